@@ -1,0 +1,207 @@
+"""Plain fp64 CPU oracle for the DashAttention forward path (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg may import
+this package.  The CUDA library never does: the two share no code.
+
+The arithmetic lives in ``dash_oracle.c`` (fp64, OpenMP over rows); this module only
+marshals numpy/torch arrays into it.  Every function widens its inputs to float64 (bf16
+inputs widen exactly) and returns float64 numpy arrays.
+
+Parity status per function (pins live in ``tests/test_oracle_pins.py``):
+  stage0            pinned (mean pooling at head_cls = 0, SDPA special case, arg-max limit)
+  entmax / stage1   pinned (sum to one, sort closed forms, brute-force supports, softmax limit)
+  stage2            pinned (dense causal attention special case, variational optimum,
+                    exact zero weight of masked chunks)
+  decode            pinned (equals the prefill row at the same position)
+  diagonal branch, GQA score averaging, bias = sigma * log p: parity unpinned by the pages
+  (they rest on stated readings; the tests pin the library to those readings).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dash_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+_dbl_p = ctypes.POINTER(ctypes.c_double)
+_i64_p = ctypes.POINTER(ctypes.c_int64)
+_L = ctypes.c_long
+
+
+def build(force: bool = False) -> str:
+    """Compile dash_oracle.c into liboracle.so (gcc, -O2, OpenMP, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        subprocess.check_call(
+            ["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-o", _LIB, _SRC, "-lm"])
+    return _LIB
+
+
+_lib = None
+
+
+def _get():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        lib.oracle_stage0.argtypes = [_dbl_p, _dbl_p, _L, _L, _L, _L, _L, _dbl_p]
+        lib.oracle_stage0.restype = None
+        for name in ("oracle_entmax", "oracle_entmax_bisect"):
+            getattr(lib, name).argtypes = (
+                [_dbl_p, _L, ctypes.c_double, _dbl_p] if name == "oracle_entmax"
+                else [_dbl_p, _L, ctypes.c_double, _dbl_p])
+            getattr(lib, name).restype = ctypes.c_double
+        for name in ("oracle_sparsemax_sort", "oracle_entmax15_sort", "oracle_softmax"):
+            getattr(lib, name).argtypes = [_dbl_p, _L, _dbl_p]
+            getattr(lib, name).restype = ctypes.c_double
+        lib.oracle_stage1.argtypes = [_dbl_p, _dbl_p, _L, _L, _L, _L, _L, _L, ctypes.c_double,
+                                      ctypes.c_double, _i64_p, _L, _dbl_p, _dbl_p, _dbl_p]
+        lib.oracle_stage1.restype = None
+        lib.oracle_stage2.argtypes = [_dbl_p, _dbl_p, _dbl_p, _dbl_p, _L, _L, _L, _L, _L, _L,
+                                      ctypes.c_double, ctypes.c_int, _i64_p, _L, _dbl_p]
+        lib.oracle_stage2.restype = None
+        lib.oracle_decode.argtypes = [_dbl_p, _dbl_p, _dbl_p, _dbl_p, _i64_p, _L, _L, _L, _L,
+                                      _L, _L, ctypes.c_double, ctypes.c_double,
+                                      ctypes.c_double, _dbl_p, _dbl_p, _dbl_p, _dbl_p]
+        lib.oracle_decode.restype = None
+        lib.oracle_num_threads.argtypes = []
+        lib.oracle_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(a) -> np.ndarray:
+    """Widen a torch tensor or array-like to a C-contiguous float64 numpy array."""
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            a = a.detach().to("cpu", torch.float64).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(_dbl_p)
+
+
+def num_threads() -> int:
+    return int(_get().oracle_num_threads())
+
+
+# --------------------------------------------------------------------------- stage 0
+def stage0(K, head_cls, chunk_size: int) -> np.ndarray:
+    """Chunk summaries [B,Hkv,T//Bc,D] of every complete chunk (gist.science summary,
+    "Stufe 0: Lokale Chunk-Zusammenfassung")."""
+    K = _f64(K)
+    hc = _f64(head_cls)
+    B, Hkv, T, D = K.shape
+    out = np.zeros((B, Hkv, T // chunk_size, D))
+    _get().oracle_stage0(_ptr(K), _ptr(hc), B, Hkv, T, D, chunk_size, _ptr(out))
+    return out
+
+
+# --------------------------------------------------------------------------- entmax
+def entmax(s, alpha: float, method: str = "auto"):
+    """alpha-entmax of one score vector s: returns (p, tau).
+
+    method: "auto" (exact sort algorithm for alpha in {1.5, 2}, softmax for 1, bisection
+    otherwise), "bisect", "sort15", "sparsemax", "softmax"."""
+    s = _f64(s).ravel()
+    n = s.size
+    p = np.zeros(n)
+    lib = _get()
+    if method == "auto":
+        tau = lib.oracle_entmax(_ptr(s), n, float(alpha), _ptr(p))
+    elif method == "bisect":
+        tau = lib.oracle_entmax_bisect(_ptr(s), n, float(alpha), _ptr(p))
+    elif method == "sort15":
+        tau = lib.oracle_entmax15_sort(_ptr(s), n, _ptr(p))
+    elif method == "sparsemax":
+        tau = lib.oracle_sparsemax_sort(_ptr(s), n, _ptr(p))
+    elif method == "softmax":
+        tau = lib.oracle_softmax(_ptr(s), n, _ptr(p))
+    else:
+        raise ValueError(method)
+    return p, float(tau)
+
+
+# --------------------------------------------------------------------------- stage 1
+def stage1(Q, summary, seq_len: int, chunk_size: int, alpha: float, gamma: float = 1.0,
+           rows=None):
+    """Routing of the given rows (default: all).  Returns (p, m, tau):
+    p, m [B,Hkv,nrows,C] (m = margin (alpha-1)s - tau on routable chunks, NaN elsewhere),
+    tau [B,Hkv,nrows].  (gist.science summary, "Stufe 1: Entmax-Chunk-Routing")."""
+    Q = _f64(Q)
+    S = _f64(summary)
+    B, Hq, T, D = Q.shape
+    assert T == seq_len
+    Hkv = S.shape[1]
+    rows = np.arange(T, dtype=np.int64) if rows is None else np.ascontiguousarray(
+        np.asarray(rows, dtype=np.int64))
+    C = (T + chunk_size - 1) // chunk_size
+    nr = rows.size
+    p = np.zeros((B, Hkv, nr, C))
+    m = np.zeros((B, Hkv, nr, C))
+    tau = np.zeros((B, Hkv, nr))
+    _get().oracle_stage1(_ptr(Q), _ptr(S), B, Hq, Hkv, T, D, chunk_size, float(alpha),
+                         float(gamma), rows.ctypes.data_as(_i64_p), nr, _ptr(p), _ptr(m),
+                         _ptr(tau))
+    return p, m, tau
+
+
+# --------------------------------------------------------------------------- stage 2
+def stage2(Q, K, V, p, chunk_size: int, sigma: float = 1.0, rows=None, dense: bool = False):
+    """Prior-induced block-sparse softmax attention for the given rows: O [B,Hq,nrows,D].
+    p is [B,Hkv,nrows,C] (ignored when dense).  (gist.science summary, "Stufe 2:
+    Prior-induzierte spaerliche Softmax")."""
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    B, Hq, T, D = Q.shape
+    Hkv = K.shape[1]
+    rows = np.arange(T, dtype=np.int64) if rows is None else np.ascontiguousarray(
+        np.asarray(rows, dtype=np.int64))
+    nr = rows.size
+    out = np.zeros((B, Hq, nr, D))
+    if dense:
+        pp = None
+    else:
+        pp = _f64(p)
+        assert pp.shape[:3] == (B, Hkv, nr)
+    _get().oracle_stage2(_ptr(Q), _ptr(K), _ptr(V), _ptr(pp) if pp is not None else None,
+                         B, Hq, Hkv, T, D, chunk_size, float(sigma), int(dense),
+                         rows.ctypes.data_as(_i64_p), nr, _ptr(out))
+    return out
+
+
+def prefill(Q, K, V, head_cls, chunk_size: int, alpha: float, gamma: float = 1.0,
+            sigma: float = 1.0, rows=None, dense: bool = False):
+    """Whole forward pass for the given rows: dict(O, p, m, tau, summary)."""
+    T = _f64(Q).shape[2] if not hasattr(Q, "shape") else Q.shape[2]
+    summary = stage0(K, head_cls, chunk_size)
+    p, m, tau = stage1(Q, summary, T, chunk_size, alpha, gamma, rows)
+    O = stage2(Q, K, V, p, chunk_size, sigma, rows, dense)
+    return dict(O=O, p=p, m=m, tau=tau, summary=summary)
+
+
+# --------------------------------------------------------------------------- decode
+def decode(q, K_cache, V_cache, head_cls, seq_lens, chunk_size: int, alpha: float,
+           gamma: float = 1.0, sigma: float = 1.0):
+    """One decode step: the row t = seq_lens[b]-1 of every sequence.  Returns dict(O
+    [B,Hq,D], p, m [B,Hkv,Ccap], tau [B,Hkv])."""
+    q, K, V, hc = _f64(q), _f64(K_cache), _f64(V_cache), _f64(head_cls)
+    B, Hq, D = q.shape
+    Hkv, cap = K.shape[1], K.shape[2]
+    sl = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int64))
+    Ccap = (cap + chunk_size - 1) // chunk_size
+    O = np.zeros((B, Hq, D))
+    p = np.zeros((B, Hkv, Ccap))
+    m = np.zeros((B, Hkv, Ccap))
+    tau = np.zeros((B, Hkv))
+    _get().oracle_decode(_ptr(q), _ptr(K), _ptr(V), _ptr(hc), sl.ctypes.data_as(_i64_p), B, Hq,
+                         Hkv, cap, D, chunk_size, float(alpha), float(gamma), float(sigma),
+                         _ptr(O), _ptr(p), _ptr(m), _ptr(tau))
+    return dict(O=O, p=p, m=m, tau=tau)

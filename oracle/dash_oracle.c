@@ -1,0 +1,331 @@
+/*
+ * dash_oracle.c -- plain, slow, fp64 CPU oracle for the DashAttention forward path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and bench.py's
+ * CPU-baseline leg may load this library.  It shares no code, header, table or
+ * constant with the CUDA library under sparse_hierarchical_attention_stage0_b200/.
+ *
+ * Sources (page title, section):
+ *   [S0] gist.science "DashAttention: Differentiable and Adaptive Sparse Hierarchical
+ *        Attention", Technische Zusammenfassung, "Stufe 0: Lokale Chunk-Zusammenfassung"
+ *        -- a learned query attends by local scaled dot-product attention over the keys
+ *        of each chunk; with the query at zero this is mean pooling; a complete chunk's
+ *        summary is frozen and cached.
+ *   [S1] same page, "Stufe 1: Entmax-Chunk-Routing" -- w = alpha-entmax(gamma * z) over
+ *        the chunk logits; GQA heads sharing a KV head share one support.
+ *   [S2] same page, "Stufe 2: Prior-induzierte spaerliche Softmax" -- softmax with the
+ *        reference distribution replaced by a prior g from the routing weights, g = 0
+ *        where w = 0 (dynamic masking); the diagonal chunk keeps a separate branch.
+ *   [E]  alpha-entmax as defined in the benchmark spec of this library:
+ *        p_c = [(alpha-1) s_c - tau]_+^{1/(alpha-1)}, sum_c p_c = 1; alpha = 1 is softmax.
+ *
+ * Readings taken where the pages are silent (listed in the design notes):
+ *   - scale 1/sqrt(D) in every stage; summaries are of the keys only;
+ *   - head_cls is one vector per KV head, query head h belongs to KV head h / G;
+ *   - GQA aggregation = mean of the G query heads' scores (= score of the mean query);
+ *   - routable chunks of row t are the complete chunks c < floor(t / Bc);
+ *   - the diagonal chunk is always attended (causal), with prior weight 1 (bias 0);
+ *   - bias of an active routed chunk = sigma * log p_c.
+ *
+ * Every array is dense, row-major, fp64.  Layouts:
+ *   Q [B,Hq,T,D], K,V [B,Hkv,T,D], head_cls [Hkv,D], summary [B,Hkv,T/Bc,D].
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#include <stdint.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static double dotd(const double *a, const double *b, long n) {
+    double s = 0.0;
+    for (long i = 0; i < n; ++i) s += a[i] * b[i];
+    return s;
+}
+
+/* ---------------------------------------------------------------- Stage 0 [S0] */
+
+/* Summary of one chunk: softmax over the chunk's keys of hc.k_j / sqrt(D), then the
+ * softmax-weighted sum of the same keys. */
+static void summarize_chunk(const double *kc, long n, const double *hc, long D, double *out) {
+    double *l = (double *)malloc(sizeof(double) * (size_t)n);
+    double mx = -INFINITY;
+    for (long j = 0; j < n; ++j) {
+        l[j] = dotd(hc, kc + j * D, D) / sqrt((double)D);
+        if (l[j] > mx) mx = l[j];
+    }
+    double den = 0.0;
+    for (long j = 0; j < n; ++j) { l[j] = exp(l[j] - mx); den += l[j]; }
+    for (long d = 0; d < D; ++d) out[d] = 0.0;
+    for (long j = 0; j < n; ++j) {
+        double w = l[j] / den;
+        for (long d = 0; d < D; ++d) out[d] += w * kc[j * D + d];
+    }
+    free(l);
+}
+
+/* Summaries of every complete chunk: summary[b,g,c,:] for c < floor(T/Bc). */
+void oracle_stage0(const double *K, const double *hc, long B, long Hkv, long T, long D,
+                   long Bc, double *summary) {
+    long Cf = T / Bc;
+#pragma omp parallel for collapse(3) schedule(static)
+    for (long b = 0; b < B; ++b)
+        for (long g = 0; g < Hkv; ++g)
+            for (long c = 0; c < Cf; ++c)
+                summarize_chunk(K + ((b * Hkv + g) * T + c * Bc) * D, Bc, hc + g * D, D,
+                                summary + ((b * Hkv + g) * Cf + c) * D);
+}
+
+/* ------------------------------------------------------------- entmax [E], [S1] */
+
+static int cmp_desc(const void *a, const void *b) {
+    double x = *(const double *)a, y = *(const double *)b;
+    return (x < y) - (x > y);
+}
+
+/* f(tau) = sum_c [x_c - tau]_+^beta  (beta = 1/(alpha-1)) */
+static double entmax_mass(const double *x, long n, double tau, double beta) {
+    double f = 0.0;
+    for (long c = 0; c < n; ++c)
+        if (x[c] > tau) f += pow(x[c] - tau, beta);
+    return f;
+}
+
+/* Any alpha > 1: bisection for the root of f(tau) = 1 on [max x - 1, max x - n^{1-alpha}],
+ * where f(lo) >= 1 >= f(hi) and f is strictly decreasing on the bracket; 200 halvings,
+ * then Newton polish steps kept inside the final bracket.  x = (alpha-1) s. */
+double oracle_entmax_bisect(const double *s, long n, double alpha, double *p) {
+    double beta = 1.0 / (alpha - 1.0);
+    double *x = (double *)malloc(sizeof(double) * (size_t)n);
+    double mx = -INFINITY;
+    for (long c = 0; c < n; ++c) { x[c] = (alpha - 1.0) * s[c]; if (x[c] > mx) mx = x[c]; }
+    double lo = mx - 1.0, hi = mx - pow((double)n, 1.0 - alpha);
+    for (int it = 0; it < 200; ++it) {
+        double mid = 0.5 * (lo + hi);
+        if (entmax_mass(x, n, mid, beta) >= 1.0) lo = mid; else hi = mid;
+    }
+    double tau = 0.5 * (lo + hi);
+    for (int it = 0; it < 4; ++it) {
+        double f = -1.0, df = 0.0;
+        for (long c = 0; c < n; ++c)
+            if (x[c] > tau) {
+                f += pow(x[c] - tau, beta);
+                df += beta * pow(x[c] - tau, beta - 1.0);
+            }
+        if (df <= 0.0) break;
+        double nt = tau + f / df;
+        if (!(nt >= lo && nt <= hi)) break;
+        tau = nt;
+    }
+    for (long c = 0; c < n; ++c) p[c] = x[c] > tau ? pow(x[c] - tau, beta) : 0.0;
+    free(x);
+    return tau;
+}
+
+/* alpha = 2 (sparsemax), exact: sort x descending; the support size k is the largest k
+ * with 1 + k z_k > sum_{j<=k} z_j; tau = (sum_{j<=k} z_j - 1) / k
+ * (Martins & Astudillo 2016, "From Softmax to Sparsemax"). */
+double oracle_sparsemax_sort(const double *s, long n, double *p) {
+    double *z = (double *)malloc(sizeof(double) * (size_t)n);
+    for (long c = 0; c < n; ++c) z[c] = s[c];          /* alpha - 1 = 1 */
+    qsort(z, (size_t)n, sizeof(double), cmp_desc);
+    double cum = 0.0, tau = 0.0;
+    for (long k = 1; k <= n; ++k) {
+        cum += z[k - 1];
+        if (1.0 + (double)k * z[k - 1] > cum) tau = (cum - 1.0) / (double)k;
+    }
+    for (long c = 0; c < n; ++c) p[c] = s[c] > tau ? s[c] - tau : 0.0;
+    free(z);
+    return tau;
+}
+
+/* alpha = 1.5, exact: sort x = s/2 descending; for the top-k set, sum (x_j - tau)^2 = 1 has
+ * the root tau_k = mean_k - sqrt((1 - k * var_k) / k) (mean_k, var_k: mean and population
+ * variance of the top k); the support is the largest k whose root lies below its k-th
+ * value (Peters, Niculae & Martins 2019, "Sparse Sequence-to-Sequence Models"). */
+double oracle_entmax15_sort(const double *s, long n, double *p) {
+    double *z = (double *)malloc(sizeof(double) * (size_t)n);
+    for (long c = 0; c < n; ++c) z[c] = 0.5 * s[c];
+    qsort(z, (size_t)n, sizeof(double), cmp_desc);
+    /* mean and M2 = k * var of the top k, updated one value at a time (Welford 1962). */
+    double mean = 0.0, M2 = 0.0, tau = z[0] - 1.0;
+    for (long k = 1; k <= n; ++k) {
+        double dlt = z[k - 1] - mean;
+        mean += dlt / (double)k;
+        M2 += dlt * (z[k - 1] - mean);
+        double disc = (1.0 - M2) / (double)k;
+        if (disc < 0.0) break;               /* M2 never decreases: no larger support fits */
+        double tk = mean - sqrt(disc);
+        if (tk < z[k - 1]) tau = tk;
+    }
+    for (long c = 0; c < n; ++c) {
+        double m = 0.5 * s[c] - tau;
+        p[c] = m > 0.0 ? m * m : 0.0;
+    }
+    free(z);
+    return tau;
+}
+
+/* alpha = 1: softmax; returns the log-sum-exp. */
+double oracle_softmax(const double *s, long n, double *p) {
+    double mx = -INFINITY;
+    for (long c = 0; c < n; ++c) if (s[c] > mx) mx = s[c];
+    double den = 0.0;
+    for (long c = 0; c < n; ++c) { p[c] = exp(s[c] - mx); den += p[c]; }
+    for (long c = 0; c < n; ++c) p[c] /= den;
+    return mx + log(den);
+}
+
+/* Dispatch: exact sort algorithms where they exist, bisection otherwise. */
+double oracle_entmax(const double *s, long n, double alpha, double *p) {
+    if (alpha == 1.0) return oracle_softmax(s, n, p);
+    if (alpha == 2.0) return oracle_sparsemax_sort(s, n, p);
+    if (alpha == 1.5) return oracle_entmax15_sort(s, n, p);
+    return oracle_entmax_bisect(s, n, alpha, p);
+}
+
+/* ---------------------------------------------------------------- Stage 1 [S1] */
+
+/* Routing of one row from its group-mean query qbar over the ct routable chunks S[0..ct).
+ * p_row, m_row have C entries: p_c and the margin m_c = (alpha-1) s_c - tau for c < ct
+ * (margin +inf for alpha = 1), p = 0 and m = NaN elsewhere.  Returns tau (the log-sum-exp
+ * for alpha = 1; NaN when ct = 0). */
+static double route_qbar(const double *qbar, const double *S, long ct, long C, long D,
+                         double alpha, double gamma, double *p_row, double *m_row) {
+    for (long c = 0; c < C; ++c) { p_row[c] = 0.0; m_row[c] = NAN; }
+    if (ct == 0) return NAN;
+    double *s = (double *)malloc(sizeof(double) * (size_t)ct);
+    for (long c = 0; c < ct; ++c)
+        s[c] = gamma * dotd(qbar, S + c * D, D) / sqrt((double)D);
+    double tau = oracle_entmax(s, ct, alpha, p_row);
+    for (long c = 0; c < ct; ++c)
+        m_row[c] = alpha == 1.0 ? INFINITY : (alpha - 1.0) * s[c] - tau;
+    free(s);
+    return tau;
+}
+
+/* Group-mean query of KV group g: the mean of the G query rows q_h, h in [gG, (g+1)G).
+ * Averaging the G heads' scores equals scoring this mean query (linearity). */
+static void group_mean(const double *q0, long stride, long G, long D, double *qbar) {
+    for (long d = 0; d < D; ++d) qbar[d] = 0.0;
+    for (long h = 0; h < G; ++h)
+        for (long d = 0; d < D; ++d) qbar[d] += q0[h * stride + d];
+    for (long d = 0; d < D; ++d) qbar[d] /= (double)G;
+}
+
+/* Stage 1 for a list of rows.  summary is [B,Hkv,T/Bc,D] (T is the sequence length the
+ * summaries were built from).  Outputs: p_out, m_out [B,Hkv,nrows,C], tau_out [B,Hkv,nrows],
+ * with C = ceil(T/Bc). */
+void oracle_stage1(const double *Q, const double *summary, long B, long Hq, long Hkv, long T,
+                   long D, long Bc, double alpha, double gamma, const int64_t *rows,
+                   long nrows, double *p_out, double *m_out, double *tau_out) {
+    long G = Hq / Hkv, Cf = T / Bc, C = (T + Bc - 1) / Bc;
+#pragma omp parallel for collapse(3) schedule(dynamic, 16)
+    for (long b = 0; b < B; ++b)
+        for (long g = 0; g < Hkv; ++g)
+            for (long r = 0; r < nrows; ++r) {
+                long o = (b * Hkv + g) * nrows + r, t = rows[r];
+                double *qbar = (double *)malloc(sizeof(double) * (size_t)D);
+                group_mean(Q + ((b * Hq + g * G) * T + t) * D, T * D, G, D, qbar);
+                tau_out[o] = route_qbar(qbar, summary + (b * Hkv + g) * Cf * D, t / Bc, C, D,
+                                        alpha, gamma, p_out + o * C, m_out + o * C);
+                free(qbar);
+            }
+}
+
+/* ---------------------------------------------------------------- Stage 2 [S2] */
+
+/* One (b, h, t) output row.  Keys j <= t; key j of chunk c = j / Bc gets
+ *   bias 0               if c == ct (diagonal branch) or dense != 0,
+ *   bias sigma * log p_c if c < ct and p_c > 0,
+ *   no weight at all     if c < ct and p_c == 0 (dynamic masking).
+ * out = sum_j softmax_j(q.k_j / sqrt(D) + bias_j) v_j, with the exact maximum. */
+static void attend_row(const double *q, const double *Kg, const double *Vg, const double *p_row,
+                       long t, long D, long Bc, double sigma, int dense, double *out) {
+    long ct = t / Bc, n = t + 1;
+    double *l = (double *)malloc(sizeof(double) * (size_t)n);
+    double mx = -INFINITY;
+    for (long j = 0; j < n; ++j) {
+        long c = j / Bc;
+        if (c == ct || dense) {
+            l[j] = dotd(q, Kg + j * D, D) / sqrt((double)D);
+        } else if (p_row[c] > 0.0) {
+            l[j] = dotd(q, Kg + j * D, D) / sqrt((double)D) + sigma * log(p_row[c]);
+        } else {
+            l[j] = -INFINITY;
+        }
+        if (l[j] > mx) mx = l[j];
+    }
+    double den = 0.0;
+    for (long d = 0; d < D; ++d) out[d] = 0.0;
+    for (long j = 0; j < n; ++j) {
+        if (l[j] == -INFINITY) continue;
+        double w = exp(l[j] - mx);
+        den += w;
+        for (long d = 0; d < D; ++d) out[d] += w * Vg[j * D + d];
+    }
+    for (long d = 0; d < D; ++d) out[d] /= den;
+    free(l);
+}
+
+/* Stage 2 for a list of rows.  p is [B,Hkv,nrows,C] (the routing of the same rows) or NULL
+ * when dense != 0.  O_out is [B,Hq,nrows,D]. */
+void oracle_stage2(const double *Q, const double *K, const double *V, const double *p, long B,
+                   long Hq, long Hkv, long T, long D, long Bc, double sigma, int dense,
+                   const int64_t *rows, long nrows, double *O_out) {
+    long G = Hq / Hkv, C = (T + Bc - 1) / Bc;
+#pragma omp parallel for collapse(3) schedule(dynamic, 4)
+    for (long b = 0; b < B; ++b)
+        for (long h = 0; h < Hq; ++h)
+            for (long r = 0; r < nrows; ++r) {
+                long g = h / G, t = rows[r];
+                const double *prow = p ? p + ((b * Hkv + g) * nrows + r) * C : NULL;
+                attend_row(Q + ((b * Hq + h) * T + t) * D, K + (b * Hkv + g) * T * D,
+                           V + (b * Hkv + g) * T * D, prow, t, D, Bc, sigma, dense,
+                           O_out + ((b * Hq + h) * nrows + r) * D);
+            }
+}
+
+/* ---------------------------------------------------------------- decode */
+
+/* One incremental-decode step for B independent sequences.  Caches K,V [B,Hkv,cap,D] hold
+ * seq_lens[b] valid tokens (the current token included); q is [B,Hq,D] for the token at
+ * t = seq_lens[b]-1.  The chunk summaries of the complete chunks are recomputed here from
+ * the cache keys (the frozen cache of [S0] holds exactly these values).  Outputs:
+ * O [B,Hq,D], p and m [B,Hkv,Ccap] (Ccap = ceil(cap/Bc)), tau [B,Hkv]. */
+void oracle_decode(const double *q, const double *K, const double *V, const double *hc,
+                   const int64_t *seq_lens, long B, long Hq, long Hkv, long cap, long D,
+                   long Bc, double alpha, double gamma, double sigma, double *O, double *p,
+                   double *m, double *tau) {
+    long G = Hq / Hkv, Ccap = (cap + Bc - 1) / Bc;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (long b = 0; b < B; ++b)
+        for (long g = 0; g < Hkv; ++g) {
+            long L = seq_lens[b], t = L - 1, ct = t / Bc;
+            const double *Kg = K + (b * Hkv + g) * cap * D;
+            const double *Vg = V + (b * Hkv + g) * cap * D;
+            double *S = (double *)malloc(sizeof(double) * (size_t)((ct > 0 ? ct : 1) * D));
+            for (long c = 0; c < ct; ++c)
+                summarize_chunk(Kg + c * Bc * D, Bc, hc + g * D, D, S + c * D);
+            double *pr = p + (b * Hkv + g) * Ccap, *mr = m + (b * Hkv + g) * Ccap;
+            double *qbar = (double *)malloc(sizeof(double) * (size_t)D);
+            group_mean(q + (b * Hq + g * G) * D, D, G, D, qbar);
+            double tv = route_qbar(qbar, S, ct, Ccap, D, alpha, gamma, pr, mr);
+            free(qbar);
+            tau[b * Hkv + g] = tv;
+            for (long h = g * G; h < (g + 1) * G; ++h)
+                attend_row(q + (b * Hq + h) * D, Kg, Vg, pr, t, D, Bc, sigma, 0,
+                           O + (b * Hq + h) * D);
+            free(S);
+        }
+}
+
+/* Number of OpenMP threads the oracle runs with (for reporting). */
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,343 @@
+"""Pins of the fp64 oracle against things other than itself (CPU only).
+
+Each pin is chosen so that a plausible slip in the oracle (a dropped 1/sqrt(D), a wrong
+sign or index, a transposed operand, a wrong support rule, a mishandled diagonal) fails at
+least one test:
+  * hand-derived examples (tests/golden/hand_examples.json);
+  * closed forms and library routines: torch SDPA in float64 for Stage 0 and for dense
+    causal attention, scipy softmax for the alpha -> 1 limit;
+  * brute force over all supports for tiny entmax problems;
+  * variational optimality: entmax maximises p.s + Tsallis entropy; the prior softmax
+    maximises z.w - KL(w || g) (gist.science "DashAttention ...", Technische
+    Zusammenfassung, "Stufe 2", variational formulation);
+  * invariants: sum to one, KKT, masked chunks contribute exactly nothing, decode == prefill.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dash_inputs import CONFIGS, make_prefill
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden", "hand_examples.json")
+RNG = np.random.default_rng(12345)
+
+
+# ----------------------------------------------------------------------------- entmax
+@pytest.mark.parametrize("case", json.load(open(GOLD))["entmax"], ids=lambda c: str(c["s"]))
+def test_entmax_hand_examples(case):
+    p, tau = oracle.entmax(np.array(case["s"]), case["alpha"])
+    np.testing.assert_allclose(p, case["p"], atol=1e-13)
+    assert abs(tau - case["tau"]) < 1e-13
+
+
+@pytest.mark.parametrize("alpha", [1.0, 1.25, 1.5, 1.75, 2.0, 2.5])
+@pytest.mark.parametrize("n", [1, 2, 7, 64, 1000])
+def test_entmax_sums_to_one_and_kkt(alpha, n):
+    s = RNG.normal(size=n) * 3
+    p, tau = oracle.entmax(s, alpha)
+    assert abs(p.sum() - 1.0) < 1e-12
+    assert (p >= 0).all()
+    if alpha > 1:
+        x = (alpha - 1) * s
+        sup = p > 0
+        # on the support p^(alpha-1) = x - tau; off it x <= tau
+        np.testing.assert_allclose(p[sup] ** (alpha - 1), x[sup] - tau, rtol=1e-9, atol=1e-12)
+        assert (x[~sup] <= tau + 1e-12).all()
+
+
+def _brute_force(s, alpha):
+    """Enumerate every support S, solve sum_{S}(x - tau)^beta = 1 in closed form (beta = 2 or
+    1), keep the self-consistent S (x > tau on S, x <= tau off S)."""
+    x = (alpha - 1) * np.asarray(s, dtype=np.float64)
+    n = x.size
+    found = []
+    for k in range(1, n + 1):
+        for S in itertools.combinations(range(n), k):
+            xs = x[list(S)]
+            if alpha == 2.0:
+                tau = (xs.sum() - 1) / k
+            else:  # alpha == 1.5: k tau^2 - 2 tau sum + sum sq - 1 = 0, smaller root
+                a, b, c = k, -2 * xs.sum(), (xs ** 2).sum() - 1
+                disc = b * b - 4 * a * c
+                if disc < 0:
+                    continue
+                tau = (-b - math.sqrt(disc)) / (2 * a)
+            inside = np.zeros(n, bool)
+            inside[list(S)] = True
+            if (x[inside] > tau).all() and (x[~inside] <= tau).all():
+                found.append(tau)
+    assert len(found) == 1, found          # the problem is strictly convex: one solution
+    tau = found[0]
+    beta = 1 / (alpha - 1)
+    return np.where(x > tau, np.maximum(x - tau, 0) ** beta, 0.0), tau
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+@pytest.mark.parametrize("trial", range(12))
+def test_entmax_brute_force(alpha, trial):
+    n = 2 + trial % 10
+    s = RNG.normal(size=n) * (0.5 + trial)
+    pb, tb = _brute_force(s, alpha)
+    for method in ("auto", "bisect"):
+        p, tau = oracle.entmax(s, alpha, method=method)
+        np.testing.assert_allclose(p, pb, atol=1e-12)
+        assert abs(tau - tb) < 1e-12
+
+
+@pytest.mark.parametrize("n", [3, 50, 2047])
+def test_sort_algorithms_agree_with_bisection(n):
+    s = RNG.normal(size=n) * 2
+    for alpha, method in ((1.5, "sort15"), (2.0, "sparsemax")):
+        p1, t1 = oracle.entmax(s, alpha, method=method)
+        p2, t2 = oracle.entmax(s, alpha, method="bisect")
+        np.testing.assert_allclose(p1, p2, atol=1e-12)
+        assert abs(t1 - t2) < 1e-12
+
+
+def _tsallis_objective(p, s, alpha):
+    return p @ s + (p - p ** alpha).sum() / (alpha * (alpha - 1))
+
+
+@pytest.mark.parametrize("alpha", [1.25, 1.5, 2.0, 3.0])
+def test_entmax_is_the_tsallis_maximiser(alpha):
+    """alpha-entmax(s) = argmax over the simplex of p.s + (1/(alpha(alpha-1))) sum(p - p^alpha)
+    (Peters, Niculae & Martins 2019); no feasible perturbation may do better."""
+    s = RNG.normal(size=9) * 2
+    p, _ = oracle.entmax(s, alpha)
+    f0 = _tsallis_objective(p, s, alpha)
+    for _ in range(2000):
+        y = p + RNG.normal(size=9) * RNG.choice([1e-3, 1e-2, 1e-1])
+        y = np.maximum(y, 0)
+        y /= y.sum()
+        assert _tsallis_objective(y, s, alpha) <= f0 + 1e-12
+    for _ in range(500):
+        y = RNG.dirichlet(np.ones(9))
+        assert _tsallis_objective(y, s, alpha) <= f0 + 1e-12
+
+
+def test_alpha_to_one_is_softmax():
+    from scipy.special import softmax
+    s = RNG.normal(size=40) * 2
+    p, _ = oracle.entmax(s, 1.0 + 1e-6, method="bisect")
+    np.testing.assert_allclose(p, softmax(s), atol=2e-5)
+    p1, lse = oracle.entmax(s, 1.0)
+    np.testing.assert_allclose(p1, softmax(s), atol=1e-14)
+    assert abs(lse - np.log(np.exp(s).sum())) < 1e-12
+
+
+def test_sparsemax_is_the_simplex_projection():
+    """sparsemax(s) is the Euclidean projection of s on the simplex: (s - p).(y - p) <= 0."""
+    s = RNG.normal(size=12)
+    p, _ = oracle.entmax(s, 2.0)
+    for _ in range(1000):
+        y = RNG.dirichlet(np.ones(12) * 0.3)
+        assert (s - p) @ (y - p) <= 1e-12
+
+
+def test_support_shrinks_with_gamma():
+    s = RNG.normal(size=300)
+    for alpha in (1.5, 2.0):
+        sizes = [int((oracle.entmax(g * s, alpha)[0] > 0).sum())
+                 for g in np.geomspace(0.05, 50, 40)]
+        assert all(a >= b for a, b in zip(sizes, sizes[1:])), sizes
+
+
+# ----------------------------------------------------------------------------- stage 0
+def _tiny_kv(B=2, Hkv=3, T=200, D=16, seed=0):
+    g = torch.Generator().manual_seed(seed)
+    K = torch.randn(B, Hkv, T, D, generator=g, dtype=torch.float64)
+    hc = torch.randn(Hkv, D, generator=g, dtype=torch.float64)
+    return K, hc
+
+
+def test_stage0_zero_query_is_mean_pooling():
+    K, hc = _tiny_kv()
+    S = oracle.stage0(K, torch.zeros_like(hc), 16)
+    ref = K[:, :, :192].reshape(2, 3, 12, 16, 16).mean(3).numpy()
+    np.testing.assert_allclose(S, ref, atol=1e-14)
+
+
+def test_stage0_is_single_query_sdpa():
+    import torch.nn.functional as F
+    K, hc = _tiny_kv()
+    Bc = 16
+    S = oracle.stage0(K, hc, Bc)
+    Kc = K[:, :, :192].reshape(2, 3, 12, Bc, 16)                  # [B,H,C,Bc,D]
+    q = hc.view(1, 3, 1, 1, 16).expand(2, 3, 12, 1, 16)
+    ref = F.scaled_dot_product_attention(q, Kc, Kc)                # scale 1/sqrt(D)
+    np.testing.assert_allclose(S, ref.squeeze(3).numpy(), atol=1e-13)
+
+
+def test_stage0_dominant_query_picks_argmax_key():
+    K, _ = _tiny_kv(D=8)
+    hc = torch.zeros(3, 8, dtype=torch.float64)
+    hc[:, 5] = 1e9            # logit gaps of 1e9/sqrt(8) * (key gap): one key wins
+    S = oracle.stage0(K, hc, 20)
+    Kc = K[:, :, :200].reshape(2, 3, 10, 20, 8)
+    idx = Kc[..., 5].argmax(-1)
+    ref = torch.gather(Kc, 3, idx[..., None, None].expand(2, 3, 10, 1, 8)).squeeze(3)
+    np.testing.assert_allclose(S, ref.numpy(), atol=1e-9)
+
+
+# ----------------------------------------------------------------------------- stage 1
+def test_stage1_single_visible_chunk_has_p_one_and_small_rows_route_nothing():
+    q, k, v, hc = make_prefill(CONFIGS["tiny"], seq_len=256)
+    S = oracle.stage0(k, hc, 64)
+    p, m, tau = oracle.stage1(q, S, 256, 64, 1.5)
+    assert (p[:, :, :64] == 0).all() and np.isnan(tau[:, :, :64]).all()
+    np.testing.assert_allclose(p[:, :, 64:128, 0], 1.0, atol=1e-15)
+    assert (p[:, :, 64:128, 1:] == 0).all()
+    np.testing.assert_allclose(p[:, :, 128:].sum(-1), 1.0, atol=1e-12)
+
+
+def test_stage1_gqa_mean_query_equals_mean_scores():
+    """GQA: the G heads' scores averaged = scores of the mean query; alpha = 1 exposes the
+    scores as log p + lse."""
+    q, k, v, hc = make_prefill(CONFIGS["tiny"], seq_len=320)
+    q = q.double()
+    qg = q.view(1, 2, 2, 320, 64)                       # 4 query heads, 2 KV heads, G = 2
+    S = oracle.stage0(k[:, :2], hc[:2], 64)
+    p, m, lse = oracle.stage1(q, S, 320, 64, 1.0)
+    scores = torch.einsum("bghtd,bgcd->bghtc", qg, torch.from_numpy(S)) / 8.0
+    mean_sc = scores.mean(2).numpy()                    # [B,Hkv,T,Cf]
+    for t in range(64, 320):
+        ct = t // 64
+        np.testing.assert_allclose(np.log(p[0, :, t, :ct]) + lse[0, :, t, None],
+                                   mean_sc[0, :, t, :ct], atol=1e-12)
+
+
+def test_stage1_margin_sign_is_the_support():
+    cfg = CONFIGS["gqa32k"]
+    q, k, v, hc = make_prefill(cfg, seq_len=2048 + 37)
+    S = oracle.stage0(k, hc, 64)
+    p, m, tau = oracle.stage1(q, S, q.shape[2], 64, 1.5)
+    T = q.shape[2]
+    ct = np.arange(T) // 64
+    vis = np.arange(p.shape[-1])[None, :] < ct[:, None]
+    assert ((m[0] > 0) == (p[0] > 0))[:, vis].all()
+    assert (p[0][:, ~vis] == 0).all()
+    rows = ct >= 1
+    np.testing.assert_allclose(p[0][:, rows].sum(-1), 1.0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- stage 2
+@pytest.mark.parametrize("case", json.load(open(GOLD))["attention"], ids=lambda c: str(c["p"]))
+def test_stage2_hand_examples(case):
+    Q = torch.ones(1, 1, 3, 1, dtype=torch.float64)
+    K = torch.zeros(1, 1, 3, 1, dtype=torch.float64)
+    V = torch.tensor([8.0, 0.0, 2.0], dtype=torch.float64).view(1, 1, 3, 1)
+    p = np.zeros((1, 1, 1, 3))
+    p[0, 0, 0, :2] = case["p"]
+    O = oracle.stage2(Q, K, V, p, chunk_size=1, rows=[2])
+    assert abs(O[0, 0, 0, 0] - case["O"]) < 1e-14
+
+
+def _small_qkv(B=1, Hq=4, Hkv=2, T=150, D=16, seed=3):
+    g = torch.Generator().manual_seed(seed)
+    Q = torch.randn(B, Hq, T, D, generator=g, dtype=torch.float64)
+    K = torch.randn(B, Hkv, T, D, generator=g, dtype=torch.float64)
+    V = torch.randn(B, Hkv, T, D, generator=g, dtype=torch.float64)
+    hc = torch.randn(Hkv, D, generator=g, dtype=torch.float64)
+    return Q, K, V, hc
+
+
+def test_stage2_dense_is_causal_sdpa():
+    import torch.nn.functional as F
+    Q, K, V, hc = _small_qkv()
+    O = oracle.stage2(Q, K, V, None, chunk_size=16, dense=True)
+    ref = F.scaled_dot_product_attention(Q, K.repeat_interleave(2, 1), V.repeat_interleave(2, 1),
+                                         is_causal=True)
+    np.testing.assert_allclose(O, ref.numpy(), atol=1e-13)
+
+
+def test_stage2_rows_in_first_chunk_are_local_causal_attention():
+    import torch.nn.functional as F
+    Q, K, V, hc = _small_qkv()
+    Bc = 32
+    S = oracle.stage0(K, hc, Bc)
+    p, m, tau = oracle.stage1(Q, S, 150, Bc, 1.5, rows=range(Bc))
+    O = oracle.stage2(Q, K, V, p, Bc, rows=range(Bc))
+    ref = F.scaled_dot_product_attention(Q[:, :, :Bc], K[:, :, :Bc].repeat_interleave(2, 1),
+                                         V[:, :, :Bc].repeat_interleave(2, 1), is_causal=True)
+    np.testing.assert_allclose(O, ref.numpy(), atol=1e-13)
+
+
+def test_stage2_masked_chunks_contribute_exactly_nothing():
+    """With the routing p fixed, rewriting K and V inside a row's zero-probability chunks
+    leaves that row's output unchanged to the bit (dynamic masking, g = 0 where w = 0)."""
+    Q, K, V, hc = _small_qkv(T=256)
+    Bc = 16
+    S = oracle.stage0(K, hc, Bc)
+    p, m, tau = oracle.stage1(Q, S, 256, Bc, 2.0)       # sparsemax: many exact zeros
+    checked = 0
+    for t in (40, 97, 150, 200, 255):
+        for g in range(2):
+            ct = t // Bc
+            dead = [c for c in range(ct) if p[0, g, t, c] == 0]
+            if not dead:
+                continue
+            K2, V2 = K.clone(), V.clone()
+            for c in dead:
+                K2[0, g, c * Bc:(c + 1) * Bc] = 1e3
+                V2[0, g, c * Bc:(c + 1) * Bc] = -7e5
+            O = oracle.stage2(Q, K, V, p[:, :, t:t + 1], Bc, rows=[t])
+            O2 = oracle.stage2(Q, K2, V2, p[:, :, t:t + 1], Bc, rows=[t])
+            for h in (2 * g, 2 * g + 1):
+                assert np.array_equal(O[0, h], O2[0, h])
+                checked += 1
+    assert checked >= 12
+
+
+def test_stage2_prior_softmax_is_the_variational_optimum():
+    """w = argmax_{w in simplex} z.w - KL(w || g): optimal value log sum_j g_j e^{z_j},
+    masked keys get exactly zero weight, and no feasible perturbation does better."""
+    T, Bc, D = 40, 8, 40
+    g_ = torch.Generator().manual_seed(9)
+    Q = torch.randn(1, 1, T, D, generator=g_, dtype=torch.float64)
+    K = torch.randn(1, 1, T, D, generator=g_, dtype=torch.float64)
+    V = torch.eye(T, D, dtype=torch.float64).view(1, 1, T, D)   # O row = attention weights
+    hc = torch.randn(1, D, generator=g_, dtype=torch.float64)
+    S = oracle.stage0(K, hc, Bc)
+    p, m, tau = oracle.stage1(Q, S, T, Bc, 1.5)
+    W = oracle.stage2(Q, K, V, p, Bc)[0, 0]                       # [T, T]
+    rng = np.random.default_rng(0)
+    for t in range(Bc, T):
+        ct = t // Bc
+        z = (K[0, 0, :t + 1] @ Q[0, 0, t]).numpy() / math.sqrt(D)
+        prior = np.array([1.0 if j // Bc == ct else p[0, 0, t, j // Bc] for j in range(t + 1)])
+        w = W[t, :t + 1]
+        assert (w[prior == 0] == 0).all() and (W[t, t + 1:] == 0).all()
+        sup = prior > 0
+        g = prior / prior.sum()
+
+        def F(u):
+            us = u[sup]
+            nz = us > 0
+            return u @ z - (us[nz] * np.log(us[nz] / g[sup][nz])).sum()
+        best = math.log((g[sup] * np.exp(z[sup])).sum())
+        assert abs(F(w) - best) < 1e-12
+        for _ in range(200):
+            u = np.zeros(t + 1)
+            u[sup] = np.maximum(w[sup] + rng.normal(size=sup.sum()) * 1e-2, 0)
+            u /= u.sum()
+            assert F(u) <= best + 1e-12
+
+
+# ----------------------------------------------------------------------------- decode
+def test_decode_equals_prefill_row():
+    q, k, v, hc = make_prefill(CONFIGS["gqa32k"], seq_len=700)
+    T = 700
+    full = oracle.prefill(q, k, v, hc, 64, 1.5, rows=[699, 640, 511])
+    for i, t in enumerate([699, 640, 511]):
+        L = t + 1
+        dec = oracle.decode(q[:, :, t], k[:, :, :L], v[:, :, :L], hc, [L], 64, 1.5)
+        np.testing.assert_allclose(dec["O"], full["O"][:, :, i], atol=1e-13)
+        C = (L + 63) // 64
+        np.testing.assert_allclose(dec["p"][:, :, :C], full["p"][:, :, i, :C], atol=1e-14)
+    assert T == 700
