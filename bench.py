@@ -1,0 +1,517 @@
+#!/usr/bin/env python
+"""Benchmark of the DashAttention forward path on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dash|reference]
+                    [--workload prefill128k|gqa32k|tiny] [--no-decode]
+
+A step is one causal prefill (Stage 0 -> Stage 1 -> Stage 2) over the workload's synthetic
+seeded inputs, already resident in HBM.  value = prefill tokens/s over all ranks (replicas:
+every rank runs the same workload on its own GPU, no data-path collective).  Also reported:
+active-FLOP TFLOP/s of Stage 2, per-stage times and roofline fractions, the library's own
+dense path, the end-to-end time through host buffers, a 256-step decode captured in one CUDA
+graph, and the fp64 oracle timed on the host cores on a bounded row sample.
+
+--impl reference times the oracle (plain fp64 C on the host cores) on the same workload and
+metric: each step runs the oracle over a bounded sample of rows, extrapolated to the
+workload's tokens/s.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from dash_inputs import CONFIGS, make_decode, make_prefill  # noqa: E402
+
+METRIC = "prefill tokens/s & active-FLOP TFLOP/s at 128K; decode tok/s; % roofline"
+GAMMA_FILE = os.path.join(ROOT, "tests", "golden", "gamma_prefill128k.json")
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(name):
+    cfg = CONFIGS[name]
+    if name == "prefill128k":
+        try:
+            with open(GAMMA_FILE) as f:
+                g = json.load(f)["gamma"]
+            from dataclasses import replace
+            cfg = replace(cfg, gamma=float(g))
+        except (OSError, ValueError, KeyError):
+            log("warning: no calibrated gamma for prefill128k; using 1.0")
+    return cfg
+
+
+# ------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of SM clock and throttle reasons during a region."""
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            self.proc.wait(timeout=10)
+
+    def summary(self):
+        if not self.proc:
+            return None
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), smax=float(f[2]), power=float(f[3]),
+                                 hw=f[5], hwt=f[6], swt=f[7], swp=f[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        loaded = [r for r in rows if r["power"] > 250] or rows
+        reasons = set()
+        for r in loaded:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("swp", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded),
+                "sm_max_mhz": max(r["smax"] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows), "samples_under_load": len(loaded)}
+
+
+# ------------------------------------------------------------------------------ helpers
+def popcount_words(words: torch.Tensor) -> torch.Tensor:
+    """Per-row popcount of int64 mask words [..., W] -> int64 [...]."""
+    b = words.contiguous().view(torch.uint8)
+    table = torch.tensor([bin(i).count("1") for i in range(256)], dtype=torch.int64,
+                         device=words.device)
+    return table[b.long()].view(*words.shape[:-1], -1).sum(-1)
+
+
+def active_stats(dash, q, k, v, hc, cfg):
+    """Realised routing of one run: active routed chunks per (b, g, t), block-weighted
+    sparsity over the routed (visible) chunks, and Stage 2's active FLOPs."""
+    res = dash.prefill(q, k, v, hc, cfg.chunk_size, cfg.alpha, cfg.gamma, enable_gqa=True,
+                       return_active_blocks=True)
+    cnt = popcount_words(res["active_blocks"]) - 1          # minus the diagonal bit
+    del res
+    T, Bc, D, G = cfg.seq_len, cfg.chunk_size, cfg.head_dim, cfg.group
+    t = torch.arange(T, device=q.device)
+    ct = t // Bc
+    visible = ct.to(torch.float64).sum() * cfg.batch * cfg.heads_kv
+    active = cnt.to(torch.float64).sum()
+    diag_keys = (t - ct * Bc + 1).to(torch.float64).sum() * cfg.batch * cfg.heads_kv
+    flops = 4.0 * D * G * (Bc * active + diag_keys)
+    dense_flops = 4.0 * D * G * cfg.batch * cfg.heads_kv * (T * (T + 1) / 2.0)
+    sparsity = 1.0 - float(active / visible) if visible > 0 else 0.0
+    return dict(active_flops=float(flops), dense_flops=float(dense_flops), sparsity=sparsity,
+                active_chunks=float(active), visible_chunks=float(visible))
+
+
+def stage01_bytes(cfg):
+    """Algorithmic HBM bytes of Stages 0-1: K read, summaries written and read once, Q read
+    once, mask words and tau written."""
+    B, Hq, Hkv, T, D, Bc = (cfg.batch, cfg.heads_q, cfg.heads_kv, cfg.seq_len, cfg.head_dim,
+                            cfg.chunk_size)
+    C = (T + Bc - 1) // Bc
+    W = (C + 63) // 64
+    k_bytes = B * Hkv * T * D * 2
+    summ = B * Hkv * (T // Bc) * D * 4
+    q_bytes = B * Hq * T * D * 2
+    mask = B * Hkv * T * W * 8
+    tau = B * Hkv * T * 4
+    return dict(stage0=k_bytes + summ, stage1=q_bytes + summ + mask + tau)
+
+
+def traffic_for(kernel, cfg_name):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on the current
+    kernel source (else None)."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+        e = d[kernel][cfg_name]
+        src = os.path.join(ROOT, "sparse_hierarchical_attention_stage0_b200", "csrc", e["source"])
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        return e["bytes_per_launch"] if h == e["source_sha256_16"] else None
+    except (OSError, ValueError, KeyError):
+        return None
+
+
+def timed(fn, steps, stream, flush=None):
+    """Per-step device times (ms) with CUDA events on `stream`; flush runs between steps."""
+    times = []
+    for _ in range(steps):
+        if flush is not None:
+            flush()
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        fn()
+        e.record(stream)
+        e.synchronize()
+        times.append(s.elapsed_time(e))
+    return times
+
+
+# ------------------------------------------------------------------------------ decode
+def bench_decode(dash, dev, steps_cap=256, warmup=3):
+    cfg = CONFIGS["decode64k"]
+    t0 = time.time()
+    d = make_decode(cfg)
+    log(f"decode inputs drawn in {time.time() - t0:.1f}s")
+    B, Hq, Hkv, D, Bc = cfg.batch, cfg.heads_q, cfg.heads_kv, cfg.head_dim, cfg.chunk_size
+    L0, S, cap = d["prefix_len"], min(d["steps"], steps_cap), d["capacity"]
+    k_all = d["k_all"].to(dev)
+    v_all = d["v_all"].to(dev)
+    hc = d["head_cls"].to(dev)
+    q_steps = d["q_steps"].to(dev)
+    kc = torch.zeros_like(k_all)
+    vc = torch.zeros_like(v_all)
+    kc[:, :, :L0] = k_all[:, :, :L0]
+    vc[:, :, :L0] = v_all[:, :, :L0]
+    cache = torch.zeros(B, Hkv, cap // Bc, D, device=dev)
+    seq = torch.full((B,), L0, dtype=torch.int32, device=dev)
+    dash.update_chunk_cache(kc, hc, seq, cache, Hq, Bc, n_recent=L0 // Bc)
+    out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
+    ws = dash.workspace(256, dev)
+    ws_u = dash.workspace(256, dev)
+
+    def step(s, with_routing=None):
+        L = L0 + s + 1
+        kc[:, :, L - 1] = k_all[:, :, L - 1]
+        vc[:, :, L - 1] = v_all[:, :, L - 1]
+        seq.fill_(L)
+        if L % Bc == 0:
+            dash.update_chunk_cache(kc, hc, seq, cache, Hq, Bc, n_recent=1, ws=ws_u)
+        if with_routing is None:
+            dash.decode(q_steps[s], kc, vc, seq, cache, Bc, cfg.alpha, out=out, ws=ws)
+        else:
+            dash.decode(q_steps[s], kc, vc, seq, cache, Bc, cfg.alpha, out=out, ws=ws,
+                        active_blocks=with_routing[s])
+
+    # Routing of every step (untimed pass) for the algorithmic byte count.
+    Wcap = ((cap + Bc - 1) // Bc + 63) // 64
+    masks = torch.zeros(S, B, Hkv, Wcap, dtype=torch.int64, device=dev)
+    for s in range(S):
+        step(s, masks)
+    torch.cuda.synchronize()
+    assert dash.read_device_status(ws) == 0
+    act = (popcount_words(masks) - 1).to(torch.float64)          # routed active per (s,b,g)
+    L = torch.arange(L0 + 1, L0 + S + 1, device=dev, dtype=torch.float64)
+    t = L - 1
+    ct = torch.floor(t / Bc)
+    diag_keys = t - ct * Bc + 1                                  # [S]
+    per_bg = (ct[:, None, None] * D * 4 + act * 2 * Bc * D * 2 + diag_keys[:, None, None] * 2 * D * 2
+              + 2 * (Hq // Hkv) * D * 2)
+    alg_bytes = float(per_bg.sum())
+    visible = float(ct.sum() * B * Hkv)
+    sparsity = 1.0 - float(act.sum()) / visible
+
+    # Reset the cache to the prefix and capture all steps in one graph.
+    kc[:, :, L0:] = 0
+    vc[:, :, L0:] = 0
+    seq.fill_(L0)
+    dash.update_chunk_cache(kc, hc, seq, cache, Hq, Bc, n_recent=L0 // Bc)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    stream = torch.cuda.Stream(dev)
+    stream.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(stream):
+        for s in range(min(warmup, S)):
+            step(s)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            for s in range(S):
+                step(s)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(3):
+        st = torch.cuda.Event(enable_timing=True)
+        en = torch.cuda.Event(enable_timing=True)
+        st.record(stream)
+        g.replay()
+        en.record(stream)
+        en.synchronize()
+        times.append(st.elapsed_time(en))
+    ms = statistics.median(times)
+    launches = S + sum(1 for s in range(S) if (L0 + s + 1) % Bc == 0)
+    del g
+    return dict(tokens_per_s=B * S / (ms / 1e3), ms_per_step=ms / S, steps=S, batch=B,
+                cache_len=L0, realised_sparsity=sparsity,
+                hbm_bytes_per_step=alg_bytes / S,
+                achieved_gbs=alg_bytes / (ms / 1e3) / 1e9, launches=launches,
+                note="steps include the K/V append copies and seq_len update (torch ops)")
+
+
+# ------------------------------------------------------------------------------ oracle
+def oracle_sample(cfg, q, k, v, hc, n_rows, seed=0):
+    """Time the fp64 oracle on n_rows sampled rows (all heads) plus Stage 0 over every chunk;
+    extrapolate linearly in rows to the workload's tokens/s."""
+    import oracle
+    q, k, v, hc = (oracle._f64(x) for x in (q, k, v, hc))     # widen outside the timing
+    g = torch.Generator().manual_seed(seed)
+    T = cfg.seq_len
+    rows = torch.sort(torch.randint(0, T, (n_rows,), generator=g)).values.numpy()
+    t0 = time.perf_counter()
+    S = oracle.stage0(k, hc, cfg.chunk_size)
+    t1 = time.perf_counter()
+    p, m, tau = oracle.stage1(q, S, T, cfg.chunk_size, cfg.alpha, cfg.gamma, rows)
+    oracle.stage2(q, k, v, p, cfg.chunk_size, 1.0, rows)
+    t2 = time.perf_counter()
+    total = (t1 - t0) + (t2 - t1) * T / n_rows
+    return dict(value=cfg.batch * T / total, unit="tokens/s", cores=oracle.num_threads(),
+                kind="oracle", seconds=t2 - t0,
+                sample=f"Stage 0 over all {T // cfg.chunk_size} chunks per KV head + Stages 1-2 "
+                       f"for {n_rows} uniformly sampled rows (all {cfg.heads_q} heads), "
+                       f"extrapolated linearly to {T} rows")
+
+
+# ------------------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="dash", choices=["dash", "reference"])
+    ap.add_argument("--workload", default="prefill128k", choices=["prefill128k", "gqa32k", "tiny"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--oracle-rows", type=int, default=0, help="0: pick by workload")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = workload_config(args.workload)
+    n_rows = args.oracle_rows or {"prefill128k": 96, "gqa32k": 256, "tiny": 1024}[args.workload]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        import oracle
+        q, k, v, hc = (oracle._f64(x) for x in make_prefill(cfg))
+        times = []
+        for i in range(args.warmup + args.steps):
+            r = oracle_sample(cfg, q, k, v, hc, max(8, n_rows // 4), seed=i)
+            if i >= args.warmup:
+                times.append(r)
+        value = statistics.median(x["value"] for x in times)
+        secs = sum(x["seconds"] for x in times)
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": cfg.batch * cfg.seq_len / value * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f64", "data": "synthetic (seeded planted-evidence generator)",
+                "config": {"workload": cfg.name, "batch": cfg.batch, "heads_q": cfg.heads_q,
+                           "heads_kv": cfg.heads_kv, "seq_len": cfg.seq_len,
+                           "head_dim": cfg.head_dim, "chunk_size": cfg.chunk_size,
+                           "alpha": cfg.alpha, "gamma": cfg.gamma, "parallelism": "replicas"},
+                "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": times[0]["cores"],
+                                 "kind": "oracle", "sample": times[0]["sample"]},
+                "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0},
+                "oracle_seconds": secs}
+        print(json.dumps(line), flush=True)
+        return
+
+    import sparse_hierarchical_attention_stage0_b200 as dash
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    t0 = time.time()
+    q_h, k_h, v_h, hc_h = make_prefill(cfg)
+    log(f"[rank {rank}] inputs drawn in {time.time() - t0:.1f}s")
+    q, k, v, hc = (x.to(dev) for x in (q_h, k_h, v_h, hc_h))
+    B, Hq, Hkv, T, D, Bc = cfg.batch, cfg.heads_q, cfg.heads_kv, cfg.seq_len, cfg.head_dim, cfg.chunk_size
+    prm = dash.make_params(B, Hq, Hkv, T, D, Bc, cfg.alpha, cfg.gamma, 1.0, True)
+    ws = dash.workspace(dash.prefill_workspace_size(prm), dev)
+    out = torch.empty_like(q)
+    flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    flush = lambda: flush_buf.zero_()                               # noqa: E731
+    stream = torch.cuda.current_stream(dev)
+
+    def prefill():
+        dash.prefill(q, k, v, hc, Bc, cfg.alpha, cfg.gamma, enable_gqa=True, out=out, ws=ws)
+
+    for _ in range(args.warmup):
+        prefill()
+    torch.cuda.synchronize()
+    assert dash.read_device_status(ws) == 0
+
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        step_ms = timed(prefill, args.steps, stream, flush)
+    torch.cuda.synchronize()
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+        torch.distributed.barrier()
+    value = world * B * T * args.steps / (total_ms / 1e3)
+
+    # Per-stage times through the stage entry points (same kernels as dash_prefill).
+    summ = torch.empty(B, Hkv, T // Bc, D, device=dev)
+    C = (T + Bc - 1) // Bc
+    W = (C + 63) // 64
+    tau = torch.empty(B, Hkv, T, device=dev)
+    mask = torch.empty(B, Hkv, T, W, dtype=torch.int64, device=dev)
+    ws_s = dash.workspace(256, dev)
+    import ctypes
+
+    def run_route():
+        dash._check(dash.lib.dash_route(ctypes.byref(prm), dash._ptr(q), dash._ptr(summ),
+                                        dash._ptr(tau), None, dash._ptr(mask), dash._ptr(ws_s),
+                                        256, dash._stream(dev)), "dash_route")
+
+    st_ms = {"stage0": [], "stage1": [], "stage2": []}
+    for i in range(args.warmup + args.steps):
+        flush()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(stream)
+        dash.stage0(k, hc, Bc, ws=ws_s, summary=summ)
+        ev[1].record(stream)
+        run_route()
+        ev[2].record(stream)
+        dash.attend(q, k, v, summ, tau, mask, Bc, cfg.alpha, cfg.gamma, 1.0, True, ws=ws_s, out=out)
+        ev[3].record(stream)
+        ev[3].synchronize()
+        if i >= args.warmup:
+            for j, name in enumerate(("stage0", "stage1", "stage2")):
+                st_ms[name].append(ev[j].elapsed_time(ev[j + 1]))
+    stage = {k_: statistics.mean(v_) for k_, v_ in st_ms.items()}
+
+    stats = active_stats(dash, q, k, v, hc, cfg)
+
+    def dense():
+        dash.prefill(q, k, v, None, Bc, enable_gqa=True, dense=True, out=out, ws=ws)
+
+    for _ in range(2):
+        dense()
+    dense_ms = statistics.mean(timed(dense, max(2, min(args.steps, 3)), stream, flush))
+
+    # End to end through host buffers: pinned H2D of q, k, v, head_cls; prefill; D2H of out.
+    hq, hk, hv, hhc = (x.pin_memory() for x in (q_h, k_h, v_h, hc_h))
+    ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def e2e():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        hc.copy_(hhc, non_blocking=True)
+        prefill()
+        ho.copy_(out, non_blocking=True)
+
+    e2e()
+    e2e_ms = statistics.mean(timed(e2e, args.steps, stream, flush))
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hhc))
+    d2h = ho.numel() * ho.element_size()
+
+    pk, pk_kind = peaks()
+    s2_tflops = stats["active_flops"] / (stage["stage2"] / 1e3) / 1e12
+    sb = stage01_bytes(cfg)
+    s01_gbs = (sb["stage0"] + sb["stage1"]) / ((stage["stage0"] + stage["stage1"]) / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded planted-evidence generator, see dash_inputs)",
+        "config": {"workload": cfg.name, "batch": B, "heads_q": Hq, "heads_kv": Hkv,
+                   "seq_len": T, "head_dim": D, "chunk_size": Bc, "alpha": cfg.alpha,
+                   "gamma": cfg.gamma, "parallelism": f"replicas x{world}",
+                   "l2": "flushed (256 MiB write) before every timed step"},
+        "active_tflops": s2_tflops,
+        "realised_sparsity": stats["sparsity"],
+        "stage_ms": stage,
+        "stage01_gbs": s01_gbs,
+        "dense_ms": dense_ms,
+        "speedup_vs_dense": dense_ms / (total_ms / args.steps),
+        "roofline": {"bound": "tensor", "kernel": "k_attend (Stage 2)",
+                     "achieved": s2_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": s2_tflops / pk["bf16_tflops"],
+                     "traffic": traffic_for("k_attend", cfg.name),
+                     "peak_source": f"{pk_kind} bf16 burst",
+                     "algorithmic": f"{stats['active_flops']:.4e} active FLOP per launch"},
+        "roofline_stage01": {"bound": "hbm", "achieved": s01_gbs, "peak": pk["hbm_gbs"],
+                             "unit": "GB/s", "frac": s01_gbs / pk["hbm_gbs"],
+                             "frac_of_8tbs_nominal": s01_gbs / 8000.0,
+                             "bytes": sb["stage0"] + sb["stage1"]},
+        "e2e": {"value": world * B * T / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk.summary(),
+    }
+    del hq, hk, hv, ho
+    if not args.no_decode and args.workload == "prefill128k":
+        del q, k, v, out, ws, mask, flush_buf
+        torch.cuda.empty_cache()
+        dec = bench_decode(dash, dev)
+        dec["roofline"] = {"bound": "hbm", "achieved": dec["achieved_gbs"], "peak": pk["hbm_gbs"],
+                           "unit": "GB/s", "frac": dec["achieved_gbs"] / pk["hbm_gbs"],
+                           "traffic": traffic_for("k_decode", "decode64k")}
+        line["decode"] = dec
+    if rank == 0 and world == 1:
+        line["cpu_baseline"] = oracle_sample(cfg, q_h, k_h, v_h, hc_h, n_rows)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,185 @@
+/*
+ * dash.h -- C ABI of libdash: the DashAttention forward path (chunk summaries, alpha-entmax
+ * block routing, prior-induced block-sparse softmax attention) for causal prefill and
+ * incremental decode on NVIDIA B200 (sm_100a).
+ *
+ * The method (page title, section):
+ *   gist.science "DashAttention: Differentiable and Adaptive Sparse Hierarchical Attention",
+ *   Technische Zusammenfassung:
+ *     "Stufe 0: Lokale Chunk-Zusammenfassung"   -> dash_stage0, dash_update_chunk_cache
+ *     "Stufe 1: Entmax-Chunk-Routing"            -> dash_route
+ *     "Stufe 2: Prior-induzierte spaerliche Softmax" -> dash_attend
+ *   aiexpert.news "DashAttention alcanca 75% de esparsidade ...", interface paragraph:
+ *     queries, keys, values, a per-head head_cls vector, chunk_size, estimate_diagonal,
+ *     enable_gqa, optional active_blocks mask -> dash_params_t, dash_prefill.
+ *   aixai.ru "DashAttention ...", "Трёхстадийная архитектура": the active-block mask is
+ *     bit-packed into 64-bit words and walked in one pass without explicit indices.
+ *   liuzhao09.github.io "DashAttention 精读", section 2: prefill and incremental decoding
+ *     with a chunk-representation cache -> dash_prefill, dash_decode.
+ *
+ * What is computed (notation: b batch, h query head, g = h / G its KV head with
+ * G = heads_q / heads_kv, t query position, Bc = chunk_size, D = head_dim, c_t = t / Bc):
+ *   Stage 0: summary[b,g,c] = sum_j softmax_j(head_cls[g].k_j / sqrt(D)) k_j over the keys j
+ *            of every complete chunk c.
+ *   Stage 1: for c < c_t:  s_c = gamma * qbar.summary[b,g,c] / sqrt(D), qbar = mean of the G
+ *            query heads of group g at t; p = alpha-entmax(s):
+ *            p_c = [(alpha-1) s_c - tau]_+^(1/(alpha-1)), sum_c p_c = 1 (alpha = 1: softmax).
+ *            Chunk c < c_t is active iff p_c > 0; the diagonal chunk c_t is always active.
+ *   Stage 2: O[b,h,t] = sum_j softmax_j(q.k_j / sqrt(D) + bias_j) v_j over keys j <= t in
+ *            active chunks, bias_j = sigma * log p_c(j) for routed chunks and 0 on the
+ *            diagonal chunk.  Zero-probability chunks are skipped.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are caller-owned DEVICE memory, dense, row-major (C order), with
+ *     the layouts stated per argument.  The library never allocates or frees memory and
+ *     keeps no global state; calls on different streams do not interact.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*; NULL = the
+ *     legacy default stream).  Arguments are checked on the host before any launch; a bad
+ *     argument returns DASH_ERR_INVALID_ARGUMENT / DASH_ERR_UNSUPPORTED /
+ *     DASH_ERR_WORKSPACE_TOO_SMALL and launches nothing.  A launch failure returns
+ *     DASH_ERR_CUDA.  Faults found on the device (a device-side bound violated, an
+ *     iteration cap reached) are written to a status word in the workspace and read with
+ *     dash_read_device_status; the kernels never trap.
+ *   - Pointers must be 16-byte aligned; workspaces 256-byte aligned.
+ *   - Supported: head_dim in {64, 128}; chunk_size in {64, 128}; heads_q % heads_kv == 0
+ *     with G = heads_q / heads_kv dividing 16 or a multiple of 16; heads_q == heads_kv when
+ *     enable_gqa == 0; alpha >= 1; seq_len >= 1 (seq_len % chunk_size may be non-zero: the
+ *     last partial chunk is only ever a diagonal chunk).
+ */
+#ifndef DASH_H_
+#define DASH_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DASH_OK = 0,
+    DASH_ERR_INVALID_ARGUMENT = 1,   /* a null/misaligned pointer, a bad size or value */
+    DASH_ERR_UNSUPPORTED = 2,        /* valid, but outside the supported shapes/flags */
+    DASH_ERR_WORKSPACE_TOO_SMALL = 3,
+    DASH_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed */
+    DASH_ERR_DEVICE_TIMEOUT = 5      /* a device wait or iteration cap ran out */
+} dash_status_t;
+
+enum {
+    /* Dense causal attention: Stages 0-1 are skipped and every chunk c <= c_t is attended
+     * with bias 0 (the uniform prior).  summary_k, p, active_blocks must be NULL. */
+    DASH_FLAG_DENSE = 1,
+    /* Stages 0-1 run and write their outputs, but Stage 2 attends every chunk c <= c_t with
+     * bias 0 (all blocks forced active, uniform prior).  Same O as DASH_FLAG_DENSE. */
+    DASH_FLAG_FORCE_ALL_ACTIVE = 2,
+    /* Reserved: the diagonal correction of the entmax normalisation ("estimate_diagonal").
+     * The pages give no formula; requesting it returns DASH_ERR_UNSUPPORTED. */
+    DASH_FLAG_ESTIMATE_DIAGONAL = 4
+};
+
+typedef struct {
+    int batch;        /* B */
+    int heads_q;      /* H_q */
+    int heads_kv;     /* H_kv */
+    int seq_len;      /* prefill: T.  decode: cache capacity (tokens per sequence). */
+    int head_dim;     /* D */
+    int chunk_size;   /* Bc */
+    float alpha;      /* entmax alpha >= 1 (1 = softmax routing, 1.5 default, 2 = sparsemax) */
+    float gamma;      /* Stage 1 score factor (1.0 default) */
+    float sigma;      /* prior strength: bias = sigma * log p (1.0 default) */
+    int enable_gqa;   /* nonzero: heads_q may be a multiple of heads_kv */
+    unsigned flags;   /* DASH_FLAG_* */
+} dash_params_t;
+
+/* Bytes of device workspace dash_prefill needs for these parameters (assuming summary_k and
+ * active_blocks are passed as NULL; they are then kept in the workspace).  0 on bad
+ * parameters. */
+size_t dash_prefill_workspace_size(const dash_params_t *params);
+
+/* Whole causal prefill: Stage 0 -> Stage 1 -> Stage 2, stream-ordered, no host syncs.
+ *   q        [B, H_q, T, D]   bf16 (in)
+ *   k, v     [B, H_kv, T, D]  bf16 (in)
+ *   head_cls [H_kv, D]        fp32 (in) the learned Stage 0 query of each KV head
+ *   out      [B, H_q, T, D]   bf16 (out)
+ *   summary_k [B, H_kv, T/Bc, D] fp32 (out, nullable) the chunk-representation cache
+ *   p        [B, H_kv, T, C]  fp32 (out, nullable) routing probabilities, C = ceil(T/Bc);
+ *            0 for c >= c_t and for inactive chunks (p[.., c_t] = 0: the diagonal is not
+ *            routed)
+ *   active_blocks [B, H_kv, T, W] uint64 (out, nullable), W = ceil(C/64); bit c % 64 of word
+ *            c / 64 (LSB first) is set iff chunk c is attended by row t (routed-active or
+ *            the diagonal); bits above c_t are 0
+ *   ws, ws_bytes: device workspace of at least dash_prefill_workspace_size(params) bytes;
+ *            its first 256 bytes hold the device status word (cleared by this call)
+ * Returns DASH_OK when every launch was issued. */
+dash_status_t dash_prefill(const dash_params_t *params, const void *q, const void *k,
+                           const void *v, const float *head_cls, void *out, float *summary_k,
+                           float *p, uint64_t *active_blocks, void *ws, size_t ws_bytes,
+                           void *stream);
+
+/* Stage 0 alone: summary_k [B, H_kv, T/Bc, D] fp32 of every complete chunk of k
+ * [B, H_kv, T, D] bf16.  Each summary is computed by one warp from a TMA (bulk-copy) staged
+ * chunk in shared memory.  ws (>= 256 bytes) holds the status word. */
+dash_status_t dash_stage0(const dash_params_t *params, const void *k, const float *head_cls,
+                          float *summary_k, void *ws, size_t ws_bytes, void *stream);
+
+/* Stage 1 alone: routing of every row from q [B,H_q,T,D] bf16 and summary_k
+ * [B,H_kv,T/Bc,D] fp32.  Writes tau [B,H_kv,T] fp32 (the entmax threshold of each row;
+ * the log-sum-exp when alpha = 1; NaN when c_t = 0), active_blocks [B,H_kv,T,W] uint64,
+ * and p [B,H_kv,T,C] fp32 when non-NULL.  ws (>= 256 bytes) holds the status word. */
+dash_status_t dash_route(const dash_params_t *params, const void *q, const float *summary_k,
+                         float *tau, float *p, uint64_t *active_blocks, void *ws,
+                         size_t ws_bytes, void *stream);
+
+/* Stage 2 alone: out [B,H_q,T,D] bf16 from q, k, v, the routing (summary_k, tau,
+ * active_blocks as written by dash_stage0 / dash_route) and the flags (DASH_FLAG_DENSE and
+ * DASH_FLAG_FORCE_ALL_ACTIVE ignore the routing, which may then be NULL).  The bias of an
+ * active chunk is recomputed from (qbar.summary, tau) bit-identically to Stage 1. */
+dash_status_t dash_attend(const dash_params_t *params, const void *q, const void *k,
+                          const void *v, const float *summary_k, const float *tau,
+                          const uint64_t *active_blocks, void *out, void *ws, size_t ws_bytes,
+                          void *stream);
+
+/* Chunk-representation cache update for decode: Stage 0 over each sequence's last n_recent
+ * complete chunks.  Idempotent (recomputing a frozen chunk writes the same bits).
+ *   k_cache       [B, H_kv, cap, D] bf16 (in), cap = params->seq_len
+ *   seq_lens      [B] int32 DEVICE (in): valid tokens per sequence, 1 <= seq_lens[b] <= cap
+ *   summary_cache [B, H_kv, cap/Bc, D] fp32 (in/out)
+ * The summaries are bit-identical to dash_stage0's for the same keys.  A seq_lens value out
+ * of range is reported through the status word in ws and that sequence is skipped. */
+dash_status_t dash_update_chunk_cache(const dash_params_t *params, const void *k_cache,
+                                      const float *head_cls, const int32_t *seq_lens,
+                                      int n_recent, float *summary_cache, void *ws,
+                                      size_t ws_bytes, void *stream);
+
+/* Bytes of device workspace dash_decode needs (status word + split partial results). */
+size_t dash_decode_workspace_size(const dash_params_t *params);
+
+/* One incremental-decode step: for each sequence b the query row is t = seq_lens[b]-1,
+ * whose K/V the caller has already written into the caches, and whose routable chunks
+ * (c < t / Bc) have summaries in summary_cache (see dash_update_chunk_cache).
+ *   q            [B, H_q, D] bf16 (in)
+ *   k_cache, v_cache [B, H_kv, cap, D] bf16 (in)
+ *   seq_lens     [B] int32 DEVICE (in)
+ *   summary_cache [B, H_kv, cap/Bc, D] fp32 (in)
+ *   out          [B, H_q, D] bf16 (out)
+ *   p            [B, H_kv, Ccap] fp32 (out, nullable), Ccap = ceil(cap/Bc)
+ *   active_blocks [B, H_kv, Wcap] uint64 (out, nullable), Wcap = ceil(Ccap/64)
+ * Same arithmetic as row t of dash_prefill.  One thread-block cluster per (b, g) routes
+ * and attends; no host sync, so a loop of steps can be captured in one CUDA graph. */
+dash_status_t dash_decode(const dash_params_t *params, const void *q, const void *k_cache,
+                          const void *v_cache, const int32_t *seq_lens,
+                          const float *summary_cache, void *out, float *p,
+                          uint64_t *active_blocks, void *ws, size_t ws_bytes, void *stream);
+
+/* Synchronises `stream`, then returns the status word the kernels wrote into ws (DASH_OK if
+ * none) and clears it.  Returns DASH_ERR_CUDA if the copy itself fails. */
+dash_status_t dash_read_device_status(void *ws, void *stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *dash_status_string(dash_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DASH_H_ */

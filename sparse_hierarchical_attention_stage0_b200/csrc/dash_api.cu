@@ -1,0 +1,337 @@
+// dash_api.cu -- the C ABI declared in include/dash.h: host-side argument checks, workspace
+// carving and stream-ordered launches.  Nothing here allocates device memory or keeps
+// global state; every failure is reported before the first launch of a call.
+#include <cmath>
+#include <cstdint>
+
+#include "kernels.cuh"
+
+using namespace dash;
+
+namespace {
+
+constexpr size_t kStatusBytes = 256;
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Shape {
+    int B, Hq, Hkv, T, D, Bc, G, C, Cf, W;
+};
+
+// Checks shared by every entry point.  `decode`: seq_len is a cache capacity.
+dash_status_t check_params(const dash_params_t *p, Shape *s) {
+    if (!p) return DASH_ERR_INVALID_ARGUMENT;
+    if (p->batch < 1 || p->heads_q < 1 || p->heads_kv < 1 || p->seq_len < 1 ||
+        p->head_dim < 1 || p->chunk_size < 1)
+        return DASH_ERR_INVALID_ARGUMENT;
+    if (p->heads_q % p->heads_kv != 0) return DASH_ERR_INVALID_ARGUMENT;
+    if (!p->enable_gqa && p->heads_q != p->heads_kv) return DASH_ERR_INVALID_ARGUMENT;
+    if (!std::isfinite(p->alpha) || p->alpha < 1.f) return DASH_ERR_INVALID_ARGUMENT;
+    if (!std::isfinite(p->gamma) || !(p->gamma > 0.f)) return DASH_ERR_INVALID_ARGUMENT;
+    if (!std::isfinite(p->sigma) || p->sigma < 0.f) return DASH_ERR_INVALID_ARGUMENT;
+    if (p->flags & ~7u) return DASH_ERR_INVALID_ARGUMENT;
+    if (p->flags & DASH_FLAG_ESTIMATE_DIAGONAL) return DASH_ERR_UNSUPPORTED;
+    if (p->head_dim != 64 && p->head_dim != 128) return DASH_ERR_UNSUPPORTED;
+    if (p->chunk_size != 64 && p->chunk_size != 128) return DASH_ERR_UNSUPPORTED;
+    const int G = p->heads_q / p->heads_kv;
+    if (!(G >= 16 ? G % 16 == 0 : 16 % G == 0)) return DASH_ERR_UNSUPPORTED;
+    // Element counts must stay well inside 64-bit indexing and grid limits.
+    const double elems = (double)p->batch * p->heads_q * p->seq_len * p->head_dim;
+    if (elems > 4e15 || (double)p->batch * p->heads_kv > 65535.0) return DASH_ERR_UNSUPPORTED;
+    s->B = p->batch;
+    s->Hq = p->heads_q;
+    s->Hkv = p->heads_kv;
+    s->T = p->seq_len;
+    s->D = p->head_dim;
+    s->Bc = p->chunk_size;
+    s->G = G;
+    s->C = (p->seq_len + p->chunk_size - 1) / p->chunk_size;
+    s->Cf = p->seq_len / p->chunk_size;
+    s->W = (s->C + 63) / 64;
+    return DASH_OK;
+}
+
+RouteConsts route_consts(const dash_params_t *p) {
+    RouteConsts rc;
+    const double a = p->alpha, g = p->gamma, sg = p->sigma, sd = std::sqrt((double)p->head_dim);
+    rc.alpha = p->alpha;
+    rc.sscale = (float)(g / sd);
+    if (a == 1.0) {
+        rc.kind = 0;
+        rc.xscale = 0.f;
+        rc.beta = 0.f;
+        rc.bscale2 = 0.f;
+    } else {
+        rc.kind = a == 1.5 ? 1 : a == 2.0 ? 2 : 3;
+        rc.xscale = (float)((a - 1.0) * g / sd);
+        rc.beta = (float)(1.0 / (a - 1.0));
+        rc.bscale2 = (float)(sg / (a - 1.0));
+    }
+    rc.sigma2 = (float)(sg * 1.4426950408889634);
+    return rc;
+}
+
+StageArgs stage_args(const dash_params_t *p, const Shape &s) {
+    StageArgs a = {};
+    a.B = s.B;
+    a.Hq = s.Hq;
+    a.Hkv = s.Hkv;
+    a.T = s.T;
+    a.D = s.D;
+    a.Bc = s.Bc;
+    a.G = s.G;
+    a.C = s.C;
+    a.Cf = s.Cf;
+    a.W = s.W;
+    a.rc = route_consts(p);
+    a.qk_scale2 = (float)(1.4426950408889634 / std::sqrt((double)s.D));
+    a.ignore_routing = (p->flags & (DASH_FLAG_DENSE | DASH_FLAG_FORCE_ALL_ACTIVE)) ? 1 : 0;
+    return a;
+}
+
+size_t bytes_tau(const Shape &s) { return align256((size_t)s.B * s.Hkv * s.T * 4); }
+size_t bytes_summary(const Shape &s) { return align256((size_t)s.B * s.Hkv * s.Cf * s.D * 4); }
+size_t bytes_mask(const Shape &s) { return align256((size_t)s.B * s.Hkv * s.T * s.W * 8); }
+
+dash_status_t clear_status(void *ws, cudaStream_t st) {
+    return cudaMemsetAsync(ws, 0, sizeof(uint32_t), st) == cudaSuccess ? DASH_OK : DASH_ERR_CUDA;
+}
+
+dash_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? DASH_OK : DASH_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char *dash_status_string(dash_status_t s) {
+    switch (s) {
+        case DASH_OK: return "DASH_OK";
+        case DASH_ERR_INVALID_ARGUMENT: return "DASH_ERR_INVALID_ARGUMENT";
+        case DASH_ERR_UNSUPPORTED: return "DASH_ERR_UNSUPPORTED";
+        case DASH_ERR_WORKSPACE_TOO_SMALL: return "DASH_ERR_WORKSPACE_TOO_SMALL";
+        case DASH_ERR_CUDA: return "DASH_ERR_CUDA";
+        case DASH_ERR_DEVICE_TIMEOUT: return "DASH_ERR_DEVICE_TIMEOUT";
+    }
+    return "DASH_ERR_UNKNOWN";
+}
+
+size_t dash_prefill_workspace_size(const dash_params_t *p) {
+    Shape s;
+    if (check_params(p, &s) != DASH_OK) return 0;
+    return kStatusBytes + bytes_tau(s) + bytes_summary(s) + bytes_mask(s);
+}
+
+dash_status_t dash_prefill(const dash_params_t *p, const void *q, const void *k, const void *v,
+                           const float *head_cls, void *out, float *summary_k, float *prob,
+                           uint64_t *active_blocks, void *ws, size_t ws_bytes, void *stream) {
+    Shape s;
+    dash_status_t rc = check_params(p, &s);
+    if (rc != DASH_OK) return rc;
+    const bool dense = (p->flags & DASH_FLAG_DENSE) != 0;
+    if (!q || !k || !v || !out || !ws) return DASH_ERR_INVALID_ARGUMENT;
+    if (!dense && !head_cls) return DASH_ERR_INVALID_ARGUMENT;
+    if (dense && (summary_k || prob || active_blocks)) return DASH_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        !aligned16(head_cls) || !aligned16(summary_k) || !aligned16(prob) ||
+        !aligned16(active_blocks) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return DASH_ERR_INVALID_ARGUMENT;
+    if (!dense && route_rows_per_cta(s.C, s.D) == 0) return DASH_ERR_UNSUPPORTED;
+    size_t need = kStatusBytes + bytes_tau(s);
+    if (!dense && !summary_k) need += bytes_summary(s);
+    if (!dense && !active_blocks) need += bytes_mask(s);
+    if (ws_bytes < need) return DASH_ERR_WORKSPACE_TOO_SMALL;
+
+    unsigned char *w = static_cast<unsigned char *>(ws);
+    StageArgs a = stage_args(p, s);
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.head_cls = head_cls;
+    a.out = out;
+    a.p = prob;
+    a.status = reinterpret_cast<uint32_t *>(w);
+    size_t off = kStatusBytes;
+    a.tau = reinterpret_cast<float *>(w + off);
+    off += bytes_tau(s);
+    if (!dense) {
+        if (summary_k) {
+            a.summary = summary_k;
+        } else {
+            a.summary = reinterpret_cast<float *>(w + off);
+            off += bytes_summary(s);
+        }
+        if (active_blocks) {
+            a.mask = active_blocks;
+        } else {
+            a.mask = reinterpret_cast<uint64_t *>(w + off);
+            off += bytes_mask(s);
+        }
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((rc = clear_status(ws, st)) != DASH_OK) return rc;
+    if (!dense) {
+        if ((rc = from_cuda(launch_stage0(a, nullptr, 0, st))) != DASH_OK) return rc;
+        if ((rc = from_cuda(launch_route(a, st))) != DASH_OK) return rc;
+    }
+    return from_cuda(launch_attend(a, st));
+}
+
+dash_status_t dash_stage0(const dash_params_t *p, const void *k, const float *head_cls,
+                          float *summary_k, void *ws, size_t ws_bytes, void *stream) {
+    Shape s;
+    dash_status_t rc = check_params(p, &s);
+    if (rc != DASH_OK) return rc;
+    if (!k || !head_cls || !summary_k || !ws) return DASH_ERR_INVALID_ARGUMENT;
+    if (!aligned16(k) || !aligned16(head_cls) || !aligned16(summary_k) ||
+        (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return DASH_ERR_INVALID_ARGUMENT;
+    if (ws_bytes < kStatusBytes) return DASH_ERR_WORKSPACE_TOO_SMALL;
+    StageArgs a = stage_args(p, s);
+    a.k = k;
+    a.head_cls = head_cls;
+    a.summary = summary_k;
+    a.status = static_cast<uint32_t *>(ws);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((rc = clear_status(ws, st)) != DASH_OK) return rc;
+    return from_cuda(launch_stage0(a, nullptr, 0, st));
+}
+
+dash_status_t dash_route(const dash_params_t *p, const void *q, const float *summary_k,
+                         float *tau, float *prob, uint64_t *active_blocks, void *ws,
+                         size_t ws_bytes, void *stream) {
+    Shape s;
+    dash_status_t rc = check_params(p, &s);
+    if (rc != DASH_OK) return rc;
+    if (!q || !summary_k || !tau || !active_blocks || !ws) return DASH_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q) || !aligned16(summary_k) || !aligned16(tau) || !aligned16(prob) ||
+        !aligned16(active_blocks) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return DASH_ERR_INVALID_ARGUMENT;
+    if (route_rows_per_cta(s.C, s.D) == 0) return DASH_ERR_UNSUPPORTED;
+    if (ws_bytes < kStatusBytes) return DASH_ERR_WORKSPACE_TOO_SMALL;
+    StageArgs a = stage_args(p, s);
+    a.q = q;
+    a.summary = const_cast<float *>(summary_k);
+    a.tau = tau;
+    a.p = prob;
+    a.mask = active_blocks;
+    a.status = static_cast<uint32_t *>(ws);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((rc = clear_status(ws, st)) != DASH_OK) return rc;
+    return from_cuda(launch_route(a, st));
+}
+
+dash_status_t dash_attend(const dash_params_t *p, const void *q, const void *k, const void *v,
+                          const float *summary_k, const float *tau,
+                          const uint64_t *active_blocks, void *out, void *ws, size_t ws_bytes,
+                          void *stream) {
+    Shape s;
+    dash_status_t rc = check_params(p, &s);
+    if (rc != DASH_OK) return rc;
+    const bool ignore = (p->flags & (DASH_FLAG_DENSE | DASH_FLAG_FORCE_ALL_ACTIVE)) != 0;
+    if (!q || !k || !v || !out || !ws) return DASH_ERR_INVALID_ARGUMENT;
+    if (!ignore && (!summary_k || !tau || !active_blocks)) return DASH_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        !aligned16(summary_k) || !aligned16(tau) || !aligned16(active_blocks) ||
+        (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return DASH_ERR_INVALID_ARGUMENT;
+    if (ws_bytes < kStatusBytes) return DASH_ERR_WORKSPACE_TOO_SMALL;
+    StageArgs a = stage_args(p, s);
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.out = out;
+    a.summary = const_cast<float *>(summary_k);
+    a.tau = const_cast<float *>(tau);
+    a.mask = const_cast<uint64_t *>(active_blocks);
+    a.status = static_cast<uint32_t *>(ws);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((rc = clear_status(ws, st)) != DASH_OK) return rc;
+    return from_cuda(launch_attend(a, st));
+}
+
+dash_status_t dash_update_chunk_cache(const dash_params_t *p, const void *k_cache,
+                                      const float *head_cls, const int32_t *seq_lens,
+                                      int n_recent, float *summary_cache, void *ws,
+                                      size_t ws_bytes, void *stream) {
+    Shape s;
+    dash_status_t rc = check_params(p, &s);
+    if (rc != DASH_OK) return rc;
+    if (!k_cache || !head_cls || !seq_lens || !summary_cache || !ws || n_recent < 1)
+        return DASH_ERR_INVALID_ARGUMENT;
+    if (!aligned16(k_cache) || !aligned16(head_cls) || !aligned16(summary_cache) ||
+        (reinterpret_cast<uintptr_t>(seq_lens) & 3u) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return DASH_ERR_INVALID_ARGUMENT;
+    if (ws_bytes < kStatusBytes) return DASH_ERR_WORKSPACE_TOO_SMALL;
+    StageArgs a = stage_args(p, s);
+    a.k = k_cache;
+    a.head_cls = head_cls;
+    a.summary = summary_cache;
+    a.status = static_cast<uint32_t *>(ws);
+    if (n_recent > s.Cf) n_recent = s.Cf > 0 ? s.Cf : 1;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((rc = clear_status(ws, st)) != DASH_OK) return rc;
+    if (s.Cf == 0) return DASH_OK;
+    return from_cuda(launch_stage0(a, seq_lens, n_recent, st));
+}
+
+size_t dash_decode_workspace_size(const dash_params_t *p) {
+    Shape s;
+    if (check_params(p, &s) != DASH_OK) return 0;
+    return kStatusBytes;
+}
+
+dash_status_t dash_decode(const dash_params_t *p, const void *q, const void *k_cache,
+                          const void *v_cache, const int32_t *seq_lens,
+                          const float *summary_cache, void *out, float *prob,
+                          uint64_t *active_blocks, void *ws, size_t ws_bytes, void *stream) {
+    Shape s;
+    dash_status_t rc = check_params(p, &s);
+    if (rc != DASH_OK) return rc;
+    if (p->flags & (DASH_FLAG_DENSE | DASH_FLAG_FORCE_ALL_ACTIVE)) return DASH_ERR_UNSUPPORTED;
+    if (!q || !k_cache || !v_cache || !seq_lens || !summary_cache || !out || !ws)
+        return DASH_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(summary_cache) ||
+        !aligned16(out) || !aligned16(prob) || !aligned16(active_blocks) ||
+        (reinterpret_cast<uintptr_t>(seq_lens) & 3u) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return DASH_ERR_INVALID_ARGUMENT;
+    if (!decode_supported(s.G, s.C, s.D)) return DASH_ERR_UNSUPPORTED;
+    if (ws_bytes < kStatusBytes) return DASH_ERR_WORKSPACE_TOO_SMALL;
+    DecodeArgs a = {};
+    a.q = q;
+    a.k = k_cache;
+    a.v = v_cache;
+    a.seq_lens = seq_lens;
+    a.summary = summary_cache;
+    a.out = out;
+    a.p = prob;
+    a.mask = active_blocks;
+    a.B = s.B;
+    a.Hq = s.Hq;
+    a.Hkv = s.Hkv;
+    a.cap = s.T;
+    a.D = s.D;
+    a.Bc = s.Bc;
+    a.G = s.G;
+    a.Ccap = s.C;
+    a.Cf = s.Cf;
+    a.Wcap = s.W;
+    a.rc = route_consts(p);
+    a.qk_scale2 = (float)(1.4426950408889634 / std::sqrt((double)s.D));
+    a.status = static_cast<uint32_t *>(ws);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((rc = clear_status(ws, st)) != DASH_OK) return rc;
+    return from_cuda(launch_decode(a, st));
+}
+
+dash_status_t dash_read_device_status(void *ws, void *stream) {
+    if (!ws) return DASH_ERR_INVALID_ARGUMENT;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return DASH_ERR_CUDA;
+    uint32_t v = 0;
+    if (cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return DASH_ERR_CUDA;
+    if (v != 0 && cudaMemset(ws, 0, sizeof(uint32_t)) != cudaSuccess) return DASH_ERR_CUDA;
+    return static_cast<dash_status_t>(v);
+}
+
+}  // extern "C"

@@ -1,0 +1,272 @@
+// dash_common.cuh -- device helpers shared by the libdash kernels (sm_100a).
+//
+// The routing arithmetic (group-mean query, routing dot product, entmax threshold) lives
+// here once, so that Stage 1 (dash_route), Stage 2 (dash_attend, which recomputes the bias
+// of each active chunk) and decode produce bit-identical values: every dot product is the
+// same sequential chain of fmaf over d = 0..D-1, every mean the same ordered sum.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/dash.h"
+
+namespace dash {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr unsigned kFull = 0xffffffffu;
+// Spin limit of every bounded device wait (each try_wait may itself sleep up to a
+// hardware time slice), and iteration cap of the entmax Newton solve.
+constexpr int kMaxSpin = 1 << 24;
+constexpr int kNewtonCap = 96;
+
+// ---------------------------------------------------------------- status word
+// The first 4 bytes of every workspace; the first error code written wins.
+__device__ __forceinline__ void report(uint32_t *status, uint32_t code) {
+    if (status) atomicCAS(status, 0u, code);
+}
+
+// ---------------------------------------------------------------- warp reductions
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+    return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+    return v;
+}
+__device__ __forceinline__ int warp_sum_i(int v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+    return v;
+}
+
+// ---------------------------------------------------------------- smem / async copies
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// 16-byte cp.async (L2 only); src_bytes = 0 fills zeros without reading global memory.
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem)),
+                 "l"(gmem), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// mbarrier + bulk (TMA engine) copy global -> shared.
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_g2s(void *smem, const void *gmem, uint32_t bytes,
+                                         uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, "
+        "[%3];\n" ::"r"(smem_u32(smem)),
+        "l"(gmem), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait on an mbarrier phase; false if the spin limit ran out.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
+    for (int i = 0; i < kMaxSpin; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
+// ---------------------------------------------------------------- ldmatrix / mma.sync
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void *smem) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(smem)));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void *smem) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_u32(smem)));
+}
+// D += A(16x16 bf16, row) * B(16x8 bf16, col), fp32 accumulate.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
+                                               uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, "
+        "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+// 2^x on the SFU (used only for attention probabilities, which are rounded to bf16).
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// ---------------------------------------------------------------- routing arithmetic
+// Group-mean query element: (sum_{h<G} q_h) / G, summed in head order.
+__device__ __forceinline__ float group_mean_elem(const __nv_bfloat16 *q0, long long head_stride,
+                                                 int G) {
+    float s = 0.f;
+    for (int h = 0; h < G; ++h) s += __bfloat162float(q0[h * head_stride]);
+    return s / (float)G;
+}
+
+// Routing dot product qbar . S_c as ONE sequential fmaf chain over d = 0..D-1.
+template <int D>
+__device__ __forceinline__ float route_dot(const float *qbar, const float *srow) {
+    float acc = 0.f;
+    const float4 *s4 = reinterpret_cast<const float4 *>(srow);
+    const float4 *q4 = reinterpret_cast<const float4 *>(qbar);
+#pragma unroll 8
+    for (int i = 0; i < D / 4; ++i) {
+        float4 s = __ldg(s4 + i);
+        float4 q = q4[i];
+        acc = fmaf(q.x, s.x, acc);
+        acc = fmaf(q.y, s.y, acc);
+        acc = fmaf(q.z, s.z, acc);
+        acc = fmaf(q.w, s.w, acc);
+    }
+    return acc;
+}
+
+// Constants of the routing, computed once on the host.
+struct RouteConsts {
+    float xscale;     // (alpha-1) * gamma / sqrt(D): x_c = dot * xscale (alpha > 1)
+    float sscale;     // gamma / sqrt(D): s_c = dot * sscale (alpha = 1)
+    float alpha;
+    float beta;       // 1 / (alpha-1)  (alpha > 1)
+    float bscale2;    // log2 of the prior: bias2 = bscale2 * log2(m) with bscale2 = sigma*beta
+    float sigma2;     // sigma * log2(e) (alpha = 1: bias2 = sigma2 * (s - lse))
+    int kind;         // 0: softmax (alpha = 1), 1: alpha = 1.5, 2: alpha = 2, 3: other alpha
+};
+
+// m^beta for the entmax probability of margin m > 0.
+__device__ __forceinline__ float pow_beta(float m, const RouteConsts &rc) {
+    if (rc.kind == 1) return m * m;
+    if (rc.kind == 2) return m;
+    return powf(m, rc.beta);
+}
+__device__ __forceinline__ float pow_beta_m1(float m, const RouteConsts &rc) {
+    if (rc.kind == 1) return m;
+    if (rc.kind == 2) return 1.f;
+    return powf(m, rc.beta - 1.f);
+}
+
+// Entmax threshold of one row held in (shared) memory xs[0..n), n >= 1, all 32 lanes of
+// the warp calling.  For alpha = 1 returns the log-sum-exp of the scores.  Otherwise x are
+// the scaled scores (alpha-1) s and the return value is tau with
+// sum_c [x_c - tau]_+^beta = 1.  For beta >= 1 (alpha <= 2) Newton's method from
+// tau0 = max x - 1 increases monotonically to the root (f is convex and decreasing); the
+// support it settles on is then fed to the exact closed form for alpha = 1.5 and 2.  For
+// alpha > 2, bisection on [max - 1, max - n^(1-alpha)].  The lane-strided sums and butterfly
+// reductions fix the summation order, so every caller gets the same bits.
+static __device__ __noinline__ float warp_entmax_tau(const float *xs, int n, const RouteConsts &rc,
+                                              uint32_t *status) {
+    const int lane = threadIdx.x & 31;
+    float mx = -INFINITY;
+    for (int c = lane; c < n; c += 32) mx = fmaxf(mx, xs[c]);
+    mx = warp_max(mx);
+    if (rc.kind == 0) {
+        float s = 0.f;
+        for (int c = lane; c < n; c += 32) s += expf(xs[c] - mx);
+        s = warp_sum(s);
+        return mx + logf(s);
+    }
+    float tau;
+    if (rc.beta >= 1.f) {
+        tau = mx - 1.f;
+        int it = 0;
+        for (; it < kNewtonCap; ++it) {
+            float f = 0.f, df = 0.f;
+            for (int c = lane; c < n; c += 32) {
+                float m = xs[c] - tau;
+                if (m > 0.f) {
+                    f += pow_beta(m, rc);
+                    df += pow_beta_m1(m, rc);
+                }
+            }
+            f = warp_sum(f);
+            df = warp_sum(df);
+            float step = (f - 1.f) / (rc.beta * df);
+            if (!(step > 0.f)) break;                 // at (or rounded past) the root
+            float nt = tau + step;
+            if (nt == tau) break;
+            tau = nt;
+            if (step <= 1e-7f * fmaxf(1.f, fabsf(tau))) break;
+        }
+        if (it == kNewtonCap) report(status, DASH_ERR_DEVICE_TIMEOUT);
+    } else {
+        float lo = mx - 1.f, hi = mx - powf((float)n, 1.f - rc.alpha);
+        for (int it = 0; it < 40; ++it) {
+            float mid = 0.5f * (lo + hi), f = 0.f;
+            for (int c = lane; c < n; c += 32) {
+                float m = xs[c] - mid;
+                if (m > 0.f) f += pow_beta(m, rc);
+            }
+            f = warp_sum(f);
+            if (f >= 1.f) lo = mid; else hi = mid;
+        }
+        tau = 0.5f * (lo + hi);
+    }
+    if (rc.kind == 1 || rc.kind == 2) {
+        // Exact closed form on the support {x > tau}; repeat while the support moves.
+        for (int rep = 0; rep < 4; ++rep) {
+            float sx = 0.f;
+            int k = 0;
+            for (int c = lane; c < n; c += 32)
+                if (xs[c] > tau) { sx += xs[c]; ++k; }
+            sx = warp_sum(sx);
+            k = warp_sum_i(k);
+            if (k == 0) break;
+            float nt;
+            if (rc.kind == 2) {
+                nt = (sx - 1.f) / (float)k;
+            } else {
+                float mean = sx / (float)k, m2 = 0.f;
+                for (int c = lane; c < n; c += 32)
+                    if (xs[c] > tau) { float d = xs[c] - mean; m2 = fmaf(d, d, m2); }
+                m2 = warp_sum(m2);
+                nt = mean - sqrtf(fmaxf(1.f - m2, 0.f) / (float)k);
+            }
+            // Same support under the new threshold?  Then it is the fixed point.
+            int moved = 0;
+            for (int c = lane; c < n; c += 32) moved |= ((xs[c] > tau) != (xs[c] > nt));
+            moved = __any_sync(kFull, moved);
+            tau = nt;
+            if (!moved) break;
+        }
+    }
+    return tau;
+}
+
+}  // namespace dash

@@ -1,0 +1,334 @@
+// decode.cu -- one incremental-decode step: Stage 1 routing and Stage 2 attention for the
+// newest token of every sequence, in a single launch.
+//
+// liuzhao09.github.io "DashAttention 精读", section 2: the three stages support incremental
+// decoding with a chunk-representation cache; gist.science "DashAttention ...", Technische
+// Zusammenfassung, "Stufe 0": complete chunks' summaries are frozen and cached (the cache is
+// maintained by dash_update_chunk_cache).  Decode is memory-bound: the step reads the
+// cached summaries and the active chunks' K/V once.
+//
+// One thread-block cluster of kDecCluster CTAs per (b, g):
+//   1. every CTA builds qbar; CTA r scores the r-th slice of the routable chunks
+//      (x_c = qbar . summary_c * (alpha-1) gamma / sqrt(D), same arithmetic as prefill);
+//   2. cluster barrier, then each CTA pulls the other slices through distributed shared
+//      memory (mapa + ld.shared::cluster), so every CTA holds the whole score row;
+//   3. every CTA solves the same tau (same code and data -> same bits); rank 0 writes the
+//      optional p row and mask words;
+//   4. the active chunks (+ the diagonal chunk, last) are dealt round-robin to the
+//      cluster's warps; each warp runs the 16-row mma.sync attention over its share;
+//   5. warp partials (max, sum, O) are merged inside the CTA, then across the cluster by
+//      rank 0 through distributed shared memory, which writes the bf16 output.
+#include "attn_warp.cuh"
+
+namespace dash {
+
+constexpr int kDecCluster = 8;
+constexpr int kDecWarps = 4;
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n"
+                 "barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+// Address of the same shared-memory variable in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t map_rank(const void *p, uint32_t rank) {
+    uint32_t out;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(out) : "r"(smem_u32(p)), "r"(rank));
+    return out;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];\n" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+int decode_supported(int G, int Ccap, int D) {
+    (void)D;
+    return G >= 1 && G <= 16 && 16 % G == 0 && Ccap <= 8192;
+}
+
+// Shared-memory layout of one decode CTA (byte offsets).
+template <int D>
+struct DecLayout {
+    static constexpr size_t tile = (size_t)kSub * D * 2;          // one K or V tile
+    static constexpr size_t warp_tiles = 2 * tile;                 // >= a warp partial
+    static constexpr size_t part = 16 * D * 4 + 2 * 16 * 4;        // O[16][D], m[16], l[16]
+    static_assert(warp_tiles >= part, "warp partial must fit in the warp's tiles");
+    size_t qbar, cta_part, tiles, xs, list, total;
+    __host__ __device__ DecLayout(int Ccap) {
+        qbar = 0;
+        cta_part = qbar + D * 4;
+        tiles = cta_part + part;
+        tiles = (tiles + 127) & ~(size_t)127;
+        xs = tiles + kDecWarps * warp_tiles;
+        list = xs + (size_t)((Ccap + 3) & ~3) * 4;
+        total = list + (size_t)(Ccap + 2) * 4;
+    }
+};
+
+template <int D, int BC>
+__global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    __shared__ float tau_s;
+    __shared__ int nact_s;
+    const DecLayout<D> L(a.Ccap);
+    float *qbar = reinterpret_cast<float *>(smem_raw + L.qbar);
+    float *cpart = reinterpret_cast<float *>(smem_raw + L.cta_part);   // O[16][D], m, l
+    float *xs = reinterpret_cast<float *>(smem_raw + L.xs);
+    int *list = reinterpret_cast<int *>(smem_raw + L.list);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = cluster_rank();
+    const int bg = blockIdx.x / kDecCluster, b = bg / a.Hkv, g = bg % a.Hkv;
+    const int G = a.G;
+    const int Lb = a.seq_lens[b];
+    if (Lb < 1 || Lb > a.cap) {                 // uniform across the cluster: no barrier
+        if (tid == 0 && rank == 0) report(a.status, DASH_ERR_INVALID_ARGUMENT);
+        return;
+    }
+    const int t = Lb - 1, ct = t / BC, n = ct;
+    const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(a.q) + (long long)b * a.Hq * D;
+
+    // 1. group-mean query and this CTA's slice of the scores.
+    for (int d = tid; d < D; d += kDecWarps * 32)
+        qbar[d] = group_mean_elem(q + (long long)g * G * D + d, D, G);
+    __syncthreads();
+    const float scale = a.rc.kind == 0 ? a.rc.sscale : a.rc.xscale;
+    const int c_lo = (int)((long long)n * rank / kDecCluster);
+    const int c_hi = (int)((long long)n * (rank + 1) / kDecCluster);
+    const float *sumg = a.summary + (long long)bg * a.Cf * D;
+    for (int c = c_lo + tid; c < c_hi; c += kDecWarps * 32)
+        xs[c] = __fmul_rn(route_dot<D>(qbar, sumg + (long long)c * D), scale);
+
+    // 2. exchange slices through distributed shared memory.
+    cluster_sync_all();
+    for (uint32_t r = 0; r < kDecCluster; ++r) {
+        if (r == rank) continue;
+        const int lo = (int)((long long)n * r / kDecCluster);
+        const int hi = (int)((long long)n * (r + 1) / kDecCluster);
+        for (int c = lo + tid; c < hi; c += kDecWarps * 32) xs[c] = ld_cluster_f32(map_rank(&xs[c], r));
+    }
+    __syncthreads();
+
+    // 3. threshold (every CTA, same bits) and the routing outputs (rank 0).
+    if (warp == 0) {
+        float tau = n > 0 ? warp_entmax_tau(xs, n, a.rc, a.status) : __int_as_float(0x7fc00000);
+        if (lane == 0) tau_s = tau;
+    }
+    __syncthreads();
+    const float tau = tau_s;
+    auto active = [&](int c) -> bool {
+        return c < n && (a.rc.kind == 0 || __fsub_rn(xs[c], tau) > 0.f);
+    };
+    if (rank == 0) {
+        if (a.mask) {
+            for (int w = warp; w < a.Wcap; w += kDecWarps) {
+                const int c0 = w * 64 + lane, c1 = c0 + 32;
+                unsigned lo = __ballot_sync(kFull, c0 == ct || active(c0));
+                unsigned hi = __ballot_sync(kFull, c1 == ct || active(c1));
+                if (lane == 0) a.mask[(long long)bg * a.Wcap + w] = ((uint64_t)hi << 32) | lo;
+            }
+        }
+        if (a.p) {
+            for (int c = tid; c < a.Ccap; c += kDecWarps * 32) {
+                float val = 0.f;
+                if (active(c)) {
+                    const float m = __fsub_rn(xs[c], tau);
+                    val = a.rc.kind == 0 ? expf(xs[c] - tau) : pow_beta(m, a.rc);
+                }
+                a.p[(long long)bg * a.Ccap + c] = val;
+            }
+        }
+    }
+
+    // 4. active list (same on every CTA): routed chunks ascending, then the diagonal.
+    if (warp == 0) {
+        int pos = 0;
+        for (int c0 = 0; c0 < n; c0 += 32) {
+            const int c = c0 + lane;
+            const bool act = active(c);
+            const unsigned bal = __ballot_sync(kFull, act);
+            if (act) list[pos + __popc(bal & ((1u << lane) - 1u))] = c;
+            pos += __popc(bal);
+        }
+        if (lane == 0) {
+            list[pos] = ct;
+            nact_s = pos + 1;
+        }
+    }
+    __syncthreads();
+    const int nact = nact_s;
+
+    // Attention over this warp's share: entries i with i % NC == rank, (i / NC) % W == warp.
+    unsigned char *ks = smem_raw + L.tiles + warp * L.warp_tiles;
+    unsigned char *vs = ks + L.tile;
+    const __nv_bfloat16 *kp = reinterpret_cast<const __nv_bfloat16 *>(a.k) + (long long)bg * a.cap * D;
+    const __nv_bfloat16 *vp = reinterpret_cast<const __nv_bfloat16 *>(a.v) + (long long)bg * a.cap * D;
+    const int r_lo = lane >> 2, r_hi = r_lo + 8, qd = lane & 3;
+    const bool ok_lo = r_lo < G, ok_hi = r_hi < G;
+    uint32_t qf[D / 16][4];
+    {
+        const __nv_bfloat16 *q_lo = q + (long long)(g * G + (ok_lo ? r_lo : 0)) * D;
+        const __nv_bfloat16 *q_hi = q + (long long)(g * G + (ok_hi ? r_hi : 0)) * D;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const int d0 = 16 * kk + 2 * qd;
+            qf[kk][0] = ok_lo ? *reinterpret_cast<const uint32_t *>(q_lo + d0) : 0u;
+            qf[kk][1] = ok_hi ? *reinterpret_cast<const uint32_t *>(q_hi + d0) : 0u;
+            qf[kk][2] = ok_lo ? *reinterpret_cast<const uint32_t *>(q_lo + d0 + 8) : 0u;
+            qf[kk][3] = ok_hi ? *reinterpret_cast<const uint32_t *>(q_hi + d0 + 8) : 0u;
+        }
+    }
+    UnitState<D> st;
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) st.o[j][e] = 0.f;
+    st.m_lo = st.m_hi = -INFINITY;
+    st.l_lo = st.l_hi = 0.f;
+
+    constexpr int NSUB = BC / kSub;
+    const int stride = kDecCluster * kDecWarps;
+    const int first = (int)rank + kDecCluster * warp;
+    const int my_n = first < nact ? (nact - first + stride - 1) / stride : 0;
+    const int nsteps = my_n * NSUB;
+    if (nsteps > 0) {
+        load_sub<D>(ks, kp, list[first] * BC, a.cap);
+        cp_async_commit();
+        load_sub<D>(vs, vp, list[first] * BC, a.cap);
+        cp_async_commit();
+    }
+    for (int s = 0; s < nsteps; ++s) {
+        const int c = list[first + (s / NSUB) * stride];
+        const int key0 = c * BC + (s % NSUB) * kSub;
+        const bool diag = c == ct, more = s + 1 < nsteps;
+        const int key_next = more ? list[first + ((s + 1) / NSUB) * stride] * BC + ((s + 1) % NSUB) * kSub : 0;
+        float bias2 = 0.f;
+        if (!diag)
+            bias2 = a.rc.kind == 0 ? a.rc.sigma2 * (xs[c] - tau)
+                                   : a.rc.bscale2 * log2f(fmaxf(__fsub_rn(xs[c], tau), 1e-37f));
+        cp_async_wait<1>();
+        __syncwarp();
+        float acc[4][4];
+        qk_sub<D>(acc, qf, ks);
+        __syncwarp();
+        if (more) {
+            load_sub<D>(ks, kp, key_next, a.cap);
+            cp_async_commit();
+        }
+        uint32_t pa[2][4];
+        softmax_sub<D>(st, acc, pa, a.qk_scale2, ok_lo ? bias2 : -INFINITY,
+                       ok_hi ? bias2 : -INFINITY, diag, key0, t, t);
+        if (more) cp_async_wait<1>(); else cp_async_wait<0>();
+        __syncwarp();
+        pv_sub<D>(st, pa, vs);
+        __syncwarp();
+        if (more) {
+            load_sub<D>(vs, vp, key_next, a.cap);
+            cp_async_commit();
+        }
+    }
+
+    // 5a. warp partial -> the warp's own tile space.
+    float l_lo = st.l_lo, l_hi = st.l_hi;
+    l_lo += __shfl_xor_sync(kFull, l_lo, 1);
+    l_lo += __shfl_xor_sync(kFull, l_lo, 2);
+    l_hi += __shfl_xor_sync(kFull, l_hi, 1);
+    l_hi += __shfl_xor_sync(kFull, l_hi, 2);
+    float *wp = reinterpret_cast<float *>(ks);          // O[16][D], m[16], l[16]
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) {
+        const int d0 = 8 * j + 2 * qd;
+        wp[r_lo * D + d0] = st.o[j][0];
+        wp[r_lo * D + d0 + 1] = st.o[j][1];
+        wp[r_hi * D + d0] = st.o[j][2];
+        wp[r_hi * D + d0 + 1] = st.o[j][3];
+    }
+    if (qd == 0) {
+        wp[16 * D + r_lo] = st.m_lo;
+        wp[16 * D + r_hi] = st.m_hi;
+        wp[16 * D + 16 + r_lo] = l_lo;
+        wp[16 * D + 16 + r_hi] = l_hi;
+    }
+    __syncthreads();
+
+    // 5b. CTA merge of the warp partials into cpart.
+    for (int idx = tid; idx < 16 * D + 16; idx += kDecWarps * 32) {
+        const int r = idx < 16 * D ? idx / D : idx - 16 * D;
+        float mstar = -INFINITY;
+        for (int w = 0; w < kDecWarps; ++w)
+            mstar = fmaxf(mstar, reinterpret_cast<float *>(smem_raw + L.tiles + w * L.warp_tiles)[16 * D + r]);
+        const float mu = mstar == -INFINITY ? 0.f : mstar;
+        float acc = 0.f;
+        for (int w = 0; w < kDecWarps; ++w) {
+            const float *pw = reinterpret_cast<float *>(smem_raw + L.tiles + w * L.warp_tiles);
+            const float f = fast_exp2(pw[16 * D + r] - mu);
+            acc += f * (idx < 16 * D ? pw[idx] : pw[16 * D + 16 + r]);
+        }
+        if (idx < 16 * D) cpart[idx] = acc;
+        else { cpart[16 * D + r] = mstar; cpart[16 * D + 16 + r] = acc; }
+    }
+
+    // 5c. cluster merge by rank 0 through distributed shared memory.
+    cluster_sync_all();
+    if (rank == 0) {
+        __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(a.out) + ((long long)b * a.Hq + g * G) * D;
+        for (int idx = tid; idx < G * D; idx += kDecWarps * 32) {
+            const int r = idx / D;
+            float mr[kDecCluster], mstar = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < kDecCluster; ++k) {
+                mr[k] = ld_cluster_f32(map_rank(&cpart[16 * D + r], k));
+                mstar = fmaxf(mstar, mr[k]);
+            }
+            const float mu = mstar == -INFINITY ? 0.f : mstar;
+            float o = 0.f, l = 0.f;
+#pragma unroll
+            for (int k = 0; k < kDecCluster; ++k) {
+                const float f = fast_exp2(mr[k] - mu);
+                o += f * ld_cluster_f32(map_rank(&cpart[idx], k));
+                l += f * ld_cluster_f32(map_rank(&cpart[16 * D + 16 + r], k));
+            }
+            out[idx] = __float2bfloat16_rn(o / l);
+        }
+    }
+    cluster_sync_all();      // peers stay resident until rank 0 has read their partials
+}
+
+template <int D, int BC>
+static cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t st) {
+    const DecLayout<D> L(a.Ccap);
+    auto kern = k_decode<D, BC>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)L.total);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(a.B * a.Hkv * kDecCluster));
+    cfg.blockDim = dim3(kDecWarps * 32);
+    cfg.dynamicSmemBytes = L.total;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kDecCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, a);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st) {
+    if (a.D == 128 && a.Bc == 64) return launch_decode_t<128, 64>(a, st);
+    if (a.D == 128 && a.Bc == 128) return launch_decode_t<128, 128>(a, st);
+    if (a.D == 64 && a.Bc == 64) return launch_decode_t<64, 64>(a, st);
+    if (a.D == 64 && a.Bc == 128) return launch_decode_t<64, 128>(a, st);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace dash

@@ -1,0 +1,50 @@
+// kernels.cuh -- launch interfaces between the C ABI (dash_api.cu) and the kernels.
+#pragma once
+
+#include "dash_common.cuh"
+
+namespace dash {
+
+constexpr int kStage0Warps = 4;     // chunks summarised per CTA
+constexpr int kRouteThreads = 256;  // Stage 1 CTA size
+constexpr int kAttnWarps = 4;       // Stage 2 (mma.sync path) units per CTA
+constexpr int kSub = 32;            // keys per Stage 2 sub-block
+
+// Everything one prefill stage needs; pointers the stage does not use may be null.
+struct StageArgs {
+    const void *q, *k, *v;
+    const float *head_cls;
+    float *summary;           // [B,Hkv,Cf,D]
+    float *tau;               // [B,Hkv,T]
+    float *p;                 // [B,Hkv,T,C] or null
+    uint64_t *mask;           // [B,Hkv,T,W]
+    void *out;                // [B,Hq,T,D]
+    int B, Hq, Hkv, T, D, Bc, G, C, Cf, W;
+    RouteConsts rc;
+    float qk_scale2;          // log2(e) / sqrt(D)
+    int ignore_routing;       // DENSE or FORCE_ALL_ACTIVE: attend every chunk, bias 0
+    uint32_t *status;
+};
+
+struct DecodeArgs {
+    const void *q, *k, *v;    // q [B,Hq,D]; caches [B,Hkv,cap,D]
+    const int32_t *seq_lens;  // [B]
+    const float *summary;     // [B,Hkv,cap/Bc,D]
+    void *out;                // [B,Hq,D]
+    float *p;                 // [B,Hkv,Ccap] or null
+    uint64_t *mask;           // [B,Hkv,Wcap] or null
+    int B, Hq, Hkv, cap, D, Bc, G, Ccap, Cf, Wcap;
+    RouteConsts rc;
+    float qk_scale2;
+    uint32_t *status;
+};
+
+cudaError_t launch_stage0(const StageArgs &a, const int32_t *seq_lens, int n_recent,
+                          cudaStream_t st);
+cudaError_t launch_route(const StageArgs &a, cudaStream_t st);
+int route_rows_per_cta(int C, int D);   // 0 if C is too large for the routing kernel
+cudaError_t launch_attend(const StageArgs &a, cudaStream_t st);
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
+int decode_supported(int G, int Ccap, int D);
+
+}  // namespace dash

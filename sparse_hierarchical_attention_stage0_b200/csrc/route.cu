@@ -1,0 +1,141 @@
+// route.cu -- Stage 1: alpha-entmax chunk routing for prefill.
+//
+// gist.science "DashAttention: Differentiable and Adaptive Sparse Hierarchical Attention",
+// Technische Zusammenfassung, "Stufe 1: Entmax-Chunk-Routing": each query scores the chunk
+// summaries, and w = alpha-entmax(gamma z) replaces top-k; query heads sharing a KV head
+// share one sparse support.  aixai.ru "DashAttention ...", "Трёхстадийная архитектура": the
+// result is handed to Stage 2 as a bit-packed active-block mask (64-bit words).
+//
+// CTA = (b, g, RT consecutive rows of one query chunk), 256 threads:
+//   1. qbar[r] = mean of the G query heads of group g at row t0 + r     (shared memory)
+//   2. x[r][c] = (qbar[r] . summary[c]) * (alpha-1) gamma / sqrt(D) for every routable
+//      chunk c < c_t: lane = chunk, each lane runs RT sequential fmaf chains over d, the
+//      summary row streamed by float4 loads, qbar broadcast from shared memory
+//   3. one warp per row solves tau (warp_entmax_tau) and emits the mask words by ballot,
+//      tau, and optionally the dense p row.
+// No top-k list and no per-row index list is ever written.
+#include "dash_common.cuh"
+#include "kernels.cuh"
+
+namespace dash {
+
+int route_rows_per_cta(int C, int D) {
+    const size_t budget = 200 * 1024;
+    for (int rt : {16, 8, 4}) {
+        size_t xstride = (size_t)((C + 3) & ~3);
+        size_t bytes = (size_t)rt * D * 4 + (size_t)rt * xstride * 4;
+        if (bytes <= budget) return rt;
+    }
+    return 0;
+}
+
+template <int D, int RT>
+__global__ void __launch_bounds__(kRouteThreads) k_route(StageArgs a) {
+    extern __shared__ __align__(16) float sm[];
+    const int xstride = (a.C + 3) & ~3;
+    float *qbar = sm;               // [RT][D]
+    float *xs = sm + RT * D;        // [RT][xstride]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bg = blockIdx.y, b = bg / a.Hkv, g = bg % a.Hkv;
+    const int t0 = blockIdx.x * RT;
+    const int ct = t0 / a.Bc;                     // every row of the tile shares c_t
+    const int n = ct;                             // routable chunks
+    const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(a.q);
+    const long long hstride = (long long)a.T * D;
+
+    for (int idx = threadIdx.x; idx < RT * D; idx += kRouteThreads) {
+        int r = idx / D, d = idx % D, t = t0 + r;
+        qbar[idx] = t < a.T ? group_mean_elem(q + ((long long)(b * a.Hq + g * a.G) * a.T + t) * D + d,
+                                              hstride, a.G)
+                            : 0.f;
+    }
+    __syncthreads();
+
+    const float scale = a.rc.kind == 0 ? a.rc.sscale : a.rc.xscale;
+    const float *sumg = a.summary + (long long)bg * a.Cf * D;
+    for (int cbase = warp * 32; cbase < n; cbase += (kRouteThreads / 32) * 32) {
+        const int c = cbase + lane;
+        const float4 *s4 = reinterpret_cast<const float4 *>(sumg + (long long)min(c, n - 1) * D);
+        float acc[RT];
+#pragma unroll
+        for (int r = 0; r < RT; ++r) acc[r] = 0.f;
+#pragma unroll 4
+        for (int i = 0; i < D / 4; ++i) {
+            const float4 s = __ldg(s4 + i);
+#pragma unroll
+            for (int r = 0; r < RT; ++r) {
+                const float4 qq = reinterpret_cast<const float4 *>(qbar + r * D)[i];
+                acc[r] = fmaf(qq.x, s.x, acc[r]);
+                acc[r] = fmaf(qq.y, s.y, acc[r]);
+                acc[r] = fmaf(qq.z, s.z, acc[r]);
+                acc[r] = fmaf(qq.w, s.w, acc[r]);
+            }
+        }
+        if (c < n) {
+#pragma unroll
+            for (int r = 0; r < RT; ++r) xs[r * xstride + c] = __fmul_rn(acc[r], scale);
+        }
+    }
+    __syncthreads();
+
+    for (int r = warp; r < RT; r += kRouteThreads / 32) {
+        const int t = t0 + r;
+        if (t >= a.T) break;
+        const long long row = (long long)bg * a.T + t;
+        const float *x = xs + r * xstride;
+        float tau = n > 0 ? warp_entmax_tau(x, n, a.rc, a.status) : __int_as_float(0x7fc00000);
+        if (lane == 0) a.tau[row] = tau;
+        uint64_t *mrow = a.mask + row * a.W;
+        for (int w = 0; w < a.W; ++w) {
+            const int c0 = w * 64 + lane, c1 = c0 + 32;
+            bool p0 = c0 == ct || (c0 < n && (a.rc.kind == 0 || __fsub_rn(x[c0], tau) > 0.f));
+            bool p1 = c1 == ct || (c1 < n && (a.rc.kind == 0 || __fsub_rn(x[c1], tau) > 0.f));
+            unsigned lo = __ballot_sync(kFull, p0), hi = __ballot_sync(kFull, p1);
+            if (lane == (w & 31)) mrow[w] = ((uint64_t)hi << 32) | lo;
+        }
+        if (a.p) {
+            float *prow = a.p + row * a.C;
+            for (int c = lane; c < a.C; c += 32) {
+                float val = 0.f;
+                if (c < n) {
+                    if (a.rc.kind == 0) {
+                        val = expf(x[c] - tau);
+                    } else {
+                        float m = __fsub_rn(x[c], tau);
+                        val = m > 0.f ? pow_beta(m, a.rc) : 0.f;
+                    }
+                }
+                prow[c] = val;
+            }
+        }
+    }
+}
+
+template <int D, int RT>
+static cudaError_t launch_route_t(const StageArgs &a, cudaStream_t st) {
+    const int xstride = (a.C + 3) & ~3;
+    size_t smem = ((size_t)RT * D + (size_t)RT * xstride) * sizeof(float);
+    auto kern = k_route<D, RT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((a.T + RT - 1) / RT, a.B * a.Hkv);
+    kern<<<grid, kRouteThreads, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_route(const StageArgs &a, cudaStream_t st) {
+    const int rt = route_rows_per_cta(a.C, a.D);
+    if (a.D == 128) {
+        if (rt == 16) return launch_route_t<128, 16>(a, st);
+        if (rt == 8) return launch_route_t<128, 8>(a, st);
+        if (rt == 4) return launch_route_t<128, 4>(a, st);
+    } else if (a.D == 64) {
+        if (rt == 16) return launch_route_t<64, 16>(a, st);
+        if (rt == 8) return launch_route_t<64, 8>(a, st);
+        if (rt == 4) return launch_route_t<64, 4>(a, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace dash

@@ -1,0 +1,147 @@
+// stage0.cu -- Stage 0: local chunk summarisation.
+//
+// gist.science "DashAttention: Differentiable and Adaptive Sparse Hierarchical Attention",
+// Technische Zusammenfassung, "Stufe 0: Lokale Chunk-Zusammenfassung": a learned query
+// (head_cls) attends by local scaled dot-product attention over the keys of each chunk; the
+// summary of a complete chunk is frozen and cached for decoding.
+//
+// One warp per chunk.  The chunk's keys (Bc x D bf16, contiguous in memory) are staged into
+// shared memory by one bulk copy on the TMA engine (cp.async.bulk + mbarrier), then
+//   l_j = head_cls . k_j / sqrt(D)      (lane-sliced dot, butterfly-reduced)
+//   summary = sum_j exp(l_j - max) k_j / sum_j exp(l_j - max)
+// with each lane owning D/32 output dims (16-byte coalesced stores for D = 128).
+// HBM-bound: it reads Bc*D*2 bytes and writes D*4 bytes per chunk.
+#include "dash_common.cuh"
+#include "kernels.cuh"
+
+namespace dash {
+
+template <int D, int BC>
+__device__ __forceinline__ void summarize_chunk_warp(const __nv_bfloat16 *ks, const float *hc,
+                                                     float *out) {
+    constexpr int PER = D / 32;          // dims per lane
+    constexpr int SLOTS = BC / 32;       // logits kept per lane
+    const int lane = threadIdx.x & 31;
+    float h[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) h[i] = hc[lane * PER + i];
+    const float inv_sqrt_d = rsqrtf((float)D);
+    float logit[SLOTS];
+#pragma unroll
+    for (int i = 0; i < SLOTS; ++i) logit[i] = 0.f;
+#pragma unroll
+    for (int sl = 0; sl < SLOTS; ++sl) {
+#pragma unroll 4
+        for (int jj = 0; jj < 32; ++jj) {
+            const __nv_bfloat16 *kr = ks + (sl * 32 + jj) * D + lane * PER;
+            float part = 0.f;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) part = fmaf(h[i], __bfloat162float(kr[i]), part);
+            part = warp_sum(part);
+            if (jj == lane) logit[sl] = part * inv_sqrt_d;
+        }
+    }
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < SLOTS; ++i) mx = fmaxf(mx, logit[i]);
+    mx = warp_max(mx);
+    float den = 0.f;
+#pragma unroll
+    for (int i = 0; i < SLOTS; ++i) { logit[i] = expf(logit[i] - mx); den += logit[i]; }
+    den = warp_sum(den);
+    float acc[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int sl = 0; sl < SLOTS; ++sl) {
+#pragma unroll 4
+        for (int jj = 0; jj < 32; ++jj) {
+            float w = __shfl_sync(kFull, logit[sl], jj);
+            const __nv_bfloat16 *kr = ks + (sl * 32 + jj) * D + lane * PER;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) acc[i] = fmaf(w, __bfloat162float(kr[i]), acc[i]);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i) out[lane * PER + i] = acc[i] / den;
+}
+
+// Grid: one warp per unit.  Prefill units are (b, g, c) for every complete chunk; decode
+// units (seq_lens != nullptr) are (b, g, r) = the r-th most recent complete chunk.
+template <int D, int BC>
+__global__ void __launch_bounds__(kStage0Warps * 32)
+k_stage0(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ head_cls,
+         float *__restrict__ summary, int B, int Hkv, int T, int Cf, const int32_t *seq_lens,
+         int n_recent, uint32_t *status) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    __shared__ __align__(8) uint64_t bars[kStage0Warps];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long unit = (long long)blockIdx.x * kStage0Warps + warp;
+    int b, g, c;
+    if (seq_lens == nullptr) {
+        if (unit >= (long long)B * Hkv * Cf) return;
+        c = (int)(unit % Cf);
+        g = (int)((unit / Cf) % Hkv);
+        b = (int)(unit / ((long long)Cf * Hkv));
+    } else {
+        if (unit >= (long long)B * Hkv * n_recent) return;
+        int r = (int)(unit % n_recent);
+        g = (int)((unit / n_recent) % Hkv);
+        b = (int)(unit / ((long long)n_recent * Hkv));
+        int L = seq_lens[b];
+        if (L < 1 || L > T) {
+            if (lane == 0) report(status, DASH_ERR_INVALID_ARGUMENT);
+            return;
+        }
+        c = L / BC - 1 - r;
+        if (c < 0) return;
+    }
+    __nv_bfloat16 *ks = reinterpret_cast<__nv_bfloat16 *>(smem_raw) + (size_t)warp * BC * D;
+    const __nv_bfloat16 *src = k + (((long long)b * Hkv + g) * T + (long long)c * BC) * D;
+    constexpr uint32_t kBytes = BC * D * sizeof(__nv_bfloat16);
+    if (lane == 0) {
+        mbar_init(&bars[warp], 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    if (lane == 0) {
+        mbar_arrive_expect_tx(&bars[warp], kBytes);
+        bulk_g2s(ks, src, kBytes, &bars[warp]);
+    }
+    if (!mbar_wait_bounded(&bars[warp], 0)) {
+        if (lane == 0) report(status, DASH_ERR_DEVICE_TIMEOUT);
+        mbar_wait_bounded(&bars[warp], 0);   // give the copy in flight one more bounded wait
+        return;
+    }
+    summarize_chunk_warp<D, BC>(ks, head_cls + (size_t)g * D,
+                                summary + (((long long)b * Hkv + g) * Cf + c) * D);
+}
+
+template <int D, int BC>
+static cudaError_t launch_stage0_t(const StageArgs &a, const int32_t *seq_lens, int n_recent,
+                                   cudaStream_t st) {
+    long long units = seq_lens ? (long long)a.B * a.Hkv * n_recent
+                               : (long long)a.B * a.Hkv * a.Cf;
+    if (units == 0) return cudaSuccess;
+    size_t smem = (size_t)kStage0Warps * BC * D * sizeof(__nv_bfloat16);
+    auto kern = k_stage0<D, BC>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    unsigned grid = (unsigned)((units + kStage0Warps - 1) / kStage0Warps);
+    kern<<<grid, kStage0Warps * 32, smem, st>>>(
+        reinterpret_cast<const __nv_bfloat16 *>(a.k), a.head_cls, a.summary, a.B, a.Hkv, a.T,
+        a.Cf, seq_lens, n_recent, a.status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_stage0(const StageArgs &a, const int32_t *seq_lens, int n_recent,
+                          cudaStream_t st) {
+    if (a.D == 128 && a.Bc == 64) return launch_stage0_t<128, 64>(a, seq_lens, n_recent, st);
+    if (a.D == 128 && a.Bc == 128) return launch_stage0_t<128, 128>(a, seq_lens, n_recent, st);
+    if (a.D == 64 && a.Bc == 64) return launch_stage0_t<64, 64>(a, seq_lens, n_recent, st);
+    if (a.D == 64 && a.Bc == 128) return launch_stage0_t<64, 128>(a, seq_lens, n_recent, st);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace dash

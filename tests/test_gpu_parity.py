@@ -1,0 +1,215 @@
+"""GPU parity of every stage against the fp64 oracle, through the C ABI (via the binding),
+at sizes the oracle finishes in seconds that still span several tiles and a ragged tail."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dash_inputs import CONFIGS, PrefillConfig, make_prefill
+from parity_util import check_output, check_routing, unpack_mask
+
+pytestmark = pytest.mark.gpu
+
+dev = "cuda"
+
+
+@pytest.fixture(scope="module")
+def dash():
+    import sparse_hierarchical_attention_stage0_b200 as d
+    return d
+
+
+def _cfg(B, Hq, Hkv, T, D, Bc, alpha, planted=True, n_max=8, seed=0, gamma=1.0):
+    return PrefillConfig("t", B, Hq, Hkv, T, D, Bc, alpha, gamma=gamma, planted=planted,
+                         n_max=n_max, seed=seed)
+
+
+def _to(*ts):
+    return [t.to(dev) for t in ts]
+
+
+# ------------------------------------------------------------------------------ stage 0
+@pytest.mark.parametrize("D,Bc,T", [(64, 64, 1000), (128, 64, 777), (128, 128, 1300),
+                                    (64, 128, 256), (128, 64, 50)])
+def test_stage0_matches_oracle(dash, D, Bc, T):
+    q, k, v, hc = make_prefill(_cfg(2, 4, 2, T, D, Bc, 1.5, planted=False, seed=D + T))
+    S = dash.stage0(k.to(dev), hc.to(dev), Bc)
+    torch.cuda.synchronize()
+    ref = oracle.stage0(k, hc, Bc)
+    assert S.shape == ref.shape
+    if ref.size:
+        rel = np.abs(S.cpu().double().numpy() - ref).max() / np.abs(ref).max()
+        assert rel <= 1e-5, rel
+
+
+def test_update_chunk_cache_is_bit_identical_to_stage0(dash):
+    B, Hkv, cap, D, Bc = 3, 2, 1024 + 64, 128, 64
+    g = torch.Generator().manual_seed(5)
+    k = torch.randn(B, Hkv, cap, D, generator=g).to(torch.bfloat16).to(dev)
+    hc = torch.randn(Hkv, D, generator=g).to(dev)
+    full = dash.stage0(k, hc, Bc)                           # every complete chunk
+    cache = torch.full_like(full, float("nan"))
+    seq = torch.tensor([64, 700, 1088], dtype=torch.int32, device=dev)
+    dash.update_chunk_cache(k, hc, seq, cache, heads_q=2 * Hkv, chunk_size=Bc, n_recent=cap // Bc)
+    torch.cuda.synchronize()
+    for b, L in enumerate([64, 700, 1088]):
+        n = L // Bc
+        assert torch.equal(cache[b, :, :n], full[b, :, :n])
+        assert torch.isnan(cache[b, :, n:]).all()           # chunks not yet complete: untouched
+
+
+def test_update_chunk_cache_reports_bad_seq_len(dash):
+    B, Hkv, cap, D = 2, 2, 512, 64
+    k = torch.zeros(B, Hkv, cap, D, dtype=torch.bfloat16, device=dev)
+    hc = torch.zeros(Hkv, D, device=dev)
+    cache = torch.zeros(B, Hkv, cap // 64, D, device=dev)
+    ws = dash.workspace(256, dev)
+    seq = torch.tensor([cap + 1, 64], dtype=torch.int32, device=dev)
+    dash.update_chunk_cache(k, hc, seq, cache, heads_q=2, chunk_size=64, ws=ws)
+    assert dash.read_device_status(ws) == 1                 # DASH_ERR_INVALID_ARGUMENT
+    assert dash.read_device_status(ws) == 0                 # read clears it
+
+
+# ------------------------------------------------------------------------------ stage 1
+@pytest.mark.parametrize("alpha", [1.0, 1.25, 1.5, 2.0])
+@pytest.mark.parametrize("G,D,Bc,T", [(16, 128, 64, 2048 + 37), (4, 128, 128, 3000),
+                                      (1, 64, 64, 1500), (2, 64, 128, 1100)])
+def test_route_matches_oracle(dash, alpha, G, D, Bc, T):
+    Hkv = 2
+    cfg = _cfg(1, G * Hkv, Hkv, T, D, Bc, alpha, seed=int(alpha * 10) + G)
+    q, k, v, hc = make_prefill(cfg)
+    qd, kd, hcd = _to(q, k, hc)
+    S = dash.stage0(kd, hcd, Bc)
+    r = dash.route(qd, S, Hkv, Bc, alpha)
+    torch.cuda.synchronize()
+    # Oracle Stage 1 on the GPU's own summaries isolates the routing arithmetic.
+    p_or, m_or, tau_or = oracle.stage1(q, S.cpu(), T, Bc, alpha)
+    C = p_or.shape[-1]
+    bits = unpack_mask(r["active_blocks"], C)
+    n_ex = check_routing(bits, r["p"].cpu().double().numpy(), p_or, m_or, np.arange(T), Bc,
+                         alpha, tag=f"a={alpha} G={G}")
+    assert n_ex <= 3
+    tau = r["tau"].cpu().double().numpy()
+    routed = np.arange(T) >= Bc
+    np.testing.assert_allclose(tau[..., routed], tau_or[..., routed], atol=2e-5)
+    assert np.isnan(tau[..., ~routed]).all()
+
+
+# ------------------------------------------------------------------------------ prefill
+@pytest.mark.parametrize("alpha", [1.0, 1.5, 2.0])
+@pytest.mark.parametrize("G,D,Bc,T", [(16, 128, 64, 1024 + 100), (4, 128, 128, 1500),
+                                      (1, 64, 64, 777), (8, 64, 64, 640), (32, 128, 64, 700)])
+def test_prefill_matches_oracle(dash, alpha, G, D, Bc, T):
+    Hkv = 2 if G <= 16 else 1
+    cfg = _cfg(1, G * Hkv, Hkv, T, D, Bc, alpha, seed=7 + G)
+    q, k, v, hc = make_prefill(cfg)
+    res = dash.prefill(*_to(q, k, v, hc), chunk_size=Bc, alpha=alpha, enable_gqa=True,
+                       return_p=True, return_active_blocks=True, return_summary=True)
+    torch.cuda.synchronize()
+    ref = oracle.prefill(q, k, v, hc, Bc, alpha)
+    C = ref["p"].shape[-1]
+    check_routing(unpack_mask(res["active_blocks"], C), res["p"].cpu().double().numpy(),
+                  ref["p"], ref["m"], np.arange(T), Bc, alpha, tag="prefill")
+    check_output(res["out"].cpu().float().numpy(), ref["O"], tag=f"G={G} a={alpha}")
+    assert dash.read_device_status(res["ws"]) == 0
+
+
+def test_prefill_single_partial_chunk(dash):
+    """T < chunk_size: every row is local causal attention inside chunk 0."""
+    q, k, v, hc = make_prefill(_cfg(2, 8, 2, 40, 64, 64, 1.5, planted=False, seed=3))
+    out = dash.prefill(*_to(q, k, v, hc), chunk_size=64, alpha=1.5, enable_gqa=True)
+    torch.cuda.synchronize()
+    ref = oracle.stage2(q, k, v, None, 64, dense=True)
+    check_output(out.cpu().float().numpy(), ref)
+
+
+def test_dense_equals_force_all_active_and_causal_attention(dash):
+    cfg = _cfg(1, 32, 2, 1200, 128, 64, 1.5, seed=11)
+    q, k, v, hc = make_prefill(cfg)
+    qd, kd, vd, hcd = _to(q, k, v, hc)
+    o_dense = dash.prefill(qd, kd, vd, None, 64, enable_gqa=True, dense=True)
+    o_force = dash.prefill(qd, kd, vd, hcd, 64, enable_gqa=True, force_all_active=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o_dense, o_force)
+    ref = oracle.stage2(q, k, v, None, 64, dense=True)
+    check_output(o_dense.cpu().float().numpy(), ref, tag="dense")
+
+
+def test_inactive_chunks_do_not_touch_the_output(dash):
+    """Rewriting V inside chunks that none of the last query chunk's 64 tokens routes to
+    leaves those tokens' outputs identical to the bit."""
+    cfg = _cfg(1, 32, 2, 2048, 128, 64, 2.0, seed=12, n_max=2)
+    q, k, v, hc = make_prefill(cfg)
+    qd, kd, vd, hcd = _to(q, k, v, hc)
+    res = dash.prefill(qd, kd, vd, hcd, 64, alpha=2.0, enable_gqa=True, return_active_blocks=True)
+    torch.cuda.synchronize()
+    bits = unpack_mask(res["active_blocks"], 32)[0, :, -64:]     # [Hkv, 64 rows, C]
+    used = bits.any(axis=1)                                       # [Hkv, C]
+    v2 = vd.clone()
+    n_dead = 0
+    for g in range(2):
+        for c in range(31):
+            if not used[g, c]:
+                v2[0, g, c * 64:(c + 1) * 64] = 1e4
+                n_dead += 1
+    assert n_dead > 0
+    out2 = dash.prefill(qd, kd, v2, hcd, 64, alpha=2.0, enable_gqa=True)
+    torch.cuda.synchronize()
+    assert torch.equal(res["out"][:, :, -64:], out2[:, :, -64:])
+
+
+# ------------------------------------------------------------------------------ decode
+def _decode_setup(dash, B, Hq, Hkv, L, D, Bc, seed):
+    cfg = _cfg(B, Hq, Hkv, L, D, Bc, 1.5, seed=seed)
+    q, k, v, hc = make_prefill(cfg)
+    return cfg, q, k, v, hc
+
+
+@pytest.mark.parametrize("G,D,Bc", [(16, 128, 64), (4, 64, 128), (1, 64, 64)])
+def test_decode_matches_oracle_and_prefill_rows(dash, G, D, Bc):
+    B, Hkv, L = 3, 2, 1500
+    cfg, q, k, v, hc = _decode_setup(dash, B, G * Hkv, Hkv, L, D, Bc, seed=20 + G)
+    qd, kd, vd, hcd = _to(q, k, v, hc)
+    pre = dash.prefill(qd, kd, vd, hcd, Bc, enable_gqa=True, return_p=True,
+                       return_active_blocks=True)
+    cap = L + 37
+    kc = torch.zeros(B, Hkv, cap, D, dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    kc[:, :, :L] = kd
+    vc[:, :, :L] = vd
+    cache = torch.zeros(B, Hkv, cap // Bc, D, device=dev)
+    lens = [L, L - 1, Bc * 3]                                 # rows t = L-1, L-2, 3Bc-1
+    seq = torch.tensor(lens, dtype=torch.int32, device=dev)
+    dash.update_chunk_cache(kc, hcd, seq, cache, heads_q=G * Hkv, chunk_size=Bc, n_recent=cap // Bc)
+    qs = torch.stack([qd[b, :, lens[b] - 1] for b in range(B)])        # [B,Hq,D]
+    ws = dash.workspace(256, dev)
+    dec = dash.decode(qs, kc, vc, seq, cache, Bc, enable_gqa=True, return_p=True,
+                      return_active_blocks=True, ws=ws)
+    torch.cuda.synchronize()
+    assert dash.read_device_status(ws) == 0
+    C = (L + Bc - 1) // Bc
+    for b in range(B):
+        t = lens[b] - 1
+        # decode row == prefill row: routing bit-identical, output within bf16 rounding
+        assert torch.equal(dec["p"][b, :, :C], pre["p"][b, :, t])
+        assert torch.equal(dec["active_blocks"][b, :, :(C + 63) // 64], pre["active_blocks"][b, :, t])
+        d = (dec["out"][b].float() - pre["out"][b, :, t].float()).abs().max().item()
+        assert d <= 2e-2, d
+    ref = oracle.decode(qs.cpu(), kc.cpu(), vc.cpu(), hc, lens, Bc, 1.5)
+    check_output(dec["out"].cpu().float().numpy(), ref["O"], tag="decode")
+    bits = unpack_mask(dec["active_blocks"], ref["p"].shape[-1])
+    for b in range(B):
+        t = lens[b] - 1
+        check_routing(bits[b][:, None], dec["p"][b][:, None].cpu().double().numpy(),
+                      ref["p"][b][:, None], ref["m"][b][:, None], [t], Bc, 1.5, tag="decode")
+
+
+def test_decode_reports_bad_seq_len(dash):
+    B, Hkv, cap, D = 2, 2, 256, 128
+    kc = torch.zeros(B, Hkv, cap, D, dtype=torch.bfloat16, device=dev)
+    cache = torch.zeros(B, Hkv, cap // 64, D, device=dev)
+    q = torch.zeros(B, 32, D, dtype=torch.bfloat16, device=dev)
+    seq = torch.tensor([cap + 5, 10], dtype=torch.int32, device=dev)
+    ws = dash.workspace(256, dev)
+    dash.decode(q, kc, kc, seq, cache, 64, enable_gqa=True, ws=ws)
+    assert dash.read_device_status(ws) == 1
