@@ -177,8 +177,9 @@ def traffic_for(kernel, cfg_name):
         with open(TRAFFIC_FILE) as f:
             d = json.load(f)
         e = d[kernel][cfg_name]
-        src = os.path.join(ROOT, "sparse_hierarchical_attention_stage0_b200", "csrc", e["source"])
-        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        csrc = os.path.join(ROOT, "sparse_hierarchical_attention_stage0_b200", "csrc")
+        blob = b"".join(open(os.path.join(csrc, n), "rb").read() for n in e["sources"])
+        h = hashlib.sha256(blob).hexdigest()[:16]
         return e["bytes_per_launch"] if h == e["source_sha256_16"] else None
     except (OSError, ValueError, KeyError):
         return None

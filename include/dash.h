@@ -118,7 +118,8 @@ dash_status_t dash_prefill(const dash_params_t *params, const void *q, const voi
 
 /* Stage 0 alone: summary_k [B, H_kv, T/Bc, D] fp32 of every complete chunk of k
  * [B, H_kv, T, D] bf16.  Each summary is computed by one warp from a TMA (bulk-copy) staged
- * chunk in shared memory.  ws (>= 256 bytes) holds the status word. */
+ * chunk in shared memory.  ws (>= 256 bytes) holds the status word.  summary_k may be NULL
+ * when T < chunk_size (no complete chunk). */
 dash_status_t dash_stage0(const dash_params_t *params, const void *k, const float *head_cls,
                           float *summary_k, void *ws, size_t ws_bytes, void *stream);
 

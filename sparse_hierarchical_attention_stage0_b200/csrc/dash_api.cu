@@ -182,7 +182,7 @@ dash_status_t dash_stage0(const dash_params_t *p, const void *k, const float *he
     Shape s;
     dash_status_t rc = check_params(p, &s);
     if (rc != DASH_OK) return rc;
-    if (!k || !head_cls || !summary_k || !ws) return DASH_ERR_INVALID_ARGUMENT;
+    if (!k || !head_cls || (!summary_k && s.Cf > 0) || !ws) return DASH_ERR_INVALID_ARGUMENT;
     if (!aligned16(k) || !aligned16(head_cls) || !aligned16(summary_k) ||
         (reinterpret_cast<uintptr_t>(ws) & 255u))
         return DASH_ERR_INVALID_ARGUMENT;
@@ -203,7 +203,8 @@ dash_status_t dash_route(const dash_params_t *p, const void *q, const float *sum
     Shape s;
     dash_status_t rc = check_params(p, &s);
     if (rc != DASH_OK) return rc;
-    if (!q || !summary_k || !tau || !active_blocks || !ws) return DASH_ERR_INVALID_ARGUMENT;
+    if (!q || (!summary_k && s.Cf > 0) || !tau || !active_blocks || !ws)
+        return DASH_ERR_INVALID_ARGUMENT;
     if (!aligned16(q) || !aligned16(summary_k) || !aligned16(tau) || !aligned16(prob) ||
         !aligned16(active_blocks) || (reinterpret_cast<uintptr_t>(ws) & 255u))
         return DASH_ERR_INVALID_ARGUMENT;
@@ -230,7 +231,8 @@ dash_status_t dash_attend(const dash_params_t *p, const void *q, const void *k, 
     if (rc != DASH_OK) return rc;
     const bool ignore = (p->flags & (DASH_FLAG_DENSE | DASH_FLAG_FORCE_ALL_ACTIVE)) != 0;
     if (!q || !k || !v || !out || !ws) return DASH_ERR_INVALID_ARGUMENT;
-    if (!ignore && (!summary_k || !tau || !active_blocks)) return DASH_ERR_INVALID_ARGUMENT;
+    if (!ignore && ((!summary_k && s.Cf > 0) || !tau || !active_blocks))
+        return DASH_ERR_INVALID_ARGUMENT;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
         !aligned16(summary_k) || !aligned16(tau) || !aligned16(active_blocks) ||
         (reinterpret_cast<uintptr_t>(ws) & 255u))
