@@ -172,6 +172,32 @@ dash_status_t dash_decode(const dash_params_t *params, const void *q, const void
                           const float *summary_cache, void *out, float *p,
                           uint64_t *active_blocks, void *ws, size_t ws_bytes, void *stream);
 
+/* Size of the device array that dash_prefill_static_ws uses as its workspace. */
+#define DASH_STATIC_WS_BYTES (16u << 20)
+
+/* dash_prefill for callers that cannot allocate device memory.  The paper has no
+ * counterpart to this entry point: it exists for callers such as a plugin inside a host
+ * application that owns all device memory through its own pool, or a loop on a latency
+ * budget that cannot afford cudaMalloc's blocking.  Same arguments, arithmetic and outputs as dash_prefill, but no
+ * workspace: the scratch (status word, tau, and the summaries / mask words not supplied by
+ * the caller) lives in one file-scope device array of DASH_STATIC_WS_BYTES, reserved on
+ * every GPU that loads the library and held until exit.
+ *   - Sizes whose scratch exceeds DASH_STATIC_WS_BYTES return DASH_ERR_WORKSPACE_TOO_SMALL
+ *     before anything runs; passing summary_k and active_blocks shrinks the need to the
+ *     status word plus tau (B*H_kv*T*4 bytes).
+ *   - The first call on a device looks up the array's device address once, with that device
+ *     current; make that first call before any stream capture.
+ *   - Every call shares the array and leaves its contents behind; the status word is cleared
+ *     per call and the rest is fully written before it is read.  Calls that overlap on the
+ *     GPU race on the array: order them.
+ *   - The device status word is not readable through this entry point's arguments; a
+ *     device-side fault shows as a wrong result only.
+ * Nothing here calls cudaMalloc, cudaFree or any allocating routine. */
+dash_status_t dash_prefill_static_ws(const dash_params_t *params, const void *q, const void *k,
+                                     const void *v, const float *head_cls, void *out,
+                                     float *summary_k, float *p, uint64_t *active_blocks,
+                                     void *stream);
+
 /* Synchronises `stream`, then returns the status word the kernels wrote into ws (DASH_OK if
  * none) and clears it.  Returns DASH_ERR_CUDA if the copy itself fails. */
 dash_status_t dash_read_device_status(void *ws, void *stream);
