@@ -16,9 +16,9 @@ namespace dash {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr unsigned kFull = 0xffffffffu;
-// Spin limit of every bounded device wait (each try_wait may itself sleep up to a
-// hardware time slice), and iteration cap of the entmax Newton solve.
-constexpr int kMaxSpin = 1 << 24;
+// Time limit of every bounded device wait (measured on %globaltimer, so the bound holds
+// whatever time each try_wait spends suspended), and iteration cap of the entmax Newton solve.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 constexpr int kNewtonCap = 96;
 
 // ---------------------------------------------------------------- status word
@@ -94,11 +94,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait on an mbarrier phase; false if the spin limit ran out.
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Bounded wait on an mbarrier phase; false once kWaitLimitNs has elapsed without it.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
-    for (int i = 0; i < kMaxSpin; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-    return false;
+        if (global_ns() - t0 > kWaitLimitNs) return false;
+    }
 }
 
 // ---------------------------------------------------------------- ldmatrix / mma.sync

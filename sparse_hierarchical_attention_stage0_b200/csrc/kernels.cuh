@@ -44,6 +44,8 @@ cudaError_t launch_stage0(const StageArgs &a, const int32_t *seq_lens, int n_rec
 cudaError_t launch_route(const StageArgs &a, cudaStream_t st);
 int route_rows_per_cta(int C, int D);   // 0 if C is too large for the routing kernel
 cudaError_t launch_attend(const StageArgs &a, cudaStream_t st);
+bool attend_tc_supported(const StageArgs &a);
+cudaError_t launch_attend_tc(const StageArgs &a, cudaStream_t st);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
 int decode_supported(int G, int Ccap, int D);
 

@@ -108,7 +108,7 @@ k_stage0(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ head_cls
         mbar_arrive_expect_tx(&bars[warp], kBytes);
         bulk_g2s(ks, src, kBytes, &bars[warp]);
     }
-    if (!mbar_wait_bounded(&bars[warp], 0)) {
+    if (!__all_sync(kFull, mbar_wait_bounded(&bars[warp], 0))) {   // warp-uniform outcome
         if (lane == 0) report(status, DASH_ERR_DEVICE_TIMEOUT);
         mbar_wait_bounded(&bars[warp], 0);   // give the copy in flight one more bounded wait
         return;

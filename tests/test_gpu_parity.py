@@ -98,7 +98,8 @@ def test_route_matches_oracle(dash, alpha, G, D, Bc, T):
 # ------------------------------------------------------------------------------ prefill
 @pytest.mark.parametrize("alpha", [1.0, 1.5, 2.0])
 @pytest.mark.parametrize("G,D,Bc,T", [(16, 128, 64, 1024 + 100), (4, 128, 128, 1500),
-                                      (1, 64, 64, 777), (8, 64, 64, 640), (32, 128, 64, 700)])
+                                      (1, 64, 64, 777), (8, 64, 64, 640), (32, 128, 64, 700),
+                                      (8, 128, 128, 1500 + 3), (16, 128, 128, 1100)])
 def test_prefill_matches_oracle(dash, alpha, G, D, Bc, T):
     Hkv = 2 if G <= 16 else 1
     cfg = _cfg(1, G * Hkv, Hkv, T, D, Bc, alpha, seed=7 + G)
