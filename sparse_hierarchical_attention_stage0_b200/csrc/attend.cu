@@ -79,12 +79,18 @@ __global__ void __launch_bounds__(kAttnWarps * 32) k_attend(StageArgs a, int TU,
 
     const bool route = !a.ignore_routing && ct > 0;
     if (route) {
-        for (int idx = lane; idx < TU * D; idx += 32) {
-            const int u = idx / D, d = idx % D, t = t0 + u;
-            qbar[idx] = t < a.T ? group_mean_elem(
-                                      q + (((long long)b * a.Hq + g * G) * a.T + t) * D + d,
-                                      (long long)a.T * D, G)
-                                : 0.f;
+        for (int idx = lane; idx < TU * (D / 8); idx += 32) {
+            const int u = idx / (D / 8), d8 = (idx % (D / 8)) * 8, t = t0 + u;
+            float m[8];
+            if (t < a.T) {
+                group_mean8(q + (((long long)b * a.Hq + g * G) * a.T + t) * D + d8,
+                            (long long)a.T * D, G, m);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) m[e] = 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) qbar[u * D + d8 + e] = m[e];
         }
     }
     __syncwarp();
@@ -253,6 +259,7 @@ static cudaError_t launch_attend_t(const StageArgs &a, cudaStream_t st) {
 }
 
 cudaError_t launch_attend(const StageArgs &a, cudaStream_t st) {
+    if (a.vt && !a.ignore_routing && attend_tok_supported(a)) return launch_attend_tok(a, st);
     if (attend_tc_supported(a)) return launch_attend_tc(a, st);
     if (a.D == 128 && a.Bc == 64) return launch_attend_t<128, 64>(a, st);
     if (a.D == 128 && a.Bc == 128) return launch_attend_t<128, 128>(a, st);

@@ -19,12 +19,11 @@
 // 32 chunks per batch, double-buffered), 4-7 softmax + epilogue.  TMEM: Q 64 columns,
 // S/P 64, O 128 = 256 columns, so two CTAs share an SM.  Every wait is bounded; on timeout
 // the CTA records DASH_ERR_DEVICE_TIMEOUT and drains.
-#include <cuda.h>
-
-#include "dash_common.cuh"
 #include "kernels.cuh"
+#include "tc_common.cuh"
 
 namespace dash {
+using namespace tcx;
 namespace {
 
 constexpr int kTcThreads = 256;
@@ -36,90 +35,6 @@ constexpr int kBiasBatch = 32;
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpBias = 2, kWarpSm0 = 4;
 constexpr uint32_t kStageBytes = 4 * 8192;  // K panels (d 0-63, 64-127), V panels
 constexpr float kRescaleThreshold = 8.f;    // log2 units, as in lazy-rescale FlashAttention
-
-// ------------------------------------------------------------------ PTX wrappers
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-    uint64_t d = 0;
-    d |= (uint64_t)((addr >> 4) & 0x3FFFu);
-    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-    d |= (uint64_t)1 << 46;                  // descriptor version for sm_100
-    d |= (uint64_t)2 << 61;                  // 128-byte swizzle
-    return d;
-}
-// kind::f16 instruction descriptor: bf16 A and B, fp32 accumulate.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn_major) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn_major << 16) |
-           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-    asm volatile("{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-                 " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
-                 "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
-}
-__device__ __forceinline__ void mma_commit(uint64_t *bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     smem_u32(bar))
-                 : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ void tma_load_3d(void *smem, const CUtensorMap *map, int x, int y, int z,
-                                            uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
-        : "memory");
-}
-// 32 lanes x 32 consecutive 32-bit columns of this warp's TMEM sub-partition.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
-          "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
-          "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
-        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
-        "r"(r[29]), "r"(r[30]), "r"(r[31]));
-}
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void named_sync(int id, int count) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
-// Bounded mbarrier wait by a whole (converged) warp, with a warp-uniform outcome: on
-// timeout it records the error once and every lane returns false.
-__device__ __forceinline__ bool wait_or_fail(uint64_t *bar, uint32_t parity, uint32_t *status,
-                                             bool &failed) {
-    if (failed) return false;
-    const bool ok = __all_sync(kFull, mbar_wait_bounded(bar, parity));
-    if (!ok) {
-        if ((threadIdx.x & 31) == 0) report(status, DASH_ERR_DEVICE_TIMEOUT);
-        failed = true;
-    }
-    return ok;
-}
 
 struct TcShared {
     uint64_t full[kStages], empty[kStages], s_full, p_full, o_full;
@@ -219,12 +134,18 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
         // Group-mean queries of the tile's tokens (Stage 1's exact arithmetic).
         if (!a.ignore_routing) {
             const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(a.q);
-            for (int idx = lane; idx < RT * D; idx += 32) {
-                const int u = idx / D, d = idx % D, t = t0 + u;
-                qbar[idx] = t < a.T ? group_mean_elem(
-                                          q + (((long long)b * a.Hq + g * G) * a.T + t) * D + d,
-                                          (long long)a.T * D, G)
-                                    : 0.f;
+            for (int idx = lane; idx < RT * (D / 8); idx += 32) {
+                const int u = idx / (D / 8), d8 = (idx % (D / 8)) * 8, t = t0 + u;
+                float m[8];
+                if (t < a.T) {
+                    group_mean8(q + (((long long)b * a.Hq + g * G) * a.T + t) * D + d8,
+                                (long long)a.T * D, G, m);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) m[e] = 0.f;
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) qbar[u * D + d8 + e] = m[e];
             }
         }
     }

@@ -148,23 +148,67 @@ __device__ __forceinline__ float group_mean_elem(const __nv_bfloat16 *q0, long l
     for (int h = 0; h < G; ++h) s += __bfloat162float(q0[h * head_stride]);
     return s / (float)G;
 }
+// The same for 8 consecutive dims (q0 16-byte aligned): one 16-byte load per head, all loads
+// issued before the ordered sums; element-wise bit-identical to group_mean_elem.
+__device__ __forceinline__ void group_mean8(const __nv_bfloat16 *q0, long long head_stride, int G,
+                                            float (&out)[8]) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) out[e] = 0.f;
+    int h = 0;
+    for (; h + 4 <= G; h += 4) {
+        uint4 v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[j] = __ldg(reinterpret_cast<const uint4 *>(q0 + (h + j) * head_stride));
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&v[j]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(b2[e]);
+                out[2 * e] += f.x;
+                out[2 * e + 1] += f.y;
+            }
+        }
+    }
+    for (; h < G; ++h) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(q0 + h * head_stride));
+        const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(b2[e]);
+            out[2 * e] += f.x;
+            out[2 * e + 1] += f.y;
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) out[e] = out[e] / (float)G;
+}
 
-// Routing dot product qbar . S_c as ONE sequential fmaf chain over d = 0..D-1.
+// Routing dot product qbar . S_c with one fixed summation order, shared by every kernel that
+// needs it: d is split into 4 interleaved slices of float4 groups (slice k = groups k, k+4,
+// k+8, ...), each slice is one sequential fmaf chain in increasing d, and the slice sums are
+// combined as (p0 + p1) + (p2 + p3).  The routing kernel computes the slices in 4 lanes and
+// combines them with two xor-shuffles, which yields exactly these bits.
 template <int D>
 __device__ __forceinline__ float route_dot(const float *qbar, const float *srow) {
-    float acc = 0.f;
     const float4 *s4 = reinterpret_cast<const float4 *>(srow);
     const float4 *q4 = reinterpret_cast<const float4 *>(qbar);
-#pragma unroll 8
-    for (int i = 0; i < D / 4; ++i) {
-        float4 s = __ldg(s4 + i);
-        float4 q = q4[i];
-        acc = fmaf(q.x, s.x, acc);
-        acc = fmaf(q.y, s.y, acc);
-        acc = fmaf(q.z, s.z, acc);
-        acc = fmaf(q.w, s.w, acc);
+    float p[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < D / 16; ++i) {
+            const float4 sv = __ldg(s4 + 4 * i + k);
+            const float4 qv = q4[4 * i + k];
+            acc = fmaf(qv.x, sv.x, acc);
+            acc = fmaf(qv.y, sv.y, acc);
+            acc = fmaf(qv.z, sv.z, acc);
+            acc = fmaf(qv.w, sv.w, acc);
+        }
+        p[k] = acc;
     }
-    return acc;
+    return (p[0] + p[1]) + (p[2] + p[3]);
 }
 
 // Constants of the routing, computed once on the host.

@@ -94,8 +94,12 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
     const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(a.q) + (long long)b * a.Hq * D;
 
     // 1. group-mean query and this CTA's slice of the scores.
-    for (int d = tid; d < D; d += kDecWarps * 32)
-        qbar[d] = group_mean_elem(q + (long long)g * G * D + d, D, G);
+    for (int d8 = tid * 8; d8 < D; d8 += kDecWarps * 32 * 8) {
+        float m[8];
+        group_mean8(q + (long long)g * G * D + d8, D, G, m);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) qbar[d8 + e] = m[e];
+    }
     __syncthreads();
     const float scale = a.rc.kind == 0 ? a.rc.sscale : a.rc.xscale;
     const int c_lo = (int)((long long)n * rank / kDecCluster);

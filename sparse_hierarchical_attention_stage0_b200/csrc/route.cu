@@ -9,8 +9,9 @@
 // CTA = (b, g, RT consecutive rows of one query chunk), 256 threads:
 //   1. qbar[r] = mean of the G query heads of group g at row t0 + r     (shared memory)
 //   2. x[r][c] = (qbar[r] . summary[c]) * (alpha-1) gamma / sqrt(D) for every routable
-//      chunk c < c_t: lane = chunk, each lane runs RT sequential fmaf chains over d, the
-//      summary row streamed by float4 loads, qbar broadcast from shared memory
+//      chunk c < c_t: 4 lanes per chunk, each owning an interleaved quarter of d (coalesced
+//      64-byte reads per chunk), RT row accumulators in registers, qbar broadcast from
+//      shared memory, slices combined with route_dot's fixed order
 //   3. one warp per row solves tau (warp_entmax_tau) and emits the mask words by ballot,
 //      tau, and optionally the dense p row.
 // No top-k list and no per-row index list is ever written.
@@ -43,35 +44,52 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(StageArgs a) {
     const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(a.q);
     const long long hstride = (long long)a.T * D;
 
-    for (int idx = threadIdx.x; idx < RT * D; idx += kRouteThreads) {
-        int r = idx / D, d = idx % D, t = t0 + r;
-        qbar[idx] = t < a.T ? group_mean_elem(q + ((long long)(b * a.Hq + g * a.G) * a.T + t) * D + d,
-                                              hstride, a.G)
-                            : 0.f;
+    for (int idx = threadIdx.x; idx < RT * (D / 8); idx += kRouteThreads) {
+        const int r = idx / (D / 8), d8 = (idx % (D / 8)) * 8, t = t0 + r;
+        float m[8];
+        if (t < a.T) {
+            group_mean8(q + ((long long)(b * a.Hq + g * a.G) * a.T + t) * D + d8, hstride, a.G, m);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) m[e] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) qbar[r * D + d8 + e] = m[e];
     }
     __syncthreads();
 
+    // Scores: 4 lanes per chunk (lane = 4*cc + k owns float4 groups k, k+4, ... of chunk cc),
+    // 8 chunks per warp and step; the RT rows' partial dots stay in registers.  The slice sums
+    // are combined with the order of route_dot: (p0 + p1) + (p2 + p3).
     const float scale = a.rc.kind == 0 ? a.rc.sscale : a.rc.xscale;
     const float *sumg = a.summary + (long long)bg * a.Cf * D;
-    for (int cbase = warp * 32; cbase < n; cbase += (kRouteThreads / 32) * 32) {
-        const int c = cbase + lane;
+    const int kslice = lane & 3, cc = lane >> 2;
+    for (int cbase = warp * 8; cbase < n; cbase += (kRouteThreads / 32) * 8) {
+        const int c = cbase + cc;
         const float4 *s4 = reinterpret_cast<const float4 *>(sumg + (long long)min(c, n - 1) * D);
         float acc[RT];
 #pragma unroll
         for (int r = 0; r < RT; ++r) acc[r] = 0.f;
-#pragma unroll 4
-        for (int i = 0; i < D / 4; ++i) {
-            const float4 s = __ldg(s4 + i);
+#pragma unroll 2
+        for (int i = 0; i < D / 16; ++i) {
+            const float4 sv = __ldg(s4 + 4 * i + kslice);
 #pragma unroll
             for (int r = 0; r < RT; ++r) {
-                const float4 qq = reinterpret_cast<const float4 *>(qbar + r * D)[i];
-                acc[r] = fmaf(qq.x, s.x, acc[r]);
-                acc[r] = fmaf(qq.y, s.y, acc[r]);
-                acc[r] = fmaf(qq.z, s.z, acc[r]);
-                acc[r] = fmaf(qq.w, s.w, acc[r]);
+                const float4 qq = reinterpret_cast<const float4 *>(qbar + r * D)[4 * i + kslice];
+                acc[r] = fmaf(qq.x, sv.x, acc[r]);
+                acc[r] = fmaf(qq.y, sv.y, acc[r]);
+                acc[r] = fmaf(qq.z, sv.z, acc[r]);
+                acc[r] = fmaf(qq.w, sv.w, acc[r]);
             }
         }
-        if (c < n) {
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+            float v = acc[r];
+            v = v + __shfl_xor_sync(kFull, v, 1);
+            v = v + __shfl_xor_sync(kFull, v, 2);
+            acc[r] = v;
+        }
+        if (kslice == 0 && c < n) {
 #pragma unroll
             for (int r = 0; r < RT; ++r) xs[r * xstride + c] = __fmul_rn(acc[r], scale);
         }
