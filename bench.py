@@ -464,6 +464,12 @@ def main():
     d2h = ho.numel() * ho.element_size()
 
     pk, pk_kind = peaks()
+    # Stage 2 kernel dash_prefill runs: the per-token kernel (after a V^T transpose, timed with
+    # it) when the workspace holds V^T scratch, else the tile kernel.
+    per_token = dash.attend_workspace_size(prm) > 256
+    s2_kernel = "k_attend_tok" if per_token else "k_attend_tc"
+    s2_note = ", V^T transpose included" if per_token else ""
+    launches_per_step = 4 if per_token else 3
     s2_tflops = stats["active_flops"] / (stage["stage2"] / 1e3) / 1e12
     sb = stage01_bytes(cfg)
     s01_gbs = (sb["stage0"] + sb["stage1"]) / ((stage["stage0"] + stage["stage1"]) / 1e3) / 1e9
@@ -482,10 +488,10 @@ def main():
         "stage01_gbs": s01_gbs,
         "dense_ms": dense_ms,
         "speedup_vs_dense": dense_ms / (total_ms / args.steps),
-        "roofline": {"bound": "tensor", "kernel": "k_attend (Stage 2)",
+        "roofline": {"bound": "tensor", "kernel": f"{s2_kernel} (Stage 2{s2_note})",
                      "achieved": s2_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": s2_tflops / pk["bf16_tflops"],
-                     "traffic": traffic_for("k_attend", cfg.name),
+                     "traffic": traffic_for(s2_kernel, cfg.name),
                      "peak_source": f"{pk_kind} bf16 burst",
                      "algorithmic": f"{stats['active_flops']:.4e} active FLOP per launch"},
         "roofline_stage01": {"bound": "hbm", "achieved": s01_gbs, "peak": pk["hbm_gbs"],
@@ -494,7 +500,7 @@ def main():
                              "bytes": sb["stage0"] + sb["stage1"]},
         "e2e": {"value": world * B * T / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }
     del hq, hk, hv, ho
