@@ -4,32 +4,43 @@
 // gist.science "DashAttention: Differentiable and Adaptive Sparse Hierarchical Attention",
 // Technische Zusammenfassung, "Stufe 2: Prior-induzierte spaerliche Softmax": the kernel
 // walks the active chunks of the bit-packed mask, adds the routing bias log p to the logits
-// of an active chunk, masks zero-probability chunks, and keeps the diagonal chunk as its own
+// of an active chunk, skips zero-probability chunks, and keeps the diagonal chunk as its own
 // (causal, bias 0) branch.
 //
-// The 16 heads of one token share one routing, so they are the N = 16 columns of the MMAs,
-// and keys (QK) or head dims (PV) are the rows:
-//   S^T[64 keys x 16] = K_c Q_t^T      A = K_c in tensor memory (M = 64), B = Q_t (smem)
-//   O_t^T[128 x 16]  += V_c^T P_t^T    A = V_c^T in tensor memory (M = 128), B = P_t (smem)
-// One CTA owns a window of 16 consecutive tokens of one (b, g) (they share the diagonal
-// chunk).  It streams the diagonal chunk first, then the union of the window's routed
-// chunks; each chunk's K and V^T are staged by TMA and copied into tensor memory once, then
-// reused by every window token that routed to it (about 16 x (1 - sparsity) of them).  Four
-// independent pipelines ("lanes") own 4 tokens each: one MMA-issuing warp and four softmax
-// warps per lane, so per-token MMAs of different lanes overlap.
+// Shapes.  The 16 heads of one token share one routing, so they are the N = 16 columns of the
+// MMAs, and keys (QK) or head dims (PV) are the M = 128 rows:
+//   S^T[128 keys x 16] = [K_a; K_b] Q_t^T   A = a chunk pair in tensor memory, B = Q_t (smem)
+//   O_t^T[128 x 16]   += V_c^T P_t^T         A = V_c^T in tensor memory, B = P_t (smem)
+// One CTA owns a window of 16 consecutive tokens of one (b, g); they share the diagonal
+// chunk.  It streams the diagonal chunk and then the union of the window's routed chunks in
+// pairs (pair 0 = diagonal + first routed chunk, pair p = list entries 2p and 2p+1).  A
+// pair's K and V^T are staged by TMA and copied into tensor memory once (tcgen05.cp), then
+// reused by every window token that routed to either chunk.  A token that routed to one chunk
+// of a pair still issues the whole M = 128 QK (an M = 64 MMA costs the same issue time) but
+// only that chunk's exponentials and PV.
 //
-// Softmax reference: the first item of every token is its diagonal chunk, whose exact
-// per-head maximum m_h becomes the fixed reference of all later chunks of that token
-// (p = 2^(s - m_h)); no running rescale of O is needed.  Logits of routed chunks can exceed
-// m_h; fp32 and bf16 hold 2^(s - m_h) exactly up to s - m_h < 127 (log2 units); larger
-// excesses are clamped and reported as DASH_ERR_RANGE_CLAMPED through the status word.
-// The lane's 4 softmax warps exchange the diagonal maxima and the row sums through an
-// mbarrier, so every wait in the kernel is bounded.
+// Pipelines.  Four independent pipelines own 4 tokens each (u = L + 4m): one MMA-issuing
+// warp and four softmax warps, one per tensor-memory sub-partition (warps 0-1 of a pipeline
+// hold chunk a's 64 keys, warps 2-3 chunk b's).  The softmax releases the S slot as soon as
+// it has loaded it, so the QK of the next item overlaps the exponentials of the current one;
+// P is double-buffered in shared memory.
 //
-// Warps: 0 TMA producer, 1 routing-bias producer, 2 TMEM owner / chunk list, 4-7 fill
-// (shared memory -> tensor memory), 8-11 MMA issuers (lane L), 12-27 softmax (lane L: warps
-// 12+4L .. 15+4L, one per TMEM sub-partition).  Tensor memory: K slots 2x64, V^T slots 2x32,
-// S slots 4x16, O 16x16 = 512 columns.  Every wait is bounded and warp-uniform.
+// Softmax reference.  The diagonal chunk (chunk a of pair 0) gives every token its exact
+// per-head maximum m_h, the fixed reference of all its chunks (p = 2^(s - m_h)), so O needs
+// no running rescale.  Routed logits can exceed m_h; fp32 and bf16 hold 2^(s - m_h) exactly
+// up to s - m_h < 127 (log2 units); larger excesses are clamped and reported as
+// DASH_ERR_RANGE_CLAMPED through the status word.
+//
+// Ordering.  K pairs are double-buffered in tensor memory, the V^T pair single-buffered.
+// Each pipeline closes the K and V phases of every pair in order (one arrival per pair, items
+// or not), and before it blocks on a resource of pair r it has closed all phases of pairs
+// below r, so the pipeline waiting on the lowest pair can always proceed.  Every wait is
+// bounded and warp-uniform.
+//
+// Warps: 0 K producer (TMA + tensor-memory copy), 1 and 3 routing-bias producers, 2 tensor
+// memory owner and chunk list, then V producer, 4-7 MMA issuers (pipeline L), 8-23 softmax
+// (pipeline L: warps 8+4L .. 11+4L).  Tensor memory (512 columns): O 16x16 | K pairs 2x64 |
+// V^T pair 64 | S 4x16.
 #include "kernels.cuh"
 #include "tc_common.cuh"
 
@@ -37,29 +48,33 @@ namespace dash {
 using namespace tcx;
 namespace {
 
-constexpr int kW = 16;
-constexpr int kLanes = 4;
-constexpr int kTpl = kW / kLanes;                 // tokens per lane
-constexpr int kNst = 2;                           // TMA stages
-constexpr uint32_t kStage = 32768;                // K panels 2 x 8 KB + V^T 16 KB
-constexpr int kBatch = 32;                        // chunk entries per bias batch
+constexpr int kW = 16;                            // tokens per window
+constexpr int kLanes = 4;                         // pipelines
+constexpr int kTpl = kW / kLanes;                 // tokens per pipeline
+constexpr uint32_t kKStage = 32768;               // K pair: 2 panels x 128 rows x 128 B
+constexpr uint32_t kVStage = 32768;               // V^T pair: 2 chunks x 128 dims x 128 B
+constexpr int kBatch = 32;                        // list entries per routing-bias batch
+constexpr int kPairsPerBatch = kBatch / 2;
 constexpr int kNBias = 4;                         // bias ring slots
-constexpr int kWarpTma = 0, kWarpBias = 1, kWarpAdmin = 2, kWarpFill0 = 4, kWarpMma0 = 8,
-              kWarpSm0 = 12;
-constexpr int kThreads = 28 * 32;
+constexpr int kWarpK = 0, kWarpBias0 = 1, kWarpAdmin = 2, kWarpBias1 = 3, kWarpMma0 = 4,
+              kWarpSm0 = 8;
+constexpr int kThreads = 24 * 32;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColK = 0, kColV = 128, kColS = 192, kColO = 256;
+constexpr uint32_t kColO = 0, kColK = 256, kColV = 384, kColS = 448;
+constexpr int kQbarStride = 132;                  // padded row of the query means (floats)
 constexpr float kMaxExcess = 126.f;               // log2 units above the reference
+constexpr int kMaxChunks = 4096;
 
 struct TokShared {
-    uint64_t tma_full[kNst], tma_empty[kNst];
-    uint64_t kv_ready[2], kv_free[2];
+    uint64_t k_full[2], k_empty[2], k_ready[2], k_free[2];
+    uint64_t v_full, v_empty, v_ready, v_free;
     uint64_t bias_full[kNBias], bias_empty[kNBias];
-    uint64_t s_full[kLanes], p_full[kLanes], o_done[kLanes], x_bar[kLanes];
+    uint64_t s_full[kLanes], s_free[kLanes], p_full[kLanes][2], o_done[kLanes], x_bar[kLanes];
     uint64_t q_full;
     uint32_t tmem_base;
     int n_ch;
     int failed;
+    int abort;
 };
 
 __device__ __forceinline__ bool wait_u(uint64_t *bar, uint32_t parity, uint32_t *status, bool &failed) {
@@ -71,13 +86,44 @@ __device__ __forceinline__ bool wait_u(uint64_t *bar, uint32_t parity, uint32_t 
     }
     return ok;
 }
+// Non-blocking, warp-uniform test of an mbarrier phase (test_wait never suspends, unlike
+// try_wait, which may sleep for a hardware-defined window before it reports "not yet").
+__device__ __forceinline__ bool test_u(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return __all_sync(kFull, ok != 0);
+}
+
+// 16 per-head values spread over a warp's 32 key lanes -> lane l holds the reduction for head
+// l >> 1 in v[0] (reduce-scatter over lane bits 4..1, then an all-reduce over bit 0).
+template <bool kMax>
+__device__ __forceinline__ float head_reduce(float (&v)[16], int lane) {
+#pragma unroll
+    for (int o = 16, n = 8; o >= 2; o >>= 1, n >>= 1) {
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < n; ++i) {
+            const float send = upper ? v[i] : v[i + n];
+            const float keep = upper ? v[i + n] : v[i];
+            const float got = __shfl_xor_sync(kFull, send, o);
+            v[i] = kMax ? fmaxf(keep, got) : keep + got;
+        }
+    }
+    const float got = __shfl_xor_sync(kFull, v[0], 1);
+    return kMax ? fmaxf(v[0], got) : v[0] + got;
+}
 
 }  // namespace
 
 struct TokArgs {
     StageArgs s;
     int n_win;             // windows per (b, g)
-    size_t off_q, off_p, off_bias, off_qbar, off_mref, off_mpart, off_lpart, off_list;
+    size_t off_q, off_k, off_v, off_p, off_bias, off_qbar, off_mref, off_mpart, off_lpart, off_list;
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -90,18 +136,20 @@ k_attend_tok(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     unsigned char *base = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~(uintptr_t)1023);
-    unsigned char *qwin = base + ta.off_q;                               // [16 tok][2 panels][16][128B]
-    unsigned char *pbuf = base + ta.off_p;                               // [lanes][2 KB]
-    float *bias_ring = reinterpret_cast<float *>(base + ta.off_bias);    // [kNBias][kBatch][16]
-    float *qbar = reinterpret_cast<float *>(base + ta.off_qbar);         // [16][D]
-    float *mref = reinterpret_cast<float *>(base + ta.off_mref);         // [16 tok][4 warps][16]
-    float *mpart = reinterpret_cast<float *>(base + ta.off_mpart);       // [16 tok][4 warps][16]
-    float *lpart = reinterpret_cast<float *>(base + ta.off_lpart);       // [16 tok][4 warps][16]
+    unsigned char *qwin = base + ta.off_q;       // [2 panels][16 tokens][16 heads][128 B]
+    unsigned char *kst = base + ta.off_k;        // [2 stages][2 panels][128 rows][128 B]
+    unsigned char *vst = base + ta.off_v;        // [2 chunks][128 dims][128 B]
+    unsigned char *pbuf = base + ta.off_p;       // [4 pipelines][2 buffers][4 KB]
+    float *bias_ring = reinterpret_cast<float *>(base + ta.off_bias);  // [kNBias][kBatch][16]
+    float *qbar = reinterpret_cast<float *>(base + ta.off_qbar);       // [16][kQbarStride]
+    float *mref = reinterpret_cast<float *>(base + ta.off_mref);       // [16 tokens][16 heads]
+    float *mpart = reinterpret_cast<float *>(base + ta.off_mpart);     // [16][2 warps][16]
+    float *lpart = reinterpret_cast<float *>(base + ta.off_lpart);     // [16][4 warps][16]
     int16_t *list = reinterpret_cast<int16_t *>(base + ta.off_list);
 
     const int BHkv = a.B * a.Hkv;
     const int wrev = blockIdx.x / BHkv, bgi = blockIdx.x % BHkv;
-    const int win = ta.n_win - 1 - wrev;
+    const int win = ta.n_win - 1 - wrev;          // longest windows first
     const int b = bgi / a.Hkv, g = bgi % a.Hkv;
     const long long bg = bgi;
     const int t0 = win * kW;
@@ -111,26 +159,33 @@ k_attend_tok(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     // ------------------------------------------------------------------ setup
     if (warp == kWarpAdmin) tmem_alloc(&sh.tmem_base, kTmemCols);
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kNst; ++s) {
-            mbar_init(&sh.tma_full[s], 1);
-            mbar_init(&sh.tma_empty[s], 4);
-        }
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&sh.kv_ready[s], 4);
-            mbar_init(&sh.kv_free[s], kLanes);
+            mbar_init(&sh.k_full[s], 1);
+            mbar_init(&sh.k_empty[s], 1);
+            mbar_init(&sh.k_ready[s], 1);
+            mbar_init(&sh.k_free[s], kLanes);
         }
+        mbar_init(&sh.v_full, 1);
+        mbar_init(&sh.v_empty, 1);
+        mbar_init(&sh.v_ready, 1);
+        mbar_init(&sh.v_free, kLanes);
         for (int k = 0; k < kNBias; ++k) {
             mbar_init(&sh.bias_full[k], 1);
             mbar_init(&sh.bias_empty[k], kLanes + 4 * kLanes);
         }
         for (int L = 0; L < kLanes; ++L) {
             mbar_init(&sh.s_full[L], 1);
-            mbar_init(&sh.p_full[L], 4);
+            mbar_init(&sh.s_free[L], 4);
+            mbar_init(&sh.p_full[L][0], 4);
+            mbar_init(&sh.p_full[L][1], 4);
             mbar_init(&sh.o_done[L], 1);
             mbar_init(&sh.x_bar[L], 4);
         }
         mbar_init(&sh.q_full, 1);
         sh.failed = 0;
+        // A CTA that starts after another one timed out does no work, so a failing launch
+        // ends within about one wave of bounded waits.
+        sh.abort = *reinterpret_cast<volatile uint32_t *>(a.status) == DASH_ERR_DEVICE_TIMEOUT;
         fence_mbar_init();
     }
     if (warp == kWarpAdmin) {
@@ -147,7 +202,7 @@ k_attend_tok(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
                 } else {
                     for (int u = 0; u < kW; ++u) {
                         const int t = t0 + u;
-                        if (t < a.T) word |= a.mask[(bg * a.T + t) * W + w];
+                        if (t < a.T) word |= __ldg(a.mask + (bg * a.T + t) * W + w);
                     }
                 }
                 const int lim = cd - 64 * w;                  // routed bits are < cd
@@ -170,9 +225,11 @@ k_attend_tok(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
         }
         if (lane == 0) sh.n_ch = pos;
     }
-    if (warp == kWarpBias && !a.ignore_routing) {
+    if ((warp == kWarpBias0 || warp == kWarpBias1) && !a.ignore_routing) {
+        // Group-mean queries of the window's tokens (the routing arithmetic of Stage 1).
         const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(a.q);
-        for (int idx = lane; idx < kW * (D / 8); idx += 32) {
+        const int l64 = lane + (warp == kWarpBias1 ? 32 : 0);
+        for (int idx = l64; idx < kW * (D / 8); idx += 64) {
             const int u = idx / (D / 8), d8 = (idx % (D / 8)) * 8, t = t0 + u;
             float m[8];
             if (t < a.T) {
@@ -183,69 +240,156 @@ k_attend_tok(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
                 for (int e = 0; e < 8; ++e) m[e] = 0.f;
             }
 #pragma unroll
-            for (int e = 0; e < 8; ++e) qbar[u * D + d8 + e] = m[e];
+            for (int e = 0; e < 8; ++e) qbar[u * kQbarStride + d8 + e] = m[e];
         }
     }
     __syncthreads();
     tc_fence_after();
     const uint32_t tb = sh.tmem_base;
+    if (sh.abort) {
+        if (warp == kWarpAdmin) tmem_dealloc(tb, kTmemCols);
+        return;
+    }
     const int n_ch = sh.n_ch;
+    const int n_pairs = (n_ch + 1) / 2;
     const int n_batches = (n_ch + kBatch - 1) / kBatch;
 
-    if (warp == kWarpTma) {
-        // ---------------------------------------------------------------- TMA producer
+    if (warp == kWarpK) {
+        // ---------------------------------------------------------------- K producer
+        auto issue_k = [&](int p) {              // lane 0: TMA of pair p into stage p & 1
+            unsigned char *stg = kst + (size_t)(p & 1) * kKStage;
+            const bool hb = 2 * p + 1 < n_ch;
+            uint64_t *bar = &sh.k_full[p & 1];
+            mbar_arrive_expect_tx(bar, hb ? kKStage : kKStage / 2);
+            const int ca = list[2 * p];
+            tma_load_3d(stg, &tmK, 0, ca * BC, (int)bg, bar);
+            tma_load_3d(stg + 16384, &tmK, 64, ca * BC, (int)bg, bar);
+            if (hb) {
+                const int cb = list[2 * p + 1];
+                tma_load_3d(stg + 8192, &tmK, 0, cb * BC, (int)bg, bar);
+                tma_load_3d(stg + 24576, &tmK, 64, cb * BC, (int)bg, bar);
+            }
+        };
         if (lane == 0) {
             mbar_arrive_expect_tx(&sh.q_full, kW * 4096);
             for (int u = 0; u < kW; ++u)
                 for (int h = 0; h < 2; ++h)
-                    tma_load_4d(qwin + u * 4096 + h * 2048, &tmQ, 64 * h, t0 + u, g * G, b, &sh.q_full);
+                    tma_load_4d(qwin + h * 32768 + u * 2048, &tmQ, 64 * h, t0 + u, g * G, b, &sh.q_full);
+            issue_k(0);
+            if (n_pairs > 1) issue_k(1);
         }
         __syncwarp();
-        int issued = 0;
-        for (int j = 0; j < n_ch; ++j) {
-            const int st = j % kNst;
-            if (!wait_u(&sh.tma_empty[st], ((uint32_t)(j / kNst) & 1u) ^ 1u, a.status, failed)) break;
-            issued = j + 1;
+        int issued = min(2, n_pairs), landed = 0, copied = 0;
+        for (int p = 0; p < n_pairs; ++p) {
+            const int st = p & 1;
+            const uint32_t ph = (uint32_t)(p >> 1) & 1u;
+            if (!wait_u(&sh.k_full[st], ph, a.status, failed)) break;
+            landed = p + 1;
+            if (!wait_u(&sh.k_free[st], ph ^ 1u, a.status, failed)) break;   // pair p-2 done
+            tc_fence_after();
             if (lane == 0) {
-                const int c = list[j];
-                unsigned char *stage = base + (size_t)st * kStage;
-                mbar_arrive_expect_tx(&sh.tma_full[st], kStage);
-                tma_load_3d(stage, &tmK, 0, c * BC, (int)bg, &sh.tma_full[st]);
-                tma_load_3d(stage + 8192, &tmK, 64, c * BC, (int)bg, &sh.tma_full[st]);
-                tma_load_3d(stage + 16384, &tmVt, c * BC, 0, (int)bg, &sh.tma_full[st]);
+                const uint32_t src = smem_u32(kst + (size_t)st * kKStage);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    tmem_cp_128x256b(tb + kColK + 64u * st + 8u * k,
+                                     smem_desc_sw128(src + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024));
+                mma_commit(&sh.k_ready[st]);
+                mma_commit(&sh.k_empty[st]);
             }
             __syncwarp();
+            copied = p + 1;
+            if (p + 2 < n_pairs) {
+                if (!wait_u(&sh.k_empty[st], ph, a.status, failed)) break;  // copy read the stage
+                if (lane == 0) issue_k(p + 2);
+                __syncwarp();
+                issued = p + 3;
+            }
         }
-        if (failed) {
+        if (failed && lane == 0) {
+            // Let the bulk copies and tensor-memory copies in flight land before exit.
             mbar_wait_bounded(&sh.q_full, 0);
-            for (int j = max(0, issued - kNst); j < issued; ++j)
-                mbar_wait_bounded(&sh.tma_full[j % kNst], (uint32_t)(j / kNst) & 1u);
-            __syncwarp();
+            for (int j = landed; j < issued; ++j) mbar_wait_bounded(&sh.k_full[j & 1], (uint32_t)(j >> 1) & 1u);
+            if (copied > 0) mbar_wait_bounded(&sh.k_empty[(copied - 1) & 1], (uint32_t)((copied - 1) >> 1) & 1u);
         }
-    } else if (warp == kWarpBias) {
+        __syncwarp();
+    } else if (warp == kWarpAdmin) {
+        // ---------------------------------------------------------------- V^T producer
+        auto issue_v = [&](int p) {
+            const bool hb = 2 * p + 1 < n_ch;
+            mbar_arrive_expect_tx(&sh.v_full, hb ? kVStage : kVStage / 2);
+            tma_load_3d(vst, &tmVt, list[2 * p] * BC, 0, (int)bg, &sh.v_full);
+            if (hb) tma_load_3d(vst + 16384, &tmVt, list[2 * p + 1] * BC, 0, (int)bg, &sh.v_full);
+        };
+        if (lane == 0 && n_pairs > 0) issue_v(0);
+        __syncwarp();
+        int issued = min(1, n_pairs), landed = 0, copied = 0;
+        for (int p = 0; p < n_pairs; ++p) {
+            const uint32_t ph = (uint32_t)p & 1u;
+            if (!wait_u(&sh.v_full, ph, a.status, failed)) break;
+            landed = p + 1;
+            if (!wait_u(&sh.v_free, ph ^ 1u, a.status, failed)) break;       // PV of pair p-1 done
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t src = smem_u32(vst);
+                const int nchunk = 2 * p + 1 < n_ch ? 2 : 1;
+                for (int c = 0; c < nchunk; ++c)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        tmem_cp_128x256b(tb + kColV + 32u * c + 8u * k,
+                                         smem_desc_sw128(src + c * 16384 + k * 32, 16, 1024));
+                mma_commit(&sh.v_ready);
+                mma_commit(&sh.v_empty);
+            }
+            __syncwarp();
+            copied = p + 1;
+            if (p + 1 < n_pairs) {
+                if (!wait_u(&sh.v_empty, ph, a.status, failed)) break;
+                if (lane == 0) issue_v(p + 1);
+                __syncwarp();
+                issued = p + 2;
+            }
+        }
+        if (failed && lane == 0) {
+            for (int j = landed; j < issued; ++j) mbar_wait_bounded(&sh.v_full, (uint32_t)j & 1u);
+            if (copied > 0) mbar_wait_bounded(&sh.v_empty, (uint32_t)(copied - 1) & 1u);
+        }
+        __syncwarp();
+    } else if (warp == kWarpBias0 || warp == kWarpBias1) {
         // ---------------------------------------------------------------- routing biases
-        for (int k = 0; k < n_batches; ++k) {
+        // Batch k (list entries 32k .. 32k+31) is produced by warp k % 2 into ring slot k % 4.
+        for (int k = (warp == kWarpBias0 ? 0 : 1); k < n_batches; k += 2) {
             const int slot = k % kNBias;
             if (!wait_u(&sh.bias_empty[slot], ((uint32_t)(k / kNBias) & 1u) ^ 1u, a.status, failed)) break;
             float *ring = bias_ring + slot * kBatch * kW;
-            for (int e = lane; e < kBatch * kW; e += 32) {
-                const int jj = e / kW, u = e % kW, j = k * kBatch + jj, t = t0 + u;
+            // Entry e = lane + 32 i: list entry j = 32k + e / 16, token u = e % 16.  Mask bits first
+            // (independent loads), then the biases of the routed entries.
+            uint32_t routed = 0;
+#pragma unroll
+            for (int i = 0; i < (kBatch * kW) / 32; ++i) {
+                const int e = lane + 32 * i, j = k * kBatch + (e >> 4), t = t0 + (e & 15);
+                if (j >= 1 && j < n_ch && t < a.T && !a.ignore_routing) {
+                    const int c = list[j];
+                    const uint64_t w = __ldg(a.mask + (bg * a.T + t) * a.W + (c >> 6));
+                    if ((w >> (c & 63)) & 1ull) routed |= 1u << i;
+                }
+            }
+#pragma unroll 1
+            for (int i = 0; i < (kBatch * kW) / 32; ++i) {
+                const int e = lane + 32 * i, j = k * kBatch + (e >> 4), u = e & 15, t = t0 + u;
                 float v = -INFINITY;
                 if (j < n_ch && t < a.T) {
                     if (j == 0 || a.ignore_routing) {
                         v = 0.f;
-                    } else {
+                    } else if ((routed >> i) & 1u) {
                         const int c = list[j];
                         const long long rowi = bg * a.T + t;
-                        if ((a.mask[rowi * a.W + (c >> 6)] >> (c & 63)) & 1ull) {
-                            const float dot = route_dot<D>(qbar + u * D, a.summary + (bg * a.Cf + c) * D);
-                            const float tau = a.tau[rowi];
-                            if (a.rc.kind == 0) {
-                                v = a.rc.sigma2 * (__fmul_rn(dot, a.rc.sscale) - tau);
-                            } else {
-                                const float m = __fsub_rn(__fmul_rn(dot, a.rc.xscale), tau);
-                                v = a.rc.bscale2 * log2f(fmaxf(m, 1e-37f));
-                            }
+                        const float dot = route_dot<D>(qbar + u * kQbarStride, a.summary + (bg * a.Cf + c) * D);
+                        const float tau = __ldg(a.tau + rowi);
+                        if (a.rc.kind == 0) {
+                            v = a.rc.sigma2 * (__fmul_rn(dot, a.rc.sscale) - tau);
+                        } else {
+                            const float m = __fsub_rn(__fmul_rn(dot, a.rc.xscale), tau);
+                            v = a.rc.bscale2 * log2f(fmaxf(m, 1e-37f));
                         }
                     }
                 }
@@ -254,219 +398,254 @@ k_attend_tok(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh.bias_full[slot]);
         }
-    } else if (warp >= kWarpFill0 && warp < kWarpFill0 + 4) {
-        // ---------------------------------------------------------------- smem -> TMEM
-        const int sp = warp & 3;
-        const uint32_t lane_addr = tb + ((uint32_t)(32 * sp) << 16);
-        const int key = 16 * sp + (lane & 15);        // M = 64 layout: lanes 0-15 of each quarter
-        const int d = 32 * sp + lane;
-        for (int j = 0; j < n_ch; ++j) {
-            const int st = j % kNst, s = j & 1;
-            if (!wait_u(&sh.tma_full[st], (uint32_t)(j / kNst) & 1u, a.status, failed)) break;
-            if (!wait_u(&sh.kv_free[s], ((uint32_t)(j / 2) & 1u) ^ 1u, a.status, failed)) break;
-            const unsigned char *stage = base + (size_t)st * kStage;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t r[32];
-                const unsigned char *row = stage + h * 8192 + key * 128;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(row + ((c ^ (key & 7)) << 4));
-                    r[4 * c] = v.x;
-                    r[4 * c + 1] = v.y;
-                    r[4 * c + 2] = v.z;
-                    r[4 * c + 3] = v.w;
-                }
-                tmem_st32(lane_addr + kColK + 64u * s + 32u * h, r);
-            }
-            {
-                uint32_t r[32];
-                const unsigned char *row = stage + 16384 + d * 128;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(row + ((c ^ (d & 7)) << 4));
-                    r[4 * c] = v.x;
-                    r[4 * c + 1] = v.y;
-                    r[4 * c + 2] = v.z;
-                    r[4 * c + 3] = v.w;
-                }
-                tmem_st32(lane_addr + kColV + 32u * s, r);
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&sh.kv_ready[s]);
-                mbar_arrive(&sh.tma_empty[st]);
-            }
-        }
     } else if (warp >= kWarpMma0 && warp < kWarpMma0 + kLanes) {
-        // ---------------------------------------------------------------- MMA issuer, lane L
+        // ---------------------------------------------------------------- MMA issuer, pipeline L
         const int L = warp - kWarpMma0;
-        constexpr uint32_t id_qk = idesc_bf16(64, 16, 0);
+        constexpr uint32_t id_qk = idesc_bf16(128, 16, 0);
         constexpr uint32_t id_pv = idesc_bf16(128, 16, 1);
         const uint32_t d_s = tb + kColS + 16u * L;
-        const uint32_t p_addr = smem_u32(pbuf + L * 2048);
+        const uint32_t p_base = smem_u32(pbuf + L * 8192);
+        // Phase bookkeeping: kw / vw = last pair whose k_ready / v_ready phase was waited,
+        // kq / vq = next pair whose k_free / v_free arrival is still owed.
+        int kw = -1, kq = 0, vw = -1, vq = 0;
+        int pend_u = -1, pend_p = 0, pend_i = 0;       // the item whose PV is still to issue
+        bool pend_a = false, pend_b = false;
         int it = 0;
-        wait_u(&sh.q_full, 0, a.status, failed);
-        for (int j = 0; j < n_ch && !failed; ++j) {
-            const int s = j & 1, k = j / kBatch, slot = k % kNBias;
-            if (j % kBatch == 0 && !wait_u(&sh.bias_full[slot], (uint32_t)(k / kNBias) & 1u, a.status, failed)) break;
-            if (!wait_u(&sh.kv_ready[s], (uint32_t)(j / 2) & 1u, a.status, failed)) break;
+        auto ensure_k = [&](int p) -> bool {
+            while (kw < p) {
+                const int r = kw + 1;
+                if (!wait_u(&sh.k_ready[r & 1], (uint32_t)(r >> 1) & 1u, a.status, failed)) return false;
+                kw = r;
+            }
+            return true;
+        };
+        auto try_k = [&](int p) -> bool {
+            while (kw < p) {
+                const int r = kw + 1;
+                if (!test_u(&sh.k_ready[r & 1], (uint32_t)(r >> 1) & 1u)) return false;
+                kw = r;
+            }
+            return true;
+        };
+        auto close_k = [&](int p) -> bool {           // arrive k_free for every pair < p
+            while (kq < p) {
+                if (!ensure_k(kq)) return false;
+                if (lane == 0) mma_commit(&sh.k_free[kq & 1]);
+                __syncwarp();
+                ++kq;
+            }
+            return true;
+        };
+        auto ensure_v = [&](int q) -> bool {
+            while (vw < q) {
+                const int r = vw + 1;
+                if (!wait_u(&sh.v_ready, (uint32_t)r & 1u, a.status, failed)) return false;
+                vw = r;
+            }
+            return true;
+        };
+        auto close_v = [&](int q) -> bool {           // arrive v_free for every pair < q
+            while (vq < q) {
+                if (!ensure_v(vq)) return false;
+                if (lane == 0) mma_commit(&sh.v_free);
+                __syncwarp();
+                ++vq;
+            }
+            return true;
+        };
+        auto do_pv = [&]() -> bool {
+            if (!close_v(pend_p) || !ensure_v(pend_p)) return false;
+            // One barrier per P buffer: the softmax can run at most one phase ahead of it.
+            if (!wait_u(&sh.p_full[L][pend_i & 1], (uint32_t)(pend_i >> 1) & 1u, a.status, failed)) return false;
             tc_fence_after();
-            const float *ring = bias_ring + slot * kBatch * kW + (j % kBatch) * kW;
+            if (lane == 0) {
+                const uint32_t pb = p_base + (uint32_t)(pend_i & 1) * 4096u;
+                const uint32_t d_o = tb + kColO + 16u * pend_u;
+                if (pend_a) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ts(d_o, tb + kColV + 8u * kk, smem_desc_noswz(pb + 256u * kk, 128, 2048), id_pv,
+                               (pend_p > 0 || kk > 0) ? 1u : 0u);
+                }
+                if (pend_b) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ts(d_o, tb + kColV + 32u + 8u * kk,
+                               smem_desc_noswz(pb + 1024u + 256u * kk, 128, 2048), id_pv, 1u);
+                }
+            }
+            __syncwarp();
+            pend_u = -1;
+            return true;
+        };
+        // Close the K and V phases of every pair below p in pair order, so that each blocking
+        // wait on a pair-r resource happens with all phases below r already closed.
+        auto close_all = [&](int p) -> bool {
+            while (kq < p || vq < p) {
+                const int r = min(kq, vq);
+                if (kq == r && !close_k(r + 1)) return false;
+                if (vq == r && r < p && !close_v(r + 1)) return false;
+            }
+            return true;
+        };
+        // Before blocking on a resource of pair p: issue the pending PV and close every phase
+        // of the pairs below p.
+        auto flush_below = [&](int p) -> bool {
+            if (pend_u >= 0 && pend_p < p && !do_pv()) return false;
+            return close_all(p);
+        };
+        bool ok = wait_u(&sh.q_full, 0, a.status, failed);
+        for (int p = 0; p < n_pairs && ok; ++p) {
+            const int k = p / kPairsPerBatch, slot = k % kNBias;
+            if (p % kPairsPerBatch == 0) {
+                const uint32_t par = (uint32_t)(k / kNBias) & 1u;
+                if (!test_u(&sh.bias_full[slot], par)) {
+                    if (!flush_below(p) || !wait_u(&sh.bias_full[slot], par, a.status, failed)) { ok = false; break; }
+                }
+            }
+            const float *ring = bias_ring + slot * kBatch * kW + (2 * p - k * kBatch) * kW;
+            const bool hb = 2 * p + 1 < n_ch;
             for (int m = 0; m < kTpl; ++m) {
                 const int u = L + kLanes * m;
-                if (ring[u] == -INFINITY) continue;                 // token did not route here
+                const bool ra = ring[u] != -INFINITY;
+                const bool rb = hb && ring[kW + u] != -INFINITY;
+                if (!ra && !rb) continue;
+                if (!try_k(p)) {
+                    if (!flush_below(p) || !ensure_k(p)) { ok = false; break; }
+                }
+                if (!close_k(p)) { ok = false; break; }
+                if (it > 0 && !wait_u(&sh.s_free[L], (uint32_t)(it - 1) & 1u, a.status, failed)) { ok = false; break; }
+                tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t qa = smem_u32(qwin + u * 4096);
+                    const uint32_t kslot = tb + kColK + 64u * (uint32_t)(p & 1);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint64_t bd = smem_desc_sw128(qa + (uint32_t)(kk / 4) * 2048u + (uint32_t)(kk % 4) * 32u, 16, 1024);
-                        mma_ts(d_s, tb + kColK + 64u * s + 8u * kk, bd, id_qk, kk > 0 ? 1u : 0u);
+                        const uint32_t qa = smem_u32(qwin + (kk >> 2) * 32768 + u * 2048) + (uint32_t)(kk & 3) * 32u;
+                        mma_ts(d_s, kslot + 8u * kk, smem_desc_sw128(qa, 16, 1024), id_qk, kk > 0 ? 1u : 0u);
                     }
                     mma_commit(&sh.s_full[L]);
                 }
                 __syncwarp();
-                if (!wait_u(&sh.p_full[L], (uint32_t)it & 1u, a.status, failed)) break;
-                tc_fence_after();
-                if (lane == 0) {
-#pragma unroll
-                    for (int kk = 0; kk < BC / 16; ++kk) {
-                        const uint64_t bd = smem_desc_noswz(p_addr + 256u * kk, 128, 1024);
-                        mma_ts(tb + kColO + 16u * u, tb + kColV + 32u * s + 8u * kk, bd, id_pv,
-                               (j > 0 || kk > 0) ? 1u : 0u);
-                    }
-                }
-                __syncwarp();
+                if (pend_u >= 0 && !do_pv()) { ok = false; break; }
+                pend_u = u;
+                pend_p = p;
+                pend_i = it;
+                pend_a = ra;
+                pend_b = rb;
                 ++it;
             }
-            if (lane == 0) mma_commit(&sh.kv_free[s]);
-            __syncwarp();
-            if ((j % kBatch == kBatch - 1 || j == n_ch - 1) && lane == 0) mbar_arrive(&sh.bias_empty[slot]);
-            __syncwarp();
+            if (!ok) break;
+            if (p % kPairsPerBatch == kPairsPerBatch - 1 || p == n_pairs - 1) {
+                if (lane == 0) mbar_arrive(&sh.bias_empty[slot]);
+                __syncwarp();
+            }
         }
-        if (lane == 0) mma_commit(&sh.o_done[L]);
+        if (ok && pend_u >= 0) ok = do_pv();
+        if (ok) ok = close_all(n_pairs);
+        if (lane == 0) mma_commit(&sh.o_done[L]);    // after the last MMA, failure or not
         __syncwarp();
-    } else if (warp >= kWarpSm0 && warp < kWarpSm0 + 4 * kLanes) {
-        // ---------------------------------------------------------------- softmax, lane L
-        const int L = (warp - kWarpSm0) / 4, sp = warp & 3;
-        const bool kl = lane < 16;                       // lanes 0-15 hold keys (M = 64 layout)
-        const int key_in = 16 * sp + (lane & 15);
+    } else if (warp >= kWarpSm0) {
+        // ---------------------------------------------------------------- softmax, pipeline L
+        const int L = (warp - kWarpSm0) >> 2, sp = warp & 3;
+        const int half = sp >> 1;                         // 0: chunk a keys, 1: chunk b keys
+        const int kp = 32 * sp + lane;                    // key row of S^T within the pair
         const uint32_t s_addr = tb + ((uint32_t)(32 * sp) << 16) + kColS + 16u * L;
-        unsigned char *pb = pbuf + L * 2048;
+        unsigned char *pb0 = pbuf + L * 8192;
         float lsum[kTpl];
 #pragma unroll
         for (int m = 0; m < kTpl; ++m) lsum[m] = 0.f;
         int it = 0, xph = 0;
-        for (int j = 0; j < n_ch; ++j) {
-            const int k = j / kBatch, slot = k % kNBias;
-            if (j % kBatch == 0) wait_u(&sh.bias_full[slot], (uint32_t)(k / kNBias) & 1u, a.status, failed);
-            const float *ring = bias_ring + slot * kBatch * kW + (j % kBatch) * kW;
-            const int c = list[j];
+        for (int p = 0; p < n_pairs; ++p) {
+            const int k = p / kPairsPerBatch, slot = k % kNBias;
+            if (p % kPairsPerBatch == 0)
+                wait_u(&sh.bias_full[slot], (uint32_t)(k / kNBias) & 1u, a.status, failed);
+            const float *ring = bias_ring + slot * kBatch * kW + (2 * p - k * kBatch) * kW;
+            const bool hb = 2 * p + 1 < n_ch;
 #pragma unroll 1
             for (int m = 0; m < kTpl; ++m) {
                 const int u = L + kLanes * m, t = t0 + u;
-                const float bias2 = ring[u];
-                if (bias2 == -INFINITY) continue;
+                const float ba = ring[u];
+                const float bb = hb ? ring[kW + u] : -INFINITY;
+                if (ba == -INFINITY && bb == -INFINITY) continue;
+                const float bias2 = half ? bb : ba;
+                const bool mine = bias2 != -INFINITY;
                 const bool ok = wait_u(&sh.s_full[L], (uint32_t)it & 1u, a.status, failed);
-                ++it;
-                float v[16];
-                if (ok) {
+                uint32_t sr[16];
+                if (ok && mine) {
                     tc_fence_after();
-                    uint32_t sr[16];
                     tmem_ld16(s_addr, sr);
                     tmem_wait_ld();
-                    const int kidx = c * BC + key_in;
-                    const bool valid = kl && (j > 0 || kidx <= t);
-#pragma unroll
-                    for (int h = 0; h < 16; ++h)
-                        v[h] = valid ? fmaf(__uint_as_float(sr[h]), a.qk_scale2, bias2) : -INFINITY;
-                } else {
-#pragma unroll
-                    for (int h = 0; h < 16; ++h) v[h] = -INFINITY;
                 }
-                float* mrow = mref + (u * 4 + sp) * 16;
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sh.s_free[L]);       // S slot free for the next QK
+                // Keys of the diagonal chunk are causal; all keys of routed chunks are < t.
+                const bool valid = ok && mine && (p > 0 || half == 1 || cd * BC + kp <= t);
                 float mh[16];
-                if (j == 0) {
-                    // Exact per-head maximum over the diagonal chunk: reduce-scatter over the
-                    // 16 key lanes, then across the lane's 4 warps.
-                    float w[16];
+                if (p == 0) {
+                    // Exact per-head maximum over the diagonal chunk (warps 0-1), shared with
+                    // the pipeline's 4 warps through an mbarrier exchange.
+                    if (half == 0) {
+                        float w[16];
 #pragma unroll
-                    for (int h = 0; h < 16; ++h) w[h] = v[h];
-#pragma unroll
-                    for (int o = 8, n = 8; o >= 1; o >>= 1, n >>= 1) {
-                        const bool upper = (lane & o) != 0;
-#pragma unroll
-                        for (int i = 0; i < n; ++i) {
-                            const float send = upper ? w[i] : w[i + n];
-                            const float keep = upper ? w[i + n] : w[i];
-                            w[i] = fmaxf(keep, __shfl_xor_sync(kFull, send, o));
-                        }
+                        for (int h = 0; h < 16; ++h) w[h] = valid ? __uint_as_float(sr[h]) * a.qk_scale2 : -INFINITY;
+                        const float mx = head_reduce<true>(w, lane);
+                        if ((lane & 1) == 0) mpart[(u * 2 + sp) * 16 + (lane >> 1)] = mx;
                     }
-                    if (kl) mpart[(u * 4 + sp) * 16 + lane] = w[0];
-                    // Exchange across the lane's 4 warps through an mbarrier (bounded wait).
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&sh.x_bar[L]);
                     wait_u(&sh.x_bar[L], (uint32_t)xph & 1u, a.status, failed);
                     ++xph;
 #pragma unroll
                     for (int h = 0; h < 16; ++h) {
-                        float x = mpart[(u * 4 + 0) * 16 + h];
-                        x = fmaxf(x, mpart[(u * 4 + 1) * 16 + h]);
-                        x = fmaxf(x, mpart[(u * 4 + 2) * 16 + h]);
-                        x = fmaxf(x, mpart[(u * 4 + 3) * 16 + h]);
+                        const float x = fmaxf(mpart[(u * 2) * 16 + h], mpart[(u * 2 + 1) * 16 + h]);
                         mh[h] = x == -INFINITY ? 0.f : x;
                     }
-                    if (kl) mrow[lane] = mh[lane & 15];
-                    __syncwarp();
+                    if (lane < 16) mref[u * 16 + lane] = mh[lane];   // same values from every warp
                 } else {
 #pragma unroll
-                    for (int h = 0; h < 16; ++h) mh[h] = mrow[h];
+                    for (int h = 0; h < 16; h += 4) {
+                        const float4 x = *reinterpret_cast<const float4 *>(mref + u * 16 + h);
+                        mh[h] = x.x;
+                        mh[h + 1] = x.y;
+                        mh[h + 2] = x.z;
+                        mh[h + 3] = x.w;
+                    }
                 }
-                if (ok) {
-                    float p[16];
-                    bool clamped = false;
+                if (mine) {
+                    float pr[16];
+                    float emax = -INFINITY;
 #pragma unroll
                     for (int h = 0; h < 16; ++h) {
-                        float e = v[h] - mh[h];
-                        if (e > kMaxExcess) { e = kMaxExcess; clamped = true; }
-                        p[h] = fast_exp2(e);
+                        const float e = valid ? fmaf(__uint_as_float(sr[h]), a.qk_scale2, bias2 - mh[h]) : -INFINITY;
+                        emax = fmaxf(emax, e);
+                        pr[h] = fast_exp2(fminf(e, kMaxExcess));
                     }
-                    if (__any_sync(kFull, clamped) && lane == 0) report(a.status, DASH_ERR_RANGE_CLAMPED);
-                    if (kl) {
-                        uint4 lo, hi;
-                        lo.x = pack_bf16x2(p[0], p[1]);
-                        lo.y = pack_bf16x2(p[2], p[3]);
-                        lo.z = pack_bf16x2(p[4], p[5]);
-                        lo.w = pack_bf16x2(p[6], p[7]);
-                        hi.x = pack_bf16x2(p[8], p[9]);
-                        hi.y = pack_bf16x2(p[10], p[11]);
-                        hi.z = pack_bf16x2(p[12], p[13]);
-                        hi.w = pack_bf16x2(p[14], p[15]);
-                        const int kq = key_in;
-                        *reinterpret_cast<uint4 *>(pb + (kq & 7) * 16 + (kq >> 3) * 128) = lo;
-                        *reinterpret_cast<uint4 *>(pb + 1024 + (kq & 7) * 16 + (kq >> 3) * 128) = hi;
-                    }
+                    if (__any_sync(kFull, emax > kMaxExcess) && lane == 0) report(a.status, DASH_ERR_RANGE_CLAMPED);
+                    uint4 lo, hi;
+                    lo.x = pack_bf16x2(pr[0], pr[1]);
+                    lo.y = pack_bf16x2(pr[2], pr[3]);
+                    lo.z = pack_bf16x2(pr[4], pr[5]);
+                    lo.w = pack_bf16x2(pr[6], pr[7]);
+                    hi.x = pack_bf16x2(pr[8], pr[9]);
+                    hi.y = pack_bf16x2(pr[10], pr[11]);
+                    hi.z = pack_bf16x2(pr[12], pr[13]);
+                    hi.w = pack_bf16x2(pr[14], pr[15]);
+                    unsigned char *pb = pb0 + (it & 1) * 4096 + (kp & 7) * 16 + (kp >> 3) * 128;
+                    *reinterpret_cast<uint4 *>(pb) = lo;
+                    *reinterpret_cast<uint4 *>(pb + 2048) = hi;
                     fence_proxy_async();
-                    tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&sh.p_full[L]);
-                    // Row sums: reduce-scatter the 16 head values over the 16 key lanes.
-#pragma unroll
-                    for (int o = 8, n = 8; o >= 1; o >>= 1, n >>= 1) {
-                        const bool upper = (lane & o) != 0;
-#pragma unroll
-                        for (int i = 0; i < n; ++i) {
-                            const float send = upper ? p[i] : p[i + n];
-                            const float keep = upper ? p[i + n] : p[i];
-                            p[i] = keep + __shfl_xor_sync(kFull, send, o);
-                        }
-                    }
-                    lsum[m] += kl ? p[0] : 0.f;
+                    if (lane == 0) mbar_arrive(&sh.p_full[L][it & 1]);
+                    const float ls = head_reduce<false>(pr, lane);
+                    if ((lane & 1) == 0) lsum[m] += ls;
+                } else {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sh.p_full[L][it & 1]);
                 }
+                ++it;
             }
-            if (j % kBatch == kBatch - 1 || j == n_ch - 1) {
+            if (p % kPairsPerBatch == kPairsPerBatch - 1 || p == n_pairs - 1) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sh.bias_empty[slot]);
             }
@@ -474,7 +653,7 @@ k_attend_tok(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
         // ------------------------------------------------------------ epilogue
 #pragma unroll
         for (int m = 0; m < kTpl; ++m)
-            if (kl) lpart[((L + kLanes * m) * 4 + sp) * 16 + lane] = lsum[m];
+            if ((lane & 1) == 0) lpart[((L + kLanes * m) * 4 + sp) * 16 + (lane >> 1)] = lsum[m];
         const bool ok = wait_u(&sh.o_done[L], 0, a.status, failed);
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.x_bar[L]);
@@ -492,7 +671,7 @@ k_attend_tok(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
                 if (t < a.T) {
 #pragma unroll
                     for (int h = 0; h < 16; ++h) {
-                        const float* lp = lpart + (u * 4) * 16 + h;
+                        const float *lp = lpart + (u * 4) * 16 + h;
                         const float l = (lp[0] + lp[16]) + (lp[32] + lp[48]);
                         const float val = l > 0.f ? __uint_as_float(orow[h]) / l : 0.f;
                         out[(((long long)b * a.Hq + g * G + h) * a.T + t) * D + dd] = __float2bfloat16_rn(val);
@@ -548,7 +727,7 @@ size_t attend_tok_vt_bytes(int B, int Hkv, int T, int D) {
 }
 
 bool attend_tok_supported(const StageArgs &a) {
-    return a.D == 128 && a.G == 16 && a.Bc == 64 && a.C <= 8192;
+    return a.D == 128 && a.G == 16 && a.Bc == 64 && a.C <= kMaxChunks;
 }
 
 cudaError_t launch_attend_tok(const StageArgs &a, cudaStream_t st) {
@@ -580,15 +759,17 @@ cudaError_t launch_attend_tok(const StageArgs &a, cudaStream_t st) {
     TokArgs ta;
     ta.s = a;
     ta.n_win = (a.T + kW - 1) / kW;
-    size_t off = (size_t)kNst * kStage;
-    ta.off_q = off;      off += (size_t)kW * 4096;
-    ta.off_p = off;      off += (size_t)kLanes * 2048;
+    size_t off = 0;
+    ta.off_q = off;      off += (size_t)2 * kW * 2048;
+    ta.off_k = off;      off += (size_t)2 * kKStage;
+    ta.off_v = off;      off += kVStage;
+    ta.off_p = off;      off += (size_t)kLanes * 2 * 4096;
     ta.off_bias = off;   off += (size_t)kNBias * kBatch * kW * 4;
-    ta.off_qbar = off;   off += (size_t)kW * 128 * 4;
-    ta.off_mref = off;   off += (size_t)kW * 4 * 16 * 4;
-    ta.off_mpart = off;  off += (size_t)kW * 4 * 16 * 4;
+    ta.off_qbar = off;   off += (size_t)kW * kQbarStride * 4;
+    ta.off_mref = off;   off += (size_t)kW * 16 * 4;
+    ta.off_mpart = off;  off += (size_t)kW * 2 * 16 * 4;
     ta.off_lpart = off;  off += (size_t)kW * 4 * 16 * 4;
-    ta.off_list = off;   off += (size_t)((a.C + 8) & ~7) * 2;
+    ta.off_list = off;   off += ((size_t)(a.C + 2) * 2 + 15) & ~(size_t)15;
     const size_t smem = off + 1024;
     e = cudaFuncSetAttribute(k_attend_tok, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -6,7 +6,7 @@
 namespace dash {
 
 constexpr int kStage0Warps = 4;     // chunks summarised per CTA
-constexpr int kRouteThreads = 256;  // Stage 1 CTA size
+constexpr int kRouteThreads = 512;  // Stage 1 CTA size (one warp per row in the tau solve)
 constexpr int kAttnWarps = 4;       // Stage 2 (mma.sync path) units per CTA
 constexpr int kSub = 32;            // keys per Stage 2 sub-block
 

@@ -6,7 +6,7 @@
 // share one sparse support.  aixai.ru "DashAttention ...", "Трёхстадийная архитектура": the
 // result is handed to Stage 2 as a bit-packed active-block mask (64-bit words).
 //
-// CTA = (b, g, RT consecutive rows of one query chunk), 256 threads:
+// CTA = (b, g, RT consecutive rows of one query chunk), 512 threads:
 //   1. qbar[r] = mean of the G query heads of group g at row t0 + r     (shared memory)
 //   2. x[r][c] = (qbar[r] . summary[c]) * (alpha-1) gamma / sqrt(D) for every routable
 //      chunk c < c_t: 4 lanes per chunk, each owning an interleaved quarter of d (coalesced
@@ -70,9 +70,12 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(StageArgs a) {
         float acc[RT];
 #pragma unroll
         for (int r = 0; r < RT; ++r) acc[r] = 0.f;
-#pragma unroll 2
+        float4 sv4[D / 16];                       // all loads of the slice in flight at once
+#pragma unroll
+        for (int i = 0; i < D / 16; ++i) sv4[i] = __ldg(s4 + 4 * i + kslice);
+#pragma unroll
         for (int i = 0; i < D / 16; ++i) {
-            const float4 sv = __ldg(s4 + 4 * i + kslice);
+            const float4 sv = sv4[i];
 #pragma unroll
             for (int r = 0; r < RT; ++r) {
                 const float4 qq = reinterpret_cast<const float4 *>(qbar + r * D)[4 * i + kslice];

@@ -120,6 +120,12 @@ __device__ __forceinline__ void tma_load_4d(void *smem, const CUtensorMap *map, 
 __device__ __forceinline__ void fence_proxy_async() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// Asynchronous copy shared memory -> tensor memory of a 128-row x 256-bit slab: row r of the
+// matrix the descriptor describes lands in lane r, its 16 bf16 elements in 8 columns.
+// Completion is tracked by tcgen05.commit like an MMA.
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t desc) {
+    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+}
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
                  "r"(ncols));
