@@ -464,12 +464,10 @@ def main():
     d2h = ho.numel() * ho.element_size()
 
     pk, pk_kind = peaks()
-    # Stage 2 kernel dash_prefill runs: the per-token kernel (after a V^T transpose, timed with
-    # it) when the workspace holds V^T scratch, else the tile kernel.
-    per_token = dash.attend_workspace_size(prm) > 256
-    s2_kernel = "k_attend_tok" if per_token else "k_attend_tc"
-    s2_note = ", V^T transpose included" if per_token else ""
-    launches_per_step = 4 if per_token else 3
+    # Stage 2 kernel dash_prefill runs for this shape (D = 128, G >= 8): the tcgen05 tile kernel.
+    s2_kernel = "k_attend_tc"
+    s2_note = ""
+    launches_per_step = 3                     # k_stage0, k_route, k_attend_tc
     s2_tflops = stats["active_flops"] / (stage["stage2"] / 1e3) / 1e12
     sb = stage01_bytes(cfg)
     s01_gbs = (sb["stage0"] + sb["stage1"]) / ((stage["stage0"] + stage["stage1"]) / 1e3) / 1e9

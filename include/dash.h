@@ -63,10 +63,10 @@ typedef enum {
     DASH_ERR_WORKSPACE_TOO_SMALL = 3,
     DASH_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed */
     DASH_ERR_DEVICE_TIMEOUT = 5,     /* a device wait or iteration cap ran out */
-    DASH_ERR_RANGE_CLAMPED = 6       /* a routed logit exceeded its token's diagonal-chunk
-                                        maximum by more than 2^126 (log2 units above the
-                                        reference); the probability was clamped, the output
-                                        of that row is not exact */
+    DASH_ERR_RANGE_CLAMPED = 6       /* a logit exceeded its row's reference (the maximum
+                                        over the first 64 keys of the diagonal chunk) by more
+                                        than 100 in log2 units; its probability was clamped,
+                                        the output of that row is not exact */
 } dash_status_t;
 
 enum {

@@ -7,17 +7,26 @@
 // zero probability are masked; the diagonal chunk keeps its own branch.
 //
 // One CTA = one tile of 128 query rows of one (b, g): 128/G consecutive tokens x G heads
-// (G >= 8).  The tile walks the UNION of its tokens' active chunks (the OR of their mask
-// words, which carry each token's diagonal bit), 64 keys per pipeline block, in ascending
-// order.  A row whose token did not route to a chunk gets bias -inf there; keys above the
-// row's position are masked.  Per block:
+// (G >= 8); the tile's tokens share one diagonal chunk.  The tile walks the UNION of its
+// tokens' active chunks (the OR of their mask words, which carry each token's diagonal bit),
+// 64 keys per pipeline block: the diagonal chunk first, then the others in ascending order.
+// A row whose token did not route to a chunk gets bias -inf there; keys above the row's
+// position are masked.  Per block:
 //   S[128 x 64]  = Q K^T      tcgen05.mma kind::f16, A = Q from TMEM, B = K (smem, TMA)
-//   softmax      one thread per row (4 warps), online max with lazy rescale, fp32
-//   O[128 x 128] += P V       tcgen05.mma, A = P (bf16, TMEM, aliased into S), B = V (smem)
-// Warp roles: 0 TMA producer (K/V blocks, 128B-swizzled, 2 stages), 1 MMA issuer and TMEM
+//   softmax      two threads per row (8 warps, 32 keys each), fp32; releases S as soon as
+//                it has loaded it, so the next block's Q K^T overlaps these exponentials
+//   O[128 x 128] += P V       tcgen05.mma, A = P (bf16, smem, 128B-swizzled, double-buffered),
+//                            B = V (smem, TMA)
+// Softmax reference: the first block (the diagonal chunk's first 64 keys, which hold at least
+// one causally visible key of every row) gives each row its exact maximum m over that block;
+// every later probability is 2^(s - m) against that fixed reference, so O is never rescaled
+// and the two threads of a row exchange nothing but their partial sums.  A logit more than
+// 2^100 above the reference (log2 units) is clamped there (no fp32 overflow for up to 2^17
+// keys) and reported as DASH_ERR_RANGE_CLAMPED.
+// Warp roles: 0 TMA producer (K and V rings, 128B-swizzled, 2 stages each), 1 MMA issuer and TMEM
 // owner, 2 routing-bias producer (recomputes qbar.summary with Stage 1's exact arithmetic,
-// 32 chunks per batch, double-buffered), 4-7 softmax + epilogue.  TMEM: Q 64 columns,
-// S/P 64, O 128 = 256 columns, so two CTAs share an SM.  Every wait is bounded; on timeout
+// 32 chunks per batch, double-buffered), 4-11 softmax + epilogue.  TMEM: Q 64 columns,
+// S 64, O 128 = 256 columns, so two CTAs share an SM.  Every wait is bounded; on timeout
 // the CTA records DASH_ERR_DEVICE_TIMEOUT and drains.
 #include "kernels.cuh"
 #include "tc_common.cuh"
@@ -26,18 +35,26 @@ namespace dash {
 using namespace tcx;
 namespace {
 
-constexpr int kTcThreads = 256;
+constexpr int kTcThreads = 384;
+constexpr int kSmThreads = 256;          // softmax warps 4-11
 constexpr int kBlk = 64;                 // keys per pipeline block
 constexpr int kStages = 2;
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColQ = 0, kColS = 64, kColP = 64, kColO = 128;
+constexpr uint32_t kColQ = 0, kColS = 64, kColO = 128;
 constexpr int kBiasBatch = 32;
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpBias = 2, kWarpSm0 = 4;
-constexpr uint32_t kStageBytes = 4 * 8192;  // K panels (d 0-63, 64-127), V panels
-constexpr float kRescaleThreshold = 8.f;    // log2 units, as in lazy-rescale FlashAttention
+constexpr uint32_t kKBytes = 2 * 8192;      // K block: panels d 0-63, 64-127 (64 keys x 128 B)
+constexpr uint32_t kVBytes = 2 * 8192;      // V block, same layout
+constexpr uint32_t kPBytes = 128 * 128;     // P block: 128 rows x 64 keys bf16
+constexpr uint32_t kOffV = kStages * kKBytes, kOffP = kOffV + kStages * kVBytes,
+                   kRingBytes = kOffP + 2 * kPBytes;
+constexpr float kMaxExcess = 100.f;         // log2 units above the row reference
 
 struct TcShared {
-    uint64_t full[kStages], empty[kStages], s_full, p_full, o_full;
+    uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
+    uint64_t s_full, s_free, p_full[2], o_full;   // p_full per P buffer: at most one phase ahead
+    float mpair[2][128];                 // partial row maxima of the first block
+    float lpair[2][128];                 // partial row sums
     uint32_t tmem_base;
     int n_chunks;
     int failed;
@@ -87,11 +104,15 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&sh.full[s], 1);
-            mbar_init(&sh.empty[s], 1);
+            mbar_init(&sh.k_full[s], 1);
+            mbar_init(&sh.k_empty[s], 1);
+            mbar_init(&sh.v_full[s], 1);
+            mbar_init(&sh.v_empty[s], 1);
         }
         mbar_init(&sh.s_full, 1);
-        mbar_init(&sh.p_full, 4);
+        mbar_init(&sh.s_free, kSmThreads / 32);
+        mbar_init(&sh.p_full[0], kSmThreads / 32);
+        mbar_init(&sh.p_full[1], kSmThreads / 32);
         mbar_init(&sh.o_full, 1);
         sh.failed = 0;
         fence_mbar_init();
@@ -149,8 +170,10 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
             }
         }
     }
-    // Softmax warps: this thread's row, its token and head; Q row into TMEM columns [0, 64).
+    // Softmax warps: this thread's row, its token and head; Q row into TMEM columns [0, 64)
+    // (warps 4-7 the first 64 dims, warps 8-11 the rest).
     const int sp = warp & 3;                     // TMEM sub-partition of this warp
+    const int khalf = (warp - kWarpSm0) >> 2;    // softmax warps: which 32 keys of a block
     const int row = 32 * sp + lane;              // valid for the softmax warps
     const int u_row = row / G;                   // token of the row within the tile
     const int t_row = t0 + u_row;
@@ -161,19 +184,17 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
     if (warp >= kWarpSm0) {
         const __nv_bfloat16 *qr = reinterpret_cast<const __nv_bfloat16 *>(a.q) +
                                   (((long long)b * a.Hq + h_row) * a.T + (row_ok ? t_row : 0)) * D;
-        for (int half = 0; half < 2; ++half) {
-            uint32_t r[32];
+        uint32_t r[32];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                uint4 v = row_ok ? *reinterpret_cast<const uint4 *>(qr + half * 64 + 8 * j)
-                                 : make_uint4(0, 0, 0, 0);
-                r[4 * j] = v.x;
-                r[4 * j + 1] = v.y;
-                r[4 * j + 2] = v.z;
-                r[4 * j + 3] = v.w;
-            }
-            tmem_st32(tb + ((uint32_t)(32 * sp) << 16) + kColQ + 32 * half, r);
+        for (int j = 0; j < 8; ++j) {
+            uint4 v = row_ok ? *reinterpret_cast<const uint4 *>(qr + khalf * 64 + 8 * j)
+                             : make_uint4(0, 0, 0, 0);
+            r[4 * j] = v.x;
+            r[4 * j + 1] = v.y;
+            r[4 * j + 2] = v.z;
+            r[4 * j + 3] = v.w;
         }
+        tmem_st32(tb + ((uint32_t)(32 * sp) << 16) + kColQ + 32 * khalf, r);
         tmem_wait_st();
     }
     tc_fence_before();
@@ -183,66 +204,90 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
     const int n_chunks = sh.n_chunks;
     const int n_blocks = n_chunks * NSUB;
     bool failed = false;
+    // Walk order: the diagonal chunk (the largest, last entry of the ascending list) first.
+    auto chunk_at = [&](int ci) -> int { return (int)list[ci == 0 ? n_chunks - 1 : ci - 1]; };
 
     if (warp == kWarpTma) {
         // ------------------------------------------------------------ TMA producer
-        // The whole warp runs the loop (converged); lane 0 issues the copies.
-        int issued = 0;
-        for (int i = 0; i < n_blocks; ++i) {
+        // The whole warp runs the loop (converged); lane 0 issues the copies.  K runs one
+        // block ahead of V: the K stage frees when Q K^T completes, the V stage after P V.
+        int k_issued = 0, v_issued = 0;
+        auto key0_of = [&](int i) { return chunk_at(i / NSUB) * BC + (i % NSUB) * kBlk; };
+        auto issue = [&](bool is_v, int i) -> bool {
             const int s = i % kStages;
             const uint32_t ph = (uint32_t)(i / kStages) & 1u;
-            if (!wait_or_fail(&sh.empty[s], ph ^ 1u, a.status, failed)) break;
-            issued = i + 1;
+            uint64_t *empty = is_v ? &sh.v_empty[s] : &sh.k_empty[s];
+            uint64_t *full = is_v ? &sh.v_full[s] : &sh.k_full[s];
+            if (!wait_or_fail(empty, ph ^ 1u, a.status, failed)) return false;
             if (lane == 0) {
-                const int key0 = (int)list[i / NSUB] * BC + (i % NSUB) * kBlk;
-                unsigned char *st = base + (size_t)s * kStageBytes;
-                mbar_arrive_expect_tx(&sh.full[s], kStageBytes);
-                tma_load_3d(st, &tmK, 0, key0, (int)bg, &sh.full[s]);
-                tma_load_3d(st + 8192, &tmK, 64, key0, (int)bg, &sh.full[s]);
-                tma_load_3d(st + 16384, &tmV, 0, key0, (int)bg, &sh.full[s]);
-                tma_load_3d(st + 24576, &tmV, 64, key0, (int)bg, &sh.full[s]);
+                const CUtensorMap *map = is_v ? &tmV : &tmK;
+                unsigned char *st = base + (is_v ? kOffV + (size_t)s * kVBytes : (size_t)s * kKBytes);
+                mbar_arrive_expect_tx(full, kKBytes);
+                tma_load_3d(st, map, 0, key0_of(i), (int)bg, full);
+                tma_load_3d(st + 8192, map, 64, key0_of(i), (int)bg, full);
             }
             __syncwarp();
+            if (is_v) v_issued = i + 1; else k_issued = i + 1;
+            return true;
+        };
+        if (n_blocks > 0) issue(false, 0);
+        for (int i = 0; i < n_blocks && !failed; ++i) {
+            if (i + 1 < n_blocks && !issue(false, i + 1)) break;
+            if (!issue(true, i)) break;
         }
         if (failed) {
-            // Bounded wait for the copies still in flight (the last one per stage).
-            for (int j = max(0, issued - kStages); j < issued; ++j)
-                mbar_wait_bounded(&sh.full[j % kStages], (uint32_t)(j / kStages) & 1u);
+            // Bounded wait for the copies still in flight (the last ones per ring).
+            for (int j = max(0, k_issued - kStages); j < k_issued; ++j)
+                mbar_wait_bounded(&sh.k_full[j % kStages], (uint32_t)(j / kStages) & 1u);
+            for (int j = max(0, v_issued - kStages); j < v_issued; ++j)
+                mbar_wait_bounded(&sh.v_full[j % kStages], (uint32_t)(j / kStages) & 1u);
             __syncwarp();
         }
     } else if (warp == kWarpMma) {
         // ------------------------------------------------------------ MMA issuer
-        // The whole warp runs the loop (converged); lane 0 issues the MMAs and commits.
+        // The whole warp runs the loop (converged); lane 0 issues the MMAs and commits.  Block
+        // i's Q K^T is issued as soon as the softmax has loaded S(i-1); P(i-1) V follows once
+        // the softmax has written P(i-1).
         constexpr uint32_t id_qk = idesc_bf16(128, kBlk, 0);
         constexpr uint32_t id_pv = idesc_bf16(128, D, 1);
-        for (int i = 0; i < n_blocks; ++i) {
-            const int s = i % kStages;
-            const uint32_t ph = (uint32_t)(i / kStages) & 1u;
-            if (!wait_or_fail(&sh.full[s], ph, a.status, failed)) break;
-            tc_fence_after();
-            const uint32_t st = smem_u32(base + (size_t)s * kStageBytes);
-            if (lane == 0) {
+        for (int i = 0; i <= n_blocks; ++i) {
+            if (i < n_blocks) {
+                const int s = i % kStages;
+                if (!wait_or_fail(&sh.k_full[s], (uint32_t)(i / kStages) & 1u, a.status, failed)) break;
+                if (i > 0 && !wait_or_fail(&sh.s_free, (uint32_t)(i - 1) & 1u, a.status, failed)) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t kst = smem_u32(base + (size_t)s * kKBytes);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t bd = smem_desc_sw128(st + (uint32_t)(kk / 4) * 8192u +
-                                                            (uint32_t)(kk % 4) * 32u,
-                                                        16, 1024);
-                    mma_ts(tb + kColS, tb + kColQ + 8u * kk, bd, id_qk, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t bd = smem_desc_sw128(kst + (uint32_t)(kk / 4) * 8192u +
+                                                                (uint32_t)(kk % 4) * 32u,
+                                                            16, 1024);
+                        mma_ts(tb + kColS, tb + kColQ + 8u * kk, bd, id_qk, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&sh.s_full);
+                    mma_commit(&sh.k_empty[s]);
                 }
-                mma_commit(&sh.s_full);
+                __syncwarp();
             }
-            __syncwarp();
-            if (!wait_or_fail(&sh.p_full, (uint32_t)i & 1u, a.status, failed)) break;
-            tc_fence_after();
-            if (lane == 0) {
+            if (i > 0) {
+                const int j = i - 1, s = j % kStages;
+                if (!wait_or_fail(&sh.v_full[s], (uint32_t)(j / kStages) & 1u, a.status, failed)) break;
+                if (!wait_or_fail(&sh.p_full[j & 1], (uint32_t)(j >> 1) & 1u, a.status, failed)) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t vst = smem_u32(base + kOffV + (size_t)s * kVBytes);
+                    const uint32_t pst = smem_u32(base + kOffP + (size_t)(j & 1) * kPBytes);
 #pragma unroll
-                for (int kk = 0; kk < kBlk / 16; ++kk) {
-                    const uint64_t bd = smem_desc_sw128(st + 16384u + (uint32_t)kk * 2048u, 8192, 1024);
-                    mma_ts(tb + kColO, tb + kColP + 8u * kk, bd, id_pv, (i > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < kBlk / 16; ++kk) {
+                        const uint64_t ad = smem_desc_sw128(pst + (uint32_t)kk * 32u, 16, 1024);
+                        const uint64_t bd = smem_desc_sw128(vst + (uint32_t)kk * 2048u, 8192, 1024);
+                        mma_ss(tb + kColO, ad, bd, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&sh.v_empty[s]);
                 }
-                mma_commit(&sh.empty[s]);
+                __syncwarp();
             }
-            __syncwarp();
         }
         if (lane == 0) mma_commit(&sh.o_full);          // tracks every MMA issued above
         __syncwarp();
@@ -255,7 +300,7 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                 const int k = e / RT, u = e % RT, ci = bt * kBiasBatch + k;
                 float v = 0.f;
                 if (ci < n_chunks && !a.ignore_routing) {
-                    const int c = list[ci], t = t0 + u;
+                    const int c = chunk_at(ci), t = t0 + u;
                     const int ctu = t / BC;
                     if (t >= a.T || c > ctu) {
                         v = -INFINITY;
@@ -279,21 +324,22 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                 buf[e] = v;
             }
             __syncwarp();
-            named_sync(1, 32 + 128);
+            named_sync(1, 32 + kSmThreads);
         }
     } else if (warp >= kWarpSm0) {
         // ------------------------------------------------------------ softmax
+        // Two threads per row: warps 4-7 take keys [0, 32) of every block, warps 8-11 keys
+        // [32, 64).  Every named barrier below is passed by all softmax warps, failure or not.
         const uint32_t lane_base = tb + ((uint32_t)(32 * sp) << 16);
         const int ct_row = t_row / BC;
-        float m_ref = -INFINITY, l_sum = 0.f;
+        float m_ref = 0.f, l_sum = 0.f, emax_all = -INFINITY;
         for (int i = 0; i < n_blocks; ++i) {
             const int ci = i / NSUB;
-            // Every batch boundary is passed even after a failure: the bias warp waits there.
-            if (ci % kBiasBatch == 0 && i % NSUB == 0) named_sync(1, 32 + 128);
-            if (!wait_or_fail(&sh.s_full, (uint32_t)i & 1u, a.status, failed)) continue;
-            tc_fence_after();
-            const int c = list[ci];
-            const int key0 = c * BC + (i % NSUB) * kBlk;
+            if (ci % kBiasBatch == 0 && i % NSUB == 0) named_sync(1, 32 + kSmThreads);
+            const bool ok = wait_or_fail(&sh.s_full, (uint32_t)i & 1u, a.status, failed);
+            if (ok) tc_fence_after();
+            const int c = chunk_at(ci);
+            const int key0 = c * BC + (i % NSUB) * kBlk + 32 * khalf;
             float bias2;
             bool diag = false;
             if (!row_ok || c > ct_row) {
@@ -306,71 +352,101 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                                          : bias_s[((ci / kBiasBatch) & 1) * kBiasBatch * RT +
                                                   (ci % kBiasBatch) * RT + u_row];
             }
-            uint32_t sv[2][32];
-            tmem_ld32(lane_base + kColS, sv[0]);
-            tmem_ld32(lane_base + kColS + 32, sv[1]);
-            tmem_wait_ld();
-            float mx = -INFINITY;
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    float v = fmaf(__uint_as_float(sv[h][j]), a.qk_scale2, bias2);
-                    if (diag && key0 + 32 * h + j > t_row) v = -INFINITY;
-                    sv[h][j] = __float_as_uint(v);
-                    mx = fmaxf(mx, v);
-                }
-            // Lazy rescale: move the reference only when the block max exceeds it by more than
-            // the threshold (values up to 2^threshold above the reference are exact in fp32).
-            float f = 1.f;
-            if (mx > m_ref + kRescaleThreshold) {
-                if (m_ref != -INFINITY && l_sum > 0.f) {
-                    f = fast_exp2(m_ref - mx);
-                    l_sum *= f;
-                }
-                m_ref = mx;
+            // The diagonal chunk is the tile's last one (every token of the tile shares it).
+            const bool dead = __all_sync(kFull, bias2 == -INFINITY);
+            uint32_t sv[32];
+            if (ok && (i == 0 || !dead)) {
+                tmem_ld32(lane_base + kColS + 32 * khalf, sv);
+                tmem_wait_ld();
             }
-            // TMEM loads/stores are warp-wide: the warp rescales its O rows together whenever
-            // any of them needs it (factor 1 for the others).  O is stable here: the commit
-            // behind s_full also tracked the previous P V.
-            if (__any_sync(kFull, f != 1.f)) {
-#pragma unroll 1
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    uint32_t o[32];
-                    tmem_ld32(lane_base + kColO + 32 * q4, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
-                    tmem_st32(lane_base + kColO + 32 * q4, o);
-                }
-            }
-            const float mu = m_ref == -INFINITY ? 0.f : m_ref;
-            uint32_t pw[32];
-            float psum = 0.f;
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float p0 = fast_exp2(__uint_as_float(sv[h][2 * j]) - mu);
-                    const float p1 = fast_exp2(__uint_as_float(sv[h][2 * j + 1]) - mu);
-                    psum += p0 + p1;
-                    pw[16 * h + j] = pack_bf16x2(p0, p1);
-                }
-            l_sum += psum;
-            tmem_st32(lane_base + kColP, pw);
-            tmem_wait_st();
+            // S is in registers: the next block's Q K^T may overwrite it.
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.p_full);
+            if (lane == 0) mbar_arrive(&sh.s_free);
+            if (i == 0) {
+                // First block: exact row maximum over the diagonal chunk's first 64 keys, the
+                // fixed reference of every later block.
+                float mx = -INFINITY;
+                if (ok) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float v = (row_ok && key0 + j <= t_row)
+                                            ? __uint_as_float(sv[j]) * a.qk_scale2 : -INFINITY;
+                        mx = fmaxf(mx, v);
+                    }
+                }
+                sh.mpair[khalf][row] = mx;
+                named_sync(2, kSmThreads);
+                const float m2 = fmaxf(sh.mpair[0][row], sh.mpair[1][row]);
+                m_ref = m2 == -INFINITY ? 0.f : m2;
+            }
+            if (!ok) continue;
+            const float c2 = bias2 - m_ref;              // -inf for rows that do not attend
+            uint32_t pw[16];
+            if (dead) {
+                // None of the warp's 32 rows attends this chunk: P = 0, no exponentials.
+#pragma unroll
+                for (int j = 0; j < 16; ++j) pw[j] = 0u;
+            } else {
+                float psum = 0.f, emax = -INFINITY;
+                if (c == ct_max) {
+                    const int lim = t_row - key0;            // keys j > lim are in the future
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float e0 = 2 * j <= lim ? fmaf(__uint_as_float(sv[2 * j]), a.qk_scale2, c2) : -INFINITY;
+                        const float e1 = 2 * j + 1 <= lim ? fmaf(__uint_as_float(sv[2 * j + 1]), a.qk_scale2, c2) : -INFINITY;
+                        emax = fmaxf(emax, fmaxf(e0, e1));
+                        const uint32_t pk = pack_bf16x2(fast_exp2(fminf(e0, kMaxExcess)),
+                                                        fast_exp2(fminf(e1, kMaxExcess)));
+                        // l sums the bf16 weights the PV MMA multiplies, so O / l is normalised
+                        // exactly even when one key dominates the row.
+                        psum += __uint_as_float(pk << 16) + __uint_as_float(pk & 0xffff0000u);
+                        pw[j] = pk;
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float e0 = fmaf(__uint_as_float(sv[2 * j]), a.qk_scale2, c2);
+                        const float e1 = fmaf(__uint_as_float(sv[2 * j + 1]), a.qk_scale2, c2);
+                        emax = fmaxf(emax, fmaxf(e0, e1));
+                        const uint32_t pk = pack_bf16x2(fast_exp2(fminf(e0, kMaxExcess)),
+                                                        fast_exp2(fminf(e1, kMaxExcess)));
+                        psum += __uint_as_float(pk << 16) + __uint_as_float(pk & 0xffff0000u);
+                        pw[j] = pk;
+                    }
+                }
+                l_sum += psum;
+                emax_all = fmaxf(emax_all, emax);
+            }
+            // P row (this thread's 32 keys = 4 16-byte chunks) into the 128B-swizzled K-major
+            // P buffer of this block: row r at (r/8)*1024 + (r%8)*128, chunk c at (c ^ r%8)*16.
+            {
+                unsigned char *prow = base + kOffP + (size_t)(i & 1) * kPBytes + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int cch = 4 * khalf + k;
+                    *reinterpret_cast<uint4 *>(prow + ((cch ^ (row & 7)) << 4)) =
+                        make_uint4(pw[4 * k], pw[4 * k + 1], pw[4 * k + 2], pw[4 * k + 3]);
+                }
+            }
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.p_full[i & 1]);
         }
-        // Epilogue: O / l -> bf16.
-        if (!failed && wait_or_fail(&sh.o_full, 0, a.status, failed)) {
+        if (__any_sync(kFull, emax_all > kMaxExcess) && lane == 0) report(a.status, DASH_ERR_RANGE_CLAMPED);
+        // Epilogue: l = sum of the two partial sums, O / l -> bf16 (each warp 64 of the dims).
+        sh.lpair[khalf][row] = l_sum;
+        const bool ok_o = wait_or_fail(&sh.o_full, 0, a.status, failed);
+        named_sync(2, kSmThreads);
+        if (ok_o) {
             tc_fence_after();
-            const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+            const float l = sh.lpair[0][row] + sh.lpair[1][row];
+            const float inv = l > 0.f ? 1.f / l : 0.f;
             __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(a.out) +
                                   (((long long)b * a.Hq + h_row) * a.T + (row_ok ? t_row : 0)) * D;
 #pragma unroll 1
-            for (int q4 = 0; q4 < 4; ++q4) {
+            for (int q2 = 0; q2 < 2; ++q2) {
+                const int q4 = 2 * khalf + q2;
                 uint32_t o[32];
                 tmem_ld32(lane_base + kColO + 32 * q4, o);
                 tmem_wait_ld();
@@ -453,7 +529,7 @@ static cudaError_t launch_tc_t(const StageArgs &a, cudaStream_t st) {
     ta.s = a;
     ta.RT = 128 / a.G;
     ta.n_tiles_bg = (a.T + ta.RT - 1) / ta.RT;
-    size_t off = (size_t)kStages * kStageBytes;
+    size_t off = kRingBytes;
     ta.off_bias = off;
     off += (size_t)2 * kBiasBatch * ta.RT * 4;
     ta.off_qbar = off;

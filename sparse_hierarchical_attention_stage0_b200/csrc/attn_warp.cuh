@@ -108,10 +108,11 @@ __device__ __forceinline__ void softmax_sub(UnitState<D> &st, float (&acc)[4][4]
     float sum_lo = 0.f, sum_hi = 0.f;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        acc[j][0] = fast_exp2(acc[j][0] - mu_lo);
-        acc[j][1] = fast_exp2(acc[j][1] - mu_lo);
-        acc[j][2] = fast_exp2(acc[j][2] - mu_hi);
-        acc[j][3] = fast_exp2(acc[j][3] - mu_hi);
+        // Weights rounded to bf16 once: the row sums add exactly what the MMA multiplies.
+        acc[j][0] = bf16_round(fast_exp2(acc[j][0] - mu_lo));
+        acc[j][1] = bf16_round(fast_exp2(acc[j][1] - mu_lo));
+        acc[j][2] = bf16_round(fast_exp2(acc[j][2] - mu_hi));
+        acc[j][3] = bf16_round(fast_exp2(acc[j][3] - mu_hi));
         sum_lo += acc[j][0] + acc[j][1];
         sum_hi += acc[j][2] + acc[j][3];
     }

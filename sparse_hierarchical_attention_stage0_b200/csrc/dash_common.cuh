@@ -133,6 +133,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
 }
+__device__ __forceinline__ float bf16_round(float x) {
+    return __bfloat162float(__float2bfloat16_rn(x));
+}
 // 2^x on the SFU (used only for attention probabilities, which are rounded to bf16).
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;
