@@ -412,7 +412,6 @@ def main():
     tau = torch.empty(B, Hkv, T, device=dev)
     mask = torch.empty(B, Hkv, T, W, dtype=torch.int64, device=dev)
     ws_s = dash.workspace(256, dev)
-    ws_a = dash.workspace(dash.attend_workspace_size(prm), dev)
     import ctypes
 
     def run_route():
@@ -429,7 +428,7 @@ def main():
         ev[1].record(stream)
         run_route()
         ev[2].record(stream)
-        dash.attend(q, k, v, summ, tau, mask, Bc, cfg.alpha, cfg.gamma, 1.0, True, ws=ws_a, out=out)
+        dash.attend(q, k, v, summ, tau, mask, Bc, cfg.alpha, cfg.gamma, 1.0, True, ws=ws_s, out=out)
         ev[3].record(stream)
         ev[3].synchronize()
         if i >= args.warmup:

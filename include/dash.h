@@ -95,11 +95,9 @@ typedef struct {
     unsigned flags;   /* DASH_FLAG_* */
 } dash_params_t;
 
-/* Bytes of device workspace dash_prefill uses for these parameters (assuming summary_k and
- * active_blocks are passed as NULL; they are then kept in the workspace), including the V^T
- * scratch that dash_attend_workspace_size describes.  dash_prefill also accepts a workspace
- * without that scratch (status, tau and the NULL-passed summaries and mask only) and then
- * runs Stage 2 on the tile kernel.  0 on bad parameters. */
+/* Bytes of device workspace dash_prefill needs for these parameters (assuming summary_k and
+ * active_blocks are passed as NULL; they are then kept in the workspace).  0 on bad
+ * parameters. */
 size_t dash_prefill_workspace_size(const dash_params_t *params);
 
 /* Whole causal prefill: Stage 0 -> Stage 1 -> Stage 2, stream-ordered, no host syncs.
@@ -114,7 +112,7 @@ size_t dash_prefill_workspace_size(const dash_params_t *params);
  *   active_blocks [B, H_kv, T, W] uint64 (out, nullable), W = ceil(C/64); bit c % 64 of word
  *            c / 64 (LSB first) is set iff chunk c is attended by row t (routed-active or
  *            the diagonal); bits above c_t are 0
- *   ws, ws_bytes: device workspace, dash_prefill_workspace_size(params) bytes for the fast path;
+ *   ws, ws_bytes: device workspace of at least dash_prefill_workspace_size(params) bytes;
  *            its first 256 bytes hold the device status word (cleared by this call)
  * Returns DASH_OK when every launch was issued. */
 dash_status_t dash_prefill(const dash_params_t *params, const void *q, const void *k,
@@ -136,13 +134,6 @@ dash_status_t dash_stage0(const dash_params_t *params, const void *k, const floa
 dash_status_t dash_route(const dash_params_t *params, const void *q, const float *summary_k,
                          float *tau, float *p, uint64_t *active_blocks, void *ws,
                          size_t ws_bytes, void *stream);
-
-/* Workspace bytes dash_attend can use with these params: 256 (the status word) plus, for
- * routed attention with head_dim 128, 16 query heads per KV head and chunk_size 64, a V^T
- * scratch of B*H_kv*128*roundup(T,8)*2 bytes (rounded up to 256) that lets the per-token
- * tensor-core kernel run.  dash_attend runs correctly with any ws_bytes >= 256; below this
- * size it takes the tile kernel instead.  Returns 0 for invalid params. */
-size_t dash_attend_workspace_size(const dash_params_t *params);
 
 /* Stage 2 alone: out [B,H_q,T,D] bf16 from q, k, v, the routing (summary_k, tau,
  * active_blocks as written by dash_stage0 / dash_route) and the flags (DASH_FLAG_DENSE and

@@ -260,7 +260,6 @@ static cudaError_t launch_attend_t(const StageArgs &a, cudaStream_t st) {
 
 cudaError_t launch_attend(const StageArgs &a, cudaStream_t st) {
     if (attend_tc_supported(a)) return launch_attend_tc(a, st);
-    if (a.vt && !a.ignore_routing && attend_tok_supported(a)) return launch_attend_tok(a, st);
     if (a.D == 128 && a.Bc == 64) return launch_attend_t<128, 64>(a, st);
     if (a.D == 128 && a.Bc == 128) return launch_attend_t<128, 128>(a, st);
     if (a.D == 64 && a.Bc == 64) return launch_attend_t<64, 64>(a, st);

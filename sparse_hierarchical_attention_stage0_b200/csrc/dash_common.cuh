@@ -231,50 +231,64 @@ __device__ __forceinline__ float pow_beta(float m, const RouteConsts &rc) {
     if (rc.kind == 2) return m;
     return powf(m, rc.beta);
 }
-__device__ __forceinline__ float pow_beta_m1(float m, const RouteConsts &rc) {
-    if (rc.kind == 1) return m;
-    if (rc.kind == 2) return 1.f;
-    return powf(m, rc.beta - 1.f);
+
+// One lane-strided pass over xs[0..n): lane l visits l, l+32, l+64, l+96, l+128, ..., with
+// four independent accumulators (one per offset mod 128, for instruction-level parallelism)
+// combined as (a0 + a1) + (a2 + a3): a fixed summation order.
+template <typename Term>
+__device__ __forceinline__ float lane_pass(const float *xs, int n, int lane, Term term) {
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    int c = lane;
+    for (; c + 96 < n; c += 128) {
+        a0 += term(xs[c]);
+        a1 += term(xs[c + 32]);
+        a2 += term(xs[c + 64]);
+        a3 += term(xs[c + 96]);
+    }
+    if (c < n) a0 += term(xs[c]);
+    if (c + 32 < n) a1 += term(xs[c + 32]);
+    if (c + 64 < n) a2 += term(xs[c + 64]);
+    return (a0 + a1) + (a2 + a3);
 }
 
 // Entmax threshold of one row held in (shared) memory xs[0..n), n >= 1, all 32 lanes of
-// the warp calling.  For alpha = 1 returns the log-sum-exp of the scores.  Otherwise x are
+// the warp calling, specialised on the kind of alpha (0 softmax, 1 alpha = 1.5, 2 alpha = 2,
+// 3 any other alpha).  For alpha = 1 returns the log-sum-exp of the scores.  Otherwise x are
 // the scaled scores (alpha-1) s and the return value is tau with
 // sum_c [x_c - tau]_+^beta = 1.  For beta >= 1 (alpha <= 2) Newton's method from
 // tau0 = max x - 1 increases monotonically to the root (f is convex and decreasing); the
 // support it settles on is then fed to the exact closed form for alpha = 1.5 and 2.  For
-// alpha > 2, bisection on [max - 1, max - n^(1-alpha)].  The lane-strided sums and butterfly
-// reductions fix the summation order, so every caller gets the same bits.
-static __device__ __noinline__ float warp_entmax_tau(const float *xs, int n, const RouteConsts &rc,
-                                              uint32_t *status) {
+// alpha > 2, bisection on [max - 1, max - n^(1-alpha)].  The fixed lane-strided sums and
+// butterfly reductions give every caller the same bits.
+template <int KIND>
+static __device__ __noinline__ float entmax_tau_k(const float *xs, int n, const RouteConsts rc,
+                                                  uint32_t *status) {
     const int lane = threadIdx.x & 31;
     float mx = -INFINITY;
     for (int c = lane; c < n; c += 32) mx = fmaxf(mx, xs[c]);
     mx = warp_max(mx);
-    if (rc.kind == 0) {
-        float s = 0.f;
-        for (int c = lane; c < n; c += 32) s += expf(xs[c] - mx);
-        s = warp_sum(s);
+    if (KIND == 0) {
+        const float s = warp_sum(lane_pass(xs, n, lane, [mx](float x) { return expf(x - mx); }));
         return mx + logf(s);
     }
+    const float beta = rc.beta;
     float tau;
-    if (rc.beta >= 1.f) {
+    if (KIND != 3 || beta >= 1.f) {
         tau = mx - 1.f;
         int it = 0;
         for (; it < kNewtonCap; ++it) {
-            float f = 0.f, df = 0.f;
-            for (int c = lane; c < n; c += 32) {
-                float m = xs[c] - tau;
-                if (m > 0.f) {
-                    f += pow_beta(m, rc);
-                    df += pow_beta_m1(m, rc);
-                }
-            }
-            f = warp_sum(f);
-            df = warp_sum(df);
-            float step = (f - 1.f) / (rc.beta * df);
+            const float t = tau;
+            const float f = warp_sum(lane_pass(xs, n, lane, [t, beta](float x) {
+                const float m = x - t;
+                return m > 0.f ? (KIND == 1 ? m * m : KIND == 2 ? m : powf(m, beta)) : 0.f;
+            }));
+            const float df = warp_sum(lane_pass(xs, n, lane, [t, beta](float x) {
+                const float m = x - t;
+                return m > 0.f ? (KIND == 1 ? m : KIND == 2 ? 1.f : powf(m, beta - 1.f)) : 0.f;
+            }));
+            const float step = (f - 1.f) / (beta * df);
             if (!(step > 0.f)) break;                 // at (or rounded past) the root
-            float nt = tau + step;
+            const float nt = tau + step;
             if (nt == tau) break;
             tau = nt;
             if (step <= 1e-7f * fmaxf(1.f, fabsf(tau))) break;
@@ -283,34 +297,31 @@ static __device__ __noinline__ float warp_entmax_tau(const float *xs, int n, con
     } else {
         float lo = mx - 1.f, hi = mx - powf((float)n, 1.f - rc.alpha);
         for (int it = 0; it < 40; ++it) {
-            float mid = 0.5f * (lo + hi), f = 0.f;
-            for (int c = lane; c < n; c += 32) {
-                float m = xs[c] - mid;
-                if (m > 0.f) f += pow_beta(m, rc);
-            }
-            f = warp_sum(f);
+            const float mid = 0.5f * (lo + hi);
+            const float f = warp_sum(lane_pass(xs, n, lane, [mid, beta](float x) {
+                const float m = x - mid;
+                return m > 0.f ? powf(m, beta) : 0.f;
+            }));
             if (f >= 1.f) lo = mid; else hi = mid;
         }
         tau = 0.5f * (lo + hi);
     }
-    if (rc.kind == 1 || rc.kind == 2) {
+    if (KIND == 1 || KIND == 2) {
         // Exact closed form on the support {x > tau}; repeat while the support moves.
         for (int rep = 0; rep < 4; ++rep) {
-            float sx = 0.f;
-            int k = 0;
-            for (int c = lane; c < n; c += 32)
-                if (xs[c] > tau) { sx += xs[c]; ++k; }
-            sx = warp_sum(sx);
-            k = warp_sum_i(k);
+            const float t = tau;
+            const float sx = warp_sum(lane_pass(xs, n, lane, [t](float x) { return x > t ? x : 0.f; }));
+            const int k = (int)warp_sum(lane_pass(xs, n, lane, [t](float x) { return x > t ? 1.f : 0.f; }));
             if (k == 0) break;
             float nt;
-            if (rc.kind == 2) {
+            if (KIND == 2) {
                 nt = (sx - 1.f) / (float)k;
             } else {
-                float mean = sx / (float)k, m2 = 0.f;
-                for (int c = lane; c < n; c += 32)
-                    if (xs[c] > tau) { float d = xs[c] - mean; m2 = fmaf(d, d, m2); }
-                m2 = warp_sum(m2);
+                const float mean = sx / (float)k;
+                const float m2 = warp_sum(lane_pass(xs, n, lane, [t, mean](float x) {
+                    const float d = x - mean;
+                    return x > t ? d * d : 0.f;
+                }));
                 nt = mean - sqrtf(fmaxf(1.f - m2, 0.f) / (float)k);
             }
             // Same support under the new threshold?  Then it is the fixed point.
@@ -322,6 +333,16 @@ static __device__ __noinline__ float warp_entmax_tau(const float *xs, int n, con
         }
     }
     return tau;
+}
+
+__device__ __forceinline__ float warp_entmax_tau(const float *xs, int n, const RouteConsts &rc,
+                                                 uint32_t *status) {
+    switch (rc.kind) {
+        case 0: return entmax_tau_k<0>(xs, n, rc, status);
+        case 1: return entmax_tau_k<1>(xs, n, rc, status);
+        case 2: return entmax_tau_k<2>(xs, n, rc, status);
+        default: return entmax_tau_k<3>(xs, n, rc, status);
+    }
 }
 
 }  // namespace dash

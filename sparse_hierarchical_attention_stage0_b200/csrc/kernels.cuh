@@ -19,7 +19,6 @@ struct StageArgs {
     float *p;                 // [B,Hkv,T,C] or null
     uint64_t *mask;           // [B,Hkv,T,W]
     void *out;                // [B,Hq,T,D]
-    void *vt;                 // [B,Hkv,D,T8] V^T scratch for the per-token kernel, or null
     int B, Hq, Hkv, T, D, Bc, G, C, Cf, W;
     RouteConsts rc;
     float qk_scale2;          // log2(e) / sqrt(D)
@@ -47,10 +46,6 @@ int route_rows_per_cta(int C, int D);   // 0 if C is too large for the routing k
 cudaError_t launch_attend(const StageArgs &a, cudaStream_t st);
 bool attend_tc_supported(const StageArgs &a);
 cudaError_t launch_attend_tc(const StageArgs &a, cudaStream_t st);
-bool attend_tok_supported(const StageArgs &a);
-size_t attend_tok_vt_bytes(int B, int Hkv, int T, int D);
-cudaError_t launch_attend_tok(const StageArgs &a, cudaStream_t st);
-cudaError_t launch_vtranspose(const void *v, void *vt, int BHkv, int T, int D, cudaStream_t st);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
 int decode_supported(int G, int Ccap, int D);
 

@@ -64,18 +64,27 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(StageArgs a) {
     const float scale = a.rc.kind == 0 ? a.rc.sscale : a.rc.xscale;
     const float *sumg = a.summary + (long long)bg * a.Cf * D;
     const int kslice = lane & 3, cc = lane >> 2;
-    for (int cbase = warp * 8; cbase < n; cbase += (kRouteThreads / 32) * 8) {
+    constexpr int kStep = (kRouteThreads / 32) * 8;       // chunks per CTA-wide step
+    // The summary slices of the next step are loaded while the current step computes, so
+    // the L2 latency of the loads overlaps the FMAs.
+    auto load_slice = [&](int cbase, float4 (&sv)[D / 16]) {
+        const float4 *s4 = reinterpret_cast<const float4 *>(sumg + (long long)min(cbase + cc, n - 1) * D);
+#pragma unroll
+        for (int i = 0; i < D / 16; ++i) sv[i] = __ldg(s4 + 4 * i + kslice);
+    };
+    float4 cur[D / 16], nxt[D / 16];
+    int cbase = warp * 8;
+    if (cbase < n) load_slice(cbase, cur);
+    for (; cbase < n; cbase += kStep) {
         const int c = cbase + cc;
-        const float4 *s4 = reinterpret_cast<const float4 *>(sumg + (long long)min(c, n - 1) * D);
+        const bool more = cbase + kStep < n;
+        if (more) load_slice(cbase + kStep, nxt);
         float acc[RT];
 #pragma unroll
         for (int r = 0; r < RT; ++r) acc[r] = 0.f;
-        float4 sv4[D / 16];                       // all loads of the slice in flight at once
-#pragma unroll
-        for (int i = 0; i < D / 16; ++i) sv4[i] = __ldg(s4 + 4 * i + kslice);
 #pragma unroll
         for (int i = 0; i < D / 16; ++i) {
-            const float4 sv = sv4[i];
+            const float4 sv = cur[i];
 #pragma unroll
             for (int r = 0; r < RT; ++r) {
                 const float4 qq = reinterpret_cast<const float4 *>(qbar + r * D)[4 * i + kslice];
@@ -95,6 +104,10 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(StageArgs a) {
         if (kslice == 0 && c < n) {
 #pragma unroll
             for (int r = 0; r < RT; ++r) xs[r * xstride + c] = __fmul_rn(acc[r], scale);
+        }
+        if (more) {
+#pragma unroll
+            for (int i = 0; i < D / 16; ++i) cur[i] = nxt[i];
         }
     }
     __syncthreads();
