@@ -63,10 +63,11 @@ typedef enum {
     DASH_ERR_WORKSPACE_TOO_SMALL = 3,
     DASH_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed */
     DASH_ERR_DEVICE_TIMEOUT = 5,     /* a device wait or iteration cap ran out */
-    DASH_ERR_RANGE_CLAMPED = 6       /* a logit exceeded its row's reference (the maximum
-                                        over the first 64 keys of the diagonal chunk) by more
-                                        than 100 in log2 units; its probability was clamped,
-                                        the output of that row is not exact */
+    DASH_ERR_RANGE_CLAMPED = 6       /* a logit lay so far above its row's softmax reference
+                                        (the maximum over the row's visible keys of the
+                                        diagonal chunk) that the row's probabilities were
+                                        clamped or their sum overflowed fp32; the output of
+                                        that row is not exact */
 } dash_status_t;
 
 enum {
@@ -95,8 +96,11 @@ typedef struct {
     unsigned flags;   /* DASH_FLAG_* */
 } dash_params_t;
 
-/* Bytes of device workspace dash_prefill needs for these parameters (assuming summary_k and
- * active_blocks are passed as NULL; they are then kept in the workspace).  0 on bad
+/* Bytes of device workspace dash_prefill uses for these parameters (assuming summary_k and
+ * active_blocks are passed as NULL; they are then kept in the workspace), including the V^T
+ * scratch that dash_attend_workspace_size describes.  dash_prefill also accepts a workspace
+ * without that scratch (status, tau and the NULL-passed summaries and mask only); Stage 2
+ * then runs on the 64-key-block tensor-core kernel, about 10% slower.  0 on bad
  * parameters. */
 size_t dash_prefill_workspace_size(const dash_params_t *params);
 
@@ -112,7 +116,7 @@ size_t dash_prefill_workspace_size(const dash_params_t *params);
  *   active_blocks [B, H_kv, T, W] uint64 (out, nullable), W = ceil(C/64); bit c % 64 of word
  *            c / 64 (LSB first) is set iff chunk c is attended by row t (routed-active or
  *            the diagonal); bits above c_t are 0
- *   ws, ws_bytes: device workspace of at least dash_prefill_workspace_size(params) bytes;
+ *   ws, ws_bytes: device workspace, dash_prefill_workspace_size(params) bytes for the fast path;
  *            its first 256 bytes hold the device status word (cleared by this call)
  * Returns DASH_OK when every launch was issued. */
 dash_status_t dash_prefill(const dash_params_t *params, const void *q, const void *k,
@@ -134,6 +138,13 @@ dash_status_t dash_stage0(const dash_params_t *params, const void *k, const floa
 dash_status_t dash_route(const dash_params_t *params, const void *q, const float *summary_k,
                          float *tau, float *p, uint64_t *active_blocks, void *ws,
                          size_t ws_bytes, void *stream);
+
+/* Workspace bytes dash_attend uses with these params: 256 (the status word) plus, when the
+ * 128-key-block tensor-core kernel applies (head_dim 128, 8 <= G <= 128 query heads per KV
+ * head with 128 % G == 0, chunk_size 64 or 128), a V^T copy of v, B*H_kv*128*roundup(T,8)*2
+ * bytes rounded up to 256, written by the call.  dash_attend runs correctly with any
+ * ws_bytes >= 256; below this size it takes the 64-key-block kernel.  0 on bad params. */
+size_t dash_attend_workspace_size(const dash_params_t *params);
 
 /* Stage 2 alone: out [B,H_q,T,D] bf16 from q, k, v, the routing (summary_k, tau,
  * active_blocks as written by dash_stage0 / dash_route) and the flags (DASH_FLAG_DENSE and

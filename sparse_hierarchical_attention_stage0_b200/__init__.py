@@ -38,7 +38,7 @@ FLAG_ESTIMATE_DIAGONAL = 4
 
 # Every symbol include/dash.h declares.
 EXPORTS = ("dash_prefill_workspace_size", "dash_prefill", "dash_stage0", "dash_route",
-           "dash_attend", "dash_update_chunk_cache", "dash_decode_workspace_size",
+           "dash_attend_workspace_size", "dash_attend", "dash_update_chunk_cache", "dash_decode_workspace_size",
            "dash_decode", "dash_read_device_status", "dash_status_string")
 
 
@@ -56,6 +56,8 @@ _P = ctypes.POINTER(Params)
 _sz = ctypes.c_size_t
 lib.dash_prefill_workspace_size.argtypes = [_P]
 lib.dash_prefill_workspace_size.restype = _sz
+lib.dash_attend_workspace_size.argtypes = [_P]
+lib.dash_attend_workspace_size.restype = _sz
 lib.dash_decode_workspace_size.argtypes = [_P]
 lib.dash_decode_workspace_size.restype = _sz
 lib.dash_prefill.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
@@ -111,6 +113,10 @@ def _need(t, dtype, shape, name):
 
 def prefill_workspace_size(params: Params) -> int:
     return int(lib.dash_prefill_workspace_size(ctypes.byref(params)))
+
+
+def attend_workspace_size(params: Params) -> int:
+    return int(lib.dash_attend_workspace_size(ctypes.byref(params)))
 
 
 def decode_workspace_size(params: Params) -> int:
@@ -199,7 +205,7 @@ def attend(q, k, v, summary, tau, active_blocks, chunk_size=64, alpha=1.5, gamma
     if out is None:
         out = torch.empty_like(q)
     if ws is None:
-        ws = workspace(256, q.device)
+        ws = workspace(lib.dash_attend_workspace_size(ctypes.byref(prm)), q.device)
     _check(lib.dash_attend(ctypes.byref(prm), _ptr(q), _ptr(k), _ptr(v), _ptr(summary),
                            _ptr(tau), _ptr(active_blocks), _ptr(out), _ptr(ws), ws.numel(),
                            _stream(q.device)), "dash_attend")

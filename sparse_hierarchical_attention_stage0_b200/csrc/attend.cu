@@ -259,6 +259,7 @@ static cudaError_t launch_attend_t(const StageArgs &a, cudaStream_t st) {
 }
 
 cudaError_t launch_attend(const StageArgs &a, cudaStream_t st) {
+    if (a.vt && attend_fa_supported(a)) return launch_attend_fa(a, st);
     if (attend_tc_supported(a)) return launch_attend_tc(a, st);
     if (a.D == 128 && a.Bc == 64) return launch_attend_t<128, 64>(a, st);
     if (a.D == 128 && a.Bc == 128) return launch_attend_t<128, 128>(a, st);

@@ -1,0 +1,621 @@
+// attend_fa.cu -- Stage 2 on the 5th-generation tensor cores with 128-key blocks, D = 128.
+//
+// gist.science "DashAttention: Differentiable and Adaptive Sparse Hierarchical Attention",
+// Technische Zusammenfassung, "Stufe 2: Prior-induzierte spaerliche Softmax": a
+// FlashAttention-style kernel iterates the active chunks given by the bit-packed mask and
+// adds the routing bias (log of the prior) to the logits before the softmax; chunks with
+// zero probability are masked; the diagonal chunk keeps its own branch.
+//
+// One CTA per SM, one tile of 128 query rows of one (b, g): 128/G consecutive tokens x G
+// heads (G >= 8), which share one diagonal chunk.  The tile walks the union of its tokens'
+// active chunks (the OR of their mask words, which carry each token's diagonal bit): the
+// diagonal chunk first, then the others in ascending order, two 64-key chunks (or one
+// 128-key chunk) per 128-key block.  A row whose token did not route to a chunk gets bias
+// -inf there; keys above the row's position are masked.  Per block j:
+//   S_j[128 x 128] = Q K^T     tcgen05.mma, A = Q (TMEM), B = K (smem, TMA), N = 128
+//   softmax        four threads per row (16 warps, 32 keys each), fp32; each thread writes
+//                  its bf16 P over its own S columns
+//   O[128 x 128]  += P V       tcgen05.mma, A = P (TMEM), B = V^T (smem, TMA; K-major: keys
+//                              contiguous per head dim), K = 128 keys
+// S is double-buffered, so Q K^T of block j+1 runs while the softmax works on block j; the
+// Q K^T and P V instructions come from two issuer warps.  Measured on B200: an N = 128
+// tcgen05.mma with a K-major B and a precomputed descriptor issues in ~66 cycles (its tensor
+// time), with an MN-major B (V as stored) in ~108, hence V^T (one transpose pass per call,
+// vtranspose.cu) and descriptors built once per ring stage.
+// Softmax reference: the first block holds the diagonal chunk, whose causally visible keys
+// (at least one per row) give each row its exact maximum m; every probability is 2^(s - m)
+// against that fixed reference, so O is never rescaled.  A logit so far above the reference
+// that the row's fp32 sum overflows (beyond about 2^110 with 2^17 keys) leaves a non-finite
+// row sum; such rows are reported as DASH_ERR_RANGE_CLAMPED.  Row sums add the bf16 weights
+// the MMA multiplies.  Off the diagonal the exponent arguments and the sums run on packed
+// fp32 pairs (fma.rn.f32x2, add.rn.f32x2): about 3.5 instructions per score.
+// Warp roles: 0 TMA producer (K and V^T rings, 3 stages each, 128B-swizzled), 1 Q K^T issuer
+// and TMEM owner, 2 routing-bias producer (recomputes qbar.summary with Stage 1's exact
+// arithmetic, 32 chunks per batch, double-buffered), 3 P V issuer, 4-19 softmax + epilogue.
+// TMEM: Q 64 columns | S0 128 | S1 128 | O 128.  Every wait is bounded; on timeout the CTA
+// records DASH_ERR_DEVICE_TIMEOUT and drains.
+#include "kernels.cuh"
+#include "tc_common.cuh"
+
+namespace dash {
+using namespace tcx;
+namespace {
+
+constexpr int kSmWarps = 16;
+constexpr int kSmThreads = kSmWarps * 32;
+constexpr int kFaThreads = 4 * 32 + kSmThreads;
+constexpr int kStages = 3;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColQ = 0, kColS = 64, kColO = 320;     // S buffer b at kColS + 128 b
+constexpr int kBiasBatch = 32;
+constexpr int kWarpTma = 0, kWarpQk = 1, kWarpBias = 2, kWarpPv = 3, kWarpSm0 = 4;
+constexpr uint32_t kBlkBytes = 32768;      // K: 2 d-panels x [128 keys][128 B]; V^T: 2 key-halves x [128 d][128 B]
+constexpr uint32_t kOffV = kStages * kBlkBytes, kRingBytes = 2 * kStages * kBlkBytes;
+
+struct FaShared {
+    uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
+    uint64_t s_full[2], p_full[2], pv_done[2];  // per S buffer: never more than one phase ahead
+    uint64_t o_full, qk_done;
+    float mpart[4][128];                   // partial row maxima of the first block
+    float lpart[4][128];                   // partial row sums
+    uint32_t tmem_base;
+    int n_chunks;
+    int failed;
+};
+
+// Packed fp32 pairs (sm_100): {lo, hi} in one 64-bit register.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+}  // namespace
+
+struct FaArgs {
+    StageArgs s;
+    int RT;              // tokens per tile (128 / G)
+    int n_tiles_bg;      // token tiles per (b, g)
+    size_t off_bias, off_qbar, off_list;  // dynamic smem offsets (bytes, from the aligned base)
+};
+
+template <int BC>
+__global__ void __launch_bounds__(kFaThreads, 1)
+k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmVt,
+            const FaArgs ta) {
+    extern __shared__ unsigned char smem_dyn[];
+    __shared__ FaShared sh;
+    const StageArgs &a = ta.s;
+    constexpr int D = 128;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    unsigned char *base = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~(uintptr_t)1023);
+    float *bias_s = reinterpret_cast<float *>(base + ta.off_bias);      // [2][kBiasBatch][RT]
+    float *qbar = reinterpret_cast<float *>(base + ta.off_qbar);        // [RT][D]
+    int16_t *list = reinterpret_cast<int16_t *>(base + ta.off_list);    // [C]
+
+    const int RT = ta.RT, G = a.G;
+    const int BHkv = a.B * a.Hkv;
+    const int tile_rev = blockIdx.x / BHkv, bgi = blockIdx.x % BHkv;
+    const int tt = ta.n_tiles_bg - 1 - tile_rev;                        // longest tiles first
+    const int b = bgi / a.Hkv, g = bgi % a.Hkv;
+    const long long bg = bgi;
+    const int t0 = tt * RT;
+    const int t_last = min(t0 + RT, a.T) - 1;
+    const int ct_max = t_last / BC;                                     // the tile's diagonal chunk
+
+    // ---------------------------------------------------------------- setup
+    if (warp == kWarpQk) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&sh.tmem_base)),
+                     "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sh.k_full[s], 1);
+            mbar_init(&sh.k_empty[s], 1);
+            mbar_init(&sh.v_full[s], 1);
+            mbar_init(&sh.v_empty[s], 1);
+        }
+        for (int bb = 0; bb < 2; ++bb) {
+            mbar_init(&sh.s_full[bb], 1);
+            mbar_init(&sh.p_full[bb], kSmWarps);
+            mbar_init(&sh.pv_done[bb], 1);
+        }
+        mbar_init(&sh.o_full, 1);
+        mbar_init(&sh.qk_done, 1);
+        sh.failed = 0;
+        fence_mbar_init();
+    }
+    if (warp == kWarpBias) {
+        // Union of the tile's tokens' mask words (each carries its token's diagonal bit).
+        const int W = a.W, wlim = ct_max / 64;
+        int pos = 0;
+        for (int w0 = 0; w0 <= wlim; w0 += 32) {
+            const int w = w0 + lane;
+            uint64_t word = 0;
+            if (w <= wlim) {
+                if (a.ignore_routing) {
+                    word = ~0ull;
+                } else {
+                    for (int u = 0; u < RT; ++u) {
+                        const int t = t0 + u;
+                        if (t < a.T) word |= a.mask[(bg * a.T + t) * W + w];
+                    }
+                }
+                const int lim = ct_max + 1 - 64 * w;          // bits [0, lim) can be attended
+                if (lim < 64) word &= (1ull << lim) - 1ull;
+            }
+            const int cnt = __popcll(word);
+            int incl = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(kFull, incl, o);
+                if (lane >= o) incl += v;
+            }
+            int p = pos + incl - cnt;
+            while (word) {
+                const int bit = __ffsll((long long)word) - 1;
+                word &= word - 1ull;
+                list[p++] = (int16_t)(w * 64 + bit);
+            }
+            pos += __shfl_sync(kFull, incl, 31);
+        }
+        if (lane == 0) sh.n_chunks = pos;
+        // Group-mean queries of the tile's tokens (Stage 1's exact arithmetic).
+        if (!a.ignore_routing) {
+            const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(a.q);
+            for (int idx = lane; idx < RT * (D / 8); idx += 32) {
+                const int u = idx / (D / 8), d8 = (idx % (D / 8)) * 8, t = t0 + u;
+                float m[8];
+                if (t < a.T) {
+                    group_mean8(q + (((long long)b * a.Hq + g * G) * a.T + t) * D + d8,
+                                (long long)a.T * D, G, m);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) m[e] = 0.f;
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) qbar[u * D + d8 + e] = m[e];
+            }
+        }
+    }
+    // Softmax warps: quadrant sp (TMEM lanes 32 sp ..), key quarter kq of every block.
+    const int sp = warp & 3;
+    const int kq = (warp - kWarpSm0) >> 2;
+    const int row = 32 * sp + lane;
+    const int u_row = row / G;
+    const int t_row = t0 + u_row;
+    const int h_row = g * G + row % G;
+    const bool row_ok = t_row < a.T;
+    __syncthreads();
+    const uint32_t tb = sh.tmem_base;
+    if (warp >= kWarpSm0) {
+        // Q row -> TMEM columns [0, 64): this warp's quarter of the dims (32 dims, 16 columns).
+        const __nv_bfloat16 *qr = reinterpret_cast<const __nv_bfloat16 *>(a.q) +
+                                  (((long long)b * a.Hq + h_row) * a.T + (row_ok ? t_row : 0)) * D +
+                                  32 * kq;
+        uint32_t r[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint4 v = row_ok ? *reinterpret_cast<const uint4 *>(qr + 8 * j) : make_uint4(0, 0, 0, 0);
+            r[4 * j] = v.x;
+            r[4 * j + 1] = v.y;
+            r[4 * j + 2] = v.z;
+            r[4 * j + 3] = v.w;
+        }
+        tmem_st16(tb + ((uint32_t)(32 * sp) << 16) + kColQ + 16 * kq, r);
+        tmem_wait_st();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const int n_chunks = sh.n_chunks;
+    const int n_blocks = BC == 64 ? (n_chunks + 1) / 2 : n_chunks;
+    bool failed = false;
+    // Walk order: the diagonal chunk (the largest, last entry of the ascending list) first.
+    auto chunk_at = [&](int e) -> int { return (int)list[e == 0 ? n_chunks - 1 : e - 1]; };
+    // List entry of half h (keys 64h .. 64h+63) of block j; -1 if that half is empty.
+    auto entry_of = [&](int j, int h) -> int {
+        if (BC == 64) return 2 * j + h < n_chunks ? 2 * j + h : -1;
+        return j;
+    };
+    auto key0_of = [&](int j, int h) -> int {
+        return BC == 64 ? chunk_at(2 * j + h) * 64 : chunk_at(j) * 128 + 64 * h;
+    };
+
+    if (warp == kWarpTma) {
+        // ------------------------------------------------------------ TMA producer
+        // K runs one block ahead of V^T (Q K^T needs it first).  K: a block's two 64-key
+        // halves land at rows 0-63 and 64-127 of each 16 KB d-panel.  V^T: key-half h is one
+        // [128 d][64 keys] box at 16 KB * h.  An empty second half is not loaded (its MMAs are
+        // not issued either).
+        int k_issued = 0, v_issued = 0;
+        auto issue = [&](bool is_v, int j) -> bool {
+            const int s = j % kStages;
+            const uint32_t ph = (uint32_t)(j / kStages) & 1u;
+            uint64_t *empty = is_v ? &sh.v_empty[s] : &sh.k_empty[s];
+            uint64_t *full = is_v ? &sh.v_full[s] : &sh.k_full[s];
+            if (!wait_or_fail(empty, ph ^ 1u, a.status, failed)) return false;
+            if (lane == 0) {
+                unsigned char *st = base + (is_v ? kOffV : 0u) + (size_t)s * kBlkBytes;
+                const int nh = entry_of(j, 1) >= 0 ? 2 : 1;
+                mbar_arrive_expect_tx(full, 16384u * nh);
+                for (int h = 0; h < nh; ++h) {
+                    const int key0 = key0_of(j, h);
+                    if (is_v) {
+                        tma_load_3d(st + 16384 * h, &tmVt, key0, 0, (int)bg, full);
+                    } else {
+                        tma_load_3d(st + 8192 * h, &tmK, 0, key0, (int)bg, full);
+                        tma_load_3d(st + 16384 + 8192 * h, &tmK, 64, key0, (int)bg, full);
+                    }
+                }
+            }
+            __syncwarp();
+            if (is_v) v_issued = j + 1; else k_issued = j + 1;
+            return true;
+        };
+        if (n_blocks > 0) issue(false, 0);
+        for (int j = 0; j < n_blocks && !failed; ++j) {
+            if (j + 1 < n_blocks && !issue(false, j + 1)) break;
+            if (!issue(true, j)) break;
+        }
+        if (failed) {
+            // Bounded wait for the copies still in flight (the last ones per ring).
+            for (int i = max(0, k_issued - kStages); i < k_issued; ++i)
+                mbar_wait_bounded(&sh.k_full[i % kStages], (uint32_t)(i / kStages) & 1u);
+            for (int i = max(0, v_issued - kStages); i < v_issued; ++i)
+                mbar_wait_bounded(&sh.v_full[i % kStages], (uint32_t)(i / kStages) & 1u);
+            __syncwarp();
+        }
+    } else if (warp == kWarpQk) {
+        // ------------------------------------------------------------ Q K^T issuer
+        // S buffer j & 1 is free once P V of block j-2 (which read P from it) has completed.
+        constexpr uint32_t id_qk128 = idesc_bf16(128, 128, 0);
+        constexpr uint32_t id_qk64 = idesc_bf16(128, 64, 0);
+        uint64_t kdesc[kStages];
+#pragma unroll
+        for (int s = 0; s < kStages; ++s) kdesc[s] = smem_desc_sw128(smem_u32(base + (size_t)s * kBlkBytes), 16, 1024);
+        for (int j = 0; j < n_blocks; ++j) {
+            const int s = j % kStages, sb = j & 1;
+            if (!wait_or_fail(&sh.k_full[s], (uint32_t)(j / kStages) & 1u, a.status, failed)) break;
+            if (j >= 2 && !wait_or_fail(&sh.pv_done[sb], (uint32_t)((j - 2) >> 1) & 1u, a.status, failed)) break;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t id = entry_of(j, 1) >= 0 ? id_qk128 : id_qk64;
+                uint64_t bd0 = 0;
+#pragma unroll
+                for (int q = 0; q < kStages; ++q) bd0 = q == s ? kdesc[q] : bd0;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    // descriptor start address advances in 16-byte units: d-panel kk/4, 32 B per 16 dims
+                    const uint64_t bd = bd0 + (uint64_t)(((kk / 4) * 16384 + (kk % 4) * 32) >> 4);
+                    mma_ts(tb + kColS + 128u * sb, tb + kColQ + 8u * kk, bd, id, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(&sh.s_full[sb]);
+                mma_commit(&sh.k_empty[s]);
+            }
+            __syncwarp();
+        }
+        if (lane == 0) mma_commit(&sh.qk_done);       // tracks every MMA issued above
+        __syncwarp();
+    } else if (warp == kWarpPv) {
+        // ------------------------------------------------------------ P V issuer
+        // P of keys 32q .. 32q+31 sits in the first 16 columns of S quarter q; B = V^T, K-major.
+        constexpr uint32_t id_pv = idesc_bf16(128, D, 0);
+        uint64_t vdesc[kStages];
+#pragma unroll
+        for (int s = 0; s < kStages; ++s) vdesc[s] = smem_desc_sw128(smem_u32(base + kOffV + (size_t)s * kBlkBytes), 16, 1024);
+        for (int j = 0; j < n_blocks; ++j) {
+            const int s = j % kStages, sb = j & 1;
+            if (!wait_or_fail(&sh.v_full[s], (uint32_t)(j / kStages) & 1u, a.status, failed)) break;
+            if (!wait_or_fail(&sh.p_full[sb], (uint32_t)(j >> 1) & 1u, a.status, failed)) break;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t pb = tb + kColS + 128u * sb;
+                const bool full_blk = entry_of(j, 1) >= 0;
+                uint64_t bd0 = 0;
+#pragma unroll
+                for (int q = 0; q < kStages; ++q) bd0 = q == s ? vdesc[q] : bd0;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    if (kk >= 4 && !full_blk) break;
+                    // key-half kk/4 of V^T at 16 KB, 32 B per 16 keys
+                    const uint64_t bd = bd0 + (uint64_t)(((kk / 4) * 16384 + (kk % 4) * 32) >> 4);
+                    mma_ts(tb + kColO, pb + 32u * (kk / 2) + 8u * (kk % 2), bd, id_pv,
+                           (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(&sh.pv_done[sb]);
+                mma_commit(&sh.v_empty[s]);
+            }
+            __syncwarp();
+        }
+        if (lane == 0) mma_commit(&sh.o_full);        // tracks every MMA issued above
+        __syncwarp();
+    } else if (warp == kWarpBias) {
+        // ------------------------------------------------------------ routing biases
+        const int n_batches = (n_chunks + kBiasBatch - 1) / kBiasBatch;
+        for (int bt = 0; bt < n_batches; ++bt) {
+            float *buf = bias_s + (bt & 1) * kBiasBatch * RT;
+            for (int e = lane; e < kBiasBatch * RT; e += 32) {
+                const int k = e / RT, u = e % RT, ci = bt * kBiasBatch + k;
+                float v = 0.f;
+                if (ci < n_chunks && !a.ignore_routing) {
+                    const int c = chunk_at(ci), t = t0 + u;
+                    const int ctu = t / BC;
+                    if (t >= a.T || c > ctu) {
+                        v = -INFINITY;
+                    } else if (c < ctu) {
+                        const long long rowi = bg * a.T + t;
+                        const bool act = (a.mask[rowi * a.W + (c >> 6)] >> (c & 63)) & 1ull;
+                        if (!act) {
+                            v = -INFINITY;
+                        } else {
+                            const float dot = route_dot<D>(qbar + u * D, a.summary + (bg * a.Cf + c) * D);
+                            const float tau = a.tau[rowi];
+                            if (a.rc.kind == 0) {
+                                v = a.rc.sigma2 * (__fmul_rn(dot, a.rc.sscale) - tau);
+                            } else {
+                                const float m = __fsub_rn(__fmul_rn(dot, a.rc.xscale), tau);
+                                v = a.rc.bscale2 * log2f(fmaxf(m, 1e-37f));
+                            }
+                        }
+                    }
+                }
+                buf[e] = v;
+            }
+            __syncwarp();
+            named_sync(1, 32 + kSmThreads);
+        }
+    } else if (warp >= kWarpSm0) {
+        // ------------------------------------------------------------ softmax
+        // Four threads per row: warp (sp, kq) owns keys 32 kq .. 32 kq + 31 of every block for
+        // the rows of TMEM quadrant sp.  Every named barrier is passed by all softmax warps,
+        // failure or not.
+        const uint32_t lane_base = tb + ((uint32_t)(32 * sp) << 16);
+        const int half = kq >> 1;
+        float m_ref = 0.f, l_sum = 0.f;
+        const uint64_t scale2 = f2_pack(a.qk_scale2, a.qk_scale2);
+        for (int j = 0; j < n_blocks; ++j) {
+            const int sb = j & 1;
+            const int e0 = BC == 64 ? 2 * j : j;              // first list entry of the block
+            if (e0 % kBiasBatch == 0) named_sync(1, 32 + kSmThreads);
+            const bool ok = wait_or_fail(&sh.s_full[sb], (uint32_t)(j >> 1) & 1u, a.status, failed);
+            if (ok) tc_fence_after();
+            const int e = entry_of(j, half);
+            int key0 = 0;
+            float bias2 = -INFINITY;
+            bool diag = false;
+            if (e >= 0 && row_ok) {
+                const int c = chunk_at(e);
+                key0 = key0_of(j, half) + 32 * (kq & 1);
+                if (c == ct_max) {
+                    bias2 = 0.f;
+                    diag = true;
+                } else {
+                    bias2 = a.ignore_routing ? 0.f
+                                             : bias_s[((e / kBiasBatch) & 1) * kBiasBatch * RT +
+                                                      (e % kBiasBatch) * RT + u_row];
+                }
+            }
+            const bool dead = __all_sync(kFull, bias2 == -INFINITY);
+            uint32_t sv[32];
+            if (ok && (j == 0 || !dead)) {
+                tmem_ld32(lane_base + kColS + 128u * sb + 32u * kq, sv);
+                tmem_wait_ld();
+            }
+            if (j == 0) {
+                // Exact row maximum over the diagonal chunk's causally visible keys (the first
+                // block holds them), shared by the row's four threads: the fixed reference.
+                float mx = -INFINITY;
+                if (ok && diag) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (key0 + i <= t_row) mx = fmaxf(mx, __uint_as_float(sv[i]) * a.qk_scale2);
+                }
+                sh.mpart[kq][row] = mx;
+                named_sync(2, kSmThreads);
+                const float m4 = fmaxf(fmaxf(sh.mpart[0][row], sh.mpart[1][row]),
+                                       fmaxf(sh.mpart[2][row], sh.mpart[3][row]));
+                m_ref = m4 == -INFINITY ? 0.f : m4;
+            }
+            if (!ok) continue;
+            const float c2 = bias2 - m_ref;                  // -inf for rows that do not attend
+            uint32_t pw[16];
+            if (dead) {
+                // None of the warp's 32 rows attends these keys: P = 0, no exponentials.
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pw[i] = 0u;
+            } else if (diag) {
+                const int lim = t_row - key0;                // keys i > lim are in the future
+                float psum = 0.f;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float x0 = 2 * i <= lim ? fmaf(__uint_as_float(sv[2 * i]), a.qk_scale2, c2) : -INFINITY;
+                    const float x1 = 2 * i + 1 <= lim ? fmaf(__uint_as_float(sv[2 * i + 1]), a.qk_scale2, c2) : -INFINITY;
+                    const uint32_t pk = pack_bf16x2(fast_exp2(x0), fast_exp2(x1));
+                    psum += __uint_as_float(pk << 16) + __uint_as_float(pk & 0xffff0000u);
+                    pw[i] = pk;
+                }
+                l_sum += psum;
+            } else {
+                const uint64_t cc = f2_pack(c2, c2);
+                uint64_t acc = f2_pack(0.f, 0.f);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), scale2, cc), x0, x1);
+                    const uint32_t pk = pack_bf16x2(fast_exp2(x0), fast_exp2(x1));
+                    // Row sums of the bf16 weights the MMA multiplies: O / l is exact.
+                    acc = f2_add(acc, f2_pack(__uint_as_float(pk << 16), __uint_as_float(pk & 0xffff0000u)));
+                    pw[i] = pk;
+                }
+                float s0, s1;
+                f2_unpack(acc, s0, s1);
+                l_sum += s0 + s1;
+            }
+            // P over this warp's own S columns (the other quarters may still be loading).
+            tmem_st16(lane_base + kColS + 128u * sb + 32u * kq, pw);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.p_full[sb]);
+        }
+        // Epilogue: l = sum of the four partial sums, O / l -> bf16 (each warp 32 of the dims).
+        sh.lpart[kq][row] = l_sum;
+        const bool ok_o = wait_or_fail(&sh.o_full, 0, a.status, failed);
+        named_sync(2, kSmThreads);
+        if (ok_o) {
+            tc_fence_after();
+            const float l = (sh.lpart[0][row] + sh.lpart[1][row]) + (sh.lpart[2][row] + sh.lpart[3][row]);
+            if (__any_sync(kFull, row_ok && !isfinite(l)) && lane == 0 && kq == 0) report(a.status, DASH_ERR_RANGE_CLAMPED);
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            uint32_t o[32];
+            tmem_ld32(lane_base + kColO + 32u * kq, o);
+            tmem_wait_ld();
+            if (row_ok) {
+                __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(a.out) +
+                                      (((long long)b * a.Hq + h_row) * a.T + t_row) * D + 32 * kq;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    uint4 v;
+                    v.x = pack_bf16x2(__uint_as_float(o[8 * i]) * inv, __uint_as_float(o[8 * i + 1]) * inv);
+                    v.y = pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv);
+                    v.z = pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv);
+                    v.w = pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv);
+                    *reinterpret_cast<uint4 *>(orow + 8 * i) = v;
+                }
+            }
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    if (failed) sh.failed = 1;
+    tc_fence_before();
+    __syncthreads();
+    if (sh.failed && lane == 0) {
+        // Each issuer committed after its last MMA, failure or not: wait (bounded) for the
+        // MMAs in flight before the tensor memory is released.
+        if (warp == kWarpQk) mbar_wait_bounded(&sh.qk_done, 0);
+        if (warp == kWarpPv) mbar_wait_bounded(&sh.o_full, 0);
+    }
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kWarpQk) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tb), "r"(kTmemCols));
+    }
+}
+
+// ---------------------------------------------------------------- host side
+namespace {
+
+using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                              const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                              const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn fa_encode() {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<EncodeFn>(fn);
+}
+
+// 3-D map over a [B*Hkv][T][128] bf16 plane set: box (64 d, 64 keys, 1), 128B swizzle,
+// zero fill out of bounds (keys >= T of the last chunk).
+bool fa_map(EncodeFn enc, CUtensorMap *m, const void *ptr, int T, int BHkv) {
+    cuuint64_t dims[3] = {128, (cuuint64_t)T, (cuuint64_t)BHkv};
+    cuuint64_t strides[2] = {128 * 2, (cuuint64_t)T * 128 * 2};
+    cuuint32_t box[3] = {64, 64, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t fa_smem_bytes(int RT, int C) {
+    size_t off = kRingBytes;
+    off += (size_t)2 * kBiasBatch * RT * 4;      // bias batches
+    off += (size_t)RT * 128 * 4;                 // qbar
+    off += (size_t)((C + 7) & ~7) * 2;           // chunk list
+    return off + 1024;                           // room to align the base to 1024 bytes
+}
+
+}  // namespace
+
+size_t attend_fa_vt_bytes(int B, int Hkv, int T, int D) {
+    const size_t T8 = (size_t)((T + 7) & ~7);
+    return (size_t)B * Hkv * D * T8 * 2;
+}
+
+bool attend_fa_supported(const StageArgs &a) {
+    if (!(a.D == 128 && a.G >= 8 && a.G <= 128 && 128 % a.G == 0 && (a.Bc == 64 || a.Bc == 128)))
+        return false;
+    return fa_smem_bytes(128 / a.G, a.C) + sizeof(FaShared) <= 227 * 1024;
+}
+
+template <int BC>
+static cudaError_t launch_fa_t(const StageArgs &a, cudaStream_t st) {
+    static EncodeFn enc = fa_encode();
+    if (!enc || !a.vt) return cudaErrorNotSupported;
+    const int BHkv = a.B * a.Hkv;
+    cudaError_t e = launch_vtranspose(a.v, a.vt, BHkv, a.T, 128, st);
+    if (e != cudaSuccess) return e;
+    CUtensorMap mk, mvt;
+    if (!fa_map(enc, &mk, a.k, a.T, BHkv)) return cudaErrorInvalidValue;
+    {
+        // V^T [B*Hkv][128][T8]: box (64 keys, 128 dims, 1), 128B swizzle.
+        const int T8 = (a.T + 7) & ~7;
+        cuuint64_t dims[3] = {(cuuint64_t)T8, 128, (cuuint64_t)BHkv};
+        cuuint64_t strides[2] = {(cuuint64_t)T8 * 2, (cuuint64_t)T8 * 2 * 128};
+        cuuint32_t box[3] = {64, 128, 1};
+        cuuint32_t estr[3] = {1, 1, 1};
+        if (enc(&mvt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.vt, dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    FaArgs ta;
+    ta.s = a;
+    ta.RT = 128 / a.G;
+    ta.n_tiles_bg = (a.T + ta.RT - 1) / ta.RT;
+    size_t off = kRingBytes;
+    ta.off_bias = off;
+    off += (size_t)2 * kBiasBatch * ta.RT * 4;
+    ta.off_qbar = off;
+    off += (size_t)ta.RT * 128 * 4;
+    ta.off_list = off;
+    const size_t smem = fa_smem_bytes(ta.RT, a.C);
+    auto kern = k_attend_fa<BC>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const long long grid = (long long)ta.n_tiles_bg * BHkv;
+    if (grid == 0) return cudaSuccess;
+    kern<<<(unsigned)grid, kFaThreads, smem, st>>>(mk, mvt, ta);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attend_fa(const StageArgs &a, cudaStream_t st) {
+    if (a.Bc == 64) return launch_fa_t<64>(a, st);
+    if (a.Bc == 128) return launch_fa_t<128>(a, st);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace dash

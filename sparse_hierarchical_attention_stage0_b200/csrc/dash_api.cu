@@ -94,6 +94,17 @@ size_t bytes_tau(const Shape &s) { return align256((size_t)s.B * s.Hkv * s.T * 4
 size_t bytes_summary(const Shape &s) { return align256((size_t)s.B * s.Hkv * s.Cf * s.D * 4); }
 size_t bytes_mask(const Shape &s) { return align256((size_t)s.B * s.Hkv * s.T * s.W * 8); }
 
+// V^T scratch of the 128-key-block Stage 2 kernel; 0 when that kernel does not apply.
+size_t bytes_vt(const Shape &s) {
+    StageArgs a = {};
+    a.D = s.D;
+    a.G = s.G;
+    a.Bc = s.Bc;
+    a.C = s.C;
+    if (!attend_fa_supported(a)) return 0;
+    return align256(attend_fa_vt_bytes(s.B, s.Hkv, s.T, s.D));
+}
+
 dash_status_t clear_status(void *ws, cudaStream_t st) {
     return cudaMemsetAsync(ws, 0, sizeof(uint32_t), st) == cudaSuccess ? DASH_OK : DASH_ERR_CUDA;
 }
@@ -120,7 +131,13 @@ const char *dash_status_string(dash_status_t s) {
 size_t dash_prefill_workspace_size(const dash_params_t *p) {
     Shape s;
     if (check_params(p, &s) != DASH_OK) return 0;
-    return kStatusBytes + bytes_tau(s) + bytes_summary(s) + bytes_mask(s);
+    return kStatusBytes + bytes_tau(s) + bytes_summary(s) + bytes_mask(s) + bytes_vt(s);
+}
+
+size_t dash_attend_workspace_size(const dash_params_t *p) {
+    Shape s;
+    if (check_params(p, &s) != DASH_OK) return 0;
+    return kStatusBytes + bytes_vt(s);
 }
 
 dash_status_t dash_prefill(const dash_params_t *p, const void *q, const void *k, const void *v,
@@ -169,6 +186,8 @@ dash_status_t dash_prefill(const dash_params_t *p, const void *q, const void *k,
             off += bytes_mask(s);
         }
     }
+    const size_t vt = bytes_vt(s);
+    if (vt && ws_bytes >= off + vt) a.vt = w + off;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if ((rc = clear_status(ws, st)) != DASH_OK) return rc;
     if (!dense) {
@@ -248,6 +267,8 @@ dash_status_t dash_attend(const dash_params_t *p, const void *q, const void *k, 
     a.tau = const_cast<float *>(tau);
     a.mask = const_cast<uint64_t *>(active_blocks);
     a.status = static_cast<uint32_t *>(ws);
+    const size_t vt = bytes_vt(s);
+    if (vt && ws_bytes >= kStatusBytes + vt) a.vt = static_cast<unsigned char *>(ws) + kStatusBytes;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if ((rc = clear_status(ws, st)) != DASH_OK) return rc;
     return from_cuda(launch_attend(a, st));

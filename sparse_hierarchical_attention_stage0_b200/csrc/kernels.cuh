@@ -6,7 +6,7 @@
 namespace dash {
 
 constexpr int kStage0Warps = 4;     // chunks summarised per CTA
-constexpr int kRouteThreads = 512;  // Stage 1 CTA size (one warp per row in the tau solve)
+constexpr int kRouteThreads = 256;  // Stage 1 CTA size
 constexpr int kAttnWarps = 4;       // Stage 2 (mma.sync path) units per CTA
 constexpr int kSub = 32;            // keys per Stage 2 sub-block
 
@@ -19,6 +19,7 @@ struct StageArgs {
     float *p;                 // [B,Hkv,T,C] or null
     uint64_t *mask;           // [B,Hkv,T,W]
     void *out;                // [B,Hq,T,D]
+    void *vt;                 // [B,Hkv,D,T8] V^T scratch for the 128-key-block kernel, or null
     int B, Hq, Hkv, T, D, Bc, G, C, Cf, W;
     RouteConsts rc;
     float qk_scale2;          // log2(e) / sqrt(D)
@@ -46,6 +47,10 @@ int route_rows_per_cta(int C, int D);   // 0 if C is too large for the routing k
 cudaError_t launch_attend(const StageArgs &a, cudaStream_t st);
 bool attend_tc_supported(const StageArgs &a);
 cudaError_t launch_attend_tc(const StageArgs &a, cudaStream_t st);
+bool attend_fa_supported(const StageArgs &a);
+size_t attend_fa_vt_bytes(int B, int Hkv, int T, int D);
+cudaError_t launch_attend_fa(const StageArgs &a, cudaStream_t st);
+cudaError_t launch_vtranspose(const void *v, void *vt, int BHkv, int T, int D, cudaStream_t st);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
 int decode_supported(int G, int Ccap, int D);
 

@@ -6,7 +6,7 @@
 // share one sparse support.  aixai.ru "DashAttention ...", "Трёхстадийная архитектура": the
 // result is handed to Stage 2 as a bit-packed active-block mask (64-bit words).
 //
-// CTA = (b, g, RT consecutive rows of one query chunk), 512 threads:
+// CTA = (b, g, RT consecutive rows of one query chunk), 256 threads:
 //   1. qbar[r] = mean of the G query heads of group g at row t0 + r     (shared memory)
 //   2. x[r][c] = (qbar[r] . summary[c]) * (alpha-1) gamma / sqrt(D) for every routable
 //      chunk c < c_t: 4 lanes per chunk, each owning an interleaved quarter of d (coalesced
@@ -21,12 +21,14 @@
 namespace dash {
 
 int route_rows_per_cta(int C, int D) {
-    const size_t budget = 200 * 1024;
-    for (int rt : {16, 8, 4}) {
-        size_t xstride = (size_t)((C + 3) & ~3);
-        size_t bytes = (size_t)rt * D * 4 + (size_t)rt * xstride * 4;
-        if (bytes <= budget) return rt;
-    }
+    // Rows per CTA: as many as keep about three CTAs resident per SM (24 warps to hide the
+    // shared-memory and FMA latencies of the score loop), within 200 KB for one CTA when C is
+    // too large for that.
+    const size_t xstride = (size_t)((C + 3) & ~3);
+    for (int rt : {16, 8, 4})
+        if ((size_t)rt * D * 4 + (size_t)rt * xstride * 4 <= 72 * 1024) return rt;
+    for (int rt : {16, 8, 4})
+        if ((size_t)rt * D * 4 + (size_t)rt * xstride * 4 <= 200 * 1024) return rt;
     return 0;
 }
 
@@ -65,20 +67,14 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(StageArgs a) {
     const float *sumg = a.summary + (long long)bg * a.Cf * D;
     const int kslice = lane & 3, cc = lane >> 2;
     constexpr int kStep = (kRouteThreads / 32) * 8;       // chunks per CTA-wide step
-    // The summary slices of the next step are loaded while the current step computes, so
-    // the L2 latency of the loads overlaps the FMAs.
-    auto load_slice = [&](int cbase, float4 (&sv)[D / 16]) {
-        const float4 *s4 = reinterpret_cast<const float4 *>(sumg + (long long)min(cbase + cc, n - 1) * D);
-#pragma unroll
-        for (int i = 0; i < D / 16; ++i) sv[i] = __ldg(s4 + 4 * i + kslice);
-    };
-    float4 cur[D / 16], nxt[D / 16];
-    int cbase = warp * 8;
-    if (cbase < n) load_slice(cbase, cur);
-    for (; cbase < n; cbase += kStep) {
+    for (int cbase = warp * 8; cbase < n; cbase += kStep) {
         const int c = cbase + cc;
-        const bool more = cbase + kStep < n;
-        if (more) load_slice(cbase + kStep, nxt);
+        float4 cur[D / 16];                       // all loads of the slice in flight at once
+        {
+            const float4 *s4 = reinterpret_cast<const float4 *>(sumg + (long long)min(c, n - 1) * D);
+#pragma unroll
+            for (int i = 0; i < D / 16; ++i) cur[i] = __ldg(s4 + 4 * i + kslice);
+        }
         float acc[RT];
 #pragma unroll
         for (int r = 0; r < RT; ++r) acc[r] = 0.f;
@@ -104,10 +100,6 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(StageArgs a) {
         if (kslice == 0 && c < n) {
 #pragma unroll
             for (int r = 0; r < RT; ++r) xs[r * xstride + c] = __fmul_rn(acc[r], scale);
-        }
-        if (more) {
-#pragma unroll
-            for (int i = 0; i < D / 16; ++i) cur[i] = nxt[i];
         }
     }
     __syncthreads();

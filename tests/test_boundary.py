@@ -58,6 +58,16 @@ def test_workspace_sizes(dash):
     r = lambda x: (x + 255) // 256 * 256
     expect = 256 + r(B * Hkv * T * 4) + r(B * Hkv * (T // Bc) * D * 4) + r(B * Hkv * T * W * 8)
     assert dash.prefill_workspace_size(prm) == expect
+    assert dash.attend_workspace_size(prm) == 256
+    g16 = _p(dash, heads_q=32, heads_kv=2, seq_len=1001)
+    T2 = 1001
+    C2 = (T2 + Bc - 1) // Bc
+    W2 = (C2 + 63) // 64
+    vt2 = r(B * Hkv * D * ((T2 + 7) // 8 * 8) * 2)
+    assert dash.attend_workspace_size(g16) == 256 + vt2
+    assert dash.prefill_workspace_size(g16) == (256 + r(B * Hkv * T2 * 4) + r(B * Hkv * (T2 // Bc) * D * 4)
+                                                + r(B * Hkv * T2 * W2 * 8) + vt2)
+    assert dash.attend_workspace_size(_p(dash, head_dim=96)) == 0
     assert dash.decode_workspace_size(prm) == 256
     assert dash.prefill_workspace_size(_p(dash, head_dim=96)) == 0
 
@@ -98,7 +108,8 @@ def test_prefill_rejects_bad_pointers_and_small_workspace(dash):
              1 << 40, None) == 1                                    # misaligned q
     assert f(ctypes.byref(prm), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, FAKE + 16,
              1 << 40, None) == 1                                    # misaligned workspace
-    need = dash.prefill_workspace_size(prm)
+    # the V^T scratch is optional: the smallest accepted workspace leaves it out
+    need = dash.prefill_workspace_size(prm) - dash.attend_workspace_size(prm) + 256
     assert f(ctypes.byref(prm), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, FAKE, need - 1,
              None) == 3
     dense = _p(dash, flags=1)
