@@ -115,6 +115,36 @@ def test_prefill_matches_oracle(dash, alpha, G, D, Bc, T):
     assert dash.read_device_status(res["ws"]) == 0
 
 
+@pytest.mark.parametrize("G,Bc,T", [(16, 64, 2100 + 37), (8, 128, 1500 + 3)])
+def test_attend_without_vt_scratch_takes_the_tile_kernel(dash, G, Bc, T):
+    """dash_attend with only the 256-byte status word cannot hold V^T, so Stage 2 runs on the
+    64-key-block tile kernel; with dash_attend_workspace_size bytes it runs the 128-key-block
+    kernel.  Both match the oracle, across several routing-bias batches (T > 32 chunks)."""
+    Hkv = 2
+    cfg = _cfg(1, G * Hkv, Hkv, T, 128, Bc, 1.5, seed=23 + G)
+    q, k, v, hc = make_prefill(cfg)
+    qd, kd, vd, hcd = _to(q, k, v, hc)
+    res = dash.prefill(qd, kd, vd, hcd, chunk_size=Bc, alpha=1.5, enable_gqa=True,
+                       return_active_blocks=True, return_summary=True)
+    torch.cuda.synchronize()
+    # tau is re-derived by Stage 1 alone (bit-identical to the prefill's)
+    summ = res["summary"]
+    r = dash.route(qd, summ, Hkv, Bc, 1.5, return_p=False)
+    tau, mask = r["tau"], r["active_blocks"]
+    assert torch.equal(mask, res["active_blocks"])
+    prm = dash.make_params(1, G * Hkv, Hkv, T, 128, Bc, 1.5, 1.0, 1.0, True)
+    assert dash.attend_workspace_size(prm) > 256
+    small = dash.workspace(256, qd.device)
+    o_tile = dash.attend(qd, kd, vd, summ, tau, mask, Bc, 1.5, ws=small)
+    o_fast = dash.attend(qd, kd, vd, summ, tau, mask, Bc, 1.5)
+    torch.cuda.synchronize()
+    assert dash.read_device_status(small) == 0
+    ref = oracle.prefill(q, k, v, hc, Bc, 1.5)
+    check_output(o_tile.cpu().float().numpy(), ref["O"], tag="tile kernel")
+    check_output(o_fast.cpu().float().numpy(), ref["O"], tag="128-key kernel")
+    assert torch.equal(o_fast, res["out"])
+
+
 def test_prefill_single_partial_chunk(dash):
     """T < chunk_size: every row is local causal attention inside chunk 0."""
     q, k, v, hc = make_prefill(_cfg(2, 8, 2, 40, 64, 64, 1.5, planted=False, seed=3))
