@@ -27,12 +27,14 @@
 // against that fixed reference, so O is never rescaled.  A logit so far above the reference
 // that the row's fp32 sum overflows (beyond about 2^110 with 2^17 keys) leaves a non-finite
 // row sum; such rows are reported as DASH_ERR_RANGE_CLAMPED.  Row sums add the bf16 weights
-// the MMA multiplies.  Off the diagonal the exponent arguments and the sums run on packed
-// fp32 pairs (fma.rn.f32x2, add.rn.f32x2): about 3.5 instructions per score.
+// the MMA multiplies, computed by the tensor core: V^T carries 16 extra rows of ones, so
+// P V (N = 144) leaves sum_k P[r, k] in O column 128.  Off the diagonal the exponent
+// arguments run on packed fp32 pairs (fma.rn.f32x2): about 2.5 instructions per score.
 // Warp roles: 0 TMA producer (K and V^T rings, 3 stages each, 128B-swizzled), 1 Q K^T issuer
 // and TMEM owner, 2 routing-bias producer (recomputes qbar.summary with Stage 1's exact
-// arithmetic, 32 chunks per batch, double-buffered), 3 P V issuer, 4-19 softmax + epilogue.
-// TMEM: Q 64 columns | S0 128 | S1 128 | O 128.  Every wait is bounded; on timeout the CTA
+// arithmetic, 32 chunks per batch, double-buffered), 3 P V issuer, 4-19 softmax + epilogue,
+// 20 V^T producer (warp 0 then streams K only).
+// TMEM: Q 64 columns | S0 128 | S1 128 | O 144 (128 dims + row sums).  Every wait is bounded; on timeout the CTA
 // records DASH_ERR_DEVICE_TIMEOUT and drains.
 #include "kernels.cuh"
 #include "tc_common.cuh"
@@ -43,21 +45,24 @@ namespace {
 
 constexpr int kSmWarps = 16;
 constexpr int kSmThreads = kSmWarps * 32;
-constexpr int kFaThreads = 4 * 32 + kSmThreads;
+constexpr int kFaThreads = 4 * 32 + kSmThreads + 32;
 constexpr int kStages = 3;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColQ = 0, kColS = 64, kColO = 320;     // S buffer b at kColS + 128 b
 constexpr int kBiasBatch = 32;
-constexpr int kWarpTma = 0, kWarpQk = 1, kWarpBias = 2, kWarpPv = 3, kWarpSm0 = 4;
-constexpr uint32_t kBlkBytes = 32768;      // K: 2 d-panels x [128 keys][128 B]; V^T: 2 key-halves x [128 d][128 B]
-constexpr uint32_t kOffV = kStages * kBlkBytes, kRingBytes = 2 * kStages * kBlkBytes;
+constexpr int kWarpTma = 0, kWarpQk = 1, kWarpBias = 2, kWarpPv = 3, kWarpSm0 = 4,
+              kWarpTmaV = kWarpSm0 + kSmWarps;
+constexpr uint32_t kBlkBytes = 32768;      // K stage: 2 d-panels x [128 keys][128 B]
+constexpr int kNv = 144;                   // P V columns: 128 dims of V, then 16 columns of ones
+constexpr uint32_t kVHalf = kNv * 128;     // V^T key-half: [144 rows][64 keys x 2 B] (rows >= 128: ones)
+constexpr uint32_t kVStage = 2 * kVHalf;
+constexpr uint32_t kOffV = kStages * kBlkBytes, kRingBytes = kOffV + kStages * kVStage;
 
 struct FaShared {
     uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
     uint64_t s_full[2], p_full[2], pv_done[2];  // per S buffer: never more than one phase ahead
     uint64_t o_full, qk_done;
     float mpart[4][128];                   // partial row maxima of the first block
-    float lpart[4][128];                   // partial row sums
     uint32_t tmem_base;
     int n_chunks;
     int failed;
@@ -77,11 +82,6 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
     return d;
 }
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
 
 }  // namespace
 
@@ -94,8 +94,8 @@ struct FaArgs {
 
 template <int BC>
 __global__ void __launch_bounds__(kFaThreads, 1)
-k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmVt,
-            const FaArgs ta) {
+k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmK128,
+            const __grid_constant__ CUtensorMap tmVt, const FaArgs ta) {
     extern __shared__ unsigned char smem_dyn[];
     __shared__ FaShared sh;
     const StageArgs &a = ta.s;
@@ -194,6 +194,16 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
             }
         }
     }
+    if (warp == kWarpTma) {
+        // Rows 128-143 of every V^T key-half stage are ones (bf16 1.0 = 0x3f80): P V then
+        // also yields the row sums of P in O columns 128-143.  TMA never writes these rows.
+        const uint4 ones = make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);
+        for (int i = lane; i < kStages * 2 * 16 * 8; i += 32) {
+            const int half = i / (16 * 8), r = (i / 8) % 16, c = i % 8;
+            *reinterpret_cast<uint4 *>(base + kOffV + (size_t)half * kVHalf + (128 + r) * 128 + c * 16) = ones;
+        }
+        fence_proxy_async();
+    }
     // Softmax warps: quadrant sp (TMEM lanes 32 sp ..), key quarter kq of every block.
     const int sp = warp & 3;
     const int kq = (warp - kWarpSm0) >> 2;
@@ -204,7 +214,7 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
     const bool row_ok = t_row < a.T;
     __syncthreads();
     const uint32_t tb = sh.tmem_base;
-    if (warp >= kWarpSm0) {
+    if (warp >= kWarpSm0 && warp < kWarpTmaV) {
         // Q row -> TMEM columns [0, 64): this warp's quarter of the dims (32 dims, 16 columns).
         const __nv_bfloat16 *qr = reinterpret_cast<const __nv_bfloat16 *>(a.q) +
                                   (((long long)b * a.Hq + h_row) * a.T + (row_ok ? t_row : 0)) * D +
@@ -239,10 +249,13 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
         return BC == 64 ? chunk_at(2 * j + h) * 64 : chunk_at(j) * 128 + 64 * h;
     };
 
-    if (warp == kWarpTma) {
+    if (warp == kWarpTma || warp == kWarpTmaV) {
         // ------------------------------------------------------------ TMA producer
         // K runs one block ahead of V^T (Q K^T needs it first).  K: a block's two 64-key
-        // halves land at rows 0-63 and 64-127 of each 16 KB d-panel.  V^T: key-half h is one
+        // halves land at rows 0-63 and 64-127 of each 16 KB d-panel, as one 128-key box per
+        // panel when the halves are adjacent keys (always for 128-key chunks, mostly in dense
+        // unions): TMA throughput per SM grows with the request size (measured on B200: about
+        // 35, 44 and 53 bytes per cycle for 8, 16 and 32 KB boxes).  V^T: key-half h is one
         // [128 d][64 keys] box at 16 KB * h.  An empty second half is not loaded (its MMAs are
         // not issued either).
         int k_issued = 0, v_issued = 0;
@@ -253,13 +266,17 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
             uint64_t *full = is_v ? &sh.v_full[s] : &sh.k_full[s];
             if (!wait_or_fail(empty, ph ^ 1u, a.status, failed)) return false;
             if (lane == 0) {
-                unsigned char *st = base + (is_v ? kOffV : 0u) + (size_t)s * kBlkBytes;
+                unsigned char *st = base + (is_v ? kOffV + (size_t)s * kVStage : (size_t)s * kBlkBytes);
                 const int nh = entry_of(j, 1) >= 0 ? 2 : 1;
                 mbar_arrive_expect_tx(full, 16384u * nh);
                 for (int h = 0; h < nh; ++h) {
                     const int key0 = key0_of(j, h);
                     if (is_v) {
-                        tma_load_3d(st + 16384 * h, &tmVt, key0, 0, (int)bg, full);
+                        tma_load_3d(st + kVHalf * h, &tmVt, key0, 0, (int)bg, full);
+                    } else if (nh == 2 && h == 0 && key0_of(j, 1) == key0 + 64) {
+                        tma_load_3d(st, &tmK128, 0, key0, (int)bg, full);
+                        tma_load_3d(st + 16384, &tmK128, 64, key0, (int)bg, full);
+                        break;
                     } else {
                         tma_load_3d(st + 8192 * h, &tmK, 0, key0, (int)bg, full);
                         tma_load_3d(st + 16384 + 8192 * h, &tmK, 64, key0, (int)bg, full);
@@ -270,11 +287,10 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
             if (is_v) v_issued = j + 1; else k_issued = j + 1;
             return true;
         };
-        if (n_blocks > 0) issue(false, 0);
-        for (int j = 0; j < n_blocks && !failed; ++j) {
-            if (j + 1 < n_blocks && !issue(false, j + 1)) break;
-            if (!issue(true, j)) break;
-        }
+        // Warp 0 streams K, warp 20 streams V^T: neither ring waits behind the other.
+        const bool is_v = warp == kWarpTmaV;
+        for (int j = 0; j < n_blocks && !failed; ++j)
+            if (!issue(is_v, j)) break;
         if (failed) {
             // Bounded wait for the copies still in flight (the last ones per ring).
             for (int i = max(0, k_issued - kStages); i < k_issued; ++i)
@@ -317,10 +333,10 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
     } else if (warp == kWarpPv) {
         // ------------------------------------------------------------ P V issuer
         // P of keys 32q .. 32q+31 sits in the first 16 columns of S quarter q; B = V^T, K-major.
-        constexpr uint32_t id_pv = idesc_bf16(128, D, 0);
+        constexpr uint32_t id_pv = idesc_bf16(128, kNv, 0);
         uint64_t vdesc[kStages];
 #pragma unroll
-        for (int s = 0; s < kStages; ++s) vdesc[s] = smem_desc_sw128(smem_u32(base + kOffV + (size_t)s * kBlkBytes), 16, 1024);
+        for (int s = 0; s < kStages; ++s) vdesc[s] = smem_desc_sw128(smem_u32(base + kOffV + (size_t)s * kVStage), 16, 1024);
         for (int j = 0; j < n_blocks; ++j) {
             const int s = j % kStages, sb = j & 1;
             if (!wait_or_fail(&sh.v_full[s], (uint32_t)(j / kStages) & 1u, a.status, failed)) break;
@@ -335,8 +351,8 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     if (kk >= 4 && !full_blk) break;
-                    // key-half kk/4 of V^T at 16 KB, 32 B per 16 keys
-                    const uint64_t bd = bd0 + (uint64_t)(((kk / 4) * 16384 + (kk % 4) * 32) >> 4);
+                    // key-half kk/4 of V^T (144 rows), 32 B per 16 keys
+                    const uint64_t bd = bd0 + (uint64_t)(((kk / 4) * kVHalf + (kk % 4) * 32) >> 4);
                     mma_ts(tb + kColO, pb + 32u * (kk / 2) + 8u * (kk % 2), bd, id_pv,
                            (j > 0 || kk > 0) ? 1u : 0u);
                 }
@@ -382,14 +398,14 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
             __syncwarp();
             named_sync(1, 32 + kSmThreads);
         }
-    } else if (warp >= kWarpSm0) {
+    } else if (warp >= kWarpSm0 && warp < kWarpTmaV) {
         // ------------------------------------------------------------ softmax
         // Four threads per row: warp (sp, kq) owns keys 32 kq .. 32 kq + 31 of every block for
         // the rows of TMEM quadrant sp.  Every named barrier is passed by all softmax warps,
         // failure or not.
         const uint32_t lane_base = tb + ((uint32_t)(32 * sp) << 16);
         const int half = kq >> 1;
-        float m_ref = 0.f, l_sum = 0.f;
+        float m_ref = 0.f;
         const uint64_t scale2 = f2_pack(a.qk_scale2, a.qk_scale2);
         for (int j = 0; j < n_blocks; ++j) {
             const int sb = j & 1;
@@ -443,31 +459,20 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                 for (int i = 0; i < 16; ++i) pw[i] = 0u;
             } else if (diag) {
                 const int lim = t_row - key0;                // keys i > lim are in the future
-                float psum = 0.f;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const float x0 = 2 * i <= lim ? fmaf(__uint_as_float(sv[2 * i]), a.qk_scale2, c2) : -INFINITY;
                     const float x1 = 2 * i + 1 <= lim ? fmaf(__uint_as_float(sv[2 * i + 1]), a.qk_scale2, c2) : -INFINITY;
-                    const uint32_t pk = pack_bf16x2(fast_exp2(x0), fast_exp2(x1));
-                    psum += __uint_as_float(pk << 16) + __uint_as_float(pk & 0xffff0000u);
-                    pw[i] = pk;
+                    pw[i] = pack_bf16x2(fast_exp2(x0), fast_exp2(x1));
                 }
-                l_sum += psum;
             } else {
                 const uint64_t cc = f2_pack(c2, c2);
-                uint64_t acc = f2_pack(0.f, 0.f);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     float x0, x1;
                     f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), scale2, cc), x0, x1);
-                    const uint32_t pk = pack_bf16x2(fast_exp2(x0), fast_exp2(x1));
-                    // Row sums of the bf16 weights the MMA multiplies: O / l is exact.
-                    acc = f2_add(acc, f2_pack(__uint_as_float(pk << 16), __uint_as_float(pk & 0xffff0000u)));
-                    pw[i] = pk;
+                    pw[i] = pack_bf16x2(fast_exp2(x0), fast_exp2(x1));
                 }
-                float s0, s1;
-                f2_unpack(acc, s0, s1);
-                l_sum += s0 + s1;
             }
             // P over this warp's own S columns (the other quarters may still be loading).
             tmem_st16(lane_base + kColS + 128u * sb + 32u * kq, pw);
@@ -476,13 +481,16 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh.p_full[sb]);
         }
-        // Epilogue: l = sum of the four partial sums, O / l -> bf16 (each warp 32 of the dims).
-        sh.lpart[kq][row] = l_sum;
+        // Epilogue: l = O column 128 (P times the ones rows of V^T: the sum of the bf16
+        // weights the MMA multiplied), O / l -> bf16 (each warp 32 of the dims).
         const bool ok_o = wait_or_fail(&sh.o_full, 0, a.status, failed);
-        named_sync(2, kSmThreads);
         if (ok_o) {
             tc_fence_after();
-            const float l = (sh.lpart[0][row] + sh.lpart[1][row]) + (sh.lpart[2][row] + sh.lpart[3][row]);
+            uint32_t lw[1];
+            asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];"
+                         : "=r"(lw[0]) : "r"(lane_base + kColO + 128u));
+            tmem_wait_ld();
+            const float l = __uint_as_float(lw[0]);
             if (__any_sync(kFull, row_ok && !isfinite(l)) && lane == 0 && kq == 0) report(a.status, DASH_ERR_RANGE_CLAMPED);
             const float inv = l > 0.f ? 1.f / l : 0.f;
             uint32_t o[32];
@@ -538,12 +546,12 @@ EncodeFn fa_encode() {
     return reinterpret_cast<EncodeFn>(fn);
 }
 
-// 3-D map over a [B*Hkv][T][128] bf16 plane set: box (64 d, 64 keys, 1), 128B swizzle,
+// 3-D map over a [B*Hkv][T][128] bf16 plane set: box (64 d, `keys` keys, 1), 128B swizzle,
 // zero fill out of bounds (keys >= T of the last chunk).
-bool fa_map(EncodeFn enc, CUtensorMap *m, const void *ptr, int T, int BHkv) {
+bool fa_map(EncodeFn enc, CUtensorMap *m, const void *ptr, int T, int BHkv, int keys) {
     cuuint64_t dims[3] = {128, (cuuint64_t)T, (cuuint64_t)BHkv};
     cuuint64_t strides[2] = {128 * 2, (cuuint64_t)T * 128 * 2};
-    cuuint32_t box[3] = {64, 64, 1};
+    cuuint32_t box[3] = {64, (cuuint32_t)keys, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -578,8 +586,9 @@ static cudaError_t launch_fa_t(const StageArgs &a, cudaStream_t st) {
     const int BHkv = a.B * a.Hkv;
     cudaError_t e = launch_vtranspose(a.v, a.vt, BHkv, a.T, 128, st);
     if (e != cudaSuccess) return e;
-    CUtensorMap mk, mvt;
-    if (!fa_map(enc, &mk, a.k, a.T, BHkv)) return cudaErrorInvalidValue;
+    CUtensorMap mk, mk128, mvt;
+    if (!fa_map(enc, &mk, a.k, a.T, BHkv, 64) || !fa_map(enc, &mk128, a.k, a.T, BHkv, 128))
+        return cudaErrorInvalidValue;
     {
         // V^T [B*Hkv][128][T8]: box (64 keys, 128 dims, 1), 128B swizzle.
         const int T8 = (a.T + 7) & ~7;
@@ -608,7 +617,7 @@ static cudaError_t launch_fa_t(const StageArgs &a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     const long long grid = (long long)ta.n_tiles_bg * BHkv;
     if (grid == 0) return cudaSuccess;
-    kern<<<(unsigned)grid, kFaThreads, smem, st>>>(mk, mvt, ta);
+    kern<<<(unsigned)grid, kFaThreads, smem, st>>>(mk, mk128, mvt, ta);
     return cudaGetLastError();
 }
 
