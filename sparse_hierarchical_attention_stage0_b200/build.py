@@ -18,7 +18,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libdash.so")
 BUILD = os.path.join(HERE, "_build")
-SOURCES = ["stage0.cu", "route.cu", "attend.cu", "attend_tc.cu", "attend_fa.cu", "vtranspose.cu",
+SOURCES = ["stage0.cu", "route.cu", "attend.cu", "attend_tc.cu", "attend_fa.cu", "attend_pair.cu", "vtranspose.cu",
            "decode.cu", "dash_api.cu", "dash_static_ws.cu"]
 HEADERS = ["dash_common.cuh", "kernels.cuh", "attn_warp.cuh", "tc_common.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

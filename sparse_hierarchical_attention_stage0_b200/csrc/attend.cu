@@ -259,6 +259,11 @@ static cudaError_t launch_attend_t(const StageArgs &a, cudaStream_t st) {
 }
 
 cudaError_t launch_attend(const StageArgs &a, cudaStream_t st) {
+    // Pairs of SMs share each K/V block between two tiles, so they walk the union of both
+    // tiles' chunks: a gain only when every visible chunk is attended anyway (dense, or every
+    // chunk forced active); with routing the larger union costs more than the halved copies
+    // save (measured at 128K: 128 ms against 117 ms).
+    if (a.vt && a.ignore_routing && attend_pair_supported(a)) return launch_attend_pair(a, st);
     if (a.vt && attend_fa_supported(a)) return launch_attend_fa(a, st);
     if (attend_tc_supported(a)) return launch_attend_tc(a, st);
     if (a.D == 128 && a.Bc == 64) return launch_attend_t<128, 64>(a, st);

@@ -30,7 +30,7 @@
 // the MMA multiplies, computed by the tensor core: V^T carries 16 extra rows of ones, so
 // P V (N = 144) leaves sum_k P[r, k] in O column 128.  Off the diagonal the exponent
 // arguments run on packed fp32 pairs (fma.rn.f32x2): about 2.5 instructions per score.
-// Warp roles: 0 TMA producer (K and V^T rings, 3 stages each, 128B-swizzled), 1 Q K^T issuer
+// Warp roles: 0 K producer (3-stage ring, 128B-swizzled), 1 Q K^T issuer
 // and TMEM owner, 2 routing-bias producer (recomputes qbar.summary with Stage 1's exact
 // arithmetic, 32 chunks per batch, double-buffered), 3 P V issuer, 4-19 softmax + epilogue,
 // 20 V^T producer (warp 0 then streams K only).
@@ -108,9 +108,10 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
     int16_t *list = reinterpret_cast<int16_t *>(base + ta.off_list);    // [C]
 
     const int RT = ta.RT, G = a.G;
-    const int BHkv = a.B * a.Hkv;
-    const int tile_rev = blockIdx.x / BHkv, bgi = blockIdx.x % BHkv;
-    const int tt = ta.n_tiles_bg - 1 - tile_rev;                        // longest tiles first
+    // (b, g)-major, longest tiles first: the CTAs in flight share one (b, g)'s K and V^T in L2
+    // (67 MB at T = 128K; both planes at once overflow the 126 MB L2: 3% slower, measured).
+    const int tile_rev = blockIdx.x % ta.n_tiles_bg, bgi = blockIdx.x / ta.n_tiles_bg;
+    const int tt = ta.n_tiles_bg - 1 - tile_rev;
     const int b = bgi / a.Hkv, g = bgi % a.Hkv;
     const long long bg = bgi;
     const int t0 = tt * RT;

@@ -50,6 +50,8 @@ cudaError_t launch_attend_tc(const StageArgs &a, cudaStream_t st);
 bool attend_fa_supported(const StageArgs &a);
 size_t attend_fa_vt_bytes(int B, int Hkv, int T, int D);
 cudaError_t launch_attend_fa(const StageArgs &a, cudaStream_t st);
+bool attend_pair_supported(const StageArgs &a);
+cudaError_t launch_attend_pair(const StageArgs &a, cudaStream_t st);
 cudaError_t launch_vtranspose(const void *v, void *vt, int BHkv, int T, int D, cudaStream_t st);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
 int decode_supported(int G, int Ccap, int D);

@@ -166,6 +166,38 @@ def test_dense_equals_force_all_active_and_causal_attention(dash):
     check_output(o_dense.cpu().float().numpy(), ref, tag="dense")
 
 
+@pytest.mark.parametrize("B,G,Bc,T", [(2, 16, 64, 993), (1, 8, 64, 1505), (1, 32, 128, 1027),
+                                      (2, 8, 128, 700)])
+def test_dense_on_sm_pairs_matches_causal_attention(dash, B, G, Bc, T):
+    """Dense mode runs on pairs of SMs, two tiles per pair.  Odd tile counts leave the last
+    pair's second tile past the end of the sequence; batch 2 covers several (b, g) planes."""
+    cfg = _cfg(B, 2 * G, 2, T, 128, Bc, 1.5, planted=False, seed=20 + G + B)
+    q, k, v, hc = make_prefill(cfg)
+    qd, kd, vd = _to(q, k, v)
+    prm = dash.make_params(B, 2 * G, 2, T, 128, Bc, enable_gqa=True)
+    ws = dash.workspace(dash.prefill_workspace_size(prm), qd.device)
+    out = dash.prefill(qd, kd, vd, None, Bc, enable_gqa=True, dense=True, ws=ws)
+    torch.cuda.synchronize()
+    assert dash.read_device_status(ws) == 0
+    ref = oracle.stage2(q, k, v, None, Bc, dense=True)
+    check_output(out.cpu().float().numpy(), ref, tag=f"dense pairs B={B} G={G} Bc={Bc}")
+
+
+def test_prefill_batch2_matches_oracle(dash):
+    """Routed prefill over four (b, g) planes (the Stage 2 grid walks them one after another)."""
+    cfg = _cfg(2, 32, 2, 700, 128, 64, 1.5, seed=31)
+    q, k, v, hc = make_prefill(cfg)
+    res = dash.prefill(*_to(q, k, v, hc), chunk_size=64, alpha=1.5, enable_gqa=True,
+                       return_p=True, return_active_blocks=True)
+    torch.cuda.synchronize()
+    ref = oracle.prefill(q, k, v, hc, 64, 1.5)
+    C = ref["p"].shape[-1]
+    check_routing(unpack_mask(res["active_blocks"], C), res["p"].cpu().double().numpy(),
+                  ref["p"], ref["m"], np.arange(700), 64, 1.5, tag="prefill B=2")
+    check_output(res["out"].cpu().float().numpy(), ref["O"], tag="prefill B=2")
+    assert dash.read_device_status(res["ws"]) == 0
+
+
 def test_inactive_chunks_do_not_touch_the_output(dash):
     """Rewriting V inside chunks that none of the last query chunk's 64 tokens routes to
     leaves those tokens' outputs identical to the bit."""
