@@ -39,6 +39,7 @@ METRIC = "prefill tokens/s & active-FLOP TFLOP/s at 128K; decode tok/s; % roofli
 GAMMA_FILE = os.path.join(ROOT, "tests", "golden", "gamma_prefill128k.json")
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+E2E_SLICES = 16         # row slices of the end-to-end prefill from host memory (8: 130 ms, 16: 128 ms at 128K)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -446,17 +447,14 @@ def main():
         dense()
     dense_ms = statistics.mean(timed(dense, max(2, min(args.steps, 3)), stream, flush))
 
-    # End to end through host buffers: pinned H2D of q, k, v, head_cls; prefill; D2H of out.
+    # End to end through host buffers: dash_prefill_host copies q, k, v, head_cls from pinned
+    # host memory and out back, in row slices overlapped with the computation.
     hq, hk, hv, hhc = (x.pin_memory() for x in (q_h, k_h, v_h, hc_h))
     ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
 
     def e2e():
-        q.copy_(hq, non_blocking=True)
-        k.copy_(hk, non_blocking=True)
-        v.copy_(hv, non_blocking=True)
-        hc.copy_(hhc, non_blocking=True)
-        prefill()
-        ho.copy_(out, non_blocking=True)
+        dash.prefill_host(hq, hk, hv, hhc, ho, q, k, v, hc, out, Bc, cfg.alpha, cfg.gamma,
+                          enable_gqa=True, n_slices=E2E_SLICES, ws=ws)
 
     e2e()
     e2e_ms = statistics.mean(timed(e2e, args.steps, stream, flush))
@@ -498,7 +496,8 @@ def main():
                              "frac_of_8tbs_nominal": s01_gbs / 8000.0,
                              "bytes": sb["stage0"] + sb["stage1"]},
         "e2e": {"value": world * B * T / (e2e_ms / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "call": f"dash_prefill_host, {E2E_SLICES} row slices"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }

@@ -124,6 +124,35 @@ dash_status_t dash_prefill(const dash_params_t *params, const void *q, const voi
                            float *p, uint64_t *active_blocks, void *ws, size_t ws_bytes,
                            void *stream);
 
+/* The same causal prefill with its inputs and output in host memory, the copies overlapped
+ * with the computation (gist.science DashAttention summary, "Stufe 2": row t attends only keys
+ * <= t, so rows [0, r) can finish before the queries of later rows arrive).
+ *   q_host, k_host, v_host, head_cls_host, out_host: host buffers of the dash_prefill shapes;
+ *            page-locked (cudaHostAlloc / cudaHostRegister) for the copies to overlap
+ *   q, k, v, head_cls, out: device buffers of the same shapes, owned by the caller (the
+ *            library allocates no memory); head_cls/head_cls_host may be NULL with
+ *            DASH_FLAG_DENSE
+ *   ws, ws_bytes: at least dash_prefill_workspace_size(params) bytes (the V^T scratch is
+ *            what lets the rows be sliced)
+ *   n_slices: row slices (1 = no overlap; at most 64 are used); each slice but the last is
+ *            a multiple of 128 rows.  With the 128-key-block Stage 2 kernel unavailable for
+ *            these parameters the call runs as one slice.
+ *   stream:  computation; h2d_stream, d2h_stream: the two copy directions.  All three must
+ *            be distinct streams of the current device.  Both copy streams first wait for
+ *            the work already queued on stream.  Order: head_cls, k and v to the device,
+ *            then q slice by slice on h2d_stream; Stage 0, then Stages 1-2 of
+ *            each slice once its q has arrived, on stream; out of each slice back to
+ *            out_host on d2h_stream once computed.  stream finally waits for the last copy,
+ *            so synchronising stream covers the whole call.
+ * The device output equals dash_prefill's bit for bit.  Creates and destroys its CUDA events
+ * (2 * slices + 3) within the call.  Returns DASH_OK when every copy and launch was issued,
+ * DASH_ERR_INVALID_ARGUMENT for a NULL buffer or n_slices < 1. */
+dash_status_t dash_prefill_host(const dash_params_t *params, const void *q_host,
+                                const void *k_host, const void *v_host,
+                                const float *head_cls_host, void *out_host, void *q, void *k,
+                                void *v, float *head_cls, void *out, void *ws, size_t ws_bytes,
+                                int n_slices, void *stream, void *h2d_stream, void *d2h_stream);
+
 /* Stage 0 alone: summary_k [B, H_kv, T/Bc, D] fp32 of every complete chunk of k
  * [B, H_kv, T, D] bf16.  Each summary is computed by one warp from a TMA (bulk-copy) staged
  * chunk in shared memory.  ws (>= 256 bytes) holds the status word.  summary_k may be NULL

@@ -37,7 +37,7 @@ FLAG_FORCE_ALL_ACTIVE = 2
 FLAG_ESTIMATE_DIAGONAL = 4
 
 # Every symbol include/dash.h declares.
-EXPORTS = ("dash_prefill_workspace_size", "dash_prefill", "dash_stage0", "dash_route",
+EXPORTS = ("dash_prefill_workspace_size", "dash_prefill", "dash_prefill_host", "dash_stage0", "dash_route",
            "dash_attend_workspace_size", "dash_attend", "dash_update_chunk_cache", "dash_decode_workspace_size",
            "dash_decode", "dash_read_device_status", "dash_status_string")
 
@@ -61,6 +61,8 @@ lib.dash_attend_workspace_size.restype = _sz
 lib.dash_decode_workspace_size.argtypes = [_P]
 lib.dash_decode_workspace_size.restype = _sz
 lib.dash_prefill.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+lib.dash_prefill_host.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                                  ctypes.c_int, _vp, _vp, _vp]
 lib.dash_stage0.argtypes = [_P, _vp, _vp, _vp, _vp, _sz, _vp]
 lib.dash_route.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 lib.dash_attend.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
@@ -163,6 +165,43 @@ def prefill(q, k, v, head_cls, chunk_size=64, alpha=1.5, gamma=1.0, sigma=1.0,
     if not (return_p or return_active_blocks or return_summary):
         return out
     return dict(out=out, p=p, active_blocks=mask, summary=summ, ws=ws)
+
+
+_copy_streams = {}
+
+
+def prefill_host(q_host, k_host, v_host, head_cls_host, out_host, q, k, v, head_cls, out,
+                 chunk_size=64, alpha=1.5, gamma=1.0, sigma=1.0, enable_gqa=False,
+                 dense=False, force_all_active=False, n_slices=8, ws=None):
+    """Causal prefill with inputs and output in page-locked host tensors (q_host, k_host,
+    v_host, head_cls_host in; out_host out), the copies overlapped with the computation in
+    row slices.  q, k, v, head_cls, out are the device buffers it fills and uses (same
+    shapes).  Enqueued on the current stream (two copy streams of its own per device); out_host
+    is valid once the current stream is synchronised."""
+    B, Hq, T, D = q.shape
+    Hkv = k.shape[1]
+    dev = q.device
+    prm = make_params(B, Hq, Hkv, T, D, chunk_size, alpha, gamma, sigma, enable_gqa,
+                      _flags(dense, force_all_active, False))
+    for name, h, d, dt in (("q", q_host, q, torch.bfloat16), ("k", k_host, k, torch.bfloat16),
+                           ("v", v_host, v, torch.bfloat16), ("out", out_host, out, torch.bfloat16)):
+        _need(d, dt, tuple(d.shape), name)
+        if h.shape != d.shape or h.dtype != dt or h.device.type != "cpu" or not h.is_contiguous():
+            raise ValueError(f"{name}_host must be a contiguous CPU {dt} tensor of shape {tuple(d.shape)}")
+    if ws is None:
+        ws = workspace(prefill_workspace_size(prm), dev)
+    if dev not in _copy_streams:
+        _copy_streams[dev] = (torch.cuda.Stream(dev), torch.cuda.Stream(dev))
+    hs, ds = _copy_streams[dev]
+    hc = None if head_cls is None else head_cls
+    _check(lib.dash_prefill_host(ctypes.byref(prm), q_host.data_ptr(), k_host.data_ptr(),
+                                 v_host.data_ptr(),
+                                 None if head_cls_host is None else head_cls_host.data_ptr(),
+                                 out_host.data_ptr(), _ptr(q), _ptr(k), _ptr(v), _ptr(hc), _ptr(out),
+                                 _ptr(ws), ws.numel(), int(n_slices), _stream(dev),
+                                 ctypes.c_void_p(hs.cuda_stream), ctypes.c_void_p(ds.cuda_stream)),
+           "dash_prefill_host")
+    return out_host
 
 
 def stage0(k, head_cls, chunk_size=64, ws=None, summary=None):

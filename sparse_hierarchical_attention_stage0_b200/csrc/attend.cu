@@ -259,6 +259,12 @@ static cudaError_t launch_attend_t(const StageArgs &a, cudaStream_t st) {
 }
 
 cudaError_t launch_attend(const StageArgs &a, cudaStream_t st) {
+    if (a.t_begin != 0 || a.t_end != a.T) {
+        // Row slices: only the 128-key-block kernels take a row range.
+        if (a.vt && a.ignore_routing && attend_pair_supported(a)) return launch_attend_pair(a, st);
+        if (a.vt && attend_fa_supported(a)) return launch_attend_fa(a, st);
+        return cudaErrorNotSupported;
+    }
     // Pairs of SMs share each K/V block between two tiles, so they walk the union of both
     // tiles' chunks: a gain only when every visible chunk is attended anyway (dense, or every
     // chunk forced active); with routing the larger union costs more than the halved copies

@@ -88,7 +88,7 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
 struct FaArgs {
     StageArgs s;
     int RT;              // tokens per tile (128 / G)
-    int n_tiles_bg;      // token tiles per (b, g)
+    int tile0, n_tiles_bg;  // first token tile and token tiles per (b, g) of the row range
     size_t off_bias, off_qbar, off_list;  // dynamic smem offsets (bytes, from the aligned base)
 };
 
@@ -111,11 +111,11 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
     // (b, g)-major, longest tiles first: the CTAs in flight share one (b, g)'s K and V^T in L2
     // (67 MB at T = 128K; both planes at once overflow the 126 MB L2: 3% slower, measured).
     const int tile_rev = blockIdx.x % ta.n_tiles_bg, bgi = blockIdx.x / ta.n_tiles_bg;
-    const int tt = ta.n_tiles_bg - 1 - tile_rev;
+    const int tt = ta.tile0 + ta.n_tiles_bg - 1 - tile_rev;
     const int b = bgi / a.Hkv, g = bgi % a.Hkv;
     const long long bg = bgi;
     const int t0 = tt * RT;
-    const int t_last = min(t0 + RT, a.T) - 1;
+    const int t_last = min(t0 + RT, a.t_end) - 1;
     const int ct_max = t_last / BC;                                     // the tile's diagonal chunk
 
     // ---------------------------------------------------------------- setup
@@ -155,7 +155,7 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                 } else {
                     for (int u = 0; u < RT; ++u) {
                         const int t = t0 + u;
-                        if (t < a.T) word |= a.mask[(bg * a.T + t) * W + w];
+                        if (t < a.t_end) word |= a.mask[(bg * a.T + t) * W + w];
                     }
                 }
                 const int lim = ct_max + 1 - 64 * w;          // bits [0, lim) can be attended
@@ -183,7 +183,7 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
             for (int idx = lane; idx < RT * (D / 8); idx += 32) {
                 const int u = idx / (D / 8), d8 = (idx % (D / 8)) * 8, t = t0 + u;
                 float m[8];
-                if (t < a.T) {
+                if (t < a.t_end) {
                     group_mean8(q + (((long long)b * a.Hq + g * G) * a.T + t) * D + d8,
                                 (long long)a.T * D, G, m);
                 } else {
@@ -212,7 +212,7 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
     const int u_row = row / G;
     const int t_row = t0 + u_row;
     const int h_row = g * G + row % G;
-    const bool row_ok = t_row < a.T;
+    const bool row_ok = t_row < a.t_end;
     __syncthreads();
     const uint32_t tb = sh.tmem_base;
     if (warp >= kWarpSm0 && warp < kWarpTmaV) {
@@ -375,7 +375,7 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                 if (ci < n_chunks && !a.ignore_routing) {
                     const int c = chunk_at(ci), t = t0 + u;
                     const int ctu = t / BC;
-                    if (t >= a.T || c > ctu) {
+                    if (t >= a.t_end || c > ctu) {
                         v = -INFINITY;
                     } else if (c < ctu) {
                         const long long rowi = bg * a.T + t;
@@ -585,7 +585,7 @@ static cudaError_t launch_fa_t(const StageArgs &a, cudaStream_t st) {
     static EncodeFn enc = fa_encode();
     if (!enc || !a.vt) return cudaErrorNotSupported;
     const int BHkv = a.B * a.Hkv;
-    cudaError_t e = launch_vtranspose(a.v, a.vt, BHkv, a.T, 128, st);
+    cudaError_t e = a.vt_ready ? cudaSuccess : launch_vtranspose(a.v, a.vt, BHkv, a.T, 128, st);
     if (e != cudaSuccess) return e;
     CUtensorMap mk, mk128, mvt;
     if (!fa_map(enc, &mk, a.k, a.T, BHkv, 64) || !fa_map(enc, &mk128, a.k, a.T, BHkv, 128))
@@ -605,7 +605,8 @@ static cudaError_t launch_fa_t(const StageArgs &a, cudaStream_t st) {
     FaArgs ta;
     ta.s = a;
     ta.RT = 128 / a.G;
-    ta.n_tiles_bg = (a.T + ta.RT - 1) / ta.RT;
+    ta.tile0 = a.t_begin / ta.RT;
+    ta.n_tiles_bg = (a.t_end + ta.RT - 1) / ta.RT - ta.tile0;
     size_t off = kRingBytes;
     ta.off_bias = off;
     off += (size_t)2 * kBiasBatch * ta.RT * 4;

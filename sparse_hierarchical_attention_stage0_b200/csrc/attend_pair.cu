@@ -157,7 +157,7 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
 struct PrArgs {
     StageArgs s;
     int RT;              // tokens per tile (128 / G)
-    int n_pairs_bg;      // tile pairs per (b, g)
+    int pair0, n_pairs_bg;  // first tile pair and tile pairs per (b, g) of the row range
     size_t off_bias, off_qbar, off_list;  // dynamic smem offsets (bytes, from the aligned base)
 };
 
@@ -184,12 +184,12 @@ k_attend_pair(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     const int pair = blockIdx.x >> 1;
     // (b, g)-major, longest pairs first: the CTAs in flight share one (b, g)'s K and V^T in L2.
     const int pair_rev = pair % ta.n_pairs_bg, bgi = pair / ta.n_pairs_bg;
-    const int pp = ta.n_pairs_bg - 1 - pair_rev;
+    const int pp = ta.pair0 + ta.n_pairs_bg - 1 - pair_rev;
     const int b = bgi / a.Hkv, g = bgi % a.Hkv;
     const long long bg = bgi;
     const int tp0 = pp * 2 * RT;                                        // the pair's first token
     const int t0 = tp0 + (int)rank * RT;                                // this CTA's first token
-    const int t_last = min(tp0 + 2 * RT, a.T) - 1;
+    const int t_last = min(tp0 + 2 * RT, a.t_end) - 1;
     const int ct_max = t_last / BC;                                     // the pair's diagonal chunk
 
     // ---------------------------------------------------------------- setup
@@ -237,7 +237,7 @@ k_attend_pair(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 } else {
                     for (int u = 0; u < 2 * RT; ++u) {
                         const int t = tp0 + u;
-                        if (t < a.T) word |= a.mask[(bg * a.T + t) * W + w];
+                        if (t < a.t_end) word |= a.mask[(bg * a.T + t) * W + w];
                     }
                 }
                 const int lim = ct_max + 1 - 64 * w;          // bits [0, lim) can be attended
@@ -265,7 +265,7 @@ k_attend_pair(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             for (int idx = lane; idx < RT * (D / 8); idx += 32) {
                 const int u = idx / (D / 8), d8 = (idx % (D / 8)) * 8, t = t0 + u;
                 float m[8];
-                if (t < a.T) {
+                if (t < a.t_end) {
                     group_mean8(q + (((long long)b * a.Hq + g * G) * a.T + t) * D + d8,
                                 (long long)a.T * D, G, m);
                 } else {
@@ -295,7 +295,7 @@ k_attend_pair(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
     const int u_row = row / G;
     const int t_row = t0 + u_row;
     const int h_row = g * G + row % G;
-    const bool row_ok = t_row < a.T;
+    const bool row_ok = t_row < a.t_end;
     __syncthreads();
     const uint32_t tb = sh.tmem_base;
     if (warp >= kWarpSm0 && warp < kWarpTmaV) {
@@ -480,7 +480,7 @@ k_attend_pair(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                 if (ci < n_chunks && !a.ignore_routing) {
                     const int c = chunk_at(ci), t = t0 + u;
                     const int ctu = t / BC;
-                    if (t >= a.T || c > ctu) {
+                    if (t >= a.t_end || c > ctu) {
                         v = -INFINITY;
                     } else if (c < ctu) {
                         const long long rowi = bg * a.T + t;
@@ -682,7 +682,7 @@ cudaError_t launch_pair_t(const StageArgs &a, cudaStream_t st) {
     static EncodeFn enc = pr_encode();
     if (!enc || !a.vt) return cudaErrorNotSupported;
     const int BHkv = a.B * a.Hkv;
-    cudaError_t e = launch_vtranspose(a.v, a.vt, BHkv, a.T, 128, st);
+    cudaError_t e = a.vt_ready ? cudaSuccess : launch_vtranspose(a.v, a.vt, BHkv, a.T, 128, st);
     if (e != cudaSuccess) return e;
     // K [B*Hkv][T][128]: box (64 dims, 64 keys).  V^T [B*Hkv][128][T8]: box (64 keys, 72 or
     // 56 dims) for the even and the odd CTA.
@@ -695,8 +695,8 @@ cudaError_t launch_pair_t(const StageArgs &a, cudaStream_t st) {
     PrArgs ta;
     ta.s = a;
     ta.RT = 128 / a.G;
-    const int n_tiles_bg = (a.T + ta.RT - 1) / ta.RT;
-    ta.n_pairs_bg = (n_tiles_bg + 1) / 2;
+    ta.pair0 = a.t_begin / (2 * ta.RT);
+    ta.n_pairs_bg = ((a.t_end + ta.RT - 1) / ta.RT + 1) / 2 - ta.pair0;
     size_t off = kRingBytes;
     ta.off_bias = off;
     off += (size_t)2 * kBiasBatch * ta.RT * 4;

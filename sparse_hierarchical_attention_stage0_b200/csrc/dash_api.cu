@@ -1,6 +1,7 @@
 // dash_api.cu -- the C ABI declared in include/dash.h: host-side argument checks, workspace
 // carving and stream-ordered launches.  Nothing here allocates device memory or keeps
 // global state; every failure is reported before the first launch of a call.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 
@@ -87,6 +88,9 @@ StageArgs stage_args(const dash_params_t *p, const Shape &s) {
     a.rc = route_consts(p);
     a.qk_scale2 = (float)(1.4426950408889634 / std::sqrt((double)s.D));
     a.ignore_routing = (p->flags & (DASH_FLAG_DENSE | DASH_FLAG_FORCE_ALL_ACTIVE)) ? 1 : 0;
+    a.t_begin = 0;
+    a.t_end = s.T;
+    a.vt_ready = 0;
     return a;
 }
 
@@ -195,6 +199,116 @@ dash_status_t dash_prefill(const dash_params_t *p, const void *q, const void *k,
         if ((rc = from_cuda(launch_route(a, st))) != DASH_OK) return rc;
     }
     return from_cuda(launch_attend(a, st));
+}
+
+dash_status_t dash_prefill_host(const dash_params_t *p, const void *q_host, const void *k_host,
+                                const void *v_host, const float *head_cls_host, void *out_host,
+                                void *q, void *k, void *v, float *head_cls, void *out, void *ws,
+                                size_t ws_bytes, int n_slices, void *stream, void *h2d_stream,
+                                void *d2h_stream) {
+    Shape s;
+    dash_status_t rc = check_params(p, &s);
+    if (rc != DASH_OK) return rc;
+    const bool dense = (p->flags & DASH_FLAG_DENSE) != 0;
+    if (!q_host || !k_host || !v_host || !out_host || (!dense && !head_cls_host) || !q || !k ||
+        !v || !out || (!dense && !head_cls) || !ws || n_slices < 1)
+        return DASH_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(head_cls) ||
+        (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return DASH_ERR_INVALID_ARGUMENT;
+    if (!dense && route_rows_per_cta(s.C, s.D) == 0) return DASH_ERR_UNSUPPORTED;
+    if (ws_bytes < dash_prefill_workspace_size(p)) return DASH_ERR_WORKSPACE_TOO_SMALL;
+
+    unsigned char *w = static_cast<unsigned char *>(ws);
+    StageArgs a = stage_args(p, s);
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.head_cls = head_cls;
+    a.out = out;
+    a.status = reinterpret_cast<uint32_t *>(w);
+    size_t off = kStatusBytes;
+    a.tau = reinterpret_cast<float *>(w + off);
+    off += bytes_tau(s);
+    if (!dense) {
+        a.summary = reinterpret_cast<float *>(w + off);
+        off += bytes_summary(s);
+        a.mask = reinterpret_cast<uint64_t *>(w + off);
+        off += bytes_mask(s);
+    }
+    const size_t vt = bytes_vt(s);
+    if (vt) a.vt = w + off;
+    // Row slices only where the Stage 2 kernel takes a row range; each slice a multiple of
+    // 128 rows (the last one ragged).
+    const bool sliceable = a.vt && (a.ignore_routing ? (attend_pair_supported(a) || attend_fa_supported(a))
+                                                     : attend_fa_supported(a));
+    constexpr int kMaxSlices = 64;
+    const int want = std::min(n_slices, kMaxSlices);
+    int rows = s.T;
+    if (sliceable && want > 1) rows = ((s.T + want - 1) / want + 127) / 128 * 128;
+    const int n = (s.T + rows - 1) / rows;                  // <= want
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaStream_t hs = static_cast<cudaStream_t>(h2d_stream);
+    cudaStream_t ds = static_cast<cudaStream_t>(d2h_stream);
+    const size_t row_bytes = (size_t)s.D * 2;
+    const size_t plane = (size_t)s.T * row_bytes;          // one (b, h) plane of q or out
+    const size_t kv_bytes = (size_t)s.B * s.Hkv * plane;
+    const int n_ev = 2 * n + 3;
+    cudaEvent_t ev[2 * kMaxSlices + 3];
+    int made = 0;
+    cudaError_t e = cudaSuccess;
+    for (; made < n_ev && e == cudaSuccess; ++made) e = cudaEventCreateWithFlags(&ev[made], cudaEventDisableTiming);
+    if (e != cudaSuccess) --made;
+    cudaEvent_t &e_kv = ev[0], &e_done = ev[1], &e_start = ev[2];
+    auto e_q = [&](int i) -> cudaEvent_t & { return ev[3 + i]; };
+    auto e_o = [&](int i) -> cudaEvent_t & { return ev[3 + n + i]; };
+    auto ok = [&](cudaError_t r) { if (e == cudaSuccess) e = r; return e == cudaSuccess; };
+    // Host -> device: head_cls, K and V (Stage 0 and every slice need all keys), then q slice
+    // by slice.  Compute: Stage 0, then Stages 1-2 of slice i once its q has landed.
+    // Device -> host: out of slice i once it is computed.
+    if (e == cudaSuccess) {
+        // Both copy streams start after the work already queued on the compute stream (which
+        // may still use these buffers).
+        ok(cudaEventRecord(e_start, st));
+        ok(cudaStreamWaitEvent(hs, e_start, 0));
+        ok(cudaStreamWaitEvent(ds, e_start, 0));
+        if (!dense) ok(cudaMemcpyAsync(head_cls, head_cls_host, (size_t)s.Hkv * s.D * 4, cudaMemcpyHostToDevice, hs));
+        ok(cudaMemcpyAsync(k, k_host, kv_bytes, cudaMemcpyHostToDevice, hs));
+        ok(cudaMemcpyAsync(v, v_host, kv_bytes, cudaMemcpyHostToDevice, hs));
+        ok(cudaEventRecord(e_kv, hs));
+        for (int i = 0; i < n; ++i) {
+            const size_t t0 = (size_t)i * rows, tr = (size_t)std::min(s.T, (i + 1) * rows) - t0;
+            ok(cudaMemcpy2DAsync(static_cast<unsigned char *>(q) + t0 * row_bytes, plane,
+                                 static_cast<const unsigned char *>(q_host) + t0 * row_bytes, plane,
+                                 tr * row_bytes, (size_t)s.B * s.Hq, cudaMemcpyHostToDevice, hs));
+            ok(cudaEventRecord(e_q(i), hs));
+        }
+        ok(cudaMemsetAsync(ws, 0, sizeof(uint32_t), st));
+        ok(cudaStreamWaitEvent(st, e_kv, 0));
+        if (!dense) ok(launch_stage0(a, nullptr, 0, st));
+        for (int i = 0; i < n && e == cudaSuccess; ++i) {
+            a.t_begin = i * rows;
+            a.t_end = std::min(s.T, (i + 1) * rows);
+            a.vt_ready = i > 0;
+            ok(cudaStreamWaitEvent(st, e_q(i), 0));
+            if (!dense) ok(launch_route(a, st));
+            ok(launch_attend(a, st));
+            ok(cudaEventRecord(e_o(i), st));
+        }
+        for (int i = 0; i < n && e == cudaSuccess; ++i) {
+            const size_t t0 = (size_t)i * rows, tr = (size_t)std::min(s.T, (i + 1) * rows) - t0;
+            ok(cudaStreamWaitEvent(ds, e_o(i), 0));
+            ok(cudaMemcpy2DAsync(static_cast<unsigned char *>(out_host) + t0 * row_bytes, plane,
+                                 static_cast<const unsigned char *>(out) + t0 * row_bytes, plane,
+                                 tr * row_bytes, (size_t)s.B * s.Hq, cudaMemcpyDeviceToHost, ds));
+        }
+        // The compute stream ends after the last copy back, so synchronising it covers the call.
+        ok(cudaEventRecord(e_done, ds));
+        ok(cudaStreamWaitEvent(st, e_done, 0));
+    }
+    for (int i = 0; i < made; ++i) cudaEventDestroy(ev[i]);   // released once complete
+    return from_cuda(e);
 }
 
 dash_status_t dash_stage0(const dash_params_t *p, const void *k, const float *head_cls,

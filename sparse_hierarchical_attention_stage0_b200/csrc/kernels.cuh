@@ -24,6 +24,9 @@ struct StageArgs {
     RouteConsts rc;
     float qk_scale2;          // log2(e) / sqrt(D)
     int ignore_routing;       // DENSE or FORCE_ALL_ACTIVE: attend every chunk, bias 0
+    int t_begin, t_end;       // Stages 1-2 compute rows [t_begin, t_end) (t_begin % 128 == 0);
+                              // T stays the row stride of q, tau, mask, p and out
+    int vt_ready;             // V^T scratch already holds the transpose of V (a later row slice)
     uint32_t *status;
 };
 

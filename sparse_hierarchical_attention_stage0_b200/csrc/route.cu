@@ -40,7 +40,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(StageArgs a) {
     float *xs = sm + RT * D;        // [RT][xstride]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bg = blockIdx.y, b = bg / a.Hkv, g = bg % a.Hkv;
-    const int t0 = blockIdx.x * RT;
+    const int t0 = a.t_begin + blockIdx.x * RT;
     const int ct = t0 / a.Bc;                     // every row of the tile shares c_t
     const int n = ct;                             // routable chunks
     const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(a.q);
@@ -49,7 +49,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(StageArgs a) {
     for (int idx = threadIdx.x; idx < RT * (D / 8); idx += kRouteThreads) {
         const int r = idx / (D / 8), d8 = (idx % (D / 8)) * 8, t = t0 + r;
         float m[8];
-        if (t < a.T) {
+        if (t < a.t_end) {
             group_mean8(q + ((long long)(b * a.Hq + g * a.G) * a.T + t) * D + d8, hstride, a.G, m);
         } else {
 #pragma unroll
@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(StageArgs a) {
 
     for (int r = warp; r < RT; r += kRouteThreads / 32) {
         const int t = t0 + r;
-        if (t >= a.T) break;
+        if (t >= a.t_end) break;
         const long long row = (long long)bg * a.T + t;
         const float *x = xs + r * xstride;
         float tau = n > 0 ? warp_entmax_tau(x, n, a.rc, a.status) : __int_as_float(0x7fc00000);
@@ -145,7 +145,7 @@ static cudaError_t launch_route_t(const StageArgs &a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((a.T + RT - 1) / RT, a.B * a.Hkv);
+    dim3 grid((a.t_end - a.t_begin + RT - 1) / RT, a.B * a.Hkv);
     kern<<<grid, kRouteThreads, smem, st>>>(a);
     return cudaGetLastError();
 }

@@ -117,6 +117,23 @@ def test_prefill_rejects_bad_pointers_and_small_workspace(dash):
              None) == 1                                             # dense + routing output
 
 
+def test_prefill_host_rejects_bad_arguments_before_any_copy(dash):
+    prm = _p(dash)
+    f = dash.lib.dash_prefill_host
+    big = 1 << 40
+    h = [FAKE] * 5                                   # q, k, v, head_cls, out on the host
+    d = [FAKE] * 5                                   # their device buffers
+    assert f(ctypes.byref(prm), *h, *d, FAKE, big, 0, None, None, None) == 1  # n_slices < 1
+    assert f(ctypes.byref(prm), None, *h[1:], *d, FAKE, big, 8, None, None, None) == 1
+    assert f(ctypes.byref(prm), *h[:4], None, *d, FAKE, big, 8, None, None, None) == 1
+    assert f(ctypes.byref(prm), *h, FAKE + 8, *d[1:], FAKE, big, 8, None, None, None) == 1
+    assert f(ctypes.byref(prm), *h, *d, FAKE, dash.prefill_workspace_size(prm) - 1, 8,
+             None, None, None) == 3
+    dense = _p(dash, flags=1)                        # no head_cls needed in dense mode
+    assert f(ctypes.byref(dense), *h[:3], None, h[4], *d[:3], None, d[4], FAKE, big, 0,
+             None, None, None) == 1
+
+
 def test_decode_and_cache_reject_bad_arguments(dash):
     prm = _p(dash, seq_len=65792)
     d = dash.lib.dash_decode

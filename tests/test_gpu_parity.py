@@ -198,6 +198,29 @@ def test_prefill_batch2_matches_oracle(dash):
     assert dash.read_device_status(res["ws"]) == 0
 
 
+@pytest.mark.parametrize("G,D,Bc,T,dense,n", [(16, 128, 64, 1100, False, 4), (8, 128, 128, 1505, True, 3),
+                                              (8, 64, 64, 640, False, 4), (32, 128, 64, 700, False, 64)])
+def test_prefill_host_equals_prefill(dash, G, D, Bc, T, dense, n):
+    """The sliced prefill from host memory gives dash_prefill's output bit for bit (row slices
+    of 128-row multiples; D = 64 runs as one slice; more slices asked than 128-row blocks)."""
+    Hkv = 2 if G <= 16 else 1
+    q, k, v, hc = make_prefill(_cfg(1, G * Hkv, Hkv, T, D, Bc, 1.5, seed=40 + G))
+    qd, kd, vd, hcd = _to(q, k, v, hc)
+    ref = dash.prefill(qd, kd, vd, None if dense else hcd, Bc, 1.5, enable_gqa=True, dense=dense)
+    torch.cuda.synchronize()
+    hq, hk, hv, hhc = (x.contiguous().pin_memory() for x in (q, k, v, hc))
+    ho = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    bq, bk, bv, bhc, bo = (torch.empty_like(x) for x in (qd, kd, vd, hcd, qd))
+    prm = dash.make_params(1, G * Hkv, Hkv, T, D, Bc, 1.5, enable_gqa=True, flags=1 if dense else 0)
+    ws = dash.workspace(dash.prefill_workspace_size(prm), qd.device)
+    dash.prefill_host(hq, hk, hv, None if dense else hhc, ho, bq, bk, bv, None if dense else bhc, bo,
+                      Bc, 1.5, enable_gqa=True, dense=dense, n_slices=n, ws=ws)
+    torch.cuda.current_stream().synchronize()
+    assert dash.read_device_status(ws) == 0
+    assert torch.equal(ho, ref.cpu())
+    assert torch.equal(bo, ref)
+
+
 def test_inactive_chunks_do_not_touch_the_output(dash):
     """Rewriting V inside chunks that none of the last query chunk's 64 tokens routes to
     leaves those tokens' outputs identical to the bit."""
