@@ -10,8 +10,9 @@
 //   1. qbar[r] = mean of the G query heads of group g at row t0 + r     (shared memory)
 //   2. x[r][c] = (qbar[r] . summary[c]) * (alpha-1) gamma / sqrt(D) for every routable
 //      chunk c < c_t: 4 lanes per chunk, each owning an interleaved quarter of d (coalesced
-//      64-byte reads per chunk), RT row accumulators in registers, qbar broadcast from
-//      shared memory, slices combined with route_dot's fixed order
+//      64-byte reads per chunk), two chunks per lane, RT row accumulators per chunk in
+//      registers, qbar from shared memory (each load feeds both chunks), slices combined with
+//      route_dot's fixed order
 //   3. one warp per row solves tau (warp_entmax_tau) and emits the mask words by ballot,
 //      tau, and optionally the dense p row.
 // No top-k list and no per-row index list is ever written.
@@ -61,45 +62,61 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(StageArgs a) {
     __syncthreads();
 
     // Scores: 4 lanes per chunk (lane = 4*cc + k owns float4 groups k, k+4, ... of chunk cc),
-    // 8 chunks per warp and step; the RT rows' partial dots stay in registers.  The slice sums
+    // two chunks per lane (cc and cc + 8), 16 chunks per warp and step; the RT rows' partial
+    // dots stay in registers, and every query float4 loaded from shared memory feeds both
+    // chunks (8 FMAs per load: the score loop is bound by the load/store pipe).  The slice sums
     // are combined with the order of route_dot: (p0 + p1) + (p2 + p3).
     const float scale = a.rc.kind == 0 ? a.rc.sscale : a.rc.xscale;
     const float *sumg = a.summary + (long long)bg * a.Cf * D;
     const int kslice = lane & 3, cc = lane >> 2;
-    constexpr int kStep = (kRouteThreads / 32) * 8;       // chunks per CTA-wide step
-    for (int cbase = warp * 8; cbase < n; cbase += kStep) {
-        const int c = cbase + cc;
-        float4 cur[D / 16];                       // all loads of the slice in flight at once
+    constexpr int kStep = (kRouteThreads / 32) * 16;      // chunks per CTA-wide step
+    for (int cbase = warp * 16; cbase < n; cbase += kStep) {
+        const int c = cbase + cc, c2 = c + 8;
+        float4 cur[D / 16], cur2[D / 16];         // all loads of both slices in flight at once
         {
             const float4 *s4 = reinterpret_cast<const float4 *>(sumg + (long long)min(c, n - 1) * D);
+            const float4 *t4 = reinterpret_cast<const float4 *>(sumg + (long long)min(c2, n - 1) * D);
 #pragma unroll
-            for (int i = 0; i < D / 16; ++i) cur[i] = __ldg(s4 + 4 * i + kslice);
+            for (int i = 0; i < D / 16; ++i) {
+                cur[i] = __ldg(s4 + 4 * i + kslice);
+                cur2[i] = __ldg(t4 + 4 * i + kslice);
+            }
         }
-        float acc[RT];
+        float acc[RT], acc2[RT];
 #pragma unroll
-        for (int r = 0; r < RT; ++r) acc[r] = 0.f;
+        for (int r = 0; r < RT; ++r) acc[r] = acc2[r] = 0.f;
 #pragma unroll
         for (int i = 0; i < D / 16; ++i) {
-            const float4 sv = cur[i];
+            const float4 sv = cur[i], tv = cur2[i];
 #pragma unroll
             for (int r = 0; r < RT; ++r) {
                 const float4 qq = reinterpret_cast<const float4 *>(qbar + r * D)[4 * i + kslice];
                 acc[r] = fmaf(qq.x, sv.x, acc[r]);
+                acc2[r] = fmaf(qq.x, tv.x, acc2[r]);
                 acc[r] = fmaf(qq.y, sv.y, acc[r]);
+                acc2[r] = fmaf(qq.y, tv.y, acc2[r]);
                 acc[r] = fmaf(qq.z, sv.z, acc[r]);
+                acc2[r] = fmaf(qq.z, tv.z, acc2[r]);
                 acc[r] = fmaf(qq.w, sv.w, acc[r]);
+                acc2[r] = fmaf(qq.w, tv.w, acc2[r]);
             }
         }
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
-            float v = acc[r];
+            float v = acc[r], w = acc2[r];
             v = v + __shfl_xor_sync(kFull, v, 1);
+            w = w + __shfl_xor_sync(kFull, w, 1);
             v = v + __shfl_xor_sync(kFull, v, 2);
+            w = w + __shfl_xor_sync(kFull, w, 2);
             acc[r] = v;
+            acc2[r] = w;
         }
-        if (kslice == 0 && c < n) {
+        if (kslice == 0) {
 #pragma unroll
-            for (int r = 0; r < RT; ++r) xs[r * xstride + c] = __fmul_rn(acc[r], scale);
+            for (int r = 0; r < RT; ++r) {
+                if (c < n) xs[r * xstride + c] = __fmul_rn(acc[r], scale);
+                if (c2 < n) xs[r * xstride + c2] = __fmul_rn(acc2[r], scale);
+            }
         }
     }
     __syncthreads();
