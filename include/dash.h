@@ -8,7 +8,8 @@
  *   Technische Zusammenfassung:
  *     "Stufe 0: Lokale Chunk-Zusammenfassung"   -> dash_stage0, dash_update_chunk_cache
  *     "Stufe 1: Entmax-Chunk-Routing"            -> dash_route
- *     "Stufe 2: Prior-induzierte spaerliche Softmax" -> dash_attend
+ *     "Stufe 2: Prior-induzierte spaerliche Softmax" -> dash_attend; its causality (row t
+ *     reads keys <= t) lets dash_prefill_host overlap host copies with row slices
  *   aiexpert.news "DashAttention alcanca 75% de esparsidade ...", interface paragraph:
  *     queries, keys, values, a per-head head_cls vector, chunk_size, estimate_diagonal,
  *     enable_gqa, optional active_blocks mask -> dash_params_t, dash_prefill.
