@@ -171,6 +171,24 @@ def stage01_bytes(cfg):
     return dict(stage0=k_bytes + summ, stage1=q_bytes + summ + mask + tau)
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The maximum of x over the ranks of the default process group (x itself when there is
+    none): every multi-rank time is the slowest rank's.  device is where the reduction runs
+    (CUDA for NCCL, CPU for gloo)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, tokens_per_rank_step: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput of `world` replicas that each processed `steps` steps of
+    `tokens_per_rank_step` tokens in at most max_ms milliseconds."""
+    return world * tokens_per_rank_step * steps / (max_ms / 1e3)
+
+
 def traffic_for(kernel, cfg_name):
     """Per-launch DRAM bytes from the committed ncu summary, if it was taken on the current
     kernel source (else None)."""
@@ -398,13 +416,10 @@ def main():
     with ClockSampler(local) as clk:
         step_ms = timed(prefill, args.steps, stream, flush)
     torch.cuda.synchronize()
-    total_ms = sum(step_ms)
+    total_ms = max_over_ranks(sum(step_ms), dev)
     if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
         torch.distributed.barrier()
-    value = world * B * T * args.steps / (total_ms / 1e3)
+    value = job_tokens_per_s(world, B * T, args.steps, total_ms)
 
     # Per-stage times through the stage entry points (same kernels as dash_prefill).
     summ = torch.empty(B, Hkv, T // Bc, D, device=dev)
@@ -457,7 +472,9 @@ def main():
                           enable_gqa=True, n_slices=E2E_SLICES, ws=ws)
 
     e2e()
-    e2e_ms = statistics.mean(timed(e2e, args.steps, stream, flush))
+    if world > 1:
+        torch.distributed.barrier()
+    e2e_ms = max_over_ranks(statistics.mean(timed(e2e, args.steps, stream, flush)), dev)
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hhc))
     d2h = ho.numel() * ho.element_size()
 
@@ -495,7 +512,7 @@ def main():
                              "unit": "GB/s", "frac": s01_gbs / pk["hbm_gbs"],
                              "frac_of_8tbs_nominal": s01_gbs / 8000.0,
                              "bytes": sb["stage0"] + sb["stage1"]},
-        "e2e": {"value": world * B * T / (e2e_ms / 1e3), "unit": "tokens/s",
+        "e2e": {"value": job_tokens_per_s(world, B * T, 1, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "call": f"dash_prefill_host, {E2E_SLICES} row slices"},
         "gpu_launches": launches_per_step * args.steps,
