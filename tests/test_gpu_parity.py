@@ -119,6 +119,19 @@ def test_prefill_matches_oracle(dash, alpha, G, D, Bc, T):
     assert dash.read_device_status(res["ws"]) == 0
 
 
+@pytest.mark.parametrize("alpha,sigma", [(1.5, 0.5), (2.0, 2.0), (1.0, 0.25)])
+def test_prefill_prior_strength_sigma(dash, alpha, sigma):
+    """sigma scales the log-prior bias of the routed chunks (the prior strength the pages
+    name for Stage 2; reading C10)."""
+    q, k, v, hc = make_prefill(_cfg(1, 32, 2, 1100, 128, 64, alpha, seed=50))
+    res = dash.prefill(*_to(q, k, v, hc), chunk_size=64, alpha=alpha, sigma=sigma,
+                       enable_gqa=True, return_active_blocks=True)
+    torch.cuda.synchronize()
+    assert dash.read_device_status(res["ws"]) == 0
+    ref = oracle.prefill(q, k, v, hc, 64, alpha, sigma=sigma)
+    check_output(res["out"].cpu().float().numpy(), ref["O"], tag=f"a={alpha} sigma={sigma}")
+
+
 @pytest.mark.parametrize("G,Bc,T", [(16, 64, 2100 + 37), (8, 128, 1500 + 3)])
 def test_attend_without_vt_scratch_takes_the_tile_kernel(dash, G, Bc, T):
     """dash_attend with only the 256-byte status word cannot hold V^T, so Stage 2 runs on the
