@@ -80,7 +80,12 @@ enum {
     DASH_FLAG_FORCE_ALL_ACTIVE = 2,
     /* Reserved: the diagonal correction of the entmax normalisation ("estimate_diagonal").
      * The pages give no formula; requesting it returns DASH_ERR_UNSUPPORTED. */
-    DASH_FLAG_ESTIMATE_DIAGONAL = 4
+    DASH_FLAG_ESTIMATE_DIAGONAL = 4,
+    /* Test hook (fault injection without a GPU fault): caps the entmax Newton solve of the
+     * routing at one iteration, so every row that needs more reports DASH_ERR_DEVICE_TIMEOUT
+     * through the device status word, the way a row that hit the real cap would.  The
+     * outputs of such a call are not meaningful. */
+    DASH_FLAG_TEST_NEWTON_CAP = 8
 };
 
 typedef struct {

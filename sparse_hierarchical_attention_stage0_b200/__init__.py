@@ -35,6 +35,7 @@ STATUS_NAMES = {0: "DASH_OK", 1: "DASH_ERR_INVALID_ARGUMENT", 2: "DASH_ERR_UNSUP
 FLAG_DENSE = 1
 FLAG_FORCE_ALL_ACTIVE = 2
 FLAG_ESTIMATE_DIAGONAL = 4
+FLAG_TEST_NEWTON_CAP = 8          # test hook: Newton solve capped at one iteration
 
 # Every symbol include/dash.h declares.
 EXPORTS = ("dash_prefill_workspace_size", "dash_prefill", "dash_prefill_host", "dash_stage0", "dash_route",

@@ -31,7 +31,7 @@ dash_status_t check_params(const dash_params_t *p, Shape *s) {
     if (!std::isfinite(p->alpha) || p->alpha < 1.f) return DASH_ERR_INVALID_ARGUMENT;
     if (!std::isfinite(p->gamma) || !(p->gamma > 0.f)) return DASH_ERR_INVALID_ARGUMENT;
     if (!std::isfinite(p->sigma) || p->sigma < 0.f) return DASH_ERR_INVALID_ARGUMENT;
-    if (p->flags & ~7u) return DASH_ERR_INVALID_ARGUMENT;
+    if (p->flags & ~15u) return DASH_ERR_INVALID_ARGUMENT;
     if (p->flags & DASH_FLAG_ESTIMATE_DIAGONAL) return DASH_ERR_UNSUPPORTED;
     if (p->head_dim != 64 && p->head_dim != 128) return DASH_ERR_UNSUPPORTED;
     if (p->chunk_size != 64 && p->chunk_size != 128) return DASH_ERR_UNSUPPORTED;
@@ -70,6 +70,7 @@ RouteConsts route_consts(const dash_params_t *p) {
         rc.bscale2 = (float)(sg / (a - 1.0));
     }
     rc.sigma2 = (float)(sg * 1.4426950408889634);
+    rc.newton_cap = (p->flags & DASH_FLAG_TEST_NEWTON_CAP) ? 1 : kNewtonCap;
     return rc;
 }
 

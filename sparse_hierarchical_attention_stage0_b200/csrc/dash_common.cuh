@@ -223,6 +223,7 @@ struct RouteConsts {
     float bscale2;    // log2 of the prior: bias2 = bscale2 * log2(m) with bscale2 = sigma*beta
     float sigma2;     // sigma * log2(e) (alpha = 1: bias2 = sigma2 * (s - lse))
     int kind;         // 0: softmax (alpha = 1), 1: alpha = 1.5, 2: alpha = 2, 3: other alpha
+    int newton_cap;   // iteration cap of the Newton solve (kNewtonCap; 1 under the test hook)
 };
 
 // m^beta for the entmax probability of margin m > 0.
@@ -276,7 +277,7 @@ static __device__ __noinline__ float entmax_tau_k(const float *xs, int n, const 
     if (KIND != 3 || beta >= 1.f) {
         tau = mx - 1.f;
         int it = 0;
-        for (; it < kNewtonCap; ++it) {
+        for (; it < rc.newton_cap; ++it) {
             const float t = tau;
             const float f = warp_sum(lane_pass(xs, n, lane, [t, beta](float x) {
                 const float m = x - t;
@@ -293,7 +294,7 @@ static __device__ __noinline__ float entmax_tau_k(const float *xs, int n, const 
             tau = nt;
             if (step <= 1e-7f * fmaxf(1.f, fabsf(tau))) break;
         }
-        if (it == kNewtonCap) report(status, DASH_ERR_DEVICE_TIMEOUT);
+        if (it == rc.newton_cap) report(status, DASH_ERR_DEVICE_TIMEOUT);
     } else {
         float lo = mx - 1.f, hi = mx - powf((float)n, 1.f - rc.alpha);
         for (int it = 0; it < 40; ++it) {

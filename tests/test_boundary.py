@@ -98,6 +98,11 @@ def test_prefill_rejects_bad_parameters_before_launch(dash, kw, code):
     assert rc == code
 
 
+def test_newton_cap_test_flag_is_accepted(dash):
+    prm = _p(dash, flags=dash.FLAG_TEST_NEWTON_CAP)
+    assert dash.prefill_workspace_size(prm) == dash.prefill_workspace_size(_p(dash))
+
+
 def test_prefill_rejects_bad_pointers_and_small_workspace(dash):
     prm = _p(dash)
     f = dash.lib.dash_prefill

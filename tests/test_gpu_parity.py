@@ -1,5 +1,6 @@
 """GPU parity of every stage against the fp64 oracle, through the C ABI (via the binding),
 at sizes the oracle finishes in seconds that still span several tiles and a ragged tail."""
+import ctypes
 import json
 import os
 from dataclasses import replace
@@ -355,6 +356,27 @@ def test_decode_matches_oracle_and_prefill_rows(dash, G, D, Bc):
         t = lens[b] - 1
         check_routing(bits[b][:, None], dec["p"][b][:, None].cpu().double().numpy(),
                       ref["p"][b][:, None], ref["m"][b][:, None], [t], Bc, 1.5, tag="decode")
+
+
+def test_newton_cap_hook_reports_device_timeout(dash):
+    """Fault injection without a GPU fault: the test flag caps the entmax Newton solve at one
+    iteration.  With i.i.d. inputs every row's scaled scores lie within 1 of their maximum, so
+    rows need a second step and report DASH_ERR_DEVICE_TIMEOUT through the status word; the
+    same call without the flag then succeeds (the context stays usable)."""
+    T, D, Bc, Hkv, Hq = 1100, 128, 64, 2, 32
+    q, k, v, hc = make_prefill(_cfg(1, Hq, Hkv, T, D, Bc, 1.5, planted=False, seed=60))
+    qd, kd, hcd = _to(q, k, hc)
+    summ = dash.stage0(kd, hcd, Bc)
+    C = (T + Bc - 1) // Bc
+    tau = torch.empty(1, Hkv, T, device=dev)
+    mask = torch.empty(1, Hkv, T, (C + 63) // 64, dtype=torch.int64, device=dev)
+    ws = dash.workspace(256, qd.device)
+    for flags, want in ((dash.FLAG_TEST_NEWTON_CAP, 5), (0, 0)):
+        prm = dash.make_params(1, Hq, Hkv, T, D, Bc, 1.5, enable_gqa=True, flags=flags)
+        rc = dash.lib.dash_route(ctypes.byref(prm), dash._ptr(qd), dash._ptr(summ), dash._ptr(tau),
+                                 None, dash._ptr(mask), dash._ptr(ws), 256, dash._stream(qd.device))
+        assert rc == 0
+        assert dash.read_device_status(ws) == want, (flags, dash.read_device_status(ws))
 
 
 def test_decode_reports_bad_seq_len(dash):
