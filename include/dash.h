@@ -85,7 +85,12 @@ enum {
      * routing at one iteration, so every row that needs more reports DASH_ERR_DEVICE_TIMEOUT
      * through the device status word, the way a row that hit the real cap would.  The
      * outputs of such a call are not meaningful. */
-    DASH_FLAG_TEST_NEWTON_CAP = 8
+    DASH_FLAG_TEST_NEWTON_CAP = 8,
+    /* Test hook (fault injection without a GPU fault): Stage 0 issues no chunk copy, so the
+     * bounded wait on its barrier runs out after 2 s and reports DASH_ERR_DEVICE_TIMEOUT;
+     * the CTA then returns with nothing in flight and the context stays usable.  Meant for
+     * a few chunks (every CTA of the grid waits its 2 s); the outputs are not meaningful. */
+    DASH_FLAG_TEST_STALL_WAIT = 16
 };
 
 typedef struct {

@@ -36,6 +36,7 @@ FLAG_DENSE = 1
 FLAG_FORCE_ALL_ACTIVE = 2
 FLAG_ESTIMATE_DIAGONAL = 4
 FLAG_TEST_NEWTON_CAP = 8          # test hook: Newton solve capped at one iteration
+FLAG_TEST_STALL_WAIT = 16         # test hook: Stage 0's bounded copy wait runs out
 
 # Every symbol include/dash.h declares.
 EXPORTS = ("dash_prefill_workspace_size", "dash_prefill", "dash_prefill_host", "dash_stage0", "dash_route",

@@ -31,7 +31,7 @@ dash_status_t check_params(const dash_params_t *p, Shape *s) {
     if (!std::isfinite(p->alpha) || p->alpha < 1.f) return DASH_ERR_INVALID_ARGUMENT;
     if (!std::isfinite(p->gamma) || !(p->gamma > 0.f)) return DASH_ERR_INVALID_ARGUMENT;
     if (!std::isfinite(p->sigma) || p->sigma < 0.f) return DASH_ERR_INVALID_ARGUMENT;
-    if (p->flags & ~15u) return DASH_ERR_INVALID_ARGUMENT;
+    if (p->flags & ~31u) return DASH_ERR_INVALID_ARGUMENT;
     if (p->flags & DASH_FLAG_ESTIMATE_DIAGONAL) return DASH_ERR_UNSUPPORTED;
     if (p->head_dim != 64 && p->head_dim != 128) return DASH_ERR_UNSUPPORTED;
     if (p->chunk_size != 64 && p->chunk_size != 128) return DASH_ERR_UNSUPPORTED;
@@ -92,6 +92,7 @@ StageArgs stage_args(const dash_params_t *p, const Shape &s) {
     a.t_begin = 0;
     a.t_end = s.T;
     a.vt_ready = 0;
+    a.test_stall = (p->flags & DASH_FLAG_TEST_STALL_WAIT) ? 1 : 0;
     return a;
 }
 

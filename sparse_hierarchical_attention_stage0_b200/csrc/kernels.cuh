@@ -27,6 +27,7 @@ struct StageArgs {
     int t_begin, t_end;       // Stages 1-2 compute rows [t_begin, t_end) (t_begin % 128 == 0);
                               // T stays the row stride of q, tau, mask, p and out
     int vt_ready;             // V^T scratch already holds the transpose of V (a later row slice)
+    int test_stall;           // test hook: Stage 0's chunk-copy wait runs out (DASH_FLAG_TEST_STALL_WAIT)
     uint32_t *status;
 };
 

@@ -72,7 +72,7 @@ template <int D, int BC>
 __global__ void __launch_bounds__(kStage0Warps * 32)
 k_stage0(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ head_cls,
          float *__restrict__ summary, int B, int Hkv, int T, int Cf, const int32_t *seq_lens,
-         int n_recent, uint32_t *status) {
+         int n_recent, uint32_t *status, int test_stall) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t bars[kStage0Warps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -104,13 +104,15 @@ k_stage0(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ head_cls
         fence_mbar_init();
     }
     __syncwarp();
-    if (lane == 0) {
+    // Test hook: with test_stall nothing arrives on the barrier (no copy is issued), so the
+    // bounded wait below runs out and reports DASH_ERR_DEVICE_TIMEOUT.
+    if (lane == 0 && !test_stall) {
         mbar_arrive_expect_tx(&bars[warp], kBytes);
         bulk_g2s(ks, src, kBytes, &bars[warp]);
     }
     if (!__all_sync(kFull, mbar_wait_bounded(&bars[warp], 0))) {   // warp-uniform outcome
         if (lane == 0) report(status, DASH_ERR_DEVICE_TIMEOUT);
-        mbar_wait_bounded(&bars[warp], 0);   // give the copy in flight one more bounded wait
+        if (!test_stall) mbar_wait_bounded(&bars[warp], 0);   // one more bounded wait for the copy
         return;
     }
     summarize_chunk_warp<D, BC>(ks, head_cls + (size_t)g * D,
@@ -131,7 +133,7 @@ static cudaError_t launch_stage0_t(const StageArgs &a, const int32_t *seq_lens, 
     unsigned grid = (unsigned)((units + kStage0Warps - 1) / kStage0Warps);
     kern<<<grid, kStage0Warps * 32, smem, st>>>(
         reinterpret_cast<const __nv_bfloat16 *>(a.k), a.head_cls, a.summary, a.B, a.Hkv, a.T,
-        a.Cf, seq_lens, n_recent, a.status);
+        a.Cf, seq_lens, n_recent, a.status, a.test_stall);
     return cudaGetLastError();
 }
 

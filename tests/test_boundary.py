@@ -98,9 +98,10 @@ def test_prefill_rejects_bad_parameters_before_launch(dash, kw, code):
     assert rc == code
 
 
-def test_newton_cap_test_flag_is_accepted(dash):
-    prm = _p(dash, flags=dash.FLAG_TEST_NEWTON_CAP)
-    assert dash.prefill_workspace_size(prm) == dash.prefill_workspace_size(_p(dash))
+def test_test_hook_flags_are_accepted(dash):
+    for f in (dash.FLAG_TEST_NEWTON_CAP, dash.FLAG_TEST_STALL_WAIT):
+        prm = _p(dash, flags=f)
+        assert dash.prefill_workspace_size(prm) == dash.prefill_workspace_size(_p(dash))
 
 
 def test_prefill_rejects_bad_pointers_and_small_workspace(dash):

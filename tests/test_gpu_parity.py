@@ -379,6 +379,27 @@ def test_newton_cap_hook_reports_device_timeout(dash):
         assert dash.read_device_status(ws) == want, (flags, dash.read_device_status(ws))
 
 
+def test_stall_hook_times_out_and_leaves_the_context_usable(dash):
+    """Fault injection without a GPU fault: the test flag makes Stage 0's bounded copy wait
+    run out (no copy is issued, so nothing arrives on its barrier).  The kernel reports
+    DASH_ERR_DEVICE_TIMEOUT after its 2 s limit and returns with nothing in flight; the next
+    call on the same context succeeds and matches the oracle."""
+    T, D, Bc = 256, 128, 64                          # 4 chunks: one CTA waits its 2 s
+    q, k, v, hc = make_prefill(_cfg(1, 2, 2, T, D, Bc, 1.5, planted=False, seed=61))
+    kd, hcd = _to(k, hc)
+    summ = torch.empty(1, 2, T // Bc, D, device=dev)
+    ws = dash.workspace(256, kd.device)
+    for flags, want in ((dash.FLAG_TEST_STALL_WAIT, 5), (0, 0)):
+        prm = dash.make_params(1, 2, 2, T, D, Bc, flags=flags)
+        rc = dash.lib.dash_stage0(ctypes.byref(prm), dash._ptr(kd), dash._ptr(hcd), dash._ptr(summ),
+                                  dash._ptr(ws), 256, dash._stream(kd.device))
+        assert rc == 0
+        assert dash.read_device_status(ws) == want, flags
+    ref = oracle.stage0(k, hc, Bc)
+    rel = np.abs(summ.cpu().double().numpy() - ref).max() / np.abs(ref).max()
+    assert rel <= 1e-5, rel
+
+
 def test_decode_reports_bad_seq_len(dash):
     B, Hkv, cap, D = 2, 2, 256, 128
     kc = torch.zeros(B, Hkv, cap, D, dtype=torch.bfloat16, device=dev)
