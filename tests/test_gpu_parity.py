@@ -133,6 +133,22 @@ def test_prefill_prior_strength_sigma(dash, alpha, sigma):
     check_output(res["out"].cpu().float().numpy(), ref["O"], tag=f"a={alpha} sigma={sigma}")
 
 
+def test_tiny_config_every_row(dash):
+    """The tiny workload as configured (B=1, 4 query heads on 4 KV heads without GQA, D=64,
+    T=1024, chunk 64, alpha 1.5, i.i.d. inputs): mask, p and O on every row."""
+    cfg = CONFIGS["tiny"]
+    q, k, v, hc = make_prefill(cfg)
+    res = dash.prefill(*_to(q, k, v, hc), chunk_size=cfg.chunk_size, alpha=cfg.alpha,
+                       enable_gqa=False, return_p=True, return_active_blocks=True)
+    torch.cuda.synchronize()
+    assert dash.read_device_status(res["ws"]) == 0
+    ref = oracle.prefill(q, k, v, hc, cfg.chunk_size, cfg.alpha)
+    C = ref["p"].shape[-1]
+    check_routing(unpack_mask(res["active_blocks"], C), res["p"].cpu().double().numpy(),
+                  ref["p"], ref["m"], np.arange(cfg.seq_len), cfg.chunk_size, cfg.alpha, tag="tiny")
+    check_output(res["out"].cpu().float().numpy(), ref["O"], tag="tiny")
+
+
 @pytest.mark.parametrize("G,Bc,T", [(16, 64, 2100 + 37), (8, 128, 1500 + 3)])
 def test_attend_without_vt_scratch_takes_the_tile_kernel(dash, G, Bc, T):
     """dash_attend with only the 256-byte status word cannot hold V^T, so Stage 2 runs on the
