@@ -294,9 +294,12 @@ def test_stage2_masked_chunks_contribute_exactly_nothing():
     assert checked >= 12
 
 
-def test_stage2_prior_softmax_is_the_variational_optimum():
-    """w = argmax_{w in simplex} z.w - KL(w || g): optimal value log sum_j g_j e^{z_j},
-    masked keys get exactly zero weight, and no feasible perturbation does better."""
+@pytest.mark.parametrize("sigma", [1.0, 0.5, 2.0, 0.0])
+def test_stage2_prior_softmax_is_the_variational_optimum(sigma):
+    """w = argmax_{w in simplex} z.w - KL(w || g) with the prior g proportional to p^sigma on
+    the routed keys (1 on the diagonal keys; sigma is the prior strength): optimal value
+    log sum_j g_j e^{z_j}, masked keys get exactly zero weight, and no feasible perturbation
+    does better."""
     T, Bc, D = 40, 8, 40
     g_ = torch.Generator().manual_seed(9)
     Q = torch.randn(1, 1, T, D, generator=g_, dtype=torch.float64)
@@ -305,7 +308,7 @@ def test_stage2_prior_softmax_is_the_variational_optimum():
     hc = torch.randn(1, D, generator=g_, dtype=torch.float64)
     S = oracle.stage0(K, hc, Bc)
     p, m, tau = oracle.stage1(Q, S, T, Bc, 1.5)
-    W = oracle.stage2(Q, K, V, p, Bc)[0, 0]                       # [T, T]
+    W = oracle.stage2(Q, K, V, p, Bc, sigma=sigma)[0, 0]          # [T, T]
     rng = np.random.default_rng(0)
     for t in range(Bc, T):
         ct = t // Bc
@@ -314,7 +317,8 @@ def test_stage2_prior_softmax_is_the_variational_optimum():
         w = W[t, :t + 1]
         assert (w[prior == 0] == 0).all() and (W[t, t + 1:] == 0).all()
         sup = prior > 0
-        g = prior / prior.sum()
+        g = np.where(sup, np.where(sup, prior, 1.0) ** sigma, 0.0)
+        g = g / g.sum()
 
         def F(u):
             us = u[sup]
