@@ -212,6 +212,35 @@ def test_stage1_gqa_mean_query_equals_mean_scores():
                                    mean_sc[0, :, t, :ct], atol=1e-12)
 
 
+@pytest.mark.parametrize("gamma", [0.2329096645116806, 3.0])
+@pytest.mark.parametrize("alpha", [1.25, 1.5, 2.0])
+def test_stage1_gamma_scales_the_scores_before_entmax(alpha, gamma):
+    """gist.science summary, "Stufe 1": the routing weights are alpha-entmax(gamma z).  The
+    scores z are computed here independently of the oracle (mean query of the KV group,
+    einsum against the summaries, 1/sqrt(D)); oracle.stage1 with gamma must give, row by
+    row, the tau and p of oracle.entmax(gamma z) (pinned on its own) and the margins
+    m = (alpha-1) gamma z - tau.  The first gamma is the one the 128K workload runs at."""
+    q, k, v, hc = make_prefill(CONFIGS["gqa32k"], seq_len=1024 + 37)
+    T, D, Bc = q.shape[2], q.shape[3], 64
+    S = oracle.stage0(k, hc, Bc)
+    qbar = q.double().view(1, 2, 16, T, D).mean(2)                    # [B,Hkv,T,D]
+    z = torch.einsum("bgtd,bgcd->bgtc", qbar, torch.from_numpy(S)).numpy() / math.sqrt(D)
+    rows = np.array([64, 65, 127, 128, 300, 640, 1000, T - 1])
+    p, m, tau = oracle.stage1(q, S, T, Bc, alpha, gamma=gamma, rows=rows)
+    for g in range(2):
+        for i, t in enumerate(rows):
+            ct = t // Bc
+            pr, tr = oracle.entmax(gamma * z[0, g, t, :ct], alpha)
+            np.testing.assert_allclose(p[0, g, i, :ct], pr, atol=1e-12)
+            assert (p[0, g, i, ct:] == 0).all()
+            assert abs(tau[0, g, i] - tr) < 1e-12
+            np.testing.assert_allclose(m[0, g, i, :ct], (alpha - 1) * gamma * z[0, g, t, :ct] - tr,
+                                       atol=1e-12)
+    # The pin bites: the gamma = 1 routing differs from the gamma routing on these rows.
+    p1, _, _ = oracle.stage1(q, S, T, Bc, alpha, gamma=1.0, rows=rows)
+    assert np.abs(p1 - p).max() > 1e-3
+
+
 def test_stage1_margin_sign_is_the_support():
     cfg = CONFIGS["gqa32k"]
     q, k, v, hc = make_prefill(cfg, seq_len=2048 + 37)
