@@ -479,11 +479,12 @@ def main():
     d2h = ho.numel() * ho.element_size()
 
     pk, pk_kind = peaks()
-    # Stage 2 kernel dash_prefill runs for this shape (D = 128, G >= 8): the V^T transpose and
-    # the 128-key-block tcgen05 kernel (timed together as Stage 2).
-    s2_kernel = "k_attend_fa"
-    s2_note = ", V^T transpose included"
-    launches_per_step = 4                     # k_stage0, k_route, k_vtranspose, k_attend_fa
+    # The Stage 2 kernel dash_attend runs with the bench's workspace (the library names it);
+    # the 128-key-block kernels also transpose V (timed together with them as Stage 2).
+    s2_kernel = dash.attend_kernel_name(prm, ws_a.numel())
+    with_vt = s2_kernel in ("k_attend_fa", "k_attend_pair")
+    s2_note = ", V^T transpose included" if with_vt else ""
+    launches_per_step = 3 + (1 if with_vt else 0)   # k_stage0, k_route, [k_vtranspose,] Stage 2
     s2_tflops = stats["active_flops"] / (stage["stage2"] / 1e3) / 1e12
     sb = stage01_bytes(cfg)
     s01_gbs = (sb["stage0"] + sb["stage1"]) / ((stage["stage0"] + stage["stage1"]) / 1e3) / 1e9

@@ -195,6 +195,15 @@ dash_status_t dash_attend(const dash_params_t *params, const void *q, const void
                           const uint64_t *active_blocks, void *out, void *ws, size_t ws_bytes,
                           void *stream);
 
+/* Name of the Stage 2 kernel dash_attend launches for these parameters with a workspace of
+ * ws_bytes (dash_prefill with the same flags and a workspace that leaves ws_bytes after its
+ * status word, tau, summaries and mask words picks the same one): "k_attend_pair" (dense
+ * modes on pairs of SMs), "k_attend_fa" (128-key blocks), "k_attend_tc" (64-key blocks, no
+ * V^T scratch) or "k_attend" (warp-level MMA: head_dim 64 or fewer than 8 query heads per KV
+ * head).  Host only, launches nothing; "" on bad parameters or ws_bytes < 256.  Static
+ * storage. */
+const char *dash_attend_kernel_name(const dash_params_t *params, size_t ws_bytes);
+
 /* Chunk-representation cache update for decode: Stage 0 over each sequence's last n_recent
  * complete chunks.  Idempotent (recomputing a frozen chunk writes the same bits).
  *   k_cache       [B, H_kv, cap, D] bf16 (in), cap = params->seq_len
@@ -240,18 +249,29 @@ dash_status_t dash_decode(const dash_params_t *params, const void *q, const void
  *   - Sizes whose scratch exceeds DASH_STATIC_WS_BYTES return DASH_ERR_WORKSPACE_TOO_SMALL
  *     before anything runs; passing summary_k and active_blocks shrinks the need to the
  *     status word plus tau (B*H_kv*T*4 bytes).
- *   - The first call on a device looks up the array's device address once, with that device
- *     current; make that first call before any stream capture.
+ *   - Every call made outside a stream capture looks up the array's device address with the
+ *     call's device current (so it stays right after a reset of the device's primary
+ *     context); a call made while `stream` is being captured uses the address the last
+ *     uncaptured call on that device found.  Make the first call on each device before any
+ *     stream capture: a captured first call returns DASH_ERR_CUDA.
  *   - Every call shares the array and leaves its contents behind; the status word is cleared
  *     per call and the rest is fully written before it is read.  Calls that overlap on the
  *     GPU race on the array: order them.
- *   - The device status word is not readable through this entry point's arguments; a
- *     device-side fault shows as a wrong result only.
+ *   - Faults found on the device go to the status word inside the array; read them with
+ *     dash_static_ws_read_status.
  * Nothing here calls cudaMalloc, cudaFree or any allocating routine. */
 dash_status_t dash_prefill_static_ws(const dash_params_t *params, const void *q, const void *k,
                                      const void *v, const float *head_cls, void *out,
                                      float *summary_k, float *p, uint64_t *active_blocks,
                                      void *stream);
+
+/* The device status word of dash_prefill_static_ws: synchronises `stream` (the stream of the
+ * calls to check), then returns the status the kernels wrote into the library's static array
+ * (DASH_OK if none) and clears it.  Like the entry point it pairs with, it allocates nothing,
+ * and the paper has no counterpart to it.  Returns DASH_ERR_CUDA if the synchronisation or
+ * the copy fails (or on a device where dash_prefill_static_ws was never called outside a
+ * stream capture while `stream` is being captured). */
+dash_status_t dash_static_ws_read_status(void *stream);
 
 /* Synchronises `stream`, then returns the status word the kernels wrote into ws (DASH_OK if
  * none) and clears it.  Returns DASH_ERR_CUDA if the copy itself fails. */

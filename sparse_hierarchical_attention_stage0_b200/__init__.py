@@ -41,7 +41,8 @@ FLAG_TEST_STALL_WAIT = 16         # test hook: Stage 0's bounded copy wait runs 
 # Every symbol include/dash.h declares.
 EXPORTS = ("dash_prefill_workspace_size", "dash_prefill", "dash_prefill_host", "dash_stage0", "dash_route",
            "dash_attend_workspace_size", "dash_attend", "dash_update_chunk_cache", "dash_decode_workspace_size",
-           "dash_decode", "dash_read_device_status", "dash_status_string")
+           "dash_decode", "dash_read_device_status", "dash_status_string", "dash_prefill_static_ws",
+           "dash_static_ws_read_status", "dash_attend_kernel_name")
 
 
 class Params(ctypes.Structure):
@@ -72,6 +73,8 @@ lib.dash_update_chunk_cache.argtypes = [_P, _vp, _vp, _vp, ctypes.c_int, _vp, _v
 lib.dash_decode.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 lib.dash_read_device_status.argtypes = [_vp, _vp]
 lib.dash_status_string.argtypes = [ctypes.c_int]
+lib.dash_attend_kernel_name.argtypes = [_P, _sz]
+lib.dash_attend_kernel_name.restype = ctypes.c_char_p
 lib.dash_status_string.restype = ctypes.c_char_p
 for _f in ("dash_prefill", "dash_stage0", "dash_route", "dash_attend",
            "dash_update_chunk_cache", "dash_decode", "dash_read_device_status"):
@@ -125,6 +128,11 @@ def attend_workspace_size(params: Params) -> int:
 
 def decode_workspace_size(params: Params) -> int:
     return int(lib.dash_decode_workspace_size(ctypes.byref(params)))
+
+
+def attend_kernel_name(params: Params, ws_bytes: int) -> str:
+    """Name of the Stage 2 kernel dash_attend launches with a workspace of ws_bytes."""
+    return lib.dash_attend_kernel_name(ctypes.byref(params), int(ws_bytes)).decode()
 
 
 def workspace(nbytes: int, device) -> torch.Tensor:

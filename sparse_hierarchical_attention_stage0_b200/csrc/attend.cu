@@ -258,25 +258,48 @@ static cudaError_t launch_attend_t(const StageArgs &a, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_attend(const StageArgs &a, cudaStream_t st) {
+AttendKernel attend_kernel(const StageArgs &a) {
     if (a.t_begin != 0 || a.t_end != a.T) {
         // Row slices: only the 128-key-block kernels take a row range.
-        if (a.vt && a.ignore_routing && attend_pair_supported(a)) return launch_attend_pair(a, st);
-        if (a.vt && attend_fa_supported(a)) return launch_attend_fa(a, st);
-        return cudaErrorNotSupported;
+        if (a.vt && a.ignore_routing && attend_pair_supported(a)) return AttendKernel::kPair;
+        if (a.vt && attend_fa_supported(a)) return AttendKernel::kFa;
+        return AttendKernel::kNone;
     }
     // Pairs of SMs share each K/V block between two tiles, so they walk the union of both
     // tiles' chunks: a gain only when every visible chunk is attended anyway (dense, or every
     // chunk forced active); with routing the larger union costs more than the halved copies
     // save (measured at 128K: 128 ms against 117 ms).
-    if (a.vt && a.ignore_routing && attend_pair_supported(a)) return launch_attend_pair(a, st);
-    if (a.vt && attend_fa_supported(a)) return launch_attend_fa(a, st);
-    if (attend_tc_supported(a)) return launch_attend_tc(a, st);
-    if (a.D == 128 && a.Bc == 64) return launch_attend_t<128, 64>(a, st);
-    if (a.D == 128 && a.Bc == 128) return launch_attend_t<128, 128>(a, st);
-    if (a.D == 64 && a.Bc == 64) return launch_attend_t<64, 64>(a, st);
-    if (a.D == 64 && a.Bc == 128) return launch_attend_t<64, 128>(a, st);
-    return cudaErrorInvalidValue;
+    if (a.vt && a.ignore_routing && attend_pair_supported(a)) return AttendKernel::kPair;
+    if (a.vt && attend_fa_supported(a)) return AttendKernel::kFa;
+    if (attend_tc_supported(a)) return AttendKernel::kTc;
+    if ((a.D == 128 || a.D == 64) && (a.Bc == 64 || a.Bc == 128)) return AttendKernel::kWarp;
+    return AttendKernel::kNone;
+}
+
+const char *attend_kernel_name(AttendKernel k) {
+    switch (k) {
+        case AttendKernel::kPair: return "k_attend_pair";
+        case AttendKernel::kFa: return "k_attend_fa";
+        case AttendKernel::kTc: return "k_attend_tc";
+        case AttendKernel::kWarp: return "k_attend";
+        default: return "";
+    }
+}
+
+cudaError_t launch_attend(const StageArgs &a, cudaStream_t st) {
+    switch (attend_kernel(a)) {
+        case AttendKernel::kPair: return launch_attend_pair(a, st);
+        case AttendKernel::kFa: return launch_attend_fa(a, st);
+        case AttendKernel::kTc: return launch_attend_tc(a, st);
+        case AttendKernel::kWarp:
+            if (a.D == 128 && a.Bc == 64) return launch_attend_t<128, 64>(a, st);
+            if (a.D == 128 && a.Bc == 128) return launch_attend_t<128, 128>(a, st);
+            if (a.D == 64 && a.Bc == 64) return launch_attend_t<64, 64>(a, st);
+            if (a.D == 64 && a.Bc == 128) return launch_attend_t<64, 128>(a, st);
+            return cudaErrorInvalidValue;
+        default:
+            return (a.t_begin != 0 || a.t_end != a.T) ? cudaErrorNotSupported : cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace dash

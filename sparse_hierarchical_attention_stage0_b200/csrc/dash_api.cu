@@ -119,6 +119,23 @@ dash_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? DASH_OK : DAS
 
 }  // namespace
 
+namespace dash {
+
+// Workspace bytes dash_prefill carves for its scratch: the status word, tau, and the
+// summaries and mask words the caller does not supply (the V^T scratch is optional and not
+// counted).  0 on bad parameters.
+size_t prefill_scratch_bytes(const dash_params_t *p, bool has_summary, bool has_mask) {
+    Shape s;
+    if (check_params(p, &s) != DASH_OK) return 0;
+    const bool dense = (p->flags & DASH_FLAG_DENSE) != 0;
+    size_t need = kStatusBytes + bytes_tau(s);
+    if (!dense && !has_summary) need += bytes_summary(s);
+    if (!dense && !has_mask) need += bytes_mask(s);
+    return need;
+}
+
+}  // namespace dash
+
 extern "C" {
 
 const char *dash_status_string(dash_status_t s) {
@@ -161,10 +178,8 @@ dash_status_t dash_prefill(const dash_params_t *p, const void *q, const void *k,
         !aligned16(active_blocks) || (reinterpret_cast<uintptr_t>(ws) & 255u))
         return DASH_ERR_INVALID_ARGUMENT;
     if (!dense && route_rows_per_cta(s.C, s.D) == 0) return DASH_ERR_UNSUPPORTED;
-    size_t need = kStatusBytes + bytes_tau(s);
-    if (!dense && !summary_k) need += bytes_summary(s);
-    if (!dense && !active_blocks) need += bytes_mask(s);
-    if (ws_bytes < need) return DASH_ERR_WORKSPACE_TOO_SMALL;
+    if (ws_bytes < prefill_scratch_bytes(p, summary_k != nullptr, active_blocks != nullptr))
+        return DASH_ERR_WORKSPACE_TOO_SMALL;
 
     unsigned char *w = static_cast<unsigned char *>(ws);
     StageArgs a = stage_args(p, s);
@@ -462,6 +477,17 @@ dash_status_t dash_decode(const dash_params_t *p, const void *q, const void *k_c
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if ((rc = clear_status(ws, st)) != DASH_OK) return rc;
     return from_cuda(launch_decode(a, st));
+}
+
+const char *dash_attend_kernel_name(const dash_params_t *p, size_t ws_bytes) {
+    Shape s;
+    if (check_params(p, &s) != DASH_OK || ws_bytes < kStatusBytes) return "";
+    StageArgs a = stage_args(p, s);
+    const size_t vt = bytes_vt(s);
+    // Only whether the V^T scratch fits matters for the choice, not where it is.
+    static unsigned char probe;
+    if (vt && ws_bytes >= kStatusBytes + vt) a.vt = &probe;
+    return attend_kernel_name(attend_kernel(a));
 }
 
 dash_status_t dash_read_device_status(void *ws, void *stream) {

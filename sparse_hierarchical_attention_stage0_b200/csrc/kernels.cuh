@@ -49,6 +49,10 @@ cudaError_t launch_stage0(const StageArgs &a, const int32_t *seq_lens, int n_rec
 cudaError_t launch_route(const StageArgs &a, cudaStream_t st);
 int route_rows_per_cta(int C, int D);   // 0 if C is too large for the routing kernel
 cudaError_t launch_attend(const StageArgs &a, cudaStream_t st);
+// The Stage 2 kernel launch_attend picks for these arguments, and its name.
+enum class AttendKernel { kNone, kPair, kFa, kTc, kWarp };
+AttendKernel attend_kernel(const StageArgs &a);
+const char *attend_kernel_name(AttendKernel k);
 bool attend_tc_supported(const StageArgs &a);
 cudaError_t launch_attend_tc(const StageArgs &a, cudaStream_t st);
 bool attend_fa_supported(const StageArgs &a);
@@ -59,5 +63,8 @@ cudaError_t launch_attend_pair(const StageArgs &a, cudaStream_t st);
 cudaError_t launch_vtranspose(const void *v, void *vt, int BHkv, int T, int D, cudaStream_t st);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
 int decode_supported(int G, int Ccap, int D);
+// Scratch bytes dash_prefill needs in its workspace (status word, tau, and the summaries /
+// mask words not supplied by the caller); 0 on bad parameters.
+size_t prefill_scratch_bytes(const dash_params_t *p, bool has_summary, bool has_mask);
 
 }  // namespace dash

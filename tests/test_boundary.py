@@ -166,3 +166,16 @@ def test_stage_entry_points_reject_missing_outputs(dash):
     assert dash.lib.dash_attend(ctypes.byref(prm), FAKE, FAKE, FAKE, None, None, None, FAKE,
                                 FAKE, 256, None) == 1       # routed mode needs the routing
     assert dash.lib.dash_read_device_status(None, None) == 1
+
+
+def test_attend_kernel_name_follows_the_dispatch(dash):
+    """The library names the Stage 2 kernel it picks (host only, nothing launched)."""
+    big = 1 << 40
+    assert dash.attend_kernel_name(_p(dash), big) == "k_attend_fa"
+    assert dash.attend_kernel_name(_p(dash), 256) == "k_attend_tc"          # no room for V^T
+    assert dash.attend_kernel_name(_p(dash, flags=1), big) == "k_attend_pair"
+    assert dash.attend_kernel_name(_p(dash, flags=2), big) == "k_attend_pair"
+    assert dash.attend_kernel_name(_p(dash, heads_q=8), big) == "k_attend"     # G = 4
+    assert dash.attend_kernel_name(_p(dash, head_dim=64), big) == "k_attend"   # D = 64
+    assert dash.attend_kernel_name(_p(dash, head_dim=96), big) == ""
+    assert dash.attend_kernel_name(_p(dash), 255) == ""
