@@ -13,6 +13,7 @@ Parity status per function (pins live in ``tests/test_oracle_pins.py``):
   stage2            pinned (dense causal attention special case, variational optimum,
                     exact zero weight of masked chunks)
   decode            pinned (equals the prefill row at the same position)
+  decode_route      pinned (equals decode's routing, which recomputes the summaries)
   diagonal branch, GQA score averaging, bias = sigma * log p: parity unpinned by the pages
   (they rest on stated readings; the tests pin the library to those readings).
 """
@@ -68,6 +69,10 @@ def _get():
                                       _L, _L, ctypes.c_double, ctypes.c_double,
                                       ctypes.c_double, _dbl_p, _dbl_p, _dbl_p, _dbl_p]
         lib.oracle_decode.restype = None
+        lib.oracle_decode_route.argtypes = [_dbl_p, _dbl_p, _i64_p, _L, _L, _L, _L, _L, _L, _L,
+                                            ctypes.c_double, ctypes.c_double, _dbl_p, _dbl_p,
+                                            _dbl_p]
+        lib.oracle_decode_route.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -205,3 +210,23 @@ def decode(q, K_cache, V_cache, head_cls, seq_lens, chunk_size: int, alpha: floa
                          Hkv, cap, D, chunk_size, float(alpha), float(gamma), float(sigma),
                          _ptr(O), _ptr(p), _ptr(m), _ptr(tau))
     return dict(O=O, p=p, m=m, tau=tau)
+
+
+def decode_route(q, summary, seq_lens, cap: int, chunk_size: int, alpha: float,
+                 gamma: float = 1.0):
+    """Routing alone of one decode step from cached summaries [B,Hkv,Cs,D]: the row
+    t = seq_lens[b]-1 of every sequence over its complete chunks.  Returns dict(p, m
+    [B,Hkv,Ccap] with Ccap = ceil(cap/Bc), tau [B,Hkv]) -- the same values as decode()."""
+    q, S = _f64(q), _f64(summary)
+    B, Hq, D = q.shape
+    Hkv, Cs = S.shape[1], S.shape[2]
+    sl = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int64))
+    assert (sl >= 1).all() and ((sl - 1) // chunk_size <= Cs).all()
+    Ccap = (cap + chunk_size - 1) // chunk_size
+    p = np.zeros((B, Hkv, Ccap))
+    m = np.zeros((B, Hkv, Ccap))
+    tau = np.zeros((B, Hkv))
+    _get().oracle_decode_route(_ptr(q), _ptr(S), sl.ctypes.data_as(_i64_p), B, Hq, Hkv, Cs,
+                               Ccap, D, chunk_size, float(alpha), float(gamma), _ptr(p),
+                               _ptr(m), _ptr(tau))
+    return dict(p=p, m=m, tau=tau)

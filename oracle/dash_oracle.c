@@ -321,6 +321,29 @@ void oracle_decode(const double *q, const double *K, const double *V, const doub
         }
 }
 
+/* Routing alone of one decode step (liuzhao09.github.io "DashAttention 精读" section 2:
+ * incremental decoding reuses the cached chunk representations; gist.science summary,
+ * "Stufe 0": a complete chunk's summary is frozen).  For each sequence b the query row is
+ * t = seq_lens[b]-1, routed over its complete chunks c < t / Bc from the given summaries
+ * [B,Hkv,Cs,D] (any Cs > t / Bc - 1): the Stage 1 routing of that row.  q is [B,Hq,D].
+ * Outputs: p and m [B,Hkv,Ccap], tau [B,Hkv] (as oracle_decode). */
+void oracle_decode_route(const double *q, const double *summary, const int64_t *seq_lens,
+                         long B, long Hq, long Hkv, long Cs, long Ccap, long D, long Bc,
+                         double alpha, double gamma, double *p, double *m, double *tau) {
+    long G = Hq / Hkv;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (long b = 0; b < B; ++b)
+        for (long g = 0; g < Hkv; ++g) {
+            long t = seq_lens[b] - 1, ct = t / Bc;
+            double *qbar = (double *)malloc(sizeof(double) * (size_t)D);
+            group_mean(q + (b * Hq + g * G) * D, D, G, D, qbar);
+            tau[b * Hkv + g] = route_qbar(qbar, summary + (b * Hkv + g) * Cs * D, ct, Ccap, D,
+                                          alpha, gamma, p + (b * Hkv + g) * Ccap,
+                                          m + (b * Hkv + g) * Ccap);
+            free(qbar);
+        }
+}
+
 /* Number of OpenMP threads the oracle runs with (for reporting). */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

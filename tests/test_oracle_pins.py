@@ -374,3 +374,28 @@ def test_decode_equals_prefill_row():
         C = (L + 63) // 64
         np.testing.assert_allclose(dec["p"][:, :, :C], full["p"][:, :, i, :C], atol=1e-14)
     assert T == 700
+
+
+def test_decode_route_from_cached_summaries_equals_decode_and_prefill_rows():
+    """Routing a decode step from summaries computed once over the whole cache (frozen
+    chunks, later chunks present but not routable) gives decode's routing, which recomputes
+    the summaries of the complete chunks, and Stage 1's routing of the same prefill row;
+    L = 640 and 641 straddle the completion of chunk 9."""
+    q, k, v, hc = make_prefill(CONFIGS["gqa32k"], seq_len=900)
+    S = oracle.stage0(k, hc, 64)                                 # 14 complete chunks
+    lens = [640, 641, 700, 129]
+    qs = torch.stack([q[0, :, L - 1] for L in lens])                    # [4, Hq, D]
+    kk = k.expand(4, -1, -1, -1)
+    vv = v.expand(4, -1, -1, -1)
+    r = oracle.decode_route(qs, np.repeat(S, 4, axis=0), lens, 900, 64, 1.5)
+    d = oracle.decode(qs, kk, vv, hc, lens, 64, 1.5)
+    np.testing.assert_array_equal(r["p"], d["p"])
+    np.testing.assert_array_equal(r["tau"], d["tau"])
+    np.testing.assert_array_equal(np.isnan(r["m"]), np.isnan(d["m"]))
+    np.testing.assert_array_equal(np.nan_to_num(r["m"]), np.nan_to_num(d["m"]))
+    rows = [L - 1 for L in lens]
+    p1, m1, tau1 = oracle.stage1(q, S, 900, 64, 1.5, rows=rows)
+    for i, L in enumerate(lens):
+        np.testing.assert_allclose(r["p"][i], p1[0, :, i], atol=1e-15)
+        np.testing.assert_allclose(r["tau"][i], tau1[0, :, i], atol=1e-15)
+    assert (r["p"][1, :, 9] >= 0).all() and (r["p"][0, :, 9] == 0).all()   # chunk 9 routable at 641 only
