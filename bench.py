@@ -2,14 +2,17 @@
 """Benchmark of the DashAttention forward path on B200 (one JSON line on stdout).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dash|reference]
-                    [--workload prefill128k|gqa32k|tiny] [--no-decode]
+                    [--workload prefill128k|gqa32k|tiny|sweep] [--no-decode]
 
 A step is one causal prefill (Stage 0 -> Stage 1 -> Stage 2) over the workload's synthetic
 seeded inputs, already resident in HBM.  value = prefill tokens/s over all ranks (replicas:
 every rank runs the same workload on its own GPU, no data-path collective).  Also reported:
 active-FLOP TFLOP/s of Stage 2, per-stage times and roofline fractions, the library's own
 dense path, the end-to-end time through host buffers, a 256-step decode captured in one CUDA
-graph, and the fp64 oracle timed on the host cores on a bounded row sample.
+graph, and the fp64 oracle timed on the host cores on a bounded row sample.  With
+--workload sweep the line covers the six alpha x chunk_size cells of the 64K sweep instead
+(per cell: tokens/s, active TFLOP/s, sparsity, Stage 0-1 GB/s, speedup vs the dense path,
+union waste).
 
 --impl reference times the oracle (plain fp64 C on the host cores) on the same workload and
 metric: each step runs the oracle over a bounded sample of rows, extrapolated to the
@@ -57,6 +60,9 @@ def peaks():
 
 
 def workload_config(name):
+    if name == "sweep64k":
+        from dash_inputs import sweep_config
+        return sweep_config(2)                    # the reference arm times the alpha 1.5, chunk 64 cell
     cfg = CONFIGS[name]
     if name == "prefill128k":
         try:
@@ -141,7 +147,8 @@ def active_stats(dash, q, k, v, hc, cfg):
     sparsity over the routed (visible) chunks, and Stage 2's active FLOPs."""
     res = dash.prefill(q, k, v, hc, cfg.chunk_size, cfg.alpha, cfg.gamma, enable_gqa=True,
                        return_active_blocks=True)
-    cnt = popcount_words(res["active_blocks"]) - 1          # minus the diagonal bit
+    words = res["active_blocks"]
+    cnt = popcount_words(words) - 1                          # minus the diagonal bit
     del res
     T, Bc, D, G = cfg.seq_len, cfg.chunk_size, cfg.head_dim, cfg.group
     t = torch.arange(T, device=q.device)
@@ -153,7 +160,45 @@ def active_stats(dash, q, k, v, hc, cfg):
     dense_flops = 4.0 * D * G * cfg.batch * cfg.heads_kv * (T * (T + 1) / 2.0)
     sparsity = 1.0 - float(active / visible) if visible > 0 else 0.0
     return dict(active_flops=float(flops), dense_flops=float(dense_flops), sparsity=sparsity,
-                active_chunks=float(active), visible_chunks=float(visible))
+                active_chunks=float(active), visible_chunks=float(visible), words=words)
+
+
+def tokens_per_tile(kernel: str, G: int) -> int:
+    """Tokens whose rows share one Stage 2 work unit (and so walk the union of their routed
+    chunks) in the named kernel: 128 rows of G heads per tile (two tiles per SM pair), or 16
+    rows per warp in the warp-MMA kernel."""
+    if kernel == "k_attend_pair":
+        return max(1, 256 // G)
+    if kernel in ("k_attend_fa", "k_attend_tc"):
+        return max(1, 128 // G)
+    return max(1, 16 // G)
+
+
+def union_stats(words: torch.Tensor, chunk_size: int, head_dim: int, G: int, tpt: int):
+    """Union waste of a Stage 2 kernel whose work units hold `tpt` consecutive tokens: each
+    unit walks the OR of its tokens' mask words, so it executes (routed chunks of the union) x
+    (its tokens) token-chunk pairs against the sum of the tokens' own active chunks.
+    words: int64 [B, Hkv, T, W].  Returns dict(factor = executed / active routed pairs,
+    executed_flops = 4 D G (Bc x executed pairs + Bc x tokens for the diagonal block))."""
+    B, Hkv, T, W = words.shape
+    pad = (-T) % tpt
+    w = words
+    if pad:
+        w = torch.cat([w, torch.zeros(B, Hkv, pad, W, dtype=w.dtype, device=w.device)], 2)
+    w = w.view(B, Hkv, (T + pad) // tpt, tpt, W)
+    u = w[:, :, :, 0]
+    for i in range(1, tpt):
+        u = u | w[:, :, :, i]
+    tok = torch.full(((T + pad) // tpt,), tpt, dtype=torch.float64, device=words.device)
+    if pad:
+        tok[-1] = tpt - pad
+    union = (popcount_words(u) - 1).clamp_min(0).to(torch.float64)      # [B,Hkv,units]
+    executed = float((union * tok).sum())
+    active = float((popcount_words(words) - 1).clamp_min(0).to(torch.float64).sum())
+    diag = float(B * Hkv * T) * chunk_size
+    return dict(factor=executed / active if active > 0 else 1.0,
+                executed_flops=4.0 * head_dim * G * (chunk_size * executed + diag),
+                tokens_per_unit=tpt)
 
 
 def stage01_bytes(cfg):
@@ -340,7 +385,8 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="dash", choices=["dash", "reference"])
-    ap.add_argument("--workload", default="prefill128k", choices=["prefill128k", "gqa32k", "tiny"])
+    ap.add_argument("--workload", default="prefill128k",
+                    choices=["prefill128k", "gqa32k", "tiny", "sweep"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--oracle-rows", type=int, default=0, help="0: pick by workload")
     args = ap.parse_args()
@@ -349,8 +395,9 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    cfg = workload_config(args.workload)
-    n_rows = args.oracle_rows or {"prefill128k": 96, "gqa32k": 256, "tiny": 1024}[args.workload]
+    cfg = workload_config(args.workload if args.workload != "sweep" else "sweep64k")
+    n_rows = args.oracle_rows or {"prefill128k": 96, "gqa32k": 256, "tiny": 1024,
+                                  "sweep": 32}[args.workload]
 
     if args.impl == "reference":
         if rank != 0:
@@ -390,9 +437,35 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=dev)
 
+    if args.workload == "sweep":
+        line = bench_sweep(dash, args, dev, world, rank)
+    else:
+        line = bench_prefill(dash, cfg, args, dev, world, rank, full=True)
+        if not args.no_decode and args.workload == "prefill128k":
+            torch.cuda.empty_cache()
+            pk, _ = peaks()
+            dec = bench_decode(dash, dev)
+            dec["roofline"] = {"bound": "hbm", "achieved": dec["achieved_gbs"], "peak": pk["hbm_gbs"],
+                               "unit": "GB/s", "frac": dec["achieved_gbs"] / pk["hbm_gbs"],
+                               "traffic": traffic_for("k_decode", "decode64k")}
+            line["decode"] = dec
+        if rank == 0 and world == 1:
+            q_h, k_h, v_h, hc_h = make_prefill(cfg)
+            line["cpu_baseline"] = oracle_sample(cfg, q_h, k_h, v_h, hc_h, n_rows)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def bench_prefill(dash, cfg, args, dev, world, rank, full=True):
+    """Time `args.steps` routed prefills of `cfg` (inputs resident in HBM, L2 flushed before
+    each), the stages one by one, the dense path, and with full=True the end-to-end prefill
+    from host buffers.  Returns the JSON line's fields (without decode and cpu_baseline)."""
     t0 = time.time()
     q_h, k_h, v_h, hc_h = make_prefill(cfg)
-    log(f"[rank {rank}] inputs drawn in {time.time() - t0:.1f}s")
+    log(f"[rank {rank}] {cfg.name}: inputs drawn in {time.time() - t0:.1f}s")
     q, k, v, hc = (x.to(dev) for x in (q_h, k_h, v_h, hc_h))
     B, Hq, Hkv, T, D, Bc = cfg.batch, cfg.heads_q, cfg.heads_kv, cfg.seq_len, cfg.head_dim, cfg.chunk_size
     prm = dash.make_params(B, Hq, Hkv, T, D, Bc, cfg.alpha, cfg.gamma, 1.0, True)
@@ -413,7 +486,7 @@ def main():
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with ClockSampler(torch.cuda.current_device()) as clk:
         step_ms = timed(prefill, args.steps, stream, flush)
     torch.cuda.synchronize()
     total_ms = max_over_ranks(sum(step_ms), dev)
@@ -452,8 +525,16 @@ def main():
             for j, name in enumerate(("stage0", "stage1", "stage2")):
                 st_ms[name].append(ev[j].elapsed_time(ev[j + 1]))
     stage = {k_: statistics.mean(v_) for k_, v_ in st_ms.items()}
+    del mask, tau
 
     stats = active_stats(dash, q, k, v, hc, cfg)
+    # The Stage 2 kernel dash_attend runs with the bench's workspace (the library names it);
+    # the 128-key-block kernels also transpose V (timed together with them as Stage 2).
+    s2_kernel = dash.attend_kernel_name(prm, ws_a.numel())
+    with_vt = s2_kernel in ("k_attend_fa", "k_attend_pair")
+    s2_note = ", V^T transpose included" if with_vt else ""
+    launches_per_step = 3 + (1 if with_vt else 0)   # k_stage0, k_route, [k_vtranspose,] Stage 2
+    un = union_stats(stats.pop("words"), Bc, D, cfg.group, tokens_per_tile(s2_kernel, cfg.group))
 
     def dense():
         dash.prefill(q, k, v, None, Bc, enable_gqa=True, dense=True, out=out, ws=ws)
@@ -461,30 +542,10 @@ def main():
     for _ in range(2):
         dense()
     dense_ms = statistics.mean(timed(dense, max(2, min(args.steps, 3)), stream, flush))
-
-    # End to end through host buffers: dash_prefill_host copies q, k, v, head_cls from pinned
-    # host memory and out back, in row slices overlapped with the computation.
-    hq, hk, hv, hhc = (x.pin_memory() for x in (q_h, k_h, v_h, hc_h))
-    ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-
-    def e2e():
-        dash.prefill_host(hq, hk, hv, hhc, ho, q, k, v, hc, out, Bc, cfg.alpha, cfg.gamma,
-                          enable_gqa=True, n_slices=E2E_SLICES, ws=ws)
-
-    e2e()
-    if world > 1:
-        torch.distributed.barrier()
-    e2e_ms = max_over_ranks(statistics.mean(timed(e2e, args.steps, stream, flush)), dev)
-    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hhc))
-    d2h = ho.numel() * ho.element_size()
+    dprm = dash.make_params(B, Hq, Hkv, T, D, Bc, enable_gqa=True, flags=1)
+    dense_kernel = dash.attend_kernel_name(dprm, ws.numel())
 
     pk, pk_kind = peaks()
-    # The Stage 2 kernel dash_attend runs with the bench's workspace (the library names it);
-    # the 128-key-block kernels also transpose V (timed together with them as Stage 2).
-    s2_kernel = dash.attend_kernel_name(prm, ws_a.numel())
-    with_vt = s2_kernel in ("k_attend_fa", "k_attend_pair")
-    s2_note = ", V^T transpose included" if with_vt else ""
-    launches_per_step = 3 + (1 if with_vt else 0)   # k_stage0, k_route, [k_vtranspose,] Stage 2
     s2_tflops = stats["active_flops"] / (stage["stage2"] / 1e3) / 1e12
     sb = stage01_bytes(cfg)
     s01_gbs = (sb["stage0"] + sb["stage1"]) / ((stage["stage0"] + stage["stage1"]) / 1e3) / 1e9
@@ -502,7 +563,14 @@ def main():
         "stage_ms": stage,
         "stage01_gbs": s01_gbs,
         "dense_ms": dense_ms,
+        "dense_kernel": dense_kernel,
+        "dense_tflops": stats["dense_flops"] / (dense_ms / 1e3) / 1e12,
         "speedup_vs_dense": dense_ms / (total_ms / args.steps),
+        "union": {"kernel": s2_kernel, "tokens_per_unit": un["tokens_per_unit"],
+                  "factor": un["factor"],
+                  "executed_tflops": un["executed_flops"] / (stage["stage2"] / 1e3) / 1e12,
+                  "note": "executed / active routed token-chunk pairs: each work unit walks "
+                          "the union of its tokens' chunks"},
         "roofline": {"bound": "tensor", "kernel": f"{s2_kernel} (Stage 2{s2_note})",
                      "achieved": s2_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": s2_tflops / pk["bf16_tflops"],
@@ -513,28 +581,69 @@ def main():
                              "unit": "GB/s", "frac": s01_gbs / pk["hbm_gbs"],
                              "frac_of_8tbs_nominal": s01_gbs / 8000.0,
                              "bytes": sb["stage0"] + sb["stage1"]},
-        "e2e": {"value": job_tokens_per_s(world, B * T, 1, e2e_ms), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                "call": f"dash_prefill_host, {E2E_SLICES} row slices"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }
-    del hq, hk, hv, ho
-    if not args.no_decode and args.workload == "prefill128k":
-        del q, k, v, out, ws, mask, flush_buf
-        torch.cuda.empty_cache()
-        dec = bench_decode(dash, dev)
-        dec["roofline"] = {"bound": "hbm", "achieved": dec["achieved_gbs"], "peak": pk["hbm_gbs"],
-                           "unit": "GB/s", "frac": dec["achieved_gbs"] / pk["hbm_gbs"],
-                           "traffic": traffic_for("k_decode", "decode64k")}
-        line["decode"] = dec
-    if rank == 0 and world == 1:
-        line["cpu_baseline"] = oracle_sample(cfg, q_h, k_h, v_h, hc_h, n_rows)
-    if world > 1:
-        torch.distributed.barrier()
-        torch.distributed.destroy_process_group()
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    if full:
+        # End to end through host buffers: dash_prefill_host copies q, k, v, head_cls from
+        # pinned host memory and out back, in row slices overlapped with the computation.
+        hq, hk, hv, hhc = (x.pin_memory() for x in (q_h, k_h, v_h, hc_h))
+        ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+        def e2e():
+            dash.prefill_host(hq, hk, hv, hhc, ho, q, k, v, hc, out, Bc, cfg.alpha, cfg.gamma,
+                              enable_gqa=True, n_slices=E2E_SLICES, ws=ws)
+
+        e2e()
+        if world > 1:
+            torch.distributed.barrier()
+        e2e_ms = max_over_ranks(statistics.mean(timed(e2e, args.steps, stream, flush)), dev)
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hhc))
+        d2h = ho.numel() * ho.element_size()
+        line["e2e"] = {"value": job_tokens_per_s(world, B * T, 1, e2e_ms), "unit": "tokens/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                       "call": f"dash_prefill_host, {E2E_SLICES} row slices"}
+        del hq, hk, hv, ho
+    del q, k, v, out, ws, flush_buf, ws_a
+    torch.cuda.empty_cache()
+    return line
+
+
+SWEEP_METRIC = ("sweep at 64K (B=2, H_kv=8): prefill tokens/s over the alpha x chunk_size "
+                "cells; per cell active TFLOP/s, sparsity, Stage 0-1 GB/s, speedup vs dense")
+
+
+def bench_sweep(dash, args, dev, world, rank):
+    """The six alpha x chunk_size cells of the 64K sweep, each timed as bench_prefill does
+    (without the host-memory leg); value = all cells' tokens over their summed step times."""
+    from dash_inputs import SWEEP_ALPHAS, SWEEP_CHUNKS, sweep_config
+    cells, tokens, ms = [], 0, 0.0
+    for i in range(len(SWEEP_ALPHAS) * len(SWEEP_CHUNKS)):
+        cfg = sweep_config(i)
+        r = bench_prefill(dash, cfg, args, dev, world, rank, full=False)
+        cells.append({"alpha": cfg.alpha, "chunk_size": cfg.chunk_size, "ms_per_step": r["ms_per_step"],
+                      "tokens_per_s": r["value"], "active_tflops": r["active_tflops"],
+                      "realised_sparsity": r["realised_sparsity"], "stage_ms": r["stage_ms"],
+                      "stage01_gbs": r["stage01_gbs"], "dense_ms": r["dense_ms"],
+                      "dense_kernel": r["dense_kernel"], "speedup_vs_dense": r["speedup_vs_dense"],
+                      "union": r["union"], "stage2_kernel": r["union"]["kernel"],
+                      "clocks": r["clocks"]})
+        tokens += cfg.batch * cfg.seq_len * args.steps * world
+        ms += r["ms_per_step"] * args.steps
+    cfg0 = sweep_config(0)
+    return {"metric": SWEEP_METRIC, "value": tokens / (ms / 1e3), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded planted-evidence generator, see dash_inputs)",
+            "config": {"workload": "sweep64k", "batch": cfg0.batch, "heads_q": cfg0.heads_q,
+                       "heads_kv": cfg0.heads_kv, "seq_len": cfg0.seq_len,
+                       "head_dim": cfg0.head_dim, "alphas": list(SWEEP_ALPHAS),
+                       "chunk_sizes": list(SWEEP_CHUNKS), "parallelism": f"replicas x{world}",
+                       "l2": "flushed (256 MiB write) before every timed step"},
+            "gpu_launches": sum(4 if c["union"]["kernel"] in ("k_attend_fa", "k_attend_pair") else 3
+                                for c in cells) * args.steps,
+            "cells": cells}
 
 
 if __name__ == "__main__":

@@ -49,3 +49,26 @@ def test_traffic_is_reported_only_for_the_captured_source(tmp_path, monkeypatch)
     _write_record(rec, "0" * 16)                        # counters taken on another source
     assert bench.traffic_for("k_x", "w") is None
     assert bench.traffic_for("k_y", "w") is None        # no record at all
+
+
+def test_union_stats_counts_the_chunks_each_unit_walks():
+    import torch
+    # 8 tokens of one query chunk (diagonal chunk 5), 4 tokens per unit.  Unit 0's tokens route
+    # to {0}, {1}, {0}, {0, 2}: union {0, 1, 2} x 4 tokens = 12 executed pairs for 5 active.
+    # Unit 1's tokens all route to {3}: 4 executed for 4 active.
+    sets = [{0}, {1}, {0}, {0, 2}, {3}, {3}, {3}, {3}]
+    words = torch.tensor([[[[sum(1 << c for c in s) | (1 << 5)] for s in sets]]], dtype=torch.int64)
+    u = bench.union_stats(words, chunk_size=64, head_dim=128, G=16, tpt=4)
+    assert abs(u["factor"] - 16 / 9) < 1e-12
+    assert u["executed_flops"] == 4.0 * 128 * 16 * (64 * 16 + 64 * 8)
+    # A ragged last unit: 6 tokens at 4 per unit, the second unit holds 2 tokens.
+    u2 = bench.union_stats(words[:, :, :6], chunk_size=64, head_dim=128, G=16, tpt=4)
+    assert abs(u2["factor"] - (12 + 2) / (5 + 2)) < 1e-12
+
+
+def test_tokens_per_tile_follow_the_kernels():
+    assert bench.tokens_per_tile("k_attend_fa", 16) == 8
+    assert bench.tokens_per_tile("k_attend_tc", 8) == 16
+    assert bench.tokens_per_tile("k_attend_pair", 16) == 16
+    assert bench.tokens_per_tile("k_attend", 4) == 4
+    assert bench.tokens_per_tile("k_attend", 32) == 1

@@ -1,10 +1,6 @@
 """GPU parity of every stage against the fp64 oracle, through the C ABI (via the binding),
 at sizes the oracle finishes in seconds that still span several tiles and a ragged tail."""
 import ctypes
-import json
-import os
-from dataclasses import replace
-
 import numpy as np
 import pytest
 import torch
@@ -78,7 +74,7 @@ def test_update_chunk_cache_reports_bad_seq_len(dash):
 # ------------------------------------------------------------------------------ stage 1
 @pytest.mark.parametrize("alpha", [1.0, 1.25, 1.5, 2.0])
 @pytest.mark.parametrize("G,D,Bc,T", [(16, 128, 64, 2048 + 37), (4, 128, 128, 3000),
-                                      (1, 64, 64, 1500), (2, 64, 128, 1100)])
+                                      (4, 128, 64, 2500 + 11), (1, 64, 64, 1500), (2, 64, 128, 1100)])
 def test_route_matches_oracle(dash, alpha, G, D, Bc, T):
     Hkv = 2
     cfg = _cfg(1, G * Hkv, Hkv, T, D, Bc, alpha, seed=int(alpha * 10) + G)
@@ -103,7 +99,7 @@ def test_route_matches_oracle(dash, alpha, G, D, Bc, T):
 # ------------------------------------------------------------------------------ prefill
 @pytest.mark.parametrize("alpha", [1.0, 1.25, 1.5, 2.0])
 @pytest.mark.parametrize("G,D,Bc,T", [(16, 128, 64, 1024 + 100), (4, 128, 128, 1500),
-                                      (1, 64, 64, 777), (8, 64, 64, 640), (32, 128, 64, 700),
+                                      (4, 128, 64, 1300 + 9), (1, 64, 64, 777), (8, 64, 64, 640), (32, 128, 64, 700),
                                       (8, 128, 128, 1500 + 3), (16, 128, 128, 1100)])
 def test_prefill_matches_oracle(dash, alpha, G, D, Bc, T):
     Hkv = 2 if G <= 16 else 1
@@ -253,56 +249,6 @@ def test_prefill_host_equals_prefill(dash, G, D, Bc, T, dense, n):
     assert dash.read_device_status(ws) == 0
     assert torch.equal(ho, ref.cpu())
     assert torch.equal(bo, ref)
-
-
-def _sample_rows(T, Bc, n_rand, seed):
-    """The first and last 16 rows, the ends and starts of the first chunks and of a chunk in
-    the middle, and n_rand uniform rows."""
-    rng = np.random.default_rng(seed)
-    mid = (T // 2) // Bc * Bc
-    r = list(range(16)) + [Bc - 1, Bc, 2 * Bc - 1, 2 * Bc, mid - 1, mid] + list(range(T - 16, T))
-    r += list(rng.integers(0, T, n_rand))
-    return np.unique(np.array(r, dtype=np.int64))
-
-
-@pytest.mark.parametrize("name,n_rand", [("gqa32k", 96), ("prefill128k", 32)])
-def test_full_size_prefill_on_sampled_rows(dash, name, n_rand):
-    """The benchmark workloads at full size, through dash_prefill with the workspace the bench
-    times (V^T scratch included: Stage 2 on the 128-key-block kernel).  Mask and p on sampled
-    rows, O on the same rows; the sliced prefill from host memory equal bit for bit."""
-    cfg = CONFIGS[name]
-    if name == "prefill128k":
-        with open(os.path.join(os.path.dirname(__file__), "golden", "gamma_prefill128k.json")) as f:
-            cfg = replace(cfg, gamma=json.load(f)["gamma"])
-    q, k, v, hc = make_prefill(cfg)
-    B, Hq, T, D = q.shape
-    Hkv, Bc = k.shape[1], cfg.chunk_size
-    C = (T + Bc - 1) // Bc
-    qd, kd, vd, hcd = _to(q, k, v, hc)
-    res = dash.prefill(qd, kd, vd, hcd, Bc, cfg.alpha, cfg.gamma, enable_gqa=True,
-                       return_p=True, return_active_blocks=True)
-    torch.cuda.synchronize()
-    assert dash.read_device_status(res["ws"]) == 0
-    rows = _sample_rows(T, Bc, n_rand, seed=cfg.seed + 100)
-    rt = torch.from_numpy(rows).to(dev)
-    ref = oracle.prefill(q, k, v, hc, Bc, cfg.alpha, cfg.gamma, rows=rows)
-    mask = unpack_mask(res["active_blocks"].index_select(2, rt), C)
-    p = res["p"].index_select(2, rt).cpu().double().numpy()
-    check_routing(mask, p, ref["p"], ref["m"], rows, Bc, cfg.alpha, tag=name)
-    check_output(res["out"].index_select(2, rt).cpu().float().numpy(), ref["O"], tag=name)
-    del res["p"]
-    # The same workload from host memory in 16 row slices.
-    hq, hk, hv, hhc = (x.contiguous().pin_memory() for x in (q, k, v, hc))
-    ho = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
-    bo = torch.empty_like(qd)
-    prm = dash.make_params(B, Hq, Hkv, T, D, Bc, cfg.alpha, cfg.gamma, enable_gqa=True)
-    ws = dash.workspace(dash.prefill_workspace_size(prm), qd.device)
-    dash.prefill_host(hq, hk, hv, hhc, ho, qd, kd, vd, hcd, bo, Bc, cfg.alpha, cfg.gamma,
-                      enable_gqa=True, n_slices=16, ws=ws)
-    torch.cuda.current_stream().synchronize()
-    assert dash.read_device_status(ws) == 0
-    assert torch.equal(bo, res["out"])
-    assert torch.equal(ho, res["out"].cpu())
 
 
 def test_inactive_chunks_do_not_touch_the_output(dash):
