@@ -14,6 +14,9 @@ Parity status per function (pins live in ``tests/test_oracle_pins.py``):
                     exact zero weight of masked chunks)
   decode            pinned (equals the prefill row at the same position)
   decode_route      pinned (equals decode's routing, which recomputes the summaries)
+  estimate_diagonal pinned (diagonal summary = single-query SDPA over the visible keys of the
+                    diagonal chunk; at a chunk's last row it is Stage 0's summary; routing =
+                    entmax of the scores written out independently)
   diagonal branch, GQA score averaging, bias = sigma * log p: parity unpinned by the pages
   (they rest on stated readings; the tests pin the library to those readings).
 """
@@ -62,16 +65,21 @@ def _get():
         lib.oracle_stage1.argtypes = [_dbl_p, _dbl_p, _L, _L, _L, _L, _L, _L, ctypes.c_double,
                                       ctypes.c_double, _i64_p, _L, _dbl_p, _dbl_p, _dbl_p]
         lib.oracle_stage1.restype = None
+        lib.oracle_stage1_diag.argtypes = [_dbl_p, _dbl_p, _dbl_p, _dbl_p, _L, _L, _L, _L, _L, _L,
+                                           ctypes.c_double, ctypes.c_double, _i64_p, _L, _dbl_p,
+                                           _dbl_p, _dbl_p]
+        lib.oracle_stage1_diag.restype = None
         lib.oracle_stage2.argtypes = [_dbl_p, _dbl_p, _dbl_p, _dbl_p, _L, _L, _L, _L, _L, _L,
                                       ctypes.c_double, ctypes.c_int, _i64_p, _L, _dbl_p]
         lib.oracle_stage2.restype = None
         lib.oracle_decode.argtypes = [_dbl_p, _dbl_p, _dbl_p, _dbl_p, _i64_p, _L, _L, _L, _L,
                                       _L, _L, ctypes.c_double, ctypes.c_double,
-                                      ctypes.c_double, _dbl_p, _dbl_p, _dbl_p, _dbl_p]
+                                      ctypes.c_double, ctypes.c_int, _dbl_p, _dbl_p, _dbl_p,
+                                      _dbl_p]
         lib.oracle_decode.restype = None
-        lib.oracle_decode_route.argtypes = [_dbl_p, _dbl_p, _i64_p, _L, _L, _L, _L, _L, _L, _L,
-                                            ctypes.c_double, ctypes.c_double, _dbl_p, _dbl_p,
-                                            _dbl_p]
+        lib.oracle_decode_route.argtypes = [_dbl_p, _dbl_p, _dbl_p, _dbl_p, _i64_p, _L, _L, _L,
+                                            _L, _L, _L, _L, ctypes.c_double, ctypes.c_double,
+                                            _dbl_p, _dbl_p, _dbl_p]
         lib.oracle_decode_route.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
@@ -137,10 +145,13 @@ def entmax(s, alpha: float, method: str = "auto"):
 
 # --------------------------------------------------------------------------- stage 1
 def stage1(Q, summary, seq_len: int, chunk_size: int, alpha: float, gamma: float = 1.0,
-           rows=None):
+           rows=None, estimate_diagonal: bool = False, K=None, head_cls=None):
     """Routing of the given rows (default: all).  Returns (p, m, tau):
     p, m [B,Hkv,nrows,C] (m = margin (alpha-1)s - tau on routable chunks, NaN elsewhere),
-    tau [B,Hkv,nrows].  (gist.science summary, "Stufe 1: Entmax-Chunk-Routing")."""
+    tau [B,Hkv,nrows].  (gist.science summary, "Stufe 1: Entmax-Chunk-Routing").
+    estimate_diagonal (needs K and head_cls): the diagonal chunk takes part in the entmax
+    normalisation with its summary estimated from the keys the row can see (p[.., c_t] is
+    then its probability; aiexpert.news interface paragraph)."""
     Q = _f64(Q)
     S = _f64(summary)
     B, Hq, T, D = Q.shape
@@ -153,9 +164,16 @@ def stage1(Q, summary, seq_len: int, chunk_size: int, alpha: float, gamma: float
     p = np.zeros((B, Hkv, nr, C))
     m = np.zeros((B, Hkv, nr, C))
     tau = np.zeros((B, Hkv, nr))
-    _get().oracle_stage1(_ptr(Q), _ptr(S), B, Hq, Hkv, T, D, chunk_size, float(alpha),
-                         float(gamma), rows.ctypes.data_as(_i64_p), nr, _ptr(p), _ptr(m),
-                         _ptr(tau))
+    if estimate_diagonal:
+        Kd, hc = _f64(K), _f64(head_cls)
+        assert Kd.shape == (B, Hkv, T, D) and hc.shape == (Hkv, D)
+        _get().oracle_stage1_diag(_ptr(Q), _ptr(S), _ptr(Kd), _ptr(hc), B, Hq, Hkv, T, D,
+                                  chunk_size, float(alpha), float(gamma),
+                                  rows.ctypes.data_as(_i64_p), nr, _ptr(p), _ptr(m), _ptr(tau))
+    else:
+        _get().oracle_stage1(_ptr(Q), _ptr(S), B, Hq, Hkv, T, D, chunk_size, float(alpha),
+                             float(gamma), rows.ctypes.data_as(_i64_p), nr, _ptr(p), _ptr(m),
+                             _ptr(tau))
     return p, m, tau
 
 
@@ -183,18 +201,20 @@ def stage2(Q, K, V, p, chunk_size: int, sigma: float = 1.0, rows=None, dense: bo
 
 
 def prefill(Q, K, V, head_cls, chunk_size: int, alpha: float, gamma: float = 1.0,
-            sigma: float = 1.0, rows=None, dense: bool = False):
+            sigma: float = 1.0, rows=None, dense: bool = False,
+            estimate_diagonal: bool = False):
     """Whole forward pass for the given rows: dict(O, p, m, tau, summary)."""
     T = _f64(Q).shape[2] if not hasattr(Q, "shape") else Q.shape[2]
     summary = stage0(K, head_cls, chunk_size)
-    p, m, tau = stage1(Q, summary, T, chunk_size, alpha, gamma, rows)
+    p, m, tau = stage1(Q, summary, T, chunk_size, alpha, gamma, rows,
+                       estimate_diagonal=estimate_diagonal, K=K, head_cls=head_cls)
     O = stage2(Q, K, V, p, chunk_size, sigma, rows, dense)
     return dict(O=O, p=p, m=m, tau=tau, summary=summary)
 
 
 # --------------------------------------------------------------------------- decode
 def decode(q, K_cache, V_cache, head_cls, seq_lens, chunk_size: int, alpha: float,
-           gamma: float = 1.0, sigma: float = 1.0):
+           gamma: float = 1.0, sigma: float = 1.0, estimate_diagonal: bool = False):
     """One decode step: the row t = seq_lens[b]-1 of every sequence.  Returns dict(O
     [B,Hq,D], p, m [B,Hkv,Ccap], tau [B,Hkv])."""
     q, K, V, hc = _f64(q), _f64(K_cache), _f64(V_cache), _f64(head_cls)
@@ -208,15 +228,18 @@ def decode(q, K_cache, V_cache, head_cls, seq_lens, chunk_size: int, alpha: floa
     tau = np.zeros((B, Hkv))
     _get().oracle_decode(_ptr(q), _ptr(K), _ptr(V), _ptr(hc), sl.ctypes.data_as(_i64_p), B, Hq,
                          Hkv, cap, D, chunk_size, float(alpha), float(gamma), float(sigma),
-                         _ptr(O), _ptr(p), _ptr(m), _ptr(tau))
+                         int(estimate_diagonal), _ptr(O), _ptr(p), _ptr(m), _ptr(tau))
     return dict(O=O, p=p, m=m, tau=tau)
 
 
 def decode_route(q, summary, seq_lens, cap: int, chunk_size: int, alpha: float,
-                 gamma: float = 1.0):
+                 gamma: float = 1.0, estimate_diagonal: bool = False, K_cache=None,
+                 head_cls=None):
     """Routing alone of one decode step from cached summaries [B,Hkv,Cs,D]: the row
-    t = seq_lens[b]-1 of every sequence over its complete chunks.  Returns dict(p, m
-    [B,Hkv,Ccap] with Ccap = ceil(cap/Bc), tau [B,Hkv]) -- the same values as decode()."""
+    t = seq_lens[b]-1 of every sequence over its complete chunks (plus, with
+    estimate_diagonal, its diagonal chunk estimated from K_cache [B,Hkv,cap,D]).  Returns
+    dict(p, m [B,Hkv,Ccap] with Ccap = ceil(cap/Bc), tau [B,Hkv]) -- the same values as
+    decode()."""
     q, S = _f64(q), _f64(summary)
     B, Hq, D = q.shape
     Hkv, Cs = S.shape[1], S.shape[2]
@@ -226,7 +249,12 @@ def decode_route(q, summary, seq_lens, cap: int, chunk_size: int, alpha: float,
     p = np.zeros((B, Hkv, Ccap))
     m = np.zeros((B, Hkv, Ccap))
     tau = np.zeros((B, Hkv))
-    _get().oracle_decode_route(_ptr(q), _ptr(S), sl.ctypes.data_as(_i64_p), B, Hq, Hkv, Cs,
-                               Ccap, D, chunk_size, float(alpha), float(gamma), _ptr(p),
-                               _ptr(m), _ptr(tau))
+    Kd = hc = None
+    if estimate_diagonal:
+        Kd, hc = _f64(K_cache), _f64(head_cls)
+        assert Kd.shape[:2] == (B, Hkv) and Kd.shape[2] == cap
+    _get().oracle_decode_route(_ptr(q), _ptr(S), _ptr(Kd) if Kd is not None else None,
+                               _ptr(hc) if hc is not None else None,
+                               sl.ctypes.data_as(_i64_p), B, Hq, Hkv, Cs, cap, D, chunk_size,
+                               float(alpha), float(gamma), _ptr(p), _ptr(m), _ptr(tau))
     return dict(p=p, m=m, tau=tau)

@@ -188,21 +188,36 @@ double oracle_entmax(const double *s, long n, double alpha, double *p) {
 /* ---------------------------------------------------------------- Stage 1 [S1] */
 
 /* Routing of one row from its group-mean query qbar over the ct routable chunks S[0..ct).
- * p_row, m_row have C entries: p_c and the margin m_c = (alpha-1) s_c - tau for c < ct
- * (margin +inf for alpha = 1), p = 0 and m = NaN elsewhere.  Returns tau (the log-sum-exp
- * for alpha = 1; NaN when ct = 0). */
+ * With dsum non-NULL (estimate_diagonal) the diagonal chunk ct takes part in the alpha-entmax
+ * normalisation as one more candidate, its score taken against the estimated summary dsum
+ * (aiexpert.news interface paragraph: estimate_diagonal is the diagonal correction of the
+ * alpha-entmax normalisation; gist.science "Stufe 2": chunks near the diagonal may have no
+ * summary).  p_row, m_row have C entries: p_c and the margin m_c = (alpha-1) s_c - tau for the
+ * routed candidates (margin +inf for alpha = 1), p = 0 and m = NaN elsewhere.  Returns tau
+ * (the log-sum-exp for alpha = 1; NaN when there is no candidate). */
 static double route_qbar(const double *qbar, const double *S, long ct, long C, long D,
-                         double alpha, double gamma, double *p_row, double *m_row) {
+                         double alpha, double gamma, const double *dsum, double *p_row,
+                         double *m_row) {
     for (long c = 0; c < C; ++c) { p_row[c] = 0.0; m_row[c] = NAN; }
-    if (ct == 0) return NAN;
-    double *s = (double *)malloc(sizeof(double) * (size_t)ct);
+    long n = ct + (dsum ? 1 : 0);
+    if (n == 0) return NAN;
+    double *s = (double *)malloc(sizeof(double) * (size_t)n);
     for (long c = 0; c < ct; ++c)
         s[c] = gamma * dotd(qbar, S + c * D, D) / sqrt((double)D);
-    double tau = oracle_entmax(s, ct, alpha, p_row);
-    for (long c = 0; c < ct; ++c)
+    if (dsum) s[ct] = gamma * dotd(qbar, dsum, D) / sqrt((double)D);
+    double tau = oracle_entmax(s, n, alpha, p_row);
+    for (long c = 0; c < n; ++c)
         m_row[c] = alpha == 1.0 ? INFINITY : (alpha - 1.0) * s[c] - tau;
     free(s);
     return tau;
+}
+
+/* Estimated summary of the diagonal chunk of row t: Stage 0's softmax-weighted key sum over
+ * the keys of chunk ct = t / Bc that the row can see (ct Bc .. t). */
+static void diag_summary(const double *Kg, long t, long Bc, const double *hc, long D,
+                         double *out) {
+    long ct = t / Bc;
+    summarize_chunk(Kg + ct * Bc * D, t - ct * Bc + 1, hc, D, out);
 }
 
 /* Group-mean query of KV group g: the mean of the G query rows q_h, h in [gG, (g+1)G).
@@ -214,12 +229,12 @@ static void group_mean(const double *q0, long stride, long G, long D, double *qb
     for (long d = 0; d < D; ++d) qbar[d] /= (double)G;
 }
 
-/* Stage 1 for a list of rows.  summary is [B,Hkv,T/Bc,D] (T is the sequence length the
- * summaries were built from).  Outputs: p_out, m_out [B,Hkv,nrows,C], tau_out [B,Hkv,nrows],
- * with C = ceil(T/Bc). */
-void oracle_stage1(const double *Q, const double *summary, long B, long Hq, long Hkv, long T,
-                   long D, long Bc, double alpha, double gamma, const int64_t *rows,
-                   long nrows, double *p_out, double *m_out, double *tau_out) {
+/* Stage 1 for a list of rows, with K [B,Hkv,T,D] and head_cls non-NULL when estimating the
+ * diagonal chunk's score (see route_qbar); outputs as oracle_stage1. */
+void oracle_stage1_diag(const double *Q, const double *summary, const double *K,
+                        const double *hc, long B, long Hq, long Hkv, long T, long D, long Bc,
+                        double alpha, double gamma, const int64_t *rows, long nrows,
+                        double *p_out, double *m_out, double *tau_out) {
     long G = Hq / Hkv, Cf = T / Bc, C = (T + Bc - 1) / Bc;
 #pragma omp parallel for collapse(3) schedule(dynamic, 16)
     for (long b = 0; b < B; ++b)
@@ -227,11 +242,27 @@ void oracle_stage1(const double *Q, const double *summary, long B, long Hq, long
             for (long r = 0; r < nrows; ++r) {
                 long o = (b * Hkv + g) * nrows + r, t = rows[r];
                 double *qbar = (double *)malloc(sizeof(double) * (size_t)D);
+                double *dsum = NULL;
                 group_mean(Q + ((b * Hq + g * G) * T + t) * D, T * D, G, D, qbar);
+                if (K) {
+                    dsum = (double *)malloc(sizeof(double) * (size_t)D);
+                    diag_summary(K + (b * Hkv + g) * T * D, t, Bc, hc + g * D, D, dsum);
+                }
                 tau_out[o] = route_qbar(qbar, summary + (b * Hkv + g) * Cf * D, t / Bc, C, D,
-                                        alpha, gamma, p_out + o * C, m_out + o * C);
+                                        alpha, gamma, dsum, p_out + o * C, m_out + o * C);
+                free(dsum);
                 free(qbar);
             }
+}
+
+/* Stage 1 for a list of rows.  summary is [B,Hkv,T/Bc,D] (T is the sequence length the
+ * summaries were built from).  Outputs: p_out, m_out [B,Hkv,nrows,C], tau_out [B,Hkv,nrows],
+ * with C = ceil(T/Bc). */
+void oracle_stage1(const double *Q, const double *summary, long B, long Hq, long Hkv, long T,
+                   long D, long Bc, double alpha, double gamma, const int64_t *rows,
+                   long nrows, double *p_out, double *m_out, double *tau_out) {
+    oracle_stage1_diag(Q, summary, NULL, NULL, B, Hq, Hkv, T, D, Bc, alpha, gamma, rows, nrows,
+                       p_out, m_out, tau_out);
 }
 
 /* ---------------------------------------------------------------- Stage 2 [S2] */
@@ -296,8 +327,8 @@ void oracle_stage2(const double *Q, const double *K, const double *V, const doub
  * O [B,Hq,D], p and m [B,Hkv,Ccap] (Ccap = ceil(cap/Bc)), tau [B,Hkv]. */
 void oracle_decode(const double *q, const double *K, const double *V, const double *hc,
                    const int64_t *seq_lens, long B, long Hq, long Hkv, long cap, long D,
-                   long Bc, double alpha, double gamma, double sigma, double *O, double *p,
-                   double *m, double *tau) {
+                   long Bc, double alpha, double gamma, double sigma, int estimate_diagonal,
+                   double *O, double *p, double *m, double *tau) {
     long G = Hq / Hkv, Ccap = (cap + Bc - 1) / Bc;
 #pragma omp parallel for collapse(2) schedule(dynamic, 1)
     for (long b = 0; b < B; ++b)
@@ -311,7 +342,13 @@ void oracle_decode(const double *q, const double *K, const double *V, const doub
             double *pr = p + (b * Hkv + g) * Ccap, *mr = m + (b * Hkv + g) * Ccap;
             double *qbar = (double *)malloc(sizeof(double) * (size_t)D);
             group_mean(q + (b * Hq + g * G) * D, D, G, D, qbar);
-            double tv = route_qbar(qbar, S, ct, Ccap, D, alpha, gamma, pr, mr);
+            double *dsum = NULL;
+            if (estimate_diagonal) {
+                dsum = (double *)malloc(sizeof(double) * (size_t)D);
+                diag_summary(Kg, t, Bc, hc + g * D, D, dsum);
+            }
+            double tv = route_qbar(qbar, S, ct, Ccap, D, alpha, gamma, dsum, pr, mr);
+            free(dsum);
             free(qbar);
             tau[b * Hkv + g] = tv;
             for (long h = g * G; h < (g + 1) * G; ++h)
@@ -325,21 +362,31 @@ void oracle_decode(const double *q, const double *K, const double *V, const doub
  * incremental decoding reuses the cached chunk representations; gist.science summary,
  * "Stufe 0": a complete chunk's summary is frozen).  For each sequence b the query row is
  * t = seq_lens[b]-1, routed over its complete chunks c < t / Bc from the given summaries
- * [B,Hkv,Cs,D] (any Cs > t / Bc - 1): the Stage 1 routing of that row.  q is [B,Hq,D].
- * Outputs: p and m [B,Hkv,Ccap], tau [B,Hkv] (as oracle_decode). */
-void oracle_decode_route(const double *q, const double *summary, const int64_t *seq_lens,
-                         long B, long Hq, long Hkv, long Cs, long Ccap, long D, long Bc,
-                         double alpha, double gamma, double *p, double *m, double *tau) {
+ * [B,Hkv,Cs,D] (any Cs > t / Bc - 1): the Stage 1 routing of that row.  q is [B,Hq,D].  With
+ * the key cache K [B,Hkv,cap,D] and head_cls non-NULL the diagonal chunk's score is estimated
+ * too (see route_qbar).  Outputs: p and m [B,Hkv,Ccap], Ccap = ceil(cap/Bc), tau [B,Hkv] (as
+ * oracle_decode). */
+void oracle_decode_route(const double *q, const double *summary, const double *K,
+                         const double *hc, const int64_t *seq_lens, long B, long Hq, long Hkv,
+                         long Cs, long cap, long D, long Bc, double alpha, double gamma,
+                         double *p, double *m, double *tau) {
+    long Ccap = (cap + Bc - 1) / Bc;
     long G = Hq / Hkv;
 #pragma omp parallel for collapse(2) schedule(dynamic, 1)
     for (long b = 0; b < B; ++b)
         for (long g = 0; g < Hkv; ++g) {
             long t = seq_lens[b] - 1, ct = t / Bc;
             double *qbar = (double *)malloc(sizeof(double) * (size_t)D);
+            double *dsum = NULL;
             group_mean(q + (b * Hq + g * G) * D, D, G, D, qbar);
+            if (K) {
+                dsum = (double *)malloc(sizeof(double) * (size_t)D);
+                diag_summary(K + (b * Hkv + g) * cap * D, t, Bc, hc + g * D, D, dsum);
+            }
             tau[b * Hkv + g] = route_qbar(qbar, summary + (b * Hkv + g) * Cs * D, ct, Ccap, D,
-                                          alpha, gamma, p + (b * Hkv + g) * Ccap,
+                                          alpha, gamma, dsum, p + (b * Hkv + g) * Ccap,
                                           m + (b * Hkv + g) * Ccap);
+            free(dsum);
             free(qbar);
         }
 }

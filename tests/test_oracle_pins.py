@@ -399,3 +399,67 @@ def test_decode_route_from_cached_summaries_equals_decode_and_prefill_rows():
         np.testing.assert_allclose(r["p"][i], p1[0, :, i], atol=1e-15)
         np.testing.assert_allclose(r["tau"][i], tau1[0, :, i], atol=1e-15)
     assert (r["p"][1, :, 9] >= 0).all() and (r["p"][0, :, 9] == 0).all()   # chunk 9 routable at 641 only
+
+
+# ----------------------------------------------------------------------------- estimate_diagonal
+@pytest.mark.parametrize("alpha", [1.0, 1.5, 2.0])
+def test_estimate_diagonal_routes_the_visible_part_of_the_diagonal_chunk(alpha):
+    """Reading of estimate_diagonal (aiexpert.news interface paragraph: the diagonal correction
+    of the alpha-entmax normalisation; gist.science "Stufe 2": chunks near the diagonal may have
+    no summary): the diagonal chunk joins the entmax as one more candidate, its summary
+    estimated as Stage 0 does for a complete chunk but over the keys the row can see.  Written
+    out here independently: the estimated summary is torch's single-query SDPA (float64) of
+    head_cls over keys c_t Bc .. t, the scores an einsum; the routing must be oracle.entmax of
+    [routed scores, diagonal score].  Rows t < Bc route to their diagonal chunk alone."""
+    import torch.nn.functional as F
+    q, k, v, hc = make_prefill(CONFIGS["gqa32k"], seq_len=700)
+    T, D, Bc = 700, 128, 64
+    S = oracle.stage0(k, hc, Bc)
+    rows = np.array([0, 5, 63, 64, 100, 127, 128, 383, 640, 699])
+    p, m, tau = oracle.stage1(q, S, T, Bc, alpha, rows=rows, estimate_diagonal=True, K=k,
+                              head_cls=hc)
+    qbar = q.double().view(1, 2, 16, T, D).mean(2)
+    kd = k.double()
+    for g in range(2):
+        for i, t in enumerate(rows):
+            ct = t // Bc
+            keys = kd[0, g, ct * Bc:t + 1]                                  # visible diagonal keys
+            dsum = F.scaled_dot_product_attention(hc.double()[g].view(1, 1, D), keys[None], keys[None])[0, 0]
+            if t == ct * Bc + Bc - 1 and ct < S.shape[2]:                    # a whole chunk: Stage 0's summary
+                np.testing.assert_allclose(dsum.numpy(), S[0, g, ct], atol=1e-13)
+            z = torch.cat([torch.from_numpy(S[0, g, :ct]) @ qbar[0, g, t], (dsum @ qbar[0, g, t])[None]])
+            z = (z / math.sqrt(D)).numpy()
+            pr, tr = oracle.entmax(z, alpha)
+            np.testing.assert_allclose(p[0, g, i, :ct + 1], pr, atol=1e-12)
+            assert (p[0, g, i, ct + 1:] == 0).all()
+            assert abs(tau[0, g, i] - tr) < 1e-12
+            assert abs(p[0, g, i].sum() - 1.0) < 1e-12
+            if ct == 0:
+                assert abs(p[0, g, i, 0] - 1.0) < 1e-12
+    # Without the flag the routed chunks hold all the mass; with it they hold 1 - p[c_t].
+    p0, _, _ = oracle.stage1(q, S, T, Bc, alpha, rows=rows)
+    ct = rows // Bc
+    routed = rows >= Bc
+    assert (np.abs(p0[0][:, routed].sum(-1) - 1) < 1e-12).all()
+    pdiag = p[0][:, np.arange(rows.size), ct]                                # [Hkv, nrows]
+    routed_mass = p[0].sum(-1) - pdiag
+    np.testing.assert_allclose(routed_mass[:, routed], 1 - pdiag[:, routed], atol=1e-12)
+    if alpha < 2:
+        assert (pdiag[:, routed] > 0).any()
+
+
+def test_estimate_diagonal_decode_equals_prefill_row():
+    q, k, v, hc = make_prefill(CONFIGS["gqa32k"], seq_len=700)
+    rows = [699, 640, 639, 511]
+    full = oracle.prefill(q, k, v, hc, 64, 1.5, rows=rows, estimate_diagonal=True)
+    S = oracle.stage0(k, hc, 64)
+    for i, t in enumerate(rows):
+        L = t + 1
+        dec = oracle.decode(q[:, :, t], k[:, :, :L], v[:, :, :L], hc, [L], 64, 1.5,
+                            estimate_diagonal=True)
+        np.testing.assert_allclose(dec["O"], full["O"][:, :, i], atol=1e-13)
+        C = (L + 63) // 64
+        np.testing.assert_allclose(dec["p"][:, :, :C], full["p"][:, :, i, :C], atol=1e-14)
+        r = oracle.decode_route(q[:, :, t], S, [L], 700, 64, 1.5, estimate_diagonal=True,
+                                K_cache=k, head_cls=hc)
+        np.testing.assert_allclose(r["p"][:, :, :C], full["p"][:, :, i, :C], atol=1e-14)
