@@ -14,6 +14,7 @@ Parity status per function (pins live in ``tests/test_oracle_pins.py``):
                     exact zero weight of masked chunks)
   decode            pinned (equals the prefill row at the same position)
   decode_route      pinned (equals decode's routing, which recomputes the summaries)
+  topk              pinned (numpy's stable argsort on the negated scores; uniform prior)
   estimate_diagonal pinned (diagonal summary = single-query SDPA over the visible keys of the
                     diagonal chunk; at a chunk's last row it is Stage 0's summary; routing =
                     entmax of the scores written out independently)
@@ -66,19 +67,21 @@ def _get():
                                       ctypes.c_double, _i64_p, _L, _dbl_p, _dbl_p, _dbl_p]
         lib.oracle_stage1.restype = None
         lib.oracle_stage1_diag.argtypes = [_dbl_p, _dbl_p, _dbl_p, _dbl_p, _L, _L, _L, _L, _L, _L,
-                                           ctypes.c_double, ctypes.c_double, _i64_p, _L, _dbl_p,
-                                           _dbl_p, _dbl_p]
+                                           ctypes.c_double, ctypes.c_double, _L, _i64_p, _L,
+                                           _dbl_p, _dbl_p, _dbl_p]
+        lib.oracle_topk.argtypes = [_dbl_p, _L, _L, _dbl_p]
+        lib.oracle_topk.restype = ctypes.c_double
         lib.oracle_stage1_diag.restype = None
         lib.oracle_stage2.argtypes = [_dbl_p, _dbl_p, _dbl_p, _dbl_p, _L, _L, _L, _L, _L, _L,
                                       ctypes.c_double, ctypes.c_int, _i64_p, _L, _dbl_p]
         lib.oracle_stage2.restype = None
         lib.oracle_decode.argtypes = [_dbl_p, _dbl_p, _dbl_p, _dbl_p, _i64_p, _L, _L, _L, _L,
                                       _L, _L, ctypes.c_double, ctypes.c_double,
-                                      ctypes.c_double, ctypes.c_int, _dbl_p, _dbl_p, _dbl_p,
-                                      _dbl_p]
+                                      ctypes.c_double, ctypes.c_int, _L, _dbl_p, _dbl_p,
+                                      _dbl_p, _dbl_p]
         lib.oracle_decode.restype = None
         lib.oracle_decode_route.argtypes = [_dbl_p, _dbl_p, _dbl_p, _dbl_p, _i64_p, _L, _L, _L,
-                                            _L, _L, _L, _L, ctypes.c_double, ctypes.c_double,
+                                            _L, _L, _L, _L, ctypes.c_double, ctypes.c_double, _L,
                                             _dbl_p, _dbl_p, _dbl_p]
         lib.oracle_decode_route.restype = None
         lib.oracle_num_threads.argtypes = []
@@ -143,15 +146,25 @@ def entmax(s, alpha: float, method: str = "auto"):
     return p, float(tau)
 
 
+def topk(s, k: int):
+    """Top-k routing of one score vector: (p, theta) with p uniform (1/min(k, n)) on the k
+    highest scores (ties: lower index first) and theta the k-th highest score."""
+    s = _f64(s).ravel()
+    p = np.zeros(s.size)
+    theta = _get().oracle_topk(_ptr(s), s.size, int(k), _ptr(p))
+    return p, float(theta)
+
+
 # --------------------------------------------------------------------------- stage 1
 def stage1(Q, summary, seq_len: int, chunk_size: int, alpha: float, gamma: float = 1.0,
-           rows=None, estimate_diagonal: bool = False, K=None, head_cls=None):
+           rows=None, estimate_diagonal: bool = False, K=None, head_cls=None, topk: int = 0):
     """Routing of the given rows (default: all).  Returns (p, m, tau):
     p, m [B,Hkv,nrows,C] (m = margin (alpha-1)s - tau on routable chunks, NaN elsewhere),
     tau [B,Hkv,nrows].  (gist.science summary, "Stufe 1: Entmax-Chunk-Routing").
     estimate_diagonal (needs K and head_cls): the diagonal chunk takes part in the entmax
     normalisation with its summary estimated from the keys the row can see (p[.., c_t] is
-    then its probability; aiexpert.news interface paragraph)."""
+    then its probability; aiexpert.news interface paragraph).  topk > 0: top-k routing
+    (p uniform over the k highest scores, m = s - theta) instead of alpha-entmax."""
     Q = _f64(Q)
     S = _f64(summary)
     B, Hq, T, D = Q.shape
@@ -164,11 +177,14 @@ def stage1(Q, summary, seq_len: int, chunk_size: int, alpha: float, gamma: float
     p = np.zeros((B, Hkv, nr, C))
     m = np.zeros((B, Hkv, nr, C))
     tau = np.zeros((B, Hkv, nr))
-    if estimate_diagonal:
-        Kd, hc = _f64(K), _f64(head_cls)
-        assert Kd.shape == (B, Hkv, T, D) and hc.shape == (Hkv, D)
-        _get().oracle_stage1_diag(_ptr(Q), _ptr(S), _ptr(Kd), _ptr(hc), B, Hq, Hkv, T, D,
-                                  chunk_size, float(alpha), float(gamma),
+    if estimate_diagonal or topk:
+        Kd = hc = None
+        if estimate_diagonal:
+            Kd, hc = _f64(K), _f64(head_cls)
+            assert Kd.shape == (B, Hkv, T, D) and hc.shape == (Hkv, D)
+        _get().oracle_stage1_diag(_ptr(Q), _ptr(S), _ptr(Kd) if Kd is not None else None,
+                                  _ptr(hc) if hc is not None else None, B, Hq, Hkv, T, D,
+                                  chunk_size, float(alpha), float(gamma), int(topk),
                                   rows.ctypes.data_as(_i64_p), nr, _ptr(p), _ptr(m), _ptr(tau))
     else:
         _get().oracle_stage1(_ptr(Q), _ptr(S), B, Hq, Hkv, T, D, chunk_size, float(alpha),
@@ -202,19 +218,21 @@ def stage2(Q, K, V, p, chunk_size: int, sigma: float = 1.0, rows=None, dense: bo
 
 def prefill(Q, K, V, head_cls, chunk_size: int, alpha: float, gamma: float = 1.0,
             sigma: float = 1.0, rows=None, dense: bool = False,
-            estimate_diagonal: bool = False):
-    """Whole forward pass for the given rows: dict(O, p, m, tau, summary)."""
+            estimate_diagonal: bool = False, topk: int = 0):
+    """Whole forward pass for the given rows: dict(O, p, m, tau, summary).  With topk > 0 the
+    routing is top-k and Stage 2 attends the selection with a uniform prior (sigma = 0)."""
     T = _f64(Q).shape[2] if not hasattr(Q, "shape") else Q.shape[2]
     summary = stage0(K, head_cls, chunk_size)
     p, m, tau = stage1(Q, summary, T, chunk_size, alpha, gamma, rows,
-                       estimate_diagonal=estimate_diagonal, K=K, head_cls=head_cls)
-    O = stage2(Q, K, V, p, chunk_size, sigma, rows, dense)
+                       estimate_diagonal=estimate_diagonal, K=K, head_cls=head_cls, topk=topk)
+    O = stage2(Q, K, V, p, chunk_size, 0.0 if topk else sigma, rows, dense)
     return dict(O=O, p=p, m=m, tau=tau, summary=summary)
 
 
 # --------------------------------------------------------------------------- decode
 def decode(q, K_cache, V_cache, head_cls, seq_lens, chunk_size: int, alpha: float,
-           gamma: float = 1.0, sigma: float = 1.0, estimate_diagonal: bool = False):
+           gamma: float = 1.0, sigma: float = 1.0, estimate_diagonal: bool = False,
+           topk: int = 0):
     """One decode step: the row t = seq_lens[b]-1 of every sequence.  Returns dict(O
     [B,Hq,D], p, m [B,Hkv,Ccap], tau [B,Hkv])."""
     q, K, V, hc = _f64(q), _f64(K_cache), _f64(V_cache), _f64(head_cls)
@@ -227,14 +245,15 @@ def decode(q, K_cache, V_cache, head_cls, seq_lens, chunk_size: int, alpha: floa
     m = np.zeros((B, Hkv, Ccap))
     tau = np.zeros((B, Hkv))
     _get().oracle_decode(_ptr(q), _ptr(K), _ptr(V), _ptr(hc), sl.ctypes.data_as(_i64_p), B, Hq,
-                         Hkv, cap, D, chunk_size, float(alpha), float(gamma), float(sigma),
-                         int(estimate_diagonal), _ptr(O), _ptr(p), _ptr(m), _ptr(tau))
+                         Hkv, cap, D, chunk_size, float(alpha), float(gamma),
+                         0.0 if topk else float(sigma), int(estimate_diagonal), int(topk),
+                         _ptr(O), _ptr(p), _ptr(m), _ptr(tau))
     return dict(O=O, p=p, m=m, tau=tau)
 
 
 def decode_route(q, summary, seq_lens, cap: int, chunk_size: int, alpha: float,
                  gamma: float = 1.0, estimate_diagonal: bool = False, K_cache=None,
-                 head_cls=None):
+                 head_cls=None, topk: int = 0):
     """Routing alone of one decode step from cached summaries [B,Hkv,Cs,D]: the row
     t = seq_lens[b]-1 of every sequence over its complete chunks (plus, with
     estimate_diagonal, its diagonal chunk estimated from K_cache [B,Hkv,cap,D]).  Returns
@@ -256,5 +275,5 @@ def decode_route(q, summary, seq_lens, cap: int, chunk_size: int, alpha: float,
     _get().oracle_decode_route(_ptr(q), _ptr(S), _ptr(Kd) if Kd is not None else None,
                                _ptr(hc) if hc is not None else None,
                                sl.ctypes.data_as(_i64_p), B, Hq, Hkv, Cs, cap, D, chunk_size,
-                               float(alpha), float(gamma), _ptr(p), _ptr(m), _ptr(tau))
+                               float(alpha), float(gamma), int(topk), _ptr(p), _ptr(m), _ptr(tau))
     return dict(p=p, m=m, tau=tau)

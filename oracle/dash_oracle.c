@@ -185,6 +185,29 @@ double oracle_entmax(const double *s, long n, double alpha, double *p) {
     return oracle_entmax_bisect(s, n, alpha, p);
 }
 
+/* Top-k routing (the fixed-k block selection of the hierarchical baselines the pages compare
+ * against -- liuzhao09.github.io "DashAttention 精读", sections 1-2: NSA and InfLLMv2 pick the
+ * top-k blocks by coarse score, then run token-level softmax inside them): the k highest of
+ * s[0..n) (ties: lower index first) are selected; p is uniform over the selection (the prior
+ * of a plain softmax inside the selected blocks).  Returns theta, the k-th highest score (the
+ * lowest one when k >= n). */
+static int cmp_desc_idx(const void *a, const void *b) {
+    const double *x = (const double *)a, *y = (const double *)b;   /* {value, index} pairs */
+    if (x[0] != y[0]) return (x[0] < y[0]) - (x[0] > y[0]);
+    return (x[1] > y[1]) - (x[1] < y[1]);
+}
+
+double oracle_topk(const double *s, long n, long k, double *p) {
+    double *v = (double *)malloc(sizeof(double) * 2 * (size_t)n);
+    for (long c = 0; c < n; ++c) { v[2 * c] = s[c]; v[2 * c + 1] = (double)c; p[c] = 0.0; }
+    qsort(v, (size_t)n, 2 * sizeof(double), cmp_desc_idx);
+    long ke = k < n ? k : n;
+    for (long i = 0; i < ke; ++i) p[(long)v[2 * i + 1]] = 1.0 / (double)ke;
+    double theta = v[2 * (ke - 1)];
+    free(v);
+    return theta;
+}
+
 /* ---------------------------------------------------------------- Stage 1 [S1] */
 
 /* Routing of one row from its group-mean query qbar over the ct routable chunks S[0..ct).
@@ -192,12 +215,14 @@ double oracle_entmax(const double *s, long n, double alpha, double *p) {
  * normalisation as one more candidate, its score taken against the estimated summary dsum
  * (aiexpert.news interface paragraph: estimate_diagonal is the diagonal correction of the
  * alpha-entmax normalisation; gist.science "Stufe 2": chunks near the diagonal may have no
- * summary).  p_row, m_row have C entries: p_c and the margin m_c = (alpha-1) s_c - tau for the
- * routed candidates (margin +inf for alpha = 1), p = 0 and m = NaN elsewhere.  Returns tau
- * (the log-sum-exp for alpha = 1; NaN when there is no candidate). */
+ * summary).  With topk > 0 the routing is the top-k selection of oracle_topk instead of
+ * alpha-entmax.  p_row, m_row have C entries: p_c and the margin m_c = (alpha-1) s_c - tau for
+ * the routed candidates (margin +inf for alpha = 1; s_c - theta for top-k), p = 0 and m = NaN
+ * elsewhere.  Returns tau (the log-sum-exp for alpha = 1; theta for top-k; NaN when there is
+ * no candidate). */
 static double route_qbar(const double *qbar, const double *S, long ct, long C, long D,
-                         double alpha, double gamma, const double *dsum, double *p_row,
-                         double *m_row) {
+                         double alpha, double gamma, const double *dsum, long topk,
+                         double *p_row, double *m_row) {
     for (long c = 0; c < C; ++c) { p_row[c] = 0.0; m_row[c] = NAN; }
     long n = ct + (dsum ? 1 : 0);
     if (n == 0) return NAN;
@@ -205,9 +230,15 @@ static double route_qbar(const double *qbar, const double *S, long ct, long C, l
     for (long c = 0; c < ct; ++c)
         s[c] = gamma * dotd(qbar, S + c * D, D) / sqrt((double)D);
     if (dsum) s[ct] = gamma * dotd(qbar, dsum, D) / sqrt((double)D);
-    double tau = oracle_entmax(s, n, alpha, p_row);
-    for (long c = 0; c < n; ++c)
-        m_row[c] = alpha == 1.0 ? INFINITY : (alpha - 1.0) * s[c] - tau;
+    double tau;
+    if (topk > 0) {                      /* margins s - theta: >= 0 on the selection */
+        tau = oracle_topk(s, n, topk, p_row);
+        for (long c = 0; c < n; ++c) m_row[c] = s[c] - tau;
+    } else {
+        tau = oracle_entmax(s, n, alpha, p_row);
+        for (long c = 0; c < n; ++c)
+            m_row[c] = alpha == 1.0 ? INFINITY : (alpha - 1.0) * s[c] - tau;
+    }
     free(s);
     return tau;
 }
@@ -230,10 +261,11 @@ static void group_mean(const double *q0, long stride, long G, long D, double *qb
 }
 
 /* Stage 1 for a list of rows, with K [B,Hkv,T,D] and head_cls non-NULL when estimating the
- * diagonal chunk's score (see route_qbar); outputs as oracle_stage1. */
+ * diagonal chunk's score, and topk > 0 for top-k routing (see route_qbar); outputs as
+ * oracle_stage1. */
 void oracle_stage1_diag(const double *Q, const double *summary, const double *K,
                         const double *hc, long B, long Hq, long Hkv, long T, long D, long Bc,
-                        double alpha, double gamma, const int64_t *rows, long nrows,
+                        double alpha, double gamma, long topk, const int64_t *rows, long nrows,
                         double *p_out, double *m_out, double *tau_out) {
     long G = Hq / Hkv, Cf = T / Bc, C = (T + Bc - 1) / Bc;
 #pragma omp parallel for collapse(3) schedule(dynamic, 16)
@@ -249,7 +281,7 @@ void oracle_stage1_diag(const double *Q, const double *summary, const double *K,
                     diag_summary(K + (b * Hkv + g) * T * D, t, Bc, hc + g * D, D, dsum);
                 }
                 tau_out[o] = route_qbar(qbar, summary + (b * Hkv + g) * Cf * D, t / Bc, C, D,
-                                        alpha, gamma, dsum, p_out + o * C, m_out + o * C);
+                                        alpha, gamma, dsum, topk, p_out + o * C, m_out + o * C);
                 free(dsum);
                 free(qbar);
             }
@@ -261,8 +293,8 @@ void oracle_stage1_diag(const double *Q, const double *summary, const double *K,
 void oracle_stage1(const double *Q, const double *summary, long B, long Hq, long Hkv, long T,
                    long D, long Bc, double alpha, double gamma, const int64_t *rows,
                    long nrows, double *p_out, double *m_out, double *tau_out) {
-    oracle_stage1_diag(Q, summary, NULL, NULL, B, Hq, Hkv, T, D, Bc, alpha, gamma, rows, nrows,
-                       p_out, m_out, tau_out);
+    oracle_stage1_diag(Q, summary, NULL, NULL, B, Hq, Hkv, T, D, Bc, alpha, gamma, 0, rows,
+                       nrows, p_out, m_out, tau_out);
 }
 
 /* ---------------------------------------------------------------- Stage 2 [S2] */
@@ -328,7 +360,7 @@ void oracle_stage2(const double *Q, const double *K, const double *V, const doub
 void oracle_decode(const double *q, const double *K, const double *V, const double *hc,
                    const int64_t *seq_lens, long B, long Hq, long Hkv, long cap, long D,
                    long Bc, double alpha, double gamma, double sigma, int estimate_diagonal,
-                   double *O, double *p, double *m, double *tau) {
+                   long topk, double *O, double *p, double *m, double *tau) {
     long G = Hq / Hkv, Ccap = (cap + Bc - 1) / Bc;
 #pragma omp parallel for collapse(2) schedule(dynamic, 1)
     for (long b = 0; b < B; ++b)
@@ -347,7 +379,7 @@ void oracle_decode(const double *q, const double *K, const double *V, const doub
                 dsum = (double *)malloc(sizeof(double) * (size_t)D);
                 diag_summary(Kg, t, Bc, hc + g * D, D, dsum);
             }
-            double tv = route_qbar(qbar, S, ct, Ccap, D, alpha, gamma, dsum, pr, mr);
+            double tv = route_qbar(qbar, S, ct, Ccap, D, alpha, gamma, dsum, topk, pr, mr);
             free(dsum);
             free(qbar);
             tau[b * Hkv + g] = tv;
@@ -369,7 +401,7 @@ void oracle_decode(const double *q, const double *K, const double *V, const doub
 void oracle_decode_route(const double *q, const double *summary, const double *K,
                          const double *hc, const int64_t *seq_lens, long B, long Hq, long Hkv,
                          long Cs, long cap, long D, long Bc, double alpha, double gamma,
-                         double *p, double *m, double *tau) {
+                         long topk, double *p, double *m, double *tau) {
     long Ccap = (cap + Bc - 1) / Bc;
     long G = Hq / Hkv;
 #pragma omp parallel for collapse(2) schedule(dynamic, 1)
@@ -384,7 +416,7 @@ void oracle_decode_route(const double *q, const double *summary, const double *K
                 diag_summary(K + (b * Hkv + g) * cap * D, t, Bc, hc + g * D, D, dsum);
             }
             tau[b * Hkv + g] = route_qbar(qbar, summary + (b * Hkv + g) * Cs * D, ct, Ccap, D,
-                                          alpha, gamma, dsum, p + (b * Hkv + g) * Ccap,
+                                          alpha, gamma, dsum, topk, p + (b * Hkv + g) * Ccap,
                                           m + (b * Hkv + g) * Ccap);
             free(dsum);
             free(qbar);

@@ -463,3 +463,43 @@ def test_estimate_diagonal_decode_equals_prefill_row():
         r = oracle.decode_route(q[:, :, t], S, [L], 700, 64, 1.5, estimate_diagonal=True,
                                 K_cache=k, head_cls=hc)
         np.testing.assert_allclose(r["p"][:, :, :C], full["p"][:, :, i, :C], atol=1e-14)
+
+
+# ----------------------------------------------------------------------------- top-k routing
+@pytest.mark.parametrize("n,k", [(1, 4), (7, 3), (50, 16), (2047, 64), (12, 12)])
+def test_topk_selects_the_k_highest_scores_with_lower_index_on_ties(n, k):
+    """Top-k routing (the fixed-k block selection of the hierarchical baselines the pages
+    compare against, liuzhao09.github.io sections 1-2): against numpy's stable sort on the
+    negated scores (which keeps the lower index first among equal scores)."""
+    s = np.round(RNG.normal(size=n) * 2, 1)          # rounding makes ties likely
+    p, theta = oracle.topk(s, k)
+    order = np.argsort(-s, kind="stable")
+    ke = min(k, n)
+    want = np.zeros(n)
+    want[order[:ke]] = 1.0 / ke
+    np.testing.assert_array_equal(p, want)
+    assert theta == s[order[ke - 1]]
+    assert abs(p.sum() - 1) < 1e-12
+
+
+def test_topk_prefill_attends_the_selection_with_a_uniform_prior():
+    """With top-k routing Stage 2 is plain softmax over the selected chunks' keys and the
+    diagonal chunk (no bias): the oracle's prefill equals its dense attention with every
+    unselected routed chunk's keys masked, written out with torch SDPA (float64)."""
+    import torch.nn.functional as F
+    q, k, v, hc = make_prefill(CONFIGS["gqa32k"], seq_len=600)
+    T, D, Bc, K = 600, 128, 64, 3
+    r = oracle.prefill(q, k, v, hc, Bc, 1.5, topk=K)
+    ct = np.arange(T) // Bc
+    sel = r["p"] > 0                                                   # [1,Hkv,T,C]
+    assert (sel.sum(-1)[0][:, ct >= 1] == np.minimum(K, ct[ct >= 1])).all()
+    keep = np.zeros((2, T, T), bool)
+    j = np.arange(T)
+    for g in range(2):
+        for t in range(T):
+            c = j // Bc
+            keep[g, t] = (j <= t) & ((c == ct[t]) | ((c < ct[t]) & sel[0, g, t, np.minimum(c, sel.shape[-1] - 1)]))
+    mask = torch.from_numpy(np.repeat(keep, 16, axis=0))[None]        # [1,Hq,T,T]
+    ref = F.scaled_dot_product_attention(q.double(), k.double().repeat_interleave(16, 1),
+                                         v.double().repeat_interleave(16, 1), attn_mask=mask)
+    np.testing.assert_allclose(r["O"], ref.numpy(), atol=1e-12)
