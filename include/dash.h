@@ -64,11 +64,15 @@ typedef enum {
     DASH_ERR_WORKSPACE_TOO_SMALL = 3,
     DASH_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed */
     DASH_ERR_DEVICE_TIMEOUT = 5,     /* a device wait or iteration cap ran out */
-    DASH_ERR_RANGE_CLAMPED = 6       /* a logit lay so far above its row's softmax reference
+    DASH_ERR_RANGE_CLAMPED = 6,      /* a logit lay so far above its row's softmax reference
                                         (the maximum over the row's visible keys of the
                                         diagonal chunk) that the row's probabilities were
                                         clamped or their sum overflowed fp32; the output of
                                         that row is not exact */
+    DASH_ERR_BOUNDS = 7              /* debug builds only (libdash_debug.so, compiled with
+                                        DASH_DEBUG): a device-side bounds check failed; the
+                                        access it guarded was skipped, the output is not
+                                        meaningful.  The release library never reports it. */
 } dash_status_t;
 
 enum {
@@ -78,8 +82,16 @@ enum {
     /* Stages 0-1 run and write their outputs, but Stage 2 attends every chunk c <= c_t with
      * bias 0 (all blocks forced active, uniform prior).  Same O as DASH_FLAG_DENSE. */
     DASH_FLAG_FORCE_ALL_ACTIVE = 2,
-    /* Reserved: the diagonal correction of the entmax normalisation ("estimate_diagonal").
-     * The pages give no formula; requesting it returns DASH_ERR_UNSUPPORTED. */
+    /* estimate_diagonal, the diagonal correction of the alpha-entmax normalisation
+     * (aiexpert.news interface paragraph; the pages give no formula, this is the reading
+     * built): the diagonal chunk c_t, which has no frozen summary (gist.science "Stufe 2"),
+     * joins the entmax as one more candidate, scored against an estimated summary -- Stage
+     * 0's softmax-weighted key sum over the keys of chunk c_t the row can see (c_t Bc .. t).
+     * The routed chunks then share 1 - p[c_t] of the mass; p[.., c_t] reports the diagonal's
+     * probability; the diagonal chunk is still always attended with bias 0.  Rows t < Bc
+     * route to the diagonal alone (p[.., 0] = 1).  Supported by dash_prefill,
+     * dash_prefill_host and dash_decode (which then needs head_cls); dash_route returns
+     * DASH_ERR_UNSUPPORTED with it (it takes no keys).  Ignored with DASH_FLAG_DENSE. */
     DASH_FLAG_ESTIMATE_DIAGONAL = 4,
     /* Test hook (fault injection without a GPU fault): caps the entmax Newton solve of the
      * routing at one iteration, so every row that needs more reports DASH_ERR_DEVICE_TIMEOUT
@@ -105,6 +117,14 @@ typedef struct {
     float sigma;      /* prior strength: bias = sigma * log p (1.0 default) */
     int enable_gqa;   /* nonzero: heads_q may be a multiple of heads_kv */
     unsigned flags;   /* DASH_FLAG_* */
+    int topk;         /* 0: alpha-entmax routing.  k > 0: top-k routing instead -- the fixed-k
+                         block selection of the hierarchical baselines the pages compare
+                         against (liuzhao09.github.io "DashAttention 精读", sections 1-2): each
+                         row attends the k chunks c < c_t with the highest Stage 1 scores (all
+                         of them when c_t <= k; the lower index first on equal scores) and its
+                         diagonal chunk, with a uniform prior (bias 0; alpha and sigma unused);
+                         p is 1/min(k, c_t) on the selection, tau the lowest selected score.
+                         Not combinable with DASH_FLAG_ESTIMATE_DIAGONAL. */
 } dash_params_t;
 
 /* Bytes of device workspace dash_prefill uses for these parameters (assuming summary_k and
@@ -122,8 +142,8 @@ size_t dash_prefill_workspace_size(const dash_params_t *params);
  *   out      [B, H_q, T, D]   bf16 (out)
  *   summary_k [B, H_kv, T/Bc, D] fp32 (out, nullable) the chunk-representation cache
  *   p        [B, H_kv, T, C]  fp32 (out, nullable) routing probabilities, C = ceil(T/Bc);
- *            0 for c >= c_t and for inactive chunks (p[.., c_t] = 0: the diagonal is not
- *            routed)
+ *            0 for c > c_t and for inactive chunks; p[.., c_t] = 0 (the diagonal is not
+ *            routed) unless DASH_FLAG_ESTIMATE_DIAGONAL gives it its estimated probability
  *   active_blocks [B, H_kv, T, W] uint64 (out, nullable), W = ceil(C/64); bit c % 64 of word
  *            c / 64 (LSB first) is set iff chunk c is attended by row t (routed-active or
  *            the diagonal); bits above c_t are 0
@@ -174,7 +194,8 @@ dash_status_t dash_stage0(const dash_params_t *params, const void *k, const floa
 /* Stage 1 alone: routing of every row from q [B,H_q,T,D] bf16 and summary_k
  * [B,H_kv,T/Bc,D] fp32.  Writes tau [B,H_kv,T] fp32 (the entmax threshold of each row;
  * the log-sum-exp when alpha = 1; NaN when c_t = 0), active_blocks [B,H_kv,T,W] uint64,
- * and p [B,H_kv,T,C] fp32 when non-NULL.  ws (>= 256 bytes) holds the status word. */
+ * and p [B,H_kv,T,C] fp32 when non-NULL.  ws (>= 256 bytes) holds the status word.
+ * DASH_FLAG_ESTIMATE_DIAGONAL returns DASH_ERR_UNSUPPORTED here (use dash_prefill). */
 dash_status_t dash_route(const dash_params_t *params, const void *q, const float *summary_k,
                          float *tau, float *p, uint64_t *active_blocks, void *ws,
                          size_t ws_bytes, void *stream);
@@ -198,8 +219,9 @@ dash_status_t dash_attend(const dash_params_t *params, const void *q, const void
 /* Name of the Stage 2 kernel dash_attend launches for these parameters with a workspace of
  * ws_bytes (dash_prefill with the same flags and a workspace that leaves ws_bytes after its
  * status word, tau, summaries and mask words picks the same one): "k_attend_pair" (dense
- * modes on pairs of SMs), "k_attend_fa" (128-key blocks), "k_attend_tc" (64-key blocks, no
- * V^T scratch) or "k_attend" (warp-level MMA: head_dim 64 or fewer than 8 query heads per KV
+ * modes on pairs of SMs), "k_attend_pp" (128-key blocks, two ping-ponged query tiles per
+ * CTA), "k_attend_fa" (128-key blocks, one query tile per CTA, where the two-tile kernel's
+ * shared memory does not fit), "k_attend_tc" (64-key blocks, no V^T scratch) or "k_attend" (warp-level MMA: head_dim 64 or fewer than 8 query heads per KV
  * head).  Host only, launches nothing; "" on bad parameters or ws_bytes < 256.  Static
  * storage. */
 const char *dash_attend_kernel_name(const dash_params_t *params, size_t ws_bytes);
@@ -226,6 +248,8 @@ size_t dash_decode_workspace_size(const dash_params_t *params);
  *   k_cache, v_cache [B, H_kv, cap, D] bf16 (in)
  *   seq_lens     [B] int32 DEVICE (in)
  *   summary_cache [B, H_kv, cap/Bc, D] fp32 (in)
+ *   head_cls     [H_kv, D] fp32 (in; only read with DASH_FLAG_ESTIMATE_DIAGONAL, may be NULL
+ *                without it)
  *   out          [B, H_q, D] bf16 (out)
  *   p            [B, H_kv, Ccap] fp32 (out, nullable), Ccap = ceil(cap/Bc)
  *   active_blocks [B, H_kv, Wcap] uint64 (out, nullable), Wcap = ceil(Ccap/64)
@@ -233,8 +257,31 @@ size_t dash_decode_workspace_size(const dash_params_t *params);
  * and attends; no host sync, so a loop of steps can be captured in one CUDA graph. */
 dash_status_t dash_decode(const dash_params_t *params, const void *q, const void *k_cache,
                           const void *v_cache, const int32_t *seq_lens,
-                          const float *summary_cache, void *out, float *p,
-                          uint64_t *active_blocks, void *ws, size_t ws_bytes, void *stream);
+                          const float *summary_cache, const float *head_cls, void *out,
+                          float *p, uint64_t *active_blocks, void *ws, size_t ws_bytes,
+                          void *stream);
+
+/* Paged KV cache (the serving layout the pages name as the first gap of the reference kernels,
+ * liuzhao09.github.io "DashAttention 精读", section 7): the cache lives in pools of pages of
+ * one chunk each, and a per-sequence block table maps logical chunk c of sequence b to its page.
+ *   k_pool, v_pool [n_pages, H_kv, Bc, D] bf16; summary_pool [n_pages, H_kv, D] fp32 (the
+ *   summary of the chunk held by the page); block_table [B, max_blocks] int32 DEVICE, entry
+ *   (b, c) the page of chunk c of sequence b (only chunks 0 .. (seq_lens[b]-1)/Bc are read);
+ *   params->seq_len must equal max_blocks * chunk_size (the capacity per sequence).
+ * A page index outside [0, n_pages) is reported as DASH_ERR_INVALID_ARGUMENT through the
+ * status word and that sequence is skipped.  Otherwise the same arithmetic and outputs as
+ * dash_update_chunk_cache / dash_decode on the gathered contiguous cache. */
+dash_status_t dash_update_chunk_cache_paged(const dash_params_t *params, const void *k_pool,
+                                            const float *head_cls, const int32_t *block_table,
+                                            int max_blocks, int n_pages, const int32_t *seq_lens,
+                                            int n_recent, float *summary_pool, void *ws,
+                                            size_t ws_bytes, void *stream);
+dash_status_t dash_decode_paged(const dash_params_t *params, const void *q, const void *k_pool,
+                                const void *v_pool, const int32_t *block_table, int max_blocks,
+                                int n_pages, const int32_t *seq_lens, const float *summary_pool,
+                                const float *head_cls, void *out, float *p,
+                                uint64_t *active_blocks, void *ws, size_t ws_bytes,
+                                void *stream);
 
 /* Size of the device array that dash_prefill_static_ws uses as its workspace. */
 #define DASH_STATIC_WS_BYTES (16u << 20)

@@ -26,12 +26,12 @@ if not os.path.exists(LIB_PATH):
         f"{LIB_PATH} is missing: build it with "
         "`python sparse_hierarchical_attention_stage0_b200/build.py` (there is no fallback)")
 
-lib = ctypes.CDLL(LIB_PATH)
+LIB_DEBUG_PATH = os.path.join(_HERE, "libdash_debug.so")
 
 DASH_OK = 0
 STATUS_NAMES = {0: "DASH_OK", 1: "DASH_ERR_INVALID_ARGUMENT", 2: "DASH_ERR_UNSUPPORTED",
                 3: "DASH_ERR_WORKSPACE_TOO_SMALL", 4: "DASH_ERR_CUDA",
-                5: "DASH_ERR_DEVICE_TIMEOUT", 6: "DASH_ERR_RANGE_CLAMPED"}
+                5: "DASH_ERR_DEVICE_TIMEOUT", 6: "DASH_ERR_RANGE_CLAMPED", 7: "DASH_ERR_BOUNDS"}
 FLAG_DENSE = 1
 FLAG_FORCE_ALL_ACTIVE = 2
 FLAG_ESTIMATE_DIAGONAL = 4
@@ -42,7 +42,8 @@ FLAG_TEST_STALL_WAIT = 16         # test hook: Stage 0's bounded copy wait runs 
 EXPORTS = ("dash_prefill_workspace_size", "dash_prefill", "dash_prefill_host", "dash_stage0", "dash_route",
            "dash_attend_workspace_size", "dash_attend", "dash_update_chunk_cache", "dash_decode_workspace_size",
            "dash_decode", "dash_read_device_status", "dash_status_string", "dash_prefill_static_ws",
-           "dash_static_ws_read_status", "dash_attend_kernel_name")
+           "dash_static_ws_read_status", "dash_attend_kernel_name", "dash_decode_paged",
+           "dash_update_chunk_cache_paged")
 
 
 class Params(ctypes.Structure):
@@ -51,34 +52,53 @@ class Params(ctypes.Structure):
                 ("seq_len", ctypes.c_int), ("head_dim", ctypes.c_int),
                 ("chunk_size", ctypes.c_int), ("alpha", ctypes.c_float),
                 ("gamma", ctypes.c_float), ("sigma", ctypes.c_float),
-                ("enable_gqa", ctypes.c_int), ("flags", ctypes.c_uint)]
+                ("enable_gqa", ctypes.c_int), ("flags", ctypes.c_uint), ("topk", ctypes.c_int)]
 
 
 _vp = ctypes.c_void_p
 _P = ctypes.POINTER(Params)
 _sz = ctypes.c_size_t
-lib.dash_prefill_workspace_size.argtypes = [_P]
-lib.dash_prefill_workspace_size.restype = _sz
-lib.dash_attend_workspace_size.argtypes = [_P]
-lib.dash_attend_workspace_size.restype = _sz
-lib.dash_decode_workspace_size.argtypes = [_P]
-lib.dash_decode_workspace_size.restype = _sz
-lib.dash_prefill.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
-lib.dash_prefill_host.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
-                                  ctypes.c_int, _vp, _vp, _vp]
-lib.dash_stage0.argtypes = [_P, _vp, _vp, _vp, _vp, _sz, _vp]
-lib.dash_route.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
-lib.dash_attend.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
-lib.dash_update_chunk_cache.argtypes = [_P, _vp, _vp, _vp, ctypes.c_int, _vp, _vp, _sz, _vp]
-lib.dash_decode.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
-lib.dash_read_device_status.argtypes = [_vp, _vp]
-lib.dash_status_string.argtypes = [ctypes.c_int]
-lib.dash_attend_kernel_name.argtypes = [_P, _sz]
-lib.dash_attend_kernel_name.restype = ctypes.c_char_p
-lib.dash_status_string.restype = ctypes.c_char_p
-for _f in ("dash_prefill", "dash_stage0", "dash_route", "dash_attend",
-           "dash_update_chunk_cache", "dash_decode", "dash_read_device_status"):
-    getattr(lib, _f).restype = ctypes.c_int
+
+
+def load_library(path: str) -> ctypes.CDLL:
+    """Load a build of libdash (libdash.so, or the bounds-checking libdash_debug.so) and
+    declare its C signatures."""
+    lib = ctypes.CDLL(path)
+    _declare(lib)
+    return lib
+
+
+def _declare(lib):
+    lib.dash_prefill_workspace_size.argtypes = [_P]
+    lib.dash_prefill_workspace_size.restype = _sz
+    lib.dash_attend_workspace_size.argtypes = [_P]
+    lib.dash_attend_workspace_size.restype = _sz
+    lib.dash_decode_workspace_size.argtypes = [_P]
+    lib.dash_decode_workspace_size.restype = _sz
+    lib.dash_prefill.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.dash_prefill_host.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                                      ctypes.c_int, _vp, _vp, _vp]
+    lib.dash_stage0.argtypes = [_P, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.dash_route.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.dash_attend.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.dash_update_chunk_cache.argtypes = [_P, _vp, _vp, _vp, ctypes.c_int, _vp, _vp, _sz, _vp]
+    lib.dash_decode.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.dash_read_device_status.argtypes = [_vp, _vp]
+    lib.dash_decode_paged.argtypes = [_P, _vp, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int, _vp, _vp,
+                                      _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.dash_update_chunk_cache_paged.argtypes = [_P, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int,
+                                                  _vp, ctypes.c_int, _vp, _vp, _sz, _vp]
+    lib.dash_status_string.argtypes = [ctypes.c_int]
+    lib.dash_attend_kernel_name.argtypes = [_P, _sz]
+    lib.dash_attend_kernel_name.restype = ctypes.c_char_p
+    lib.dash_status_string.restype = ctypes.c_char_p
+    for _f in ("dash_prefill", "dash_stage0", "dash_route", "dash_attend",
+               "dash_update_chunk_cache", "dash_decode", "dash_read_device_status",
+               "dash_decode_paged", "dash_update_chunk_cache_paged"):
+        getattr(lib, _f).restype = ctypes.c_int
+
+
+lib = load_library(LIB_PATH)
 
 
 class DashError(RuntimeError):
@@ -101,10 +121,10 @@ def _stream(device):
 
 
 def make_params(batch, heads_q, heads_kv, seq_len, head_dim, chunk_size=64, alpha=1.5,
-                gamma=1.0, sigma=1.0, enable_gqa=False, flags=0) -> Params:
+                gamma=1.0, sigma=1.0, enable_gqa=False, flags=0, topk=0) -> Params:
     return Params(int(batch), int(heads_q), int(heads_kv), int(seq_len), int(head_dim),
                   int(chunk_size), float(alpha), float(gamma), float(sigma),
-                  1 if enable_gqa else 0, int(flags))
+                  1 if enable_gqa else 0, int(flags), int(topk))
 
 
 def _flags(dense, force_all_active, estimate_diagonal):
@@ -142,7 +162,7 @@ def workspace(nbytes: int, device) -> torch.Tensor:
 def prefill(q, k, v, head_cls, chunk_size=64, alpha=1.5, gamma=1.0, sigma=1.0,
             enable_gqa=False, return_p=False, return_active_blocks=False,
             return_summary=False, dense=False, force_all_active=False,
-            estimate_diagonal=False, out=None, ws=None):
+            estimate_diagonal=False, out=None, ws=None, topk=0):
     """Causal prefill.  q [B,Hq,T,D], k/v [B,Hkv,T,D] bf16 CUDA; head_cls [Hkv,D] fp32.
 
     Returns out [B,Hq,T,D] bf16, or a dict with out and the requested p [B,Hkv,T,C] fp32,
@@ -153,7 +173,7 @@ def prefill(q, k, v, head_cls, chunk_size=64, alpha=1.5, gamma=1.0, sigma=1.0,
     W = (C + 63) // 64
     dev = q.device
     prm = make_params(B, Hq, Hkv, T, D, chunk_size, alpha, gamma, sigma, enable_gqa,
-                      _flags(dense, force_all_active, estimate_diagonal))
+                      _flags(dense, force_all_active, estimate_diagonal), topk)
     _need(q, torch.bfloat16, (B, Hq, T, D), "q")
     _need(k, torch.bfloat16, (B, Hkv, T, D), "k")
     _need(v, torch.bfloat16, (B, Hkv, T, D), "v")
@@ -227,12 +247,12 @@ def stage0(k, head_cls, chunk_size=64, ws=None, summary=None):
 
 
 def route(q, summary, heads_kv, chunk_size=64, alpha=1.5, gamma=1.0, enable_gqa=True,
-          return_p=True, ws=None):
+          return_p=True, ws=None, topk=0):
     """Stage 1 alone: returns dict(tau [B,Hkv,T], active_blocks [B,Hkv,T,W], p or None)."""
     B, Hq, T, D = q.shape
     C = (T + chunk_size - 1) // chunk_size
     W = (C + 63) // 64
-    prm = make_params(B, Hq, heads_kv, T, D, chunk_size, alpha, gamma, 1.0, enable_gqa)
+    prm = make_params(B, Hq, heads_kv, T, D, chunk_size, alpha, gamma, 1.0, enable_gqa, 0, topk)
     dev = q.device
     tau = torch.empty(B, heads_kv, T, dtype=torch.float32, device=dev)
     mask = torch.empty(B, heads_kv, T, W, dtype=torch.int64, device=dev)
@@ -245,12 +265,13 @@ def route(q, summary, heads_kv, chunk_size=64, alpha=1.5, gamma=1.0, enable_gqa=
 
 
 def attend(q, k, v, summary, tau, active_blocks, chunk_size=64, alpha=1.5, gamma=1.0,
-           sigma=1.0, enable_gqa=True, dense=False, force_all_active=False, ws=None, out=None):
+           sigma=1.0, enable_gqa=True, dense=False, force_all_active=False, ws=None, out=None,
+           topk=0):
     """Stage 2 alone from a given routing."""
     B, Hq, T, D = q.shape
     Hkv = k.shape[1]
     prm = make_params(B, Hq, Hkv, T, D, chunk_size, alpha, gamma, sigma, enable_gqa,
-                      _flags(dense, force_all_active, False))
+                      _flags(dense, force_all_active, False), topk)
     if out is None:
         out = torch.empty_like(q)
     if ws is None:
@@ -277,14 +298,16 @@ def update_chunk_cache(k_cache, head_cls, seq_lens, summary_cache, heads_q, chun
 
 def decode(q, k_cache, v_cache, seq_lens, summary_cache, chunk_size=64, alpha=1.5, gamma=1.0,
            sigma=1.0, enable_gqa=True, return_p=False, return_active_blocks=False, out=None,
-           ws=None, p=None, active_blocks=None):
-    """One decode step for the token at seq_lens[b]-1 of every sequence.  q [B,Hq,D]."""
+           ws=None, p=None, active_blocks=None, estimate_diagonal=False, head_cls=None, topk=0):
+    """One decode step for the token at seq_lens[b]-1 of every sequence.  q [B,Hq,D];
+    head_cls [Hkv,D] fp32 is needed with estimate_diagonal."""
     B, Hq, D = q.shape
     Hkv, cap = k_cache.shape[1], k_cache.shape[2]
     Ccap = (cap + chunk_size - 1) // chunk_size
     Wcap = (Ccap + 63) // 64
     dev = q.device
-    prm = make_params(B, Hq, Hkv, cap, D, chunk_size, alpha, gamma, sigma, enable_gqa)
+    prm = make_params(B, Hq, Hkv, cap, D, chunk_size, alpha, gamma, sigma, enable_gqa,
+                      _flags(False, False, estimate_diagonal), topk)
     if out is None:
         out = torch.empty_like(q)
     if return_p and p is None:
@@ -294,12 +317,58 @@ def decode(q, k_cache, v_cache, seq_lens, summary_cache, chunk_size=64, alpha=1.
     if ws is None:
         ws = workspace(decode_workspace_size(prm), dev)
     _check(lib.dash_decode(ctypes.byref(prm), _ptr(q), _ptr(k_cache), _ptr(v_cache),
-                           _ptr(seq_lens), _ptr(summary_cache), _ptr(out), _ptr(p),
+                           _ptr(seq_lens), _ptr(summary_cache), _ptr(head_cls), _ptr(out), _ptr(p),
                            _ptr(active_blocks), _ptr(ws), ws.numel(), _stream(dev)),
            "dash_decode")
     if not (return_p or return_active_blocks):
         return out
     return dict(out=out, p=p, active_blocks=active_blocks)
+
+
+def update_chunk_cache_paged(k_pool, head_cls, block_table, seq_lens, summary_pool, heads_q,
+                             chunk_size=64, n_recent=1, ws=None):
+    """Stage 0 over each sequence's last n_recent complete chunks of a paged cache (in place):
+    k_pool [n_pages,Hkv,Bc,D] bf16, block_table [B,max_blocks] int32, summary_pool
+    [n_pages,Hkv,D] fp32."""
+    n_pages, Hkv, Bc, D = k_pool.shape
+    B, max_blocks = block_table.shape
+    prm = make_params(B, heads_q, Hkv, max_blocks * chunk_size, D, chunk_size, enable_gqa=True)
+    if ws is None:
+        ws = workspace(256, k_pool.device)
+    _check(lib.dash_update_chunk_cache_paged(ctypes.byref(prm), _ptr(k_pool), _ptr(head_cls),
+                                             _ptr(block_table), int(max_blocks), int(n_pages),
+                                             _ptr(seq_lens), int(n_recent), _ptr(summary_pool),
+                                             _ptr(ws), ws.numel(), _stream(k_pool.device)),
+           "dash_update_chunk_cache_paged")
+    return summary_pool
+
+
+def decode_paged(q, k_pool, v_pool, block_table, seq_lens, summary_pool, chunk_size=64,
+                 alpha=1.5, gamma=1.0, sigma=1.0, enable_gqa=True, return_p=False,
+                 return_active_blocks=False, out=None, ws=None, estimate_diagonal=False,
+                 head_cls=None, topk=0):
+    """One decode step on a paged cache (see update_chunk_cache_paged for the layouts)."""
+    B, Hq, D = q.shape
+    n_pages, Hkv = k_pool.shape[0], k_pool.shape[1]
+    max_blocks = block_table.shape[1]
+    cap = max_blocks * chunk_size
+    Ccap = max_blocks
+    Wcap = (Ccap + 63) // 64
+    dev = q.device
+    prm = make_params(B, Hq, Hkv, cap, D, chunk_size, alpha, gamma, sigma, enable_gqa,
+                      _flags(False, False, estimate_diagonal), topk)
+    out = torch.empty_like(q) if out is None else out
+    p = torch.empty(B, Hkv, Ccap, dtype=torch.float32, device=dev) if return_p else None
+    mask = torch.empty(B, Hkv, Wcap, dtype=torch.int64, device=dev) if return_active_blocks else None
+    if ws is None:
+        ws = workspace(decode_workspace_size(prm), dev)
+    _check(lib.dash_decode_paged(ctypes.byref(prm), _ptr(q), _ptr(k_pool), _ptr(v_pool),
+                                 _ptr(block_table), int(max_blocks), int(n_pages), _ptr(seq_lens),
+                                 _ptr(summary_pool), _ptr(head_cls), _ptr(out), _ptr(p), _ptr(mask),
+                                 _ptr(ws), ws.numel(), _stream(dev)), "dash_decode_paged")
+    if not (return_p or return_active_blocks):
+        return out
+    return dict(out=out, p=p, active_blocks=mask)
 
 
 def read_device_status(ws) -> int:

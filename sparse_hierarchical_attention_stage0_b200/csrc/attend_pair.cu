@@ -254,7 +254,8 @@ k_attend_pair(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
             while (word) {
                 const int bit = __ffsll((long long)word) - 1;
                 word &= word - 1ull;
-                list[p++] = (int16_t)(w * 64 + bit);
+                const int cl = w * 64 + bit;
+                list[p++] = (int16_t)(dash_check(cl <= ct_max && cl < a.C, a.status) ? cl : ct_max);
             }
             pos += __shfl_sync(kFull, incl, 31);
         }
@@ -484,13 +485,16 @@ k_attend_pair(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ C
                         v = -INFINITY;
                     } else if (c < ctu) {
                         const long long rowi = bg * a.T + t;
-                        const bool act = (a.mask[rowi * a.W + (c >> 6)] >> (c & 63)) & 1ull;
+                        const bool act = dash_check(t < a.T && c < a.Cf, a.status) &&
+                                         ((a.mask[rowi * a.W + (c >> 6)] >> (c & 63)) & 1ull);
                         if (!act) {
                             v = -INFINITY;
                         } else {
                             const float dot = route_dot<D>(qbar + u * D, a.summary + (bg * a.Cf + c) * D);
                             const float tau = a.tau[rowi];
-                            if (a.rc.kind == 0) {
+                            if (a.rc.kind == kKindTopk) {
+                                v = 0.f;                        // top-k: uniform prior
+                            } else if (a.rc.kind == 0) {
                                 v = a.rc.sigma2 * (__fmul_rn(dot, a.rc.sscale) - tau);
                             } else {
                                 const float m = __fsub_rn(__fmul_rn(dot, a.rc.xscale), tau);

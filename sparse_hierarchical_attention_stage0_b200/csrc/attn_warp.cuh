@@ -139,6 +139,7 @@ __device__ __forceinline__ void softmax_sub(UnitState<D> &st, float (&acc)[4][4]
 template <int D>
 __device__ __forceinline__ float routed_bias2(const float *qb, const float *srow, float tau,
                                               const RouteConsts &rc) {
+    if (rc.kind == kKindTopk) return 0.f;            // top-k: uniform prior
     const float dot = route_dot<D>(qb, srow);
     if (rc.kind == 0) return rc.sigma2 * (__fmul_rn(dot, rc.sscale) - tau);
     const float m = __fsub_rn(__fmul_rn(dot, rc.xscale), tau);

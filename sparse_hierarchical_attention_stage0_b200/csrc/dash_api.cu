@@ -32,7 +32,8 @@ dash_status_t check_params(const dash_params_t *p, Shape *s) {
     if (!std::isfinite(p->gamma) || !(p->gamma > 0.f)) return DASH_ERR_INVALID_ARGUMENT;
     if (!std::isfinite(p->sigma) || p->sigma < 0.f) return DASH_ERR_INVALID_ARGUMENT;
     if (p->flags & ~31u) return DASH_ERR_INVALID_ARGUMENT;
-    if (p->flags & DASH_FLAG_ESTIMATE_DIAGONAL) return DASH_ERR_UNSUPPORTED;
+    if (p->topk < 0) return DASH_ERR_INVALID_ARGUMENT;
+    if (p->topk > 0 && (p->flags & DASH_FLAG_ESTIMATE_DIAGONAL)) return DASH_ERR_UNSUPPORTED;
     if (p->head_dim != 64 && p->head_dim != 128) return DASH_ERR_UNSUPPORTED;
     if (p->chunk_size != 64 && p->chunk_size != 128) return DASH_ERR_UNSUPPORTED;
     const int G = p->heads_q / p->heads_kv;
@@ -71,6 +72,15 @@ RouteConsts route_consts(const dash_params_t *p) {
     }
     rc.sigma2 = (float)(sg * 1.4426950408889634);
     rc.newton_cap = (p->flags & DASH_FLAG_TEST_NEWTON_CAP) ? 1 : kNewtonCap;
+    rc.est_diag = (p->flags & DASH_FLAG_ESTIMATE_DIAGONAL) ? 1 : 0;
+    rc.topk = p->topk;
+    if (p->topk > 0) {                     // scores as for softmax routing, uniform prior
+        rc.kind = kKindTopk;
+        rc.xscale = rc.sscale;
+        rc.bscale2 = 0.f;
+        rc.sigma2 = 0.f;
+    }
+    rc.inv_sqrt_d = (float)(1.0 / sd);
     return rc;
 }
 
@@ -136,6 +146,61 @@ size_t prefill_scratch_bytes(const dash_params_t *p, bool has_summary, bool has_
 
 }  // namespace dash
 
+namespace {
+
+// One decode step on a contiguous cache (block_table null) or a paged one.
+dash_status_t decode_common(const dash_params_t *p, const void *q, const void *k_cache,
+                            const void *v_cache, const int32_t *block_table, int max_blocks,
+                            int n_pages, const int32_t *seq_lens, const float *summary_cache,
+                            const float *head_cls, void *out, float *prob,
+                            uint64_t *active_blocks, void *ws, size_t ws_bytes, void *stream) {
+    Shape s;
+    dash_status_t rc = check_params(p, &s);
+    if (rc != DASH_OK) return rc;
+    if (p->flags & (DASH_FLAG_DENSE | DASH_FLAG_FORCE_ALL_ACTIVE)) return DASH_ERR_UNSUPPORTED;
+    if (!q || !k_cache || !v_cache || !seq_lens || !summary_cache || !out || !ws)
+        return DASH_ERR_INVALID_ARGUMENT;
+    if ((p->flags & DASH_FLAG_ESTIMATE_DIAGONAL) && !head_cls) return DASH_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(summary_cache) ||
+        !aligned16(head_cls) ||
+        !aligned16(out) || !aligned16(prob) || !aligned16(active_blocks) ||
+        (reinterpret_cast<uintptr_t>(seq_lens) & 3u) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return DASH_ERR_INVALID_ARGUMENT;
+    if (!decode_supported(s.G, s.C, s.D)) return DASH_ERR_UNSUPPORTED;
+    if (ws_bytes < kStatusBytes) return DASH_ERR_WORKSPACE_TOO_SMALL;
+    DecodeArgs a = {};
+    a.q = q;
+    a.k = k_cache;
+    a.v = v_cache;
+    a.seq_lens = seq_lens;
+    a.summary = summary_cache;
+    a.head_cls = head_cls;
+    a.block_table = block_table;
+    a.max_blocks = max_blocks;
+    a.n_pages = n_pages;
+    a.out = out;
+    a.p = prob;
+    a.mask = active_blocks;
+    a.B = s.B;
+    a.Hq = s.Hq;
+    a.Hkv = s.Hkv;
+    a.cap = s.T;
+    a.D = s.D;
+    a.Bc = s.Bc;
+    a.G = s.G;
+    a.Ccap = s.C;
+    a.Cf = s.Cf;
+    a.Wcap = s.W;
+    a.rc = route_consts(p);
+    a.qk_scale2 = (float)(1.4426950408889634 / std::sqrt((double)s.D));
+    a.status = static_cast<uint32_t *>(ws);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((rc = clear_status(ws, st)) != DASH_OK) return rc;
+    return from_cuda(launch_decode(a, st));
+}
+
+}  // namespace
+
 extern "C" {
 
 const char *dash_status_string(dash_status_t s) {
@@ -147,6 +212,7 @@ const char *dash_status_string(dash_status_t s) {
         case DASH_ERR_CUDA: return "DASH_ERR_CUDA";
         case DASH_ERR_DEVICE_TIMEOUT: return "DASH_ERR_DEVICE_TIMEOUT";
         case DASH_ERR_RANGE_CLAMPED: return "DASH_ERR_RANGE_CLAMPED";
+        case DASH_ERR_BOUNDS: return "DASH_ERR_BOUNDS";
     }
     return "DASH_ERR_UNKNOWN";
 }
@@ -356,6 +422,8 @@ dash_status_t dash_route(const dash_params_t *p, const void *q, const float *sum
     if (rc != DASH_OK) return rc;
     if (!q || (!summary_k && s.Cf > 0) || !tau || !active_blocks || !ws)
         return DASH_ERR_INVALID_ARGUMENT;
+    // The estimated diagonal needs the keys and head_cls, which this entry point does not take.
+    if (p->flags & DASH_FLAG_ESTIMATE_DIAGONAL) return DASH_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(summary_k) || !aligned16(tau) || !aligned16(prob) ||
         !aligned16(active_blocks) || (reinterpret_cast<uintptr_t>(ws) & 255u))
         return DASH_ERR_INVALID_ARGUMENT;
@@ -438,45 +506,52 @@ size_t dash_decode_workspace_size(const dash_params_t *p) {
 
 dash_status_t dash_decode(const dash_params_t *p, const void *q, const void *k_cache,
                           const void *v_cache, const int32_t *seq_lens,
-                          const float *summary_cache, void *out, float *prob,
-                          uint64_t *active_blocks, void *ws, size_t ws_bytes, void *stream) {
+                          const float *summary_cache, const float *head_cls, void *out,
+                          float *prob, uint64_t *active_blocks, void *ws, size_t ws_bytes,
+                          void *stream) {
+    return decode_common(p, q, k_cache, v_cache, nullptr, 0, 0, seq_lens, summary_cache,
+                         head_cls, out, prob, active_blocks, ws, ws_bytes, stream);
+}
+
+dash_status_t dash_decode_paged(const dash_params_t *p, const void *q, const void *k_pool,
+                                const void *v_pool, const int32_t *block_table, int max_blocks,
+                                int n_pages, const int32_t *seq_lens, const float *summary_pool,
+                                const float *head_cls, void *out, float *prob,
+                                uint64_t *active_blocks, void *ws, size_t ws_bytes,
+                                void *stream) {
+    if (!p || !block_table || max_blocks < 1 || n_pages < 1 ||
+        (reinterpret_cast<uintptr_t>(block_table) & 3u))
+        return DASH_ERR_INVALID_ARGUMENT;
+    if ((long long)max_blocks * p->chunk_size != (long long)p->seq_len) return DASH_ERR_INVALID_ARGUMENT;
+    return decode_common(p, q, k_pool, v_pool, block_table, max_blocks, n_pages, seq_lens,
+                         summary_pool, head_cls, out, prob, active_blocks, ws, ws_bytes, stream);
+}
+
+dash_status_t dash_update_chunk_cache_paged(const dash_params_t *p, const void *k_pool,
+                                            const float *head_cls, const int32_t *block_table,
+                                            int max_blocks, int n_pages, const int32_t *seq_lens,
+                                            int n_recent, float *summary_pool, void *ws,
+                                            size_t ws_bytes, void *stream) {
     Shape s;
     dash_status_t rc = check_params(p, &s);
     if (rc != DASH_OK) return rc;
-    if (p->flags & (DASH_FLAG_DENSE | DASH_FLAG_FORCE_ALL_ACTIVE)) return DASH_ERR_UNSUPPORTED;
-    if (!q || !k_cache || !v_cache || !seq_lens || !summary_cache || !out || !ws)
+    if (!k_pool || !head_cls || !block_table || !seq_lens || !summary_pool || !ws || n_recent < 1 ||
+        max_blocks < 1 || n_pages < 1 || (long long)max_blocks * s.Bc != (long long)s.T)
         return DASH_ERR_INVALID_ARGUMENT;
-    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(summary_cache) ||
-        !aligned16(out) || !aligned16(prob) || !aligned16(active_blocks) ||
-        (reinterpret_cast<uintptr_t>(seq_lens) & 3u) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    if (!aligned16(k_pool) || !aligned16(head_cls) || !aligned16(summary_pool) ||
+        (reinterpret_cast<uintptr_t>(seq_lens) & 3u) || (reinterpret_cast<uintptr_t>(block_table) & 3u) ||
+        (reinterpret_cast<uintptr_t>(ws) & 255u))
         return DASH_ERR_INVALID_ARGUMENT;
-    if (!decode_supported(s.G, s.C, s.D)) return DASH_ERR_UNSUPPORTED;
     if (ws_bytes < kStatusBytes) return DASH_ERR_WORKSPACE_TOO_SMALL;
-    DecodeArgs a = {};
-    a.q = q;
-    a.k = k_cache;
-    a.v = v_cache;
-    a.seq_lens = seq_lens;
-    a.summary = summary_cache;
-    a.out = out;
-    a.p = prob;
-    a.mask = active_blocks;
-    a.B = s.B;
-    a.Hq = s.Hq;
-    a.Hkv = s.Hkv;
-    a.cap = s.T;
-    a.D = s.D;
-    a.Bc = s.Bc;
-    a.G = s.G;
-    a.Ccap = s.C;
-    a.Cf = s.Cf;
-    a.Wcap = s.W;
-    a.rc = route_consts(p);
-    a.qk_scale2 = (float)(1.4426950408889634 / std::sqrt((double)s.D));
+    StageArgs a = stage_args(p, s);
+    a.k = k_pool;
+    a.head_cls = head_cls;
+    a.summary = summary_pool;
     a.status = static_cast<uint32_t *>(ws);
+    if (n_recent > s.Cf) n_recent = s.Cf;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if ((rc = clear_status(ws, st)) != DASH_OK) return rc;
-    return from_cuda(launch_decode(a, st));
+    return from_cuda(launch_stage0_paged(a, seq_lens, n_recent, block_table, max_blocks, n_pages, st));
 }
 
 const char *dash_attend_kernel_name(const dash_params_t *p, size_t ws_bytes) {

@@ -27,6 +27,21 @@ __device__ __forceinline__ void report(uint32_t *status, uint32_t code) {
     if (status) atomicCAS(status, 0u, code);
 }
 
+// Device-side bounds checks of the DASH_DEBUG build (build.py --debug -> libdash_debug.so):
+// dash_check(ok, status) returns ok; a false check is reported as DASH_ERR_BOUNDS through the
+// status word, and the caller then skips (or clamps) the access it guards.  In the release
+// build it returns true and compiles away.
+__device__ __forceinline__ bool dash_check(bool ok, uint32_t *status) {
+#ifdef DASH_DEBUG
+    if (!ok) report(status, DASH_ERR_BOUNDS);
+    return ok;
+#else
+    (void)ok;
+    (void)status;
+    return true;
+#endif
+}
+
 // ---------------------------------------------------------------- warp reductions
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -214,6 +229,9 @@ __device__ __forceinline__ float route_dot(const float *qbar, const float *srow)
     return (p[0] + p[1]) + (p[2] + p[3]);
 }
 
+// RouteConsts::kind of top-k routing (the k highest scores, uniform prior in Stage 2).
+constexpr int kKindTopk = 4;
+
 // Constants of the routing, computed once on the host.
 struct RouteConsts {
     float xscale;     // (alpha-1) * gamma / sqrt(D): x_c = dot * xscale (alpha > 1)
@@ -222,9 +240,105 @@ struct RouteConsts {
     float beta;       // 1 / (alpha-1)  (alpha > 1)
     float bscale2;    // log2 of the prior: bias2 = bscale2 * log2(m) with bscale2 = sigma*beta
     float sigma2;     // sigma * log2(e) (alpha = 1: bias2 = sigma2 * (s - lse))
-    int kind;         // 0: softmax (alpha = 1), 1: alpha = 1.5, 2: alpha = 2, 3: other alpha
+    int kind;         // 0: softmax (alpha = 1), 1: alpha = 1.5, 2: alpha = 2, 3: other alpha,
+                      // kKindTopk: top-k routing
+    int topk;         // k of top-k routing
     int newton_cap;   // iteration cap of the Newton solve (kNewtonCap; 1 under the test hook)
+    int est_diag;     // estimate_diagonal: the diagonal chunk joins the entmax (diag_dot)
+    float inv_sqrt_d; // 1 / sqrt(D): Stage 0's logit scale
 };
+
+// estimate_diagonal: the routing dot qbar . dsum of the diagonal chunk of one row, where dsum
+// is Stage 0's summary taken over the n_vis keys of that chunk the row can see:
+// dsum = sum_j w_j k_j, w = softmax_j(hc . k_j / sqrt(D)), so qbar . dsum = sum_j w_j (qbar . k_j).
+// keys: the chunk's first key, bf16 rows of D (16-byte aligned); 1 <= n_vis <= 128; all 32
+// lanes of one warp call it and get the same value.
+template <int D>
+__device__ __forceinline__ float diag_dot(const __nv_bfloat16 *keys, int n_vis, const float *hc,
+                                          const float *qbar, float inv_sqrt_d) {
+    const int lane = threadIdx.x & 31;
+    float l[4], kq[4];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int j = lane + 32 * i;
+        l[i] = -INFINITY;
+        kq[i] = 0.f;
+        if (j < n_vis) {
+            const uint4 *kr = reinterpret_cast<const uint4 *>(keys + (long long)j * D);
+            float a = 0.f, b = 0.f;
+#pragma unroll 4
+            for (int d8 = 0; d8 < D / 8; ++d8) {
+                const uint4 v = __ldg(kr + d8);
+                const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(b2[e]);
+                    a = fmaf(__ldg(hc + 8 * d8 + 2 * e), f.x, a);
+                    a = fmaf(__ldg(hc + 8 * d8 + 2 * e + 1), f.y, a);
+                    b = fmaf(qbar[8 * d8 + 2 * e], f.x, b);
+                    b = fmaf(qbar[8 * d8 + 2 * e + 1], f.y, b);
+                }
+            }
+            l[i] = a * inv_sqrt_d;
+            kq[i] = b;
+            mx = fmaxf(mx, l[i]);
+        }
+    }
+    mx = warp_max(mx);
+    float den = 0.f, num = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float e = lane + 32 * i < n_vis ? expf(l[i] - mx) : 0.f;
+        den += e;
+        num = fmaf(e, kq[i], num);
+    }
+    return warp_sum(num) / warp_sum(den);
+}
+
+// Order-preserving map of fp32 to uint32: a > b as floats iff key(a) > key(b) (no NaN).
+__device__ __forceinline__ uint32_t f32_key(float x) {
+    const uint32_t u = __float_as_uint(x);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_f32(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Top-k threshold of one row xs[0..n) (all 32 lanes of a warp, 1 <= k < n): the key of the
+// k-th largest score, built bit by bit from the most significant one, and in `need` how many
+// scores equal to it are selected (the lowest indices first: the row's selection is every
+// score above the threshold plus the first `need` equal to it).
+__device__ __forceinline__ uint32_t warp_topk_key(const float *xs, int n, int k, int &need) {
+    const int lane = threadIdx.x & 31;
+    uint32_t ans = 0;
+    for (int b = 31; b >= 0; --b) {
+        const uint32_t t = ans | (1u << b);
+        int cnt = 0;
+        for (int c = lane; c < n; c += 32) cnt += f32_key(xs[c]) >= t ? 1 : 0;
+        if (warp_sum_i(cnt) >= k) ans = t;
+    }
+    int gt = 0;
+    for (int c = lane; c < n; c += 32) gt += f32_key(xs[c]) > ans ? 1 : 0;
+    need = k - warp_sum_i(gt);
+    return ans;
+}
+
+// Walks a top-k selection in index order, 32 entries per call and warp: entry c (= 32 i + lane
+// of the i-th call) is selected if it is one of the n scores and either all of them are
+// selected (sel_all), or its key is above `key`, or it equals `key` and fewer than `need`
+// equal keys came before it (`run` counts those, and is updated).
+__device__ __forceinline__ bool topk_selected(const float *xs, int c, int n, bool sel_all,
+                                              uint32_t key, int need, int &run) {
+    const int lane = threadIdx.x & 31;
+    const bool in = c < n;
+    const uint32_t kc = in ? f32_key(xs[c]) : 0u;
+    const bool eq = in && !sel_all && kc == key;
+    const unsigned bal = __ballot_sync(kFull, eq);
+    const bool sel = in && (sel_all || kc > key || (eq && run + __popc(bal & ((1u << lane) - 1u)) < need));
+    run += __popc(bal);
+    return sel;
+}
 
 // m^beta for the entmax probability of margin m > 0.
 __device__ __forceinline__ float pow_beta(float m, const RouteConsts &rc) {

@@ -58,7 +58,7 @@ struct DecLayout {
     static constexpr size_t warp_tiles = 2 * tile;                 // >= a warp partial
     static constexpr size_t part = 16 * D * 4 + 2 * 16 * 4;        // O[16][D], m[16], l[16]
     static_assert(warp_tiles >= part, "warp partial must fit in the warp's tiles");
-    size_t qbar, cta_part, tiles, xs, list, total;
+    size_t qbar, cta_part, tiles, xs, list, sel, total;
     __host__ __device__ DecLayout(int Ccap) {
         qbar = 0;
         cta_part = qbar + D * 4;
@@ -66,7 +66,8 @@ struct DecLayout {
         tiles = (tiles + 127) & ~(size_t)127;
         xs = tiles + kDecWarps * warp_tiles;
         list = xs + (size_t)((Ccap + 3) & ~3) * 4;
-        total = list + (size_t)(Ccap + 2) * 4;
+        sel = list + (size_t)(Ccap + 2) * 4;
+        total = sel + (size_t)((Ccap + 63) / 32) * 4;
     }
 };
 
@@ -80,6 +81,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
     float *cpart = reinterpret_cast<float *>(smem_raw + L.cta_part);   // O[16][D], m, l
     float *xs = reinterpret_cast<float *>(smem_raw + L.xs);
     int *list = reinterpret_cast<int *>(smem_raw + L.list);
+    uint32_t *sel = reinterpret_cast<uint32_t *>(smem_raw + L.sel);   // top-k selection bits
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_rank();
@@ -92,6 +94,29 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
     }
     const int t = Lb - 1, ct = t / BC, n = ct;
     const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(a.q) + (long long)b * a.Hq * D;
+    // Paged cache: every page the step reads (chunks 0 .. c_t) must lie in the pools; the
+    // check gives the same answer in every CTA of the cluster, so all return together.
+    const int32_t *bt = a.block_table ? a.block_table + (long long)b * a.max_blocks : nullptr;
+    if (bt) {
+        int bad = 0;
+        for (int c = tid; c <= ct; c += kDecWarps * 32) bad |= (bt[c] < 0 || bt[c] >= a.n_pages);
+        if (__syncthreads_or(bad)) {
+            if (tid == 0 && rank == 0) report(a.status, DASH_ERR_INVALID_ARGUMENT);
+            return;
+        }
+    }
+    // Keys / values of chunk c (its first key) and the summary of chunk c.
+    auto kv_base = [&](const void *pool, int c) -> const __nv_bfloat16 * {
+        const __nv_bfloat16 *p0 = reinterpret_cast<const __nv_bfloat16 *>(pool);
+        if (bt) return p0 + ((long long)bt[c] * a.Hkv + g) * BC * D;
+        return p0 + ((long long)bg * a.cap + (long long)c * BC) * D;
+    };
+    // Keys of chunk c that exist in memory (a contiguous cache may end inside its last chunk).
+    auto kv_rows = [&](int c) -> int { return bt ? BC : min(BC, a.cap - c * BC); };
+    auto summary_of = [&](int c) -> const float * {
+        if (bt) return a.summary + ((long long)bt[c] * a.Hkv + g) * D;
+        return a.summary + ((long long)bg * a.Cf + c) * D;
+    };
 
     // 1. group-mean query and this CTA's slice of the scores.
     for (int d8 = tid * 8; d8 < D; d8 += kDecWarps * 32 * 8) {
@@ -104,9 +129,8 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
     const float scale = a.rc.kind == 0 ? a.rc.sscale : a.rc.xscale;
     const int c_lo = (int)((long long)n * rank / kDecCluster);
     const int c_hi = (int)((long long)n * (rank + 1) / kDecCluster);
-    const float *sumg = a.summary + (long long)bg * a.Cf * D;
     for (int c = c_lo + tid; c < c_hi; c += kDecWarps * 32)
-        xs[c] = __fmul_rn(route_dot<D>(qbar, sumg + (long long)c * D), scale);
+        xs[c] = __fmul_rn(route_dot<D>(qbar, summary_of(c)), scale);
 
     // 2. exchange slices through distributed shared memory.
     cluster_sync_all();
@@ -118,14 +142,45 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
     }
     __syncthreads();
 
-    // 3. threshold (every CTA, same bits) and the routing outputs (rank 0).
+    // 3. threshold (every CTA, same bits) and the routing outputs (rank 0).  With
+    // estimate_diagonal the diagonal chunk's score joins the candidates as entry n.
+    const int n_eff = n + (a.rc.est_diag ? 1 : 0);
     if (warp == 0) {
-        float tau = n > 0 ? warp_entmax_tau(xs, n, a.rc, a.status) : __int_as_float(0x7fc00000);
+        if (a.rc.est_diag) {
+            const float dd = diag_dot<D>(kv_base(a.k, ct), t - ct * BC + 1,
+                                         a.head_cls + (long long)g * D, qbar, a.rc.inv_sqrt_d);
+            if (lane == 0) xs[n] = __fmul_rn(dd, scale);
+            __syncwarp();
+        }
+        float tau;
+        if (a.rc.kind == kKindTopk) {
+            // Top-k: selection bits in index order (lower index first on ties); tau = the
+            // lowest selected score.
+            const bool all = n <= a.rc.topk;
+            int need = 0;
+            uint32_t key = 0;
+            if (!all) key = warp_topk_key(xs, n, a.rc.topk, need);
+            int run = 0;
+            for (int c0 = 0; c0 < n; c0 += 32) {
+                const unsigned bal = __ballot_sync(kFull, topk_selected(xs, c0 + lane, n, all, key, need, run));
+                if (lane == 0) sel[c0 >> 5] = bal;
+            }
+            if (n > 0 && all) {
+                float mn = INFINITY;
+                for (int c = lane; c < n; c += 32) mn = fminf(mn, xs[c]);
+                tau = -warp_max(-mn);
+            } else {
+                tau = n > 0 ? key_f32(key) : __int_as_float(0x7fc00000);
+            }
+        } else {
+            tau = n_eff > 0 ? warp_entmax_tau(xs, n_eff, a.rc, a.status) : __int_as_float(0x7fc00000);
+        }
         if (lane == 0) tau_s = tau;
     }
     __syncthreads();
     const float tau = tau_s;
     auto active = [&](int c) -> bool {
+        if (a.rc.kind == kKindTopk) return c < n && ((sel[c >> 5] >> (c & 31)) & 1u);
         return c < n && (a.rc.kind == 0 || __fsub_rn(xs[c], tau) > 0.f);
     };
     if (rank == 0) {
@@ -140,9 +195,11 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
         if (a.p) {
             for (int c = tid; c < a.Ccap; c += kDecWarps * 32) {
                 float val = 0.f;
-                if (active(c)) {
+                if (a.rc.kind == kKindTopk) {
+                    val = active(c) ? 1.f / (float)min(n, a.rc.topk) : 0.f;
+                } else if (active(c) || (c == n && n < n_eff)) {   // routed, or the estimated diagonal
                     const float m = __fsub_rn(xs[c], tau);
-                    val = a.rc.kind == 0 ? expf(xs[c] - tau) : pow_beta(m, a.rc);
+                    val = a.rc.kind == 0 ? expf(xs[c] - tau) : m > 0.f ? pow_beta(m, a.rc) : 0.f;
                 }
                 a.p[(long long)bg * a.Ccap + c] = val;
             }
@@ -154,7 +211,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
         int pos = 0;
         for (int c0 = 0; c0 < n; c0 += 32) {
             const int c = c0 + lane;
-            const bool act = active(c);
+            const bool act = active(c) && dash_check(c < a.Cf && (c + 1) * BC <= a.cap, a.status);
             const unsigned bal = __ballot_sync(kFull, act);
             if (act) list[pos + __popc(bal & ((1u << lane) - 1u))] = c;
             pos += __popc(bal);
@@ -170,8 +227,6 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
     // Attention over this warp's share: entries i with i % NC == rank, (i / NC) % W == warp.
     unsigned char *ks = smem_raw + L.tiles + warp * L.warp_tiles;
     unsigned char *vs = ks + L.tile;
-    const __nv_bfloat16 *kp = reinterpret_cast<const __nv_bfloat16 *>(a.k) + (long long)bg * a.cap * D;
-    const __nv_bfloat16 *vp = reinterpret_cast<const __nv_bfloat16 *>(a.v) + (long long)bg * a.cap * D;
     const int r_lo = lane >> 2, r_hi = r_lo + 8, qd = lane & 3;
     const bool ok_lo = r_lo < G, ok_hi = r_hi < G;
     uint32_t qf[D / 16][4];
@@ -200,28 +255,33 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
     const int first = (int)rank + kDecCluster * warp;
     const int my_n = first < nact ? (nact - first + stride - 1) / stride : 0;
     const int nsteps = my_n * NSUB;
+    // Sub-block s of this warp's share: kSub keys from key (s % NSUB) * kSub of chunk
+    // list[first + (s / NSUB) * stride]; keys past the end of a contiguous cache are zero-filled,
+    // keys after t in the diagonal chunk are masked by the softmax.
     if (nsteps > 0) {
-        load_sub<D>(ks, kp, list[first] * BC, a.cap);
+        load_sub<D>(ks, kv_base(a.k, list[first]), 0, kv_rows(list[first]));
         cp_async_commit();
-        load_sub<D>(vs, vp, list[first] * BC, a.cap);
+        load_sub<D>(vs, kv_base(a.v, list[first]), 0, kv_rows(list[first]));
         cp_async_commit();
     }
     for (int s = 0; s < nsteps; ++s) {
         const int c = list[first + (s / NSUB) * stride];
         const int key0 = c * BC + (s % NSUB) * kSub;
         const bool diag = c == ct, more = s + 1 < nsteps;
-        const int key_next = more ? list[first + ((s + 1) / NSUB) * stride] * BC + ((s + 1) % NSUB) * kSub : 0;
+        const int c_next = more ? list[first + ((s + 1) / NSUB) * stride] : 0;
+        const int sub_next = ((s + 1) % NSUB) * kSub;
         float bias2 = 0.f;
         if (!diag)
-            bias2 = a.rc.kind == 0 ? a.rc.sigma2 * (xs[c] - tau)
-                                   : a.rc.bscale2 * log2f(fmaxf(__fsub_rn(xs[c], tau), 1e-37f));
+            bias2 = a.rc.kind == kKindTopk ? 0.f                 // top-k: uniform prior
+                    : a.rc.kind == 0 ? a.rc.sigma2 * (xs[c] - tau)
+                                     : a.rc.bscale2 * log2f(fmaxf(__fsub_rn(xs[c], tau), 1e-37f));
         cp_async_wait<1>();
         __syncwarp();
         float acc[4][4];
         qk_sub<D>(acc, qf, ks);
         __syncwarp();
         if (more) {
-            load_sub<D>(ks, kp, key_next, a.cap);
+            load_sub<D>(ks, kv_base(a.k, c_next), sub_next, kv_rows(c_next));
             cp_async_commit();
         }
         uint32_t pa[2][4];
@@ -232,7 +292,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
         pv_sub<D>(st, pa, vs);
         __syncwarp();
         if (more) {
-            load_sub<D>(vs, vp, key_next, a.cap);
+            load_sub<D>(vs, kv_base(a.v, c_next), sub_next, kv_rows(c_next));
             cp_async_commit();
         }
     }

@@ -35,6 +35,9 @@ struct DecodeArgs {
     const void *q, *k, *v;    // q [B,Hq,D]; caches [B,Hkv,cap,D]
     const int32_t *seq_lens;  // [B]
     const float *summary;     // [B,Hkv,cap/Bc,D]
+    const float *head_cls;    // [Hkv,D] (estimate_diagonal only)
+    const int32_t *block_table;  // paged cache: [B, max_blocks] page of each logical chunk, or null
+    int max_blocks, n_pages;  // paged cache: table row length, pages in the pools
     void *out;                // [B,Hq,D]
     float *p;                 // [B,Hkv,Ccap] or null
     uint64_t *mask;           // [B,Hkv,Wcap] or null
@@ -46,11 +49,16 @@ struct DecodeArgs {
 
 cudaError_t launch_stage0(const StageArgs &a, const int32_t *seq_lens, int n_recent,
                           cudaStream_t st);
+// Stage 0 over the newest complete chunks of a paged cache: k_pool [n_pages, Hkv, Bc, D],
+// summary_pool [n_pages, Hkv, D], block_table [B, max_blocks].
+cudaError_t launch_stage0_paged(const StageArgs &a, const int32_t *seq_lens, int n_recent,
+                                const int32_t *block_table, int max_blocks, int n_pages,
+                                cudaStream_t st);
 cudaError_t launch_route(const StageArgs &a, cudaStream_t st);
 int route_rows_per_cta(int C, int D);   // 0 if C is too large for the routing kernel
 cudaError_t launch_attend(const StageArgs &a, cudaStream_t st);
 // The Stage 2 kernel launch_attend picks for these arguments, and its name.
-enum class AttendKernel { kNone, kPair, kFa, kTc, kWarp };
+enum class AttendKernel { kNone, kPair, kPp, kFa, kTc, kWarp };
 AttendKernel attend_kernel(const StageArgs &a);
 const char *attend_kernel_name(AttendKernel k);
 bool attend_tc_supported(const StageArgs &a);
@@ -58,6 +66,8 @@ cudaError_t launch_attend_tc(const StageArgs &a, cudaStream_t st);
 bool attend_fa_supported(const StageArgs &a);
 size_t attend_fa_vt_bytes(int B, int Hkv, int T, int D);
 cudaError_t launch_attend_fa(const StageArgs &a, cudaStream_t st);
+bool attend_pp_supported(const StageArgs &a);
+cudaError_t launch_attend_pp(const StageArgs &a, cudaStream_t st);
 bool attend_pair_supported(const StageArgs &a);
 cudaError_t launch_attend_pair(const StageArgs &a, cudaStream_t st);
 cudaError_t launch_vtranspose(const void *v, void *vt, int BHkv, int T, int D, cudaStream_t st);

@@ -13,7 +13,9 @@
 //      64-byte reads per chunk), two chunks per lane, RT row accumulators per chunk in
 //      registers, qbar from shared memory (each load feeds both chunks), slices combined with
 //      route_dot's fixed order
-//   3. one warp per row solves tau (warp_entmax_tau) and emits the mask words by ballot,
+//   3. with estimate_diagonal, one warp per row adds the diagonal chunk's score against its
+//      estimated summary (diag_dot) as one more candidate;
+//   4. one warp per row solves tau (warp_entmax_tau) and emits the mask words by ballot,
 //      tau, and optionally the dense p row.
 // No top-k list and no per-row index list is ever written.
 #include "dash_common.cuh"
@@ -43,7 +45,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(StageArgs a) {
     const int bg = blockIdx.y, b = bg / a.Hkv, g = bg % a.Hkv;
     const int t0 = a.t_begin + blockIdx.x * RT;
     const int ct = t0 / a.Bc;                     // every row of the tile shares c_t
-    const int n = ct;                             // routable chunks
+    const int n = dash_check(ct <= a.Cf, a.status) ? ct : a.Cf;   // routable chunks
     const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(a.q);
     const long long hstride = (long long)a.T * D;
 
@@ -121,12 +123,61 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(StageArgs a) {
     }
     __syncthreads();
 
+    // estimate_diagonal: the diagonal chunk's score joins each row's candidates as entry n.
+    const int n_eff = n + (a.rc.est_diag ? 1 : 0);
+    if (a.rc.est_diag) {
+        const __nv_bfloat16 *kd = reinterpret_cast<const __nv_bfloat16 *>(a.k) +
+                                  ((long long)bg * a.T + (long long)ct * a.Bc) * D;
+        for (int r = warp; r < RT; r += kRouteThreads / 32) {
+            const int t = t0 + r;
+            if (t >= a.t_end) break;
+            const float dd = diag_dot<D>(kd, t - ct * a.Bc + 1, a.head_cls + (long long)g * D,
+                                         qbar + r * D, a.rc.inv_sqrt_d);
+            if (lane == 0) xs[r * xstride + n] = __fmul_rn(dd, scale);
+        }
+        __syncthreads();
+    }
+
     for (int r = warp; r < RT; r += kRouteThreads / 32) {
         const int t = t0 + r;
         if (t >= a.t_end) break;
         const long long row = (long long)bg * a.T + t;
         const float *x = xs + r * xstride;
-        float tau = n > 0 ? warp_entmax_tau(x, n, a.rc, a.status) : __int_as_float(0x7fc00000);
+        if (a.rc.kind == kKindTopk) {
+            // Top-k: the topk highest scores (all of them when there are no more), lower
+            // index first on ties; p uniform over the selection; tau = the lowest selected.
+            const bool all = n <= a.rc.topk;
+            int need = 0;
+            uint32_t key = 0;
+            if (!all) key = warp_topk_key(x, n, a.rc.topk, need);
+            float tau = __int_as_float(0x7fc00000);
+            if (n > 0 && all) {
+                float mn = INFINITY;
+                for (int c = lane; c < n; c += 32) mn = fminf(mn, x[c]);
+                tau = -warp_max(-mn);
+            } else if (n > 0) {
+                tau = key_f32(key);
+            }
+            if (lane == 0) a.tau[row] = tau;
+            const float pv = n > 0 ? 1.f / (float)min(n, a.rc.topk) : 0.f;
+            uint64_t *mrow = a.mask + row * a.W;
+            float *prow = a.p ? a.p + row * a.C : nullptr;
+            int run = 0;
+            for (int w = 0; w < a.W; ++w) {
+                const int c0 = w * 64 + lane, c1 = c0 + 32;
+                const bool s0 = topk_selected(x, c0, n, all, key, need, run);
+                const bool s1 = topk_selected(x, c1, n, all, key, need, run);
+                const unsigned lo = __ballot_sync(kFull, c0 == ct || s0);
+                const unsigned hi = __ballot_sync(kFull, c1 == ct || s1);
+                if (lane == (w & 31)) mrow[w] = ((uint64_t)hi << 32) | lo;
+                if (prow) {
+                    if (c0 < a.C) prow[c0] = s0 ? pv : 0.f;
+                    if (c1 < a.C) prow[c1] = s1 ? pv : 0.f;
+                }
+            }
+            continue;
+        }
+        float tau = n_eff > 0 ? warp_entmax_tau(x, n_eff, a.rc, a.status) : __int_as_float(0x7fc00000);
         if (lane == 0) a.tau[row] = tau;
         uint64_t *mrow = a.mask + row * a.W;
         for (int w = 0; w < a.W; ++w) {
@@ -140,7 +191,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route(StageArgs a) {
             float *prow = a.p + row * a.C;
             for (int c = lane; c < a.C; c += 32) {
                 float val = 0.f;
-                if (c < n) {
+                if (c < n_eff) {
                     if (a.rc.kind == 0) {
                         val = expf(x[c] - tau);
                     } else {

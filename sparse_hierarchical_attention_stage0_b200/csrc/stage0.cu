@@ -68,11 +68,15 @@ __device__ __forceinline__ void summarize_chunk_warp(const __nv_bfloat16 *ks, co
 
 // Grid: one warp per unit.  Prefill units are (b, g, c) for every complete chunk; decode
 // units (seq_lens != nullptr) are (b, g, r) = the r-th most recent complete chunk.
+// Paged caches (block_table != nullptr): the keys of logical chunk c of sequence b live in
+// page block_table[b * max_blocks + c] of k [n_pages, Hkv, BC, D], and its summary goes to
+// summary [n_pages, Hkv, D]; a page index out of [0, n_pages) is reported and skipped.
 template <int D, int BC>
 __global__ void __launch_bounds__(kStage0Warps * 32)
 k_stage0(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ head_cls,
          float *__restrict__ summary, int B, int Hkv, int T, int Cf, const int32_t *seq_lens,
-         int n_recent, uint32_t *status, int test_stall) {
+         int n_recent, uint32_t *status, int test_stall, const int32_t *block_table,
+         int max_blocks, int n_pages) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t bars[kStage0Warps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -96,8 +100,19 @@ k_stage0(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ head_cls
         c = L / BC - 1 - r;
         if (c < 0) return;
     }
+    if (!dash_check(c >= 0 && c < Cf && b < B && (long long)(c + 1) * BC <= T, status)) return;
     __nv_bfloat16 *ks = reinterpret_cast<__nv_bfloat16 *>(smem_raw) + (size_t)warp * BC * D;
     const __nv_bfloat16 *src = k + (((long long)b * Hkv + g) * T + (long long)c * BC) * D;
+    float *dst = summary + (((long long)b * Hkv + g) * Cf + c) * D;
+    if (block_table) {
+        const int page = block_table[(long long)b * max_blocks + c];
+        if (page < 0 || page >= n_pages) {
+            if (lane == 0) report(status, DASH_ERR_INVALID_ARGUMENT);
+            return;
+        }
+        src = k + ((long long)page * Hkv + g) * BC * D;
+        dst = summary + ((long long)page * Hkv + g) * D;
+    }
     constexpr uint32_t kBytes = BC * D * sizeof(__nv_bfloat16);
     if (lane == 0) {
         mbar_init(&bars[warp], 1);
@@ -115,13 +130,13 @@ k_stage0(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ head_cls
         if (!test_stall) mbar_wait_bounded(&bars[warp], 0);   // one more bounded wait for the copy
         return;
     }
-    summarize_chunk_warp<D, BC>(ks, head_cls + (size_t)g * D,
-                                summary + (((long long)b * Hkv + g) * Cf + c) * D);
+    summarize_chunk_warp<D, BC>(ks, head_cls + (size_t)g * D, dst);
 }
 
 template <int D, int BC>
 static cudaError_t launch_stage0_t(const StageArgs &a, const int32_t *seq_lens, int n_recent,
-                                   cudaStream_t st) {
+                                   cudaStream_t st, const int32_t *block_table = nullptr,
+                                   int max_blocks = 0, int n_pages = 0) {
     long long units = seq_lens ? (long long)a.B * a.Hkv * n_recent
                                : (long long)a.B * a.Hkv * a.Cf;
     if (units == 0) return cudaSuccess;
@@ -133,7 +148,7 @@ static cudaError_t launch_stage0_t(const StageArgs &a, const int32_t *seq_lens, 
     unsigned grid = (unsigned)((units + kStage0Warps - 1) / kStage0Warps);
     kern<<<grid, kStage0Warps * 32, smem, st>>>(
         reinterpret_cast<const __nv_bfloat16 *>(a.k), a.head_cls, a.summary, a.B, a.Hkv, a.T,
-        a.Cf, seq_lens, n_recent, a.status, a.test_stall);
+        a.Cf, seq_lens, n_recent, a.status, a.test_stall, block_table, max_blocks, n_pages);
     return cudaGetLastError();
 }
 
@@ -143,6 +158,20 @@ cudaError_t launch_stage0(const StageArgs &a, const int32_t *seq_lens, int n_rec
     if (a.D == 128 && a.Bc == 128) return launch_stage0_t<128, 128>(a, seq_lens, n_recent, st);
     if (a.D == 64 && a.Bc == 64) return launch_stage0_t<64, 64>(a, seq_lens, n_recent, st);
     if (a.D == 64 && a.Bc == 128) return launch_stage0_t<64, 128>(a, seq_lens, n_recent, st);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_stage0_paged(const StageArgs &a, const int32_t *seq_lens, int n_recent,
+                                const int32_t *block_table, int max_blocks, int n_pages,
+                                cudaStream_t st) {
+    if (a.D == 128 && a.Bc == 64)
+        return launch_stage0_t<128, 64>(a, seq_lens, n_recent, st, block_table, max_blocks, n_pages);
+    if (a.D == 128 && a.Bc == 128)
+        return launch_stage0_t<128, 128>(a, seq_lens, n_recent, st, block_table, max_blocks, n_pages);
+    if (a.D == 64 && a.Bc == 64)
+        return launch_stage0_t<64, 64>(a, seq_lens, n_recent, st, block_table, max_blocks, n_pages);
+    if (a.D == 64 && a.Bc == 128)
+        return launch_stage0_t<64, 128>(a, seq_lens, n_recent, st, block_table, max_blocks, n_pages);
     return cudaErrorInvalidValue;
 }
 

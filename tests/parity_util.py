@@ -61,3 +61,30 @@ def check_output(o_gpu, o_or, tag=""):
     assert err.max() <= O_MAX_TOL, f"{tag}: O max abs err {err.max():.3e}"
     assert err.mean() <= O_MEAN_TOL, f"{tag}: O mean abs err {err.mean():.3e}"
     return float(err.max()), float(err.mean())
+
+
+def check_topk(mask_bits, p_gpu, p_or, m_or, rows, chunk_size, k, tol=1e-4, tag=""):
+    """Top-k routing: every row selects min(k, c_t) routed chunks plus its diagonal; the
+    selection is a valid top-k of the oracle's scores up to `tol` (a selected chunk's oracle
+    margin s - theta >= -tol, an unselected one's <= tol: near-ties may fall either way under
+    fp32 rounding), and p is uniform over it.  Returns the boolean per-row mask of rows whose
+    selection equals the oracle's exactly."""
+    rows = np.asarray(rows)
+    C = p_or.shape[-1]
+    ct = rows // chunk_size
+    col = np.arange(C)
+    routed = col[None, :] < ct[:, None]
+    diag = col[None, :] == ct[:, None]
+    above = col[None, :] > ct[:, None]
+    assert mask_bits[..., diag].all(), f"{tag}: diagonal bit missing"
+    assert not mask_bits[..., above].any(), f"{tag}: bit above the diagonal set"
+    sel = mask_bits & routed
+    ke = np.minimum(k, ct)
+    assert (sel.sum(-1) == ke).all(), f"{tag}: selection sizes differ from min(k, c_t)"
+    m = np.where(routed, m_or, 0.0)
+    assert (m[sel] >= -tol).all(), f"{tag}: a selected chunk lies below the k-th score"
+    assert (m[routed & ~sel] <= tol).all(), f"{tag}: an unselected chunk lies above the k-th score"
+    want = np.where(sel, 1.0 / np.maximum(ke, 1)[:, None], 0.0)
+    if p_gpu is not None:
+        assert np.abs(p_gpu - want).max() <= 1e-6, f"{tag}: p is not uniform over the selection"
+    return (sel == ((p_or > 0) & routed)).all(-1)

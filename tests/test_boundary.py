@@ -83,7 +83,8 @@ FAKE = 1 << 20      # a 256-aligned fake device address; never dereferenced on t
     (dict(gamma=0.0), 1),
     (dict(sigma=-1.0), 1),
     (dict(flags=64), 1),                        # unknown flag bit
-    (dict(flags=4), 2),                         # estimate_diagonal: reserved
+    (dict(topk=-1), 1),
+    (dict(topk=8, flags=4), 2),                 # top-k with estimate_diagonal
     (dict(head_dim=96), 2),
     (dict(chunk_size=32), 2),
     (dict(heads_q=6, heads_kv=2), 2),           # G = 3 neither divides 16 nor is a multiple
@@ -96,6 +97,17 @@ def test_prefill_rejects_bad_parameters_before_launch(dash, kw, code):
     rc = dash.lib.dash_prefill(ctypes.byref(prm), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None,
                                FAKE, 1 << 40, None)
     assert rc == code
+
+
+def test_estimate_diagonal_is_accepted_by_prefill_and_refused_by_route(dash):
+    prm = _p(dash, flags=dash.FLAG_ESTIMATE_DIAGONAL)
+    assert dash.prefill_workspace_size(prm) == dash.prefill_workspace_size(_p(dash))
+    rc = dash.lib.dash_route(ctypes.byref(prm), FAKE, FAKE, FAKE, None, FAKE, FAKE, 256, None)
+    assert rc == 2                                  # needs the keys: dash_prefill only
+    # decode with the flag needs head_cls
+    rc = dash.lib.dash_decode(ctypes.byref(prm), FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, None,
+                              None, FAKE, 256, None)
+    assert rc == 1
 
 
 def test_test_hook_flags_are_accepted(dash):
@@ -143,15 +155,15 @@ def test_prefill_host_rejects_bad_arguments_before_any_copy(dash):
 def test_decode_and_cache_reject_bad_arguments(dash):
     prm = _p(dash, seq_len=65792)
     d = dash.lib.dash_decode
-    assert d(ctypes.byref(prm), FAKE, FAKE, FAKE, None, FAKE, FAKE, None, None, FAKE, 256,
+    assert d(ctypes.byref(prm), FAKE, FAKE, FAKE, None, FAKE, None, FAKE, None, None, FAKE, 256,
              None) == 1                                             # no seq_lens
-    assert d(ctypes.byref(prm), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, 255,
+    assert d(ctypes.byref(prm), FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, None, FAKE, 255,
              None) == 3
     dense = _p(dash, seq_len=65792, flags=1)
-    assert d(ctypes.byref(dense), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, 256,
+    assert d(ctypes.byref(dense), FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, None, FAKE, 256,
              None) == 2
     wide = _p(dash, heads_q=64, heads_kv=2, seq_len=65792)         # G = 32: decode is G <= 16
-    assert d(ctypes.byref(wide), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, 256,
+    assert d(ctypes.byref(wide), FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, None, FAKE, 256,
              None) == 2
     u = dash.lib.dash_update_chunk_cache
     assert u(ctypes.byref(prm), FAKE, FAKE, FAKE, 0, FAKE, FAKE, 256, None) == 1   # n_recent 0
@@ -171,7 +183,7 @@ def test_stage_entry_points_reject_missing_outputs(dash):
 def test_attend_kernel_name_follows_the_dispatch(dash):
     """The library names the Stage 2 kernel it picks (host only, nothing launched)."""
     big = 1 << 40
-    assert dash.attend_kernel_name(_p(dash), big) == "k_attend_fa"
+    assert dash.attend_kernel_name(_p(dash), big) == "k_attend_pp"
     assert dash.attend_kernel_name(_p(dash), 256) == "k_attend_tc"          # no room for V^T
     assert dash.attend_kernel_name(_p(dash, flags=1), big) == "k_attend_pair"
     assert dash.attend_kernel_name(_p(dash, flags=2), big) == "k_attend_pair"

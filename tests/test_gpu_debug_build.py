@@ -1,0 +1,108 @@
+"""The bounds-checking build libdash_debug.so (the same kernels compiled with DASH_DEBUG: every
+checked index is compared with its buffer's bounds, a failed check reports DASH_ERR_BOUNDS
+through the status word and skips the access).  On odd shapes (ragged sequence lengths,
+batch > 1, every Stage 2 kernel, sliced prefill from host memory, decode with ragged cache
+lengths) it must report no violation and give the release library's output bit for bit."""
+import pytest
+import torch
+
+from dash_inputs import PrefillConfig, make_prefill
+
+pytestmark = pytest.mark.gpu
+dev = "cuda"
+
+
+@pytest.fixture(scope="module")
+def libs():
+    import sparse_hierarchical_attention_stage0_b200 as dash
+    return dash, dash.lib, dash.load_library(dash.LIB_DEBUG_PATH)
+
+
+def _both(dash, rel, dbg, monkeypatch, fn):
+    """fn() run with the release and then the debug library behind the binding."""
+    monkeypatch.setattr(dash, "lib", rel)
+    a = fn()
+    torch.cuda.synchronize()
+    monkeypatch.setattr(dash, "lib", dbg)
+    b = fn()
+    torch.cuda.synchronize()
+    monkeypatch.setattr(dash, "lib", rel)
+    return a, b
+
+
+@pytest.mark.parametrize("B,G,D,Bc,T,flags", [
+    (2, 16, 128, 64, 1100 + 5, {}),                          # two-tile tensor-core kernel
+    (1, 8, 128, 128, 1500 + 3, {}),
+    (1, 4, 128, 128, 777, {}),                               # warp-MMA kernel
+    (2, 1, 64, 64, 333, {}),
+    (2, 8, 128, 128, 700, {"dense": True}),                  # pairs of SMs
+    (1, 16, 128, 64, 640 + 17, {"estimate_diagonal": True}),
+])
+def test_debug_build_matches_release_without_violations(libs, monkeypatch, B, G, D, Bc, T, flags):
+    dash, rel, dbg = libs
+    Hkv = 2
+    q, k, v, hc = (x.to(dev) for x in make_prefill(
+        PrefillConfig("dbg", B, G * Hkv, Hkv, T, D, Bc, 1.5, planted=True, n_max=6, seed=90 + G)))
+    dense = flags.get("dense", False)
+    fl = (dash.FLAG_DENSE if dense else 0) | (dash.FLAG_ESTIMATE_DIAGONAL if flags.get("estimate_diagonal") else 0)
+    prm = dash.make_params(B, G * Hkv, Hkv, T, D, Bc, 1.5, enable_gqa=True, flags=fl)
+
+    def run():
+        ws = dash.workspace(dash.prefill_workspace_size(prm), dev)
+        r = dash.prefill(q, k, v, None if dense else hc, Bc, 1.5, enable_gqa=True, ws=ws,
+                         return_active_blocks=not dense, return_p=not dense, **flags)
+        r = r if isinstance(r, dict) else {"out": r}
+        r["status"] = dash.read_device_status(ws)
+        return r
+
+    a, b = _both(dash, rel, dbg, monkeypatch, run)
+    assert a["status"] == 0 and b["status"] == 0, (a["status"], b["status"])
+    for key in ("out", "p", "active_blocks"):
+        if a.get(key) is not None:
+            assert torch.equal(a[key], b[key]), key
+
+
+def test_debug_build_host_prefill_and_decode(libs, monkeypatch):
+    dash, rel, dbg = libs
+    B, Hkv, G, L, D, Bc = 3, 2, 16, 1300 + 9, 128, 64
+    q, k, v, hc = make_prefill(PrefillConfig("dbg", B, G * Hkv, Hkv, L, D, Bc, 1.5, planted=True,
+                                             n_max=6, seed=99))
+    qd, kd, vd, hcd = (x.to(dev) for x in (q, k, v, hc))
+    hq, hk, hv, hhc = (x.contiguous().pin_memory() for x in (q, k, v, hc))
+    prm = dash.make_params(B, G * Hkv, Hkv, L, D, Bc, 1.5, enable_gqa=True)
+    ws = dash.workspace(dash.prefill_workspace_size(prm), dev)
+
+    def host():
+        ho = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+        bo = torch.empty_like(qd)
+        dash.prefill_host(hq, hk, hv, hhc, ho, qd.clone(), kd.clone(), vd.clone(), hcd.clone(), bo,
+                          Bc, 1.5, enable_gqa=True, n_slices=5, ws=ws)
+        torch.cuda.current_stream().synchronize()
+        assert dash.read_device_status(ws) == 0
+        return ho
+
+    a, b = _both(dash, rel, dbg, monkeypatch, host)
+    assert torch.equal(a, b)
+
+    cap = L + 100
+    kc = torch.zeros(B, Hkv, cap, D, dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    kc[:, :, :L] = kd
+    vc[:, :, :L] = vd
+    lens = [L, Bc * 5, 17]
+    seq = torch.tensor(lens, dtype=torch.int32, device=dev)
+    qs = torch.stack([qd[b, :, lens[b] - 1] for b in range(B)])
+
+    def dec():
+        cache = torch.zeros(B, Hkv, cap // Bc, D, device=dev)
+        wsu, wsd = dash.workspace(256, dev), dash.workspace(256, dev)
+        dash.update_chunk_cache(kc, hcd, seq, cache, heads_q=G * Hkv, chunk_size=Bc,
+                                n_recent=cap // Bc, ws=wsu)
+        r = dash.decode(qs, kc, vc, seq, cache, Bc, return_p=True, return_active_blocks=True, ws=wsd)
+        assert dash.read_device_status(wsu) == 0 and dash.read_device_status(wsd) == 0
+        r["cache"] = cache
+        return r
+
+    a, b = _both(dash, rel, dbg, monkeypatch, dec)
+    for key in ("out", "p", "active_blocks", "cache"):
+        assert torch.equal(a[key], b[key]), key

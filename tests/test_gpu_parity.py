@@ -371,3 +371,163 @@ def test_decode_reports_bad_seq_len(dash):
     ws = dash.workspace(256, dev)
     dash.decode(q, kc, kc, seq, cache, 64, enable_gqa=True, ws=ws)
     assert dash.read_device_status(ws) == 1
+
+
+# ------------------------------------------------------------------------------ estimate_diagonal
+@pytest.mark.parametrize("alpha", [1.0, 1.5, 2.0])
+@pytest.mark.parametrize("G,D,Bc,T", [(16, 128, 64, 1100 + 5), (4, 128, 128, 1300), (1, 64, 64, 777)])
+def test_prefill_estimate_diagonal_matches_oracle(dash, alpha, G, D, Bc, T):
+    """estimate_diagonal: the diagonal chunk joins the entmax with its summary estimated over
+    the keys each row can see; p[.., c_t] is its probability, the routed chunks share the rest,
+    Stage 2 attends the diagonal with bias 0 as before."""
+    Hkv = 2
+    q, k, v, hc = make_prefill(_cfg(1, G * Hkv, Hkv, T, D, Bc, alpha, seed=70 + G))
+    res = dash.prefill(*_to(q, k, v, hc), chunk_size=Bc, alpha=alpha, enable_gqa=True,
+                       estimate_diagonal=True, return_p=True, return_active_blocks=True)
+    torch.cuda.synchronize()
+    assert dash.read_device_status(res["ws"]) == 0
+    ref = oracle.prefill(q, k, v, hc, Bc, alpha, estimate_diagonal=True)
+    C = ref["p"].shape[-1]
+    p = res["p"].cpu().double().numpy()
+    check_routing(unpack_mask(res["active_blocks"], C), p, ref["p"], ref["m"], np.arange(T), Bc,
+                  alpha, tag=f"estimate_diagonal G={G} a={alpha}")
+    ct = np.arange(T) // Bc
+    pdiag = p[0][:, np.arange(T), ct]
+    assert np.abs(p[0].sum(-1) - 1).max() < 1e-4          # the diagonal is part of the simplex
+    if alpha < 2:
+        assert (pdiag > 0).any()
+    check_output(res["out"].cpu().float().numpy(), ref["O"], tag=f"estimate_diagonal G={G}")
+
+
+def test_decode_estimate_diagonal_matches_oracle(dash):
+    B, Hkv, G, L, D, Bc = 3, 2, 16, 1500, 128, 64
+    q, k, v, hc = make_prefill(_cfg(B, G * Hkv, Hkv, L, D, Bc, 1.5, seed=71))
+    qd, kd, vd, hcd = _to(q, k, v, hc)
+    cap = L + 37
+    kc = torch.zeros(B, Hkv, cap, D, dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    kc[:, :, :L] = kd
+    vc[:, :, :L] = vd
+    cache = torch.zeros(B, Hkv, cap // Bc, D, device=dev)
+    lens = [L, Bc * 3 + 1, 40]                                # the last row routes to chunk 0 alone
+    seq = torch.tensor(lens, dtype=torch.int32, device=dev)
+    dash.update_chunk_cache(kc, hcd, seq, cache, heads_q=G * Hkv, chunk_size=Bc, n_recent=cap // Bc)
+    qs = torch.stack([qd[b, :, lens[b] - 1] for b in range(B)])
+    ws = dash.workspace(256, dev)
+    dec = dash.decode(qs, kc, vc, seq, cache, Bc, enable_gqa=True, return_p=True,
+                      return_active_blocks=True, ws=ws, estimate_diagonal=True, head_cls=hcd)
+    pre = dash.prefill(qd, kd, vd, hcd, Bc, enable_gqa=True, estimate_diagonal=True, return_p=True)
+    torch.cuda.synchronize()
+    assert dash.read_device_status(ws) == 0
+    ref = oracle.decode(qs.cpu(), kc.cpu(), vc.cpu(), hc, lens, Bc, 1.5, estimate_diagonal=True)
+    check_output(dec["out"].cpu().float().numpy(), ref["O"], tag="decode estimate_diagonal")
+    bits = unpack_mask(dec["active_blocks"], ref["p"].shape[-1])
+    for b in range(B):
+        t = lens[b] - 1
+        check_routing(bits[b][:, None], dec["p"][b][:, None].cpu().double().numpy(),
+                      ref["p"][b][:, None], ref["m"][b][:, None], [t], Bc, 1.5, tag="decode est")
+        C = (L + Bc - 1) // Bc
+        assert torch.equal(dec["p"][b, :, :C], pre["p"][b, :, t])        # same routing as prefill
+    assert torch.allclose(dec["p"][2, :, 0], torch.ones(Hkv, device=dev))
+
+
+# ------------------------------------------------------------------------------ top-k routing
+@pytest.mark.parametrize("G,D,Bc,T,k", [(16, 128, 64, 1100 + 5, 4), (4, 128, 128, 1500, 3),
+                                        (1, 64, 64, 777, 2), (8, 128, 128, 1300, 64)])
+def test_prefill_topk_matches_oracle(dash, G, D, Bc, T, k):
+    """Top-k routing: the k highest-scoring chunks plus the diagonal, a uniform prior in Stage 2
+    (the fixed-k selection of the hierarchical baselines); k = 64 exceeds every row's c_t here,
+    so all visible chunks are selected."""
+    from parity_util import check_topk
+    Hkv = 2
+    q, k_, v, hc = make_prefill(_cfg(1, G * Hkv, Hkv, T, D, Bc, 1.5, seed=80 + G))
+    res = dash.prefill(*_to(q, k_, v, hc), chunk_size=Bc, enable_gqa=True, topk=k,
+                       return_p=True, return_active_blocks=True)
+    torch.cuda.synchronize()
+    assert dash.read_device_status(res["ws"]) == 0
+    ref = oracle.prefill(q, k_, v, hc, Bc, 1.5, topk=k)
+    C = ref["p"].shape[-1]
+    same = check_topk(unpack_mask(res["active_blocks"], C)[0], res["p"].cpu().double().numpy()[0],
+                      ref["p"][0], ref["m"][0], np.arange(T), Bc, k, tag=f"topk G={G}")
+    assert same.mean() >= 0.999, same.mean()
+    rows = np.nonzero(same.all(0))[0]                      # rows whose selection is the oracle's
+    check_output(res["out"].cpu().float().numpy()[:, :, rows], ref["O"][:, :, rows], tag="topk")
+
+
+def test_decode_topk_equals_prefill_row(dash):
+    B, Hkv, G, L, D, Bc, K = 3, 2, 16, 1500, 128, 64, 5
+    q, k, v, hc = make_prefill(_cfg(B, G * Hkv, Hkv, L, D, Bc, 1.5, seed=81))
+    qd, kd, vd, hcd = _to(q, k, v, hc)
+    pre = dash.prefill(qd, kd, vd, hcd, Bc, enable_gqa=True, topk=K, return_p=True,
+                       return_active_blocks=True)
+    cap = L + 37
+    kc = torch.zeros(B, Hkv, cap, D, dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    kc[:, :, :L] = kd
+    vc[:, :, :L] = vd
+    cache = torch.zeros(B, Hkv, cap // Bc, D, device=dev)
+    lens = [L, Bc * 4 + 3, 100]
+    seq = torch.tensor(lens, dtype=torch.int32, device=dev)
+    dash.update_chunk_cache(kc, hcd, seq, cache, heads_q=G * Hkv, chunk_size=Bc, n_recent=cap // Bc)
+    qs = torch.stack([qd[b, :, lens[b] - 1] for b in range(B)])
+    ws = dash.workspace(256, dev)
+    dec = dash.decode(qs, kc, vc, seq, cache, Bc, enable_gqa=True, topk=K, return_p=True,
+                      return_active_blocks=True, ws=ws)
+    torch.cuda.synchronize()
+    assert dash.read_device_status(ws) == 0
+    C = (L + Bc - 1) // Bc
+    for b in range(B):
+        t = lens[b] - 1
+        assert torch.equal(dec["p"][b, :, :C], pre["p"][b, :, t])
+        assert torch.equal(dec["active_blocks"][b, :, :(C + 63) // 64], pre["active_blocks"][b, :, t])
+    ref = oracle.decode(qs.cpu(), kc.cpu(), vc.cpu(), hc, lens, Bc, 1.5, topk=K)
+    check_output(dec["out"].cpu().float().numpy(), ref["O"], tag="decode topk")
+
+
+# ------------------------------------------------------------------------------ paged KV cache
+def test_paged_decode_equals_contiguous_decode(dash):
+    """A paged cache (pages of one chunk, a per-sequence block table with the pages scattered
+    through the pools) gives the contiguous cache's summaries, routing and output bit for bit,
+    and the oracle's output on the gathered cache; a page index outside the pools is reported
+    through the status word."""
+    B, Hkv, G, D, Bc = 3, 2, 16, 128, 64
+    max_blocks = 24
+    cap = max_blocks * Bc
+    q, k, v, hc = make_prefill(_cfg(B, G * Hkv, Hkv, cap, D, Bc, 1.5, seed=85))
+    qd, kd, vd, hcd = _to(q, k, v, hc)
+    lens = [cap, Bc * 7 + 5, 64]
+    seq = torch.tensor(lens, dtype=torch.int32, device=dev)
+    n_pages = B * max_blocks + 5
+    perm = torch.randperm(n_pages, generator=torch.Generator().manual_seed(3))[:B * max_blocks]
+    table = perm.view(B, max_blocks).to(torch.int32).to(dev)
+    k_pool = torch.zeros(n_pages, Hkv, Bc, D, dtype=torch.bfloat16, device=dev)
+    v_pool = torch.zeros_like(k_pool)
+    for b in range(B):
+        for c in range(max_blocks):
+            k_pool[table[b, c]] = kd[b, :, c * Bc:(c + 1) * Bc]
+            v_pool[table[b, c]] = vd[b, :, c * Bc:(c + 1) * Bc]
+    s_pool = torch.zeros(n_pages, Hkv, D, device=dev)
+    dash.update_chunk_cache_paged(k_pool, hcd, table, seq, s_pool, G * Hkv, Bc, n_recent=max_blocks)
+    cache = torch.zeros(B, Hkv, max_blocks, D, device=dev)
+    dash.update_chunk_cache(kd, hcd, seq, cache, heads_q=G * Hkv, chunk_size=Bc, n_recent=max_blocks)
+    qs = torch.stack([qd[b, :, lens[b] - 1] for b in range(B)])
+    ws = dash.workspace(256, dev)
+    for kw in (dict(), dict(topk=3), dict(estimate_diagonal=True, head_cls=hcd)):
+        pg = dash.decode_paged(qs, k_pool, v_pool, table, seq, s_pool, Bc, return_p=True,
+                               return_active_blocks=True, ws=ws, **kw)
+        ct = dash.decode(qs, kd, vd, seq, cache, Bc, return_p=True, return_active_blocks=True, **kw)
+        torch.cuda.synchronize()
+        assert dash.read_device_status(ws) == 0
+        for key in ("out", "p", "active_blocks"):
+            assert torch.equal(pg[key], ct[key]), (kw, key)
+    for b in range(B):
+        for c in range(lens[b] // Bc):
+            assert torch.equal(s_pool[table[b, c]], cache[b, :, c])
+    ref = oracle.decode(qs.cpu(), k, v, hc, lens, Bc, 1.5)
+    out = dash.decode_paged(qs, k_pool, v_pool, table, seq, s_pool, Bc, ws=ws)
+    torch.cuda.synchronize()
+    check_output(out.cpu().float().numpy(), ref["O"], tag="paged decode")
+    bad = table.clone()
+    bad[1, 2] = n_pages + 7
+    dash.decode_paged(qs, k_pool, v_pool, bad, seq, s_pool, Bc, ws=ws)
+    assert dash.read_device_status(ws) == 1
