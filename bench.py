@@ -165,9 +165,9 @@ def active_stats(dash, q, k, v, hc, cfg):
 
 def tokens_per_tile(kernel: str, G: int) -> int:
     """Tokens whose rows share one Stage 2 work unit (and so walk the union of their routed
-    chunks) in the named kernel: 128 rows of G heads per tile (two tiles per SM pair or per ping-pong CTA), or 16
+    chunks) in the named kernel: 128 rows of G heads per tile (two tiles per SM pair), or 16
     rows per warp in the warp-MMA kernel."""
-    if kernel in ("k_attend_pair", "k_attend_pp"):
+    if kernel == "k_attend_pair":
         return max(1, 256 // G)
     if kernel in ("k_attend_fa", "k_attend_tc"):
         return max(1, 128 // G)
@@ -531,7 +531,7 @@ def bench_prefill(dash, cfg, args, dev, world, rank, full=True):
     # The Stage 2 kernel dash_attend runs with the bench's workspace (the library names it);
     # the 128-key-block kernels also transpose V (timed together with them as Stage 2).
     s2_kernel = dash.attend_kernel_name(prm, ws_a.numel())
-    with_vt = s2_kernel in ("k_attend_fa", "k_attend_pp", "k_attend_pair")
+    with_vt = s2_kernel in ("k_attend_fa", "k_attend_pair")
     s2_note = ", V^T transpose included" if with_vt else ""
     launches_per_step = 3 + (1 if with_vt else 0)   # k_stage0, k_route, [k_vtranspose,] Stage 2
     un = union_stats(stats.pop("words"), Bc, D, cfg.group, tokens_per_tile(s2_kernel, cfg.group))
@@ -641,7 +641,7 @@ def bench_sweep(dash, args, dev, world, rank):
                        "head_dim": cfg0.head_dim, "alphas": list(SWEEP_ALPHAS),
                        "chunk_sizes": list(SWEEP_CHUNKS), "parallelism": f"replicas x{world}",
                        "l2": "flushed (256 MiB write) before every timed step"},
-            "gpu_launches": sum(4 if c["union"]["kernel"] in ("k_attend_fa", "k_attend_pp", "k_attend_pair") else 3
+            "gpu_launches": sum(4 if c["union"]["kernel"] in ("k_attend_fa", "k_attend_pair") else 3
                                 for c in cells) * args.steps,
             "cells": cells}
 

@@ -219,9 +219,8 @@ dash_status_t dash_attend(const dash_params_t *params, const void *q, const void
 /* Name of the Stage 2 kernel dash_attend launches for these parameters with a workspace of
  * ws_bytes (dash_prefill with the same flags and a workspace that leaves ws_bytes after its
  * status word, tau, summaries and mask words picks the same one): "k_attend_pair" (dense
- * modes on pairs of SMs), "k_attend_pp" (128-key blocks, two ping-ponged query tiles per
- * CTA), "k_attend_fa" (128-key blocks, one query tile per CTA, where the two-tile kernel's
- * shared memory does not fit), "k_attend_tc" (64-key blocks, no V^T scratch) or "k_attend" (warp-level MMA: head_dim 64 or fewer than 8 query heads per KV
+ * modes on pairs of SMs), "k_attend_fa" (128-key blocks), "k_attend_tc" (64-key blocks, no
+ * V^T scratch) or "k_attend" (warp-level MMA: head_dim 64 or fewer than 8 query heads per KV
  * head).  Host only, launches nothing; "" on bad parameters or ws_bytes < 256.  Static
  * storage. */
 const char *dash_attend_kernel_name(const dash_params_t *params, size_t ws_bytes);

@@ -23,7 +23,7 @@ LIB = os.path.join(HERE, "libdash.so")
 BUILD = os.path.join(HERE, "_build")
 LIB_DEBUG = os.path.join(HERE, "libdash_debug.so")
 BUILD_DEBUG = os.path.join(HERE, "_build_debug")
-SOURCES = ["stage0.cu", "route.cu", "attend.cu", "attend_tc.cu", "attend_fa.cu", "attend_pp.cu", "attend_pair.cu", "vtranspose.cu",
+SOURCES = ["stage0.cu", "route.cu", "attend.cu", "attend_tc.cu", "attend_fa.cu", "attend_pair.cu", "vtranspose.cu",
            "decode.cu", "dash_api.cu", "dash_static_ws.cu"]
 HEADERS = ["dash_common.cuh", "kernels.cuh", "attn_warp.cuh", "tc_common.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -262,7 +262,6 @@ AttendKernel attend_kernel(const StageArgs &a) {
     if (a.t_begin != 0 || a.t_end != a.T) {
         // Row slices: only the 128-key-block kernels take a row range.
         if (a.vt && a.ignore_routing && attend_pair_supported(a)) return AttendKernel::kPair;
-        if (a.vt && attend_pp_supported(a)) return AttendKernel::kPp;
         if (a.vt && attend_fa_supported(a)) return AttendKernel::kFa;
         return AttendKernel::kNone;
     }
@@ -271,7 +270,6 @@ AttendKernel attend_kernel(const StageArgs &a) {
     // chunk forced active); with routing the larger union costs more than the halved copies
     // save (measured at 128K: 128 ms against 117 ms).
     if (a.vt && a.ignore_routing && attend_pair_supported(a)) return AttendKernel::kPair;
-    if (a.vt && attend_pp_supported(a)) return AttendKernel::kPp;
     if (a.vt && attend_fa_supported(a)) return AttendKernel::kFa;
     if (attend_tc_supported(a)) return AttendKernel::kTc;
     if ((a.D == 128 || a.D == 64) && (a.Bc == 64 || a.Bc == 128)) return AttendKernel::kWarp;
@@ -281,7 +279,6 @@ AttendKernel attend_kernel(const StageArgs &a) {
 const char *attend_kernel_name(AttendKernel k) {
     switch (k) {
         case AttendKernel::kPair: return "k_attend_pair";
-        case AttendKernel::kPp: return "k_attend_pp";
         case AttendKernel::kFa: return "k_attend_fa";
         case AttendKernel::kTc: return "k_attend_tc";
         case AttendKernel::kWarp: return "k_attend";
@@ -292,7 +289,6 @@ const char *attend_kernel_name(AttendKernel k) {
 cudaError_t launch_attend(const StageArgs &a, cudaStream_t st) {
     switch (attend_kernel(a)) {
         case AttendKernel::kPair: return launch_attend_pair(a, st);
-        case AttendKernel::kPp: return launch_attend_pp(a, st);
         case AttendKernel::kFa: return launch_attend_fa(a, st);
         case AttendKernel::kTc: return launch_attend_tc(a, st);
         case AttendKernel::kWarp:

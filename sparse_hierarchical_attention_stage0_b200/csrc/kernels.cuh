@@ -58,7 +58,7 @@ cudaError_t launch_route(const StageArgs &a, cudaStream_t st);
 int route_rows_per_cta(int C, int D);   // 0 if C is too large for the routing kernel
 cudaError_t launch_attend(const StageArgs &a, cudaStream_t st);
 // The Stage 2 kernel launch_attend picks for these arguments, and its name.
-enum class AttendKernel { kNone, kPair, kPp, kFa, kTc, kWarp };
+enum class AttendKernel { kNone, kPair, kFa, kTc, kWarp };
 AttendKernel attend_kernel(const StageArgs &a);
 const char *attend_kernel_name(AttendKernel k);
 bool attend_tc_supported(const StageArgs &a);
@@ -66,8 +66,6 @@ cudaError_t launch_attend_tc(const StageArgs &a, cudaStream_t st);
 bool attend_fa_supported(const StageArgs &a);
 size_t attend_fa_vt_bytes(int B, int Hkv, int T, int D);
 cudaError_t launch_attend_fa(const StageArgs &a, cudaStream_t st);
-bool attend_pp_supported(const StageArgs &a);
-cudaError_t launch_attend_pp(const StageArgs &a, cudaStream_t st);
 bool attend_pair_supported(const StageArgs &a);
 cudaError_t launch_attend_pair(const StageArgs &a, cudaStream_t st);
 cudaError_t launch_vtranspose(const void *v, void *vt, int BHkv, int T, int D, cudaStream_t st);

@@ -70,6 +70,5 @@ def test_tokens_per_tile_follow_the_kernels():
     assert bench.tokens_per_tile("k_attend_fa", 16) == 8
     assert bench.tokens_per_tile("k_attend_tc", 8) == 16
     assert bench.tokens_per_tile("k_attend_pair", 16) == 16
-    assert bench.tokens_per_tile("k_attend_pp", 8) == 32
     assert bench.tokens_per_tile("k_attend", 4) == 4
     assert bench.tokens_per_tile("k_attend", 32) == 1

@@ -183,7 +183,7 @@ def test_stage_entry_points_reject_missing_outputs(dash):
 def test_attend_kernel_name_follows_the_dispatch(dash):
     """The library names the Stage 2 kernel it picks (host only, nothing launched)."""
     big = 1 << 40
-    assert dash.attend_kernel_name(_p(dash), big) == "k_attend_pp"
+    assert dash.attend_kernel_name(_p(dash), big) == "k_attend_fa"
     assert dash.attend_kernel_name(_p(dash), 256) == "k_attend_tc"          # no room for V^T
     assert dash.attend_kernel_name(_p(dash, flags=1), big) == "k_attend_pair"
     assert dash.attend_kernel_name(_p(dash, flags=2), big) == "k_attend_pair"

@@ -73,7 +73,7 @@ def test_full_size_prefill_every_row(dash, name, n_rand):
     Hkv, Bc = k.shape[1], cfg.chunk_size
     qd, kd, vd, hcd = (x.to(dev) for x in (q, k, v, hc))
     prm = dash.make_params(B, Hq, Hkv, T, D, Bc, cfg.alpha, cfg.gamma, enable_gqa=True)
-    assert dash.attend_kernel_name(prm, dash.prefill_workspace_size(prm)) in ("k_attend_pp", "k_attend_fa")
+    assert dash.attend_kernel_name(prm, dash.prefill_workspace_size(prm)) == "k_attend_fa"
     res = dash.prefill(qd, kd, vd, hcd, Bc, cfg.alpha, cfg.gamma, enable_gqa=True,
                        return_p=True, return_active_blocks=True)
     torch.cuda.synchronize()
