@@ -2,7 +2,7 @@
 """Benchmark of the DashAttention forward path on B200 (one JSON line on stdout).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dash|reference]
-                    [--workload prefill128k|gqa32k|tiny|sweep] [--no-decode]
+                    [--workload prefill128k|gqa32k|tiny|sweep|decode64k] [--no-decode]
 
 A step is one causal prefill (Stage 0 -> Stage 1 -> Stage 2) over the workload's synthetic
 seeded inputs, already resident in HBM.  value = prefill tokens/s over all ranks (replicas:
@@ -378,6 +378,35 @@ def oracle_sample(cfg, q, k, v, hc, n_rows, seed=0):
                        f"extrapolated linearly to {T} rows")
 
 
+def reference_decode_line(args):
+    """The oracle's decode on the host cores: each step one decode of the 16 sequences at a
+    sampled step of the workload (its summaries recomputed by the oracle, as decode does)."""
+    import oracle
+    cfg = CONFIGS["decode64k"]
+    d = make_decode(cfg)
+    k64, v64 = oracle._f64(d["k_all"]), oracle._f64(d["v_all"])
+    times = []
+    for i in range(args.warmup + args.steps):
+        s = (37 * i) % d["steps"]
+        L = d["prefix_len"] + s + 1
+        t0 = time.perf_counter()
+        oracle.decode(d["q_steps"][s], k64, v64, d["head_cls"], [L] * cfg.batch, cfg.chunk_size,
+                      cfg.alpha)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    value = cfg.batch / statistics.median(times)
+    sample = f"{args.steps} decode steps of all {cfg.batch} sequences (oracle recomputes summaries)"
+    return {"impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 / value * cfg.batch, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "batch": cfg.batch, "cache_len": cfg.prefix_len},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
 # ------------------------------------------------------------------------------ main
 def main():
     ap = argparse.ArgumentParser()
@@ -386,7 +415,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="dash", choices=["dash", "reference"])
     ap.add_argument("--workload", default="prefill128k",
-                    choices=["prefill128k", "gqa32k", "tiny", "sweep"])
+                    choices=["prefill128k", "gqa32k", "tiny", "sweep", "decode64k"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--oracle-rows", type=int, default=0, help="0: pick by workload")
     args = ap.parse_args()
@@ -395,10 +424,14 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    cfg = workload_config(args.workload if args.workload != "sweep" else "sweep64k")
+    cfg = workload_config({"sweep": "sweep64k", "decode64k": "gqa32k"}.get(args.workload, args.workload))
     n_rows = args.oracle_rows or {"prefill128k": 96, "gqa32k": 256, "tiny": 1024,
-                                  "sweep": 32}[args.workload]
+                                  "sweep": 32, "decode64k": 0}[args.workload]
 
+    if args.impl == "reference" and args.workload == "decode64k":
+        if rank == 0:
+            print(json.dumps(reference_decode_line(args)), flush=True)
+        return
     if args.impl == "reference":
         if rank != 0:
             return
@@ -439,6 +472,8 @@ def main():
 
     if args.workload == "sweep":
         line = bench_sweep(dash, args, dev, world, rank)
+    elif args.workload == "decode64k":
+        line = bench_decode_line(dash, args, dev, world)
     else:
         line = bench_prefill(dash, cfg, args, dev, world, rank, full=True)
         if not args.no_decode and args.workload == "prefill128k":
@@ -607,6 +642,34 @@ def bench_prefill(dash, cfg, args, dev, world, rank, full=True):
     del q, k, v, out, ws, flush_buf, ws_a
     torch.cuda.empty_cache()
     return line
+
+
+DECODE_METRIC = "decode tok/s (16 sequences x 64K cached tokens, 256 steps in one CUDA graph)"
+
+
+def bench_decode_line(dash, args, dev, world):
+    """The decode workload alone as the JSON line (value = decode tokens/s over all ranks)."""
+    pk, pk_kind = peaks()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        dec = bench_decode(dash, dev)
+    ms = max_over_ranks(dec["ms_per_step"] * dec["steps"], dev)
+    cfg = CONFIGS["decode64k"]
+    return {"metric": DECODE_METRIC, "value": world * dec["batch"] * dec["steps"] / (ms / 1e3),
+            "unit": "tokens/s", "n_gpus": world, "steps": dec["steps"], "warmup": 3,
+            "ms_per_step": ms / dec["steps"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded planted-evidence generator, see dash_inputs)",
+            "config": {"workload": cfg.name, "batch": cfg.batch, "heads_q": cfg.heads_q,
+                       "heads_kv": cfg.heads_kv, "cache_len": cfg.prefix_len, "steps": cfg.steps,
+                       "head_dim": cfg.head_dim, "chunk_size": cfg.chunk_size, "alpha": cfg.alpha,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "not flushed between steps (one graph of 256 steps)"},
+            "roofline": {"bound": "hbm", "kernel": "k_decode", "achieved": dec["achieved_gbs"],
+                         "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": dec["achieved_gbs"] / pk["hbm_gbs"],
+                         "traffic": traffic_for("k_decode", "decode64k"),
+                         "peak_source": f"{pk_kind} copy bandwidth"},
+            "decode": dec, "gpu_launches": dec["launches"], "clocks": clk.summary()}
 
 
 SWEEP_METRIC = ("sweep at 64K (B=2, H_kv=8): prefill tokens/s over the alpha x chunk_size "
