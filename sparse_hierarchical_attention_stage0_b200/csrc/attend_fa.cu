@@ -63,6 +63,7 @@ struct FaShared {
     uint64_t s_full[2], p_full[2], pv_done[2];  // per S buffer: never more than one phase ahead
     uint64_t o_full, qk_done;
     float mpart[4][128];                   // partial row maxima of the first block
+    float tau[32];                         // fused routing: tau of the tile's tokens
     uint32_t tmem_base;
     int n_chunks;
     int failed;
@@ -85,11 +86,70 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
 
 }  // namespace
 
+// Fused routing of one tile (see the kernel): scores of the RT tokens over chunks [0, n) into
+// xs (stride roundup(C, 4)), then per token tau, the mask words (maskw [RT][W], and mem_mask /
+// mem_tau / mem_p in memory when given).  Every thread of the CTA calls it.
+template <int D>
+__device__ __noinline__ void fa_route_tile(const float *sumg, int C, int W, float *mem_tau,
+                                           uint64_t *mem_mask, float *mem_p, const RouteConsts rc,
+                                           uint32_t *status, long long row0, int t0, int t_end,
+                                           int RT, int n, float *xs, const float *qbar,
+                                           uint64_t *maskw, float *tau_s, int warp, int lane) {
+    const int xstride = (C + 3) & ~3;
+    const float scale = rc.kind == 0 ? rc.sscale : rc.xscale;
+    if (warp >= kWarpSm0 && warp < kWarpTmaV) {
+        const int wi = warp - kWarpSm0;
+        if (RT == 8) route_scores_lean<D, 8>(xs, xstride, qbar, sumg, n, wi, kSmWarps, scale);
+        else if (RT == 16) route_scores_lean<D, 16>(xs, xstride, qbar, sumg, n, wi, kSmWarps, scale);
+        else if (RT == 4) route_scores_lean<D, 4>(xs, xstride, qbar, sumg, n, wi, kSmWarps, scale);
+        else if (RT == 2) route_scores_lean<D, 2>(xs, xstride, qbar, sumg, n, wi, kSmWarps, scale);
+        else route_scores_lean<D, 1>(xs, xstride, qbar, sumg, n, wi, kSmWarps, scale);
+    }
+    __syncthreads();
+    for (int u = warp - kWarpSm0; u >= 0 && u < RT && warp < kWarpTmaV; u += kSmWarps) {
+        const int t = t0 + u;
+        const bool live = t < t_end;
+        const float *x = xs + u * xstride;
+        const float tau = live && n > 0 ? warp_entmax_tau(x, n, rc, status) : __int_as_float(0x7fc00000);
+        const long long rowi = row0 + t;
+        if (lane == 0) {
+            tau_s[u] = tau;
+            if (live && mem_tau) mem_tau[rowi] = tau;
+        }
+        for (int w = 0; w < W; ++w) {
+            const int c0 = w * 64 + lane, c1 = c0 + 32;
+            const bool p0 = c0 == n || (c0 < n && (rc.kind == 0 || __fsub_rn(x[c0], tau) > 0.f));
+            const bool p1 = c1 == n || (c1 < n && (rc.kind == 0 || __fsub_rn(x[c1], tau) > 0.f));
+            const unsigned lo = __ballot_sync(kFull, p0), hi = __ballot_sync(kFull, p1);
+            const uint64_t word = live ? ((uint64_t)hi << 32) | lo : 0ull;
+            if (lane == (w & 31)) {
+                maskw[u * W + w] = word;
+                if (live && mem_mask) mem_mask[rowi * W + w] = word;
+            }
+        }
+        if (live && mem_p) {
+            float *prow = mem_p + rowi * C;
+            for (int c = lane; c < C; c += 32) {
+                float val = 0.f;
+                if (c < n) {
+                    if (rc.kind == 0) {
+                        val = expf(x[c] - tau);
+                    } else {
+                        const float m = __fsub_rn(x[c], tau);
+                        val = m > 0.f ? pow_beta(m, rc) : 0.f;
+                    }
+                }
+                prow[c] = val;
+            }
+        }
+    }
+}
+
 struct FaArgs {
     StageArgs s;
     int RT;              // tokens per tile (128 / G)
     int tile0, n_tiles_bg;  // first token tile and token tiles per (b, g) of the row range
-    size_t off_bias, off_qbar, off_list;  // dynamic smem offsets (bytes, from the aligned base)
+    size_t off_bias, off_qbar, off_list, off_mask;  // dynamic smem offsets (from the aligned base)
 };
 
 template <int BC>
@@ -142,8 +202,11 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
         sh.failed = 0;
         fence_mbar_init();
     }
-    if (warp == kWarpBias) {
-        // Union of the tile's tokens' mask words (each carries its token's diagonal bit).
+    const bool fuse = a.fuse_route != 0;
+    uint64_t *maskw = reinterpret_cast<uint64_t *>(base + ta.off_mask);  // [RT][W], fused routing
+    // Union of the tile's tokens' mask words (each carries its token's diagonal bit): from the
+    // routing in memory, or from this kernel's own routing (maskw) when it is fused.
+    auto build_list = [&](bool from_smem) {
         const int W = a.W, wlim = ct_max / 64;
         int pos = 0;
         for (int w0 = 0; w0 <= wlim; w0 += 32) {
@@ -155,7 +218,7 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                 } else {
                     for (int u = 0; u < RT; ++u) {
                         const int t = t0 + u;
-                        if (t < a.t_end) word |= a.mask[(bg * a.T + t) * W + w];
+                        if (t < a.t_end) word |= from_smem ? maskw[u * W + w] : a.mask[(bg * a.T + t) * W + w];
                     }
                 }
                 const int lim = ct_max + 1 - 64 * w;          // bits [0, lim) can be attended
@@ -178,6 +241,9 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
             pos += __shfl_sync(kFull, incl, 31);
         }
         if (lane == 0) sh.n_chunks = pos;
+    };
+    if (warp == kWarpBias) {
+        if (!fuse) build_list(false);
         // Group-mean queries of the tile's tokens (Stage 1's exact arithmetic).
         if (!a.ignore_routing) {
             const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(a.q);
@@ -196,16 +262,18 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
             }
         }
     }
-    if (warp == kWarpTma) {
-        // Rows 128-143 of every V^T key-half stage are ones (bf16 1.0 = 0x3f80): P V then
-        // also yields the row sums of P in O columns 128-143.  TMA never writes these rows.
+    // Rows 128-143 of every V^T key-half stage are ones (bf16 1.0 = 0x3f80): P V then also
+    // yields the row sums of P in O columns 128-143.  TMA never writes these rows.  (With the
+    // routing fused, the ring holds the routing scores first; the ones are written after.)
+    auto write_ones = [&]() {
         const uint4 ones = make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);
         for (int i = lane; i < kStages * 2 * 16 * 8; i += 32) {
             const int half = i / (16 * 8), r = (i / 8) % 16, c = i % 8;
             *reinterpret_cast<uint4 *>(base + kOffV + (size_t)half * kVHalf + (128 + r) * 128 + c * 16) = ones;
         }
         fence_proxy_async();
-    }
+    };
+    if (warp == kWarpTma && !fuse) write_ones();
     // Softmax warps: quadrant sp (TMEM lanes 32 sp ..), key quarter kq of every block.
     const int sp = warp & 3;
     const int kq = (warp - kWarpSm0) >> 2;
@@ -237,6 +305,24 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
     __syncthreads();
     tc_fence_after();
 
+    if (fuse) {
+        // Stage 1 inside the tile (fused route-and-attend): every token of the tile has its
+        // diagonal chunk ct_max, so all route over chunks [0, ct_max).  The 16 softmax warps
+        // score them with Stage 1's arithmetic into the K/V ring (free until the copies
+        // start), one warp per token solves tau and emits its mask words (to shared memory,
+        // and to memory for the caller), then the union list is built as usual.  Kept out of
+        // line so that its registers do not press on the attention loop's.
+        fa_route_tile<D>(a.summary + bg * a.Cf * D, a.C, a.W, a.tau, a.mask, a.p, a.rc, a.status,
+                         bg * a.T, t0, a.t_end, RT, ct_max, reinterpret_cast<float *>(base), qbar,
+                         maskw, sh.tau, warp, lane);
+        // The scores went through the generic proxy; the copies that reuse the ring next go
+        // through the async proxy.
+        fence_proxy_async();
+        __syncthreads();
+        if (warp == kWarpBias) build_list(true);
+        if (warp == kWarpTma) write_ones();
+        __syncthreads();
+    }
     const int n_chunks = sh.n_chunks;
     const int n_blocks = BC == 64 ? (n_chunks + 1) / 2 : n_chunks;
     bool failed = false;
@@ -380,13 +466,13 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                         v = -INFINITY;
                     } else if (c < ctu) {
                         const long long rowi = bg * a.T + t;
-                        const bool act = dash_check(t < a.T && c < a.Cf, a.status) &&
-                                         ((a.mask[rowi * a.W + (c >> 6)] >> (c & 63)) & 1ull);
+                        const uint64_t word = fuse ? maskw[u * a.W + (c >> 6)] : a.mask[rowi * a.W + (c >> 6)];
+                        const bool act = dash_check(t < a.T && c < a.Cf, a.status) && ((word >> (c & 63)) & 1ull);
                         if (!act) {
                             v = -INFINITY;
                         } else {
                             const float dot = route_dot<D>(qbar + u * D, a.summary + (bg * a.Cf + c) * D);
-                            const float tau = a.tau[rowi];
+                            const float tau = fuse ? sh.tau[u] : a.tau[rowi];
                             if (a.rc.kind == kKindTopk) {
                                 v = 0.f;                        // top-k: uniform prior
                             } else if (a.rc.kind == 0) {
@@ -563,11 +649,13 @@ bool fa_map(EncodeFn enc, CUtensorMap *m, const void *ptr, int T, int BHkv, int 
                CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-size_t fa_smem_bytes(int RT, int C) {
+size_t fa_smem_bytes(int RT, int C, bool fuse) {
     size_t off = kRingBytes;
     off += (size_t)2 * kBiasBatch * RT * 4;      // bias batches
     off += (size_t)RT * 128 * 4;                 // qbar
     off += (size_t)((C + 7) & ~7) * 2;           // chunk list
+    off = (off + 7) & ~(size_t)7;
+    if (fuse) off += (size_t)RT * ((C + 63) / 64) * 8;   // the tile's mask words
     return off + 1024;                           // room to align the base to 1024 bytes
 }
 
@@ -581,7 +669,14 @@ size_t attend_fa_vt_bytes(int B, int Hkv, int T, int D) {
 bool attend_fa_supported(const StageArgs &a) {
     if (!(a.D == 128 && a.G >= 8 && a.G <= 128 && 128 % a.G == 0 && (a.Bc == 64 || a.Bc == 128)))
         return false;
-    return fa_smem_bytes(128 / a.G, a.C) + sizeof(FaShared) <= 227 * 1024;
+    return fa_smem_bytes(128 / a.G, a.C, false) + sizeof(FaShared) <= 227 * 1024;
+}
+
+bool attend_fa_fuse_supported(const StageArgs &a) {
+    if (!attend_fa_supported(a) || a.ignore_routing || a.rc.kind > 3 || a.rc.est_diag) return false;
+    const int RT = 128 / a.G;
+    if ((size_t)RT * ((a.C + 3) & ~3) * 4 > kRingBytes) return false;   // the scores fit the ring
+    return fa_smem_bytes(RT, a.C, true) + sizeof(FaShared) <= 227 * 1024;
 }
 
 template <int BC>
@@ -617,7 +712,9 @@ static cudaError_t launch_fa_t(const StageArgs &a, cudaStream_t st) {
     ta.off_qbar = off;
     off += (size_t)ta.RT * 128 * 4;
     ta.off_list = off;
-    const size_t smem = fa_smem_bytes(ta.RT, a.C);
+    off += (size_t)((a.C + 7) & ~7) * 2;
+    ta.off_mask = (off + 7) & ~(size_t)7;
+    const size_t smem = fa_smem_bytes(ta.RT, a.C, a.fuse_route != 0);
     auto kern = k_attend_fa<BC>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -277,9 +277,13 @@ dash_status_t dash_prefill(const dash_params_t *p, const void *q, const void *k,
     if (vt && ws_bytes >= off + vt) a.vt = w + off;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if ((rc = clear_status(ws, st)) != DASH_OK) return rc;
+    // Fused route-and-attend where the 128-key-block kernel takes it: Stage 2 runs Stage 1 for
+    // its own tiles (liuzhao09.github.io "DashAttention 精读", section 2: fused kernels), so q
+    // is read once and the routing never makes a round trip through memory.
+    a.fuse_route = !dense && attend_kernel(a) == AttendKernel::kFa && attend_fa_fuse_supported(a);
     if (!dense) {
         if ((rc = from_cuda(launch_stage0(a, nullptr, 0, st))) != DASH_OK) return rc;
-        if ((rc = from_cuda(launch_route(a, st))) != DASH_OK) return rc;
+        if (!a.fuse_route && (rc = from_cuda(launch_route(a, st))) != DASH_OK) return rc;
     }
     return from_cuda(launch_attend(a, st));
 }
@@ -374,8 +378,9 @@ dash_status_t dash_prefill_host(const dash_params_t *p, const void *q_host, cons
             a.t_begin = i * rows;
             a.t_end = std::min(s.T, (i + 1) * rows);
             a.vt_ready = i > 0;
+            a.fuse_route = !dense && attend_kernel(a) == AttendKernel::kFa && attend_fa_fuse_supported(a);
             ok(cudaStreamWaitEvent(st, e_q(i), 0));
-            if (!dense) ok(launch_route(a, st));
+            if (!dense && !a.fuse_route) ok(launch_route(a, st));
             ok(launch_attend(a, st));
             ok(cudaEventRecord(e_o(i), st));
         }

@@ -232,6 +232,56 @@ __device__ __forceinline__ float route_dot(const float *qbar, const float *srow)
 // RouteConsts::kind of top-k routing (the k highest scores, uniform prior in Stage 2).
 constexpr int kKindTopk = 4;
 
+// Routing scores of RT query rows against chunks [0, n) into xs[r * xstride + c], computed
+// by n_warps warps (this one is warp_idx of them): 4 lanes per chunk, each an interleaved
+// quarter of d as one sequential fmaf chain, two chunks (c, c + 8) per lane, slices combined
+// as (p0 + p1) + (p2 + p3) -- route_dot's order, so every score has route_dot's bits.  The
+// summary rows are loaded one float4 group at a time (few registers: usable inside a kernel
+// with a tight register budget).  qbar: [RT][D] in shared memory.
+template <int D, int RT>
+__device__ __forceinline__ void route_scores_lean(float *xs, int xstride, const float *qbar,
+                                                  const float *sumg, int n, int warp_idx,
+                                                  int n_warps, float scale) {
+    const int lane = threadIdx.x & 31;
+    const int kslice = lane & 3, cc = lane >> 2;
+    for (int cbase = warp_idx * 16; cbase < n; cbase += n_warps * 16) {
+        const int c = cbase + cc, c2 = c + 8;
+        const float4 *s4 = reinterpret_cast<const float4 *>(sumg + (long long)min(c, n - 1) * D);
+        const float4 *t4 = reinterpret_cast<const float4 *>(sumg + (long long)min(c2, n - 1) * D);
+        float acc[RT], acc2[RT];
+#pragma unroll
+        for (int r = 0; r < RT; ++r) acc[r] = acc2[r] = 0.f;
+#pragma unroll 2
+        for (int i = 0; i < D / 16; ++i) {
+            const float4 sv = __ldg(s4 + 4 * i + kslice), tv = __ldg(t4 + 4 * i + kslice);
+#pragma unroll
+            for (int r = 0; r < RT; ++r) {
+                const float4 qq = reinterpret_cast<const float4 *>(qbar + r * D)[4 * i + kslice];
+                acc[r] = fmaf(qq.x, sv.x, acc[r]);
+                acc2[r] = fmaf(qq.x, tv.x, acc2[r]);
+                acc[r] = fmaf(qq.y, sv.y, acc[r]);
+                acc2[r] = fmaf(qq.y, tv.y, acc2[r]);
+                acc[r] = fmaf(qq.z, sv.z, acc[r]);
+                acc2[r] = fmaf(qq.z, tv.z, acc2[r]);
+                acc[r] = fmaf(qq.w, sv.w, acc[r]);
+                acc2[r] = fmaf(qq.w, tv.w, acc2[r]);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+            float v = acc[r], w = acc2[r];
+            v = v + __shfl_xor_sync(kFull, v, 1);
+            w = w + __shfl_xor_sync(kFull, w, 1);
+            v = v + __shfl_xor_sync(kFull, v, 2);
+            w = w + __shfl_xor_sync(kFull, w, 2);
+            if (kslice == 0) {
+                if (c < n) xs[r * xstride + c] = __fmul_rn(v, scale);
+                if (c2 < n) xs[r * xstride + c2] = __fmul_rn(w, scale);
+            }
+        }
+    }
+}
+
 // Constants of the routing, computed once on the host.
 struct RouteConsts {
     float xscale;     // (alpha-1) * gamma / sqrt(D): x_c = dot * xscale (alpha > 1)

@@ -28,6 +28,7 @@ struct StageArgs {
                               // T stays the row stride of q, tau, mask, p and out
     int vt_ready;             // V^T scratch already holds the transpose of V (a later row slice)
     int test_stall;           // test hook: Stage 0's chunk-copy wait runs out (DASH_FLAG_TEST_STALL_WAIT)
+    int fuse_route;           // Stage 2 computes the routing itself (fused route-and-attend)
     uint32_t *status;
 };
 
@@ -64,6 +65,8 @@ const char *attend_kernel_name(AttendKernel k);
 bool attend_tc_supported(const StageArgs &a);
 cudaError_t launch_attend_tc(const StageArgs &a, cudaStream_t st);
 bool attend_fa_supported(const StageArgs &a);
+// The 128-key-block kernel can run Stage 1 itself for these arguments (fused route-and-attend).
+bool attend_fa_fuse_supported(const StageArgs &a);
 size_t attend_fa_vt_bytes(int B, int Hkv, int T, int D);
 cudaError_t launch_attend_fa(const StageArgs &a, cudaStream_t st);
 bool attend_pair_supported(const StageArgs &a);

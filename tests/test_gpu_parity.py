@@ -531,3 +531,29 @@ def test_paged_decode_equals_contiguous_decode(dash):
     bad[1, 2] = n_pages + 7
     dash.decode_paged(qs, k_pool, v_pool, bad, seq, s_pool, Bc, ws=ws)
     assert dash.read_device_status(ws) == 1
+
+
+# ------------------------------------------------------------------------------ fused route-and-attend
+@pytest.mark.parametrize("alpha", [1.0, 1.5, 2.0, 1.25])
+@pytest.mark.parametrize("G,Bc,T", [(16, 64, 2100 + 37), (8, 128, 1500 + 3), (32, 64, 1300)])
+def test_fused_route_and_attend_equals_the_separate_stages(dash, alpha, G, Bc, T):
+    """dash_prefill runs Stage 1 inside the 128-key-block Stage 2 kernel (each tile routes its
+    own tokens with Stage 1's arithmetic).  Its mask, p and output equal those of the separate
+    Stage 1 and Stage 2 launches bit for bit, and the oracle's."""
+    Hkv = 2 if G <= 16 else 1
+    q, k, v, hc = make_prefill(_cfg(1, G * Hkv, Hkv, T, 128, Bc, alpha, seed=95 + G))
+    qd, kd, vd, hcd = _to(q, k, v, hc)
+    res = dash.prefill(qd, kd, vd, hcd, Bc, alpha, enable_gqa=True, return_p=True,
+                       return_active_blocks=True, return_summary=True)
+    r = dash.route(qd, res["summary"], Hkv, Bc, alpha)
+    o = dash.attend(qd, kd, vd, res["summary"], r["tau"], r["active_blocks"], Bc, alpha)
+    torch.cuda.synchronize()
+    assert dash.read_device_status(res["ws"]) == 0
+    assert torch.equal(res["active_blocks"], r["active_blocks"])
+    assert torch.equal(res["p"], r["p"])
+    assert torch.equal(res["out"], o)
+    ref = oracle.prefill(q, k, v, hc, Bc, alpha)
+    C = ref["p"].shape[-1]
+    check_routing(unpack_mask(res["active_blocks"], C), res["p"].cpu().double().numpy(),
+                  ref["p"], ref["m"], np.arange(T), Bc, alpha, tag="fused")
+    check_output(res["out"].cpu().float().numpy(), ref["O"], tag="fused")
