@@ -720,7 +720,9 @@ cudaError_t launch_pair_t(const StageArgs &a, cudaStream_t st) {
 }  // namespace
 
 bool attend_pair_supported(const StageArgs &a) {
-    if (!(a.D == 128 && a.G >= 8 && a.G <= 128 && 128 % a.G == 0 && (a.Bc == 64 || a.Bc == 128)))
+    // A pair's two tiles (2 x 128/G tokens) must share one diagonal chunk.
+    if (!(a.D == 128 && a.G >= 2 && a.G <= 128 && 128 % a.G == 0 && (a.Bc == 64 || a.Bc == 128) &&
+          2 * (128 / a.G) <= a.Bc))
         return false;
     return pr_smem_bytes(128 / a.G, a.C) + sizeof(PrShared) <= 227 * 1024;
 }

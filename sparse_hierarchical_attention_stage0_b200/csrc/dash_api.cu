@@ -110,15 +110,20 @@ size_t bytes_tau(const Shape &s) { return align256((size_t)s.B * s.Hkv * s.T * 4
 size_t bytes_summary(const Shape &s) { return align256((size_t)s.B * s.Hkv * s.Cf * s.D * 4); }
 size_t bytes_mask(const Shape &s) { return align256((size_t)s.B * s.Hkv * s.T * s.W * 8); }
 
-// V^T scratch of the 128-key-block Stage 2 kernel; 0 when that kernel does not apply.
-size_t bytes_vt(const Shape &s) {
+// V^T scratch of the 128-key-block Stage 2 kernels; 0 when none of them applies (the routed
+// kernel, or with `dense` the one on pairs of SMs, which also serves fewer query heads per KV
+// head).
+size_t bytes_vt(const Shape &s, bool dense) {
     StageArgs a = {};
     a.D = s.D;
     a.G = s.G;
     a.Bc = s.Bc;
     a.C = s.C;
-    if (!attend_fa_supported(a)) return 0;
+    if (!attend_fa_supported(a) && !(dense && attend_pair_supported(a))) return 0;
     return align256(attend_fa_vt_bytes(s.B, s.Hkv, s.T, s.D));
+}
+bool dense_flags(const dash_params_t *p) {
+    return (p->flags & (DASH_FLAG_DENSE | DASH_FLAG_FORCE_ALL_ACTIVE)) != 0;
 }
 
 dash_status_t clear_status(void *ws, cudaStream_t st) {
@@ -220,13 +225,13 @@ const char *dash_status_string(dash_status_t s) {
 size_t dash_prefill_workspace_size(const dash_params_t *p) {
     Shape s;
     if (check_params(p, &s) != DASH_OK) return 0;
-    return kStatusBytes + bytes_tau(s) + bytes_summary(s) + bytes_mask(s) + bytes_vt(s);
+    return kStatusBytes + bytes_tau(s) + bytes_summary(s) + bytes_mask(s) + bytes_vt(s, dense_flags(p));
 }
 
 size_t dash_attend_workspace_size(const dash_params_t *p) {
     Shape s;
     if (check_params(p, &s) != DASH_OK) return 0;
-    return kStatusBytes + bytes_vt(s);
+    return kStatusBytes + bytes_vt(s, dense_flags(p));
 }
 
 dash_status_t dash_prefill(const dash_params_t *p, const void *q, const void *k, const void *v,
@@ -273,7 +278,7 @@ dash_status_t dash_prefill(const dash_params_t *p, const void *q, const void *k,
             off += bytes_mask(s);
         }
     }
-    const size_t vt = bytes_vt(s);
+    const size_t vt = bytes_vt(s, dense_flags(p));
     if (vt && ws_bytes >= off + vt) a.vt = w + off;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if ((rc = clear_status(ws, st)) != DASH_OK) return rc;
@@ -323,7 +328,7 @@ dash_status_t dash_prefill_host(const dash_params_t *p, const void *q_host, cons
         a.mask = reinterpret_cast<uint64_t *>(w + off);
         off += bytes_mask(s);
     }
-    const size_t vt = bytes_vt(s);
+    const size_t vt = bytes_vt(s, dense_flags(p));
     if (vt) a.vt = w + off;
     // Row slices only where the Stage 2 kernel takes a row range; each slice a multiple of
     // 128 rows (the last one ragged).
@@ -471,7 +476,7 @@ dash_status_t dash_attend(const dash_params_t *p, const void *q, const void *k, 
     a.tau = const_cast<float *>(tau);
     a.mask = const_cast<uint64_t *>(active_blocks);
     a.status = static_cast<uint32_t *>(ws);
-    const size_t vt = bytes_vt(s);
+    const size_t vt = bytes_vt(s, dense_flags(p));
     if (vt && ws_bytes >= kStatusBytes + vt) a.vt = static_cast<unsigned char *>(ws) + kStatusBytes;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if ((rc = clear_status(ws, st)) != DASH_OK) return rc;
@@ -563,7 +568,7 @@ const char *dash_attend_kernel_name(const dash_params_t *p, size_t ws_bytes) {
     Shape s;
     if (check_params(p, &s) != DASH_OK || ws_bytes < kStatusBytes) return "";
     StageArgs a = stage_args(p, s);
-    const size_t vt = bytes_vt(s);
+    const size_t vt = bytes_vt(s, dense_flags(p));
     // Only whether the V^T scratch fits matters for the choice, not where it is.
     static unsigned char probe;
     if (vt && ws_bytes >= kStatusBytes + vt) a.vt = &probe;

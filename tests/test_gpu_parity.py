@@ -197,7 +197,7 @@ def test_dense_equals_force_all_active_and_causal_attention(dash):
 
 
 @pytest.mark.parametrize("B,G,Bc,T", [(2, 16, 64, 993), (1, 8, 64, 1505), (1, 32, 128, 1027),
-                                      (2, 8, 128, 700)])
+                                      (2, 8, 128, 700), (2, 4, 64, 777), (1, 2, 128, 1100 + 9)])
 def test_dense_on_sm_pairs_matches_causal_attention(dash, B, G, Bc, T):
     """Dense mode runs on pairs of SMs, two tiles per pair.  Odd tile counts leave the last
     pair's second tile past the end of the sequence; batch 2 covers several (b, g) planes."""
