@@ -348,11 +348,79 @@ def bench_decode(dash, dev, steps_cap=256, warmup=3):
     ms = statistics.median(times)
     launches = S + sum(1 for s in range(S) if (L0 + s + 1) % Bc == 0)
     del g
+    paged_ms = bench_decode_paged(dash, dev, d, cfg, S, warmup)
     return dict(tokens_per_s=B * S / (ms / 1e3), ms_per_step=ms / S, steps=S, batch=B,
+                paged={"ms_per_step": paged_ms / S, "tokens_per_s": B * S / (paged_ms / 1e3),
+                       "layout": "pages of one chunk, scattered through the pools by a random "
+                                 "block table"},
                 cache_len=L0, realised_sparsity=sparsity,
                 hbm_bytes_per_step=alg_bytes / S,
                 achieved_gbs=alg_bytes / (ms / 1e3) / 1e9, launches=launches,
                 note="steps include the K/V append copies and seq_len update (torch ops)")
+
+
+def bench_decode_paged(dash, dev, d, cfg, S, warmup):
+    """The same 256 decode steps on a paged cache (pages of one chunk, a random block table),
+    captured in one graph; returns the median graph time in ms."""
+    B, Hq, Hkv, D, Bc = cfg.batch, cfg.heads_q, cfg.heads_kv, cfg.head_dim, cfg.chunk_size
+    L0, cap = d["prefix_len"], d["capacity"]
+    nb = cap // Bc
+    n_pages = B * nb
+    gen = torch.Generator().manual_seed(11)
+    table = torch.randperm(n_pages, generator=gen).view(B, nb).to(torch.int32).to(dev)
+    k_all, v_all = d["k_all"].to(dev), d["v_all"].to(dev)
+    hc, q_steps = d["head_cls"].to(dev), d["q_steps"].to(dev)
+    # pool[table[b, c]] = chunk c of sequence b (positions >= L0 zero until appended)
+    flat = table.view(-1).long()
+    kp = torch.zeros(n_pages, Hkv, Bc, D, dtype=torch.bfloat16, device=dev)
+    vp = torch.zeros_like(kp)
+    src_k = k_all.clone()
+    src_v = v_all.clone()
+    src_k[:, :, L0:] = 0
+    src_v[:, :, L0:] = 0
+    kp[flat] = src_k.view(B, Hkv, nb, Bc, D).permute(0, 2, 1, 3, 4).reshape(n_pages, Hkv, Bc, D)
+    vp[flat] = src_v.view(B, Hkv, nb, Bc, D).permute(0, 2, 1, 3, 4).reshape(n_pages, Hkv, Bc, D)
+    sp = torch.zeros(n_pages, Hkv, D, device=dev)
+    seq = torch.full((B,), L0, dtype=torch.int32, device=dev)
+    dash.update_chunk_cache_paged(kp, hc, table, seq, sp, Hq, Bc, n_recent=L0 // Bc)
+    out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
+    ws, ws_u = dash.workspace(256, dev), dash.workspace(256, dev)
+    bidx = torch.arange(B, device=dev)
+
+    def step(s):
+        L = L0 + s + 1
+        c, r = (L - 1) // Bc, (L - 1) % Bc
+        pages = table[:, c].long()
+        kp[pages, :, r] = k_all[bidx, :, L - 1]
+        vp[pages, :, r] = v_all[bidx, :, L - 1]
+        seq.fill_(L)
+        if L % Bc == 0:
+            dash.update_chunk_cache_paged(kp, hc, table, seq, sp, Hq, Bc, n_recent=1, ws=ws_u)
+        dash.decode_paged(q_steps[s], kp, vp, table, seq, sp, Bc, cfg.alpha, out=out, ws=ws)
+
+    g = torch.cuda.CUDAGraph()
+    stream = torch.cuda.Stream(dev)
+    stream.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(stream):
+        for s in range(min(warmup, S)):
+            step(s)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            for s in range(S):
+                step(s)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(3):
+        st = torch.cuda.Event(enable_timing=True)
+        en = torch.cuda.Event(enable_timing=True)
+        st.record(stream)
+        g.replay()
+        en.record(stream)
+        en.synchronize()
+        times.append(st.elapsed_time(en))
+    assert dash.read_device_status(ws) == 0 and dash.read_device_status(ws_u) == 0
+    del g
+    return statistics.median(times)
 
 
 # ------------------------------------------------------------------------------ oracle
@@ -620,6 +688,22 @@ def bench_prefill(dash, cfg, args, dev, world, rank, full=True):
         "clocks": clk.summary(),
     }
     if full:
+        # The routing variants, each timed as the main prefill (L2 flushed before each step):
+        # top-k routing at the entmax's mean active-chunk count (equal sparsity), and the
+        # estimated diagonal.
+        k_eq = max(1, int(round(stats["active_chunks"] / (B * Hkv * T))))
+        variants = {}
+        for name, kw in (("topk", dict(topk=k_eq)), ("estimate_diagonal", dict(estimate_diagonal=True))):
+            def run_variant(kw=kw):
+                dash.prefill(q, k, v, hc, Bc, cfg.alpha, cfg.gamma, enable_gqa=True, out=out,
+                             ws=ws, **kw)
+            for _ in range(2):
+                run_variant()
+            vms = statistics.mean(timed(run_variant, max(2, min(args.steps, 3)), stream, flush))
+            variants[name] = {"ms_per_step": vms, "tokens_per_s": B * T / (vms / 1e3), **kw}
+        torch.cuda.synchronize()
+        assert dash.read_device_status(ws) == 0
+        line["routing_variants"] = variants
         # End to end through host buffers: dash_prefill_host copies q, k, v, head_cls from
         # pinned host memory and out back, in row slices overlapped with the computation.
         hq, hk, hv, hhc = (x.pin_memory() for x in (q_h, k_h, v_h, hc_h))
