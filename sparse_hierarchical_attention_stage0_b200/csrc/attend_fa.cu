@@ -56,14 +56,16 @@ constexpr uint32_t kBlkBytes = 32768;      // K stage: 2 d-panels x [128 keys][1
 constexpr int kNv = 144;                   // P V columns: 128 dims of V, then 16 columns of ones
 constexpr uint32_t kVHalf = kNv * 128;     // V^T key-half: [144 rows][64 keys x 2 B] (rows >= 128: ones)
 constexpr uint32_t kVStage = 2 * kVHalf;
-constexpr uint32_t kOffV = kStages * kBlkBytes, kRingBytes = kOffV + kStages * kVStage;
+// K/V ring of NST stages (3, or 2 where larger tiles of tokens need the shared memory).
+constexpr uint32_t ring_offv(int nst) { return (uint32_t)nst * kBlkBytes; }
+constexpr uint32_t ring_bytes(int nst) { return ring_offv(nst) + (uint32_t)nst * kVStage; }
 
 struct FaShared {
     uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
     uint64_t s_full[2], p_full[2], pv_done[2];  // per S buffer: never more than one phase ahead
     uint64_t o_full, qk_done;
     float mpart[4][128];                   // partial row maxima of the first block
-    float tau[32];                         // fused routing: tau of the tile's tokens
+    float tau[64];                         // fused routing: tau of the tile's tokens
     uint32_t tmem_base;
     int n_chunks;
     int failed;
@@ -99,11 +101,19 @@ __device__ __noinline__ void fa_route_tile(const float *sumg, int C, int W, floa
     const float scale = rc.kind == 0 ? rc.sscale : rc.xscale;
     if (warp >= kWarpSm0 && warp < kWarpTmaV) {
         const int wi = warp - kWarpSm0;
-        if (RT == 8) route_scores_lean<D, 8>(xs, xstride, qbar, sumg, n, wi, kSmWarps, scale);
-        else if (RT == 16) route_scores_lean<D, 16>(xs, xstride, qbar, sumg, n, wi, kSmWarps, scale);
-        else if (RT == 4) route_scores_lean<D, 4>(xs, xstride, qbar, sumg, n, wi, kSmWarps, scale);
-        else if (RT == 2) route_scores_lean<D, 2>(xs, xstride, qbar, sumg, n, wi, kSmWarps, scale);
-        else route_scores_lean<D, 1>(xs, xstride, qbar, sumg, n, wi, kSmWarps, scale);
+        if (RT >= 16) {
+            // Rows in groups of 16 (register budget); each row's arithmetic is unchanged.
+            for (int r0 = 0; r0 < RT; r0 += 16)
+                route_scores_lean<D, 16>(xs + r0 * xstride, xstride, qbar + r0 * D, sumg, n, wi, kSmWarps, scale);
+        } else if (RT == 8) {
+            route_scores_lean<D, 8>(xs, xstride, qbar, sumg, n, wi, kSmWarps, scale);
+        } else if (RT == 4) {
+            route_scores_lean<D, 4>(xs, xstride, qbar, sumg, n, wi, kSmWarps, scale);
+        } else if (RT == 2) {
+            route_scores_lean<D, 2>(xs, xstride, qbar, sumg, n, wi, kSmWarps, scale);
+        } else {
+            route_scores_lean<D, 1>(xs, xstride, qbar, sumg, n, wi, kSmWarps, scale);
+        }
     }
     __syncthreads();
     for (int u = warp - kWarpSm0; u >= 0 && u < RT && warp < kWarpTmaV; u += kSmWarps) {
@@ -152,12 +162,13 @@ struct FaArgs {
     size_t off_bias, off_qbar, off_list, off_mask;  // dynamic smem offsets (from the aligned base)
 };
 
-template <int BC>
+template <int BC, int NST>
 __global__ void __launch_bounds__(kFaThreads, 1)
 k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmK128,
             const __grid_constant__ CUtensorMap tmVt, const FaArgs ta) {
     extern __shared__ unsigned char smem_dyn[];
     __shared__ FaShared sh;
+    constexpr uint32_t kOffVn = ring_offv(NST);
     const StageArgs &a = ta.s;
     constexpr int D = 128;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -186,7 +197,7 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < NST; ++s) {
             mbar_init(&sh.k_full[s], 1);
             mbar_init(&sh.k_empty[s], 1);
             mbar_init(&sh.v_full[s], 1);
@@ -267,9 +278,9 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
     // routing fused, the ring holds the routing scores first; the ones are written after.)
     auto write_ones = [&]() {
         const uint4 ones = make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);
-        for (int i = lane; i < kStages * 2 * 16 * 8; i += 32) {
+        for (int i = lane; i < NST * 2 * 16 * 8; i += 32) {
             const int half = i / (16 * 8), r = (i / 8) % 16, c = i % 8;
-            *reinterpret_cast<uint4 *>(base + kOffV + (size_t)half * kVHalf + (128 + r) * 128 + c * 16) = ones;
+            *reinterpret_cast<uint4 *>(base + kOffVn + (size_t)half * kVHalf + (128 + r) * 128 + c * 16) = ones;
         }
         fence_proxy_async();
     };
@@ -348,13 +359,13 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
         // not issued either).
         int k_issued = 0, v_issued = 0;
         auto issue = [&](bool is_v, int j) -> bool {
-            const int s = j % kStages;
-            const uint32_t ph = (uint32_t)(j / kStages) & 1u;
+            const int s = j % NST;
+            const uint32_t ph = (uint32_t)(j / NST) & 1u;
             uint64_t *empty = is_v ? &sh.v_empty[s] : &sh.k_empty[s];
             uint64_t *full = is_v ? &sh.v_full[s] : &sh.k_full[s];
             if (!wait_or_fail(empty, ph ^ 1u, a.status, failed)) return false;
             if (lane == 0) {
-                unsigned char *st = base + (is_v ? kOffV + (size_t)s * kVStage : (size_t)s * kBlkBytes);
+                unsigned char *st = base + (is_v ? kOffVn + (size_t)s * kVStage : (size_t)s * kBlkBytes);
                 const int nh = entry_of(j, 1) >= 0 ? 2 : 1;
                 mbar_arrive_expect_tx(full, 16384u * nh);
                 for (int h = 0; h < nh; ++h) {
@@ -381,10 +392,10 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
             if (!issue(is_v, j)) break;
         if (failed) {
             // Bounded wait for the copies still in flight (the last ones per ring).
-            for (int i = max(0, k_issued - kStages); i < k_issued; ++i)
-                mbar_wait_bounded(&sh.k_full[i % kStages], (uint32_t)(i / kStages) & 1u);
-            for (int i = max(0, v_issued - kStages); i < v_issued; ++i)
-                mbar_wait_bounded(&sh.v_full[i % kStages], (uint32_t)(i / kStages) & 1u);
+            for (int i = max(0, k_issued - NST); i < k_issued; ++i)
+                mbar_wait_bounded(&sh.k_full[i % NST], (uint32_t)(i / NST) & 1u);
+            for (int i = max(0, v_issued - NST); i < v_issued; ++i)
+                mbar_wait_bounded(&sh.v_full[i % NST], (uint32_t)(i / NST) & 1u);
             __syncwarp();
         }
     } else if (warp == kWarpQk) {
@@ -392,19 +403,19 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
         // S buffer j & 1 is free once P V of block j-2 (which read P from it) has completed.
         constexpr uint32_t id_qk128 = idesc_bf16(128, 128, 0);
         constexpr uint32_t id_qk64 = idesc_bf16(128, 64, 0);
-        uint64_t kdesc[kStages];
+        uint64_t kdesc[NST];
 #pragma unroll
-        for (int s = 0; s < kStages; ++s) kdesc[s] = smem_desc_sw128(smem_u32(base + (size_t)s * kBlkBytes), 16, 1024);
+        for (int s = 0; s < NST; ++s) kdesc[s] = smem_desc_sw128(smem_u32(base + (size_t)s * kBlkBytes), 16, 1024);
         for (int j = 0; j < n_blocks; ++j) {
-            const int s = j % kStages, sb = j & 1;
-            if (!wait_or_fail(&sh.k_full[s], (uint32_t)(j / kStages) & 1u, a.status, failed)) break;
+            const int s = j % NST, sb = j & 1;
+            if (!wait_or_fail(&sh.k_full[s], (uint32_t)(j / NST) & 1u, a.status, failed)) break;
             if (j >= 2 && !wait_or_fail(&sh.pv_done[sb], (uint32_t)((j - 2) >> 1) & 1u, a.status, failed)) break;
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t id = entry_of(j, 1) >= 0 ? id_qk128 : id_qk64;
                 uint64_t bd0 = 0;
 #pragma unroll
-                for (int q = 0; q < kStages; ++q) bd0 = q == s ? kdesc[q] : bd0;
+                for (int q = 0; q < NST; ++q) bd0 = q == s ? kdesc[q] : bd0;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     // descriptor start address advances in 16-byte units: d-panel kk/4, 32 B per 16 dims
@@ -422,12 +433,12 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
         // ------------------------------------------------------------ P V issuer
         // P of keys 32q .. 32q+31 sits in the first 16 columns of S quarter q; B = V^T, K-major.
         constexpr uint32_t id_pv = idesc_bf16(128, kNv, 0);
-        uint64_t vdesc[kStages];
+        uint64_t vdesc[NST];
 #pragma unroll
-        for (int s = 0; s < kStages; ++s) vdesc[s] = smem_desc_sw128(smem_u32(base + kOffV + (size_t)s * kVStage), 16, 1024);
+        for (int s = 0; s < NST; ++s) vdesc[s] = smem_desc_sw128(smem_u32(base + kOffVn + (size_t)s * kVStage), 16, 1024);
         for (int j = 0; j < n_blocks; ++j) {
-            const int s = j % kStages, sb = j & 1;
-            if (!wait_or_fail(&sh.v_full[s], (uint32_t)(j / kStages) & 1u, a.status, failed)) break;
+            const int s = j % NST, sb = j & 1;
+            if (!wait_or_fail(&sh.v_full[s], (uint32_t)(j / NST) & 1u, a.status, failed)) break;
             if (!wait_or_fail(&sh.p_full[sb], (uint32_t)(j >> 1) & 1u, a.status, failed)) break;
             tc_fence_after();
             if (lane == 0) {
@@ -435,7 +446,7 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                 const bool full_blk = entry_of(j, 1) >= 0;
                 uint64_t bd0 = 0;
 #pragma unroll
-                for (int q = 0; q < kStages; ++q) bd0 = q == s ? vdesc[q] : bd0;
+                for (int q = 0; q < NST; ++q) bd0 = q == s ? vdesc[q] : bd0;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     if (kk >= 4 && !full_blk) break;
@@ -649,8 +660,8 @@ bool fa_map(EncodeFn enc, CUtensorMap *m, const void *ptr, int T, int BHkv, int 
                CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-size_t fa_smem_bytes(int RT, int C, bool fuse) {
-    size_t off = kRingBytes;
+size_t fa_smem_bytes(int RT, int C, bool fuse, int nst) {
+    size_t off = ring_bytes(nst);
     off += (size_t)2 * kBiasBatch * RT * 4;      // bias batches
     off += (size_t)RT * 128 * 4;                 // qbar
     off += (size_t)((C + 7) & ~7) * 2;           // chunk list
@@ -666,20 +677,27 @@ size_t attend_fa_vt_bytes(int B, int Hkv, int T, int D) {
     return (size_t)B * Hkv * D * T8 * 2;
 }
 
-bool attend_fa_supported(const StageArgs &a) {
-    if (!(a.D == 128 && a.G >= 8 && a.G <= 128 && 128 % a.G == 0 && (a.Bc == 64 || a.Bc == 128)))
-        return false;
-    return fa_smem_bytes(128 / a.G, a.C, false) + sizeof(FaShared) <= 227 * 1024;
+// Ring stages for these arguments: 3, or 2 when 3 do not fit (0: neither fits).
+static int fa_stages(const StageArgs &a, bool fuse) {
+    if (!(a.D == 128 && a.G >= 2 && a.G <= 128 && 128 % a.G == 0 && (a.Bc == 64 || a.Bc == 128) &&
+          128 / a.G <= a.Bc))                  // a tile's tokens share one diagonal chunk
+        return 0;
+    const int RT = 128 / a.G;
+    for (int nst : {3, 2}) {
+        if (fuse && (size_t)RT * ((a.C + 3) & ~3) * 4 > ring_bytes(nst)) continue;   // scores fit the ring
+        if (fa_smem_bytes(RT, a.C, fuse, nst) + sizeof(FaShared) <= 227 * 1024) return nst;
+    }
+    return 0;
 }
+
+bool attend_fa_supported(const StageArgs &a) { return fa_stages(a, false) != 0; }
 
 bool attend_fa_fuse_supported(const StageArgs &a) {
-    if (!attend_fa_supported(a) || a.ignore_routing || a.rc.kind > 3 || a.rc.est_diag) return false;
-    const int RT = 128 / a.G;
-    if ((size_t)RT * ((a.C + 3) & ~3) * 4 > kRingBytes) return false;   // the scores fit the ring
-    return fa_smem_bytes(RT, a.C, true) + sizeof(FaShared) <= 227 * 1024;
+    if (a.ignore_routing || a.rc.kind > 3 || a.rc.est_diag) return false;
+    return fa_stages(a, true) != 0;
 }
 
-template <int BC>
+template <int BC, int NST>
 static cudaError_t launch_fa_t(const StageArgs &a, cudaStream_t st) {
     static EncodeFn enc = fa_encode();
     if (!enc || !a.vt) return cudaErrorNotSupported;
@@ -706,7 +724,7 @@ static cudaError_t launch_fa_t(const StageArgs &a, cudaStream_t st) {
     ta.RT = 128 / a.G;
     ta.tile0 = a.t_begin / ta.RT;
     ta.n_tiles_bg = (a.t_end + ta.RT - 1) / ta.RT - ta.tile0;
-    size_t off = kRingBytes;
+    size_t off = ring_bytes(NST);
     ta.off_bias = off;
     off += (size_t)2 * kBiasBatch * ta.RT * 4;
     ta.off_qbar = off;
@@ -714,8 +732,8 @@ static cudaError_t launch_fa_t(const StageArgs &a, cudaStream_t st) {
     ta.off_list = off;
     off += (size_t)((a.C + 7) & ~7) * 2;
     ta.off_mask = (off + 7) & ~(size_t)7;
-    const size_t smem = fa_smem_bytes(ta.RT, a.C, a.fuse_route != 0);
-    auto kern = k_attend_fa<BC>;
+    const size_t smem = fa_smem_bytes(ta.RT, a.C, a.fuse_route != 0, NST);
+    auto kern = k_attend_fa<BC, NST>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const long long grid = (long long)ta.n_tiles_bg * BHkv;
@@ -725,8 +743,11 @@ static cudaError_t launch_fa_t(const StageArgs &a, cudaStream_t st) {
 }
 
 cudaError_t launch_attend_fa(const StageArgs &a, cudaStream_t st) {
-    if (a.Bc == 64) return launch_fa_t<64>(a, st);
-    if (a.Bc == 128) return launch_fa_t<128>(a, st);
+    const int nst = fa_stages(a, a.fuse_route != 0);
+    if (a.Bc == 64 && nst == 3) return launch_fa_t<64, 3>(a, st);
+    if (a.Bc == 64 && nst == 2) return launch_fa_t<64, 2>(a, st);
+    if (a.Bc == 128 && nst == 3) return launch_fa_t<128, 3>(a, st);
+    if (a.Bc == 128 && nst == 2) return launch_fa_t<128, 2>(a, st);
     return cudaErrorInvalidValue;
 }
 

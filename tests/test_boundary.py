@@ -187,10 +187,12 @@ def test_attend_kernel_name_follows_the_dispatch(dash):
     assert dash.attend_kernel_name(_p(dash), 256) == "k_attend_tc"          # no room for V^T
     assert dash.attend_kernel_name(_p(dash, flags=1), big) == "k_attend_pair"
     assert dash.attend_kernel_name(_p(dash, flags=2), big) == "k_attend_pair"
-    assert dash.attend_kernel_name(_p(dash, heads_q=8), big) == "k_attend"     # G = 4
+    assert dash.attend_kernel_name(_p(dash, heads_q=8), big) == "k_attend_fa"  # G = 4: 32-token tiles
+    assert dash.attend_kernel_name(_p(dash, heads_q=8), 256) == "k_attend"    # no V^T room, G < 8
     assert dash.attend_kernel_name(_p(dash, heads_q=8, flags=1), big) == "k_attend_pair"
-    assert dash.attend_kernel_name(_p(dash, heads_q=4, flags=1), big) == "k_attend"  # G = 2, chunk 64
+    assert dash.attend_kernel_name(_p(dash, heads_q=4, flags=1), big) == "k_attend_fa"  # G = 2, chunk 64
     assert dash.attend_kernel_name(_p(dash, heads_q=4, chunk_size=128, flags=2), big) == "k_attend_pair"
+    assert dash.attend_kernel_name(_p(dash, heads_q=2), big) == "k_attend"     # G = 1: 128 tokens per tile
     assert dash.attend_kernel_name(_p(dash, head_dim=64), big) == "k_attend"   # D = 64
     assert dash.attend_kernel_name(_p(dash, head_dim=96), big) == ""
     assert dash.attend_kernel_name(_p(dash), 255) == ""

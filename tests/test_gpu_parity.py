@@ -535,7 +535,8 @@ def test_paged_decode_equals_contiguous_decode(dash):
 
 # ------------------------------------------------------------------------------ fused route-and-attend
 @pytest.mark.parametrize("alpha", [1.0, 1.5, 2.0, 1.25])
-@pytest.mark.parametrize("G,Bc,T", [(16, 64, 2100 + 37), (8, 128, 1500 + 3), (32, 64, 1300)])
+@pytest.mark.parametrize("G,Bc,T", [(16, 64, 2100 + 37), (8, 128, 1500 + 3), (32, 64, 1300),
+                                    (4, 64, 1500 + 3), (2, 128, 900)])
 def test_fused_route_and_attend_equals_the_separate_stages(dash, alpha, G, Bc, T):
     """dash_prefill runs Stage 1 inside the 128-key-block Stage 2 kernel (each tile routes its
     own tokens with Stage 1's arithmetic).  Its mask, p and output equal those of the separate
