@@ -14,6 +14,8 @@ Parity status per function (pins live in ``tests/test_oracle_pins.py``):
                     exact zero weight of masked chunks)
   decode            pinned (equals the prefill row at the same position)
   decode_route      pinned (equals decode's routing, which recomputes the summaries)
+  backward          pinned (central finite differences of sum(O dO) for every input; dense
+                    mode against torch autograd of SDPA in float64)
   topk              pinned (numpy's stable argsort on the negated scores; uniform prior)
   estimate_diagonal pinned (diagonal summary = single-query SDPA over the visible keys of the
                     diagonal chunk; at a chunk's last row it is Stage 0's summary; routing =
@@ -84,6 +86,8 @@ def _get():
                                             _L, _L, _L, _L, ctypes.c_double, ctypes.c_double, _L,
                                             _dbl_p, _dbl_p, _dbl_p]
         lib.oracle_decode_route.restype = None
+        lib.oracle_backward.argtypes = [_dbl_p] * 5 + [_L] * 6 + [ctypes.c_double] * 3 + [_dbl_p] * 4
+        lib.oracle_backward.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -277,3 +281,22 @@ def decode_route(q, summary, seq_lens, cap: int, chunk_size: int, alpha: float,
                                sl.ctypes.data_as(_i64_p), B, Hq, Hkv, Cs, cap, D, chunk_size,
                                float(alpha), float(gamma), int(topk), _ptr(p), _ptr(m), _ptr(tau))
     return dict(p=p, m=m, tau=tau)
+
+
+# --------------------------------------------------------------------------- backward
+def backward(Q, K, V, head_cls, dO, chunk_size: int, alpha: float, gamma: float = 1.0,
+             sigma: float = 1.0):
+    """Gradients of sum(O * dO) w.r.t. Q, K, V, head_cls through Stages 2, 1 and 0 (default
+    routing mode).  Returns dict(dQ [B,Hq,T,D], dK, dV [B,Hkv,T,D], dhc [Hkv,D]).
+    (gist.science summary, "Stufe 1": gradients flow through the routing back to Stage 0.)"""
+    Q, K, V, hc, dO = (_f64(x) for x in (Q, K, V, head_cls, dO))
+    B, Hq, T, D = Q.shape
+    Hkv = K.shape[1]
+    dQ = np.zeros_like(Q)
+    dK = np.zeros_like(K)
+    dV = np.zeros_like(V)
+    dhc = np.zeros_like(hc)
+    _get().oracle_backward(_ptr(Q), _ptr(K), _ptr(V), _ptr(hc), _ptr(dO), B, Hq, Hkv, T, D,
+                           chunk_size, float(alpha), float(gamma), float(sigma), _ptr(dQ),
+                           _ptr(dK), _ptr(dV), _ptr(dhc))
+    return dict(dQ=dQ, dK=dK, dV=dV, dhc=dhc)

@@ -423,6 +423,137 @@ void oracle_decode_route(const double *q, const double *summary, const double *K
         }
 }
 
+/* ---------------------------------------------------------------- backward */
+
+/* Gradients of L = sum(O * dO) with respect to Q, K, V and head_cls, through all three stages
+ * (gist.science summary, "Stufe 1": alpha-entmax is differentiable, so gradients flow from the
+ * Stage 2 softmax through the routing back to the chunk summaries of Stage 0;
+ * liuzhao09.github.io "DashAttention 精读", section 2: the hierarchy trains end to end).
+ * Written from the chain rule of the forward above, one stage at a time (prefill, default
+ * mode: entmax routing, bias sigma * log p on routed chunks, diagonal with bias 0):
+ *   Stage 2, row (h, t), attention weights a_j over its attended keys, O = sum a_j v_j:
+ *     dl_j = a_j (dO . v_j - dO . O);  dq += sum_j dl_j k_j / sqrt(D);  dk_j += dl_j q / sqrt(D);
+ *     dv_j += a_j dO;  a routed chunk c (p_c > 0) collects dlogp_c += sigma * sum_{j in c} dl_j.
+ *   Routing, row (g, t): dp_c = dlogp_c / p_c on the support; with g_c = p_c^(2 - alpha)
+ *     (p_c for alpha = 1) the entmax Jacobian (Peters, Niculae & Martins 2019) gives
+ *     ds_c = g_c dp_c - g_c (sum g dp) / (sum g);  s_c = gamma qbar . S_c / sqrt(D), so
+ *     dqbar = sum_c ds_c gamma S_c / sqrt(D) (each of the G heads gets dqbar / G) and
+ *     dS_c += ds_c gamma qbar / sqrt(D).
+ *   Stage 0, chunk c with weights w = softmax(hc . k_j / sqrt(D)), S_c = sum w_j k_j:
+ *     dk_j += w_j dS_c;  dl_j = w_j (k_j . dS_c - S_c . dS_c);  dk_j += dl_j hc / sqrt(D);
+ *     dhc += dl_j k_j / sqrt(D).
+ * Outputs are overwritten; dhc [Hkv, D] sums over the batch. */
+void oracle_backward(const double *Q, const double *K, const double *V, const double *hc,
+                     const double *dO, long B, long Hq, long Hkv, long T, long D, long Bc,
+                     double alpha, double gamma, double sigma, double *dQ, double *dK,
+                     double *dV, double *dhc) {
+    long G = Hq / Hkv, Cf = T / Bc, C = (T + Bc - 1) / Bc;
+    double rs = 1.0 / sqrt((double)D);
+    for (long i = 0; i < B * Hq * T * D; ++i) dQ[i] = 0.0;
+    for (long i = 0; i < B * Hkv * T * D; ++i) { dK[i] = 0.0; dV[i] = 0.0; }
+    double *dhc_bg = (double *)calloc((size_t)(B * Hkv * D), sizeof(double));
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (long b = 0; b < B; ++b)
+        for (long g = 0; g < Hkv; ++g) {
+            const double *Kg = K + (b * Hkv + g) * T * D, *Vg = V + (b * Hkv + g) * T * D;
+            double *dKg = dK + (b * Hkv + g) * T * D, *dVg = dV + (b * Hkv + g) * T * D;
+            const double *hcg = hc + g * D;
+            /* forward: summaries */
+            double *S = (double *)calloc((size_t)((Cf > 0 ? Cf : 1) * D), sizeof(double));
+            double *dS = (double *)calloc((size_t)((Cf > 0 ? Cf : 1) * D), sizeof(double));
+            for (long c = 0; c < Cf; ++c) summarize_chunk(Kg + c * Bc * D, Bc, hcg, D, S + c * D);
+            double *qbar = (double *)malloc(sizeof(double) * (size_t)D);
+            double *pr = (double *)malloc(sizeof(double) * (size_t)C);
+            double *mr = (double *)malloc(sizeof(double) * (size_t)C);
+            double *dlogp = (double *)malloc(sizeof(double) * (size_t)C);
+            double *l = (double *)malloc(sizeof(double) * (size_t)T);
+            double *O = (double *)malloc(sizeof(double) * (size_t)D);
+            for (long t = 0; t < T; ++t) {
+                long ct = t / Bc, n = t + 1;
+                group_mean(Q + ((b * Hq + g * G) * T + t) * D, T * D, G, D, qbar);
+                route_qbar(qbar, S, ct, C, D, alpha, gamma, NULL, 0, pr, mr);
+                for (long c = 0; c < C; ++c) dlogp[c] = 0.0;
+                for (long h = g * G; h < (g + 1) * G; ++h) {
+                    const double *q = Q + ((b * Hq + h) * T + t) * D;
+                    const double *dOr = dO + ((b * Hq + h) * T + t) * D;
+                    double *dq = dQ + ((b * Hq + h) * T + t) * D;
+                    /* forward row: logits, weights (exact maximum), O */
+                    double mx = -INFINITY;
+                    for (long j = 0; j < n; ++j) {
+                        long c = j / Bc;
+                        if (c == ct) l[j] = dotd(q, Kg + j * D, D) * rs;
+                        else if (pr[c] > 0.0) l[j] = dotd(q, Kg + j * D, D) * rs + sigma * log(pr[c]);
+                        else l[j] = -INFINITY;
+                        if (l[j] > mx) mx = l[j];
+                    }
+                    double den = 0.0;
+                    for (long j = 0; j < n; ++j) { l[j] = l[j] == -INFINITY ? 0.0 : exp(l[j] - mx); den += l[j]; }
+                    for (long d = 0; d < D; ++d) O[d] = 0.0;
+                    for (long j = 0; j < n; ++j) {
+                        l[j] /= den;                                /* l now holds a_j */
+                        for (long d = 0; d < D; ++d) O[d] += l[j] * Vg[j * D + d];
+                    }
+                    double dOO = dotd(dOr, O, D);
+                    for (long j = 0; j < n; ++j) {
+                        if (l[j] == 0.0) continue;
+                        double dl = l[j] * (dotd(dOr, Vg + j * D, D) - dOO);
+                        for (long d = 0; d < D; ++d) {
+                            dq[d] += dl * Kg[j * D + d] * rs;
+                            dKg[j * D + d] += dl * q[d] * rs;
+                            dVg[j * D + d] += l[j] * dOr[d];
+                        }
+                        long c = j / Bc;
+                        if (c < ct) dlogp[c] += sigma * dl;
+                    }
+                }
+                if (ct == 0) continue;
+                /* routing backward: entmax Jacobian on the support */
+                double sg = 0.0, sgdp = 0.0;
+                for (long c = 0; c < ct; ++c) {
+                    if (!(pr[c] > 0.0)) continue;
+                    double gc = alpha == 1.0 ? pr[c] : pow(pr[c], 2.0 - alpha);
+                    sg += gc;
+                    sgdp += gc * dlogp[c] / pr[c];
+                }
+                for (long c = 0; c < ct; ++c) {
+                    if (!(pr[c] > 0.0)) continue;
+                    double gc = alpha == 1.0 ? pr[c] : pow(pr[c], 2.0 - alpha);
+                    double ds = gc * dlogp[c] / pr[c] - gc * sgdp / sg;
+                    for (long d = 0; d < D; ++d) {
+                        double dqb = ds * gamma * S[c * D + d] * rs;
+                        for (long h = g * G; h < (g + 1) * G; ++h)
+                            dQ[((b * Hq + h) * T + t) * D + d] += dqb / (double)G;
+                        dS[c * D + d] += ds * gamma * qbar[d] * rs;
+                    }
+                }
+            }
+            /* Stage 0 backward */
+            double *w = (double *)malloc(sizeof(double) * (size_t)Bc);
+            for (long c = 0; c < Cf; ++c) {
+                const double *kc = Kg + c * Bc * D;
+                double mx = -INFINITY, den = 0.0, sdS = dotd(S + c * D, dS + c * D, D);
+                for (long j = 0; j < Bc; ++j) { w[j] = dotd(hcg, kc + j * D, D) * rs; if (w[j] > mx) mx = w[j]; }
+                for (long j = 0; j < Bc; ++j) { w[j] = exp(w[j] - mx); den += w[j]; }
+                for (long j = 0; j < Bc; ++j) {
+                    w[j] /= den;
+                    double dl = w[j] * (dotd(kc + j * D, dS + c * D, D) - sdS);
+                    for (long d = 0; d < D; ++d) {
+                        dKg[(c * Bc + j) * D + d] += w[j] * dS[c * D + d] + dl * hcg[d] * rs;
+                        dhc_bg[(b * Hkv + g) * D + d] += dl * kc[j * D + d] * rs;
+                    }
+                }
+            }
+            free(w); free(S); free(dS); free(qbar); free(pr); free(mr); free(dlogp); free(l); free(O);
+        }
+    for (long g = 0; g < Hkv; ++g)
+        for (long d = 0; d < D; ++d) {
+            double acc = 0.0;
+            for (long b = 0; b < B; ++b) acc += dhc_bg[(b * Hkv + g) * D + d];
+            dhc[g * D + d] = acc;
+        }
+    free(dhc_bg);
+}
+
 /* Number of OpenMP threads the oracle runs with (for reporting). */
 int oracle_num_threads(void) {
 #ifdef _OPENMP

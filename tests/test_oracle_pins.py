@@ -503,3 +503,79 @@ def test_topk_prefill_attends_the_selection_with_a_uniform_prior():
     ref = F.scaled_dot_product_attention(q.double(), k.double().repeat_interleave(16, 1),
                                          v.double().repeat_interleave(16, 1), attn_mask=mask)
     np.testing.assert_allclose(r["O"], ref.numpy(), atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- backward
+def _tiny_problem(seed, B=1, Hq=4, Hkv=2, T=40, D=8, Bc=8):
+    g = torch.Generator().manual_seed(seed)
+    Q = torch.randn(B, Hq, T, D, generator=g, dtype=torch.float64)
+    K = torch.randn(B, Hkv, T, D, generator=g, dtype=torch.float64)
+    V = torch.randn(B, Hkv, T, D, generator=g, dtype=torch.float64)
+    hc = torch.randn(Hkv, D, generator=g, dtype=torch.float64)
+    dO = torch.randn(B, Hq, T, D, generator=g, dtype=torch.float64)
+    return Q, K, V, hc, dO
+
+
+def _loss(Q, K, V, hc, dO, Bc, alpha, sigma):
+    return float((oracle.prefill(Q, K, V, hc, Bc, alpha, sigma=sigma)["O"] * dO.numpy()).sum())
+
+
+@pytest.mark.parametrize("alpha,sigma", [(1.5, 1.0), (2.0, 0.5), (1.0, 1.0), (1.25, 2.0)])
+def test_backward_matches_central_finite_differences(alpha, sigma):
+    """The oracle's gradients of sum(O * dO) through Stages 2, 1 and 0 against central finite
+    differences of its own forward, for sampled entries of every input (the entmax supports
+    are fixed under the perturbation: every margin lies well away from zero)."""
+    Bc = 8
+    for seed in range(40):                       # a problem whose routing margins are not tiny
+        Q, K, V, hc, dO = _tiny_problem(seed)
+        r = oracle.prefill(Q, K, V, hc, Bc, alpha, sigma=sigma)
+        m = r["m"][np.isfinite(r["m"])]
+        if alpha == 1.0 or np.abs(m).min() > 1e-3:
+            break
+    else:
+        pytest.skip("no problem with clear margins")
+    gr = oracle.backward(Q, K, V, hc, dO, Bc, alpha, sigma=sigma)
+    rng = np.random.default_rng(seed)
+    eps = 1e-6
+    for name, X, dX in (("Q", Q, gr["dQ"]), ("K", K, gr["dK"]), ("V", V, gr["dV"]), ("hc", hc, gr["dhc"])):
+        flat = X.view(-1)
+        for idx in rng.choice(flat.numel(), 12, replace=False):
+            old = float(flat[idx])
+            flat[idx] = old + eps
+            lp = _loss(Q, K, V, hc, dO, Bc, alpha, sigma)
+            flat[idx] = old - eps
+            lm = _loss(Q, K, V, hc, dO, Bc, alpha, sigma)
+            flat[idx] = old
+            fd = (lp - lm) / (2 * eps)
+            an = dX.reshape(-1)[idx]
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(fd)), (name, idx, fd, an)
+    # the routing gradient reaches head_cls (Stage 0): not identically zero
+    assert np.abs(gr["dhc"]).max() > 1e-6
+
+
+def test_backward_without_the_prior_is_masked_attention_backward():
+    """sigma = 0 removes the routing from the gradient (the bias is zero on every attended key),
+    so dQ, dK, dV are the gradients of plain softmax attention restricted to the routed chunks
+    and the diagonal -- torch autograd through scaled_dot_product_attention in float64 with
+    that mask -- and head_cls gets no gradient."""
+    import torch.nn.functional as F
+    Q, K, V, hc, dO = _tiny_problem(3, T=48)
+    Bc, T = 8, 48
+    r = oracle.prefill(Q, K, V, hc, Bc, 1.5, sigma=0.0)
+    gr = oracle.backward(Q, K, V, hc, dO, Bc, 1.5, sigma=0.0)
+    ct = np.arange(T) // Bc
+    keep = np.zeros((2, T, T), bool)
+    for g in range(2):
+        for t in range(T):
+            for j in range(t + 1):
+                c = j // Bc
+                keep[g, t, j] = c == ct[t] or r["p"][0, g, t, c] > 0
+    mask = torch.from_numpy(np.repeat(keep, 2, axis=0))[None]
+    q, k, v = (x.clone().requires_grad_(True) for x in (Q, K, V))
+    O = F.scaled_dot_product_attention(q, k.repeat_interleave(2, 1), v.repeat_interleave(2, 1),
+                                       attn_mask=mask)
+    (O * dO).sum().backward()
+    np.testing.assert_allclose(gr["dQ"], q.grad.numpy(), atol=1e-12)
+    np.testing.assert_allclose(gr["dK"], k.grad.numpy(), atol=1e-12)
+    np.testing.assert_allclose(gr["dV"], v.grad.numpy(), atol=1e-12)
+    assert np.abs(gr["dhc"]).max() == 0.0
