@@ -282,6 +282,29 @@ dash_status_t dash_decode_paged(const dash_params_t *params, const void *q, cons
                                 uint64_t *active_blocks, void *ws, size_t ws_bytes,
                                 void *stream);
 
+/* Bytes of device workspace dash_backward needs (the routing it recomputes with p, the
+ * gradient into p, per-row softmax statistics, group-mean queries, the routing transposed to
+ * per-chunk token lists, and the summaries' gradient).  0 on bad parameters. */
+size_t dash_backward_workspace_size(const dash_params_t *params);
+
+/* Backward pass of the causal prefill: the gradients of L = sum(out * dout) with respect to q,
+ * k, v and head_cls, through Stage 2 (the attention and its prior bias sigma * log p), Stage 1
+ * (the alpha-entmax routing: its Jacobian on the support) and Stage 0 (the chunk summaries).
+ * gist.science "DashAttention ..." summary, "Stufe 1": alpha-entmax is differentiable, so the
+ * gradient flows from the Stage 2 softmax through the routing back to the summaries of Stage 0.
+ *   q, k, v, head_cls: the forward's inputs (layouts of dash_prefill); out: its output;
+ *   dout [B, H_q, T, D] bf16: the gradient of L with respect to out;
+ *   dq [B, H_q, T, D], dk, dv [B, H_kv, T, D], dhc [H_kv, D] fp32 (out, overwritten; dhc sums
+ *   over the batch).
+ * The default routing only: DASH_FLAG_DENSE, DASH_FLAG_FORCE_ALL_ACTIVE,
+ * DASH_FLAG_ESTIMATE_DIAGONAL and top-k return DASH_ERR_UNSUPPORTED.  Probabilities are
+ * recomputed in fp32 (not rounded to bf16 as in the forward's P V); the gradient operands of
+ * the warp-level MMAs are rounded to bf16. */
+dash_status_t dash_backward(const dash_params_t *params, const void *q, const void *k,
+                            const void *v, const float *head_cls, const void *out,
+                            const void *dout, float *dq, float *dk, float *dv, float *dhc,
+                            void *ws, size_t ws_bytes, void *stream);
+
 /* Size of the device array that dash_prefill_static_ws uses as its workspace. */
 #define DASH_STATIC_WS_BYTES (16u << 20)
 

@@ -43,7 +43,7 @@ EXPORTS = ("dash_prefill_workspace_size", "dash_prefill", "dash_prefill_host", "
            "dash_attend_workspace_size", "dash_attend", "dash_update_chunk_cache", "dash_decode_workspace_size",
            "dash_decode", "dash_read_device_status", "dash_status_string", "dash_prefill_static_ws",
            "dash_static_ws_read_status", "dash_attend_kernel_name", "dash_decode_paged",
-           "dash_update_chunk_cache_paged")
+           "dash_update_chunk_cache_paged", "dash_backward", "dash_backward_workspace_size")
 
 
 class Params(ctypes.Structure):
@@ -84,6 +84,10 @@ def _declare(lib):
     lib.dash_update_chunk_cache.argtypes = [_P, _vp, _vp, _vp, ctypes.c_int, _vp, _vp, _sz, _vp]
     lib.dash_decode.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
     lib.dash_read_device_status.argtypes = [_vp, _vp]
+    lib.dash_backward_workspace_size.argtypes = [_P]
+    lib.dash_backward_workspace_size.restype = _sz
+    lib.dash_backward.argtypes = [_P] + [_vp] * 11 + [_sz, _vp]
+    lib.dash_backward.restype = ctypes.c_int
     lib.dash_decode_paged.argtypes = [_P, _vp, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int, _vp, _vp,
                                       _vp, _vp, _vp, _vp, _vp, _sz, _vp]
     lib.dash_update_chunk_cache_paged.argtypes = [_P, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int,
@@ -339,7 +343,7 @@ def update_chunk_cache_paged(k_pool, head_cls, block_table, seq_lens, summary_po
                                              _ptr(block_table), int(max_blocks), int(n_pages),
                                              _ptr(seq_lens), int(n_recent), _ptr(summary_pool),
                                              _ptr(ws), ws.numel(), _stream(k_pool.device)),
-           "dash_update_chunk_cache_paged")
+           "dash_update_chunk_cache_paged", "dash_backward", "dash_backward_workspace_size")
     return summary_pool
 
 
@@ -369,6 +373,29 @@ def decode_paged(q, k_pool, v_pool, block_table, seq_lens, summary_pool, chunk_s
     if not (return_p or return_active_blocks):
         return out
     return dict(out=out, p=p, active_blocks=mask)
+
+
+def backward(q, k, v, head_cls, out, dout, chunk_size=64, alpha=1.5, gamma=1.0, sigma=1.0,
+             enable_gqa=True, ws=None):
+    """Gradients of sum(out * dout) w.r.t. q, k, v, head_cls (fp32 tensors) through the three
+    stages.  out is the forward's output for the same arguments."""
+    B, Hq, T, D = q.shape
+    Hkv = k.shape[1]
+    dev = q.device
+    prm = make_params(B, Hq, Hkv, T, D, chunk_size, alpha, gamma, sigma, enable_gqa)
+    for name, t_, dt in (("q", q, torch.bfloat16), ("k", k, torch.bfloat16), ("v", v, torch.bfloat16),
+                         ("out", out, torch.bfloat16), ("dout", dout, torch.bfloat16)):
+        _need(t_, dt, tuple(t_.shape), name)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=dev)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=dev)
+    dhc = torch.empty(head_cls.shape, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = workspace(lib.dash_backward_workspace_size(ctypes.byref(prm)), dev)
+    _check(lib.dash_backward(ctypes.byref(prm), _ptr(q), _ptr(k), _ptr(v), _ptr(head_cls), _ptr(out),
+                             _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dhc), _ptr(ws), ws.numel(),
+                             _stream(dev)), "dash_backward")
+    return dict(dq=dq, dk=dk, dv=dv, dhc=dhc, ws=ws)
 
 
 def read_device_status(ws) -> int:

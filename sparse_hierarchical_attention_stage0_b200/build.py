@@ -24,7 +24,7 @@ BUILD = os.path.join(HERE, "_build")
 LIB_DEBUG = os.path.join(HERE, "libdash_debug.so")
 BUILD_DEBUG = os.path.join(HERE, "_build_debug")
 SOURCES = ["stage0.cu", "route.cu", "attend.cu", "attend_tc.cu", "attend_fa.cu", "attend_pair.cu", "vtranspose.cu",
-           "decode.cu", "dash_api.cu", "dash_static_ws.cu"]
+           "decode.cu", "backward.cu", "dash_api.cu", "dash_static_ws.cu"]
 HEADERS = ["dash_common.cuh", "kernels.cuh", "attn_warp.cuh", "tc_common.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

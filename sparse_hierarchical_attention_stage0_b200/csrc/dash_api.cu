@@ -564,6 +564,79 @@ dash_status_t dash_update_chunk_cache_paged(const dash_params_t *p, const void *
     return from_cuda(launch_stage0_paged(a, seq_lens, n_recent, block_table, max_blocks, n_pages, st));
 }
 
+size_t dash_backward_workspace_size(const dash_params_t *p) {
+    Shape s;
+    if (check_params(p, &s) != DASH_OK) return 0;
+    const size_t bhkv = (size_t)s.B * s.Hkv;
+    size_t n = kStatusBytes + bytes_tau(s) + bytes_summary(s) + bytes_mask(s);
+    n += 2 * align256(bhkv * s.T * s.C * 4);                     // p, d log p
+    n += 3 * align256((size_t)s.B * s.Hq * s.T * 4);             // row max, sum, delta
+    n += align256(bhkv * s.T * s.D * 4);                         // qbar
+    n += align256(bhkv * s.C * 4) + align256(bhkv * (s.C + 1) * 8);   // list counts, offsets
+    n += align256(bhkv * (size_t)backward_nnz_max(s.T, s.Bc) * 4);     // lists
+    n += align256(bytes_summary(s));                             // d summaries
+    return n;
+}
+
+dash_status_t dash_backward(const dash_params_t *p, const void *q, const void *k, const void *v,
+                            const float *head_cls, const void *out, const void *dout, float *dq,
+                            float *dk, float *dv, float *dhc, void *ws, size_t ws_bytes,
+                            void *stream) {
+    Shape s;
+    dash_status_t rc = check_params(p, &s);
+    if (rc != DASH_OK) return rc;
+    if (p->flags & (DASH_FLAG_DENSE | DASH_FLAG_FORCE_ALL_ACTIVE | DASH_FLAG_ESTIMATE_DIAGONAL) ||
+        p->topk > 0)
+        return DASH_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !head_cls || !out || !dout || !dq || !dk || !dv || !dhc || !ws)
+        return DASH_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(head_cls) || !aligned16(out) ||
+        !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(dhc) ||
+        (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return DASH_ERR_INVALID_ARGUMENT;
+    if (route_rows_per_cta(s.C, s.D) == 0) return DASH_ERR_UNSUPPORTED;
+    if (ws_bytes < dash_backward_workspace_size(p)) return DASH_ERR_WORKSPACE_TOO_SMALL;
+    unsigned char *w = static_cast<unsigned char *>(ws);
+    const size_t bhkv = (size_t)s.B * s.Hkv;
+    StageArgs a = stage_args(p, s);
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.head_cls = head_cls;
+    a.status = reinterpret_cast<uint32_t *>(w);
+    size_t off = kStatusBytes;
+    auto take = [&](size_t bytes) { unsigned char *r = w + off; off += align256(bytes); return r; };
+    a.tau = reinterpret_cast<float *>(take((size_t)s.B * s.Hkv * s.T * 4));
+    a.summary = reinterpret_cast<float *>(take((size_t)s.B * s.Hkv * s.Cf * s.D * 4));
+    a.mask = reinterpret_cast<uint64_t *>(take((size_t)s.B * s.Hkv * s.T * s.W * 8));
+    a.p = reinterpret_cast<float *>(take(bhkv * s.T * s.C * 4));
+    BackwardBuffers bb;
+    bb.dout = dout;
+    bb.out = out;
+    bb.dq = dq;
+    bb.dk = dk;
+    bb.dv = dv;
+    bb.dhc = dhc;
+    bb.dlogp = reinterpret_cast<float *>(take(bhkv * s.T * s.C * 4));
+    bb.row_m = reinterpret_cast<float *>(take((size_t)s.B * s.Hq * s.T * 4));
+    bb.row_l = reinterpret_cast<float *>(take((size_t)s.B * s.Hq * s.T * 4));
+    bb.row_delta = reinterpret_cast<float *>(take((size_t)s.B * s.Hq * s.T * 4));
+    bb.qbar = reinterpret_cast<float *>(take(bhkv * s.T * s.D * 4));
+    bb.list_cnt = reinterpret_cast<int *>(take(bhkv * s.C * 4));
+    bb.list_off = reinterpret_cast<long long *>(take(bhkv * (s.C + 1) * 8));
+    bb.list = reinterpret_cast<int *>(take(bhkv * (size_t)backward_nnz_max(s.T, s.Bc) * 4));
+    bb.dsum = reinterpret_cast<float *>(take((size_t)s.B * s.Hkv * s.Cf * s.D * 4));
+    bb.sigma = p->sigma;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((rc = clear_status(ws, st)) != DASH_OK) return rc;
+    if ((rc = from_cuda(cudaMemsetAsync(bb.dlogp, 0, bhkv * s.T * s.C * 4, st))) != DASH_OK) return rc;
+    if ((rc = from_cuda(cudaMemsetAsync(dhc, 0, (size_t)s.Hkv * s.D * 4, st))) != DASH_OK) return rc;
+    // The forward's routing (with p), then the backward kernels.
+    if ((rc = from_cuda(launch_stage0(a, nullptr, 0, st))) != DASH_OK) return rc;
+    if ((rc = from_cuda(launch_route(a, st))) != DASH_OK) return rc;
+    return from_cuda(launch_backward(a, bb, st));
+}
+
 const char *dash_attend_kernel_name(const dash_params_t *p, size_t ws_bytes) {
     Shape s;
     if (check_params(p, &s) != DASH_OK || ws_bytes < kStatusBytes) return "";

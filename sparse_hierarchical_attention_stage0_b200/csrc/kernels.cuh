@@ -73,6 +73,25 @@ bool attend_pair_supported(const StageArgs &a);
 cudaError_t launch_attend_pair(const StageArgs &a, cudaStream_t st);
 cudaError_t launch_vtranspose(const void *v, void *vt, int BHkv, int T, int D, cudaStream_t st);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
+
+// Buffers of the backward pass (dash_backward); the StageArgs carry the forward's routing
+// (summary, tau, mask, p).
+struct BackwardBuffers {
+    const void *dout, *out;   // [B,Hq,T,D] bf16
+    float *dq;                // [B,Hq,T,D]
+    float *dk, *dv;           // [B,Hkv,T,D]
+    float *dhc;               // [Hkv,D]
+    float *dlogp;             // [B,Hkv,T,C]
+    float *row_m, *row_l, *row_delta;   // [B,Hq,T]
+    float *qbar;              // [B,Hkv,T,D]
+    int *list_cnt;            // [B*Hkv][C]
+    long long *list_off;      // [B*Hkv][C+1]
+    int *list;                // [B*Hkv][backward_nnz_max]
+    float *dsum;              // [B,Hkv,Cf,D]
+    float sigma;
+};
+long long backward_nnz_max(int T, int Bc);
+cudaError_t launch_backward(const StageArgs &s, const BackwardBuffers &bb, cudaStream_t st);
 int decode_supported(int G, int Ccap, int D);
 // Scratch bytes dash_prefill needs in its workspace (status word, tau, and the summaries /
 // mask words not supplied by the caller); 0 on bad parameters.

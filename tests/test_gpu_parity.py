@@ -558,3 +558,36 @@ def test_fused_route_and_attend_equals_the_separate_stages(dash, alpha, G, Bc, T
     check_routing(unpack_mask(res["active_blocks"], C), res["p"].cpu().double().numpy(),
                   ref["p"], ref["m"], np.arange(T), Bc, alpha, tag="fused")
     check_output(res["out"].cpu().float().numpy(), ref["O"], tag="fused")
+
+
+# ------------------------------------------------------------------------------ backward
+def _grad_check(name, got, ref, rel_max=2e-2, rel_mean=2e-3):
+    """Gradient parity: errors measured against the largest reference magnitude (the gradients
+    sum many terms, each rounded to bf16 on its way into the warp-level MMAs)."""
+    got = np.asarray(got, dtype=np.float64)
+    scale = max(np.abs(ref).max(), 1e-30)
+    err = np.abs(got - ref)
+    assert np.isfinite(got).all(), f"{name}: non-finite"
+    assert err.max() <= rel_max * scale, f"{name}: max err {err.max():.3e} vs scale {scale:.3e}"
+    assert err.mean() <= rel_mean * scale, f"{name}: mean err {err.mean():.3e} vs scale {scale:.3e}"
+    return err.max() / scale
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0, 1.0])
+@pytest.mark.parametrize("G,D,Bc,T", [(16, 128, 64, 700), (4, 128, 128, 600 + 7), (1, 64, 64, 333),
+                                      (32, 128, 64, 400)])
+def test_backward_matches_oracle(dash, alpha, G, D, Bc, T):
+    """The gradients of sum(out * dout) w.r.t. q, k, v and head_cls through Stages 2, 1 and 0
+    (dash_backward) against the oracle's backward."""
+    Hkv = 2 if G <= 16 else 1
+    q, k, v, hc = make_prefill(_cfg(1, G * Hkv, Hkv, T, D, Bc, alpha, seed=110 + G))
+    g_ = torch.Generator().manual_seed(7)
+    dout = torch.randn(q.shape, generator=g_).to(torch.bfloat16)
+    qd, kd, vd, hcd, dd = _to(q, k, v, hc, dout)
+    out = dash.prefill(qd, kd, vd, hcd, Bc, alpha, enable_gqa=True)
+    gr = dash.backward(qd, kd, vd, hcd, out, dd, Bc, alpha)
+    torch.cuda.synchronize()
+    assert dash.read_device_status(gr["ws"]) == 0
+    ref = oracle.backward(q, k, v, hc, dout, Bc, alpha)
+    for name, key in (("dq", "dQ"), ("dk", "dK"), ("dv", "dV"), ("dhc", "dhc")):
+        _grad_check(f"{name} G={G} a={alpha}", gr[name].cpu().numpy(), ref[key])
