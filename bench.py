@@ -160,7 +160,27 @@ def active_stats(dash, q, k, v, hc, cfg):
     dense_flops = 4.0 * D * G * cfg.batch * cfg.heads_kv * (T * (T + 1) / 2.0)
     sparsity = 1.0 - float(active / visible) if visible > 0 else 0.0
     return dict(active_flops=float(flops), dense_flops=float(dense_flops), sparsity=sparsity,
-                active_chunks=float(active), visible_chunks=float(visible), words=words)
+                active_chunks=float(active), visible_chunks=float(visible), words=words,
+                support=support_histogram(cnt))
+
+
+def support_histogram(cnt: torch.Tensor) -> dict:
+    """Entmax support sizes (routed active chunks per row, diagonal excluded) as a histogram
+    over power-of-two bins, with quantiles: how adaptive the routing was."""
+    c = cnt.flatten().to(torch.int64)
+    edges = [0, 1, 2, 4, 8, 16, 32, 64, 128, 256, 512, 1024, 2048, 4096, 8192]
+    bins = {}
+    for lo, hi in zip(edges[:-1], edges[1:]):
+        n = int(((c >= lo) & (c < hi)).sum())
+        if n:
+            bins[f"{lo}-{hi - 1}"] = n
+    n_big = int((c >= edges[-1]).sum())
+    if n_big:
+        bins[f">={edges[-1]}"] = n_big
+    q = torch.quantile(c[:1 << 24].to(torch.float64), torch.tensor([0.1, 0.5, 0.9, 0.99], dtype=torch.float64, device=c.device))
+    return {"rows": int(c.numel()), "bins": bins, "mean": float(c.to(torch.float64).mean()),
+            "p10": float(q[0]), "p50": float(q[1]), "p90": float(q[2]), "p99": float(q[3]),
+            "max": int(c.max()) if c.numel() else 0}
 
 
 def tokens_per_tile(kernel: str, G: int) -> int:
@@ -340,14 +360,16 @@ def bench_decode(dash, dev, steps_cap=256, warmup=3):
     for _ in range(3):
         st = torch.cuda.Event(enable_timing=True)
         en = torch.cuda.Event(enable_timing=True)
-        st.record(stream)
-        g.replay()
-        en.record(stream)
+        with torch.cuda.stream(stream):               # replay launches on the current stream
+            st.record(stream)
+            g.replay()
+            en.record(stream)
         en.synchronize()
         times.append(st.elapsed_time(en))
     ms = statistics.median(times)
     launches = S + sum(1 for s in range(S) if (L0 + s + 1) % Bc == 0)
     del g
+    kern = bench_decode_kernel(dash, dev, cfg, q_steps, kc, vc, seq, cache, out, ws, S, stream)
     paged_ms = bench_decode_paged(dash, dev, d, cfg, S, warmup)
     return dict(tokens_per_s=B * S / (ms / 1e3), ms_per_step=ms / S, steps=S, batch=B,
                 paged={"ms_per_step": paged_ms / S, "tokens_per_s": B * S / (paged_ms / 1e3),
@@ -356,7 +378,56 @@ def bench_decode(dash, dev, steps_cap=256, warmup=3):
                 cache_len=L0, realised_sparsity=sparsity,
                 hbm_bytes_per_step=alg_bytes / S,
                 achieved_gbs=alg_bytes / (ms / 1e3) / 1e9, launches=launches,
+                kernel=dict(us_l2_warm=kern["warm_us"], us_l2_cold=kern["cold_us"],
+                            gbs_l2_cold=alg_bytes / S / (kern["cold_us"] / 1e6) / 1e9,
+                            note="k_decode alone, 256 launches per graph at the last step's cache "
+                                 "length; cold: each launch after a 256 MiB L2-flushing write, "
+                                 "the graph of writes alone subtracted"),
                 note="steps include the K/V append copies and seq_len update (torch ops)")
+
+
+def bench_decode_kernel(dash, dev, cfg, q_steps, kc, vc, seq, cache, out, ws, S, stream):
+    """k_decode alone: S launches in one graph (L2 warm across launches), and S launches each
+    after an L2-flushing write, minus the graph of the writes alone (L2 cold).  Microseconds per
+    launch, medians of three replays."""
+    Bc = cfg.chunk_size
+    flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def graph_us(body):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            body()
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g, stream=stream):
+                body()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(3):
+            st = torch.cuda.Event(enable_timing=True)
+            en = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                st.record(stream)
+                g.replay()
+                en.record(stream)
+            en.synchronize()
+            ts.append(st.elapsed_time(en) * 1e3)
+        del g
+        return statistics.median(ts)
+
+    def decodes(flush):
+        for s in range(S):
+            if flush:
+                flush_buf.zero_()
+            dash.decode(q_steps[s], kc, vc, seq, cache, Bc, cfg.alpha, out=out, ws=ws)
+
+    def flushes():
+        for _ in range(S):
+            flush_buf.zero_()
+
+    warm = graph_us(lambda: decodes(False)) / S
+    cold = (graph_us(lambda: decodes(True)) - graph_us(flushes)) / S
+    assert dash.read_device_status(ws) == 0
+    return {"warm_us": warm, "cold_us": cold}
 
 
 def bench_decode_paged(dash, dev, d, cfg, S, warmup):
@@ -413,9 +484,10 @@ def bench_decode_paged(dash, dev, d, cfg, S, warmup):
     for _ in range(3):
         st = torch.cuda.Event(enable_timing=True)
         en = torch.cuda.Event(enable_timing=True)
-        st.record(stream)
-        g.replay()
-        en.record(stream)
+        with torch.cuda.stream(stream):               # replay launches on the current stream
+            st.record(stream)
+            g.replay()
+            en.record(stream)
         en.synchronize()
         times.append(st.elapsed_time(en))
     assert dash.read_device_status(ws) == 0 and dash.read_device_status(ws_u) == 0
@@ -548,8 +620,10 @@ def main():
             torch.cuda.empty_cache()
             pk, _ = peaks()
             dec = bench_decode(dash, dev)
-            dec["roofline"] = {"bound": "hbm", "achieved": dec["achieved_gbs"], "peak": pk["hbm_gbs"],
-                               "unit": "GB/s", "frac": dec["achieved_gbs"] / pk["hbm_gbs"],
+            kg = dec["kernel"]["gbs_l2_cold"]
+            dec["roofline"] = {"bound": "hbm", "kernel": "k_decode (alone, L2 flushed before each launch)",
+                               "achieved": kg, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                               "frac": kg / pk["hbm_gbs"],
                                "traffic": traffic_for("k_decode", "decode64k")}
             line["decode"] = dec
         if rank == 0 and world == 1:
@@ -633,10 +707,13 @@ def bench_prefill(dash, cfg, args, dev, world, rank, full=True):
     stats = active_stats(dash, q, k, v, hc, cfg)
     # The Stage 2 kernel dash_attend runs with the bench's workspace (the library names it);
     # the 128-key-block kernels also transpose V (timed together with them as Stage 2).
-    s2_kernel = dash.attend_kernel_name(prm, ws_a.numel())
-    with_vt = s2_kernel in ("k_attend_fa", "k_attend_pair")
+    s2_dispatch = dash.attend_kernel_name(prm, ws_a.numel())
+    with_vt = s2_dispatch in ("k_attend_fa", "k_attend_pair", "k_attend_fa|k_attend")
+    # Chosen at run time (fewer than 8 query heads per KV head): the kernel the timed calls ran.
+    s2_kernel = (dash.stage2_kernel_ran(ws_a) or s2_dispatch) if "|" in s2_dispatch else s2_dispatch
     s2_note = ", V^T transpose included" if with_vt else ""
-    launches_per_step = 3 + (1 if with_vt else 0)   # k_stage0, k_route, [k_vtranspose,] Stage 2
+    # k_stage0, [k_route,] [k_vtranspose,] Stage 2: as the library reports for this workspace
+    launches_per_step = dash.prefill_kernel_count(prm, ws.numel())
     un = union_stats(stats.pop("words"), Bc, D, cfg.group, tokens_per_tile(s2_kernel, cfg.group))
 
     def dense():
@@ -663,6 +740,7 @@ def bench_prefill(dash, cfg, args, dev, world, rank, full=True):
                    "l2": "flushed (256 MiB write) before every timed step"},
         "active_tflops": s2_tflops,
         "realised_sparsity": stats["sparsity"],
+        "support": stats.pop("support"),
         "stage_ms": stage,
         "stage01_gbs": s01_gbs,
         "dense_ms": dense_ms,
@@ -748,11 +826,13 @@ def bench_decode_line(dash, args, dev, world):
                        "head_dim": cfg.head_dim, "chunk_size": cfg.chunk_size, "alpha": cfg.alpha,
                        "parallelism": f"replicas x{world}",
                        "l2": "not flushed between steps (one graph of 256 steps)"},
-            "roofline": {"bound": "hbm", "kernel": "k_decode", "achieved": dec["achieved_gbs"],
+            "roofline": {"bound": "hbm", "kernel": "k_decode (alone, L2 flushed before each launch)",
+                         "achieved": dec["kernel"]["gbs_l2_cold"],
                          "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": dec["achieved_gbs"] / pk["hbm_gbs"],
+                         "frac": dec["kernel"]["gbs_l2_cold"] / pk["hbm_gbs"],
                          "traffic": traffic_for("k_decode", "decode64k"),
-                         "peak_source": f"{pk_kind} copy bandwidth"},
+                         "peak_source": f"{pk_kind} copy bandwidth",
+                         "algorithmic": f"{dec['hbm_bytes_per_step']:.4e} bytes per launch"},
             "decode": dec, "gpu_launches": dec["launches"], "clocks": clk.summary()}
 
 
@@ -770,11 +850,12 @@ def bench_sweep(dash, args, dev, world, rank):
         r = bench_prefill(dash, cfg, args, dev, world, rank, full=False)
         cells.append({"alpha": cfg.alpha, "chunk_size": cfg.chunk_size, "ms_per_step": r["ms_per_step"],
                       "tokens_per_s": r["value"], "active_tflops": r["active_tflops"],
-                      "realised_sparsity": r["realised_sparsity"], "stage_ms": r["stage_ms"],
+                      "realised_sparsity": r["realised_sparsity"], "support": r["support"],
+                      "stage_ms": r["stage_ms"],
                       "stage01_gbs": r["stage01_gbs"], "dense_ms": r["dense_ms"],
                       "dense_kernel": r["dense_kernel"], "speedup_vs_dense": r["speedup_vs_dense"],
                       "union": r["union"], "stage2_kernel": r["union"]["kernel"],
-                      "clocks": r["clocks"]})
+                      "gpu_launches": r["gpu_launches"], "clocks": r["clocks"]})
         tokens += cfg.batch * cfg.seq_len * args.steps * world
         ms += r["ms_per_step"] * args.steps
     cfg0 = sweep_config(0)
@@ -788,8 +869,7 @@ def bench_sweep(dash, args, dev, world, rank):
                        "head_dim": cfg0.head_dim, "alphas": list(SWEEP_ALPHAS),
                        "chunk_sizes": list(SWEEP_CHUNKS), "parallelism": f"replicas x{world}",
                        "l2": "flushed (256 MiB write) before every timed step"},
-            "gpu_launches": sum(4 if c["union"]["kernel"] in ("k_attend_fa", "k_attend_pair") else 3
-                                for c in cells) * args.steps,
+            "gpu_launches": sum(c["gpu_launches"] for c in cells),
             "cells": cells}
 
 

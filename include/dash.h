@@ -69,10 +69,11 @@ typedef enum {
                                         diagonal chunk) that the row's probabilities were
                                         clamped or their sum overflowed fp32; the output of
                                         that row is not exact */
-    DASH_ERR_BOUNDS = 7              /* debug builds only (libdash_debug.so, compiled with
-                                        DASH_DEBUG): a device-side bounds check failed; the
-                                        access it guarded was skipped, the output is not
-                                        meaningful.  The release library never reports it. */
+    DASH_ERR_BOUNDS = 7              /* a device-side bounds check failed; the access it
+                                        guarded was skipped, the output is not meaningful.
+                                        Debug builds (libdash_debug.so, compiled with
+                                        DASH_DEBUG) check every kernel; the release library
+                                        checks only the index lists dash_backward builds. */
 } dash_status_t;
 
 enum {
@@ -220,10 +221,28 @@ dash_status_t dash_attend(const dash_params_t *params, const void *q, const void
  * ws_bytes (dash_prefill with the same flags and a workspace that leaves ws_bytes after its
  * status word, tau, summaries and mask words picks the same one): "k_attend_pair" (dense
  * modes on pairs of SMs), "k_attend_fa" (128-key blocks), "k_attend_tc" (64-key blocks, no
- * V^T scratch) or "k_attend" (warp-level MMA: head_dim 64 or fewer than 8 query heads per KV
- * head).  Host only, launches nothing; "" on bad parameters or ws_bytes < 256.  Static
- * storage. */
+ * V^T scratch), "k_attend" (warp-level MMA: head_dim 64, a single query head per KV head,
+ * or tiles of 128/G tokens that would span two chunks) or "k_attend_fa|k_attend" (chosen at
+ * run time, see dash_stage2_kernel_ran).  Host only, launches nothing; "" on bad parameters
+ * or ws_bytes < 256.  Static storage. */
 const char *dash_attend_kernel_name(const dash_params_t *params, size_t ws_bytes);
+
+/* After a dash_prefill or dash_attend call with workspace ws, on `stream` (synchronised
+ * here): the Stage 2 kernel a run-time choice ran, "k_attend_fa" or "k_attend", or "" if that
+ * call made no run-time choice.  dash_attend_kernel_name reports "k_attend_fa|k_attend" for
+ * calls that choose at run time: routed, full-range calls with 2 or 4 query heads per KV
+ * head, where a small kernel first counts from the mask words the token-chunk pairs each
+ * kernel would execute (the 128-key-block kernel walks the union of 128/G tokens' chunks,
+ * the warp-MMA kernel of 16/G tokens'), both kernels are launched, and every CTA of the
+ * one with the larger estimated time exits at once.  Static storage. */
+const char *dash_stage2_kernel_ran(void *ws, void *stream);
+
+/* Number of kernels one dash_prefill call with these parameters launches when its workspace
+ * is ws_bytes and the caller passes neither summary_k nor active_blocks: Stage 0, Stage 1
+ * (absent where the 128-key-block kernel routes its own tiles), the V^T transpose (for the
+ * 128-key-block kernels) and Stage 2 (with a run-time choice: the cost kernel and both Stage 2
+ * kernels).  Host only; 0 on bad parameters. */
+int dash_prefill_kernel_count(const dash_params_t *params, size_t ws_bytes);
 
 /* Chunk-representation cache update for decode: Stage 0 over each sequence's last n_recent
  * complete chunks.  Idempotent (recomputing a frozen chunk writes the same bits).

@@ -42,8 +42,9 @@ FLAG_TEST_STALL_WAIT = 16         # test hook: Stage 0's bounded copy wait runs 
 EXPORTS = ("dash_prefill_workspace_size", "dash_prefill", "dash_prefill_host", "dash_stage0", "dash_route",
            "dash_attend_workspace_size", "dash_attend", "dash_update_chunk_cache", "dash_decode_workspace_size",
            "dash_decode", "dash_read_device_status", "dash_status_string", "dash_prefill_static_ws",
-           "dash_static_ws_read_status", "dash_attend_kernel_name", "dash_decode_paged",
-           "dash_update_chunk_cache_paged", "dash_backward", "dash_backward_workspace_size")
+           "dash_static_ws_read_status", "dash_attend_kernel_name", "dash_prefill_kernel_count", "dash_decode_paged",
+           "dash_update_chunk_cache_paged", "dash_backward_workspace_size", "dash_backward",
+           "dash_stage2_kernel_ran")
 
 
 class Params(ctypes.Structure):
@@ -95,6 +96,10 @@ def _declare(lib):
     lib.dash_status_string.argtypes = [ctypes.c_int]
     lib.dash_attend_kernel_name.argtypes = [_P, _sz]
     lib.dash_attend_kernel_name.restype = ctypes.c_char_p
+    lib.dash_stage2_kernel_ran.argtypes = [_vp, _vp]
+    lib.dash_stage2_kernel_ran.restype = ctypes.c_char_p
+    lib.dash_prefill_kernel_count.argtypes = [_P, _sz]
+    lib.dash_prefill_kernel_count.restype = ctypes.c_int
     lib.dash_status_string.restype = ctypes.c_char_p
     for _f in ("dash_prefill", "dash_stage0", "dash_route", "dash_attend",
                "dash_update_chunk_cache", "dash_decode", "dash_read_device_status",
@@ -157,6 +162,17 @@ def decode_workspace_size(params: Params) -> int:
 def attend_kernel_name(params: Params, ws_bytes: int) -> str:
     """Name of the Stage 2 kernel dash_attend launches with a workspace of ws_bytes."""
     return lib.dash_attend_kernel_name(ctypes.byref(params), int(ws_bytes)).decode()
+
+
+def stage2_kernel_ran(ws) -> str:
+    """The Stage 2 kernel a run-time choice ran in the last call with workspace ws ("" if that
+    call made no run-time choice); synchronises the current stream."""
+    return lib.dash_stage2_kernel_ran(_ptr(ws), _stream(ws.device)).decode()
+
+
+def prefill_kernel_count(params: Params, ws_bytes: int) -> int:
+    """Kernels one dash_prefill call launches with a workspace of ws_bytes."""
+    return int(lib.dash_prefill_kernel_count(ctypes.byref(params), int(ws_bytes)))
 
 
 def workspace(nbytes: int, device) -> torch.Tensor:
@@ -343,7 +359,7 @@ def update_chunk_cache_paged(k_pool, head_cls, block_table, seq_lens, summary_po
                                              _ptr(block_table), int(max_blocks), int(n_pages),
                                              _ptr(seq_lens), int(n_recent), _ptr(summary_pool),
                                              _ptr(ws), ws.numel(), _stream(k_pool.device)),
-           "dash_update_chunk_cache_paged", "dash_backward", "dash_backward_workspace_size")
+           "dash_update_chunk_cache_paged")
     return summary_pool
 
 

@@ -28,6 +28,10 @@ __global__ void __launch_bounds__(kAttnWarps * 32) k_attend(StageArgs a, int TU,
                                                             long long n_units) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (a.cost) {                           // run-time choice against the 128-key-block kernel
+        if (attend_fa_chosen(a)) return;
+        attend_record_ran(a, 2);
+    }
     const long long unit = (long long)blockIdx.x * kAttnWarps + warp;
     if (unit >= n_units) return;
 
@@ -258,6 +262,59 @@ static cudaError_t launch_attend_t(const StageArgs &a, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+// Token-chunk pairs the two Stage 2 kernels would execute for a routed call with G < 8: the
+// 128-key-block kernel walks, per tile of 128/G tokens, the union of their chunks
+// (cost[0] += |union| x 128/G), the warp-MMA kernel per unit of 16/G tokens
+// (cost[1] += |union| x 16/G).  Each token's mask words carry its diagonal bit, so the
+// tile's diagonal chunk counts in both.  One warp per tile, lanes over mask words.
+__global__ void __launch_bounds__(128) k_union_cost(StageArgs a, unsigned long long *cost,
+                                                    int n_tiles_bg) {
+    const int lane = threadIdx.x & 31;
+    const long long tile = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
+    if (tile >= (long long)n_tiles_bg * a.B * a.Hkv) return;
+    const int RT = 128 / a.G, TU = 16 / a.G;
+    const long long bg = tile / n_tiles_bg;
+    const int t0 = (int)(tile % n_tiles_bg) * RT;
+    const int t_last = min(t0 + RT, a.T) - 1;
+    const int wlim = (t_last / a.Bc) / 64;       // the last word with a bit the tile can hold
+    unsigned long long cf = 0, cw = 0;
+    for (int w = lane; w <= wlim; w += 32) {
+        uint64_t tile_word = 0;
+        for (int u0 = 0; u0 < RT; u0 += TU) {
+            uint64_t unit_word = 0;
+            for (int u = u0; u < u0 + TU; ++u) {
+                const int t = t0 + u;
+                if (t < a.T) unit_word |= a.mask[(bg * a.T + t) * a.W + w];
+            }
+            cw += (unsigned long long)__popcll(unit_word) * TU;
+            tile_word |= unit_word;
+        }
+        cf += (unsigned long long)__popcll(tile_word) * RT;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        cf += __shfl_xor_sync(kFull, cf, o);
+        cw += __shfl_xor_sync(kFull, cw, o);
+    }
+    if (lane == 0) {
+        atomicAdd(&cost[0], cf);
+        atomicAdd(&cost[1], cw);
+    }
+}
+
+// Executed token-chunk pairs per unit of time of the two kernels for G = 4 (TFLOP/s on
+// executed blocks measured on B200 over the 64K sweep cells: 128-key blocks about 355 with
+// 64-key chunks and 620 with 128-key chunks, warp MMA about 135); only their ratio is used.
+constexpr float kRateFa64 = 355.f, kRateFa128 = 620.f, kRateWarp = 135.f;
+
+// A run-time choice applies to full-range routed calls with fewer than 8 query heads per KV
+// head: there the 128-key-block kernel's tiles (128/G tokens) walk much larger unions than
+// the warp kernel's units (16/G tokens), and which costs less depends on the sparsity.
+static bool attend_dynamic(const StageArgs &a) {
+    return !a.ignore_routing && a.G < 8 && a.D == 128 && (a.Bc == 64 || a.Bc == 128) &&
+           a.t_begin == 0 && a.t_end == a.T;
+}
+
 AttendKernel attend_kernel(const StageArgs &a) {
     if (a.t_begin != 0 || a.t_end != a.T) {
         // Row slices: only the 128-key-block kernels take a row range.
@@ -270,7 +327,7 @@ AttendKernel attend_kernel(const StageArgs &a) {
     // chunk forced active); with routing the larger union costs more than the halved copies
     // save (measured at 128K: 128 ms against 117 ms).
     if (a.vt && a.ignore_routing && attend_pair_supported(a)) return AttendKernel::kPair;
-    if (a.vt && attend_fa_supported(a)) return AttendKernel::kFa;
+    if (a.vt && attend_fa_supported(a)) return attend_dynamic(a) ? AttendKernel::kFaOrWarp : AttendKernel::kFa;
     if (attend_tc_supported(a)) return AttendKernel::kTc;
     if ((a.D == 128 || a.D == 64) && (a.Bc == 64 || a.Bc == 128)) return AttendKernel::kWarp;
     return AttendKernel::kNone;
@@ -282,8 +339,17 @@ const char *attend_kernel_name(AttendKernel k) {
         case AttendKernel::kFa: return "k_attend_fa";
         case AttendKernel::kTc: return "k_attend_tc";
         case AttendKernel::kWarp: return "k_attend";
+        case AttendKernel::kFaOrWarp: return "k_attend_fa|k_attend";
         default: return "";
     }
+}
+
+static cudaError_t launch_warp(const StageArgs &a, cudaStream_t st) {
+    if (a.D == 128 && a.Bc == 64) return launch_attend_t<128, 64>(a, st);
+    if (a.D == 128 && a.Bc == 128) return launch_attend_t<128, 128>(a, st);
+    if (a.D == 64 && a.Bc == 64) return launch_attend_t<64, 64>(a, st);
+    if (a.D == 64 && a.Bc == 128) return launch_attend_t<64, 128>(a, st);
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_attend(const StageArgs &a, cudaStream_t st) {
@@ -291,12 +357,26 @@ cudaError_t launch_attend(const StageArgs &a, cudaStream_t st) {
         case AttendKernel::kPair: return launch_attend_pair(a, st);
         case AttendKernel::kFa: return launch_attend_fa(a, st);
         case AttendKernel::kTc: return launch_attend_tc(a, st);
-        case AttendKernel::kWarp:
-            if (a.D == 128 && a.Bc == 64) return launch_attend_t<128, 64>(a, st);
-            if (a.D == 128 && a.Bc == 128) return launch_attend_t<128, 128>(a, st);
-            if (a.D == 64 && a.Bc == 64) return launch_attend_t<64, 64>(a, st);
-            if (a.D == 64 && a.Bc == 128) return launch_attend_t<64, 128>(a, st);
-            return cudaErrorInvalidValue;
+        case AttendKernel::kWarp: return launch_warp(a, st);
+        case AttendKernel::kFaOrWarp: {
+            // Costs from the mask, then both kernels; the one not chosen exits per CTA.
+            unsigned char *blk = reinterpret_cast<unsigned char *>(a.status);
+            unsigned long long *cost = reinterpret_cast<unsigned long long *>(blk + kStatusCostOff);
+            cudaError_t e = cudaMemsetAsync(cost, 0, 2 * sizeof(unsigned long long), st);
+            if (e != cudaSuccess) return e;
+            const int RT = 128 / a.G;
+            const int n_tiles_bg = (a.T + RT - 1) / RT;
+            const long long tiles = (long long)n_tiles_bg * a.B * a.Hkv;
+            if (tiles > 0) {
+                k_union_cost<<<(unsigned)((tiles + 3) / 4), 128, 0, st>>>(a, cost, n_tiles_bg);
+                if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            }
+            StageArgs d = a;
+            d.cost = cost;
+            d.cost_ratio = (a.Bc == 64 ? kRateFa64 : kRateFa128) / kRateWarp;
+            if ((e = launch_attend_fa(d, st)) != cudaSuccess) return e;
+            return launch_warp(d, st);
+        }
         default:
             return (a.t_begin != 0 || a.t_end != a.T) ? cudaErrorNotSupported : cudaErrorInvalidValue;
     }

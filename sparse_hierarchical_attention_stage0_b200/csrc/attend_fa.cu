@@ -178,6 +178,10 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
     float *qbar = reinterpret_cast<float *>(base + ta.off_qbar);        // [RT][D]
     int16_t *list = reinterpret_cast<int16_t *>(base + ta.off_list);    // [C]
 
+    if (a.cost) {                           // run-time choice against the warp-MMA kernel
+        if (!attend_fa_chosen(a)) return;
+        attend_record_ran(a, 1);
+    }
     const int RT = ta.RT, G = a.G;
     // (b, g)-major, longest tiles first: the CTAs in flight share one (b, g)'s K and V^T in L2
     // (67 MB at T = 128K; both planes at once overflow the 126 MB L2: 3% slower, measured).

@@ -440,10 +440,14 @@ __global__ void k_bwd_lists(BwdArgs ba, int mode) {
             const unsigned bal = __ballot_sync(kFull, (word >> bit) & 1ull);
             if (!bal) continue;
             const int c = 64 * w + bit;
+            // The chunk's running count sits on lane bit % 32; every lane takes part in the
+            // shuffle, whether or not its token routes to the chunk.
+            const int run_c = bit < 32 ? __shfl_sync(kFull, run_lo, bit) : __shfl_sync(kFull, run_hi, bit - 32);
             if (mode == 1 && ((word >> bit) & 1ull)) {
-                const int before = (bit < 32 ? __shfl_sync(kFull, run_lo, bit) : __shfl_sync(kFull, run_hi, bit - 32)) +
-                                   __popc(bal & ((1u << lane) - 1u));
-                ba.list[bg * ba.nnz_max + ba.list_off[bg * (a.C + 1) + c] + before] = t;
+                const int before = run_c + __popc(bal & ((1u << lane) - 1u));
+                const long long pos = ba.list_off[bg * (a.C + 1) + c] + before;
+                if (pos >= 0 && pos < ba.nnz_max) ba.list[bg * ba.nnz_max + pos] = t;
+                else report(a.status, DASH_ERR_BOUNDS);
             }
             if (lane == (bit & 31)) {
                 if (bit < 32) run_lo += __popc(bal); else run_hi += __popc(bal);
@@ -528,6 +532,10 @@ __global__ void __launch_bounds__(BC / 16 * 32) k_bwd_kv(BwdArgs ba, int UPT) {
         const int kunit = (int)(e % UPT);
         const bool diag = ti < n_diag;
         const int t = diag ? c * BC + (int)ti : ba.list[bg * ba.nnz_max + off + (ti - n_diag)];
+        if (t < 0 || t >= a.T) {                             // same entry in every thread
+            if (tid == 0) report(a.status, DASH_ERR_BOUNDS);
+            continue;
+        }
         __syncthreads();                                     // the previous entry's tiles are read
         // rows r < Gu of the entry: heads g G + kunit 16 + r of token t
         for (int i = tid; i < 16 * CH; i += NW * 32) {
@@ -687,6 +695,10 @@ __global__ void __launch_bounds__(128) k_bwd_dsum(BwdArgs ba) {
     for (int i = 0; i < D / 32; ++i) acc[i] = 0.f;
     for (long long e = 0; e < n; ++e) {
         const int t = ba.list[bg * ba.nnz_max + off + e];
+        if (t < 0 || t >= a.T) {
+            if (lane == 0) report(a.status, DASH_ERR_BOUNDS);
+            continue;
+        }
         const float ds = ba.dlogp[(bg * a.T + t) * a.C + c];
         const float *qb = ba.qbar + (bg * a.T + t) * D;
 #pragma unroll

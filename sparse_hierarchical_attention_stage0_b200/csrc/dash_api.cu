@@ -55,7 +55,7 @@ dash_status_t check_params(const dash_params_t *p, Shape *s) {
 }
 
 RouteConsts route_consts(const dash_params_t *p) {
-    RouteConsts rc;
+    RouteConsts rc = {};
     const double a = p->alpha, g = p->gamma, sg = p->sigma, sd = std::sqrt((double)p->head_dim);
     rc.alpha = p->alpha;
     rc.sscale = (float)(g / sd);
@@ -69,6 +69,8 @@ RouteConsts route_consts(const dash_params_t *p) {
         rc.xscale = (float)((a - 1.0) * g / sd);
         rc.beta = (float)(1.0 / (a - 1.0));
         rc.bscale2 = (float)(sg / (a - 1.0));
+        const double b = 1.0 / (a - 1.0), br = std::round(b);
+        rc.beta_int = (rc.kind == 3 && br >= 3.0 && br <= 8.0 && std::fabs(b - br) < 1e-9) ? (int)br : 0;
     }
     rc.sigma2 = (float)(sg * 1.4426950408889634);
     rc.newton_cap = (p->flags & DASH_FLAG_TEST_NEWTON_CAP) ? 1 : kNewtonCap;
@@ -126,8 +128,9 @@ bool dense_flags(const dash_params_t *p) {
     return (p->flags & (DASH_FLAG_DENSE | DASH_FLAG_FORCE_ALL_ACTIVE)) != 0;
 }
 
+// The status word and the record of a run-time Stage 2 choice (bytes 0-31 of the block).
 dash_status_t clear_status(void *ws, cudaStream_t st) {
-    return cudaMemsetAsync(ws, 0, sizeof(uint32_t), st) == cudaSuccess ? DASH_OK : DASH_ERR_CUDA;
+    return cudaMemsetAsync(ws, 0, 32, st) == cudaSuccess ? DASH_OK : DASH_ERR_CUDA;
 }
 
 dash_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? DASH_OK : DASH_ERR_CUDA; }
@@ -646,6 +649,34 @@ const char *dash_attend_kernel_name(const dash_params_t *p, size_t ws_bytes) {
     static unsigned char probe;
     if (vt && ws_bytes >= kStatusBytes + vt) a.vt = &probe;
     return attend_kernel_name(attend_kernel(a));
+}
+
+int dash_prefill_kernel_count(const dash_params_t *p, size_t ws_bytes) {
+    Shape s;
+    if (check_params(p, &s) != DASH_OK) return 0;
+    const bool dense = (p->flags & DASH_FLAG_DENSE) != 0;
+    StageArgs a = stage_args(p, s);
+    size_t off = kStatusBytes + bytes_tau(s);
+    if (!dense) off += bytes_summary(s) + bytes_mask(s);
+    const size_t vt = bytes_vt(s, dense_flags(p));
+    static unsigned char probe;               // only whether V^T fits matters, as in dash_prefill
+    if (vt && ws_bytes >= off + vt) a.vt = &probe;
+    const AttendKernel kern = attend_kernel(a);
+    if (kern == AttendKernel::kNone) return 0;
+    const bool fused = !dense && kern == AttendKernel::kFa && attend_fa_fuse_supported(a);
+    const bool with_vt = kern == AttendKernel::kFa || kern == AttendKernel::kPair || kern == AttendKernel::kFaOrWarp;
+    // a run-time choice adds the cost kernel and launches both Stage 2 kernels
+    const int extra = kern == AttendKernel::kFaOrWarp ? 2 : 0;
+    return (dense ? 0 : 1) + (dense || fused ? 0 : 1) + (with_vt ? 1 : 0) + 1 + extra;
+}
+
+const char *dash_stage2_kernel_ran(void *ws, void *stream) {
+    if (!ws) return "";
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return "";
+    unsigned char id = 0;
+    if (cudaMemcpy(&id, static_cast<unsigned char *>(ws) + kStatusRanOff, 1, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return "";
+    return id == 1 ? "k_attend_fa" : id == 2 ? "k_attend" : "";
 }
 
 dash_status_t dash_read_device_status(void *ws, void *stream) {

@@ -296,7 +296,16 @@ struct RouteConsts {
     int newton_cap;   // iteration cap of the Newton solve (kNewtonCap; 1 under the test hook)
     int est_diag;     // estimate_diagonal: the diagonal chunk joins the entmax (diag_dot)
     float inv_sqrt_d; // 1 / sqrt(D): Stage 0's logit scale
+    int beta_int;     // kind 3: beta when it is an integer 3..8 (alpha = 1 + 1/beta), else 0;
+                      // the powers m^beta, m^(beta-1) are then products, not powf
 };
+
+// m^e for a small integer e >= 0 (products, left to right).
+__device__ __forceinline__ float ipow(float m, int e) {
+    float r = 1.f;
+    for (int i = 0; i < e; ++i) r = __fmul_rn(r, m);
+    return r;
+}
 
 // estimate_diagonal: the routing dot qbar . dsum of the diagonal chunk of one row, where dsum
 // is Stage 0's summary taken over the n_vis keys of that chunk the row can see:
@@ -394,63 +403,160 @@ __device__ __forceinline__ bool topk_selected(const float *xs, int c, int n, boo
 __device__ __forceinline__ float pow_beta(float m, const RouteConsts &rc) {
     if (rc.kind == 1) return m * m;
     if (rc.kind == 2) return m;
-    return powf(m, rc.beta);
+    return rc.beta_int ? ipow(m, rc.beta_int) : powf(m, rc.beta);
+}
+// m^(beta-1), the derivative's power.
+__device__ __forceinline__ float pow_beta_m1(float m, const RouteConsts &rc) {
+    if (rc.kind == 1) return m;
+    if (rc.kind == 2) return 1.f;
+    return rc.beta_int ? ipow(m, rc.beta_int - 1) : powf(m, rc.beta - 1.f);
 }
 
 // One lane-strided pass over xs[0..n): lane l visits l, l+32, l+64, l+96, l+128, ..., with
 // four independent accumulators (one per offset mod 128, for instruction-level parallelism)
-// combined as (a0 + a1) + (a2 + a3): a fixed summation order.
+// combined as (a0 + a1) + (a2 + a3): a fixed summation order.  The adds are explicit (never
+// contracted into a product of the term), so every source of the row gives the same bits.
 template <typename Term>
 __device__ __forceinline__ float lane_pass(const float *xs, int n, int lane, Term term) {
     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
     int c = lane;
     for (; c + 96 < n; c += 128) {
-        a0 += term(xs[c]);
-        a1 += term(xs[c + 32]);
-        a2 += term(xs[c + 64]);
-        a3 += term(xs[c + 96]);
+        a0 = __fadd_rn(a0, term(xs[c]));
+        a1 = __fadd_rn(a1, term(xs[c + 32]));
+        a2 = __fadd_rn(a2, term(xs[c + 64]));
+        a3 = __fadd_rn(a3, term(xs[c + 96]));
     }
-    if (c < n) a0 += term(xs[c]);
-    if (c + 32 < n) a1 += term(xs[c + 32]);
-    if (c + 64 < n) a2 += term(xs[c + 64]);
+    if (c < n) a0 = __fadd_rn(a0, term(xs[c]));
+    if (c + 32 < n) a1 = __fadd_rn(a1, term(xs[c + 32]));
+    if (c + 64 < n) a2 = __fadd_rn(a2, term(xs[c + 64]));
     return (a0 + a1) + (a2 + a3);
 }
 
-// Entmax threshold of one row held in (shared) memory xs[0..n), n >= 1, all 32 lanes of
-// the warp calling, specialised on the kind of alpha (0 softmax, 1 alpha = 1.5, 2 alpha = 2,
-// 3 any other alpha).  For alpha = 1 returns the log-sum-exp of the scores.  Otherwise x are
-// the scaled scores (alpha-1) s and the return value is tau with
-// sum_c [x_c - tau]_+^beta = 1.  For beta >= 1 (alpha <= 2) Newton's method from
-// tau0 = max x - 1 increases monotonically to the root (f is convex and decreasing); the
-// support it settles on is then fed to the exact closed form for alpha = 1.5 and 2.  For
-// alpha > 2, bisection on [max - 1, max - n^(1-alpha)].  The fixed lane-strided sums and
-// butterfly reductions give every caller the same bits.
-template <int KIND>
-static __device__ __noinline__ float entmax_tau_k(const float *xs, int n, const RouteConsts rc,
-                                                  uint32_t *status) {
-    const int lane = threadIdx.x & 31;
-    float mx = -INFINITY;
-    for (int c = lane; c < n; c += 32) mx = fmaxf(mx, xs[c]);
-    mx = warp_max(mx);
+// Two sums in one lane-strided pass: each with lane_pass's order, so each has lane_pass's
+// bits; xs is read once for both.
+template <typename Term1, typename Term2>
+__device__ __forceinline__ void lane_pass2(const float *xs, int n, int lane, Term1 t1, Term2 t2,
+                                           float &s1, float &s2) {
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, b0 = 0.f, b1 = 0.f, b2 = 0.f, b3 = 0.f;
+    int c = lane;
+    for (; c + 96 < n; c += 128) {
+        const float x0 = xs[c], x1 = xs[c + 32], x2 = xs[c + 64], x3 = xs[c + 96];
+        a0 = __fadd_rn(a0, t1(x0));
+        b0 = __fadd_rn(b0, t2(x0));
+        a1 = __fadd_rn(a1, t1(x1));
+        b1 = __fadd_rn(b1, t2(x1));
+        a2 = __fadd_rn(a2, t1(x2));
+        b2 = __fadd_rn(b2, t2(x2));
+        a3 = __fadd_rn(a3, t1(x3));
+        b3 = __fadd_rn(b3, t2(x3));
+    }
+    if (c < n) { const float x = xs[c]; a0 = __fadd_rn(a0, t1(x)); b0 = __fadd_rn(b0, t2(x)); }
+    if (c + 32 < n) { const float x = xs[c + 32]; a1 = __fadd_rn(a1, t1(x)); b1 = __fadd_rn(b1, t2(x)); }
+    if (c + 64 < n) { const float x = xs[c + 64]; a2 = __fadd_rn(a2, t1(x)); b2 = __fadd_rn(b2, t2(x)); }
+    s1 = (a0 + a1) + (a2 + a3);
+    s2 = (b0 + b1) + (b2 + b3);
+}
+
+// A row of n scores as seen by one warp: lane l owns the values c = l + 32 k, k = 0, 1, ...
+// Two sources with the same summation order, so the same bits: the row in (shared) memory,
+// or the lane's values in registers (n <= 32 NV).
+struct RowInMemory {
+    const float *xs;
+    int n, lane;
+    __device__ float max() const {
+        float mx = -INFINITY;
+        for (int c = lane; c < n; c += 32) mx = fmaxf(mx, xs[c]);
+        return mx;
+    }
+    template <typename T>
+    __device__ float pass(T term) const { return lane_pass(xs, n, lane, term); }
+    template <typename T1, typename T2>
+    __device__ void pass2(T1 t1, T2 t2, float &s1, float &s2) const { lane_pass2(xs, n, lane, t1, t2, s1, s2); }
+    // Does any value lie on different sides of t and nt?
+    __device__ int moved(float t, float nt) const {
+        int m = 0;
+        for (int c = lane; c < n; c += 32) m |= ((xs[c] > t) != (xs[c] > nt));
+        return m;
+    }
+};
+template <int NV>
+struct RowInRegisters {
+    const float (&v)[NV];                // v[k] = score l + 32 k of lane l (valid for k < nk)
+    int nk;
+    __device__ float max() const {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < NV; ++k)
+            if (k < nk) mx = fmaxf(mx, v[k]);
+        return mx;
+    }
+    // lane_pass's order: accumulator k % 4 takes the values k, k + 4, ... in turn.
+    template <typename T>
+    __device__ float pass(T term) const {
+        float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k = 0; k < NV; ++k)
+            if (k < nk) a[k & 3] = __fadd_rn(a[k & 3], term(v[k]));
+        return (a[0] + a[1]) + (a[2] + a[3]);
+    }
+    template <typename T1, typename T2>
+    __device__ void pass2(T1 t1, T2 t2, float &s1, float &s2) const {
+        float a[4] = {0.f, 0.f, 0.f, 0.f}, b[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k = 0; k < NV; ++k)
+            if (k < nk) {
+                a[k & 3] = __fadd_rn(a[k & 3], t1(v[k]));
+                b[k & 3] = __fadd_rn(b[k & 3], t2(v[k]));
+            }
+        s1 = (a[0] + a[1]) + (a[2] + a[3]);
+        s2 = (b[0] + b[1]) + (b[2] + b[3]);
+    }
+    __device__ int moved(float t, float nt) const {
+        int m = 0;
+#pragma unroll
+        for (int k = 0; k < NV; ++k)
+            if (k < nk) m |= ((v[k] > t) != (v[k] > nt));
+        return m;
+    }
+};
+
+// Entmax threshold of one row (n >= 1 scores, all 32 lanes of the warp calling), specialised
+// on the kind of alpha (0 softmax, 1 alpha = 1.5, 2 alpha = 2, 3 any other alpha).  For
+// alpha = 1 returns the log-sum-exp of the scores.  Otherwise x are the scaled scores
+// (alpha-1) s and the return value is tau with sum_c [x_c - tau]_+^beta = 1.  For beta >= 1
+// (alpha <= 2) Newton's method from tau0 = max x - 1 increases monotonically to the root (f
+// is convex and decreasing); the support it settles on is then fed to the exact closed form
+// for alpha = 1.5 and 2.  For alpha > 2, bisection on [max - 1, max - n^(1-alpha)].  The
+// fixed lane-strided sums and butterfly reductions give every caller the same bits.
+template <int KIND, typename Row>
+__device__ __forceinline__ float entmax_tau_row(const Row &row, int n, const RouteConsts &rc,
+                                                uint32_t *status) {
+    const float mx = warp_max(row.max());
     if (KIND == 0) {
-        const float s = warp_sum(lane_pass(xs, n, lane, [mx](float x) { return expf(x - mx); }));
+        const float s = warp_sum(row.pass([mx](float x) { return expf(x - mx); }));
         return mx + logf(s);
     }
     const float beta = rc.beta;
     float tau;
     if (KIND != 3 || beta >= 1.f) {
         tau = mx - 1.f;
+        const int bi = rc.beta_int;
         int it = 0;
         for (; it < rc.newton_cap; ++it) {
             const float t = tau;
-            const float f = warp_sum(lane_pass(xs, n, lane, [t, beta](float x) {
-                const float m = x - t;
-                return m > 0.f ? (KIND == 1 ? m * m : KIND == 2 ? m : powf(m, beta)) : 0.f;
-            }));
-            const float df = warp_sum(lane_pass(xs, n, lane, [t, beta](float x) {
-                const float m = x - t;
-                return m > 0.f ? (KIND == 1 ? m : KIND == 2 ? 1.f : powf(m, beta - 1.f)) : 0.f;
-            }));
+            float f, df;
+            row.pass2(
+                [t, beta, bi](float x) {
+                    const float m = x - t;
+                    return m > 0.f ? (KIND == 1 ? __fmul_rn(m, m) : KIND == 2 ? m : bi ? ipow(m, bi) : powf(m, beta)) : 0.f;
+                },
+                [t, beta, bi](float x) {
+                    const float m = x - t;
+                    return m > 0.f ? (KIND == 1 ? m : KIND == 2 ? 1.f : bi ? ipow(m, bi - 1) : powf(m, beta - 1.f)) : 0.f;
+                },
+                f, df);
+            f = warp_sum(f);
+            df = warp_sum(df);
             const float step = (f - 1.f) / (beta * df);
             if (!(step > 0.f)) break;                 // at (or rounded past) the root
             const float nt = tau + step;
@@ -463,7 +569,7 @@ static __device__ __noinline__ float entmax_tau_k(const float *xs, int n, const 
         float lo = mx - 1.f, hi = mx - powf((float)n, 1.f - rc.alpha);
         for (int it = 0; it < 40; ++it) {
             const float mid = 0.5f * (lo + hi);
-            const float f = warp_sum(lane_pass(xs, n, lane, [mid, beta](float x) {
+            const float f = warp_sum(row.pass([mid, beta](float x) {
                 const float m = x - mid;
                 return m > 0.f ? powf(m, beta) : 0.f;
             }));
@@ -475,29 +581,38 @@ static __device__ __noinline__ float entmax_tau_k(const float *xs, int n, const 
         // Exact closed form on the support {x > tau}; repeat while the support moves.
         for (int rep = 0; rep < 4; ++rep) {
             const float t = tau;
-            const float sx = warp_sum(lane_pass(xs, n, lane, [t](float x) { return x > t ? x : 0.f; }));
-            const int k = (int)warp_sum(lane_pass(xs, n, lane, [t](float x) { return x > t ? 1.f : 0.f; }));
+            float sx, kf;
+            row.pass2([t](float x) { return x > t ? x : 0.f; }, [t](float x) { return x > t ? 1.f : 0.f; },
+                      sx, kf);
+            sx = warp_sum(sx);
+            const int k = (int)warp_sum(kf);
             if (k == 0) break;
             float nt;
             if (KIND == 2) {
                 nt = (sx - 1.f) / (float)k;
             } else {
                 const float mean = sx / (float)k;
-                const float m2 = warp_sum(lane_pass(xs, n, lane, [t, mean](float x) {
+                const float m2 = warp_sum(row.pass([t, mean](float x) {
                     const float d = x - mean;
-                    return x > t ? d * d : 0.f;
+                    return x > t ? __fmul_rn(d, d) : 0.f;
                 }));
                 nt = mean - sqrtf(fmaxf(1.f - m2, 0.f) / (float)k);
             }
             // Same support under the new threshold?  Then it is the fixed point.
-            int moved = 0;
-            for (int c = lane; c < n; c += 32) moved |= ((xs[c] > tau) != (xs[c] > nt));
-            moved = __any_sync(kFull, moved);
+            const int moved = __any_sync(kFull, row.moved(tau, nt));
             tau = nt;
             if (!moved) break;
         }
     }
     return tau;
+}
+
+// The row in (shared) memory xs[0..n); kept out of line (its callers' register budgets).
+template <int KIND>
+static __device__ __noinline__ float entmax_tau_k(const float *xs, int n, const RouteConsts rc,
+                                                  uint32_t *status) {
+    const RowInMemory row{xs, n, (int)(threadIdx.x & 31)};
+    return entmax_tau_row<KIND>(row, n, rc, status);
 }
 
 __device__ __forceinline__ float warp_entmax_tau(const float *xs, int n, const RouteConsts &rc,
@@ -507,6 +622,21 @@ __device__ __forceinline__ float warp_entmax_tau(const float *xs, int n, const R
         case 1: return entmax_tau_k<1>(xs, n, rc, status);
         case 2: return entmax_tau_k<2>(xs, n, rc, status);
         default: return entmax_tau_k<3>(xs, n, rc, status);
+    }
+}
+
+// The same threshold from the lane's values in registers: v[k] = xs[lane + 32 k], k < NV,
+// n <= 32 NV.  Same bits as warp_entmax_tau on the row in memory.
+template <int NV>
+__device__ __forceinline__ float warp_entmax_tau_regs(const float (&v)[NV], int n,
+                                                      const RouteConsts &rc, uint32_t *status) {
+    const int lane = threadIdx.x & 31;
+    const RowInRegisters<NV> row{v, n > lane ? (n - lane + 31) / 32 : 0};
+    switch (rc.kind) {
+        case 0: return entmax_tau_row<0>(row, n, rc, status);
+        case 1: return entmax_tau_row<1>(row, n, rc, status);
+        case 2: return entmax_tau_row<2>(row, n, rc, status);
+        default: return entmax_tau_row<3>(row, n, rc, status);
     }
 }
 

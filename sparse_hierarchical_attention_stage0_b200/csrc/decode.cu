@@ -5,25 +5,34 @@
 // decoding with a chunk-representation cache; gist.science "DashAttention ...", Technische
 // Zusammenfassung, "Stufe 0": complete chunks' summaries are frozen and cached (the cache is
 // maintained by dash_update_chunk_cache).  Decode is memory-bound: the step reads the
-// cached summaries and the active chunks' K/V once.
+// cached summaries and the active chunks' K/V once.  At one token per sequence the step is
+// short, so the kernel is laid out to keep its memory latencies off one serial path.
 //
 // One thread-block cluster of kDecCluster CTAs per (b, g):
-//   1. every CTA builds qbar; CTA r scores the r-th slice of the routable chunks
-//      (x_c = qbar . summary_c * (alpha-1) gamma / sqrt(D), same arithmetic as prefill);
-//   2. cluster barrier, then each CTA pulls the other slices through distributed shared
-//      memory (mapa + ld.shared::cluster), so every CTA holds the whole score row;
-//   3. every CTA solves the same tau (same code and data -> same bits); rank 0 writes the
-//      optional p row and mask words;
-//   4. the active chunks (+ the diagonal chunk, last) are dealt round-robin to the
-//      cluster's warps; each warp runs the 16-row mma.sync attention over its share;
-//   5. warp partials (max, sum, O) are merged inside the CTA, then across the cluster by
-//      rank 0 through distributed shared memory, which writes the bf16 output.
+//   1. every CTA builds qbar; CTA r scores the r-th slice of the routable chunks, four lanes
+//      per chunk (x_c = qbar . summary_c * (alpha-1) gamma / sqrt(D), route_dot's arithmetic
+//      and summation order, so prefill and decode route alike) and stores each score into
+//      every CTA's score row through distributed shared memory (st.shared::cluster); one
+//      cluster barrier later every CTA holds the whole row;
+//   2. warp 0 of every CTA solves the same tau (same code and data -> same bits).  Meanwhile
+//      one warp attends over the diagonal chunk (always active, bias 0: it needs no tau;
+//      its first K/V copies were issued at kernel entry).  (An L2 prefetch of the chunks
+//      above a lower bound of tau, by the idle warps, measured slower: the bound from a few
+//      Newton steps still leaves several times the support above it.);
+//   3. rank 0 writes the optional p row and mask words; the routed sub-blocks (32 keys of an
+//      active chunk) are dealt round-robin to the cluster's warps, which run the 16-row
+//      mma.sync attention over their share (K/V double-buffered per warp);
+//   4. warp partials (max, sum, O) merge inside each CTA; after a cluster barrier each CTA
+//      merges one eighth of the output (row, dim) pairs across the cluster through
+//      distributed shared memory and writes them in bf16.
 #include "attn_warp.cuh"
 
 namespace dash {
 
 constexpr int kDecCluster = 8;
 constexpr int kDecWarps = 4;
+constexpr int kDecSlots = kDecCluster * kDecWarps;          // warps of one cluster
+constexpr int kTauRegs = 33;                                // tau solved in registers up to 1056 scores
 
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
@@ -33,6 +42,14 @@ __device__ __forceinline__ uint32_t cluster_rank() {
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n"
                  "barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+// Split cluster barrier: arrive at entry, wait before the first access to a peer's shared
+// memory (a peer's shared memory may be used only once the peer has started).
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.aligned;\n" ::: "memory");
 }
 // Address of the same shared-memory variable in CTA `rank` of this cluster.
 __device__ __forceinline__ uint32_t map_rank(const void *p, uint32_t rank) {
@@ -44,6 +61,9 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
     float v;
     asm volatile("ld.shared::cluster.f32 %0, [%1];\n" : "=f"(v) : "r"(addr) : "memory");
     return v;
+}
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;\n" ::"r"(addr), "f"(v) : "memory");
 }
 
 int decode_supported(int G, int Ccap, int D) {
@@ -105,6 +125,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
             return;
         }
     }
+    cluster_arrive_relaxed();
     // Keys / values of chunk c (its first key) and the summary of chunk c.
     auto kv_base = [&](const void *pool, int c) -> const __nv_bfloat16 * {
         const __nv_bfloat16 *p0 = reinterpret_cast<const __nv_bfloat16 *>(pool);
@@ -118,31 +139,148 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
         return a.summary + ((long long)bg * a.Cf + c) * D;
     };
 
-    // 1. group-mean query and this CTA's slice of the scores.
+    // Per-warp attention state: 16 rows (the group's G heads), K/V tiles of kSub keys.
+    unsigned char *ks = smem_raw + L.tiles + warp * L.warp_tiles;
+    unsigned char *vs = ks + L.tile;
+    constexpr int NSUB = BC / kSub;
+    const bool diag_warp = rank == 0 && warp == 1;
+    const int n_diag = (t - ct * BC) / kSub + 1;   // sub-blocks of the diagonal chunk up to t
+    if (diag_warp) {
+        // The diagonal chunk is always attended: start its first copies now.
+        load_sub<D>(ks, kv_base(a.k, ct), 0, kv_rows(ct));
+        cp_async_commit();
+        load_sub<D>(vs, kv_base(a.v, ct), 0, kv_rows(ct));
+        cp_async_commit();
+    }
+
+    // 1. group-mean query and this CTA's slice of the scores, stored into every CTA's row.
+    // Four lanes per chunk: lane quarter k accumulates route_dot's partial sum p_k (the float4
+    // groups 4i + k, one sequential fmaf chain), combined as (p0 + p1) + (p2 + p3).  Each
+    // warp scores 8 chunks per step; the summaries of its next step are loaded while this
+    // one is scored (its first step's before qbar, which they do not depend on).
+    const int c_lo = (int)((long long)n * rank / kDecCluster);
+    const int c_hi = (int)((long long)n * (rank + 1) / kDecCluster);
+    const int kslice = lane & 3, cc = lane >> 2;
+    float4 sv[D / 16];
+    auto load_summaries = [&](int cb) {
+        const int c = cb + cc;
+        const float4 *s4 = reinterpret_cast<const float4 *>(summary_of(c < c_hi ? c : cb));
+#pragma unroll
+        for (int i = 0; i < D / 16; ++i) sv[i] = __ldg(s4 + 4 * i + kslice);
+    };
+    if (c_lo + warp * 8 < c_hi) load_summaries(c_lo + warp * 8);
     for (int d8 = tid * 8; d8 < D; d8 += kDecWarps * 32 * 8) {
         float m[8];
         group_mean8(q + (long long)g * G * D + d8, D, G, m);
 #pragma unroll
         for (int e = 0; e < 8; ++e) qbar[d8 + e] = m[e];
     }
-    __syncthreads();
-    const float scale = a.rc.kind == 0 ? a.rc.sscale : a.rc.xscale;
-    const int c_lo = (int)((long long)n * rank / kDecCluster);
-    const int c_hi = (int)((long long)n * (rank + 1) / kDecCluster);
-    for (int c = c_lo + tid; c < c_hi; c += kDecWarps * 32)
-        xs[c] = __fmul_rn(route_dot<D>(qbar, summary_of(c)), scale);
-
-    // 2. exchange slices through distributed shared memory.
-    cluster_sync_all();
-    for (uint32_t r = 0; r < kDecCluster; ++r) {
-        if (r == rank) continue;
-        const int lo = (int)((long long)n * r / kDecCluster);
-        const int hi = (int)((long long)n * (r + 1) / kDecCluster);
-        for (int c = lo + tid; c < hi; c += kDecWarps * 32) xs[c] = ld_cluster_f32(map_rank(&xs[c], r));
+    const int r_lo = lane >> 2, r_hi = r_lo + 8, qd = lane & 3;
+    const bool ok_lo = r_lo < G, ok_hi = r_hi < G;
+    uint32_t qf[D / 16][4];
+    {
+        const __nv_bfloat16 *q_lo = q + (long long)(g * G + (ok_lo ? r_lo : 0)) * D;
+        const __nv_bfloat16 *q_hi = q + (long long)(g * G + (ok_hi ? r_hi : 0)) * D;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const int d0 = 16 * kk + 2 * qd;
+            qf[kk][0] = ok_lo ? *reinterpret_cast<const uint32_t *>(q_lo + d0) : 0u;
+            qf[kk][1] = ok_hi ? *reinterpret_cast<const uint32_t *>(q_hi + d0) : 0u;
+            qf[kk][2] = ok_lo ? *reinterpret_cast<const uint32_t *>(q_lo + d0 + 8) : 0u;
+            qf[kk][3] = ok_hi ? *reinterpret_cast<const uint32_t *>(q_hi + d0 + 8) : 0u;
+        }
     }
     __syncthreads();
+    const float scale = a.rc.kind == 0 ? a.rc.sscale : a.rc.xscale;
+    cluster_wait();                               // every peer has started
+    {
+        uint32_t xs_at[kDecCluster];              // the score row of every CTA
+#pragma unroll
+        for (int r = 0; r < kDecCluster; ++r) xs_at[r] = map_rank(xs, (uint32_t)r);
+        const float4 *q4 = reinterpret_cast<const float4 *>(qbar);
+        for (int cb = c_lo + warp * 8; cb < c_hi; cb += kDecWarps * 8) {
+            float4 cur[D / 16];
+#pragma unroll
+            for (int i = 0; i < D / 16; ++i) cur[i] = sv[i];
+            if (cb + kDecWarps * 8 < c_hi) load_summaries(cb + kDecWarps * 8);
+            float acc = 0.f;
+#pragma unroll
+            for (int i = 0; i < D / 16; ++i) {
+                const float4 qq = q4[4 * i + kslice];
+                acc = fmaf(qq.x, cur[i].x, acc);
+                acc = fmaf(qq.y, cur[i].y, acc);
+                acc = fmaf(qq.z, cur[i].z, acc);
+                acc = fmaf(qq.w, cur[i].w, acc);
+            }
+            const float pair = acc + __shfl_down_sync(kFull, acc, 1);      // p0+p1 | p2+p3
+            const float dot = pair + __shfl_down_sync(kFull, pair, 2);
+            const int c = cb + cc;
+            if (c < c_hi && kslice == 0) {
+                const float x = __fmul_rn(dot, scale);
+#pragma unroll
+                for (int r = 0; r < kDecCluster; ++r)
+                    st_cluster_f32(xs_at[r] + 4u * (uint32_t)c, x);
+            }
+        }
+    }
+    cluster_sync_all();                           // every CTA holds the whole score row
 
-    // 3. threshold (every CTA, same bits) and the routing outputs (rank 0).  With
+    UnitState<D> st;
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) st.o[j][e] = 0.f;
+    st.m_lo = st.m_hi = -INFINITY;
+    st.l_lo = st.l_hi = 0.f;
+    float tau = 0.f;
+    // Attention over `cnt` sub-blocks: sub-block i is keys [sub_of(i) kSub, +kSub) of chunk
+    // chunk_of(i); keys past the end of a contiguous cache are zero-filled, keys after t in the
+    // diagonal chunk are masked by the softmax.  K/V double-buffered through the warp's tiles;
+    // `preloaded`: the copies of sub-block 0 are already in flight.
+    auto attend = [&](int cnt, auto chunk_of, auto sub_of, bool preloaded) {
+        if (cnt <= 0) return;
+        if (!preloaded) {
+            const int c0 = chunk_of(0);
+            load_sub<D>(ks, kv_base(a.k, c0), sub_of(0) * kSub, kv_rows(c0));
+            cp_async_commit();
+            load_sub<D>(vs, kv_base(a.v, c0), sub_of(0) * kSub, kv_rows(c0));
+            cp_async_commit();
+        }
+        for (int s = 0; s < cnt; ++s) {
+            const int c = chunk_of(s);
+            const int key0 = c * BC + sub_of(s) * kSub;
+            const bool diag = c == ct, more = s + 1 < cnt;
+            const int c_next = more ? chunk_of(s + 1) : 0;
+            const int sub_next = more ? sub_of(s + 1) * kSub : 0;
+            float bias2 = 0.f;
+            if (!diag)
+                bias2 = a.rc.kind == kKindTopk ? 0.f                 // top-k: uniform prior
+                        : a.rc.kind == 0 ? a.rc.sigma2 * (xs[c] - tau)
+                                         : a.rc.bscale2 * log2f(fmaxf(__fsub_rn(xs[c], tau), 1e-37f));
+            cp_async_wait<1>();
+            __syncwarp();
+            float acc[4][4];
+            qk_sub<D>(acc, qf, ks);
+            __syncwarp();
+            if (more) {
+                load_sub<D>(ks, kv_base(a.k, c_next), sub_next, kv_rows(c_next));
+                cp_async_commit();
+            }
+            uint32_t pa[2][4];
+            softmax_sub<D>(st, acc, pa, a.qk_scale2, ok_lo ? bias2 : -INFINITY,
+                           ok_hi ? bias2 : -INFINITY, diag, key0, t, t);
+            if (more) cp_async_wait<1>(); else cp_async_wait<0>();
+            __syncwarp();
+            pv_sub<D>(st, pa, vs);
+            __syncwarp();
+            if (more) {
+                load_sub<D>(vs, kv_base(a.v, c_next), sub_next, kv_rows(c_next));
+                cp_async_commit();
+            }
+        }
+    };
+
+    // 2. threshold (warp 0 of every CTA, same bits) and the diagonal chunk.  With
     // estimate_diagonal the diagonal chunk's score joins the candidates as entry n.
     const int n_eff = n + (a.rc.est_diag ? 1 : 0);
     if (warp == 0) {
@@ -152,7 +290,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
             if (lane == 0) xs[n] = __fmul_rn(dd, scale);
             __syncwarp();
         }
-        float tau;
+        float tw;
         if (a.rc.kind == kKindTopk) {
             // Top-k: selection bits in index order (lower index first on ties); tau = the
             // lowest selected score.
@@ -168,17 +306,25 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
             if (n > 0 && all) {
                 float mn = INFINITY;
                 for (int c = lane; c < n; c += 32) mn = fminf(mn, xs[c]);
-                tau = -warp_max(-mn);
+                tw = -warp_max(-mn);
             } else {
-                tau = n > 0 ? key_f32(key) : __int_as_float(0x7fc00000);
+                tw = n > 0 ? key_f32(key) : __int_as_float(0x7fc00000);
             }
+        } else if (n_eff > 0 && n_eff <= 32 * kTauRegs) {
+            // The row in registers (same bits as the solve on the row in shared memory).
+            float v[kTauRegs];
+#pragma unroll
+            for (int k = 0; k < kTauRegs; ++k) v[k] = lane + 32 * k < n_eff ? xs[lane + 32 * k] : 0.f;
+            tw = warp_entmax_tau_regs(v, n_eff, a.rc, a.status);
         } else {
-            tau = n_eff > 0 ? warp_entmax_tau(xs, n_eff, a.rc, a.status) : __int_as_float(0x7fc00000);
+            tw = n_eff > 0 ? warp_entmax_tau(xs, n_eff, a.rc, a.status) : __int_as_float(0x7fc00000);
         }
-        if (lane == 0) tau_s = tau;
+        if (lane == 0) tau_s = tw;
+    } else if (diag_warp) {
+        attend(n_diag, [&](int) { return ct; }, [&](int i) { return i; }, true);
     }
     __syncthreads();
-    const float tau = tau_s;
+    tau = tau_s;
     auto active = [&](int c) -> bool {
         if (a.rc.kind == kKindTopk) return c < n && ((sel[c >> 5] >> (c & 31)) & 1u);
         return c < n && (a.rc.kind == 0 || __fsub_rn(xs[c], tau) > 0.f);
@@ -206,98 +352,46 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
         }
     }
 
-    // 4. active list (same on every CTA): routed chunks ascending, then the diagonal.
+    // 3. active list (same on every CTA): the routed chunks (the diagonal is attended
+    // separately above).
+    // Lane l lists its chunks l, l + 32, ... of each block of 1024, the lanes in order.
     if (warp == 0) {
         int pos = 0;
-        for (int c0 = 0; c0 < n; c0 += 32) {
-            const int c = c0 + lane;
-            const bool act = active(c) && dash_check(c < a.Cf && (c + 1) * BC <= a.cap, a.status);
-            const unsigned bal = __ballot_sync(kFull, act);
-            if (act) list[pos + __popc(bal & ((1u << lane) - 1u))] = c;
-            pos += __popc(bal);
+        for (int c0 = 0; c0 < n; c0 += 32 * 32) {
+            uint32_t bits = 0;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                const int c = c0 + lane + 32 * k;
+                if (active(c) && dash_check(c < a.Cf && (c + 1) * BC <= a.cap, a.status)) bits |= 1u << k;
+            }
+            const int cnt = __popc(bits);
+            int incl = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(kFull, incl, o);
+                if (lane >= o) incl += y;
+            }
+            int p = pos + incl - cnt;
+            while (bits) {
+                const int k = __ffs(bits) - 1;
+                bits &= bits - 1u;
+                list[p++] = c0 + lane + 32 * k;
+            }
+            pos += __shfl_sync(kFull, incl, 31);
         }
-        if (lane == 0) {
-            list[pos] = ct;
-            nact_s = pos + 1;
-        }
+        if (lane == 0) nact_s = pos;
     }
     __syncthreads();
-    const int nact = nact_s;
-
-    // Attention over this warp's share: entries i with i % NC == rank, (i / NC) % W == warp.
-    unsigned char *ks = smem_raw + L.tiles + warp * L.warp_tiles;
-    unsigned char *vs = ks + L.tile;
-    const int r_lo = lane >> 2, r_hi = r_lo + 8, qd = lane & 3;
-    const bool ok_lo = r_lo < G, ok_hi = r_hi < G;
-    uint32_t qf[D / 16][4];
     {
-        const __nv_bfloat16 *q_lo = q + (long long)(g * G + (ok_lo ? r_lo : 0)) * D;
-        const __nv_bfloat16 *q_hi = q + (long long)(g * G + (ok_hi ? r_hi : 0)) * D;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-            const int d0 = 16 * kk + 2 * qd;
-            qf[kk][0] = ok_lo ? *reinterpret_cast<const uint32_t *>(q_lo + d0) : 0u;
-            qf[kk][1] = ok_hi ? *reinterpret_cast<const uint32_t *>(q_hi + d0) : 0u;
-            qf[kk][2] = ok_lo ? *reinterpret_cast<const uint32_t *>(q_lo + d0 + 8) : 0u;
-            qf[kk][3] = ok_hi ? *reinterpret_cast<const uint32_t *>(q_hi + d0 + 8) : 0u;
-        }
-    }
-    UnitState<D> st;
-#pragma unroll
-    for (int j = 0; j < D / 8; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) st.o[j][e] = 0.f;
-    st.m_lo = st.m_hi = -INFINITY;
-    st.l_lo = st.l_hi = 0.f;
-
-    constexpr int NSUB = BC / kSub;
-    const int stride = kDecCluster * kDecWarps;
-    const int first = (int)rank + kDecCluster * warp;
-    const int my_n = first < nact ? (nact - first + stride - 1) / stride : 0;
-    const int nsteps = my_n * NSUB;
-    // Sub-block s of this warp's share: kSub keys from key (s % NSUB) * kSub of chunk
-    // list[first + (s / NSUB) * stride]; keys past the end of a contiguous cache are zero-filled,
-    // keys after t in the diagonal chunk are masked by the softmax.
-    if (nsteps > 0) {
-        load_sub<D>(ks, kv_base(a.k, list[first]), 0, kv_rows(list[first]));
-        cp_async_commit();
-        load_sub<D>(vs, kv_base(a.v, list[first]), 0, kv_rows(list[first]));
-        cp_async_commit();
-    }
-    for (int s = 0; s < nsteps; ++s) {
-        const int c = list[first + (s / NSUB) * stride];
-        const int key0 = c * BC + (s % NSUB) * kSub;
-        const bool diag = c == ct, more = s + 1 < nsteps;
-        const int c_next = more ? list[first + ((s + 1) / NSUB) * stride] : 0;
-        const int sub_next = ((s + 1) % NSUB) * kSub;
-        float bias2 = 0.f;
-        if (!diag)
-            bias2 = a.rc.kind == kKindTopk ? 0.f                 // top-k: uniform prior
-                    : a.rc.kind == 0 ? a.rc.sigma2 * (xs[c] - tau)
-                                     : a.rc.bscale2 * log2f(fmaxf(__fsub_rn(xs[c], tau), 1e-37f));
-        cp_async_wait<1>();
-        __syncwarp();
-        float acc[4][4];
-        qk_sub<D>(acc, qf, ks);
-        __syncwarp();
-        if (more) {
-            load_sub<D>(ks, kv_base(a.k, c_next), sub_next, kv_rows(c_next));
-            cp_async_commit();
-        }
-        uint32_t pa[2][4];
-        softmax_sub<D>(st, acc, pa, a.qk_scale2, ok_lo ? bias2 : -INFINITY,
-                       ok_hi ? bias2 : -INFINITY, diag, key0, t, t);
-        if (more) cp_async_wait<1>(); else cp_async_wait<0>();
-        __syncwarp();
-        pv_sub<D>(st, pa, vs);
-        __syncwarp();
-        if (more) {
-            load_sub<D>(vs, kv_base(a.v, c_next), sub_next, kv_rows(c_next));
-            cp_async_commit();
-        }
+        // This warp's share of the routed sub-blocks: entries e = first + i * kDecSlots.
+        const int n_ent = nact_s * NSUB;
+        const int first = (int)rank + kDecCluster * warp;
+        const int my_n = first < n_ent ? (n_ent - first + kDecSlots - 1) / kDecSlots : 0;
+        attend(my_n, [&](int i) { return list[(first + i * kDecSlots) / NSUB]; },
+               [&](int i) { return (first + i * kDecSlots) % NSUB; }, false);
     }
 
-    // 5a. warp partial -> the warp's own tile space.
+    // 4a. warp partial -> the warp's own tile space.
     float l_lo = st.l_lo, l_hi = st.l_hi;
     l_lo += __shfl_xor_sync(kFull, l_lo, 1);
     l_lo += __shfl_xor_sync(kFull, l_lo, 2);
@@ -320,7 +414,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
     }
     __syncthreads();
 
-    // 5b. CTA merge of the warp partials into cpart.
+    // 4b. CTA merge of the warp partials into cpart.
     for (int idx = tid; idx < 16 * D + 16; idx += kDecWarps * 32) {
         const int r = idx < 16 * D ? idx / D : idx - 16 * D;
         float mstar = -INFINITY;
@@ -337,30 +431,35 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
         else { cpart[16 * D + r] = mstar; cpart[16 * D + 16 + r] = acc; }
     }
 
-    // 5c. cluster merge by rank 0 through distributed shared memory.
+    // 4c. cluster merge: CTA r combines the r-th eighth of the (row, dim) outputs.
     cluster_sync_all();
-    if (rank == 0) {
+    {
         __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(a.out) + ((long long)b * a.Hq + g * G) * D;
-        for (int idx = tid; idx < G * D; idx += kDecWarps * 32) {
+        const int total = G * D, per = (total + kDecCluster - 1) / kDecCluster;
+        const int i_end = min(total, ((int)rank + 1) * per);
+        for (int idx = (int)rank * per + tid; idx < i_end; idx += kDecWarps * 32) {
             const int r = idx / D;
-            float mr[kDecCluster], mstar = -INFINITY;
+            float mr[kDecCluster], lr[kDecCluster], orr[kDecCluster], mstar = -INFINITY;
 #pragma unroll
             for (int k = 0; k < kDecCluster; ++k) {
                 mr[k] = ld_cluster_f32(map_rank(&cpart[16 * D + r], k));
-                mstar = fmaxf(mstar, mr[k]);
+                lr[k] = ld_cluster_f32(map_rank(&cpart[16 * D + 16 + r], k));
+                orr[k] = ld_cluster_f32(map_rank(&cpart[idx], k));
             }
+#pragma unroll
+            for (int k = 0; k < kDecCluster; ++k) mstar = fmaxf(mstar, mr[k]);
             const float mu = mstar == -INFINITY ? 0.f : mstar;
             float o = 0.f, l = 0.f;
 #pragma unroll
             for (int k = 0; k < kDecCluster; ++k) {
                 const float f = fast_exp2(mr[k] - mu);
-                o += f * ld_cluster_f32(map_rank(&cpart[idx], k));
-                l += f * ld_cluster_f32(map_rank(&cpart[16 * D + 16 + r], k));
+                o += f * orr[k];
+                l += f * lr[k];
             }
             out[idx] = __float2bfloat16_rn(o / l);
         }
     }
-    cluster_sync_all();      // peers stay resident until rank 0 has read their partials
+    cluster_sync_all();      // peers stay resident until every CTA has read their partials
 }
 
 template <int D, int BC>

@@ -29,6 +29,11 @@ struct StageArgs {
     int vt_ready;             // V^T scratch already holds the transpose of V (a later row slice)
     int test_stall;           // test hook: Stage 0's chunk-copy wait runs out (DASH_FLAG_TEST_STALL_WAIT)
     int fuse_route;           // Stage 2 computes the routing itself (fused route-and-attend)
+    // Run-time choice between the 128-key-block and the warp-MMA Stage 2 kernels (null: none):
+    // cost[0] / cost[1] are the token-chunk pairs each would execute (k_union_cost), and the
+    // 128-key-block kernel runs iff cost[0] <= cost[1] * cost_ratio.
+    const unsigned long long *cost;
+    float cost_ratio;
     uint32_t *status;
 };
 
@@ -48,6 +53,22 @@ struct DecodeArgs {
     uint32_t *status;
 };
 
+// Byte offsets in the 256-byte status block at the start of every workspace: the status word
+// (0), the run-time Stage 2 choice's two costs (8, 16) and the kernel that ran (24: 1 the
+// 128-key-block kernel, 2 the warp-MMA kernel, 0 no run-time choice in the last call).
+constexpr int kStatusCostOff = 8;
+constexpr int kStatusRanOff = 24;
+
+// With a run-time Stage 2 choice: whether the 128-key-block kernel is the one that runs.
+__device__ __forceinline__ bool attend_fa_chosen(const StageArgs &a) {
+    return (double)a.cost[0] <= (double)a.cost[1] * (double)a.cost_ratio;
+}
+// Records, once per launch, which kernel a run-time choice ran (1: 128-key blocks, 2: warp MMA).
+__device__ __forceinline__ void attend_record_ran(const StageArgs &a, unsigned char id) {
+    if (blockIdx.x == 0 && threadIdx.x == 0)
+        reinterpret_cast<volatile unsigned char *>(a.status)[kStatusRanOff] = id;
+}
+
 cudaError_t launch_stage0(const StageArgs &a, const int32_t *seq_lens, int n_recent,
                           cudaStream_t st);
 // Stage 0 over the newest complete chunks of a paged cache: k_pool [n_pages, Hkv, Bc, D],
@@ -59,7 +80,9 @@ cudaError_t launch_route(const StageArgs &a, cudaStream_t st);
 int route_rows_per_cta(int C, int D);   // 0 if C is too large for the routing kernel
 cudaError_t launch_attend(const StageArgs &a, cudaStream_t st);
 // The Stage 2 kernel launch_attend picks for these arguments, and its name.
-enum class AttendKernel { kNone, kPair, kFa, kTc, kWarp };
+// kFaOrWarp: both are launched after k_union_cost; each CTA of the one not chosen exits at
+// once (see StageArgs::cost).
+enum class AttendKernel { kNone, kPair, kFa, kTc, kWarp, kFaOrWarp };
 AttendKernel attend_kernel(const StageArgs &a);
 const char *attend_kernel_name(AttendKernel k);
 bool attend_tc_supported(const StageArgs &a);

@@ -72,3 +72,13 @@ def test_tokens_per_tile_follow_the_kernels():
     assert bench.tokens_per_tile("k_attend_pair", 16) == 16
     assert bench.tokens_per_tile("k_attend", 4) == 4
     assert bench.tokens_per_tile("k_attend", 32) == 1
+
+
+def test_support_histogram_bins_and_quantiles():
+    """The support-size histogram counts rows per power-of-two bin and reports quantiles."""
+    import torch
+    cnt = torch.tensor([0, 1, 1, 2, 3, 5, 40, 40, 40, 5000], dtype=torch.int64)
+    h = bench.support_histogram(cnt)
+    assert h["rows"] == 10 and h["max"] == 5000
+    assert h["bins"] == {"0-0": 1, "1-1": 2, "2-3": 2, "4-7": 1, "32-63": 3, "4096-8191": 1}
+    assert h["p50"] == 4.0 and abs(h["mean"] - 513.2) < 1e-9

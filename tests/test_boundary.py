@@ -34,7 +34,7 @@ def test_header_declares_the_documented_entry_points():
 def test_library_exports_every_declared_symbol(dash):
     for name in _declared():
         assert hasattr(dash.lib, name), name          # ctypes resolves via dlsym
-    assert set(dash.EXPORTS) <= set(_declared())
+    assert set(dash.EXPORTS) == set(_declared())
 
 
 def test_status_strings(dash):
@@ -187,7 +187,7 @@ def test_attend_kernel_name_follows_the_dispatch(dash):
     assert dash.attend_kernel_name(_p(dash), 256) == "k_attend_tc"          # no room for V^T
     assert dash.attend_kernel_name(_p(dash, flags=1), big) == "k_attend_pair"
     assert dash.attend_kernel_name(_p(dash, flags=2), big) == "k_attend_pair"
-    assert dash.attend_kernel_name(_p(dash, heads_q=8), big) == "k_attend_fa"  # G = 4: 32-token tiles
+    assert dash.attend_kernel_name(_p(dash, heads_q=8), big) == "k_attend_fa|k_attend"  # G = 4: chosen at run time
     assert dash.attend_kernel_name(_p(dash, heads_q=8), 256) == "k_attend"    # no V^T room, G < 8
     assert dash.attend_kernel_name(_p(dash, heads_q=8, flags=1), big) == "k_attend_pair"
     assert dash.attend_kernel_name(_p(dash, heads_q=4, flags=1), big) == "k_attend_fa"  # G = 2, chunk 64
@@ -196,3 +196,17 @@ def test_attend_kernel_name_follows_the_dispatch(dash):
     assert dash.attend_kernel_name(_p(dash, head_dim=64), big) == "k_attend"   # D = 64
     assert dash.attend_kernel_name(_p(dash, head_dim=96), big) == ""
     assert dash.attend_kernel_name(_p(dash), 255) == ""
+
+
+def test_prefill_kernel_count_follows_the_dispatch(dash):
+    """The library counts the kernels one dash_prefill call launches (host only)."""
+    big = 1 << 40
+    assert dash.prefill_kernel_count(_p(dash), big) == 3              # stage 0, V^T, fused route + attend
+    assert dash.prefill_kernel_count(_p(dash), 256) == 3              # stage 0, route, 64-key blocks
+    assert dash.prefill_kernel_count(_p(dash, flags=1), big) == 2     # dense: V^T, SM pairs
+    assert dash.prefill_kernel_count(_p(dash, head_dim=64), big) == 3  # stage 0, route, warp MMA
+    assert dash.prefill_kernel_count(_p(dash, flags=4), big) == 4     # estimated diagonal: not fused
+    assert dash.prefill_kernel_count(_p(dash, head_dim=96), big) == 0
+    # G = 4: stage 0, route, cost kernel, V^T, both Stage 2 kernels (one exits per CTA)
+    assert dash.prefill_kernel_count(_p(dash, heads_q=8), big) == 6
+    assert dash.prefill_kernel_count(_p(dash, heads_q=8, flags=1), big) == 2   # dense: V^T, SM pairs

@@ -106,3 +106,29 @@ def test_debug_build_host_prefill_and_decode(libs, monkeypatch):
     a, b = _both(dash, rel, dbg, monkeypatch, dec)
     for key in ("out", "p", "active_blocks", "cache"):
         assert torch.equal(a[key], b[key]), key
+
+
+@pytest.mark.parametrize("G,D,Bc,T", [(16, 128, 64, 300 + 5), (4, 128, 128, 607), (1, 64, 64, 333)])
+def test_debug_build_backward_without_violations(libs, monkeypatch, G, D, Bc, T):
+    """dash_backward (routing, the per-chunk token lists, query- and key-side kernels) under the
+    bounds-checking build first, then the release build: no violation, and the same gradients
+    up to the order of the atomic sums (d log p over head groups, dhc over chunks)."""
+    dash, rel, dbg = libs
+    Hkv = 2
+    q, k, v, hc = (x.to(dev) for x in make_prefill(
+        PrefillConfig("dbg", 1, G * Hkv, Hkv, T, D, Bc, 1.5, planted=True, n_max=6, seed=70 + G)))
+    g_ = torch.Generator().manual_seed(5)
+    dout = torch.randn(q.shape, generator=g_).to(torch.bfloat16).to(dev)
+    res = {}
+    for name, lib in (("debug", dbg), ("release", rel)):
+        monkeypatch.setattr(dash, "lib", lib)
+        out = dash.prefill(q, k, v, hc, Bc, 1.5, enable_gqa=True)
+        gr = dash.backward(q, k, v, hc, out, dout, Bc, 1.5)
+        torch.cuda.synchronize()
+        assert dash.read_device_status(gr["ws"]) == 0, name
+        res[name] = gr
+    monkeypatch.setattr(dash, "lib", rel)
+    for key in ("dq", "dk", "dv", "dhc"):
+        a, b = res["debug"][key], res["release"][key]
+        scale = b.abs().max().item()
+        assert (a - b).abs().max().item() <= 1e-4 * max(scale, 1e-30), key

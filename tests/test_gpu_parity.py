@@ -591,3 +591,38 @@ def test_backward_matches_oracle(dash, alpha, G, D, Bc, T):
     ref = oracle.backward(q, k, v, hc, dout, Bc, alpha)
     for name, key in (("dq", "dQ"), ("dk", "dK"), ("dv", "dV"), ("dhc", "dhc")):
         _grad_check(f"{name} G={G} a={alpha}", gr[name].cpu().numpy(), ref[key])
+
+
+# ------------------------------------------------------------------------------ run-time choice
+@pytest.mark.parametrize("alpha,Bc,T", [(1.25, 64, 1500), (2.0, 64, 1500), (1.25, 128, 1400 + 7),
+                                        (2.0, 128, 2100)])
+def test_stage2_choice_at_run_time(dash, alpha, Bc, T):
+    """G = 4 routed prefill: a cost kernel picks the 128-key-block or the warp-MMA Stage 2 from
+    the mask.  The output matches the oracle and equals, bit for bit, the chosen kernel run on
+    its own: the warp kernel through dash_attend without V^T room, the 128-key-block kernel
+    through the sliced host prefill (row slices always take it)."""
+    G, Hkv, D = 4, 2, 128
+    q, k, v, hc = make_prefill(_cfg(1, G * Hkv, Hkv, T, D, Bc, alpha, n_max=12, seed=130 + T))
+    qd, kd, vd, hcd = _to(q, k, v, hc)
+    prm = dash.make_params(1, G * Hkv, Hkv, T, D, Bc, alpha, enable_gqa=True)
+    assert dash.attend_kernel_name(prm, dash.prefill_workspace_size(prm)) == "k_attend_fa|k_attend"
+    res = dash.prefill(qd, kd, vd, hcd, Bc, alpha, enable_gqa=True, return_active_blocks=True)
+    ran = dash.stage2_kernel_ran(res["ws"])
+    assert ran in ("k_attend_fa", "k_attend")
+    assert dash.read_device_status(res["ws"]) == 0
+    ref = oracle.prefill(q, k, v, hc, Bc, alpha)
+    check_output(res["out"].cpu().float().numpy(), ref["O"], tag=f"run-time choice {ran}")
+    if ran == "k_attend":
+        S = dash.stage0(kd, hcd, Bc)
+        r = dash.route(qd, S, Hkv, Bc, alpha)
+        o = dash.attend(qd, kd, vd, S, r["tau"], r["active_blocks"], Bc, alpha, ws=dash.workspace(256, dev))
+        assert dash.attend_kernel_name(prm, 256) == "k_attend"
+    else:
+        hq, hk, hv, hhc = (x.contiguous().pin_memory() for x in (q, k, v, hc))
+        ho = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+        dash.prefill_host(hq, hk, hv, hhc, ho, qd.clone(), kd.clone(), vd.clone(), hcd.clone(),
+                          torch.empty_like(qd), Bc, alpha, enable_gqa=True, n_slices=3)
+        torch.cuda.current_stream().synchronize()
+        o = ho
+    torch.cuda.synchronize()
+    assert torch.equal(o.cpu(), res["out"].cpu())
