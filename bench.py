@@ -21,6 +21,7 @@ workload's tokens/s.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import math
@@ -286,7 +287,39 @@ def timed(fn, steps, stream, flush=None):
 
 
 # ------------------------------------------------------------------------------ decode
+def graph_us(body, stream, reset=None, replays=3):
+    """Median device time (us) of one replay of a CUDA graph of body(), timed with events on
+    `stream`; reset() (outside the timing) restores the state body() mutates."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        if reset is not None:
+            reset()
+        body()                                        # warm-up outside the capture
+        if reset is not None:
+            reset()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            body()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(replays):
+        with torch.cuda.stream(stream):
+            if reset is not None:
+                reset()
+            st = torch.cuda.Event(enable_timing=True)
+            en = torch.cuda.Event(enable_timing=True)
+            st.record(stream)
+            g.replay()                                # replay launches on the current stream
+            en.record(stream)
+        en.synchronize()
+        ts.append(st.elapsed_time(en) * 1e3)
+    del g
+    return statistics.median(ts)
+
+
 def bench_decode(dash, dev, steps_cap=256, warmup=3):
+    """The decode workload: 256 steps of dash_decode_step (append the new K/V, route, attend,
+    summarise a completed chunk, advance seq_lens: one launch per step), in one CUDA graph."""
     cfg = CONFIGS["decode64k"]
     t0 = time.time()
     d = make_decode(cfg)
@@ -297,6 +330,8 @@ def bench_decode(dash, dev, steps_cap=256, warmup=3):
     v_all = d["v_all"].to(dev)
     hc = d["head_cls"].to(dev)
     q_steps = d["q_steps"].to(dev)
+    k_new = k_all[:, :, L0:L0 + S].permute(2, 0, 1, 3).contiguous()       # [S, B, Hkv, D]
+    v_new = v_all[:, :, L0:L0 + S].permute(2, 0, 1, 3).contiguous()
     kc = torch.zeros_like(k_all)
     vc = torch.zeros_like(v_all)
     kc[:, :, :L0] = k_all[:, :, :L0]
@@ -305,29 +340,27 @@ def bench_decode(dash, dev, steps_cap=256, warmup=3):
     seq = torch.full((B,), L0, dtype=torch.int32, device=dev)
     dash.update_chunk_cache(kc, hc, seq, cache, Hq, Bc, n_recent=L0 // Bc)
     out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
-    ws = dash.workspace(256, dev)
-    ws_u = dash.workspace(256, dev)
+    prm = dash.make_params(B, Hq, Hkv, cap, D, Bc, cfg.alpha, enable_gqa=True)
+    ws = dash.workspace(dash.lib.dash_decode_step_workspace_size(ctypes.byref(prm)), dev)
 
-    def step(s, with_routing=None):
-        L = L0 + s + 1
-        kc[:, :, L - 1] = k_all[:, :, L - 1]
-        vc[:, :, L - 1] = v_all[:, :, L - 1]
-        seq.fill_(L)
-        if L % Bc == 0:
-            dash.update_chunk_cache(kc, hc, seq, cache, Hq, Bc, n_recent=1, ws=ws_u)
-        if with_routing is None:
-            dash.decode(q_steps[s], kc, vc, seq, cache, Bc, cfg.alpha, out=out, ws=ws)
-        else:
-            dash.decode(q_steps[s], kc, vc, seq, cache, Bc, cfg.alpha, out=out, ws=ws,
-                        active_blocks=with_routing[s])
+    def reset():
+        seq.fill_(L0)
+
+    def steps(masks=None, flush=None):
+        for s in range(S):
+            if flush is not None:
+                flush()
+            dash.decode_step(q_steps[s], k_new[s], v_new[s], kc, vc, seq, cache, hc, Bc, cfg.alpha,
+                             out=out, ws=ws, active_blocks=None if masks is None else masks[s])
 
     # Routing of every step (untimed pass) for the algorithmic byte count.
     Wcap = ((cap + Bc - 1) // Bc + 63) // 64
     masks = torch.zeros(S, B, Hkv, Wcap, dtype=torch.int64, device=dev)
-    for s in range(S):
-        step(s, masks)
+    reset()
+    steps(masks)
     torch.cuda.synchronize()
     assert dash.read_device_status(ws) == 0
+    assert int(seq.min()) == L0 + S
     act = (popcount_words(masks) - 1).to(torch.float64)          # routed active per (s,b,g)
     L = torch.arange(L0 + 1, L0 + S + 1, device=dev, dtype=torch.float64)
     t = L - 1
@@ -339,100 +372,33 @@ def bench_decode(dash, dev, steps_cap=256, warmup=3):
     visible = float(ct.sum() * B * Hkv)
     sparsity = 1.0 - float(act.sum()) / visible
 
-    # Reset the cache to the prefix and capture all steps in one graph.
-    kc[:, :, L0:] = 0
-    vc[:, :, L0:] = 0
-    seq.fill_(L0)
-    dash.update_chunk_cache(kc, hc, seq, cache, Hq, Bc, n_recent=L0 // Bc)
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
     stream = torch.cuda.Stream(dev)
     stream.wait_stream(torch.cuda.current_stream(dev))
-    with torch.cuda.stream(stream):
-        for s in range(min(warmup, S)):
-            step(s)
-        torch.cuda.synchronize()
-        with torch.cuda.graph(g, stream=stream):
-            for s in range(S):
-                step(s)
-    torch.cuda.synchronize()
-    times = []
-    for _ in range(3):
-        st = torch.cuda.Event(enable_timing=True)
-        en = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):               # replay launches on the current stream
-            st.record(stream)
-            g.replay()
-            en.record(stream)
-        en.synchronize()
-        times.append(st.elapsed_time(en))
-    ms = statistics.median(times)
-    launches = S + sum(1 for s in range(S) if (L0 + s + 1) % Bc == 0)
-    del g
-    kern = bench_decode_kernel(dash, dev, cfg, q_steps, kc, vc, seq, cache, out, ws, S, stream)
-    paged_ms = bench_decode_paged(dash, dev, d, cfg, S, warmup)
+    warm_us = graph_us(steps, stream, reset)
+    flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    flush = flush_buf.zero_
+    cold_us = graph_us(lambda: steps(flush=flush), stream, reset) - graph_us(lambda: [flush() for _ in range(S)], stream)
+    assert dash.read_device_status(ws) == 0
+    ms = warm_us / 1e3
+    paged_us = bench_decode_paged(dash, dev, d, cfg, S, k_new, v_new, stream)
     return dict(tokens_per_s=B * S / (ms / 1e3), ms_per_step=ms / S, steps=S, batch=B,
-                paged={"ms_per_step": paged_ms / S, "tokens_per_s": B * S / (paged_ms / 1e3),
+                paged={"ms_per_step": paged_us / 1e3 / S, "tokens_per_s": B * S / (paged_us / 1e6),
                        "layout": "pages of one chunk, scattered through the pools by a random "
                                  "block table"},
                 cache_len=L0, realised_sparsity=sparsity,
                 hbm_bytes_per_step=alg_bytes / S,
-                achieved_gbs=alg_bytes / (ms / 1e3) / 1e9, launches=launches,
-                kernel=dict(us_l2_warm=kern["warm_us"], us_l2_cold=kern["cold_us"],
-                            gbs_l2_cold=alg_bytes / S / (kern["cold_us"] / 1e6) / 1e9,
-                            note="k_decode alone, 256 launches per graph at the last step's cache "
-                                 "length; cold: each launch after a 256 MiB L2-flushing write, "
-                                 "the graph of writes alone subtracted"),
-                note="steps include the K/V append copies and seq_len update (torch ops)")
+                achieved_gbs=alg_bytes / (ms / 1e3) / 1e9, launches=S,
+                kernel=dict(us_l2_warm=warm_us / S, us_l2_cold=cold_us / S,
+                            gbs_l2_cold=alg_bytes / (cold_us / 1e6) / 1e9,
+                            note="cold: each step after a 256 MiB L2-flushing write, the graph "
+                                 "of writes alone subtracted"),
+                note="one dash_decode_step launch per step (append, route, attend, chunk "
+                     "summary, length update); steps consecutive, L2 warm across them")
 
 
-def bench_decode_kernel(dash, dev, cfg, q_steps, kc, vc, seq, cache, out, ws, S, stream):
-    """k_decode alone: S launches in one graph (L2 warm across launches), and S launches each
-    after an L2-flushing write, minus the graph of the writes alone (L2 cold).  Microseconds per
-    launch, medians of three replays."""
-    Bc = cfg.chunk_size
-    flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-
-    def graph_us(body):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.stream(stream):
-            body()
-            torch.cuda.synchronize()
-            with torch.cuda.graph(g, stream=stream):
-                body()
-        torch.cuda.synchronize()
-        ts = []
-        for _ in range(3):
-            st = torch.cuda.Event(enable_timing=True)
-            en = torch.cuda.Event(enable_timing=True)
-            with torch.cuda.stream(stream):
-                st.record(stream)
-                g.replay()
-                en.record(stream)
-            en.synchronize()
-            ts.append(st.elapsed_time(en) * 1e3)
-        del g
-        return statistics.median(ts)
-
-    def decodes(flush):
-        for s in range(S):
-            if flush:
-                flush_buf.zero_()
-            dash.decode(q_steps[s], kc, vc, seq, cache, Bc, cfg.alpha, out=out, ws=ws)
-
-    def flushes():
-        for _ in range(S):
-            flush_buf.zero_()
-
-    warm = graph_us(lambda: decodes(False)) / S
-    cold = (graph_us(lambda: decodes(True)) - graph_us(flushes)) / S
-    assert dash.read_device_status(ws) == 0
-    return {"warm_us": warm, "cold_us": cold}
-
-
-def bench_decode_paged(dash, dev, d, cfg, S, warmup):
-    """The same 256 decode steps on a paged cache (pages of one chunk, a random block table),
-    captured in one graph; returns the median graph time in ms."""
+def bench_decode_paged(dash, dev, d, cfg, S, k_new, v_new, stream):
+    """The same 256 steps on a paged cache (pages of one chunk, a random block table),
+    captured in one graph; returns the median graph time in us."""
     B, Hq, Hkv, D, Bc = cfg.batch, cfg.heads_q, cfg.heads_kv, cfg.head_dim, cfg.chunk_size
     L0, cap = d["prefix_len"], d["capacity"]
     nb = cap // Bc
@@ -455,44 +421,17 @@ def bench_decode_paged(dash, dev, d, cfg, S, warmup):
     seq = torch.full((B,), L0, dtype=torch.int32, device=dev)
     dash.update_chunk_cache_paged(kp, hc, table, seq, sp, Hq, Bc, n_recent=L0 // Bc)
     out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
-    ws, ws_u = dash.workspace(256, dev), dash.workspace(256, dev)
-    bidx = torch.arange(B, device=dev)
+    prm = dash.make_params(B, Hq, Hkv, cap, D, Bc, cfg.alpha, enable_gqa=True)
+    ws = dash.workspace(dash.lib.dash_decode_step_workspace_size(ctypes.byref(prm)), dev)
 
-    def step(s):
-        L = L0 + s + 1
-        c, r = (L - 1) // Bc, (L - 1) % Bc
-        pages = table[:, c].long()
-        kp[pages, :, r] = k_all[bidx, :, L - 1]
-        vp[pages, :, r] = v_all[bidx, :, L - 1]
-        seq.fill_(L)
-        if L % Bc == 0:
-            dash.update_chunk_cache_paged(kp, hc, table, seq, sp, Hq, Bc, n_recent=1, ws=ws_u)
-        dash.decode_paged(q_steps[s], kp, vp, table, seq, sp, Bc, cfg.alpha, out=out, ws=ws)
+    def steps():
+        for s in range(S):
+            dash.decode_step(q_steps[s], k_new[s], v_new[s], kp, vp, seq, sp, hc, Bc, cfg.alpha,
+                             out=out, ws=ws, block_table=table)
 
-    g = torch.cuda.CUDAGraph()
-    stream = torch.cuda.Stream(dev)
-    stream.wait_stream(torch.cuda.current_stream(dev))
-    with torch.cuda.stream(stream):
-        for s in range(min(warmup, S)):
-            step(s)
-        torch.cuda.synchronize()
-        with torch.cuda.graph(g, stream=stream):
-            for s in range(S):
-                step(s)
-    torch.cuda.synchronize()
-    times = []
-    for _ in range(3):
-        st = torch.cuda.Event(enable_timing=True)
-        en = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):               # replay launches on the current stream
-            st.record(stream)
-            g.replay()
-            en.record(stream)
-        en.synchronize()
-        times.append(st.elapsed_time(en))
-    assert dash.read_device_status(ws) == 0 and dash.read_device_status(ws_u) == 0
-    del g
-    return statistics.median(times)
+    us = graph_us(steps, stream, lambda: seq.fill_(L0))
+    assert dash.read_device_status(ws) == 0
+    return us
 
 
 # ------------------------------------------------------------------------------ oracle

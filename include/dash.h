@@ -301,6 +301,37 @@ dash_status_t dash_decode_paged(const dash_params_t *params, const void *q, cons
                                 uint64_t *active_blocks, void *ws, size_t ws_bytes,
                                 void *stream);
 
+/* Bytes of device workspace dash_decode_step / dash_decode_step_paged need (the status word
+ * and one counter per sequence). */
+size_t dash_decode_step_workspace_size(const dash_params_t *params);
+
+/* A whole decode step in one launch (liuzhao09.github.io "DashAttention 精读", section 2:
+ * incremental decoding with the chunk-representation cache): for each sequence b with
+ * L = seq_lens[b] tokens in the cache,
+ *   1. k_new[b], v_new[b] ([B, H_kv, D] bf16, in) are written into row L of the caches;
+ *   2. the query q[b] is routed and attends exactly as dash_decode with seq_lens[b] = L + 1;
+ *   3. if L + 1 is a multiple of chunk_size, the chunk it completes gets its summary in
+ *      summary_cache (bit-identical to dash_update_chunk_cache's);
+ *   4. seq_lens[b] (int32 DEVICE, in/out) becomes L + 1.
+ * k_cache, v_cache and summary_cache are in/out; head_cls [H_kv, D] fp32 is required; L + 1
+ * must not exceed the capacity (params->seq_len), else DASH_ERR_INVALID_ARGUMENT through
+ * the status word and the sequence is left unchanged.  The other arguments as dash_decode.
+ * The step reads seq_lens[b] before any write, so a loop of steps needs no host work between
+ * them and can be captured in one CUDA graph. */
+dash_status_t dash_decode_step(const dash_params_t *params, const void *q, const void *k_new,
+                               const void *v_new, void *k_cache, void *v_cache, int32_t *seq_lens,
+                               float *summary_cache, const float *head_cls, void *out, float *p,
+                               uint64_t *active_blocks, void *ws, size_t ws_bytes, void *stream);
+/* The same on a paged cache (pools, block table and capacity as dash_decode_paged; the page
+ * of the chunk that holds row L must already be in the block table). */
+dash_status_t dash_decode_step_paged(const dash_params_t *params, const void *q,
+                                     const void *k_new, const void *v_new, void *k_pool,
+                                     void *v_pool, const int32_t *block_table, int max_blocks,
+                                     int n_pages, int32_t *seq_lens, float *summary_pool,
+                                     const float *head_cls, void *out, float *p,
+                                     uint64_t *active_blocks, void *ws, size_t ws_bytes,
+                                     void *stream);
+
 /* Bytes of device workspace dash_backward needs (the routing it recomputes with p, the
  * gradient into p, per-row softmax statistics, group-mean queries, the routing transposed to
  * per-chunk token lists, and the summaries' gradient).  0 on bad parameters. */

@@ -44,7 +44,8 @@ EXPORTS = ("dash_prefill_workspace_size", "dash_prefill", "dash_prefill_host", "
            "dash_decode", "dash_read_device_status", "dash_status_string", "dash_prefill_static_ws",
            "dash_static_ws_read_status", "dash_attend_kernel_name", "dash_prefill_kernel_count", "dash_decode_paged",
            "dash_update_chunk_cache_paged", "dash_backward_workspace_size", "dash_backward",
-           "dash_stage2_kernel_ran")
+           "dash_stage2_kernel_ran", "dash_decode_step_workspace_size", "dash_decode_step",
+           "dash_decode_step_paged")
 
 
 class Params(ctypes.Structure):
@@ -91,6 +92,11 @@ def _declare(lib):
     lib.dash_backward.restype = ctypes.c_int
     lib.dash_decode_paged.argtypes = [_P, _vp, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int, _vp, _vp,
                                       _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.dash_decode_step_workspace_size.argtypes = [_P]
+    lib.dash_decode_step_workspace_size.restype = _sz
+    lib.dash_decode_step.argtypes = [_P] + [_vp] * 12 + [_sz, _vp]
+    lib.dash_decode_step_paged.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int,
+                                           _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
     lib.dash_update_chunk_cache_paged.argtypes = [_P, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int,
                                                   _vp, ctypes.c_int, _vp, _vp, _sz, _vp]
     lib.dash_status_string.argtypes = [ctypes.c_int]
@@ -386,6 +392,50 @@ def decode_paged(q, k_pool, v_pool, block_table, seq_lens, summary_pool, chunk_s
                                  _ptr(block_table), int(max_blocks), int(n_pages), _ptr(seq_lens),
                                  _ptr(summary_pool), _ptr(head_cls), _ptr(out), _ptr(p), _ptr(mask),
                                  _ptr(ws), ws.numel(), _stream(dev)), "dash_decode_paged")
+    if not (return_p or return_active_blocks):
+        return out
+    return dict(out=out, p=p, active_blocks=mask)
+
+
+def decode_step(q, k_new, v_new, k_cache, v_cache, seq_lens, summary_cache, head_cls,
+                chunk_size=64, alpha=1.5, gamma=1.0, sigma=1.0, enable_gqa=True, return_p=False,
+                return_active_blocks=False, out=None, ws=None, estimate_diagonal=False, topk=0,
+                block_table=None, p=None, active_blocks=None):
+    """A whole decode step in one launch: k_new, v_new [B,Hkv,D] bf16 are appended at row
+    seq_lens[b] of the caches, q [B,Hq,D] attends over seq_lens[b] + 1 tokens, a chunk the new
+    token completes gets its summary, and seq_lens is incremented (all in place).  With
+    block_table the caches are page pools (see update_chunk_cache_paged)."""
+    B, Hq, D = q.shape
+    dev = q.device
+    if block_table is None:
+        Hkv, cap = k_cache.shape[1], k_cache.shape[2]
+    else:
+        Hkv = k_cache.shape[1]
+        cap = block_table.shape[1] * chunk_size
+    Ccap = (cap + chunk_size - 1) // chunk_size
+    Wcap = (Ccap + 63) // 64
+    prm = make_params(B, Hq, Hkv, cap, D, chunk_size, alpha, gamma, sigma, enable_gqa,
+                      _flags(False, False, estimate_diagonal), topk)
+    out = torch.empty_like(q) if out is None else out
+    if p is None and return_p:
+        p = torch.empty(B, Hkv, Ccap, dtype=torch.float32, device=dev)
+    mask = active_blocks
+    if mask is None and return_active_blocks:
+        mask = torch.empty(B, Hkv, Wcap, dtype=torch.int64, device=dev)
+    if ws is None:
+        ws = workspace(lib.dash_decode_step_workspace_size(ctypes.byref(prm)), dev)
+    if block_table is None:
+        _check(lib.dash_decode_step(ctypes.byref(prm), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+                                    _ptr(v_cache), _ptr(seq_lens), _ptr(summary_cache), _ptr(head_cls),
+                                    _ptr(out), _ptr(p), _ptr(mask), _ptr(ws), ws.numel(), _stream(dev)),
+               "dash_decode_step")
+    else:
+        _check(lib.dash_decode_step_paged(ctypes.byref(prm), _ptr(q), _ptr(k_new), _ptr(v_new),
+                                          _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                          int(block_table.shape[1]), int(k_cache.shape[0]),
+                                          _ptr(seq_lens), _ptr(summary_cache), _ptr(head_cls), _ptr(out),
+                                          _ptr(p), _ptr(mask), _ptr(ws), ws.numel(), _stream(dev)),
+               "dash_decode_step_paged")
     if not (return_p or return_active_blocks):
         return out
     return dict(out=out, p=p, active_blocks=mask)

@@ -161,11 +161,18 @@ dash_status_t decode_common(const dash_params_t *p, const void *q, const void *k
                             const void *v_cache, const int32_t *block_table, int max_blocks,
                             int n_pages, const int32_t *seq_lens, const float *summary_cache,
                             const float *head_cls, void *out, float *prob,
-                            uint64_t *active_blocks, void *ws, size_t ws_bytes, void *stream) {
+                            uint64_t *active_blocks, void *ws, size_t ws_bytes, void *stream,
+                            const void *k_new = nullptr, const void *v_new = nullptr,
+                            int32_t *seq_inout = nullptr, float *summary_out = nullptr) {
     Shape s;
     dash_status_t rc = check_params(p, &s);
     if (rc != DASH_OK) return rc;
     if (p->flags & (DASH_FLAG_DENSE | DASH_FLAG_FORCE_ALL_ACTIVE)) return DASH_ERR_UNSUPPORTED;
+    const bool step = k_new != nullptr;
+    if (step && (!v_new || !seq_inout || !summary_out || !head_cls || !aligned16(k_new) ||
+                 !aligned16(v_new)))
+        return DASH_ERR_INVALID_ARGUMENT;
+    if (step && ws_bytes < kStatusBytes + align256((size_t)s.B * 4)) return DASH_ERR_WORKSPACE_TOO_SMALL;
     if (!q || !k_cache || !v_cache || !seq_lens || !summary_cache || !out || !ws)
         return DASH_ERR_INVALID_ARGUMENT;
     if ((p->flags & DASH_FLAG_ESTIMATE_DIAGONAL) && !head_cls) return DASH_ERR_INVALID_ARGUMENT;
@@ -203,6 +210,24 @@ dash_status_t decode_common(const dash_params_t *p, const void *q, const void *k
     a.qk_scale2 = (float)(1.4426950408889634 / std::sqrt((double)s.D));
     a.status = static_cast<uint32_t *>(ws);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (step) {
+        a.k_new = k_new;
+        a.v_new = v_new;
+        a.seq_out = seq_inout;
+        a.summary_out = summary_out;
+        // Per-sequence arrival counters: in the status block's free bytes (32..255) for up to
+        // 56 sequences, cleared with the status word by one memset; else after the block.
+        unsigned char *w = static_cast<unsigned char *>(ws);
+        if (s.B <= (int)((kStatusBytes - 32) / 4)) {
+            a.arrive = reinterpret_cast<int *>(w + 32);
+            if ((rc = from_cuda(cudaMemsetAsync(w, 0, 32 + (size_t)s.B * 4, st))) != DASH_OK) return rc;
+        } else {
+            a.arrive = reinterpret_cast<int *>(w + kStatusBytes);
+            if ((rc = clear_status(ws, st)) != DASH_OK) return rc;
+            if ((rc = from_cuda(cudaMemsetAsync(a.arrive, 0, (size_t)s.B * 4, st))) != DASH_OK) return rc;
+        }
+        return from_cuda(launch_decode(a, st));
+    }
     if ((rc = clear_status(ws, st)) != DASH_OK) return rc;
     return from_cuda(launch_decode(a, st));
 }
@@ -538,6 +563,38 @@ dash_status_t dash_decode_paged(const dash_params_t *p, const void *q, const voi
     if ((long long)max_blocks * p->chunk_size != (long long)p->seq_len) return DASH_ERR_INVALID_ARGUMENT;
     return decode_common(p, q, k_pool, v_pool, block_table, max_blocks, n_pages, seq_lens,
                          summary_pool, head_cls, out, prob, active_blocks, ws, ws_bytes, stream);
+}
+
+size_t dash_decode_step_workspace_size(const dash_params_t *p) {
+    Shape s;
+    if (check_params(p, &s) != DASH_OK) return 0;
+    return kStatusBytes + align256((size_t)s.B * 4);
+}
+
+dash_status_t dash_decode_step(const dash_params_t *p, const void *q, const void *k_new,
+                               const void *v_new, void *k_cache, void *v_cache, int32_t *seq_lens,
+                               float *summary_cache, const float *head_cls, void *out,
+                               float *prob, uint64_t *active_blocks, void *ws, size_t ws_bytes,
+                               void *stream) {
+    if (!k_new) return DASH_ERR_INVALID_ARGUMENT;
+    return decode_common(p, q, k_cache, v_cache, nullptr, 0, 0, seq_lens, summary_cache,
+                         head_cls, out, prob, active_blocks, ws, ws_bytes, stream, k_new, v_new,
+                         seq_lens, summary_cache);
+}
+
+dash_status_t dash_decode_step_paged(const dash_params_t *p, const void *q, const void *k_new,
+                                     const void *v_new, void *k_pool, void *v_pool,
+                                     const int32_t *block_table, int max_blocks, int n_pages,
+                                     int32_t *seq_lens, float *summary_pool, const float *head_cls,
+                                     void *out, float *prob, uint64_t *active_blocks, void *ws,
+                                     size_t ws_bytes, void *stream) {
+    if (!p || !k_new || !block_table || max_blocks < 1 || n_pages < 1 ||
+        (reinterpret_cast<uintptr_t>(block_table) & 3u))
+        return DASH_ERR_INVALID_ARGUMENT;
+    if ((long long)max_blocks * p->chunk_size != (long long)p->seq_len) return DASH_ERR_INVALID_ARGUMENT;
+    return decode_common(p, q, k_pool, v_pool, block_table, max_blocks, n_pages, seq_lens,
+                         summary_pool, head_cls, out, prob, active_blocks, ws, ws_bytes, stream,
+                         k_new, v_new, seq_lens, summary_pool);
 }
 
 dash_status_t dash_update_chunk_cache_paged(const dash_params_t *p, const void *k_pool,

@@ -307,12 +307,68 @@ __device__ __forceinline__ float ipow(float m, int e) {
     return r;
 }
 
+// Stage 0 summary of one chunk by one warp: l_j = head_cls . k_j / sqrt(D),
+// summary = sum_j exp(l_j - max) k_j / sum_j exp(l_j - max); ks: the chunk's BC keys
+// ([BC][D] bf16, shared or global memory), out: D floats.  The prefill / cache-update kernel
+// and the decode step both call it, so a chunk's summary has the same bits either way.
+template <int D, int BC>
+__device__ __forceinline__ void summarize_chunk_warp(const __nv_bfloat16 *ks, const float *hc,
+                                                     float *out) {
+    constexpr int PER = D / 32;          // dims per lane
+    constexpr int SLOTS = BC / 32;       // logits kept per lane
+    const int lane = threadIdx.x & 31;
+    float h[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) h[i] = hc[lane * PER + i];
+    const float inv_sqrt_d = rsqrtf((float)D);
+    float logit[SLOTS];
+#pragma unroll
+    for (int i = 0; i < SLOTS; ++i) logit[i] = 0.f;
+#pragma unroll
+    for (int sl = 0; sl < SLOTS; ++sl) {
+#pragma unroll 4
+        for (int jj = 0; jj < 32; ++jj) {
+            const __nv_bfloat16 *kr = ks + (sl * 32 + jj) * D + lane * PER;
+            float part = 0.f;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) part = fmaf(h[i], __bfloat162float(kr[i]), part);
+            part = warp_sum(part);
+            if (jj == lane) logit[sl] = part * inv_sqrt_d;
+        }
+    }
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < SLOTS; ++i) mx = fmaxf(mx, logit[i]);
+    mx = warp_max(mx);
+    float den = 0.f;
+#pragma unroll
+    for (int i = 0; i < SLOTS; ++i) { logit[i] = expf(logit[i] - mx); den += logit[i]; }
+    den = warp_sum(den);
+    float acc[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int sl = 0; sl < SLOTS; ++sl) {
+#pragma unroll 4
+        for (int jj = 0; jj < 32; ++jj) {
+            float w = __shfl_sync(kFull, logit[sl], jj);
+            const __nv_bfloat16 *kr = ks + (sl * 32 + jj) * D + lane * PER;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) acc[i] = fmaf(w, __bfloat162float(kr[i]), acc[i]);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i) out[lane * PER + i] = acc[i] / den;
+}
+
 // estimate_diagonal: the routing dot qbar . dsum of the diagonal chunk of one row, where dsum
 // is Stage 0's summary taken over the n_vis keys of that chunk the row can see:
 // dsum = sum_j w_j k_j, w = softmax_j(hc . k_j / sqrt(D)), so qbar . dsum = sum_j w_j (qbar . k_j).
 // keys: the chunk's first key, bf16 rows of D (16-byte aligned); 1 <= n_vis <= 128; all 32
 // lanes of one warp call it and get the same value.
-template <int D>
+// kCoherent: the keys may have been written earlier in the same kernel (plain loads instead
+// of the read-only path).
+template <int D, bool kCoherent = false>
 __device__ __forceinline__ float diag_dot(const __nv_bfloat16 *keys, int n_vis, const float *hc,
                                           const float *qbar, float inv_sqrt_d) {
     const int lane = threadIdx.x & 31;
@@ -328,7 +384,7 @@ __device__ __forceinline__ float diag_dot(const __nv_bfloat16 *keys, int n_vis, 
             float a = 0.f, b = 0.f;
 #pragma unroll 4
             for (int d8 = 0; d8 < D / 8; ++d8) {
-                const uint4 v = __ldg(kr + d8);
+                const uint4 v = kCoherent ? kr[d8] : __ldg(kr + d8);
                 const __nv_bfloat162 *b2 = reinterpret_cast<const __nv_bfloat162 *>(&v);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {

@@ -107,7 +107,8 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
     const uint32_t rank = cluster_rank();
     const int bg = blockIdx.x / kDecCluster, b = bg / a.Hkv, g = bg % a.Hkv;
     const int G = a.G;
-    const int Lb = a.seq_lens[b];
+    const bool append = a.k_new != nullptr;
+    const int Lb = a.seq_lens[b] + (append ? 1 : 0);   // tokens attended, the new one included
     if (Lb < 1 || Lb > a.cap) {                 // uniform across the cluster: no barrier
         if (tid == 0 && rank == 0) report(a.status, DASH_ERR_INVALID_ARGUMENT);
         return;
@@ -146,6 +147,21 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
     const bool diag_warp = rank == 0 && warp == 1;
     const int n_diag = (t - ct * BC) / kSub + 1;   // sub-blocks of the diagonal chunk up to t
     if (diag_warp) {
+        if (append) {
+            // Decode step: the new token's key and value into row t of the cache first (the
+            // cluster barrier after the scores publishes them to the other CTAs).
+            const long long src = ((long long)b * a.Hkv + g) * D;
+            __nv_bfloat16 *kd = const_cast<__nv_bfloat16 *>(kv_base(a.k, ct)) + (long long)(t - ct * BC) * D;
+            __nv_bfloat16 *vd = const_cast<__nv_bfloat16 *>(kv_base(a.v, ct)) + (long long)(t - ct * BC) * D;
+            const uint2 *ksrc = reinterpret_cast<const uint2 *>(reinterpret_cast<const __nv_bfloat16 *>(a.k_new) + src);
+            const uint2 *vsrc = reinterpret_cast<const uint2 *>(reinterpret_cast<const __nv_bfloat16 *>(a.v_new) + src);
+            for (int i = lane; i < D / 4; i += 32) {
+                reinterpret_cast<uint2 *>(kd)[i] = ksrc[i];
+                reinterpret_cast<uint2 *>(vd)[i] = vsrc[i];
+            }
+            __threadfence();
+            __syncwarp();
+        }
         // The diagonal chunk is always attended: start its first copies now.
         load_sub<D>(ks, kv_base(a.k, ct), 0, kv_rows(ct));
         cp_async_commit();
@@ -285,8 +301,11 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
     const int n_eff = n + (a.rc.est_diag ? 1 : 0);
     if (warp == 0) {
         if (a.rc.est_diag) {
-            const float dd = diag_dot<D>(kv_base(a.k, ct), t - ct * BC + 1,
-                                         a.head_cls + (long long)g * D, qbar, a.rc.inv_sqrt_d);
+            // (with a decode step, row t was written in this launch: coherent loads)
+            const float dd = append ? diag_dot<D, true>(kv_base(a.k, ct), t - ct * BC + 1,
+                                                        a.head_cls + (long long)g * D, qbar, a.rc.inv_sqrt_d)
+                                    : diag_dot<D>(kv_base(a.k, ct), t - ct * BC + 1,
+                                                  a.head_cls + (long long)g * D, qbar, a.rc.inv_sqrt_d);
             if (lane == 0) xs[n] = __fmul_rn(dd, scale);
             __syncwarp();
         }
@@ -460,6 +479,23 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
         }
     }
     cluster_sync_all();      // peers stay resident until every CTA has read their partials
+    if (append && rank == 0) {
+        // Decode step: the chunk the new token completed gets its Stage 0 summary (the same
+        // function as the cache-update kernel; the keys were written by this CTA), and the
+        // sequence's last cluster to finish stores the new length.
+        if (warp == 2 && (t + 1) % BC == 0) {
+            float *dst = bt ? a.summary_out + ((long long)bt[ct] * a.Hkv + g) * D
+                            : a.summary_out + ((long long)bg * a.Cf + ct) * D;
+            summarize_chunk_warp<D, BC>(kv_base(a.k, ct), a.head_cls + (long long)g * D, dst);
+        }
+        if (tid == 0) {
+            __threadfence();
+            if (atomicAdd(&a.arrive[b], 1) == a.Hkv - 1) {
+                a.arrive[b] = 0;
+                a.seq_out[b] = Lb;
+            }
+        }
+    }
 }
 
 template <int D, int BC>

@@ -50,12 +50,21 @@ struct DecodeArgs {
     int B, Hq, Hkv, cap, D, Bc, G, Ccap, Cf, Wcap;
     RouteConsts rc;
     float qk_scale2;
+    // Decode step (k_new != null): the new token's k/v [B,Hkv,D] go to position seq_lens[b]
+    // of the cache before the step attends over seq_lens[b] + 1 tokens; the last of the
+    // sequence's Hkv clusters to finish (arrive[b] counts them) stores seq_lens[b] + 1 into
+    // seq_out[b]; a chunk completed by the new token gets its summary in summary_out.
+    const void *k_new, *v_new;
+    int32_t *seq_out;
+    int *arrive;
+    float *summary_out;
     uint32_t *status;
 };
 
 // Byte offsets in the 256-byte status block at the start of every workspace: the status word
 // (0), the run-time Stage 2 choice's two costs (8, 16) and the kernel that ran (24: 1 the
-// 128-key-block kernel, 2 the warp-MMA kernel, 0 no run-time choice in the last call).
+// 128-key-block kernel, 2 the warp-MMA kernel, 0 no run-time choice in the last call); a
+// decode step keeps its per-sequence counters at 32.. when they fit.
 constexpr int kStatusCostOff = 8;
 constexpr int kStatusRanOff = 24;
 

@@ -16,56 +16,6 @@
 
 namespace dash {
 
-template <int D, int BC>
-__device__ __forceinline__ void summarize_chunk_warp(const __nv_bfloat16 *ks, const float *hc,
-                                                     float *out) {
-    constexpr int PER = D / 32;          // dims per lane
-    constexpr int SLOTS = BC / 32;       // logits kept per lane
-    const int lane = threadIdx.x & 31;
-    float h[PER];
-#pragma unroll
-    for (int i = 0; i < PER; ++i) h[i] = hc[lane * PER + i];
-    const float inv_sqrt_d = rsqrtf((float)D);
-    float logit[SLOTS];
-#pragma unroll
-    for (int i = 0; i < SLOTS; ++i) logit[i] = 0.f;
-#pragma unroll
-    for (int sl = 0; sl < SLOTS; ++sl) {
-#pragma unroll 4
-        for (int jj = 0; jj < 32; ++jj) {
-            const __nv_bfloat16 *kr = ks + (sl * 32 + jj) * D + lane * PER;
-            float part = 0.f;
-#pragma unroll
-            for (int i = 0; i < PER; ++i) part = fmaf(h[i], __bfloat162float(kr[i]), part);
-            part = warp_sum(part);
-            if (jj == lane) logit[sl] = part * inv_sqrt_d;
-        }
-    }
-    float mx = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < SLOTS; ++i) mx = fmaxf(mx, logit[i]);
-    mx = warp_max(mx);
-    float den = 0.f;
-#pragma unroll
-    for (int i = 0; i < SLOTS; ++i) { logit[i] = expf(logit[i] - mx); den += logit[i]; }
-    den = warp_sum(den);
-    float acc[PER];
-#pragma unroll
-    for (int i = 0; i < PER; ++i) acc[i] = 0.f;
-#pragma unroll
-    for (int sl = 0; sl < SLOTS; ++sl) {
-#pragma unroll 4
-        for (int jj = 0; jj < 32; ++jj) {
-            float w = __shfl_sync(kFull, logit[sl], jj);
-            const __nv_bfloat16 *kr = ks + (sl * 32 + jj) * D + lane * PER;
-#pragma unroll
-            for (int i = 0; i < PER; ++i) acc[i] = fmaf(w, __bfloat162float(kr[i]), acc[i]);
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < PER; ++i) out[lane * PER + i] = acc[i] / den;
-}
-
 // Grid: one warp per unit.  Prefill units are (b, g, c) for every complete chunk; decode
 // units (seq_lens != nullptr) are (b, g, r) = the r-th most recent complete chunk.
 // Paged caches (block_table != nullptr): the keys of logical chunk c of sequence b live in

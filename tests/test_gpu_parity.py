@@ -626,3 +626,77 @@ def test_stage2_choice_at_run_time(dash, alpha, Bc, T):
         o = ho
     torch.cuda.synchronize()
     assert torch.equal(o.cpu(), res["out"].cpu())
+
+
+# ------------------------------------------------------------------------------ decode step
+@pytest.mark.parametrize("kw", [dict(), dict(estimate_diagonal=True), dict(topk=4)])
+def test_decode_step_equals_append_update_and_decode(dash, kw):
+    """dash_decode_step (append the new K/V, route, attend, summarise a completed chunk,
+    increment seq_lens, one launch) over 70 steps of three ragged sequences, each crossing
+    chunk boundaries, equals bit for bit the separate path (K/V rows written by the host,
+    dash_update_chunk_cache, dash_decode): outputs and routing every step, caches, summaries
+    and lengths at the end; the paged step equals the contiguous one."""
+    B, Hkv, G, D, Bc = 3, 2, 16, 128, 64
+    max_blocks = 24
+    cap = max_blocks * Bc
+    steps = 70
+    q, k, v, hc = make_prefill(_cfg(B, G * Hkv, Hkv, cap, D, Bc, 1.5, seed=87))
+    qd, kd, vd, hcd = _to(q, k, v, hc)
+    L0 = [Bc * 11 + 3, Bc * 5 - 1, 17]
+    # separate path (A), fused step (Bc), fused step on pages (Bp)
+    kA, vA = torch.zeros_like(kd), torch.zeros_like(vd)
+    for b in range(B):
+        kA[b, :, :L0[b]] = kd[b, :, :L0[b]]
+        vA[b, :, :L0[b]] = vd[b, :, :L0[b]]
+    kB, vB = kA.clone(), vA.clone()
+    seqA = torch.tensor(L0, dtype=torch.int32, device=dev)
+    seqB, seqP = seqA.clone(), seqA.clone()
+    cA = torch.zeros(B, Hkv, max_blocks, D, device=dev)
+    dash.update_chunk_cache(kA, hcd, seqA, cA, heads_q=G * Hkv, chunk_size=Bc, n_recent=max_blocks)
+    cB = cA.clone()
+    n_pages = B * max_blocks + 3
+    table = torch.randperm(n_pages, generator=torch.Generator().manual_seed(5))[:B * max_blocks]
+    table = table.view(B, max_blocks).to(torch.int32).to(dev)
+    kP = torch.zeros(n_pages, Hkv, Bc, D, dtype=torch.bfloat16, device=dev)
+    vP = torch.zeros_like(kP)
+    sP = torch.zeros(n_pages, Hkv, D, device=dev)
+    for b in range(B):
+        for c in range(max_blocks):
+            kP[table[b, c]] = kA[b, :, c * Bc:(c + 1) * Bc]
+            vP[table[b, c]] = vA[b, :, c * Bc:(c + 1) * Bc]
+            sP[table[b, c]] = cA[b, :, c]
+    wsA, wsB, wsP, wsU = (dash.workspace(4096, dev) for _ in range(4))
+    hk = hcd if kw.get("estimate_diagonal") else None
+    for s in range(steps):
+        pos = [L0[b] + s for b in range(B)]
+        qs = torch.stack([qd[b, :, pos[b]] for b in range(B)])
+        kn = torch.stack([kd[b, :, pos[b]] for b in range(B)])
+        vn = torch.stack([vd[b, :, pos[b]] for b in range(B)])
+        for b in range(B):
+            kA[b, :, pos[b]] = kn[b]
+            vA[b, :, pos[b]] = vn[b]
+        seqA += 1
+        dash.update_chunk_cache(kA, hcd, seqA, cA, heads_q=G * Hkv, chunk_size=Bc, n_recent=1, ws=wsU)
+        ra = dash.decode(qs, kA, vA, seqA, cA, Bc, return_p=True, return_active_blocks=True, ws=wsA,
+                         head_cls=hk, **kw)
+        rb = dash.decode_step(qs, kn, vn, kB, vB, seqB, cB, hcd, Bc, return_p=True,
+                              return_active_blocks=True, ws=wsB, **kw)
+        rp = dash.decode_step(qs, kn, vn, kP, vP, seqP, sP, hcd, Bc, return_p=True,
+                              return_active_blocks=True, ws=wsP, block_table=table, **kw)
+        for key in ("out", "p", "active_blocks"):
+            assert torch.equal(ra[key], rb[key]), (s, key)
+            assert torch.equal(rb[key], rp[key]), (s, key, "paged")
+    torch.cuda.synchronize()
+    for ws in (wsA, wsB, wsP, wsU):
+        assert dash.read_device_status(ws) == 0
+    assert torch.equal(seqA, seqB) and torch.equal(seqA, seqP)
+    assert torch.equal(kA, kB) and torch.equal(vA, vB) and torch.equal(cA, cB)
+    for b in range(B):
+        for c in range(int(seqA[b]) // Bc):
+            assert torch.equal(sP[table[b, c]], cA[b, :, c])
+            assert torch.equal(kP[table[b, c]], kA[b, :, c * Bc:(c + 1) * Bc])
+    # a step past the capacity is refused on the device and leaves the sequence unchanged
+    full = torch.tensor([cap, 5, 5], dtype=torch.int32, device=dev)
+    dash.decode_step(qs, kn, vn, kB, vB, full, cB, hcd, Bc, ws=wsB)
+    assert dash.read_device_status(wsB) == 1
+    assert full[0].item() == cap
