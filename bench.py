@@ -286,6 +286,33 @@ def timed(fn, steps, stream, flush=None):
     return times
 
 
+def bench_backward(dash, q, k, v, hc, out, cfg, stream, flush, stats):
+    """dash_backward (gradients w.r.t. q, k, v, head_cls of sum(out * dout) through the three
+    stages) on the same inputs, L2 flushed before each call.  Algorithmic FLOPs: the five
+    products of attention backward per attended (token, key, head) (S, dP, dQ, dK, dV:
+    10 D) = 2.5 x the forward's active FLOPs; the routing backward is not counted."""
+    dash.prefill(q, k, v, hc, cfg.chunk_size, cfg.alpha, cfg.gamma, enable_gqa=True, out=out)
+    dout = torch.randn(q.shape, generator=torch.Generator(device=q.device).manual_seed(1),
+                       device=q.device).to(torch.bfloat16)
+    prm = dash.make_params(q.shape[0], q.shape[1], k.shape[1], q.shape[2], q.shape[3], cfg.chunk_size,
+                           cfg.alpha, cfg.gamma, 1.0, True)
+    ws = dash.workspace(dash.lib.dash_backward_workspace_size(ctypes.byref(prm)), q.device)
+
+    def run():
+        dash.backward(q, k, v, hc, out, dout, cfg.chunk_size, cfg.alpha, cfg.gamma, ws=ws)
+
+    run()
+    ms = statistics.mean(timed(run, 2, stream, flush))
+    assert dash.read_device_status(ws) == 0
+    flops = 2.5 * stats["active_flops"]
+    del ws, dout
+    torch.cuda.empty_cache()
+    return {"ms": ms, "tflops": flops / (ms / 1e3) / 1e12, "algorithmic_flop": flops,
+            "kernels": "k_stage0, k_route (with p), k_bwd_q, k_bwd_lists x2, k_bwd_scan, k_bwd_kv, "
+                       "k_bwd_route, k_bwd_dsum, k_bwd_stage0 (warp-level MMA)",
+            "note": "2.5 x the forward's active FLOPs (S, dP, dQ, dK, dV per attended pair)"}
+
+
 # ------------------------------------------------------------------------------ decode
 def graph_us(body, stream, reset=None, replays=3):
     """Median device time (us) of one replay of a CUDA graph of body(), timed with events on
@@ -721,6 +748,7 @@ def bench_prefill(dash, cfg, args, dev, world, rank, full=True):
         torch.cuda.synchronize()
         assert dash.read_device_status(ws) == 0
         line["routing_variants"] = variants
+        line["backward"] = bench_backward(dash, q, k, v, hc, out, cfg, stream, flush, stats)
         # End to end through host buffers: dash_prefill_host copies q, k, v, head_cls from
         # pinned host memory and out back, in row slices overlapped with the computation.
         hq, hk, hv, hhc = (x.pin_memory() for x in (q_h, k_h, v_h, hc_h))
