@@ -237,6 +237,20 @@ def stage01_bytes(cfg):
     return dict(stage0=k_bytes + summ, stage1=q_bytes + summ + mask + tau)
 
 
+def stage1_score_flops(cfg):
+    """FLOPs of Stage 1's scores: qbar . summary_c (2 D) for every row and routable chunk
+    c < c_t (the group mean and the entmax solve not counted)."""
+    B, Hkv, T, D, Bc = cfg.batch, cfg.heads_kv, cfg.seq_len, cfg.head_dim, cfg.chunk_size
+    Cf = T // Bc
+    pairs = Bc * Cf * (Cf - 1) // 2 + (T - Cf * Bc) * Cf       # sum over t of floor(t / Bc)
+    return 2.0 * D * B * Hkv * pairs
+
+
+# FP32 FMA peak of the CUDA cores: 148 SMs x 128 FMA lanes x 2 FLOP x the maximum SM clock
+# (1965 MHz); the Stage 1 scores run there (fp32 FMA chains in a fixed order).
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
 def max_over_ranks(x: float, device) -> float:
     """The maximum of x over the ranks of the default process group (x itself when there is
     none): every multi-rank time is the slowest rank's.  device is where the reduction runs
@@ -728,6 +742,13 @@ def bench_prefill(dash, cfg, args, dev, world, rank, full=True):
                              "unit": "GB/s", "frac": s01_gbs / pk["hbm_gbs"],
                              "frac_of_8tbs_nominal": s01_gbs / 8000.0,
                              "bytes": sb["stage0"] + sb["stage1"]},
+        "roofline_stage1_alu": {"bound": "alu",
+                                "achieved": stage1_score_flops(cfg) / (stage["stage1"] / 1e3) / 1e12,
+                                "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
+                                "frac": stage1_score_flops(cfg) / (stage["stage1"] / 1e3) / 1e12 / FP32_PEAK_TFLOPS,
+                                "note": "Stage 1's score FLOPs (2 D per row and routable chunk) over its "
+                                        "time through dash_route, against the fp32 FMA peak of the CUDA "
+                                        "cores (148 SMs x 128 lanes x 2 x 1965 MHz)"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }

@@ -82,3 +82,14 @@ def test_support_histogram_bins_and_quantiles():
     assert h["rows"] == 10 and h["max"] == 5000
     assert h["bins"] == {"0-0": 1, "1-1": 2, "2-3": 2, "4-7": 1, "32-63": 3, "4096-8191": 1}
     assert h["p50"] == 4.0 and abs(h["mean"] - 513.2) < 1e-9
+
+
+def test_stage1_score_flops_counts_routable_pairs():
+    """Stage 1's score FLOPs: 2 D per (row, routable chunk), routable chunks of row t being
+    floor(t / Bc) — checked by brute force on a small shape."""
+    import bench
+    from dash_inputs import PrefillConfig
+    cfg = PrefillConfig("t", 2, 8, 2, 1000, 128, 64, 1.5)
+    brute = sum(t // 64 for t in range(1000)) * 2 * 128 * 2 * 2
+    assert bench.stage1_score_flops(cfg) == brute
+    assert abs(bench.FP32_PEAK_TFLOPS - 148 * 128 * 2 * 1.965e-3) < 1e-9
