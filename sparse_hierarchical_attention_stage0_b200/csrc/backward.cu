@@ -33,6 +33,7 @@ namespace dash {
 namespace {
 
 constexpr int kBwdWarps = 4;
+constexpr int kBwdSlice = 1024;        // k_bwd_kv entries per CTA
 
 struct BwdArgs {
     StageArgs s;                 // shapes, q, k, v, head_cls, summary, tau, mask, p (routing)
@@ -482,10 +483,13 @@ __global__ void k_bwd_scan(BwdArgs ba) {
 }
 
 // ---------------------------------------------------------------- k_bwd_kv
-// One CTA per (b, g, chunk c), BC / 16 warps (warp w: keys c BC + 16 w .. + 15).  Entries are
-// (token, group of up to 16 heads): the chunk's own tokens (diagonal, bias 0, causal), then
-// its routed tokens (bias = sigma log p).  Per entry, each warp computes S^T = K_w Q^T,
-// P^T, dP^T = V_w dO^T, dS^T and accumulates dv += P^T dO, dk += dS^T Q in registers.
+// One CTA per (b, g, chunk c, slice of kBwdSlice entries), BC / 16 warps (warp w: keys
+// c BC + 16 w .. + 15).  Entries are (token, group of up to 16 heads): the chunk's own tokens
+// (diagonal, bias 0, causal), then its routed tokens (bias = sigma log p); the first chunks of
+// a long sequence are routed to by up to a quarter of it, so each CTA takes one slice of
+// the entries and adds its partial dk, dv into memory (zeroed first).  Per entry, each warp
+// computes S^T = K_w Q^T, P^T, dP^T = V_w dO^T, dS^T and accumulates dv += P^T dO,
+// dk += dS^T Q in registers.
 template <int D, int BC>
 __global__ void __launch_bounds__(BC / 16 * 32) k_bwd_kv(BwdArgs ba, int UPT) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -505,6 +509,13 @@ __global__ void __launch_bounds__(BC / 16 * 32) k_bwd_kv(BwdArgs ba, int UPT) {
     const __nv_bfloat16 *kp = reinterpret_cast<const __nv_bfloat16 *>(a.k) + bg * a.T * D;
     const __nv_bfloat16 *vp = reinterpret_cast<const __nv_bfloat16 *>(a.v) + bg * a.T * D;
     const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(a.q);
+    const int n_diag = min(BC, a.T - c * BC);
+    const long long n_routed = c < a.Cf ? ba.list_cnt[bg * a.C + c] : 0;
+    const long long off = c < a.Cf ? ba.list_off[bg * (a.C + 1) + c] : 0;
+    const long long n_entries = ((long long)n_diag + n_routed) * UPT;
+    const long long e_begin = (long long)blockIdx.z * kBwdSlice;
+    const long long e_end = min(n_entries, e_begin + kBwdSlice);
+    if (e_begin >= n_entries) return;                        // the same in every thread
     constexpr int CH = D / 8;
     for (int i = tid; i < BC * CH; i += NW * 32) {
         const int row = i / CH, ch = i % CH, key = c * BC + row;
@@ -523,11 +534,7 @@ __global__ void __launch_bounds__(BC / 16 * 32) k_bwd_kv(BwdArgs ba, int UPT) {
     const int r_lo = lane >> 2, qd = lane & 3;                // key rows r_lo, r_lo + 8 of the warp
     const int key_lo = c * BC + 16 * warp + r_lo, key_hi = key_lo + 8;
 
-    const int n_diag = min(BC, a.T - c * BC);
-    const long long n_routed = c < a.Cf ? ba.list_cnt[bg * a.C + c] : 0;
-    const long long off = c < a.Cf ? ba.list_off[bg * (a.C + 1) + c] : 0;
-    const long long n_entries = ((long long)n_diag + n_routed) * UPT;
-    for (long long e = 0; e < n_entries; ++e) {
+    for (long long e = e_begin; e < e_end; ++e) {
         const long long ti = e / UPT;
         const int kunit = (int)(e % UPT);
         const bool diag = ti < n_diag;
@@ -606,17 +613,17 @@ __global__ void __launch_bounds__(BC / 16 * 32) k_bwd_kv(BwdArgs ba, int UPT) {
         const int d0 = 8 * j + 2 * qd;
         if (key_lo < a.T) {
             const long long o = (bg * a.T + key_lo) * D + d0;
-            ba.dk[o] = dka[j][0] * rs;
-            ba.dk[o + 1] = dka[j][1] * rs;
-            ba.dv[o] = dva[j][0];
-            ba.dv[o + 1] = dva[j][1];
+            atomicAdd(&ba.dk[o], dka[j][0] * rs);
+            atomicAdd(&ba.dk[o + 1], dka[j][1] * rs);
+            atomicAdd(&ba.dv[o], dva[j][0]);
+            atomicAdd(&ba.dv[o + 1], dva[j][1]);
         }
         if (key_hi < a.T) {
             const long long o = (bg * a.T + key_hi) * D + d0;
-            ba.dk[o] = dka[j][2] * rs;
-            ba.dk[o + 1] = dka[j][3] * rs;
-            ba.dv[o] = dva[j][2];
-            ba.dv[o + 1] = dva[j][3];
+            atomicAdd(&ba.dk[o], dka[j][2] * rs);
+            atomicAdd(&ba.dk[o + 1], dka[j][3] * rs);
+            atomicAdd(&ba.dv[o], dva[j][2]);
+            atomicAdd(&ba.dv[o + 1], dva[j][3]);
         }
     }
 }
@@ -807,7 +814,9 @@ cudaError_t launch_bwd_t(BwdArgs ba, cudaStream_t st) {
         const size_t smem = 2 * (size_t)BC * D * 2 + 2 * (size_t)16 * D * 2 + 48 * 4;
         auto kern = k_bwd_kv<D, BC>;
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
-        kern<<<dim3((unsigned)a.C, (unsigned)(a.B * a.Hkv)), BC / 16 * 32, smem, st>>>(ba, UPT);
+        // slices: enough for the longest possible list (chunk 0: every token of the sequence)
+        const unsigned slices = (unsigned)(((long long)a.T * UPT + kBwdSlice - 1) / kBwdSlice);
+        kern<<<dim3((unsigned)a.C, (unsigned)(a.B * a.Hkv), slices), BC / 16 * 32, smem, st>>>(ba, UPT);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     // 4-6. routing, summaries, Stage 0

@@ -691,6 +691,10 @@ dash_status_t dash_backward(const dash_params_t *p, const void *q, const void *k
     if ((rc = clear_status(ws, st)) != DASH_OK) return rc;
     if ((rc = from_cuda(cudaMemsetAsync(bb.dlogp, 0, bhkv * s.T * s.C * 4, st))) != DASH_OK) return rc;
     if ((rc = from_cuda(cudaMemsetAsync(dhc, 0, (size_t)s.Hkv * s.D * 4, st))) != DASH_OK) return rc;
+    // dk and dv are summed over the key-side kernel's slices
+    const size_t kv_bytes = (size_t)s.B * s.Hkv * s.T * s.D * 4;
+    if ((rc = from_cuda(cudaMemsetAsync(dk, 0, kv_bytes, st))) != DASH_OK) return rc;
+    if ((rc = from_cuda(cudaMemsetAsync(dv, 0, kv_bytes, st))) != DASH_OK) return rc;
     // The forward's routing (with p), then the backward kernels.
     if ((rc = from_cuda(launch_stage0(a, nullptr, 0, st))) != DASH_OK) return rc;
     if ((rc = from_cuda(launch_route(a, st))) != DASH_OK) return rc;
