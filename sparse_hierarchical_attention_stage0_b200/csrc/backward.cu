@@ -34,6 +34,7 @@ namespace {
 
 constexpr int kBwdWarps = 4;
 constexpr int kBwdSlice = 1024;        // k_bwd_kv entries per CTA
+constexpr int kListBlock = 2048;       // tokens per block of the routing transpose
 
 struct BwdArgs {
     StageArgs s;                 // shapes, q, k, v, head_cls, summary, tau, mask, p (routing)
@@ -47,6 +48,8 @@ struct BwdArgs {
     float *qbar;                 // [B,Hkv,T,D]
     int *list_cnt;               // [B*Hkv][C]
     long long *list_off;         // [B*Hkv][C + 1]
+    int *blk_cnt;                // [B*Hkv][C][nblk]: routed tokens per (chunk, token block)
+    long long *blk_off;          // [B*Hkv][C][nblk]
     int *list;                   // [B*Hkv][nnz_max]
     long long nnz_max;
     float *dsum;                 // [B,Hkv,Cf,D]
@@ -141,12 +144,12 @@ __global__ void __launch_bounds__(kBwdWarps * 32) k_bwd_q(BwdArgs ba, int TU, in
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long unit = (long long)blockIdx.x * kBwdWarps + warp;
     if (unit >= n_units) return;
+    // Per warp: a K and a V tile, and the routing biases of the current batch of chunks.
     const size_t tile_bytes = (size_t)kSub * D * 2;
-    const size_t warp_bytes = 2 * tile_bytes + (size_t)TU * D * 4 + (size_t)TU * 32 * 4;
+    const size_t warp_bytes = 2 * tile_bytes + (size_t)TU * 32 * 4;
     unsigned char *base = smem_raw + warp * warp_bytes;
     unsigned char *ks = base, *vs = base + tile_bytes;
-    float *qbar = reinterpret_cast<float *>(base + 2 * tile_bytes);
-    float *bias_s = qbar + TU * D;
+    float *bias_s = reinterpret_cast<float *>(base + 2 * tile_bytes);
 
     const int G = a.G, Gu = G >= 16 ? 16 : G;
     const int kunit = (int)(unit % UPT);
@@ -201,8 +204,6 @@ __global__ void __launch_bounds__(kBwdWarps * 32) k_bwd_q(BwdArgs ba, int TU, in
 #pragma unroll
                 for (int e = 0; e < 8; ++e) m[e] = 0.f;
             }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) qbar[u * D + d8 + e] = m[e];
             if (kunit == 0 && t < a.T)
 #pragma unroll
                 for (int e = 0; e < 8; ++e) ba.qbar[(bg * a.T + t) * D + d8 + e] = m[e];
@@ -268,17 +269,12 @@ __global__ void __launch_bounds__(kBwdWarps * 32) k_bwd_q(BwdArgs ba, int TU, in
             if (nb == 0) break;
             const int n_routed = batch_has_diag ? nb - 1 : nb;
             if (lane < n_routed) {
+                // bias = sigma log p of the token's routing (-inf where the token's p is 0:
+                // a chunk of the union the token itself did not route to)
                 for (int u = 0; u < TU; ++u) {
                     const int t = t0 + u;
-                    float b2 = -INFINITY;
-                    if (t < a.T) {
-                        const long long row = bg * a.T + t;
-                        const bool act = TU == 1 || ((a.mask[row * a.W + (my_c >> 6)] >> (my_c & 63)) & 1ull);
-                        if (act)
-                            b2 = routed_bias2<D>(qbar + u * D, a.summary + (bg * a.Cf + my_c) * D,
-                                                 a.tau[row], a.rc);
-                    }
-                    bias_s[u * 32 + lane] = b2;
+                    bias_s[u * 32 + lane] =
+                        t < a.T ? ba.sigma * log2f(a.p[(bg * a.T + t) * a.C + my_c]) : -INFINITY;
                 }
             }
             __syncwarp();
@@ -289,14 +285,9 @@ __global__ void __launch_bounds__(kBwdWarps * 32) k_bwd_q(BwdArgs ba, int TU, in
                 const bool diag = c == ct;
                 const int key0 = c * BC + sb * kSub;
                 load_sub<D>(ks, kp, key0, a.T);
+                if (pass == 1) load_sub<D>(vs, vp, key0, a.T);
                 cp_async_commit();
-                if (pass == 1) {
-                    load_sub<D>(vs, vp, key0, a.T);
-                    cp_async_commit();
-                    cp_async_wait<0>();
-                } else {
-                    cp_async_wait<0>();
-                }
+                cp_async_wait<0>();
                 __syncwarp();
                 float b_lo = 0.f, b_hi = 0.f;
                 if (!diag) {
@@ -419,20 +410,23 @@ __global__ void __launch_bounds__(kBwdWarps * 32) k_bwd_q(BwdArgs ba, int TU, in
 }
 
 // ---------------------------------------------------------------- k_bwd_lists
-// Per (b, g) and mask word w: the routed tokens of chunks 64 w .. 64 w + 63 (the diagonal bit
-// excluded), in token order.  mode 0 counts into list_cnt, mode 1 writes list entries at
-// list_off.  One warp per (b, g, w), 32 tokens per step.
-__global__ void k_bwd_lists(BwdArgs ba, int mode) {
+// Per (b, g), mask word w and block of kListBlock tokens: the block's routed tokens of chunks
+// 64 w .. 64 w + 63 (the diagonal bit excluded), in token order.  mode 0 counts them into
+// blk_cnt[(bg C + c) nblk + blk]; mode 1 writes them from blk_off (the same index).  One warp
+// per (b, g, w, block), 32 tokens per step; chunks of word w are routed to only by tokens from
+// 64 w Bc on, so earlier blocks have nothing to do.
+__global__ void k_bwd_lists(BwdArgs ba, int mode, int nblk) {
     const StageArgs &a = ba.s;
     const int lane = threadIdx.x & 31;
-    const int w = blockIdx.x, bgi = blockIdx.y;
+    const int w = blockIdx.x, bgi = blockIdx.y, blk = blockIdx.z;
     const long long bg = bgi;
     int run_lo = 0, run_hi = 0;                  // per chunk 64 w + lane and 64 w + 32 + lane
-    int c_lo = 64 * w + lane, c_hi = c_lo + 32;
-    for (int t0 = 64 * w * a.Bc; t0 < a.T; t0 += 32) {
+    const int c_lo = 64 * w + lane, c_hi = c_lo + 32;
+    const int t_begin = max(blk * kListBlock, 64 * w * a.Bc), t_end = min(a.T, (blk + 1) * kListBlock);
+    for (int t0 = t_begin; t0 < t_end; t0 += 32) {
         const int t = t0 + lane;
         uint64_t word = 0;
-        if (t < a.T) {
+        if (t < t_end) {
             word = a.mask[(bg * a.T + t) * a.W + w];
             const int ct = t / a.Bc;
             if (ct / 64 == w) word &= ~(1ull << (ct & 63));
@@ -446,7 +440,7 @@ __global__ void k_bwd_lists(BwdArgs ba, int mode) {
             const int run_c = bit < 32 ? __shfl_sync(kFull, run_lo, bit) : __shfl_sync(kFull, run_hi, bit - 32);
             if (mode == 1 && ((word >> bit) & 1ull)) {
                 const int before = run_c + __popc(bal & ((1u << lane) - 1u));
-                const long long pos = ba.list_off[bg * (a.C + 1) + c] + before;
+                const long long pos = ba.blk_off[(bg * a.C + c) * nblk + blk] + before;
                 if (pos >= 0 && pos < ba.nnz_max) ba.list[bg * ba.nnz_max + pos] = t;
                 else report(a.status, DASH_ERR_BOUNDS);
             }
@@ -456,28 +450,37 @@ __global__ void k_bwd_lists(BwdArgs ba, int mode) {
         }
     }
     if (mode == 0) {
-        if (c_lo < a.C) ba.list_cnt[bg * a.C + c_lo] = run_lo;
-        if (c_hi < a.C) ba.list_cnt[bg * a.C + c_hi] = run_hi;
+        if (c_lo < a.C) ba.blk_cnt[(bg * a.C + c_lo) * nblk + blk] = run_lo;
+        if (c_hi < a.C) ba.blk_cnt[(bg * a.C + c_hi) * nblk + blk] = run_hi;
     }
 }
 
-// Exclusive prefix sum of list_cnt per (b, g) into list_off (one warp per (b, g)).
-__global__ void k_bwd_scan(BwdArgs ba) {
+// Exclusive prefix sum per (b, g) over (chunk, block) in chunk-major order into blk_off, and
+// per chunk its count (list_cnt) and first offset (list_off).  One warp per (b, g).
+__global__ void k_bwd_scan(BwdArgs ba, int nblk) {
     const StageArgs &a = ba.s;
     const int lane = threadIdx.x & 31;
     const long long bg = blockIdx.x;
+    const long long n = (long long)a.C * nblk;
     long long base = 0;
-    for (int c0 = 0; c0 < a.C; c0 += 32) {
-        const int c = c0 + lane;
-        const int v = c < a.C ? ba.list_cnt[bg * a.C + c] : 0;
+    for (long long i0 = 0; i0 < n; i0 += 32) {
+        const long long i = i0 + lane;
+        const int v = i < n ? ba.blk_cnt[bg * n + i] : 0;
         int incl = v;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int x = __shfl_up_sync(kFull, incl, o);
             if (lane >= o) incl += x;
         }
-        if (c < a.C) ba.list_off[bg * (a.C + 1) + c] = base + incl - v;
+        if (i < n) ba.blk_off[bg * n + i] = base + incl - v;
         base += __shfl_sync(kFull, incl, 31);
+    }
+    __syncwarp();
+    for (int c = lane; c < a.C; c += 32) {
+        const long long first = ba.blk_off[bg * n + (long long)c * nblk];
+        const long long next = c + 1 < a.C ? ba.blk_off[bg * n + (long long)(c + 1) * nblk] : base;
+        ba.list_off[bg * (a.C + 1) + c] = first;
+        ba.list_cnt[bg * a.C + c] = (int)(next - first);
     }
     if (lane == 0) ba.list_off[bg * (a.C + 1) + a.C] = base;
 }
@@ -502,10 +505,11 @@ __global__ void __launch_bounds__(BC / 16 * 32) k_bwd_kv(BwdArgs ba, int UPT) {
     const int G = a.G, Gu = G >= 16 ? 16 : G;
     unsigned char *kt = smem_raw;                             // [BC][D] bf16
     unsigned char *vt = kt + (size_t)BC * D * 2;              // [BC][D]
-    unsigned char *qt = vt + (size_t)BC * D * 2;              // [16][D]
-    unsigned char *ot = qt + (size_t)16 * D * 2;              // [16][D] (dO)
-    float *st = reinterpret_cast<float *>(ot + (size_t)16 * D * 2);   // m[16], il[16], delta[16], bias
-    __shared__ float bias_sh;
+    // Two buffers per entry (the next entry's rows and statistics are copied while this one
+    // is computed): q rows [16][D], dO rows [16][D], and per row m, l, delta, then the bias p.
+    unsigned char *qt0 = vt + (size_t)BC * D * 2;
+    unsigned char *ot0 = qt0 + (size_t)2 * 16 * D * 2;
+    float *st0 = reinterpret_cast<float *>(ot0 + (size_t)2 * 16 * D * 2);   // [2][52]
     const __nv_bfloat16 *kp = reinterpret_cast<const __nv_bfloat16 *>(a.k) + bg * a.T * D;
     const __nv_bfloat16 *vp = reinterpret_cast<const __nv_bfloat16 *>(a.v) + bg * a.T * D;
     const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(a.q);
@@ -524,8 +528,6 @@ __global__ void __launch_bounds__(BC / 16 * 32) k_bwd_kv(BwdArgs ba, int UPT) {
         cp_async16(vt + swz<D>(row, ch), vp + (long long)(ok ? key : 0) * D + ch * 8, ok ? 16 : 0);
     }
     cp_async_commit();
-    cp_async_wait<0>();
-    __syncthreads();
     float dka[D / 8][4], dva[D / 8][4];
 #pragma unroll
     for (int j = 0; j < D / 8; ++j)
@@ -534,44 +536,59 @@ __global__ void __launch_bounds__(BC / 16 * 32) k_bwd_kv(BwdArgs ba, int UPT) {
     const int r_lo = lane >> 2, qd = lane & 3;                // key rows r_lo, r_lo + 8 of the warp
     const int key_lo = c * BC + 16 * warp + r_lo, key_hi = key_lo + 8;
 
-    for (long long e = e_begin; e < e_end; ++e) {
+    // Entry e: token t (the chunk's own tokens first, then its routed ones) and head group.
+    struct Ent { int t, kunit; bool diag, valid; };
+    auto entry = [&](long long e) -> Ent {
+        Ent en;
         const long long ti = e / UPT;
-        const int kunit = (int)(e % UPT);
-        const bool diag = ti < n_diag;
-        const int t = diag ? c * BC + (int)ti : ba.list[bg * ba.nnz_max + off + (ti - n_diag)];
-        if (t < 0 || t >= a.T) {                             // same entry in every thread
-            if (tid == 0) report(a.status, DASH_ERR_BOUNDS);
-            continue;
-        }
-        __syncthreads();                                     // the previous entry's tiles are read
-        // rows r < Gu of the entry: heads g G + kunit 16 + r of token t
-        for (int i = tid; i < 16 * CH; i += NW * 32) {
-            const int r = i / CH, ch = i % CH;
-            const bool ok = r < Gu;
-            const long long row = ((long long)b * a.Hq + g * G + kunit * 16 + (ok ? r : 0)) * a.T + t;
-            cp_async16(qt + swz<D>(r, ch), q + row * D + ch * 8, ok ? 16 : 0);
-            cp_async16(ot + swz<D>(r, ch), ba.dout + row * D + ch * 8, ok ? 16 : 0);
+        en.kunit = (int)(e % UPT);
+        en.diag = ti < n_diag;
+        en.t = en.diag ? c * BC + (int)ti : ba.list[bg * ba.nnz_max + off + (ti - n_diag)];
+        en.valid = en.t >= 0 && en.t < a.T;
+        return en;
+    };
+    // Copies of an entry's rows and statistics into buffer buf; every thread commits one group.
+    auto prefetch = [&](const Ent &en, int buf) {
+        if (en.valid) {
+            unsigned char *qt = qt0 + (size_t)buf * 16 * D * 2, *ot = ot0 + (size_t)buf * 16 * D * 2;
+            float *st = st0 + buf * 52;
+            for (int i = tid; i < 16 * CH; i += NW * 32) {
+                const int r = i / CH, ch = i % CH;
+                const bool ok = r < Gu;
+                const long long row = ((long long)b * a.Hq + g * G + en.kunit * 16 + (ok ? r : 0)) * a.T + en.t;
+                cp_async16(qt + swz<D>(r, ch), q + row * D + ch * 8, ok ? 16 : 0);
+                cp_async16(ot + swz<D>(r, ch), ba.dout + row * D + ch * 8, ok ? 16 : 0);
+            }
+            if (tid < Gu) {
+                const long long row = ((long long)b * a.Hq + g * G + en.kunit * 16 + tid) * a.T + en.t;
+                cp_async4(st + tid, ba.row_m + row);
+                cp_async4(st + 16 + tid, ba.row_l + row);
+                cp_async4(st + 32 + tid, ba.row_delta + row);
+            }
+            // the routing bias of a routed entry is sigma log p (p > 0 on the routed chunks)
+            if (tid == 0 && !en.diag) cp_async4(st + 48, a.p + (bg * a.T + en.t) * a.C + c);
         }
         cp_async_commit();
-        if (tid < 16) {
-            const bool ok = tid < Gu;
-            const long long row = ((long long)b * a.Hq + g * G + kunit * 16 + (ok ? tid : 0)) * a.T + t;
-            st[tid] = ok ? ba.row_m[row] : 0.f;
-            const float l = ok ? ba.row_l[row] : 0.f;
-            st[16 + tid] = l > 0.f ? 1.f / l : 0.f;
-            st[32 + tid] = ok ? ba.row_delta[row] : 0.f;
-        }
-        if (warp == 0) {
-            float b2 = 0.f;
-            if (!diag && lane == 0) {
-                const long long row = bg * a.T + t;
-                b2 = routed_bias2<D>(ba.qbar + row * D, a.summary + (bg * a.Cf + c) * D, a.tau[row], a.rc);
-            }
-            if (lane == 0) bias_sh = b2;
-        }
-        cp_async_wait<0>();
+    };
+    Ent cur = entry(e_begin);
+    prefetch(cur, 0);
+    for (long long e = e_begin; e < e_end; ++e) {
+        const int buf = (int)((e - e_begin) & 1);
+        const Ent nxt = e + 1 < e_end ? entry(e + 1) : Ent{0, 0, false, false};
+        __syncthreads();                                     // entry e-1's buffer is read
+        prefetch(nxt, buf ^ 1);
+        cp_async_wait<1>();                                  // entry e's copies (and K, V)
         __syncthreads();
-        const float b2 = bias_sh;
+        if (!cur.valid) {                                    // same entry in every thread
+            if (tid == 0) report(a.status, DASH_ERR_BOUNDS);
+            cur = nxt;
+            continue;
+        }
+        const int t = cur.t;
+        const bool diag = cur.diag;
+        const unsigned char *qt = qt0 + (size_t)buf * 16 * D * 2, *ot = ot0 + (size_t)buf * 16 * D * 2;
+        const float *st = st0 + buf * 52;
+        const float b2 = diag ? 0.f : ba.sigma * log2f(st[48]);
         // S^T (16 keys x 16 rows) in log2 units, P^T, dP^T, dS^T
         float sa[2][4], dpa[2][4];
         {
@@ -591,7 +608,8 @@ __global__ void __launch_bounds__(BC / 16 * 32) k_bwd_kv(BwdArgs ba, int UPT) {
                 const int key = e2 >= 2 ? key_hi : key_lo;
                 float x = fmaf(sa[j][e2], a.qk_scale2, b2);
                 if ((diag && key > t) || key >= a.T || r >= Gu) x = -INFINITY;
-                const float p = x == -INFINITY ? 0.f : exp2f(x - st[r]) * st[16 + r];
+                const float l = st[16 + r];
+                const float p = x == -INFINITY ? 0.f : exp2f(x - st[r]) * (l > 0.f ? 1.f / l : 0.f);
                 pv[j][e2] = p;
                 dsv[j][e2] = p * (dpa[j][e2] - st[32 + r]);
             }
@@ -606,6 +624,7 @@ __global__ void __launch_bounds__(BC / 16 * 32) k_bwd_kv(BwdArgs ba, int UPT) {
         dsa[3] = pack_bf16x2(dsv[1][2], dsv[1][3]);
         mm_acc_kd<D>(dva, pa, ot);
         mm_acc_kd<D>(dka, dsa, qt);
+        cur = nxt;
     }
     const float rs = a.qk_scale2 * 0.69314718055994531f;
 #pragma unroll
@@ -794,7 +813,7 @@ cudaError_t launch_bwd_t(BwdArgs ba, cudaStream_t st) {
     {
         const long long NTG = (a.T + TU - 1) / TU;
         const long long n_units = NTG * a.B * a.Hkv * UPT;
-        const size_t warp_bytes = 2 * (size_t)kSub * D * 2 + (size_t)TU * D * 4 + (size_t)TU * 32 * 4;
+        const size_t warp_bytes = 2 * (size_t)kSub * D * 2 + (size_t)TU * 32 * 4;
         const size_t smem = warp_bytes * kBwdWarps;
         auto kern = k_bwd_q<D, BC>;
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
@@ -803,15 +822,16 @@ cudaError_t launch_bwd_t(BwdArgs ba, cudaStream_t st) {
     }
     // 2. the routing transposed
     {
-        dim3 grid((unsigned)a.W, (unsigned)(a.B * a.Hkv));
-        k_bwd_lists<<<grid, 32, 0, st>>>(ba, 0);
-        k_bwd_scan<<<(unsigned)(a.B * a.Hkv), 32, 0, st>>>(ba);
-        k_bwd_lists<<<grid, 32, 0, st>>>(ba, 1);
+        const int nblk = backward_list_blocks(a.T);
+        dim3 grid((unsigned)a.W, (unsigned)(a.B * a.Hkv), (unsigned)nblk);
+        k_bwd_lists<<<grid, 32, 0, st>>>(ba, 0, nblk);
+        k_bwd_scan<<<(unsigned)(a.B * a.Hkv), 32, 0, st>>>(ba, nblk);
+        k_bwd_lists<<<grid, 32, 0, st>>>(ba, 1, nblk);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     // 3. key side
     {
-        const size_t smem = 2 * (size_t)BC * D * 2 + 2 * (size_t)16 * D * 2 + 48 * 4;
+        const size_t smem = 2 * (size_t)BC * D * 2 + 4 * (size_t)16 * D * 2 + 2 * 52 * 4;
         auto kern = k_bwd_kv<D, BC>;
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
         // slices: enough for the longest possible list (chunk 0: every token of the sequence)
@@ -835,6 +855,8 @@ cudaError_t launch_bwd_t(BwdArgs ba, cudaStream_t st) {
 
 }  // namespace
 
+int backward_list_blocks(int T) { return (T + kListBlock - 1) / kListBlock; }
+
 long long backward_nnz_max(int T, int Bc) {
     // routed (token, chunk) pairs of one (b, g) at most: sum over t of floor(t / Bc)
     const long long Cf = T / Bc;
@@ -857,6 +879,8 @@ cudaError_t launch_backward(const StageArgs &s, const BackwardBuffers &bb, cudaS
     ba.qbar = bb.qbar;
     ba.list_cnt = bb.list_cnt;
     ba.list_off = bb.list_off;
+    ba.blk_cnt = bb.blk_cnt;
+    ba.blk_off = bb.blk_off;
     ba.list = bb.list;
     ba.nnz_max = backward_nnz_max(s.T, s.Bc);
     ba.dsum = bb.dsum;

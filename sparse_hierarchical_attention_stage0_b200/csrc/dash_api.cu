@@ -633,6 +633,8 @@ size_t dash_backward_workspace_size(const dash_params_t *p) {
     n += 3 * align256((size_t)s.B * s.Hq * s.T * 4);             // row max, sum, delta
     n += align256(bhkv * s.T * s.D * 4);                         // qbar
     n += align256(bhkv * s.C * 4) + align256(bhkv * (s.C + 1) * 8);   // list counts, offsets
+    const size_t nblk = (size_t)backward_list_blocks(s.T);
+    n += align256(bhkv * s.C * nblk * 4) + align256(bhkv * s.C * nblk * 8);   // per token block
     n += align256(bhkv * (size_t)backward_nnz_max(s.T, s.Bc) * 4);     // lists
     n += align256(bytes_summary(s));                             // d summaries
     return n;
@@ -684,6 +686,9 @@ dash_status_t dash_backward(const dash_params_t *p, const void *q, const void *k
     bb.qbar = reinterpret_cast<float *>(take(bhkv * s.T * s.D * 4));
     bb.list_cnt = reinterpret_cast<int *>(take(bhkv * s.C * 4));
     bb.list_off = reinterpret_cast<long long *>(take(bhkv * (s.C + 1) * 8));
+    const size_t nblk = (size_t)backward_list_blocks(s.T);
+    bb.blk_cnt = reinterpret_cast<int *>(take(bhkv * s.C * nblk * 4));
+    bb.blk_off = reinterpret_cast<long long *>(take(bhkv * s.C * nblk * 8));
     bb.list = reinterpret_cast<int *>(take(bhkv * (size_t)backward_nnz_max(s.T, s.Bc) * 4));
     bb.dsum = reinterpret_cast<float *>(take((size_t)s.B * s.Hkv * s.Cf * s.D * 4));
     bb.sigma = p->sigma;

@@ -70,6 +70,11 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem, int src
                  "l"(gmem), "r"(src_bytes)
                  : "memory");
 }
+// 4-byte cp.async (through L1), for scattered scalars.
+__device__ __forceinline__ void cp_async4(void *smem, const void *gmem) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(smem_u32(smem)), "l"(gmem)
+                 : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() {
     asm volatile("cp.async.commit_group;\n" ::: "memory");
 }

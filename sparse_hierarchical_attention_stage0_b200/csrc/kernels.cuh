@@ -118,11 +118,14 @@ struct BackwardBuffers {
     float *qbar;              // [B,Hkv,T,D]
     int *list_cnt;            // [B*Hkv][C]
     long long *list_off;      // [B*Hkv][C+1]
+    int *blk_cnt;             // [B*Hkv][C][backward_list_blocks(T)]
+    long long *blk_off;       // [B*Hkv][C][backward_list_blocks(T)]
     int *list;                // [B*Hkv][backward_nnz_max]
     float *dsum;              // [B,Hkv,Cf,D]
     float sigma;
 };
 long long backward_nnz_max(int T, int Bc);
+int backward_list_blocks(int T);            // token blocks of the routing transpose
 cudaError_t launch_backward(const StageArgs &s, const BackwardBuffers &bb, cudaStream_t st);
 int decode_supported(int G, int Ccap, int D);
 // Scratch bytes dash_prefill needs in its workspace (status word, tau, and the summaries /
