@@ -585,9 +585,9 @@ struct RowInRegisters {
 // on the kind of alpha (0 softmax, 1 alpha = 1.5, 2 alpha = 2, 3 any other alpha).  For
 // alpha = 1 returns the log-sum-exp of the scores.  Otherwise x are the scaled scores
 // (alpha-1) s and the return value is tau with sum_c [x_c - tau]_+^beta = 1.  For beta >= 1
-// (alpha <= 2) Newton's method from tau0 = max x - 1 increases monotonically to the root (f
-// is convex and decreasing); the support it settles on is then fed to the exact closed form
-// for alpha = 1.5 and 2.  For alpha > 2, bisection on [max - 1, max - n^(1-alpha)].  The
+// (alpha <= 2) Newton's method on f^(1/beta) = 1 from tau0 = max x - 1 increases
+// monotonically to the root (the function is convex and decreasing); the support it settles
+// on is then fed to the exact closed form for alpha = 1.5 and 2.  For alpha > 2, bisection on [max - 1, max - n^(1-alpha)].  The
 // fixed lane-strided sums and butterfly reductions give every caller the same bits.
 template <int KIND, typename Row>
 __device__ __forceinline__ float entmax_tau_row(const Row &row, int n, const RouteConsts &rc,
@@ -618,7 +618,13 @@ __device__ __forceinline__ float entmax_tau_row(const Row &row, int n, const Rou
                 f, df);
             f = warp_sum(f);
             df = warp_sum(df);
-            const float step = (f - 1.f) / (beta * df);
+            // Newton on f^(1/beta) = 1, which is nearly linear in tau (a beta-norm of the
+            // margins), so far fewer steps than on f = 1 when the support is large; it is
+            // convex and decreasing too, so the steps still rise monotonically to the root.
+            // Step = (f - f^(1 - 1/beta)) / sum m^(beta-1).
+            const float step = KIND == 2 ? (f - 1.f) / df
+                             : KIND == 1 ? (f - sqrtf(f)) / df
+                                         : (f - powf(f, 1.f - 1.f / beta)) / df;
             if (!(step > 0.f)) break;                 // at (or rounded past) the root
             const float nt = tau + step;
             if (nt == tau) break;
