@@ -376,12 +376,16 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
     // Lane l lists its chunks l, l + 32, ... of each block of 1024, the lanes in order.
     if (warp == 0) {
         int pos = 0;
+        const int kind = a.rc.kind;
+        const float tv = tau;
         for (int c0 = 0; c0 < n; c0 += 32 * 32) {
             uint32_t bits = 0;
 #pragma unroll
             for (int k = 0; k < 32; ++k) {
                 const int c = c0 + lane + 32 * k;
-                if (active(c) && dash_check(c < a.Cf && (c + 1) * BC <= a.cap, a.status)) bits |= 1u << k;
+                const bool act = c < n && (kind == kKindTopk ? ((sel[c >> 5] >> (c & 31)) & 1u) != 0
+                                                             : (kind == 0 || __fsub_rn(xs[c], tv) > 0.f));
+                if (act && dash_check(c < a.Cf && (c + 1) * BC <= a.cap, a.status)) bits |= 1u << k;
             }
             const int cnt = __popc(bits);
             int incl = cnt;
