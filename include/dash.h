@@ -171,13 +171,15 @@ dash_status_t dash_prefill(const dash_params_t *params, const void *q, const voi
  *            these parameters the call runs as one slice.
  *   stream:  computation; h2d_stream, d2h_stream: the two copy directions.  All three must
  *            be distinct streams of the current device.  Both copy streams first wait for
- *            the work already queued on stream.  Order: head_cls, k and v to the device,
- *            then q slice by slice on h2d_stream; Stage 0, then Stages 1-2 of
- *            each slice once its q has arrived, on stream; out of each slice back to
- *            out_host on d2h_stream once computed.  stream finally waits for the last copy,
- *            so synchronising stream covers the whole call.
+ *            the work already queued on stream.  Order on h2d_stream: head_cls, then per
+ *            slice its q rows, preceded where one starts by a piece of k and v rows (pieces
+ *            of 1, 2, 4, ... slices: rows below t route and attend only to keys below t).
+ *            On stream: per piece of keys, Stage 0 on the chunks it completes and the V^T
+ *            transpose of its rows; Stages 1-2 of each slice once its q has arrived.  Out of
+ *            each slice back to out_host on d2h_stream once computed.  stream finally waits
+ *            for the last copy, so synchronising stream covers the whole call.
  * The device output equals dash_prefill's bit for bit.  Creates and destroys its CUDA events
- * (2 * slices + 3) within the call.  Returns DASH_OK when every copy and launch was issued,
+ * (3 * slices + 2) within the call.  Returns DASH_OK when every copy and launch was issued,
  * DASH_ERR_INVALID_ARGUMENT for a NULL buffer or n_slices < 1. */
 dash_status_t dash_prefill_host(const dash_params_t *params, const void *q_host,
                                 const void *k_host, const void *v_host,

@@ -706,7 +706,8 @@ static cudaError_t launch_fa_t(const StageArgs &a, cudaStream_t st) {
     static EncodeFn enc = fa_encode();
     if (!enc || !a.vt) return cudaErrorNotSupported;
     const int BHkv = a.B * a.Hkv;
-    cudaError_t e = a.vt_ready ? cudaSuccess : launch_vtranspose(a.v, a.vt, BHkv, a.T, 128, st);
+    cudaError_t e = a.vt_ready ? cudaSuccess
+                               : launch_vtranspose(a.v, a.vt, BHkv, a.T, 128, st, a.vt_begin, a.vt_end);
     if (e != cudaSuccess) return e;
     CUtensorMap mk, mk128, mvt;
     if (!fa_map(enc, &mk, a.k, a.T, BHkv, 64) || !fa_map(enc, &mk128, a.k, a.T, BHkv, 128))

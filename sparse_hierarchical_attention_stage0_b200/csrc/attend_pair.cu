@@ -686,7 +686,8 @@ cudaError_t launch_pair_t(const StageArgs &a, cudaStream_t st) {
     static EncodeFn enc = pr_encode();
     if (!enc || !a.vt) return cudaErrorNotSupported;
     const int BHkv = a.B * a.Hkv;
-    cudaError_t e = a.vt_ready ? cudaSuccess : launch_vtranspose(a.v, a.vt, BHkv, a.T, 128, st);
+    cudaError_t e = a.vt_ready ? cudaSuccess
+                               : launch_vtranspose(a.v, a.vt, BHkv, a.T, 128, st, a.vt_begin, a.vt_end);
     if (e != cudaSuccess) return e;
     // K [B*Hkv][T][128]: box (64 dims, 64 keys).  V^T [B*Hkv][128][T8]: box (64 keys, 72 or
     // 56 dims) for the even and the odd CTA.

@@ -321,6 +321,14 @@ dash_status_t dash_prefill(const dash_params_t *p, const void *q, const void *k,
     return from_cuda(launch_attend(a, st));
 }
 
+// Keys go up in pieces that double in slices: slice 0, slices 1-2, slices 3-6, ... (a piece
+// starts at slice 2^j - 1). The first slice's computation starts after a small copy, and the
+// number of copies and of Stage 0 / transpose launches stays logarithmic in the slices.
+// Returns the slice after the piece that starts at slice i, or 0 when no piece starts there.
+static int kv_piece_end(int i, int n) {
+    return ((i + 1) & i) == 0 ? std::min(n, 2 * i + 1) : 0;
+}
+
 dash_status_t dash_prefill_host(const dash_params_t *p, const void *q_host, const void *k_host,
                                 const void *v_host, const float *head_cls_host, void *out_host,
                                 void *q, void *k, void *v, float *head_cls, void *out, void *ws,
@@ -373,19 +381,30 @@ dash_status_t dash_prefill_host(const dash_params_t *p, const void *q_host, cons
     cudaStream_t ds = static_cast<cudaStream_t>(d2h_stream);
     const size_t row_bytes = (size_t)s.D * 2;
     const size_t plane = (size_t)s.T * row_bytes;          // one (b, h) plane of q or out
-    const size_t kv_bytes = (size_t)s.B * s.Hkv * plane;
-    const int n_ev = 2 * n + 3;
-    cudaEvent_t ev[2 * kMaxSlices + 3];
+    const int n_ev = 3 * n + 2;
+    cudaEvent_t ev[3 * kMaxSlices + 2];
     int made = 0;
     cudaError_t e = cudaSuccess;
     for (; made < n_ev && e == cudaSuccess; ++made) e = cudaEventCreateWithFlags(&ev[made], cudaEventDisableTiming);
     if (e != cudaSuccess) --made;
-    cudaEvent_t &e_kv = ev[0], &e_done = ev[1], &e_start = ev[2];
-    auto e_q = [&](int i) -> cudaEvent_t & { return ev[3 + i]; };
-    auto e_o = [&](int i) -> cudaEvent_t & { return ev[3 + n + i]; };
+    cudaEvent_t &e_done = ev[0], &e_start = ev[1];
+    auto e_kv = [&](int i) -> cudaEvent_t & { return ev[2 + i]; };
+    auto e_q = [&](int i) -> cudaEvent_t & { return ev[2 + n + i]; };
+    auto e_o = [&](int i) -> cudaEvent_t & { return ev[2 + 2 * n + i]; };
     auto ok = [&](cudaError_t r) { if (e == cudaSuccess) e = r; return e == cudaSuccess; };
-    // Host -> device: head_cls, K and V (Stage 0 and every slice need all keys), then q slice
-    // by slice.  Compute: Stage 0, then Stages 1-2 of slice i once its q has landed.
+    // Rows [t0, t1) of every (b, h) plane of a [B, H, T, D] tensor in one strided copy.
+    auto rows_copy = [&](void *dst, const void *src, int planes, size_t t0, size_t t1,
+                         cudaMemcpyKind kind, cudaStream_t cs) {
+        return cudaMemcpy2DAsync(static_cast<unsigned char *>(dst) + t0 * row_bytes, plane,
+                                 static_cast<const unsigned char *>(src) + t0 * row_bytes, plane,
+                                 (t1 - t0) * row_bytes, (size_t)planes, kind, cs);
+    };
+    // Causal attention and routing of the rows below t1 read only keys below t1 and the
+    // summaries of the chunks that end at or before t1. So slice i uploads its own rows of
+    // K, V and q; the compute stream summarises the chunks completed by the new keys,
+    // transposes the new rows of V, then routes and attends the slice.
+    // Host -> device: head_cls, then per slice K, V rows and q rows.
+    // Compute: per slice Stage 0 on the new chunks once K has landed, Stages 1-2 once q has.
     // Device -> host: out of slice i once it is computed.
     if (e == cudaSuccess) {
         // Both copy streams start after the work already queued on the compute stream (which
@@ -394,35 +413,44 @@ dash_status_t dash_prefill_host(const dash_params_t *p, const void *q_host, cons
         ok(cudaStreamWaitEvent(hs, e_start, 0));
         ok(cudaStreamWaitEvent(ds, e_start, 0));
         if (!dense) ok(cudaMemcpyAsync(head_cls, head_cls_host, (size_t)s.Hkv * s.D * 4, cudaMemcpyHostToDevice, hs));
-        ok(cudaMemcpyAsync(k, k_host, kv_bytes, cudaMemcpyHostToDevice, hs));
-        ok(cudaMemcpyAsync(v, v_host, kv_bytes, cudaMemcpyHostToDevice, hs));
-        ok(cudaEventRecord(e_kv, hs));
         for (int i = 0; i < n; ++i) {
-            const size_t t0 = (size_t)i * rows, tr = (size_t)std::min(s.T, (i + 1) * rows) - t0;
-            ok(cudaMemcpy2DAsync(static_cast<unsigned char *>(q) + t0 * row_bytes, plane,
-                                 static_cast<const unsigned char *>(q_host) + t0 * row_bytes, plane,
-                                 tr * row_bytes, (size_t)s.B * s.Hq, cudaMemcpyHostToDevice, hs));
+            const size_t t0 = (size_t)i * rows, t1 = (size_t)std::min(s.T, (i + 1) * rows);
+            if (const int pe = kv_piece_end(i, n)) {
+                const size_t k1 = (size_t)std::min(s.T, pe * rows);
+                ok(rows_copy(k, k_host, s.B * s.Hkv, t0, k1, cudaMemcpyHostToDevice, hs));
+                ok(rows_copy(v, v_host, s.B * s.Hkv, t0, k1, cudaMemcpyHostToDevice, hs));
+                ok(cudaEventRecord(e_kv(i), hs));
+            }
+            ok(rows_copy(q, q_host, s.B * s.Hq, t0, t1, cudaMemcpyHostToDevice, hs));
             ok(cudaEventRecord(e_q(i), hs));
         }
         ok(cudaMemsetAsync(ws, 0, sizeof(uint32_t), st));
-        ok(cudaStreamWaitEvent(st, e_kv, 0));
-        if (!dense) ok(launch_stage0(a, nullptr, 0, st));
         for (int i = 0; i < n && e == cudaSuccess; ++i) {
             a.t_begin = i * rows;
             a.t_end = std::min(s.T, (i + 1) * rows);
-            a.vt_ready = i > 0;
             a.fuse_route = !dense && attend_kernel(a) == AttendKernel::kFa && attend_fa_fuse_supported(a);
+            a.vt_ready = 1;
+            if (const int pe = kv_piece_end(i, n)) {
+                // A new piece of keys: summarise the chunks it completes, transpose its V rows
+                // (one piece: every chunk and every key, ranges 0 meaning "all").
+                const int k1 = std::min(s.T, pe * rows);
+                a.s0_begin = n > 1 ? a.t_begin / s.Bc : 0;
+                a.s0_end = n > 1 ? k1 / s.Bc : 0;
+                a.vt_begin = n > 1 ? a.t_begin : 0;
+                a.vt_end = n > 1 ? k1 : 0;
+                a.vt_ready = 0;
+                ok(cudaStreamWaitEvent(st, e_kv(i), 0));
+                if (!dense && (n == 1 || a.s0_end > a.s0_begin)) ok(launch_stage0(a, nullptr, 0, st));
+            }
             ok(cudaStreamWaitEvent(st, e_q(i), 0));
             if (!dense && !a.fuse_route) ok(launch_route(a, st));
             ok(launch_attend(a, st));
             ok(cudaEventRecord(e_o(i), st));
         }
         for (int i = 0; i < n && e == cudaSuccess; ++i) {
-            const size_t t0 = (size_t)i * rows, tr = (size_t)std::min(s.T, (i + 1) * rows) - t0;
             ok(cudaStreamWaitEvent(ds, e_o(i), 0));
-            ok(cudaMemcpy2DAsync(static_cast<unsigned char *>(out_host) + t0 * row_bytes, plane,
-                                 static_cast<const unsigned char *>(out) + t0 * row_bytes, plane,
-                                 tr * row_bytes, (size_t)s.B * s.Hq, cudaMemcpyDeviceToHost, ds));
+            ok(rows_copy(out_host, out, s.B * s.Hq, (size_t)i * rows, (size_t)std::min(s.T, (i + 1) * rows),
+                         cudaMemcpyDeviceToHost, ds));
         }
         // The compute stream ends after the last copy back, so synchronising it covers the call.
         ok(cudaEventRecord(e_done, ds));

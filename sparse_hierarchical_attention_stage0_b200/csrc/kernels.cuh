@@ -26,7 +26,9 @@ struct StageArgs {
     int ignore_routing;       // DENSE or FORCE_ALL_ACTIVE: attend every chunk, bias 0
     int t_begin, t_end;       // Stages 1-2 compute rows [t_begin, t_end) (t_begin % 128 == 0);
                               // T stays the row stride of q, tau, mask, p and out
-    int vt_ready;             // V^T scratch already holds the transpose of V (a later row slice)
+    int vt_ready;             // V^T scratch already holds the keys this call reads
+    int vt_begin, vt_end;     // keys [vt_begin, vt_end) to transpose when !vt_ready (vt_end 0: all)
+    int s0_begin, s0_end;     // Stage 0 over chunks [s0_begin, s0_end) (s0_end 0: every chunk)
     int test_stall;           // test hook: Stage 0's chunk-copy wait runs out (DASH_FLAG_TEST_STALL_WAIT)
     int fuse_route;           // Stage 2 computes the routing itself (fused route-and-attend)
     // Run-time choice between the 128-key-block and the warp-MMA Stage 2 kernels (null: none):
@@ -103,7 +105,10 @@ size_t attend_fa_vt_bytes(int B, int Hkv, int T, int D);
 cudaError_t launch_attend_fa(const StageArgs &a, cudaStream_t st);
 bool attend_pair_supported(const StageArgs &a);
 cudaError_t launch_attend_pair(const StageArgs &a, cudaStream_t st);
-cudaError_t launch_vtranspose(const void *v, void *vt, int BHkv, int T, int D, cudaStream_t st);
+// Keys [k_begin, k_end) of V (k_begin a multiple of 64; k_end 0: all), the zero padding to T8
+// included when the range reaches T.
+cudaError_t launch_vtranspose(const void *v, void *vt, int BHkv, int T, int D, cudaStream_t st,
+                              int k_begin = 0, int k_end = 0);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
 
 // Buffers of the backward pass (dash_backward); the StageArgs carry the forward's routing

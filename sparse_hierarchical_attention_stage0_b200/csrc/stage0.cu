@@ -11,6 +11,8 @@
 //   summary = sum_j exp(l_j - max) k_j / sum_j exp(l_j - max)
 // with each lane owning D/32 output dims (16-byte coalesced stores for D = 128).
 // HBM-bound: it reads Bc*D*2 bytes and writes D*4 bytes per chunk.
+#include <algorithm>
+
 #include "dash_common.cuh"
 #include "kernels.cuh"
 
@@ -26,17 +28,17 @@ __global__ void __launch_bounds__(kStage0Warps * 32)
 k_stage0(const __nv_bfloat16 *__restrict__ k, const float *__restrict__ head_cls,
          float *__restrict__ summary, int B, int Hkv, int T, int Cf, const int32_t *seq_lens,
          int n_recent, uint32_t *status, int test_stall, const int32_t *block_table,
-         int max_blocks, int n_pages) {
+         int max_blocks, int n_pages, int c_begin, int nc) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t bars[kStage0Warps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long unit = (long long)blockIdx.x * kStage0Warps + warp;
     int b, g, c;
-    if (seq_lens == nullptr) {
-        if (unit >= (long long)B * Hkv * Cf) return;
-        c = (int)(unit % Cf);
-        g = (int)((unit / Cf) % Hkv);
-        b = (int)(unit / ((long long)Cf * Hkv));
+    if (seq_lens == nullptr) {                    // chunks [c_begin, c_begin + nc) of every (b, g)
+        if (unit >= (long long)B * Hkv * nc) return;
+        c = c_begin + (int)(unit % nc);
+        g = (int)((unit / nc) % Hkv);
+        b = (int)(unit / ((long long)nc * Hkv));
     } else {
         if (unit >= (long long)B * Hkv * n_recent) return;
         int r = (int)(unit % n_recent);
@@ -87,8 +89,11 @@ template <int D, int BC>
 static cudaError_t launch_stage0_t(const StageArgs &a, const int32_t *seq_lens, int n_recent,
                                    cudaStream_t st, const int32_t *block_table = nullptr,
                                    int max_blocks = 0, int n_pages = 0) {
+    const int c_begin = seq_lens || a.s0_end <= 0 ? 0 : a.s0_begin;
+    const int nc = seq_lens ? 0 : (a.s0_end <= 0 ? a.Cf : std::min(a.s0_end, a.Cf) - c_begin);
+    if (!seq_lens && nc <= 0) return cudaSuccess;
     long long units = seq_lens ? (long long)a.B * a.Hkv * n_recent
-                               : (long long)a.B * a.Hkv * a.Cf;
+                               : (long long)a.B * a.Hkv * nc;
     if (units == 0) return cudaSuccess;
     size_t smem = (size_t)kStage0Warps * BC * D * sizeof(__nv_bfloat16);
     auto kern = k_stage0<D, BC>;
@@ -98,7 +103,7 @@ static cudaError_t launch_stage0_t(const StageArgs &a, const int32_t *seq_lens, 
     unsigned grid = (unsigned)((units + kStage0Warps - 1) / kStage0Warps);
     kern<<<grid, kStage0Warps * 32, smem, st>>>(
         reinterpret_cast<const __nv_bfloat16 *>(a.k), a.head_cls, a.summary, a.B, a.Hkv, a.T,
-        a.Cf, seq_lens, n_recent, a.status, a.test_stall, block_table, max_blocks, n_pages);
+        a.Cf, seq_lens, n_recent, a.status, a.test_stall, block_table, max_blocks, n_pages, c_begin, nc);
     return cudaGetLastError();
 }
 

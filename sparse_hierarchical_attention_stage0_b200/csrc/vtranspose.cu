@@ -13,9 +13,10 @@ constexpr int kTrTile = 64;
 
 template <int D>
 __global__ void __launch_bounds__(256) k_vtranspose(const __nv_bfloat16 *__restrict__ v,
-                                                    __nv_bfloat16 *__restrict__ vt, int T, int T8) {
+                                                    __nv_bfloat16 *__restrict__ vt, int T, int T8,
+                                                    int t_base) {
     __shared__ __nv_bfloat16 tile[kTrTile][kTrTile + 2];
-    const int bg = blockIdx.z, t0 = blockIdx.x * kTrTile, d0 = blockIdx.y * kTrTile;
+    const int bg = blockIdx.z, t0 = t_base + blockIdx.x * kTrTile, d0 = blockIdx.y * kTrTile;
     const __nv_bfloat16 *src = v + (long long)bg * T * D;
     __nv_bfloat16 *dst = vt + (long long)bg * D * T8;
     for (int i = threadIdx.x; i < kTrTile * kTrTile; i += 256) {
@@ -31,15 +32,18 @@ __global__ void __launch_bounds__(256) k_vtranspose(const __nv_bfloat16 *__restr
     }
 }
 
-cudaError_t launch_vtranspose(const void *v, void *vt, int BHkv, int T, int D, cudaStream_t st) {
+cudaError_t launch_vtranspose(const void *v, void *vt, int BHkv, int T, int D, cudaStream_t st,
+                              int k_begin, int k_end) {
     const int T8 = (T + 7) & ~7;
-    dim3 grid((T8 + kTrTile - 1) / kTrTile, D / kTrTile, BHkv);
+    if (k_end <= 0 || k_end >= T) k_end = T8;            // the range reaching T covers the padding
+    if (k_begin < 0 || (k_begin % kTrTile) != 0 || k_begin >= k_end) return cudaErrorInvalidValue;
+    dim3 grid((k_end - k_begin + kTrTile - 1) / kTrTile, D / kTrTile, BHkv);
     if (D == 128)
         k_vtranspose<128><<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(v),
-                                                reinterpret_cast<__nv_bfloat16 *>(vt), T, T8);
+                                                reinterpret_cast<__nv_bfloat16 *>(vt), T, T8, k_begin);
     else if (D == 64)
         k_vtranspose<64><<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(v),
-                                               reinterpret_cast<__nv_bfloat16 *>(vt), T, T8);
+                                               reinterpret_cast<__nv_bfloat16 *>(vt), T, T8, k_begin);
     else
         return cudaErrorInvalidValue;
     return cudaGetLastError();

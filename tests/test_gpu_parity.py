@@ -232,7 +232,10 @@ def test_prefill_batch2_matches_oracle(dash):
                                               (8, 64, 64, 640, False, 4), (32, 128, 64, 700, False, 64)])
 def test_prefill_host_equals_prefill(dash, G, D, Bc, T, dense, n):
     """The sliced prefill from host memory gives dash_prefill's output bit for bit (row slices
-    of 128-row multiples; D = 64 runs as one slice; more slices asked than 128-row blocks)."""
+    of 128-row multiples; D = 64 runs as one slice; more slices asked than 128-row blocks).
+    K, V and q arrive slice by slice, each slice summarising and transposing only its own rows:
+    the device buffers and the workspace start as NaN bytes, so a row that no slice covered
+    shows up in the output."""
     Hkv = 2 if G <= 16 else 1
     q, k, v, hc = make_prefill(_cfg(1, G * Hkv, Hkv, T, D, Bc, 1.5, seed=40 + G))
     qd, kd, vd, hcd = _to(q, k, v, hc)
@@ -241,8 +244,12 @@ def test_prefill_host_equals_prefill(dash, G, D, Bc, T, dense, n):
     hq, hk, hv, hhc = (x.contiguous().pin_memory() for x in (q, k, v, hc))
     ho = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
     bq, bk, bv, bhc, bo = (torch.empty_like(x) for x in (qd, kd, vd, hcd, qd))
+    for x in (bq, bk, bv, bo):
+        x.view(torch.int16).fill_(-1)                   # 0xFFFF: a bf16 NaN
     prm = dash.make_params(1, G * Hkv, Hkv, T, D, Bc, 1.5, enable_gqa=True, flags=1 if dense else 0)
     ws = dash.workspace(dash.prefill_workspace_size(prm), qd.device)
+    ws.fill_(255)
+    ws[:256].zero_()
     dash.prefill_host(hq, hk, hv, None if dense else hhc, ho, bq, bk, bv, None if dense else bhc, bo,
                       Bc, 1.5, enable_gqa=True, dense=dense, n_slices=n, ws=ws)
     torch.cuda.current_stream().synchronize()
