@@ -311,6 +311,15 @@ __device__ __forceinline__ float ipow(float m, int e) {
     for (int i = 0; i < e; ++i) r = __fmul_rn(r, m);
     return r;
 }
+// The same product chain with the exponent known at compile time (E >= 1): bit-identical to
+// ipow(m, E), and ipow_c<E - 1>(m) * m is ipow(m, E).
+template <int E>
+__device__ __forceinline__ float ipow_c(float m) {
+    float r = m;
+#pragma unroll
+    for (int i = 1; i < E; ++i) r = __fmul_rn(r, m);
+    return r;
+}
 
 // Stage 0 summary of one chunk by one warp: l_j = head_cls . k_j / sqrt(D),
 // summary = sum_j exp(l_j - max) k_j / sum_j exp(l_j - max); ks: the chunk's BC keys
@@ -581,6 +590,54 @@ struct RowInRegisters {
     }
 };
 
+// Newton's method on f^(1/beta) = 1, f(tau) = sum_c [x_c - tau]_+^beta, from tau0 = max x - 1
+// (beta >= 1).  f^(1/beta) is a beta-norm of the margins, nearly linear in tau, so it takes
+// far fewer steps than Newton on f = 1 when the support is large; it is convex and decreasing
+// too, so the steps rise monotonically to the root.  Step = (f - f^(1 - 1/beta)) / sum m^(beta-1).
+// BI > 0: beta = BI, the powers as ipow's product chain unrolled (m^BI = m^(BI-1) * m, the
+// same bits as ipow(m, BI)); BI = 0 with KIND 3: powf.
+template <int KIND, int BI, typename Row>
+__device__ __forceinline__ float newton_tau(const Row &row, float mx, const RouteConsts &rc,
+                                            uint32_t *status) {
+    const float beta = rc.beta;
+    float tau = mx - 1.f;
+    int it = 0;
+    for (; it < rc.newton_cap; ++it) {
+        const float t = tau;
+        float f, df;
+        row.pass2(
+            [t, beta](float x) {
+                const float m = x - t;
+                if (!(m > 0.f)) return 0.f;
+                if constexpr (KIND == 1) return __fmul_rn(m, m);
+                else if constexpr (KIND == 2) return m;
+                else if constexpr (BI > 0) return __fmul_rn(ipow_c<BI - 1>(m), m);
+                else return powf(m, beta);
+            },
+            [t, beta](float x) {
+                const float m = x - t;
+                if (!(m > 0.f)) return 0.f;
+                if constexpr (KIND == 1) return m;
+                else if constexpr (KIND == 2) return 1.f;
+                else if constexpr (BI > 0) return ipow_c<BI - 1>(m);
+                else return powf(m, beta - 1.f);
+            },
+            f, df);
+        f = warp_sum(f);
+        df = warp_sum(df);
+        const float step = KIND == 2 ? (f - 1.f) / df
+                         : KIND == 1 ? (f - sqrtf(f)) / df
+                                     : (f - powf(f, 1.f - 1.f / beta)) / df;
+        if (!(step > 0.f)) break;                 // at (or rounded past) the root
+        const float nt = tau + step;
+        if (nt == tau) break;
+        tau = nt;
+        if (step <= 1e-7f * fmaxf(1.f, fabsf(tau))) break;
+    }
+    if (it == rc.newton_cap) report(status, DASH_ERR_DEVICE_TIMEOUT);
+    return tau;
+}
+
 // Entmax threshold of one row (n >= 1 scores, all 32 lanes of the warp calling), specialised
 // on the kind of alpha (0 softmax, 1 alpha = 1.5, 2 alpha = 2, 3 any other alpha).  For
 // alpha = 1 returns the log-sum-exp of the scores.  Otherwise x are the scaled scores
@@ -597,42 +654,23 @@ __device__ __forceinline__ float entmax_tau_row(const Row &row, int n, const Rou
         const float s = warp_sum(row.pass([mx](float x) { return expf(x - mx); }));
         return mx + logf(s);
     }
-    const float beta = rc.beta;
     float tau;
-    if (KIND != 3 || beta >= 1.f) {
-        tau = mx - 1.f;
-        const int bi = rc.beta_int;
-        int it = 0;
-        for (; it < rc.newton_cap; ++it) {
-            const float t = tau;
-            float f, df;
-            row.pass2(
-                [t, beta, bi](float x) {
-                    const float m = x - t;
-                    return m > 0.f ? (KIND == 1 ? __fmul_rn(m, m) : KIND == 2 ? m : bi ? ipow(m, bi) : powf(m, beta)) : 0.f;
-                },
-                [t, beta, bi](float x) {
-                    const float m = x - t;
-                    return m > 0.f ? (KIND == 1 ? m : KIND == 2 ? 1.f : bi ? ipow(m, bi - 1) : powf(m, beta - 1.f)) : 0.f;
-                },
-                f, df);
-            f = warp_sum(f);
-            df = warp_sum(df);
-            // Newton on f^(1/beta) = 1, which is nearly linear in tau (a beta-norm of the
-            // margins), so far fewer steps than on f = 1 when the support is large; it is
-            // convex and decreasing too, so the steps still rise monotonically to the root.
-            // Step = (f - f^(1 - 1/beta)) / sum m^(beta-1).
-            const float step = KIND == 2 ? (f - 1.f) / df
-                             : KIND == 1 ? (f - sqrtf(f)) / df
-                                         : (f - powf(f, 1.f - 1.f / beta)) / df;
-            if (!(step > 0.f)) break;                 // at (or rounded past) the root
-            const float nt = tau + step;
-            if (nt == tau) break;
-            tau = nt;
-            if (step <= 1e-7f * fmaxf(1.f, fabsf(tau))) break;
+    if (KIND != 3 || rc.beta >= 1.f) {
+        if (KIND != 3) {
+            tau = newton_tau<KIND, 0>(row, mx, rc, status);
+        } else {
+            switch (rc.beta_int) {              // integer beta: the power chain unrolled
+                case 3: tau = newton_tau<3, 3>(row, mx, rc, status); break;
+                case 4: tau = newton_tau<3, 4>(row, mx, rc, status); break;
+                case 5: tau = newton_tau<3, 5>(row, mx, rc, status); break;
+                case 6: tau = newton_tau<3, 6>(row, mx, rc, status); break;
+                case 7: tau = newton_tau<3, 7>(row, mx, rc, status); break;
+                case 8: tau = newton_tau<3, 8>(row, mx, rc, status); break;
+                default: tau = newton_tau<3, 0>(row, mx, rc, status); break;
+            }
         }
-        if (it == rc.newton_cap) report(status, DASH_ERR_DEVICE_TIMEOUT);
     } else {
+        const float beta = rc.beta;
         float lo = mx - 1.f, hi = mx - powf((float)n, 1.f - rc.alpha);
         for (int it = 0; it < 40; ++it) {
             const float mid = 0.5f * (lo + hi);
