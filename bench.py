@@ -382,7 +382,8 @@ def bench_decode(dash, dev, steps_cap=256, warmup=3):
     dash.update_chunk_cache(kc, hc, seq, cache, Hq, Bc, n_recent=L0 // Bc)
     out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
     prm = dash.make_params(B, Hq, Hkv, cap, D, Bc, cfg.alpha, enable_gqa=True)
-    ws = dash.workspace(dash.lib.dash_decode_step_workspace_size(ctypes.byref(prm)), dev)
+    ws = torch.zeros(max(256, dash.lib.dash_decode_step_workspace_size(ctypes.byref(prm))),
+                     dtype=torch.uint8, device=dev)             # zeroed before the first step
 
     def reset():
         seq.fill_(L0)
@@ -463,7 +464,8 @@ def bench_decode_paged(dash, dev, d, cfg, S, k_new, v_new, stream):
     dash.update_chunk_cache_paged(kp, hc, table, seq, sp, Hq, Bc, n_recent=L0 // Bc)
     out = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
     prm = dash.make_params(B, Hq, Hkv, cap, D, Bc, cfg.alpha, enable_gqa=True)
-    ws = dash.workspace(dash.lib.dash_decode_step_workspace_size(ctypes.byref(prm)), dev)
+    ws = torch.zeros(max(256, dash.lib.dash_decode_step_workspace_size(ctypes.byref(prm))),
+                     dtype=torch.uint8, device=dev)             # zeroed before the first step
 
     def steps():
         for s in range(S):

@@ -304,7 +304,8 @@ dash_status_t dash_decode_paged(const dash_params_t *params, const void *q, cons
                                 void *stream);
 
 /* Bytes of device workspace dash_decode_step / dash_decode_step_paged need (the status word
- * and one counter per sequence). */
+ * and one counter per sequence).  The workspace must be zero-filled before its first step;
+ * every step leaves its counters at zero again. */
 size_t dash_decode_step_workspace_size(const dash_params_t *params);
 
 /* A whole decode step in one launch (liuzhao09.github.io "DashAttention 精读", section 2:
@@ -319,7 +320,11 @@ size_t dash_decode_step_workspace_size(const dash_params_t *params);
  * must not exceed the capacity (params->seq_len), else DASH_ERR_INVALID_ARGUMENT through
  * the status word and the sequence is left unchanged.  The other arguments as dash_decode.
  * The step reads seq_lens[b] before any write, so a loop of steps needs no host work between
- * them and can be captured in one CUDA graph. */
+ * them and can be captured in one CUDA graph.  ws: dash_decode_step_workspace_size bytes,
+ * zero-filled before the first step.  Unlike the other entry points the step does not clear
+ * the status word (it is one launch, with no memset before it): the first error of any step
+ * since the last dash_read_device_status stays in it, so one read after a loop of steps (or
+ * a graph replay) covers all of them. */
 dash_status_t dash_decode_step(const dash_params_t *params, const void *q, const void *k_new,
                                const void *v_new, void *k_cache, void *v_cache, int32_t *seq_lens,
                                float *summary_cache, const float *head_cls, void *out, float *p,

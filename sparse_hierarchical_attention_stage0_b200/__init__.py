@@ -404,7 +404,9 @@ def decode_step(q, k_new, v_new, k_cache, v_cache, seq_lens, summary_cache, head
     """A whole decode step in one launch: k_new, v_new [B,Hkv,D] bf16 are appended at row
     seq_lens[b] of the caches, q [B,Hq,D] attends over seq_lens[b] + 1 tokens, a chunk the new
     token completes gets its summary, and seq_lens is incremented (all in place).  With
-    block_table the caches are page pools (see update_chunk_cache_paged)."""
+    block_table the caches are page pools (see update_chunk_cache_paged).  A ws passed in
+    must have been zero-filled before its first step; the step does not clear its status
+    word (read_device_status does)."""
     B, Hq, D = q.shape
     dev = q.device
     if block_table is None:
@@ -422,8 +424,9 @@ def decode_step(q, k_new, v_new, k_cache, v_cache, seq_lens, summary_cache, head
     mask = active_blocks
     if mask is None and return_active_blocks:
         mask = torch.empty(B, Hkv, Wcap, dtype=torch.int64, device=dev)
-    if ws is None:
-        ws = workspace(lib.dash_decode_step_workspace_size(ctypes.byref(prm)), dev)
+    if ws is None:       # zero-filled before its first step (the arrival counters)
+        ws = torch.zeros(max(256, lib.dash_decode_step_workspace_size(ctypes.byref(prm))),
+                         dtype=torch.uint8, device=dev)
     if block_table is None:
         _check(lib.dash_decode_step(ctypes.byref(prm), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
                                     _ptr(v_cache), _ptr(seq_lens), _ptr(summary_cache), _ptr(head_cls),

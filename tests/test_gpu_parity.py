@@ -672,7 +672,8 @@ def test_decode_step_equals_append_update_and_decode(dash, kw):
             kP[table[b, c]] = kA[b, :, c * Bc:(c + 1) * Bc]
             vP[table[b, c]] = vA[b, :, c * Bc:(c + 1) * Bc]
             sP[table[b, c]] = cA[b, :, c]
-    wsA, wsB, wsP, wsU = (dash.workspace(4096, dev) for _ in range(4))
+    wsA, wsU = (dash.workspace(4096, dev) for _ in range(2))
+    wsB, wsP = (torch.zeros(4096, dtype=torch.uint8, device=dev) for _ in range(2))   # step: zeroed once
     hk = hcd if kw.get("estimate_diagonal") else None
     for s in range(steps):
         pos = [L0[b] + s for b in range(B)]
@@ -696,6 +697,8 @@ def test_decode_step_equals_append_update_and_decode(dash, kw):
     torch.cuda.synchronize()
     for ws in (wsA, wsB, wsP, wsU):
         assert dash.read_device_status(ws) == 0
+    for ws in (wsB, wsP):                     # every step left its arrival counters at zero
+        assert not ws[32:32 + 4 * B].any()
     assert torch.equal(seqA, seqB) and torch.equal(seqA, seqP)
     assert torch.equal(kA, kB) and torch.equal(vA, vB) and torch.equal(cA, cB)
     for b in range(B):
@@ -705,5 +708,10 @@ def test_decode_step_equals_append_update_and_decode(dash, kw):
     # a step past the capacity is refused on the device and leaves the sequence unchanged
     full = torch.tensor([cap, 5, 5], dtype=torch.int32, device=dev)
     dash.decode_step(qs, kn, vn, kB, vB, full, cB, hcd, Bc, ws=wsB)
+    # the status word is not cleared by a step: the error stays through a clean step after it
+    dash.decode_step(qs, kn, vn, kB, vB, torch.tensor([5, 5, 5], dtype=torch.int32, device=dev),
+                     cB, hcd, Bc, ws=wsB)
     assert dash.read_device_status(wsB) == 1
-    assert full[0].item() == cap
+    assert dash.read_device_status(wsB) == 0
+    assert full[0].item() == cap and full[1].item() == 6
+    assert not wsB[32:32 + 4 * B].any()
