@@ -32,7 +32,8 @@
 // arguments run on packed fp32 pairs (fma.rn.f32x2): about 2.5 instructions per score.
 // Warp roles: 0 K producer (3-stage ring, 128B-swizzled), 1 Q K^T issuer
 // and TMEM owner, 2 routing-bias producer (recomputes qbar.summary with Stage 1's exact
-// arithmetic, 32 chunks per batch, double-buffered), 3 P V issuer, 4-19 softmax + epilogue,
+// arithmetic for the active (token, chunk) pairs, 32 chunks per batch, double-buffered), 3 P V
+// issuer, 4-19 softmax + epilogue,
 // 20 V^T producer (warp 0 then streams K only).
 // TMEM: Q 64 columns | S0 128 | S1 128 | O 144 (128 dims + row sums).  Every wait is bounded; on timeout the CTA
 // records DASH_ERR_DEVICE_TIMEOUT and drains.
@@ -50,6 +51,11 @@ constexpr int kStages = 3;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColQ = 0, kColS = 64, kColO = 320;     // S buffer b at kColS + 128 b
 constexpr int kBiasBatch = 32;
+// Row stride (floats) of the tile's group-mean queries in shared memory: 4 floats of padding
+// put consecutive rows 4 banks apart, so the routing-bias warp, whose lanes read different
+// rows at the same column, loads them without bank conflicts (a stride of 128 floats made
+// every 16-byte load a 32-way conflict with 32 tokens per tile).
+constexpr int kQs = 128 + 4;
 constexpr int kWarpTma = 0, kWarpQk = 1, kWarpBias = 2, kWarpPv = 3, kWarpSm0 = 4,
               kWarpTmaV = kWarpSm0 + kSmWarps;
 constexpr uint32_t kBlkBytes = 32768;      // K stage: 2 d-panels x [128 keys][128 B]
@@ -104,15 +110,15 @@ __device__ __noinline__ void fa_route_tile(const float *sumg, int C, int W, floa
         if (RT >= 16) {
             // Rows in groups of 16 (register budget); each row's arithmetic is unchanged.
             for (int r0 = 0; r0 < RT; r0 += 16)
-                route_scores_lean<D, 16>(xs + r0 * xstride, xstride, qbar + r0 * D, sumg, n, wi, kSmWarps, scale);
+                route_scores_lean<D, 16>(xs + r0 * xstride, xstride, qbar + r0 * kQs, kQs, sumg, n, wi, kSmWarps, scale);
         } else if (RT == 8) {
-            route_scores_lean<D, 8>(xs, xstride, qbar, sumg, n, wi, kSmWarps, scale);
+            route_scores_lean<D, 8>(xs, xstride, qbar, kQs, sumg, n, wi, kSmWarps, scale);
         } else if (RT == 4) {
-            route_scores_lean<D, 4>(xs, xstride, qbar, sumg, n, wi, kSmWarps, scale);
+            route_scores_lean<D, 4>(xs, xstride, qbar, kQs, sumg, n, wi, kSmWarps, scale);
         } else if (RT == 2) {
-            route_scores_lean<D, 2>(xs, xstride, qbar, sumg, n, wi, kSmWarps, scale);
+            route_scores_lean<D, 2>(xs, xstride, qbar, kQs, sumg, n, wi, kSmWarps, scale);
         } else {
-            route_scores_lean<D, 1>(xs, xstride, qbar, sumg, n, wi, kSmWarps, scale);
+            route_scores_lean<D, 1>(xs, xstride, qbar, kQs, sumg, n, wi, kSmWarps, scale);
         }
     }
     __syncthreads();
@@ -155,11 +161,43 @@ __device__ __noinline__ void fa_route_tile(const float *sumg, int C, int W, floa
     }
 }
 
+// Two dot products qa . sa and qb . sb, each with route_dot's slices and order (the same
+// bits), their loads and multiply-adds interleaved.
+template <int D>
+__device__ __forceinline__ void route_dot2(const float *qa, const float *sa, const float *qb,
+                                           const float *sb, float &da, float &db) {
+    const float4 *qa4 = reinterpret_cast<const float4 *>(qa), *sa4 = reinterpret_cast<const float4 *>(sa);
+    const float4 *qb4 = reinterpret_cast<const float4 *>(qb), *sb4 = reinterpret_cast<const float4 *>(sb);
+    float pa[4], pb[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        float x = 0.f, y = 0.f;
+#pragma unroll
+        for (int i = 0; i < D / 16; ++i) {
+            const float4 s1 = __ldg(sa4 + 4 * i + k), s2 = __ldg(sb4 + 4 * i + k);
+            const float4 q1 = qa4[4 * i + k], q2 = qb4[4 * i + k];
+            x = fmaf(q1.x, s1.x, x);
+            y = fmaf(q2.x, s2.x, y);
+            x = fmaf(q1.y, s1.y, x);
+            y = fmaf(q2.y, s2.y, y);
+            x = fmaf(q1.z, s1.z, x);
+            y = fmaf(q2.z, s2.z, y);
+            x = fmaf(q1.w, s1.w, x);
+            y = fmaf(q2.w, s2.w, y);
+        }
+        pa[k] = x;
+        pb[k] = y;
+    }
+    da = (pa[0] + pa[1]) + (pa[2] + pa[3]);
+    db = (pb[0] + pb[1]) + (pb[2] + pb[3]);
+}
+
 struct FaArgs {
     StageArgs s;
     int RT;              // tokens per tile (128 / G)
     int tile0, n_tiles_bg;  // first token tile and token tiles per (b, g) of the row range
-    size_t off_bias, off_qbar, off_list, off_mask;  // dynamic smem offsets (from the aligned base)
+    size_t off_bias, off_qbar, off_list, off_mask, off_blist;  // dynamic smem offsets (aligned base)
+    int mask_smem;       // the tile's mask words are copied to shared memory (always when fused)
 };
 
 template <int BC, int NST>
@@ -175,7 +213,7 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
     unsigned char *base = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~(uintptr_t)1023);
     float *bias_s = reinterpret_cast<float *>(base + ta.off_bias);      // [2][kBiasBatch][RT]
-    float *qbar = reinterpret_cast<float *>(base + ta.off_qbar);        // [RT][D]
+    float *qbar = reinterpret_cast<float *>(base + ta.off_qbar);        // [RT][kQs]
     int16_t *list = reinterpret_cast<int16_t *>(base + ta.off_list);    // [C]
 
     if (a.cost) {                           // run-time choice against the warp-MMA kernel
@@ -218,7 +256,8 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
         fence_mbar_init();
     }
     const bool fuse = a.fuse_route != 0;
-    uint64_t *maskw = reinterpret_cast<uint64_t *>(base + ta.off_mask);  // [RT][W], fused routing
+    uint64_t *maskw = reinterpret_cast<uint64_t *>(base + ta.off_mask);  // [RT][W] (routed)
+    int16_t *blist = reinterpret_cast<int16_t *>(base + ta.off_blist);  // [kBiasBatch * RT]
     // Union of the tile's tokens' mask words (each carries its token's diagonal bit): from the
     // routing in memory, or from this kernel's own routing (maskw) when it is fused.
     auto build_list = [&](bool from_smem) {
@@ -258,7 +297,21 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
         if (lane == 0) sh.n_chunks = pos;
     };
     if (warp == kWarpBias) {
-        if (!fuse) build_list(false);
+        if (!fuse && !a.ignore_routing) {
+            // tau and, where they fit, the tile's mask words (up to its diagonal chunk) into
+            // shared memory, as the fused routing leaves them: the bias loop then reads no
+            // memory but the summaries.
+            if (ta.mask_smem) {
+                const int W = a.W, nw = ct_max / 64 + 1;
+                for (int idx = lane; idx < RT * nw; idx += 32) {
+                    const int u = idx / nw, w = idx % nw, t = t0 + u;
+                    maskw[u * W + w] = t < a.t_end ? a.mask[(bg * a.T + t) * W + w] : 0ull;
+                }
+            }
+            for (int u = lane; u < RT; u += 32) sh.tau[u] = t0 + u < a.t_end ? a.tau[bg * a.T + t0 + u] : 0.f;
+            __syncwarp();
+        }
+        if (!fuse) build_list(ta.mask_smem != 0);
         // Group-mean queries of the tile's tokens (Stage 1's exact arithmetic).
         if (!a.ignore_routing) {
             const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(a.q);
@@ -273,7 +326,7 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                     for (int e = 0; e < 8; ++e) m[e] = 0.f;
                 }
 #pragma unroll
-                for (int e = 0; e < 8; ++e) qbar[u * D + d8 + e] = m[e];
+                for (int e = 0; e < 8; ++e) qbar[u * kQs + d8 + e] = m[e];
             }
         }
     }
@@ -468,38 +521,55 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
         __syncwarp();
     } else if (warp == kWarpBias) {
         // ------------------------------------------------------------ routing biases
+        // Per batch of kBiasBatch list entries: first the entries that need no dot product
+        // (invisible or inactive: -inf; the diagonal chunk and top-k: 0) and the list of the
+        // others; then those, two per lane and step with their dot products interleaved
+        // (each with route_dot's order, so the same bits).
+        auto bias_of = [&](float dot, float tau) -> float {
+            if (a.rc.kind == 0) return a.rc.sigma2 * (__fmul_rn(dot, a.rc.sscale) - tau);
+            const float m = __fsub_rn(__fmul_rn(dot, a.rc.xscale), tau);
+            return a.rc.bscale2 * log2f(fmaxf(m, 1e-37f));
+        };
+        const float *sumg = a.summary + bg * a.Cf * D;
+        const bool msm = fuse || ta.mask_smem;
         const int n_batches = (n_chunks + kBiasBatch - 1) / kBiasBatch;
         for (int bt = 0; bt < n_batches; ++bt) {
             float *buf = bias_s + (bt & 1) * kBiasBatch * RT;
-            for (int e = lane; e < kBiasBatch * RT; e += 32) {
+            int nact = 0;
+            for (int e0 = 0; e0 < kBiasBatch * RT; e0 += 32) {
+                const int e = e0 + lane;
                 const int k = e / RT, u = e % RT, ci = bt * kBiasBatch + k;
                 float v = 0.f;
+                bool need = false;
                 if (ci < n_chunks && !a.ignore_routing) {
                     const int c = chunk_at(ci), t = t0 + u;
                     const int ctu = t / BC;
                     if (t >= a.t_end || c > ctu) {
                         v = -INFINITY;
                     } else if (c < ctu) {
-                        const long long rowi = bg * a.T + t;
-                        const uint64_t word = fuse ? maskw[u * a.W + (c >> 6)] : a.mask[rowi * a.W + (c >> 6)];
+                        const uint64_t word = msm ? maskw[u * a.W + (c >> 6)]
+                                                  : a.mask[(bg * a.T + t) * a.W + (c >> 6)];
                         const bool act = dash_check(t < a.T && c < a.Cf, a.status) && ((word >> (c & 63)) & 1ull);
-                        if (!act) {
-                            v = -INFINITY;
-                        } else {
-                            const float dot = route_dot<D>(qbar + u * D, a.summary + (bg * a.Cf + c) * D);
-                            const float tau = fuse ? sh.tau[u] : a.tau[rowi];
-                            if (a.rc.kind == kKindTopk) {
-                                v = 0.f;                        // top-k: uniform prior
-                            } else if (a.rc.kind == 0) {
-                                v = a.rc.sigma2 * (__fmul_rn(dot, a.rc.sscale) - tau);
-                            } else {
-                                const float m = __fsub_rn(__fmul_rn(dot, a.rc.xscale), tau);
-                                v = a.rc.bscale2 * log2f(fmaxf(m, 1e-37f));
-                            }
-                        }
+                        if (!act) v = -INFINITY;
+                        else if (a.rc.kind != kKindTopk) need = true;   // top-k: uniform prior, 0
                     }
                 }
                 buf[e] = v;
+                const unsigned bal = __ballot_sync(kFull, need);
+                if (need) blist[nact + __popc(bal & ((1u << lane) - 1u))] = (int16_t)e;
+                nact += __popc(bal);
+            }
+            __syncwarp();
+            for (int j = lane; j < nact; j += 64) {
+                const bool two = j + 32 < nact;
+                const int ea = blist[j], eb = two ? blist[j + 32] : ea;
+                const int ua = ea % RT, ub = eb % RT;
+                const int ca = chunk_at(bt * kBiasBatch + ea / RT), cb = chunk_at(bt * kBiasBatch + eb / RT);
+                float da, db;
+                route_dot2<D>(qbar + ua * kQs, sumg + (long long)ca * D, qbar + ub * kQs,
+                              sumg + (long long)cb * D, da, db);
+                buf[ea] = bias_of(da, sh.tau[ua]);
+                if (two) buf[eb] = bias_of(db, sh.tau[ub]);
             }
             __syncwarp();
             named_sync(1, 32 + kSmThreads);
@@ -664,13 +734,14 @@ bool fa_map(EncodeFn enc, CUtensorMap *m, const void *ptr, int T, int BHkv, int 
                CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-size_t fa_smem_bytes(int RT, int C, bool fuse, int nst) {
+size_t fa_smem_bytes(int RT, int C, bool mask_words, int nst) {
     size_t off = ring_bytes(nst);
     off += (size_t)2 * kBiasBatch * RT * 4;      // bias batches
-    off += (size_t)RT * 128 * 4;                 // qbar
+    off += (size_t)RT * kQs * 4;                 // qbar
     off += (size_t)((C + 7) & ~7) * 2;           // chunk list
     off = (off + 7) & ~(size_t)7;
-    if (fuse) off += (size_t)RT * ((C + 63) / 64) * 8;   // the tile's mask words
+    if (mask_words) off += (size_t)RT * ((C + 63) / 64) * 8;   // the tile's mask words
+    off += (size_t)kBiasBatch * RT * 2;          // a batch's entries that need a dot product
     return off + 1024;                           // room to align the base to 1024 bytes
 }
 
@@ -681,28 +752,38 @@ size_t attend_fa_vt_bytes(int B, int Hkv, int T, int D) {
     return (size_t)B * Hkv * D * T8 * 2;
 }
 
-// Ring stages for these arguments: 3, or 2 when 3 do not fit (0: neither fits).
-static int fa_stages(const StageArgs &a, bool fuse) {
+// Ring stages for these arguments (3, or 2 when 3 do not fit; 0: neither fits) and whether the
+// tile's mask words go to shared memory: the deepest ring first, with the mask words where
+// they fit beside it (the fused routing needs them there).
+struct FaPlan {
+    int nst;
+    bool mask_smem;
+};
+static FaPlan fa_plan(const StageArgs &a, bool fuse) {
     if (!(a.D == 128 && a.G >= 2 && a.G <= 128 && 128 % a.G == 0 && (a.Bc == 64 || a.Bc == 128) &&
           128 / a.G <= a.Bc))                  // a tile's tokens share one diagonal chunk
-        return 0;
+        return {0, false};
     const int RT = 128 / a.G;
     for (int nst : {3, 2}) {
         if (fuse && (size_t)RT * ((a.C + 3) & ~3) * 4 > ring_bytes(nst)) continue;   // scores fit the ring
-        if (fa_smem_bytes(RT, a.C, fuse, nst) + sizeof(FaShared) <= 227 * 1024) return nst;
+        for (bool ms : {true, false}) {
+            if (!ms && fuse) continue;
+            const bool m = ms && !a.ignore_routing;
+            if (fa_smem_bytes(RT, a.C, m, nst) + sizeof(FaShared) <= 227 * 1024) return {nst, m};
+        }
     }
-    return 0;
+    return {0, false};
 }
 
-bool attend_fa_supported(const StageArgs &a) { return fa_stages(a, false) != 0; }
+bool attend_fa_supported(const StageArgs &a) { return fa_plan(a, false).nst != 0; }
 
 bool attend_fa_fuse_supported(const StageArgs &a) {
     if (a.ignore_routing || a.rc.kind > 3 || a.rc.est_diag) return false;
-    return fa_stages(a, true) != 0;
+    return fa_plan(a, true).nst != 0;
 }
 
 template <int BC, int NST>
-static cudaError_t launch_fa_t(const StageArgs &a, cudaStream_t st) {
+static cudaError_t launch_fa_t(const StageArgs &a, bool mask_smem, cudaStream_t st) {
     static EncodeFn enc = fa_encode();
     if (!enc || !a.vt) return cudaErrorNotSupported;
     const int BHkv = a.B * a.Hkv;
@@ -733,11 +814,13 @@ static cudaError_t launch_fa_t(const StageArgs &a, cudaStream_t st) {
     ta.off_bias = off;
     off += (size_t)2 * kBiasBatch * ta.RT * 4;
     ta.off_qbar = off;
-    off += (size_t)ta.RT * 128 * 4;
+    off += (size_t)ta.RT * kQs * 4;
     ta.off_list = off;
     off += (size_t)((a.C + 7) & ~7) * 2;
     ta.off_mask = (off + 7) & ~(size_t)7;
-    const size_t smem = fa_smem_bytes(ta.RT, a.C, a.fuse_route != 0, NST);
+    ta.mask_smem = mask_smem ? 1 : 0;
+    ta.off_blist = ta.off_mask + (mask_smem ? (size_t)ta.RT * ((a.C + 63) / 64) * 8 : 0);
+    const size_t smem = fa_smem_bytes(ta.RT, a.C, mask_smem, NST);
     auto kern = k_attend_fa<BC, NST>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -748,11 +831,11 @@ static cudaError_t launch_fa_t(const StageArgs &a, cudaStream_t st) {
 }
 
 cudaError_t launch_attend_fa(const StageArgs &a, cudaStream_t st) {
-    const int nst = fa_stages(a, a.fuse_route != 0);
-    if (a.Bc == 64 && nst == 3) return launch_fa_t<64, 3>(a, st);
-    if (a.Bc == 64 && nst == 2) return launch_fa_t<64, 2>(a, st);
-    if (a.Bc == 128 && nst == 3) return launch_fa_t<128, 3>(a, st);
-    if (a.Bc == 128 && nst == 2) return launch_fa_t<128, 2>(a, st);
+    const FaPlan pl = fa_plan(a, a.fuse_route != 0);
+    if (a.Bc == 64 && pl.nst == 3) return launch_fa_t<64, 3>(a, pl.mask_smem, st);
+    if (a.Bc == 64 && pl.nst == 2) return launch_fa_t<64, 2>(a, pl.mask_smem, st);
+    if (a.Bc == 128 && pl.nst == 3) return launch_fa_t<128, 3>(a, pl.mask_smem, st);
+    if (a.Bc == 128 && pl.nst == 2) return launch_fa_t<128, 2>(a, pl.mask_smem, st);
     return cudaErrorInvalidValue;
 }
 

@@ -242,11 +242,11 @@ constexpr int kKindTopk = 4;
 // quarter of d as one sequential fmaf chain, two chunks (c, c + 8) per lane, slices combined
 // as (p0 + p1) + (p2 + p3) -- route_dot's order, so every score has route_dot's bits.  The
 // summary rows are loaded one float4 group at a time (few registers: usable inside a kernel
-// with a tight register budget).  qbar: [RT][D] in shared memory.
+// with a tight register budget).  qbar: RT rows of D in shared memory, qstride floats apart.
 template <int D, int RT>
 __device__ __forceinline__ void route_scores_lean(float *xs, int xstride, const float *qbar,
-                                                  const float *sumg, int n, int warp_idx,
-                                                  int n_warps, float scale) {
+                                                  int qstride, const float *sumg, int n,
+                                                  int warp_idx, int n_warps, float scale) {
     const int lane = threadIdx.x & 31;
     const int kslice = lane & 3, cc = lane >> 2;
     for (int cbase = warp_idx * 16; cbase < n; cbase += n_warps * 16) {
@@ -261,7 +261,7 @@ __device__ __forceinline__ void route_scores_lean(float *xs, int xstride, const 
             const float4 sv = __ldg(s4 + 4 * i + kslice), tv = __ldg(t4 + 4 * i + kslice);
 #pragma unroll
             for (int r = 0; r < RT; ++r) {
-                const float4 qq = reinterpret_cast<const float4 *>(qbar + r * D)[4 * i + kslice];
+                const float4 qq = reinterpret_cast<const float4 *>(qbar + r * qstride)[4 * i + kslice];
                 acc[r] = fmaf(qq.x, sv.x, acc[r]);
                 acc2[r] = fmaf(qq.x, tv.x, acc2[r]);
                 acc[r] = fmaf(qq.y, sv.y, acc[r]);
