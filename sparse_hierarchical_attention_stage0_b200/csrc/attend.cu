@@ -302,10 +302,13 @@ __global__ void __launch_bounds__(128) k_union_cost(StageArgs a, unsigned long l
     }
 }
 
-// Executed token-chunk pairs per unit of time of the two kernels for G = 4 (TFLOP/s on
-// executed blocks measured on B200 over the 64K sweep cells: 128-key blocks about 355 with
-// 64-key chunks and 620 with 128-key chunks, warp MMA about 135); only their ratio is used.
-constexpr float kRateFa64 = 355.f, kRateFa128 = 620.f, kRateWarp = 135.f;
+// Executed token-chunk pairs per unit of time of the two kernels for G = 4, as TFLOP/s on
+// executed blocks measured on B200 over the 64K sweep cells: 128-key blocks 470-940 with
+// 64-key chunks and 610-1000 with 128-key chunks (lower where more of a batch's pairs are
+// active and need a routing dot product), warp MMA 128-155.  Only their ratio is used; these
+// values pick the faster kernel in all six cells (the closest, alpha 1.5 and 2 with 64-key
+// chunks, lie at ratios 4.5 and 5.9 on either side of 690 / 135 = 5.1).
+constexpr float kRateFa64 = 690.f, kRateFa128 = 900.f, kRateWarp = 135.f;
 
 // A run-time choice applies to full-range routed calls with fewer than 8 query heads per KV
 // head: there the 128-key-block kernel's tiles (128/G tokens) walk much larger unions than
