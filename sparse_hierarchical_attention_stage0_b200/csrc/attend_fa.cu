@@ -70,6 +70,7 @@ struct FaShared {
     uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
     uint64_t s_full[2], p_full[2], pv_done[2];  // per S buffer: never more than one phase ahead
     uint64_t o_full, qk_done;
+    uint64_t sum_full[2];                  // a routing-bias batch's summary rows have landed
     float mpart[4][128];                   // partial row maxima of the first block
     float tau[64];                         // fused routing: tau of the tile's tokens
     uint32_t tmem_base;
@@ -162,8 +163,9 @@ __device__ __noinline__ void fa_route_tile(const float *sumg, int C, int W, floa
 }
 
 // Two dot products qa . sa and qb . sb, each with route_dot's slices and order (the same
-// bits), their loads and multiply-adds interleaved.
-template <int D>
+// bits), their loads and multiply-adds interleaved.  kLdg: sa, sb in global memory (read-only
+// path); otherwise in shared memory.
+template <int D, bool kLdg>
 __device__ __forceinline__ void route_dot2(const float *qa, const float *sa, const float *qb,
                                            const float *sb, float &da, float &db) {
     const float4 *qa4 = reinterpret_cast<const float4 *>(qa), *sa4 = reinterpret_cast<const float4 *>(sa);
@@ -174,7 +176,8 @@ __device__ __forceinline__ void route_dot2(const float *qa, const float *sa, con
         float x = 0.f, y = 0.f;
 #pragma unroll
         for (int i = 0; i < D / 16; ++i) {
-            const float4 s1 = __ldg(sa4 + 4 * i + k), s2 = __ldg(sb4 + 4 * i + k);
+            const float4 s1 = kLdg ? __ldg(sa4 + 4 * i + k) : sa4[4 * i + k];
+            const float4 s2 = kLdg ? __ldg(sb4 + 4 * i + k) : sb4[4 * i + k];
             const float4 q1 = qa4[4 * i + k], q2 = qb4[4 * i + k];
             x = fmaf(q1.x, s1.x, x);
             y = fmaf(q2.x, s2.x, y);
@@ -196,8 +199,9 @@ struct FaArgs {
     StageArgs s;
     int RT;              // tokens per tile (128 / G)
     int tile0, n_tiles_bg;  // first token tile and token tiles per (b, g) of the row range
-    size_t off_bias, off_qbar, off_list, off_mask, off_blist;  // dynamic smem offsets (aligned base)
+    size_t off_bias, off_qbar, off_list, off_mask, off_blist, off_sum;  // dynamic smem offsets (aligned base)
     int mask_smem;       // the tile's mask words are copied to shared memory (always when fused)
+    int sum_smem;        // the bias batches' summary rows are staged in shared memory
 };
 
 template <int BC, int NST>
@@ -252,6 +256,8 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
         }
         mbar_init(&sh.o_full, 1);
         mbar_init(&sh.qk_done, 1);
+        mbar_init(&sh.sum_full[0], 1);
+        mbar_init(&sh.sum_full[1], 1);
         sh.failed = 0;
         fence_mbar_init();
     }
@@ -533,8 +539,40 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
         const float *sumg = a.summary + bg * a.Cf * D;
         const bool msm = fuse || ta.mask_smem;
         const int n_batches = (n_chunks + kBiasBatch - 1) / kBiasBatch;
+        // Staged summaries: the rows of a batch's chunks below the diagonal one (the only ones
+        // with a dot product) are copied by the TMA engine into sum_s[bt & 1][k] (rows of kQs
+        // floats: lanes reading different rows at the same column hit different banks), two
+        // batches in flight, so the dot products read shared memory instead of waiting on L2.
+        float *sum_s = reinterpret_cast<float *>(base + ta.off_sum);     // [2][kBiasBatch][kQs]
+        const bool stage = ta.sum_smem && !a.ignore_routing;
+        int last_issued = -1;
+        auto issue_batch = [&](int bt2) {
+            if (bt2 >= n_batches) return;
+            last_issued = bt2;
+            const int ci = bt2 * kBiasBatch + lane;
+            const int c = ci < n_chunks ? chunk_at(ci) : ct_max;
+            const bool row = c < ct_max && c < a.Cf;
+            const unsigned bal = __ballot_sync(kFull, row);
+            if (lane == 0) mbar_arrive_expect_tx(&sh.sum_full[bt2 & 1], (uint32_t)__popc(bal) * D * 4);
+            __syncwarp();
+            if (row)
+                bulk_g2s(sum_s + ((bt2 & 1) * kBiasBatch + lane) * kQs, sumg + (long long)c * D, D * 4,
+                         &sh.sum_full[bt2 & 1]);
+        };
+        if (stage) {
+            issue_batch(0);
+            issue_batch(1);
+        }
+        bool sum_failed = false;
         for (int bt = 0; bt < n_batches; ++bt) {
             float *buf = bias_s + (bt & 1) * kBiasBatch * RT;
+            // A timed-out copy leaves the biases of this and later batches unset (the status
+            // word reports it); the batches' barriers are still passed.
+            if (stage && !wait_or_fail(&sh.sum_full[bt & 1], (uint32_t)(bt >> 1) & 1u, a.status, sum_failed)) {
+                __syncwarp();
+                named_sync(1, 32 + kSmThreads);
+                continue;
+            }
             int nact = 0;
             for (int e0 = 0; e0 < kBiasBatch * RT; e0 += 32) {
                 const int e = e0 + lane;
@@ -566,13 +604,32 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                 const int ua = ea % RT, ub = eb % RT;
                 const int ca = chunk_at(bt * kBiasBatch + ea / RT), cb = chunk_at(bt * kBiasBatch + eb / RT);
                 float da, db;
-                route_dot2<D>(qbar + ua * kQs, sumg + (long long)ca * D, qbar + ub * kQs,
-                              sumg + (long long)cb * D, da, db);
+                if (stage) {
+                    const float *sb0 = sum_s + (bt & 1) * kBiasBatch * kQs;
+                    route_dot2<D, false>(qbar + ua * kQs, sb0 + (ea / RT) * kQs, qbar + ub * kQs,
+                                         sb0 + (eb / RT) * kQs, da, db);
+                } else {
+                    route_dot2<D, true>(qbar + ua * kQs, sumg + (long long)ca * D, qbar + ub * kQs,
+                                        sumg + (long long)cb * D, da, db);
+                }
                 buf[ea] = bias_of(da, sh.tau[ua]);
                 if (two) buf[eb] = bias_of(db, sh.tau[ub]);
             }
             __syncwarp();
+            if (stage) {
+                // This batch's rows are read: order those reads before the copies that refill
+                // the buffer.
+                fence_proxy_async();
+                issue_batch(bt + 2);
+            }
             named_sync(1, 32 + kSmThreads);
+        }
+        if (sum_failed) {
+            // Copies issued after the timeout may still be in flight: wait for them (bounded)
+            // before the CTA can exit.
+            failed = true;
+            for (int bb = max(last_issued - 1, 0); bb <= last_issued; ++bb)
+                mbar_wait_bounded(&sh.sum_full[bb & 1], (uint32_t)(bb >> 1) & 1u);
         }
     } else if (warp >= kWarpSm0 && warp < kWarpTmaV) {
         // ------------------------------------------------------------ softmax
@@ -734,7 +791,7 @@ bool fa_map(EncodeFn enc, CUtensorMap *m, const void *ptr, int T, int BHkv, int 
                CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-size_t fa_smem_bytes(int RT, int C, bool mask_words, int nst) {
+size_t fa_smem_bytes(int RT, int C, bool mask_words, int nst, bool sum_rows) {
     size_t off = ring_bytes(nst);
     off += (size_t)2 * kBiasBatch * RT * 4;      // bias batches
     off += (size_t)RT * kQs * 4;                 // qbar
@@ -742,6 +799,8 @@ size_t fa_smem_bytes(int RT, int C, bool mask_words, int nst) {
     off = (off + 7) & ~(size_t)7;
     if (mask_words) off += (size_t)RT * ((C + 63) / 64) * 8;   // the tile's mask words
     off += (size_t)kBiasBatch * RT * 2;          // a batch's entries that need a dot product
+    off = (off + 15) & ~(size_t)15;
+    if (sum_rows) off += (size_t)2 * kBiasBatch * kQs * 4;     // two batches' summary rows
     return off + 1024;                           // room to align the base to 1024 bytes
 }
 
@@ -752,27 +811,31 @@ size_t attend_fa_vt_bytes(int B, int Hkv, int T, int D) {
     return (size_t)B * Hkv * D * T8 * 2;
 }
 
-// Ring stages for these arguments (3, or 2 when 3 do not fit; 0: neither fits) and whether the
-// tile's mask words go to shared memory: the deepest ring first, with the mask words where
-// they fit beside it (the fused routing needs them there).
+// Ring stages for these arguments (3, or 2 when 3 do not fit; 0: neither fits), whether the
+// tile's mask words go to shared memory and whether the bias batches' summary rows are staged
+// there: the deepest ring first, with the mask words and then the staged rows where they fit
+// beside it (the fused routing needs the mask words there).
 struct FaPlan {
     int nst;
-    bool mask_smem;
+    bool mask_smem, sum_smem;
 };
 static FaPlan fa_plan(const StageArgs &a, bool fuse) {
     if (!(a.D == 128 && a.G >= 2 && a.G <= 128 && 128 % a.G == 0 && (a.Bc == 64 || a.Bc == 128) &&
           128 / a.G <= a.Bc))                  // a tile's tokens share one diagonal chunk
-        return {0, false};
+        return {0, false, false};
     const int RT = 128 / a.G;
     for (int nst : {3, 2}) {
         if (fuse && (size_t)RT * ((a.C + 3) & ~3) * 4 > ring_bytes(nst)) continue;   // scores fit the ring
-        for (bool ms : {true, false}) {
+        for (int v = 0; v < 3; ++v) {
+            const bool ms = v < 2, ss = v == 0;   // mask and rows, mask only, neither
             if (!ms && fuse) continue;
-            const bool m = ms && !a.ignore_routing;
-            if (fa_smem_bytes(RT, a.C, m, nst) + sizeof(FaShared) <= 227 * 1024) return {nst, m};
+            // (bulk copies need 16-byte aligned summary rows)
+            const bool m = ms && !a.ignore_routing,
+                       sr = ss && !a.ignore_routing && (reinterpret_cast<uintptr_t>(a.summary) & 15) == 0;
+            if (fa_smem_bytes(RT, a.C, m, nst, sr) + sizeof(FaShared) <= 227 * 1024) return {nst, m, sr};
         }
     }
-    return {0, false};
+    return {0, false, false};
 }
 
 bool attend_fa_supported(const StageArgs &a) { return fa_plan(a, false).nst != 0; }
@@ -783,7 +846,7 @@ bool attend_fa_fuse_supported(const StageArgs &a) {
 }
 
 template <int BC, int NST>
-static cudaError_t launch_fa_t(const StageArgs &a, bool mask_smem, cudaStream_t st) {
+static cudaError_t launch_fa_t(const StageArgs &a, bool mask_smem, bool sum_smem, cudaStream_t st) {
     static EncodeFn enc = fa_encode();
     if (!enc || !a.vt) return cudaErrorNotSupported;
     const int BHkv = a.B * a.Hkv;
@@ -820,7 +883,9 @@ static cudaError_t launch_fa_t(const StageArgs &a, bool mask_smem, cudaStream_t 
     ta.off_mask = (off + 7) & ~(size_t)7;
     ta.mask_smem = mask_smem ? 1 : 0;
     ta.off_blist = ta.off_mask + (mask_smem ? (size_t)ta.RT * ((a.C + 63) / 64) * 8 : 0);
-    const size_t smem = fa_smem_bytes(ta.RT, a.C, mask_smem, NST);
+    ta.sum_smem = sum_smem ? 1 : 0;
+    ta.off_sum = (ta.off_blist + (size_t)kBiasBatch * ta.RT * 2 + 15) & ~(size_t)15;
+    const size_t smem = fa_smem_bytes(ta.RT, a.C, mask_smem, NST, sum_smem);
     auto kern = k_attend_fa<BC, NST>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -832,10 +897,10 @@ static cudaError_t launch_fa_t(const StageArgs &a, bool mask_smem, cudaStream_t 
 
 cudaError_t launch_attend_fa(const StageArgs &a, cudaStream_t st) {
     const FaPlan pl = fa_plan(a, a.fuse_route != 0);
-    if (a.Bc == 64 && pl.nst == 3) return launch_fa_t<64, 3>(a, pl.mask_smem, st);
-    if (a.Bc == 64 && pl.nst == 2) return launch_fa_t<64, 2>(a, pl.mask_smem, st);
-    if (a.Bc == 128 && pl.nst == 3) return launch_fa_t<128, 3>(a, pl.mask_smem, st);
-    if (a.Bc == 128 && pl.nst == 2) return launch_fa_t<128, 2>(a, pl.mask_smem, st);
+    if (a.Bc == 64 && pl.nst == 3) return launch_fa_t<64, 3>(a, pl.mask_smem, pl.sum_smem, st);
+    if (a.Bc == 64 && pl.nst == 2) return launch_fa_t<64, 2>(a, pl.mask_smem, pl.sum_smem, st);
+    if (a.Bc == 128 && pl.nst == 3) return launch_fa_t<128, 3>(a, pl.mask_smem, pl.sum_smem, st);
+    if (a.Bc == 128 && pl.nst == 2) return launch_fa_t<128, 2>(a, pl.mask_smem, pl.sum_smem, st);
     return cudaErrorInvalidValue;
 }
 
