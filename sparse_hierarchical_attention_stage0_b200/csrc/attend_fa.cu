@@ -31,10 +31,10 @@
 // P V (N = 144) leaves sum_k P[r, k] in O column 128.  Off the diagonal the exponent
 // arguments run on packed fp32 pairs (fma.rn.f32x2): about 2.5 instructions per score.
 // Warp roles: 0 K producer (3-stage ring, 128B-swizzled), 1 Q K^T issuer
-// and TMEM owner, 2 routing-bias producer (recomputes qbar.summary with Stage 1's exact
-// arithmetic for the active (token, chunk) pairs, 32 chunks per batch, double-buffered), 3 P V
-// issuer, 4-19 softmax + epilogue,
-// 20 V^T producer (warp 0 then streams K only).
+// and TMEM owner, 2 and 21 routing-bias producers (recompute qbar.summary with Stage 1's exact
+// arithmetic for the active (token, chunk) pairs, 32 chunks per batch, half a batch each,
+// double-buffered; at G <= 4 the batch's summary rows are staged in shared memory), 3 P V
+// issuer, 4-19 softmax + epilogue, 20 V^T producer (warp 0 then streams K only).
 // TMEM: Q 64 columns | S0 128 | S1 128 | O 144 (128 dims + row sums).  Every wait is bounded; on timeout the CTA
 // records DASH_ERR_DEVICE_TIMEOUT and drains.
 #include "kernels.cuh"
@@ -46,7 +46,7 @@ namespace {
 
 constexpr int kSmWarps = 16;
 constexpr int kSmThreads = kSmWarps * 32;
-constexpr int kFaThreads = 4 * 32 + kSmThreads + 32;
+constexpr int kFaThreads = 4 * 32 + kSmThreads + 64;
 constexpr int kStages = 3;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColQ = 0, kColS = 64, kColO = 320;     // S buffer b at kColS + 128 b
@@ -57,7 +57,8 @@ constexpr int kBiasBatch = 32;
 // every 16-byte load a 32-way conflict with 32 tokens per tile).
 constexpr int kQs = 128 + 4;
 constexpr int kWarpTma = 0, kWarpQk = 1, kWarpBias = 2, kWarpPv = 3, kWarpSm0 = 4,
-              kWarpTmaV = kWarpSm0 + kSmWarps;
+              kWarpTmaV = kWarpSm0 + kSmWarps, kWarpBias2 = kWarpTmaV + 1;
+constexpr int kBiasThreads = 64;           // the two routing-bias warps
 constexpr uint32_t kBlkBytes = 32768;      // K stage: 2 d-panels x [128 keys][128 B]
 constexpr int kNv = 144;                   // P V columns: 128 dims of V, then 16 columns of ones
 constexpr uint32_t kVHalf = kNv * 128;     // V^T key-half: [144 rows][64 keys x 2 B] (rows >= 128: ones)
@@ -525,12 +526,16 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
         }
         if (lane == 0) mma_commit(&sh.o_full);        // tracks every MMA issued above
         __syncwarp();
-    } else if (warp == kWarpBias) {
+    } else if (warp == kWarpBias || warp == kWarpBias2) {
         // ------------------------------------------------------------ routing biases
-        // Per batch of kBiasBatch list entries: first the entries that need no dot product
-        // (invisible or inactive: -inf; the diagonal chunk and top-k: 0) and the list of the
-        // others; then those, two per lane and step with their dot products interleaved
-        // (each with route_dot's order, so the same bits).
+        // Two warps; each takes half of every batch of kBiasBatch list entries (bw: which
+        // half).  Per half: first the entries that need no dot product (invisible or inactive:
+        // -inf; the diagonal chunk and top-k: 0) and the list of the others; then those, two
+        // per lane and step with their dot products interleaved (each with route_dot's order,
+        // so the same bits).
+        const int bw = warp == kWarpBias ? 0 : 1;
+        const int half_n = kBiasBatch * RT / 2;   // entries per warp and batch (RT even)
+        int16_t *my_list = blist + bw * half_n;
         auto bias_of = [&](float dot, float tau) -> float {
             if (a.rc.kind == 0) return a.rc.sigma2 * (__fmul_rn(dot, a.rc.sscale) - tau);
             const float m = __fsub_rn(__fmul_rn(dot, a.rc.xscale), tau);
@@ -546,7 +551,7 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
         float *sum_s = reinterpret_cast<float *>(base + ta.off_sum);     // [2][kBiasBatch][kQs]
         const bool stage = ta.sum_smem && !a.ignore_routing;
         int last_issued = -1;
-        auto issue_batch = [&](int bt2) {
+        auto issue_batch = [&](int bt2) {       // the first bias warp issues the copies
             if (bt2 >= n_batches) return;
             last_issued = bt2;
             const int ci = bt2 * kBiasBatch + lane;
@@ -559,7 +564,7 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                 bulk_g2s(sum_s + ((bt2 & 1) * kBiasBatch + lane) * kQs, sumg + (long long)c * D, D * 4,
                          &sh.sum_full[bt2 & 1]);
         };
-        if (stage) {
+        if (stage && bw == 0) {
             issue_batch(0);
             issue_batch(1);
         }
@@ -568,18 +573,15 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
             float *buf = bias_s + (bt & 1) * kBiasBatch * RT;
             // A timed-out copy leaves the biases of this and later batches unset (the status
             // word reports it); the batches' barriers are still passed.
-            if (stage && !wait_or_fail(&sh.sum_full[bt & 1], (uint32_t)(bt >> 1) & 1u, a.status, sum_failed)) {
-                __syncwarp();
-                named_sync(1, 32 + kSmThreads);
-                continue;
-            }
+            const bool ready = !stage || wait_or_fail(&sh.sum_full[bt & 1], (uint32_t)(bt >> 1) & 1u, a.status, sum_failed);
             int nact = 0;
-            for (int e0 = 0; e0 < kBiasBatch * RT; e0 += 32) {
+            for (int e0 = bw * half_n; e0 < (bw + 1) * half_n && ready; e0 += 32) {
                 const int e = e0 + lane;
+                const bool mine = e < (bw + 1) * half_n;   // (a half holds 16 entries at RT = 1)
                 const int k = e / RT, u = e % RT, ci = bt * kBiasBatch + k;
                 float v = 0.f;
                 bool need = false;
-                if (ci < n_chunks && !a.ignore_routing) {
+                if (mine && ci < n_chunks && !a.ignore_routing) {
                     const int c = chunk_at(ci), t = t0 + u;
                     const int ctu = t / BC;
                     if (t >= a.t_end || c > ctu) {
@@ -592,15 +594,15 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
                         else if (a.rc.kind != kKindTopk) need = true;   // top-k: uniform prior, 0
                     }
                 }
-                buf[e] = v;
+                if (mine) buf[e] = v;
                 const unsigned bal = __ballot_sync(kFull, need);
-                if (need) blist[nact + __popc(bal & ((1u << lane) - 1u))] = (int16_t)e;
+                if (need) my_list[nact + __popc(bal & ((1u << lane) - 1u))] = (int16_t)e;
                 nact += __popc(bal);
             }
             __syncwarp();
             for (int j = lane; j < nact; j += 64) {
                 const bool two = j + 32 < nact;
-                const int ea = blist[j], eb = two ? blist[j + 32] : ea;
+                const int ea = my_list[j], eb = two ? my_list[j + 32] : ea;
                 const int ua = ea % RT, ub = eb % RT;
                 const int ca = chunk_at(bt * kBiasBatch + ea / RT), cb = chunk_at(bt * kBiasBatch + eb / RT);
                 float da, db;
@@ -617,19 +619,21 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
             }
             __syncwarp();
             if (stage) {
-                // This batch's rows are read: order those reads before the copies that refill
-                // the buffer.
+                // This batch's rows are read by both warps: order those reads before the
+                // copies that refill the buffer.
                 fence_proxy_async();
-                issue_batch(bt + 2);
+                named_sync(3, kBiasThreads);
+                if (bw == 0 && !sum_failed) issue_batch(bt + 2);
             }
-            named_sync(1, 32 + kSmThreads);
+            named_sync(1, kBiasThreads + kSmThreads);
         }
         if (sum_failed) {
-            // Copies issued after the timeout may still be in flight: wait for them (bounded)
-            // before the CTA can exit.
+            // Copies issued after the timeout may still be in flight: the issuing warp waits
+            // for them (bounded) before the CTA can exit.
             failed = true;
-            for (int bb = max(last_issued - 1, 0); bb <= last_issued; ++bb)
-                mbar_wait_bounded(&sh.sum_full[bb & 1], (uint32_t)(bb >> 1) & 1u);
+            if (bw == 0)
+                for (int bb = max(last_issued - 1, 0); bb <= last_issued; ++bb)
+                    mbar_wait_bounded(&sh.sum_full[bb & 1], (uint32_t)(bb >> 1) & 1u);
         }
     } else if (warp >= kWarpSm0 && warp < kWarpTmaV) {
         // ------------------------------------------------------------ softmax
@@ -643,7 +647,7 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
         for (int j = 0; j < n_blocks; ++j) {
             const int sb = j & 1;
             const int e0 = BC == 64 ? 2 * j : j;              // first list entry of the block
-            if (e0 % kBiasBatch == 0) named_sync(1, 32 + kSmThreads);
+            if (e0 % kBiasBatch == 0) named_sync(1, kBiasThreads + kSmThreads);
             const bool ok = wait_or_fail(&sh.s_full[sb], (uint32_t)(j >> 1) & 1u, a.status, failed);
             if (ok) tc_fence_after();
             const int e = entry_of(j, half);
