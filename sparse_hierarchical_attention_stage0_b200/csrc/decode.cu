@@ -96,6 +96,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     __shared__ float tau_s;
     __shared__ int nact_s;
+    __shared__ float wfac[kDecWarps][16], wmax[16];   // the CTA merge's per-row weights
     const DecLayout<D> L(a.Ccap);
     float *qbar = reinterpret_cast<float *>(smem_raw + L.qbar);
     float *cpart = reinterpret_cast<float *>(smem_raw + L.cta_part);   // O[16][D], m, l
@@ -437,21 +438,29 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(DecodeArgs a) {
     }
     __syncthreads();
 
-    // 4b. CTA merge of the warp partials into cpart.
-    for (int idx = tid; idx < 16 * D + 16; idx += kDecWarps * 32) {
-        const int r = idx < 16 * D ? idx / D : idx - 16 * D;
+    // 4b. CTA merge of the warp partials into cpart: each row's warp weights 2^(m_w - m*)
+    // once, then every output of the row with them.
+    if (tid < 16) {
+        const int r = tid;
         float mstar = -INFINITY;
         for (int w = 0; w < kDecWarps; ++w)
             mstar = fmaxf(mstar, reinterpret_cast<float *>(smem_raw + L.tiles + w * L.warp_tiles)[16 * D + r]);
         const float mu = mstar == -INFINITY ? 0.f : mstar;
+        for (int w = 0; w < kDecWarps; ++w)
+            wfac[w][r] = fast_exp2(reinterpret_cast<float *>(smem_raw + L.tiles + w * L.warp_tiles)[16 * D + r] - mu);
+        wmax[r] = mstar;
+    }
+    __syncthreads();
+    for (int idx = tid; idx < 16 * D + 16; idx += kDecWarps * 32) {
+        const int r = idx < 16 * D ? idx / D : idx - 16 * D;
         float acc = 0.f;
         for (int w = 0; w < kDecWarps; ++w) {
             const float *pw = reinterpret_cast<float *>(smem_raw + L.tiles + w * L.warp_tiles);
-            const float f = fast_exp2(pw[16 * D + r] - mu);
+            const float f = wfac[w][r];
             acc += f * (idx < 16 * D ? pw[idx] : pw[16 * D + 16 + r]);
         }
         if (idx < 16 * D) cpart[idx] = acc;
-        else { cpart[16 * D + r] = mstar; cpart[16 * D + 16 + r] = acc; }
+        else { cpart[16 * D + r] = wmax[r]; cpart[16 * D + 16 + r] = acc; }
     }
 
     // 4c. cluster merge: CTA r combines the r-th eighth of the (row, dim) outputs.
