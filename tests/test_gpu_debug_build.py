@@ -108,6 +108,37 @@ def test_debug_build_host_prefill_and_decode(libs, monkeypatch):
         assert torch.equal(a[key], b[key]), key
 
 
+@pytest.mark.parametrize("Bc,L", [(64, 1300 + 9), (128, 900 + 3)])
+def test_debug_build_four_heads_per_kv_head(libs, monkeypatch, Bc, L):
+    """G = 4 at low sparsity (alpha 1.25): the 128-key-block kernel with 32-token tiles, whose
+    routing biases come from two warps over summary rows staged in shared memory, through the
+    full-range prefill (chosen at run time) and the sliced prefill from host memory (fused
+    routing).  Ragged lengths leave a diagonal chunk without a summary row."""
+    dash, rel, dbg = libs
+    B, Hkv, G, D, alpha = 2, 2, 4, 128, 1.25
+    q, k, v, hc = make_prefill(PrefillConfig("dbg", B, G * Hkv, Hkv, L, D, Bc, alpha, planted=True,
+                                             n_max=6, seed=101 + Bc))
+    qd, kd, vd, hcd = (x.to(dev) for x in (q, k, v, hc))
+    hq, hk, hv, hhc = (x.contiguous().pin_memory() for x in (q, k, v, hc))
+    prm = dash.make_params(B, G * Hkv, Hkv, L, D, Bc, alpha, enable_gqa=True)
+
+    def run():
+        ws = dash.workspace(dash.prefill_workspace_size(prm), dev)
+        r = dash.prefill(qd, kd, vd, hcd, Bc, alpha, enable_gqa=True, ws=ws, return_active_blocks=True)
+        st = dash.read_device_status(ws)
+        ho = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+        dash.prefill_host(hq, hk, hv, hhc, ho, qd.clone(), kd.clone(), vd.clone(), hcd.clone(),
+                          torch.empty_like(qd), Bc, alpha, enable_gqa=True, n_slices=3, ws=ws)
+        torch.cuda.current_stream().synchronize()
+        return {"out": r["out"], "active_blocks": r["active_blocks"], "host": ho,
+                "status": (st, dash.read_device_status(ws))}
+
+    a, b = _both(dash, rel, dbg, monkeypatch, run)
+    assert a["status"] == (0, 0) and b["status"] == (0, 0), (a["status"], b["status"])
+    for key in ("out", "active_blocks", "host"):
+        assert torch.equal(a[key], b[key]), key
+
+
 @pytest.mark.parametrize("G,D,Bc,T", [(16, 128, 64, 300 + 5), (4, 128, 128, 607), (1, 64, 64, 333)])
 def test_debug_build_backward_without_violations(libs, monkeypatch, G, D, Bc, T):
     """dash_backward (routing, the per-chunk token lists, query- and key-side kernels) under the
