@@ -164,25 +164,24 @@ def test_decode_workload_at_full_size(dash):
 
 
 @pytest.mark.parametrize("cell", range(6))
-def test_sweep_cell_on_sampled_rows(dash, cell):
+def test_sweep_cell_every_row(dash, cell):
     """One alpha x chunk_size cell of the 64K sweep (B = 2, H_q = 32, H_kv = 8: four query
-    heads per KV head), mask, p and O on sampled rows of both sequences."""
+    heads per KV head): mask and p on every row of both sequences, O on sampled rows."""
     cfg = sweep_config(cell)
     q, k, v, hc = make_prefill(cfg)
     B, Hq, T, D = q.shape
     Hkv, Bc = k.shape[1], cfg.chunk_size
-    C = (T + Bc - 1) // Bc
     qd, kd, vd, hcd = (x.to(dev) for x in (q, k, v, hc))
     res = dash.prefill(qd, kd, vd, hcd, Bc, cfg.alpha, cfg.gamma, enable_gqa=True,
                        return_p=True, return_active_blocks=True)
     torch.cuda.synchronize()
     assert dash.read_device_status(res["ws"]) == 0
+    n_ex = _routing_every_row(res, oracle._f64(q), oracle.stage0(k, hc, Bc), cfg)
+    assert n_ex <= 1e-5 * B * Hkv * T * T / Bc / 2, n_ex       # near-threshold flips are rare
+    del res["p"]
     rows = _sample_rows(T, Bc, 64, seed=cfg.seed + 100)
     rt = torch.from_numpy(rows).to(dev)
     ref = oracle.prefill(q, k, v, hc, Bc, cfg.alpha, cfg.gamma, rows=rows)
-    check_routing(unpack_mask(res["active_blocks"].index_select(2, rt), C),
-                  res["p"].index_select(2, rt).cpu().double().numpy(), ref["p"], ref["m"], rows,
-                  Bc, cfg.alpha, tag=cfg.name)
     check_output(res["out"].index_select(2, rt).cpu().float().numpy(), ref["O"], tag=cfg.name)
 
 
