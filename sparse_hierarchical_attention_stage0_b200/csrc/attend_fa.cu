@@ -303,26 +303,26 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
         }
         if (lane == 0) sh.n_chunks = pos;
     };
-    if (warp == kWarpBias) {
+    if (warp >= kWarpSm0 && warp < kWarpTmaV) {
+        // The tile's setup, spread over the 16 softmax warps (idle until the first block).
+        const int st = threadIdx.x - kWarpSm0 * 32;
         if (!fuse && !a.ignore_routing) {
             // tau and, where they fit, the tile's mask words (up to its diagonal chunk) into
             // shared memory, as the fused routing leaves them: the bias loop then reads no
             // memory but the summaries.
             if (ta.mask_smem) {
                 const int W = a.W, nw = ct_max / 64 + 1;
-                for (int idx = lane; idx < RT * nw; idx += 32) {
+                for (int idx = st; idx < RT * nw; idx += kSmThreads) {
                     const int u = idx / nw, w = idx % nw, t = t0 + u;
                     maskw[u * W + w] = t < a.t_end ? a.mask[(bg * a.T + t) * W + w] : 0ull;
                 }
             }
-            for (int u = lane; u < RT; u += 32) sh.tau[u] = t0 + u < a.t_end ? a.tau[bg * a.T + t0 + u] : 0.f;
-            __syncwarp();
+            for (int u = st; u < RT; u += kSmThreads) sh.tau[u] = t0 + u < a.t_end ? a.tau[bg * a.T + t0 + u] : 0.f;
         }
-        if (!fuse) build_list(ta.mask_smem != 0);
         // Group-mean queries of the tile's tokens (Stage 1's exact arithmetic).
         if (!a.ignore_routing) {
             const __nv_bfloat16 *q = reinterpret_cast<const __nv_bfloat16 *>(a.q);
-            for (int idx = lane; idx < RT * (D / 8); idx += 32) {
+            for (int idx = st; idx < RT * (D / 8); idx += kSmThreads) {
                 const int u = idx / (D / 8), d8 = (idx % (D / 8)) * 8, t = t0 + u;
                 float m[8];
                 if (t < a.t_end) {
@@ -376,6 +376,8 @@ k_attend_fa(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
         tmem_st16(tb + ((uint32_t)(32 * sp) << 16) + kColQ + 16 * kq, r);
         tmem_wait_st();
     }
+    // The union list (from the mask words staged above, or from memory), beside the Q stores.
+    if (warp == kWarpBias && !fuse) build_list(ta.mask_smem != 0);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
