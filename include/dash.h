@@ -103,7 +103,16 @@ enum {
      * bounded wait on its barrier runs out after 2 s and reports DASH_ERR_DEVICE_TIMEOUT;
      * the CTA then returns with nothing in flight and the context stays usable.  Meant for
      * a few chunks (every CTA of the grid waits its 2 s); the outputs are not meaningful. */
-    DASH_FLAG_TEST_STALL_WAIT = 16
+    DASH_FLAG_TEST_STALL_WAIT = 16,
+    /* Fused route-and-attend (dash_prefill and dash_prefill_host): where the 128-key-block
+     * Stage 2 kernel applies (D = 128, G >= 8, entmax routing, no estimated diagonal), it
+     * routes its own tile's tokens with Stage 1's arithmetic instead of a separate Stage 1
+     * launch; q is read once and the routing makes no round trip through memory.  Mask, p,
+     * tau and the output are bit-identical to the separate launches.  Off by default: on B200
+     * the separate launches measured faster (32K: 3.74 against 4.04 ms per step; 128K: 124.3
+     * against 126.3 ms), because the routing inside the kernel runs at one CTA per SM while
+     * the tensor cores wait, and the routing kernel alone runs three. */
+    DASH_FLAG_FUSE_ROUTE = 32
 };
 
 typedef struct {

@@ -37,6 +37,7 @@ FLAG_FORCE_ALL_ACTIVE = 2
 FLAG_ESTIMATE_DIAGONAL = 4
 FLAG_TEST_NEWTON_CAP = 8          # test hook: Newton solve capped at one iteration
 FLAG_TEST_STALL_WAIT = 16         # test hook: Stage 0's bounded copy wait runs out
+FLAG_FUSE_ROUTE = 32              # Stage 1 inside the Stage 2 kernel where it applies (off by default)
 
 # Every symbol include/dash.h declares.
 EXPORTS = ("dash_prefill_workspace_size", "dash_prefill", "dash_prefill_host", "dash_stage0", "dash_route",
@@ -188,7 +189,7 @@ def workspace(nbytes: int, device) -> torch.Tensor:
 def prefill(q, k, v, head_cls, chunk_size=64, alpha=1.5, gamma=1.0, sigma=1.0,
             enable_gqa=False, return_p=False, return_active_blocks=False,
             return_summary=False, dense=False, force_all_active=False,
-            estimate_diagonal=False, out=None, ws=None, topk=0):
+            estimate_diagonal=False, out=None, ws=None, topk=0, fuse_route=False):
     """Causal prefill.  q [B,Hq,T,D], k/v [B,Hkv,T,D] bf16 CUDA; head_cls [Hkv,D] fp32.
 
     Returns out [B,Hq,T,D] bf16, or a dict with out and the requested p [B,Hkv,T,C] fp32,
@@ -199,7 +200,8 @@ def prefill(q, k, v, head_cls, chunk_size=64, alpha=1.5, gamma=1.0, sigma=1.0,
     W = (C + 63) // 64
     dev = q.device
     prm = make_params(B, Hq, Hkv, T, D, chunk_size, alpha, gamma, sigma, enable_gqa,
-                      _flags(dense, force_all_active, estimate_diagonal), topk)
+                      _flags(dense, force_all_active, estimate_diagonal)
+                      | (FLAG_FUSE_ROUTE if fuse_route else 0), topk)
     _need(q, torch.bfloat16, (B, Hq, T, D), "q")
     _need(k, torch.bfloat16, (B, Hkv, T, D), "k")
     _need(v, torch.bfloat16, (B, Hkv, T, D), "v")
@@ -228,7 +230,7 @@ _copy_streams = {}
 
 def prefill_host(q_host, k_host, v_host, head_cls_host, out_host, q, k, v, head_cls, out,
                  chunk_size=64, alpha=1.5, gamma=1.0, sigma=1.0, enable_gqa=False,
-                 dense=False, force_all_active=False, n_slices=8, ws=None):
+                 dense=False, force_all_active=False, n_slices=8, ws=None, fuse_route=False):
     """Causal prefill with inputs and output in page-locked host tensors (q_host, k_host,
     v_host, head_cls_host in; out_host out), the copies overlapped with the computation in
     row slices.  q, k, v, head_cls, out are the device buffers it fills and uses (same
@@ -238,7 +240,7 @@ def prefill_host(q_host, k_host, v_host, head_cls_host, out_host, q, k, v, head_
     Hkv = k.shape[1]
     dev = q.device
     prm = make_params(B, Hq, Hkv, T, D, chunk_size, alpha, gamma, sigma, enable_gqa,
-                      _flags(dense, force_all_active, False))
+                      _flags(dense, force_all_active, False) | (FLAG_FUSE_ROUTE if fuse_route else 0))
     for name, h, d, dt in (("q", q_host, q, torch.bfloat16), ("k", k_host, k, torch.bfloat16),
                            ("v", v_host, v, torch.bfloat16), ("out", out_host, out, torch.bfloat16)):
         _need(d, dt, tuple(d.shape), name)

@@ -20,6 +20,9 @@ struct Shape {
     int B, Hq, Hkv, T, D, Bc, G, C, Cf, W;
 };
 
+// Whether the caller asked for the routing inside the Stage 2 kernel (DASH_FLAG_FUSE_ROUTE).
+bool fuse_requested(const dash_params_t *p) { return (p->flags & DASH_FLAG_FUSE_ROUTE) != 0; }
+
 // Checks shared by every entry point.  `decode`: seq_len is a cache capacity.
 dash_status_t check_params(const dash_params_t *p, Shape *s) {
     if (!p) return DASH_ERR_INVALID_ARGUMENT;
@@ -31,7 +34,7 @@ dash_status_t check_params(const dash_params_t *p, Shape *s) {
     if (!std::isfinite(p->alpha) || p->alpha < 1.f) return DASH_ERR_INVALID_ARGUMENT;
     if (!std::isfinite(p->gamma) || !(p->gamma > 0.f)) return DASH_ERR_INVALID_ARGUMENT;
     if (!std::isfinite(p->sigma) || p->sigma < 0.f) return DASH_ERR_INVALID_ARGUMENT;
-    if (p->flags & ~31u) return DASH_ERR_INVALID_ARGUMENT;
+    if (p->flags & ~63u) return DASH_ERR_INVALID_ARGUMENT;
     if (p->topk < 0) return DASH_ERR_INVALID_ARGUMENT;
     if (p->topk > 0 && (p->flags & DASH_FLAG_ESTIMATE_DIAGONAL)) return DASH_ERR_UNSUPPORTED;
     if (p->head_dim != 64 && p->head_dim != 128) return DASH_ERR_UNSUPPORTED;
@@ -306,10 +309,11 @@ dash_status_t dash_prefill(const dash_params_t *p, const void *q, const void *k,
     if (vt && ws_bytes >= off + vt) a.vt = w + off;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if ((rc = clear_status(ws, st)) != DASH_OK) return rc;
-    // Fused route-and-attend where the 128-key-block kernel takes it: Stage 2 runs Stage 1 for
-    // its own tiles (liuzhao09.github.io "DashAttention 精读", section 2: fused kernels), so q
-    // is read once and the routing never makes a round trip through memory.
-    a.fuse_route = !dense && attend_kernel(a) == AttendKernel::kFa && attend_fa_fuse_supported(a);
+    // Fused route-and-attend on request, where the 128-key-block kernel takes it: Stage 2 runs
+    // Stage 1 for its own tiles (liuzhao09.github.io "DashAttention 精读", section 2: fused
+    // kernels), so q is read once and the routing never makes a round trip through memory.
+    a.fuse_route = fuse_requested(p) && !dense && attend_kernel(a) == AttendKernel::kFa &&
+                   attend_fa_fuse_supported(a);
     if (!dense) {
         if ((rc = from_cuda(launch_stage0(a, nullptr, 0, st))) != DASH_OK) return rc;
         if (!a.fuse_route && (rc = from_cuda(launch_route(a, st))) != DASH_OK) return rc;
@@ -424,7 +428,8 @@ dash_status_t dash_prefill_host(const dash_params_t *p, const void *q_host, cons
         for (int i = 0; i < n && e == cudaSuccess; ++i) {
             a.t_begin = i * rows;
             a.t_end = std::min(s.T, (i + 1) * rows);
-            a.fuse_route = !dense && attend_kernel(a) == AttendKernel::kFa && attend_fa_fuse_supported(a);
+            a.fuse_route = fuse_requested(p) && !dense && attend_kernel(a) == AttendKernel::kFa &&
+                           attend_fa_fuse_supported(a);
             a.vt_ready = 1;
             if (const int pe = kv_piece_end(i, n)) {
                 // A new piece of keys: summarise the chunks it completes, transpose its V rows
@@ -753,7 +758,7 @@ int dash_prefill_kernel_count(const dash_params_t *p, size_t ws_bytes) {
     if (vt && ws_bytes >= off + vt) a.vt = &probe;
     const AttendKernel kern = attend_kernel(a);
     if (kern == AttendKernel::kNone) return 0;
-    const bool fused = !dense && kern == AttendKernel::kFa && attend_fa_fuse_supported(a);
+    const bool fused = fuse_requested(p) && !dense && kern == AttendKernel::kFa && attend_fa_fuse_supported(a);
     const bool with_vt = kern == AttendKernel::kFa || kern == AttendKernel::kPair || kern == AttendKernel::kFaOrWarp;
     // a run-time choice adds the cost kernel and launches both Stage 2 kernels
     const int extra = kern == AttendKernel::kFaOrWarp ? 2 : 0;

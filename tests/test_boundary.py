@@ -83,6 +83,7 @@ FAKE = 1 << 20      # a 256-aligned fake device address; never dereferenced on t
     (dict(gamma=0.0), 1),
     (dict(sigma=-1.0), 1),
     (dict(flags=64), 1),                        # unknown flag bit
+    (dict(flags=128), 1),
     (dict(topk=-1), 1),
     (dict(topk=8, flags=4), 2),                 # top-k with estimate_diagonal
     (dict(head_dim=96), 2),
@@ -201,11 +202,12 @@ def test_attend_kernel_name_follows_the_dispatch(dash):
 def test_prefill_kernel_count_follows_the_dispatch(dash):
     """The library counts the kernels one dash_prefill call launches (host only)."""
     big = 1 << 40
-    assert dash.prefill_kernel_count(_p(dash), big) == 3              # stage 0, V^T, fused route + attend
+    assert dash.prefill_kernel_count(_p(dash), big) == 4              # stage 0, route, V^T, 128-key blocks
+    assert dash.prefill_kernel_count(_p(dash, flags=32), big) == 3    # fused route + attend on request
     assert dash.prefill_kernel_count(_p(dash), 256) == 3              # stage 0, route, 64-key blocks
     assert dash.prefill_kernel_count(_p(dash, flags=1), big) == 2     # dense: V^T, SM pairs
     assert dash.prefill_kernel_count(_p(dash, head_dim=64), big) == 3  # stage 0, route, warp MMA
-    assert dash.prefill_kernel_count(_p(dash, flags=4), big) == 4     # estimated diagonal: not fused
+    assert dash.prefill_kernel_count(_p(dash, flags=4 | 32), big) == 4   # estimated diagonal: never fused
     assert dash.prefill_kernel_count(_p(dash, head_dim=96), big) == 0
     # G = 4: stage 0, route, cost kernel, V^T, both Stage 2 kernels (one exits per CTA)
     assert dash.prefill_kernel_count(_p(dash, heads_q=8), big) == 6

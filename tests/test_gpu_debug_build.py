@@ -76,7 +76,7 @@ def test_debug_build_host_prefill_and_decode(libs, monkeypatch):
         ho = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
         bo = torch.empty_like(qd)
         dash.prefill_host(hq, hk, hv, hhc, ho, qd.clone(), kd.clone(), vd.clone(), hcd.clone(), bo,
-                          Bc, 1.5, enable_gqa=True, n_slices=5, ws=ws)
+                          Bc, 1.5, enable_gqa=True, n_slices=5, ws=ws, fuse_route=True)
         torch.cuda.current_stream().synchronize()
         assert dash.read_device_status(ws) == 0
         return ho
@@ -112,8 +112,8 @@ def test_debug_build_host_prefill_and_decode(libs, monkeypatch):
 def test_debug_build_four_heads_per_kv_head(libs, monkeypatch, Bc, L):
     """G = 4 at low sparsity (alpha 1.25): the 128-key-block kernel with 32-token tiles, whose
     routing biases come from two warps over summary rows staged in shared memory, through the
-    full-range prefill (chosen at run time) and the sliced prefill from host memory (fused
-    routing).  Ragged lengths leave a diagonal chunk without a summary row."""
+    full-range prefill (chosen at run time) and the sliced prefill from host memory (with the
+    routing fused).  Ragged lengths leave a diagonal chunk without a summary row."""
     dash, rel, dbg = libs
     B, Hkv, G, D, alpha = 2, 2, 4, 128, 1.25
     q, k, v, hc = make_prefill(PrefillConfig("dbg", B, G * Hkv, Hkv, L, D, Bc, alpha, planted=True,
@@ -128,7 +128,8 @@ def test_debug_build_four_heads_per_kv_head(libs, monkeypatch, Bc, L):
         st = dash.read_device_status(ws)
         ho = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
         dash.prefill_host(hq, hk, hv, hhc, ho, qd.clone(), kd.clone(), vd.clone(), hcd.clone(),
-                          torch.empty_like(qd), Bc, alpha, enable_gqa=True, n_slices=3, ws=ws)
+                          torch.empty_like(qd), Bc, alpha, enable_gqa=True, n_slices=3, ws=ws,
+                          fuse_route=True)
         torch.cuda.current_stream().synchronize()
         return {"out": r["out"], "active_blocks": r["active_blocks"], "host": ho,
                 "status": (st, dash.read_device_status(ws))}

@@ -545,14 +545,17 @@ def test_paged_decode_equals_contiguous_decode(dash):
 @pytest.mark.parametrize("G,Bc,T", [(16, 64, 2100 + 37), (8, 128, 1500 + 3), (32, 64, 1300),
                                     (4, 64, 1500 + 3), (2, 128, 900)])
 def test_fused_route_and_attend_equals_the_separate_stages(dash, alpha, G, Bc, T):
-    """dash_prefill runs Stage 1 inside the 128-key-block Stage 2 kernel (each tile routes its
-    own tokens with Stage 1's arithmetic).  Its mask, p and output equal those of the separate
-    Stage 1 and Stage 2 launches bit for bit, and the oracle's."""
+    """dash_prefill with DASH_FLAG_FUSE_ROUTE runs Stage 1 inside the 128-key-block Stage 2
+    kernel (each tile routes its own tokens with Stage 1's arithmetic).  Its mask, p and output
+    equal those of the separate Stage 1 and Stage 2 launches bit for bit, and the oracle's;
+    the sliced prefill from host memory with the same flag gives the same output."""
     Hkv = 2 if G <= 16 else 1
     q, k, v, hc = make_prefill(_cfg(1, G * Hkv, Hkv, T, 128, Bc, alpha, seed=95 + G))
     qd, kd, vd, hcd = _to(q, k, v, hc)
+    prm = dash.make_params(1, G * Hkv, Hkv, T, 128, Bc, alpha, enable_gqa=True, flags=dash.FLAG_FUSE_ROUTE)
+    assert dash.prefill_kernel_count(prm, dash.prefill_workspace_size(prm)) == 3   # no Stage 1 launch
     res = dash.prefill(qd, kd, vd, hcd, Bc, alpha, enable_gqa=True, return_p=True,
-                       return_active_blocks=True, return_summary=True)
+                       return_active_blocks=True, return_summary=True, fuse_route=True)
     r = dash.route(qd, res["summary"], Hkv, Bc, alpha)
     o = dash.attend(qd, kd, vd, res["summary"], r["tau"], r["active_blocks"], Bc, alpha)
     torch.cuda.synchronize()
@@ -565,6 +568,12 @@ def test_fused_route_and_attend_equals_the_separate_stages(dash, alpha, G, Bc, T
     check_routing(unpack_mask(res["active_blocks"], C), res["p"].cpu().double().numpy(),
                   ref["p"], ref["m"], np.arange(T), Bc, alpha, tag="fused")
     check_output(res["out"].cpu().float().numpy(), ref["O"], tag="fused")
+    hq, hk, hv, hhc = (x.contiguous().pin_memory() for x in (q, k, v, hc))
+    ho = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    dash.prefill_host(hq, hk, hv, hhc, ho, qd.clone(), kd.clone(), vd.clone(), hcd.clone(),
+                      torch.empty_like(qd), Bc, alpha, enable_gqa=True, n_slices=3, fuse_route=True)
+    torch.cuda.current_stream().synchronize()
+    assert torch.equal(ho, res["out"].cpu())
 
 
 # ------------------------------------------------------------------------------ backward
