@@ -553,7 +553,10 @@ def test_fused_route_and_attend_equals_the_separate_stages(dash, alpha, G, Bc, T
     q, k, v, hc = make_prefill(_cfg(1, G * Hkv, Hkv, T, 128, Bc, alpha, seed=95 + G))
     qd, kd, vd, hcd = _to(q, k, v, hc)
     prm = dash.make_params(1, G * Hkv, Hkv, T, 128, Bc, alpha, enable_gqa=True, flags=dash.FLAG_FUSE_ROUTE)
-    assert dash.prefill_kernel_count(prm, dash.prefill_workspace_size(prm)) == 3   # no Stage 1 launch
+    # With G < 8 the full-range call chooses its Stage 2 kernel at run time and is not fused;
+    # the sliced prefill from host memory below still routes inside the kernel.
+    if G >= 8:
+        assert dash.prefill_kernel_count(prm, dash.prefill_workspace_size(prm)) == 3   # no Stage 1 launch
     res = dash.prefill(qd, kd, vd, hcd, Bc, alpha, enable_gqa=True, return_p=True,
                        return_active_blocks=True, return_summary=True, fuse_route=True)
     r = dash.route(qd, res["summary"], Hkv, Bc, alpha)
